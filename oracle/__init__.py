@@ -1,0 +1,230 @@
+"""CPU oracle for quantized-KV decode attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s
+``cpu_baseline`` / ``--impl reference`` legs may import this package.  The
+product path (the CUDA library and its binding) never imports or links it,
+and the two share no code: the oracle is plain C (``kvq_oracle.c``) built
+with gcc, fp32 codec arithmetic in a fixed order and fp64 attention.
+
+Every function cites the page passage it follows; see ``kvq_oracle.c``.
+Pinned by ``tests/test_oracle_*.py`` against hand-worked cases, closed forms,
+library routines (scipy's Hadamard matrix, numpy's float16, torch's fp64
+scaled-dot-product attention) and brute force.  Parity of the bound's
+magnitude against the pages is unpinned: the pages print no worked bound.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libkvq_oracle.so")
+
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc into oracle/_build/libkvq_oracle.so."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        L = _lib
+        L.oc_f16_value.restype = ctypes.c_double
+        L.oc_f16_value.argtypes = [ctypes.c_uint16]
+        L.oc_f16_round.restype = ctypes.c_uint16
+        L.oc_f16_round.argtypes = [ctypes.c_float, ctypes.c_int]
+        L.oc_block_bytes.restype = ctypes.c_int64
+        for name in ("oc_quantize_sym", "oc_quantize_asym", "oc_append", "oc_decode",
+                     "oc_dense", "oc_f16_round_n"):
+            getattr(L, name).restype = ctypes.c_int
+    return _lib
+
+
+class OcCfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("d", "hkv", "kbits", "kgroup", "krotate", "vbits", "vgroup", "num_pages")]
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+PAGE_SIZE = 16
+OK, ERR_ARG, ERR_RANGE = 0, -1, -3
+
+
+# ---------------------------------------------------------------- fp16 ----
+def f16_round(x, up: bool) -> np.ndarray:
+    """Directed rounding fp32 -> binary16 bits (up: toward +inf, else -inf)."""
+    x = _c(x, np.float32).ravel()
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib().oc_f16_round_n(_p(x), ctypes.c_int64(x.size), int(bool(up)), _p(out))
+    return out
+
+
+def f16_value(h) -> np.ndarray:
+    h = _c(h, np.uint16).ravel()
+    out = np.empty(h.shape, dtype=np.float64)
+    lib().oc_f16_value_n(_p(h), ctypes.c_int64(h.size), _p(out))
+    return out
+
+
+# ------------------------------------------------------------ rotation ----
+def rotate(x, signs) -> np.ndarray:
+    """Randomized Walsh-Hadamard rotation of the last axis, fp32, fixed order."""
+    x = _c(x, np.float32)
+    d = x.shape[-1]
+    out = np.empty_like(x)
+    lib().oc_rotate_n(_p(x), ctypes.c_int64(x.size // d), d, _p(_c(signs, np.int8)), _p(out))
+    return out
+
+
+# -------------------------------------------------------------- codecs ----
+def quantize_sym(x, bits: int):
+    """Symmetric group quantizer: returns (rc, scale_bits, codes int8)."""
+    x = _c(x, np.float32).ravel()
+    codes = np.zeros(x.size, dtype=np.int8)
+    sb = np.zeros(1, dtype=np.uint16)
+    rc = lib().oc_quantize_sym(_p(x), x.size, 127 if bits == 8 else 7, _p(sb), _p(codes))
+    return rc, int(sb[0]), codes
+
+
+def quantize_asym(x):
+    """Asymmetric 4-bit group quantizer: (rc, scale_bits, zero_bits, codes, max_err)."""
+    x = _c(x, np.float32).ravel()
+    codes = np.zeros(x.size, dtype=np.uint8)
+    sb = np.zeros(1, dtype=np.uint16)
+    zb = np.zeros(1, dtype=np.uint16)
+    e = np.zeros(1, dtype=np.float32)
+    rc = lib().oc_quantize_asym(_p(x), x.size, _p(sb), _p(zb), _p(codes), _p(e))
+    return rc, int(sb[0]), int(zb[0]), codes, float(e[0])
+
+
+class Cache:
+    """The oracle's own paged Tier-1 cache (same byte format as the library's)."""
+
+    def __init__(self, head_dim, num_kv_heads, num_pages, k_bits=8, k_group=128,
+                 k_rotate=False, v_bits=4, v_group=32, rot_signs=None):
+        self.cfg = OcCfg(head_dim, num_kv_heads, k_bits, k_group, int(bool(k_rotate)),
+                         v_bits, v_group, num_pages)
+        bb = lib().oc_block_bytes(ctypes.byref(self.cfg))
+        if bb < 0:
+            raise ValueError("unsupported cache configuration")
+        self.block_bytes = int(bb)
+        self.pool = np.zeros(num_pages * num_kv_heads * self.block_bytes, dtype=np.uint8)
+        self.eta = np.zeros((num_pages, num_kv_heads), dtype=np.float32)
+        self.signs = None if rot_signs is None else _c(rot_signs, np.int8)
+
+    @property
+    def head_dim(self):
+        return self.cfg.d
+
+    def append(self, k, v, page_table, start_pos, valid=None):
+        """Quantize k, v [num_seqs][Hkv][T][d] (fp32 or bf16 bits) into the pool."""
+        k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v)
+        assert k.shape == v.shape and k.dtype == v.dtype and k.ndim == 4
+        B, H, T, d = k.shape
+        is_f32 = int(k.dtype == np.float32)
+        pt = _c(page_table, np.int32)
+        sp = _c(start_pos, np.int32)
+        vl = None if valid is None else _c(valid, np.int32)
+        rc = lib().oc_append(ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(k), _p(v),
+                             is_f32, ctypes.c_int64(H * T * d), ctypes.c_int64(T * d),
+                             ctypes.c_int64(d), B, T, _p(vl), _p(pt), pt.shape[1], _p(sp),
+                             _p(self.signs))
+        return rc
+
+    def decode(self, q, page_table, seq_lens, scale=None, tau=math.inf, row_mask=None):
+        """Returns (o_hat f64 [rows][d], bound f64 [rows], flags u8 [rows], diag [rows][8])."""
+        q = np.ascontiguousarray(q)
+        B, NQ, HQ, d = q.shape
+        rows = B * NQ * HQ
+        scale = default_scale(d) if scale is None else np.float32(scale)
+        out = np.zeros((rows, d), dtype=np.float64)
+        bound = np.zeros(rows, dtype=np.float64)
+        flags = np.zeros(rows, dtype=np.uint8)
+        diag = np.zeros((rows, 8), dtype=np.float64)
+        pt = _c(page_table, np.int32)
+        sl = _c(seq_lens, np.int32)
+        rm = None if row_mask is None else _c(row_mask, np.uint8)
+        rc = lib().oc_decode(ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(q),
+                             int(q.dtype == np.float32), B, NQ, HQ, _p(pt), pt.shape[1], _p(sl),
+                             ctypes.c_float(scale), ctypes.c_float(tau), _p(self.signs),
+                             _p(out), _p(bound), _p(flags), _p(diag), _p(rm))
+        if rc != OK:
+            raise ValueError(f"oracle decode failed: {rc}")
+        return out, bound, flags, diag
+
+
+    def decode_terms(self, q, page_table, n, b, i, h, scale=None):
+        """Per-token (z_hat, Delta) of one query row over the first n tokens."""
+        q = np.ascontiguousarray(q)
+        B, NQ, HQ, d = q.shape
+        scale = default_scale(d) if scale is None else np.float32(scale)
+        z = np.zeros(n, dtype=np.float64)
+        dl = np.zeros(n, dtype=np.float64)
+        pt = _c(page_table, np.int32)
+        rc = lib().oc_decode_terms(ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(q),
+                                   int(q.dtype == np.float32), NQ, HQ, b, i, h, _p(pt),
+                                   pt.shape[1], n, ctypes.c_float(scale), _p(self.signs),
+                                   _p(z), _p(dl))
+        if rc != OK:
+            raise ValueError(f"oracle decode_terms failed: {rc}")
+        return z, dl
+
+
+def default_scale(d: int) -> np.float32:
+    """Scaled-dot-product default 1/sqrt(d), as the fp32 value the path receives."""
+    return np.float32(1.0 / math.sqrt(d))
+
+
+def dense(q, k, v, seq_lens, scale=None, row_mask=None) -> np.ndarray:
+    """Exact fp64 attention over originals k, v [num_seqs][Hkv][T][d]."""
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    B, NQ, HQ, d = q.shape
+    _, H, T, _ = k.shape
+    scale = default_scale(d) if scale is None else np.float32(scale)
+    out = np.zeros((B * NQ * HQ, d), dtype=np.float64)
+    sl = _c(seq_lens, np.int32)
+    rm = None if row_mask is None else _c(row_mask, np.uint8)
+    rc = lib().oc_dense(_p(q), int(q.dtype == np.float32), _p(k), _p(v),
+                        int(k.dtype == np.float32), ctypes.c_int64(H * T * d),
+                        ctypes.c_int64(T * d), ctypes.c_int64(d), B, NQ, HQ, H, d, _p(sl),
+                        ctypes.c_float(scale), _p(out), _p(rm))
+    if rc != OK:
+        raise ValueError(f"oracle dense failed: {rc}")
+    return out
+
+
+def certified(o_hat, o_dense, flags) -> np.ndarray:
+    """Final output: exact dense attention for flagged rows, else o_hat."""
+    return np.where(np.asarray(flags, bool)[:, None], o_dense, o_hat)

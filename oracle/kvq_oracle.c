@@ -1,0 +1,639 @@
+/*
+ * kvq_oracle.c -- plain, slow CPU oracle for quantized-KV decode attention
+ * with a certified per-query error bound.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * load this file: only tests/, __graft_entry__.smoke() and bench.py's
+ * cpu_baseline leg use it.  It shares no code, header, table or constant
+ * generator with the CUDA library.
+ *
+ * What it follows ("Runtime-Certified Bounded-Error Quantized Attention"):
+ *   - Methodology 1, Tier 1: keys stored as INT8 codes, values as per-group
+ *     INT4 codes with scale/offset metadata and a per-block error annotation
+ *     eta_b; Tier 2: unquantized originals kept for exact recomputation.
+ *   - Methodology 1, fallback: exact dense attention (scaled-dot-product
+ *     semantics) on the originals for a query whose bound is exceeded.
+ *   - Methodology 2: the error splits into a key term E_key (total-variation
+ *     distance between exact and approximate softmax, bounded through the
+ *     per-token score perturbation Delta) and a value term E_val (block
+ *     errors eta_b weighted by attention mass), both computed from the
+ *     quantization scales, the query norms and the value range.
+ * and ("Statistical Inference and Quality Measures of KV Cache Quantisations
+ * Inspired by TurboQuant", Quantisation schemes, KQV): a Walsh-Hadamard
+ * rotation applied to K before scalar quantization.
+ *
+ * Readings taken where the pages are silent (all listed in the design notes):
+ *   keys per token and group, symmetric, codes in [-Q, Q] with Q = 127 (8 bit)
+ *   or 7 (4 bit); values per token and 32-channel group, asymmetric, codes in
+ *   [0, 15]; scale rounded UP to fp16 and zero rounded DOWN to fp16 so codes
+ *   never clip; rounding half-to-even after an IEEE fp32 division; block =
+ *   one 16-token page of one kv head, eta = max |v - v_hat| rounded up by one
+ *   fp32 ulp; softmax scale 1/sqrt(d); GQA head h reads kv head h/(Hq/Hkv);
+ *   error norm = max-abs over the d output channels; flag = bound > tau.
+ *
+ * Codec arithmetic is fp32 in the exact operation order below (the decision
+ * of every integer code is taken in fp32, as the CUDA path takes it);
+ * attention, softmax and the bound are fp64.  Compile without FMA
+ * contraction (-ffp-contract=off) and without fast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OC_PAGE 16
+#define OC_OK 0
+#define OC_ERR_ARG (-1)
+#define OC_ERR_RANGE (-3)
+
+/* Slack factor applied to the bound: absorbs fp32 rounding of the quantizer
+ * (x/s rounded before rint), of the value dequantization and of the
+ * fixed-order Hadamard rotation. */
+#define OC_KAPPA (1.0 + 1.0 / 1024.0)
+/* Relative size of the fp32 rotation error term added to Delta for rotated
+ * keys (the fp32 FWHT of q and k deviates from an exact orthogonal map by far
+ * less than this fraction of |q|*|k|). */
+#define OC_ROT_SLACK (1.0 / 65536.0)
+
+/* ------------------------------------------------------------------------ */
+/* IEEE-754 binary16, from its definition.                                   */
+/* ------------------------------------------------------------------------ */
+
+/* value of a binary16 bit pattern: sign, 5-bit exponent (bias 15),
+ * 10-bit fraction; exponent 0 = subnormal, 31 = inf/nan */
+double oc_f16_value(uint16_t h) {
+  int sign = (h >> 15) & 1, e = (h >> 10) & 31, f = h & 1023;
+  double v;
+  if (e == 31) v = f ? NAN : INFINITY;
+  else if (e == 0) v = ldexp((double)f, -24);            /* f/1024 * 2^-14 */
+  else v = ldexp(1.0 + f / 1024.0, e - 15);
+  return sign ? -v : v;
+}
+
+typedef struct { double v; uint16_t h; } oc_f16_entry;
+static oc_f16_entry oc_tab[63490];  /* all finite binary16 values, sorted */
+static int oc_tab_n = 0;
+
+static int oc_cmp(const void* a, const void* b) {
+  double x = ((const oc_f16_entry*)a)->v, y = ((const oc_f16_entry*)b)->v;
+  return (x > y) - (x < y);
+}
+
+static void oc_tab_init(void) {
+  if (oc_tab_n) return;
+  int n = 0;
+  for (uint32_t h = 0; h < 65536u; ++h) {
+    if (((h >> 10) & 31) == 31) continue;       /* skip inf / nan */
+    if (h == 0x8000u) continue;                  /* -0 handled by sign rule */
+    oc_tab[n].v = oc_f16_value((uint16_t)h);
+    oc_tab[n].h = (uint16_t)h;
+    ++n;
+  }
+  qsort(oc_tab, n, sizeof(oc_tab[0]), oc_cmp);
+  oc_tab_n = n;
+}
+
+/* Directed rounding of a finite fp32 to binary16:
+ *   up   -> smallest binary16 >= x (or +inf),
+ *   down -> largest  binary16 <= x (or -inf).
+ * A zero result keeps the sign of x (IEEE rule for directed rounding). */
+uint16_t oc_f16_round(float xf, int up) {
+  oc_tab_init();
+  double x = (double)xf;
+  if (isnan(x)) return 0x7E00u;
+  int lo = 0, hi = oc_tab_n - 1;
+  uint16_t r;
+  if (up) {
+    if (x > oc_tab[hi].v) return 0x7C00u;           /* +inf */
+    /* first entry with v >= x */
+    while (lo < hi) { int mid = (lo + hi) / 2; if (oc_tab[mid].v >= x) hi = mid; else lo = mid + 1; }
+    r = oc_tab[lo].h;
+  } else {
+    if (x < oc_tab[0].v) return 0xFC00u;            /* -inf */
+    /* last entry with v <= x */
+    while (lo < hi) { int mid = (lo + hi + 1) / 2; if (oc_tab[mid].v <= x) lo = mid; else hi = mid - 1; }
+    r = oc_tab[lo].h;
+  }
+  if ((r & 0x7FFFu) == 0) r = signbit(xf) ? 0x8000u : 0x0000u;
+  return r;
+}
+
+int oc_f16_round_n(const float* x, int64_t n, int up, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oc_f16_round(x[i], up);
+  return OC_OK;
+}
+
+void oc_f16_value_n(const uint16_t* h, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oc_f16_value(h[i]);
+}
+
+static float oc_bf16_to_f32(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Randomized Walsh-Hadamard rotation (KQV scheme: WHT before quantization). */
+/* y = c * H_d * (sigma o x), H_d the Sylvester Hadamard matrix,             */
+/* c = fp32(1/sqrt(d)).  Butterflies in a fixed order: stride 1, 2, ...,     */
+/* d/2; each pair (a, b) at (j, j + stride) becomes (a + b, a - b).  Then    */
+/* every element is multiplied by c.  All in fp32.                           */
+/* ------------------------------------------------------------------------ */
+void oc_rotate(const float* x, const int8_t* sigma, int d, float* y) {
+  float c = (float)(1.0 / sqrt((double)d));
+  for (int i = 0; i < d; ++i) y[i] = sigma[i] < 0 ? -x[i] : x[i];
+  for (int h = 1; h < d; h *= 2)
+    for (int i = 0; i < d; i += 2 * h)
+      for (int j = i; j < i + h; ++j) {
+        float a = y[j], b = y[j + h];
+        y[j] = a + b;
+        y[j + h] = a - b;
+      }
+  for (int i = 0; i < d; ++i) y[i] = y[i] * c;
+}
+
+void oc_rotate_n(const float* x, int64_t n, int d, const int8_t* sigma, float* y) {
+  for (int64_t i = 0; i < n; ++i) oc_rotate(x + i * d, sigma, d, y + i * d);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Scalar codecs (Tier 1: INT8/INT4 keys, INT4 values with scale/offset).     */
+/* ------------------------------------------------------------------------ */
+
+/* Symmetric group quantizer for keys.
+ * a = max|x|; s = fp16_up(a / Q); code = clamp(rint(x / s), -Q, Q); s = 0 -> 0.
+ * Returns OC_ERR_RANGE (and zero codes/scale) on a non-finite input or an
+ * fp16-overflowing scale. */
+int oc_quantize_sym(const float* x, int n, int Q, uint16_t* scale_bits, int8_t* codes) {
+  float a = 0.0f;
+  for (int c = 0; c < n; ++c) {
+    if (!isfinite(x[c])) { *scale_bits = 0; memset(codes, 0, n); return OC_ERR_RANGE; }
+    float m = fabsf(x[c]);
+    if (m > a) a = m;
+  }
+  float t = a / (float)Q;
+  uint16_t sb = oc_f16_round(t, 1);
+  if ((sb & 0x7C00u) == 0x7C00u) { *scale_bits = 0; memset(codes, 0, n); return OC_ERR_RANGE; }
+  float s = (float)oc_f16_value(sb);
+  *scale_bits = sb;
+  for (int c = 0; c < n; ++c) {
+    if (s == 0.0f) { codes[c] = 0; continue; }
+    float r = rintf(x[c] / s);
+    if (r > (float)Q) r = (float)Q;
+    if (r < (float)-Q) r = (float)-Q;
+    codes[c] = (int8_t)r;
+  }
+  return OC_OK;
+}
+
+/* Asymmetric 4-bit group quantizer for values.
+ * z = fp16_down(min x); s = fp16_up((max x - z) / 15);
+ * code = clamp(rint((x - z) / s), 0, 15) (s = 0 -> 0);
+ * v_hat = fmaf(code, s, z); max_err = max |x - v_hat| (fp32). */
+int oc_quantize_asym(const float* x, int n, uint16_t* scale_bits, uint16_t* zero_bits,
+                     uint8_t* codes, float* max_err) {
+  float lo = x[0], hi = x[0];
+  for (int c = 0; c < n; ++c) {
+    if (!isfinite(x[c])) goto range;
+    if (x[c] < lo) lo = x[c];
+    if (x[c] > hi) hi = x[c];
+  }
+  {
+    uint16_t zb = oc_f16_round(lo, 0);
+    if ((zb & 0x7C00u) == 0x7C00u) goto range;
+    float z = (float)oc_f16_value(zb);
+    float t = (hi - z) / 15.0f;
+    uint16_t sb = oc_f16_round(t, 1);
+    if ((sb & 0x7C00u) == 0x7C00u) goto range;
+    float s = (float)oc_f16_value(sb);
+    float e = 0.0f;
+    for (int c = 0; c < n; ++c) {
+      float r = 0.0f;
+      if (s != 0.0f) {
+        r = rintf((x[c] - z) / s);
+        if (r > 15.0f) r = 15.0f;
+        if (r < 0.0f) r = 0.0f;
+      }
+      codes[c] = (uint8_t)r;
+      float vh = fmaf(r, s, z);
+      float err = fabsf(x[c] - vh);
+      if (err > e) e = err;
+    }
+    *scale_bits = sb;
+    *zero_bits = zb;
+    *max_err = e;
+    return OC_OK;
+  }
+range:
+  *scale_bits = 0;
+  *zero_bits = 0;
+  memset(codes, 0, n);
+  *max_err = 0.0f;
+  return OC_ERR_RANGE;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Paged Tier-1 layout.  One block per (physical page, kv head), 16 tokens:  */
+/*   [K codes][V codes][K scales fp16 [16][d/gk]][V scale,zero fp16 [16][d/32][2]] */
+/* K codes, 8 bit: row-major int8 [16][d].                                    */
+/* K codes, 4 bit: per token d/2 bytes; channel c (block b = c/32, w = c%32)  */
+/*   sits in byte (w/8)*(4*nb) + 4*b + (w%8)/2, low nibble for even c,       */
+/*   4-bit two's complement; nb = d/32.                                       */
+/* V codes: per token d/2 bytes; channel c (group g = c/32, w = c%32) sits in */
+/*   byte (w/4)*(2*nb) + 2*g + (w%4)/2, low nibble for even c, unsigned.     */
+/* eta is a separate fp32 array [num_pages][Hkv].                             */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t d, hkv, kbits, kgroup, krotate, vbits, vgroup, num_pages;
+} oc_cfg;
+
+static int oc_cfg_ok(const oc_cfg* c) {
+  if (!c || (c->d != 64 && c->d != 128) || c->hkv <= 0 || c->num_pages < 0) return 0;
+  if (c->kbits != 8 && c->kbits != 4) return 0;
+  if (c->kgroup <= 0 || c->kgroup % 32 || c->d % c->kgroup) return 0;
+  if (c->vbits != 4 || c->vgroup != 32) return 0;
+  return 1;
+}
+
+static int64_t oc_kcode_bytes(const oc_cfg* c) { return (int64_t)OC_PAGE * c->d * c->kbits / 8; }
+static int64_t oc_vcode_bytes(const oc_cfg* c) { return (int64_t)OC_PAGE * c->d / 2; }
+static int64_t oc_kscale_bytes(const oc_cfg* c) { return (int64_t)OC_PAGE * (c->d / c->kgroup) * 2; }
+static int64_t oc_vmeta_bytes(const oc_cfg* c) { return (int64_t)OC_PAGE * (c->d / 32) * 4; }
+
+int64_t oc_block_bytes(const oc_cfg* c) {
+  if (!oc_cfg_ok(c)) return -1;
+  return oc_kcode_bytes(c) + oc_vcode_bytes(c) + oc_kscale_bytes(c) + oc_vmeta_bytes(c);
+}
+
+static int64_t oc_k4_byte(int d, int ch) {
+  int nb = d / 32, b = ch / 32, w = ch % 32;
+  return (int64_t)(w / 8) * (4 * nb) + 4 * b + (w % 8) / 2;
+}
+static int64_t oc_v4_byte(int d, int ch) {
+  int nb = d / 32, g = ch / 32, w = ch % 32;
+  return (int64_t)(w / 4) * (2 * nb) + 2 * g + (w % 4) / 2;
+}
+
+static void oc_put_nibble(uint8_t* row, int64_t byte, int ch, unsigned v) {
+  if (ch % 2 == 0) row[byte] = (uint8_t)((row[byte] & 0xF0u) | (v & 0xFu));
+  else row[byte] = (uint8_t)((row[byte] & 0x0Fu) | ((v & 0xFu) << 4));
+}
+static unsigned oc_get_nibble(const uint8_t* row, int64_t byte, int ch) {
+  return ch % 2 == 0 ? (row[byte] & 0xFu) : (row[byte] >> 4);
+}
+
+static uint16_t oc_rd16(const uint8_t* p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+static void oc_wr16(uint8_t* p, uint16_t v) { p[0] = (uint8_t)(v & 0xFF); p[1] = (uint8_t)(v >> 8); }
+
+/* Quantize one token of one kv head into slot `slot` of block `blk`.
+ * x_k, x_v: fp32 [d]; returns the token's fp32 max value error through *verr. */
+static int oc_quantize_token(const oc_cfg* c, uint8_t* blk, int slot, const float* xk_in,
+                             const float* xv, const int8_t* sigma, float* verr) {
+  int d = c->d, rc = OC_OK;
+  float xk_rot[128];
+  const float* xk = xk_in;
+  if (c->krotate) { oc_rotate(xk_in, sigma, d, xk_rot); xk = xk_rot; }
+  /* keys */
+  int Q = c->kbits == 8 ? 127 : 7;
+  uint8_t* kcodes = blk;
+  uint8_t* kscales = blk + oc_kcode_bytes(c) + oc_vcode_bytes(c);
+  for (int g = 0; g < d / c->kgroup; ++g) {
+    int8_t codes[128];
+    uint16_t sb;
+    int r = oc_quantize_sym(xk + g * c->kgroup, c->kgroup, Q, &sb, codes);
+    if (r != OC_OK) rc = r;
+    oc_wr16(kscales + ((int64_t)slot * (d / c->kgroup) + g) * 2, sb);
+    for (int i = 0; i < c->kgroup; ++i) {
+      int ch = g * c->kgroup + i;
+      if (c->kbits == 8) {
+        kcodes[(int64_t)slot * d + ch] = (uint8_t)codes[i];
+      } else {
+        uint8_t* row = kcodes + (int64_t)slot * (d / 2);
+        oc_put_nibble(row, oc_k4_byte(d, ch), ch, (unsigned)(codes[i] & 0xF));
+      }
+    }
+  }
+  /* values */
+  uint8_t* vrow = blk + oc_kcode_bytes(c) + (int64_t)slot * (d / 2);
+  uint8_t* vmeta = blk + oc_kcode_bytes(c) + oc_vcode_bytes(c) + oc_kscale_bytes(c);
+  float e = 0.0f;
+  for (int g = 0; g < d / 32; ++g) {
+    uint8_t codes[32];
+    uint16_t sb, zb;
+    float ge;
+    int r = oc_quantize_asym(xv + g * 32, 32, &sb, &zb, codes, &ge);
+    if (r != OC_OK) rc = r;
+    oc_wr16(vmeta + ((int64_t)slot * (d / 32) + g) * 4, sb);
+    oc_wr16(vmeta + ((int64_t)slot * (d / 32) + g) * 4 + 2, zb);
+    for (int i = 0; i < 32; ++i) {
+      int ch = g * 32 + i;
+      oc_put_nibble(vrow, oc_v4_byte(d, ch), ch, codes[i]);
+    }
+    if (ge > e) e = ge;
+  }
+  *verr = e;
+  return rc;
+}
+
+static void oc_load_vec(const void* base, int is_f32, int64_t off, int d, float* out) {
+  if (is_f32) memcpy(out, (const float*)base + off, sizeof(float) * d);
+  else for (int i = 0; i < d; ++i) out[i] = oc_bf16_to_f32(((const uint16_t*)base)[off + i]);
+}
+
+/* Quantize-on-append.  Token t (< valid[b], or < num_tokens if valid is NULL)
+ * of sequence b goes to logical position start_pos[b] + t, i.e. physical page
+ * page_table[b][pos/16], slot pos%16.  Element (b, h, t, ch) of k and v is at
+ * b*seq_stride + h*head_stride + t*tok_stride + ch.
+ * eta[page][h] = max(eta, nextafter(token max error, +inf)). */
+int oc_append(const oc_cfg* c, uint8_t* pool, float* eta, const void* k, const void* v,
+              int in_is_f32, int64_t seq_stride, int64_t head_stride, int64_t tok_stride,
+              int num_seqs, int num_tokens, const int32_t* valid, const int32_t* page_table,
+              int max_pages, const int32_t* start_pos, const int8_t* sigma) {
+  if (!oc_cfg_ok(c) || (c->krotate && !sigma)) return OC_ERR_ARG;
+  int64_t bb = oc_block_bytes(c);
+  int rc = OC_OK;
+  float xk[128], xv[128];
+  for (int b = 0; b < num_seqs; ++b) {
+    int nt = valid ? valid[b] : num_tokens;
+    for (int t = 0; t < nt; ++t) {
+      int pos = start_pos[b] + t;
+      int lp = pos / OC_PAGE;
+      if (lp >= max_pages) return OC_ERR_ARG;
+      int page = page_table[(int64_t)b * max_pages + lp];
+      if (page < 0 || page >= c->num_pages) return OC_ERR_ARG;
+      for (int h = 0; h < c->hkv; ++h) {
+        int64_t off = b * seq_stride + h * head_stride + t * tok_stride;
+        oc_load_vec(k, in_is_f32, off, c->d, xk);
+        oc_load_vec(v, in_is_f32, off, c->d, xv);
+        uint8_t* blk = pool + ((int64_t)page * c->hkv + h) * bb;
+        float e;
+        int r = oc_quantize_token(c, blk, pos % OC_PAGE, xk, xv, sigma, &e);
+        if (r != OC_OK) rc = r;
+        float eu = nextafterf(e, INFINITY);
+        float* ep = eta + (int64_t)page * c->hkv + h;
+        if (eu > *ep) *ep = eu;
+      }
+    }
+  }
+  return rc;
+}
+
+/* Dequantized view of one token of one kv head, read back from the layout. */
+static void oc_read_token(const oc_cfg* c, const uint8_t* blk, int slot, double* khat,
+                          double* kscale, double* vhat, double* vs, double* vz,
+                          double* vtop) {
+  int d = c->d, ngk = d / c->kgroup;
+  const uint8_t* kcodes = blk;
+  const uint8_t* vrow = blk + oc_kcode_bytes(c) + (int64_t)slot * (d / 2);
+  const uint8_t* kscales = blk + oc_kcode_bytes(c) + oc_vcode_bytes(c);
+  const uint8_t* vmeta = kscales + oc_kscale_bytes(c);
+  for (int g = 0; g < ngk; ++g)
+    kscale[g] = oc_f16_value(oc_rd16(kscales + ((int64_t)slot * ngk + g) * 2));
+  for (int ch = 0; ch < d; ++ch) {
+    int code;
+    if (c->kbits == 8) code = (int8_t)kcodes[(int64_t)slot * d + ch];
+    else {
+      unsigned nib = oc_get_nibble(kcodes + (int64_t)slot * (d / 2), oc_k4_byte(d, ch), ch);
+      code = nib >= 8 ? (int)nib - 16 : (int)nib;
+    }
+    khat[ch] = kscale[ch / c->kgroup] * code;
+  }
+  for (int g = 0; g < d / 32; ++g) {
+    uint16_t sb = oc_rd16(vmeta + ((int64_t)slot * (d / 32) + g) * 4);
+    uint16_t zb = oc_rd16(vmeta + ((int64_t)slot * (d / 32) + g) * 4 + 2);
+    vs[g] = oc_f16_value(sb);
+    vz[g] = oc_f16_value(zb);
+    /* top of the representable range of this group: fmaf(15, s, z) in fp32 */
+    vtop[g] = (double)fmaf(15.0f, (float)vs[g], (float)vz[g]);
+  }
+  for (int ch = 0; ch < d; ++ch) {
+    unsigned code = oc_get_nibble(vrow, oc_v4_byte(d, ch), ch);
+    vhat[ch] = vs[ch / 32] * (double)code + vz[ch / 32];   /* exact in fp64 */
+  }
+}
+
+/* Quantized decode attention and its certified bound, for every query row
+ * (sequence b, query i, q head h), kv head h / (Hq/Hkv):
+ *   q'   = rotated q if keys are rotated (same fp32 rotation as the keys)
+ *   z^_j = scale * q' . k^_j                          (fp64)
+ *   p^   = softmax(z^),  o^ = sum_j p^_j v^_j
+ *   Delta_j = kappa*scale*( sum_g |q'_g|_1 * sK_{j,g} / 2
+ *                           + [rotated] 2^-16*sqrt(d)*Q*|q'|_2*max_g sK_{j,g} )
+ *   A = sum_j p^_j (exp(Delta_j) - 1),  B = sum_j p^_j exp(-Delta_j)
+ *   TV = min(tanh(max_j Delta_j / 2), A / B)
+ *   range = max_g ( max_j fmaf(15, sV_{j,g}, zV_{j,g}) - min_j zV_{j,g} )
+ *   E_key = TV * (range + 2 * max_b eta_b)
+ *   E_val = sum_j p^_j eta_{block(j)}
+ *   bound = kappa * (E_key + E_val);  flag = bound > tau.
+ * An empty context gives o^ = 0, bound = 0, flag = 0.
+ * diag (optional) gets per row: TV, E_key, E_val, max Delta, A, B, range, eta_max.
+ * row_mask (optional): only rows with a nonzero entry are computed. */
+/* Per-token terms of one query row over its context of n tokens:
+ * z[j] = z^_j, dl[j] = Delta_j, et[j] = eta of token j's block; also the
+ * value range and the largest eta of the context. */
+static void oc_row_terms(const oc_cfg* c, const uint8_t* pool, const float* eta,
+                         const float* qp, int b, int kv, int n, const int32_t* page_table,
+                         int max_pages, double sc, double* z, double* dl, double* et,
+                         double* range_out, double* eta_max_out) {
+  int d = c->d, ngk = d / c->kgroup, ngv = d / 32;
+  int Q = c->kbits == 8 ? 127 : 7;
+  int64_t bb = oc_block_bytes(c);
+  double qn1[4] = {0, 0, 0, 0}, qn2 = 0.0;
+  for (int ch = 0; ch < d; ++ch) {
+    qn1[ch / c->kgroup] += fabs((double)qp[ch]);
+    qn2 += (double)qp[ch] * (double)qp[ch];
+  }
+  qn2 = sqrt(qn2);
+  double rot = c->krotate ? OC_ROT_SLACK * sqrt((double)d) * Q * qn2 : 0.0;
+  double vtop_max[4], vz_min[4], eta_max = 0.0;
+  for (int g = 0; g < ngv; ++g) { vtop_max[g] = -INFINITY; vz_min[g] = INFINITY; }
+  double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+  for (int j = 0; j < n; ++j) {
+    int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
+    const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+    oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+    double dot = 0.0, smax = 0.0, qs = 0.0;
+    for (int ch = 0; ch < d; ++ch) dot += (double)qp[ch] * khat[ch];
+    for (int g = 0; g < ngk; ++g) {
+      qs += qn1[g] * ks[g] / 2.0;
+      if (ks[g] > smax) smax = ks[g];
+    }
+    z[j] = sc * dot;
+    dl[j] = OC_KAPPA * sc * (qs + rot * smax);
+    et[j] = (double)eta[(int64_t)page * c->hkv + kv];
+    if (et[j] > eta_max) eta_max = et[j];
+    for (int g = 0; g < ngv; ++g) {
+      if (vtop[g] > vtop_max[g]) vtop_max[g] = vtop[g];
+      if (vz[g] < vz_min[g]) vz_min[g] = vz[g];
+    }
+  }
+  double range = 0.0;
+  for (int g = 0; g < ngv; ++g)
+    if (vtop_max[g] - vz_min[g] > range) range = vtop_max[g] - vz_min[g];
+  *range_out = range;
+  *eta_max_out = eta_max;
+}
+
+static const float* oc_row_query(const oc_cfg* c, const void* q, int q_is_f32, int64_t row,
+                                 const int8_t* sigma, float* qf, float* qr) {
+  oc_load_vec(q, q_is_f32, row * c->d, c->d, qf);
+  if (!c->krotate) return qf;
+  oc_rotate(qf, sigma, c->d, qr);
+  return qr;
+}
+
+/* Quantized decode attention and its certified bound, for every query row
+ * (sequence b, query i, q head h), kv head h / (Hq/Hkv):
+ *   q'   = rotated q if keys are rotated (same fp32 rotation as the keys)
+ *   z^_j = scale * q' . k^_j                          (fp64)
+ *   p^   = softmax(z^),  o^ = sum_j p^_j v^_j
+ *   Delta_j = kappa*scale*( sum_g |q'_g|_1 * sK_{j,g} / 2
+ *                           + [rotated] 2^-16*sqrt(d)*Q*|q'|_2*max_g sK_{j,g} )
+ *   A = sum_j p^_j (exp(Delta_j) - 1),  B = sum_j p^_j exp(-Delta_j)
+ *   TV = min(tanh(max_j Delta_j / 2), A / B)
+ *   range = max_g ( max_j fmaf(15, sV_{j,g}, zV_{j,g}) - min_j zV_{j,g} )
+ *   E_key = TV * (range + 2 * max_b eta_b)
+ *   E_val = sum_j p^_j eta_{block(j)}
+ *   bound = kappa * (E_key + E_val);  flag = bound > tau.
+ * An empty context gives o^ = 0, bound = 0, flag = 0.
+ * diag (optional) gets per row: TV, E_key, E_val, max Delta, A, B, range, eta_max.
+ * row_mask (optional): only rows with a nonzero entry are computed. */
+int oc_decode(const oc_cfg* c, const uint8_t* pool, const float* eta, const void* q,
+              int q_is_f32, int num_seqs, int nq, int hq, const int32_t* page_table,
+              int max_pages, const int32_t* seq_lens, float scale, float tau,
+              const int8_t* sigma, double* out, double* bound, uint8_t* flags, double* diag,
+              const uint8_t* row_mask) {
+  if (!oc_cfg_ok(c) || hq % c->hkv || (c->krotate && !sigma)) return OC_ERR_ARG;
+  int d = c->d, G = hq / c->hkv;
+  int64_t bb = oc_block_bytes(c);
+  double sc = (double)scale;
+  for (int b = 0; b < num_seqs; ++b) {
+    int n = seq_lens[b];
+    double* z = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* dl = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* et = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    for (int i = 0; i < nq; ++i)
+      for (int h = 0; h < hq; ++h) {
+        int64_t row = ((int64_t)b * nq + i) * hq + h;
+        if (row_mask && !row_mask[row]) continue;
+        int kv = h / G;
+        double* o = out + row * d;
+        for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+        if (n == 0) {
+          bound[row] = 0.0;
+          flags[row] = 0;
+          if (diag) for (int t = 0; t < 8; ++t) diag[row * 8 + t] = 0.0;
+          continue;
+        }
+        float qf[128], qr[128];
+        const float* qp = oc_row_query(c, q, q_is_f32, row, sigma, qf, qr);
+        double range, eta_max;
+        oc_row_terms(c, pool, eta, qp, b, kv, n, page_table, max_pages, sc, z, dl, et, &range,
+                     &eta_max);
+        double m = -INFINITY;
+        for (int j = 0; j < n; ++j) if (z[j] > m) m = z[j];
+        double l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
+        double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+        for (int j = 0; j < n; ++j) {
+          double p = exp(z[j] - m) / l;
+          int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
+          const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+          oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+          for (int ch = 0; ch < d; ++ch) o[ch] += p * vhat[ch];
+          A += p * expm1(dl[j]);
+          B += p * exp(-dl[j]);
+          Ev += p * et[j];
+          if (dl[j] > dmax) dmax = dl[j];
+        }
+        double tv = tanh(dmax / 2.0);
+        if (A / B < tv) tv = A / B;
+        double ekey = tv * (range + 2.0 * eta_max);
+        double bd = OC_KAPPA * (ekey + Ev);
+        bound[row] = bd;
+        flags[row] = bd > (double)tau ? 1 : 0;
+        if (diag) {
+          double* dg = diag + row * 8;
+          dg[0] = tv; dg[1] = ekey; dg[2] = Ev; dg[3] = dmax;
+          dg[4] = A; dg[5] = B; dg[6] = range; dg[7] = eta_max;
+        }
+      }
+    free(z);
+    free(dl);
+    free(et);
+  }
+  return OC_OK;
+}
+
+/* Per-token scores z^_j and perturbation bounds Delta_j of one query row
+ * (for tests of the bound's ingredients). */
+int oc_decode_terms(const oc_cfg* c, const uint8_t* pool, const float* eta, const void* q,
+                    int q_is_f32, int nq, int hq, int b, int i, int h,
+                    const int32_t* page_table, int max_pages, int n, float scale,
+                    const int8_t* sigma, double* z, double* dl) {
+  if (!oc_cfg_ok(c) || hq % c->hkv || (c->krotate && !sigma) || n <= 0) return OC_ERR_ARG;
+  int64_t row = ((int64_t)b * nq + i) * hq + h;
+  float qf[128], qr[128];
+  const float* qp = oc_row_query(c, q, q_is_f32, row, sigma, qf, qr);
+  double* et = (double*)malloc(sizeof(double) * n);
+  double range, eta_max;
+  oc_row_terms(c, pool, eta, qp, b, h / (hq / c->hkv), n, page_table, max_pages,
+               (double)scale, z, dl, et, &range, &eta_max);
+  free(et);
+  return OC_OK;
+}
+
+/* Exact dense attention on the originals (the fallback's ground truth):
+ * o = softmax(scale * q . k_j) v, fp64, no quantization, no rotation.
+ * k, v element (b, h, t, ch) at b*seq_stride + h*head_stride + t*tok_stride + ch. */
+int oc_dense(const void* q, int q_is_f32, const void* k, const void* v, int kv_is_f32,
+             int64_t seq_stride, int64_t head_stride, int64_t tok_stride, int num_seqs,
+             int nq, int hq, int hkv, int d, const int32_t* seq_lens, float scale, double* out,
+             const uint8_t* row_mask) {
+  if (d <= 0 || d > 128 || hkv <= 0 || hq % hkv) return OC_ERR_ARG;
+  int G = hq / hkv;
+  double sc = (double)scale;
+  float qf[128], kf[128], vf[128];
+  for (int b = 0; b < num_seqs; ++b) {
+    int n = seq_lens[b];
+    double* z = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    for (int i = 0; i < nq; ++i)
+      for (int h = 0; h < hq; ++h) {
+        int64_t row = ((int64_t)b * nq + i) * hq + h;
+        if (row_mask && !row_mask[row]) continue;
+        int kv = h / G;
+        double* o = out + row * d;
+        for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+        if (n == 0) continue;
+        oc_load_vec(q, q_is_f32, row * d, d, qf);
+        double m = -INFINITY;
+        for (int j = 0; j < n; ++j) {
+          oc_load_vec(k, kv_is_f32, b * seq_stride + kv * head_stride + j * tok_stride, d, kf);
+          double dot = 0.0;
+          for (int ch = 0; ch < d; ++ch) dot += (double)qf[ch] * (double)kf[ch];
+          z[j] = sc * dot;
+          if (z[j] > m) m = z[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        for (int j = 0; j < n; ++j) {
+          double p = exp(z[j] - m) / l;
+          oc_load_vec(v, kv_is_f32, b * seq_stride + kv * head_stride + j * tok_stride, d, vf);
+          for (int ch = 0; ch < d; ++ch) o[ch] += p * (double)vf[ch];
+        }
+      }
+    free(z);
+  }
+  return OC_OK;
+}
+
+/* Certified output: o = exact dense attention where flag is set, else o^. */
+void oc_certified_output(const double* ohat, const double* odense, const uint8_t* flags,
+                         int64_t rows, int d, double* out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int ch = 0; ch < d; ++ch)
+      out[r * d + ch] = flags[r] ? odense[r * d + ch] : ohat[r * d + ch];
+}
