@@ -1,0 +1,472 @@
+"""Benchmark of one decode step of quantized-KV attention with the certified bound.
+
+A step is one pass of the whole hot path over one batch: quantize-on-append of
+the step's new K/V token of every sequence into the paged cache, then the fused
+split-K decode attention with its per-query bound and flags over the full
+context (and, when tau is finite and a query is flagged, the exact fallback).
+The metric is KV token-heads processed per second (sum of context lengths x kv
+heads per step) and the achieved HBM bandwidth of the decode kernel against the
+measured peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b]
+    python bench.py --impl reference ...   # the CPU oracle as the reference arm
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the path
+has no exchange step); the time is the max over ranks and the value is the
+work of all ranks over that time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_decode_attention_kvq_b200 import inputs as synth  # noqa: E402
+
+METRIC = ("quantized-KV decode attention: KV tokens·heads/s and achieved HBM GB/s "
+          "vs peak")
+UNIT = "KV token-heads/s"
+L2_BYTES = 126 * 2 ** 20
+DECODE_SRC = os.path.join(ROOT, "quantized_decode_attention_kvq_b200", "csrc",
+                          "decode_attention.cu")
+
+
+def _workload_desc(wl) -> str:
+    ctx = f"ctx {wl.ctx}" if wl.ctx_min is None else f"ctx U[{wl.ctx_min},{wl.ctx}]"
+    rot = "Hadamard-rotated " if wl.k_rotate else ""
+    return (f"{wl.name}: B={wl.num_seqs}, Hq={wl.num_q_heads}, Hkv={wl.num_kv_heads}, "
+            f"d={wl.head_dim}, {ctx}, {rot}INT{wl.k_bits}-K g{wl.k_group}, "
+            f"INT{wl.v_bits}-V g{wl.v_group}, 16-token pages (seeded permutation), "
+            f"tau={wl.tau}")
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _traffic_record():
+    """dram bytes per decode launch from the committed ncu summary, if it was taken
+    on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "decode_attention_llama8b_traffic.md")
+    if not os.path.exists(p):
+        return None
+    src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
+    rec = {}
+    for line in open(p):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            rec[k.strip()] = v.strip()
+    if rec.get("decode_source_sha256_16") != src_hash:
+        return None
+    try:
+        return float(rec["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------- GPU --
+def _dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class GpuStep:
+    """Device-resident workload and the raw C-ABI calls of one step."""
+
+    def __init__(self, wl_name: str, seed: int, replicas: int):
+        import ctypes
+
+        import torch
+
+        from quantized_decode_attention_kvq_b200 import kvq
+        self.kvq = kvq
+        self.torch = torch
+        inp = synth.make(wl_name, seed)
+        wl = inp.wl
+        self.inp, self.wl = inp, wl
+        k, v = inp.kv()
+        q = inp.q()
+
+        def dev(x):
+            t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if x.dtype == np.uint16 \
+                else torch.from_numpy(x)
+            return t.cuda()
+
+        T = k.shape[2]
+        self.kd, self.vd, self.qd = dev(k), dev(v), dev(q)
+        self.pt = torch.from_numpy(inp.page_table).cuda()
+        self.sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
+        base = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, k_bits=wl.k_bits,
+                              k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+        zeros = torch.zeros(wl.num_seqs, dtype=torch.int32, device="cuda")
+        base.append(self.kd, self.vd, self.pt, zeros, self.sl)
+        torch.cuda.synchronize()
+        # the step's new token: position seq_len - 1 of every sequence
+        self.new_pos = (self.sl - 1).to(torch.int32)
+        last = torch.tensor(inp.seq_lens, device="cuda").long() - 1
+        idx = last.view(-1, 1, 1, 1).expand(-1, wl.num_kv_heads, 1, wl.head_dim)
+        self.k_new = torch.gather(self.kd, 2, idx).contiguous()       # [B][Hkv][1][d]
+        self.v_new = torch.gather(self.vd, 2, idx).contiguous()
+        self.caches = [base]
+        for _ in range(replicas - 1):
+            c = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, k_bits=wl.k_bits,
+                               k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+            c.pool.copy_(base.pool)
+            c.eta.copy_(base.eta)
+            self.caches.append(c)
+        self.ws = [c.workspace(wl.num_seqs, wl.num_queries, wl.num_q_heads, self.pt.shape[1])
+                   for c in self.caches]
+        B, NQ, HQ, d = q.shape
+        self.out = torch.empty((B, NQ, HQ, d), dtype=torch.float32, device="cuda")
+        self.bound = torch.empty((B, NQ, HQ), dtype=torch.float32, device="cuda")
+        self.flags = torch.empty((B, NQ, HQ), dtype=torch.uint8, device="cuda")
+        self.stream = torch.cuda.current_stream()
+        s = self.stream.cuda_stream
+        L = kvq.lib()
+        self.L = L
+        dt = kvq.KVQ_BF16 if self.kd.dtype == torch.bfloat16 else kvq.KVQ_F32
+        qdt = kvq.KVQ_BF16 if self.qd.dtype == torch.bfloat16 else kvq.KVQ_F32
+        kn, vn = self.k_new, self.v_new
+        self.append_args = [
+            (ctypes.byref(c.desc), kn.data_ptr(), vn.data_ptr(), dt, kn.stride(0), kn.stride(1),
+             kn.stride(2), wl.num_seqs, 1, None, self.new_pos.data_ptr(), self.pt.data_ptr(),
+             self.pt.shape[1], s) for c in self.caches]
+        self.decode_args = [
+            (ctypes.byref(c.desc), self.qd.data_ptr(), qdt, B, NQ, HQ, self.pt.data_ptr(),
+             self.pt.shape[1], self.sl.data_ptr(), 0.0, wl.tau, self.out.data_ptr(),
+             self.bound.data_ptr(), self.flags.data_ptr(), w.data_ptr(), w.numel(), s)
+            for c, w in zip(self.caches, self.ws)]
+        self.token_heads = int(sum(inp.seq_lens)) * wl.num_kv_heads
+        bb = base.block_bytes
+        self.decode_bytes = (sum(inp.seq_lens) * wl.num_kv_heads * bb // 16
+                             + sum(inp.pages_per_seq) * wl.num_kv_heads * 4)
+        self.cache_bytes = inp.num_pages * wl.num_kv_heads * bb
+        self.replicas = replicas
+        self.launches_per_step = 2
+
+    def step(self, i, ev=None):
+        r = i % self.replicas
+        rc = self.L.kvq_quantize_append(*self.append_args[r])
+        if rc:
+            raise RuntimeError(self.kvq.last_error())
+        if ev is not None:
+            ev[0].record(self.stream)
+        rc = self.L.kvq_decode_attention(*self.decode_args[r])
+        if rc:
+            raise RuntimeError(self.kvq.last_error())
+        if ev is not None:
+            ev[1].record(self.stream)
+
+
+def run_gpu(args):
+    import torch
+    rank, world, local = _dist_setup(args.gpus)
+    wl = synth.WORKLOADS[args.workload]
+    reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl))))
+    reps = min(reps, 8)
+    st = GpuStep(args.workload, args.seed, reps)
+    for i in range(args.warmup):
+        st.step(i)
+    torch.cuda.synchronize()
+    err = st.caches[0].device_error()
+    if err:
+        raise RuntimeError(f"device error {err} during warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local) if rank == 0 else None
+    _barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t0.record()
+    for i in range(args.steps):
+        st.step(args.warmup + i, evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    _barrier(world)
+    ms_total = t0.elapsed_time(t1)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    ms_total = _max_over_ranks(ms_total, world)
+    dec_ms = _max_over_ranks(dec_ms, world)
+    ms_step = ms_total / args.steps
+
+    # end to end through the public API with host buffers: H2D of the step's inputs
+    # (q and the new K/V token) from pinned memory, the two calls, D2H of the results
+    q_h = st.qd.cpu().pin_memory()
+    kn_h = st.k_new.cpu().pin_memory()
+    vn_h = st.v_new.cpu().pin_memory()
+    out_h = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
+    bound_h = torch.empty(st.bound.shape, dtype=torch.float32).pin_memory()
+    flags_h = torch.empty(st.flags.shape, dtype=torch.uint8).pin_memory()
+    h2d = q_h.numel() * q_h.element_size() + 2 * kn_h.numel() * kn_h.element_size()
+    d2h = out_h.numel() * 4 + bound_h.numel() * 4 + flags_h.numel()
+    e_steps = max(1, args.steps)
+    _barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e_steps):
+        st.qd.copy_(q_h, non_blocking=True)
+        st.k_new.copy_(kn_h, non_blocking=True)
+        st.v_new.copy_(vn_h, non_blocking=True)
+        st.step(i)
+        out_h.copy_(st.out, non_blocking=True)
+        bound_h.copy_(st.bound, non_blocking=True)
+        flags_h.copy_(st.flags, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e_steps, world)
+
+    peak, peak_kind = _peaks()
+    achieved = st.decode_bytes / (dec_ms * 1e-3) / 1e9
+    traffic = _traffic_record()
+    res = {
+        "metric": METRIC,
+        "value": st.token_heads * world / (ms_step * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8xs8->s32 (QK), f16xf16->f32 (PV), f32 softmax/bound",
+        "data": "synthetic (seeded N(0,1) bf16 + outlier channels, as the workload states)",
+        "config": {"workload": _workload_desc(wl),
+                   "l2": f"inputs larger than L2: {reps} cache replicas of "
+                         f"{st.cache_bytes / 1e6:.1f} MB rotated per step",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "token_heads_per_step": st.token_heads,
+                   "decode_bytes_per_launch": st.decode_bytes},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} copy bandwidth",
+                     "kernel": "decode_mma_kernel", "kernel_ms": dec_ms},
+        "e2e": {"value": st.token_heads * world / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": st.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(args.workload, args.seed, args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def _cache_bytes_estimate(wl) -> int:
+    per_tok = wl.head_dim * wl.k_bits // 8 + wl.head_dim // 2 + 2 * wl.head_dim // wl.k_group \
+        + 4 * wl.head_dim // 32
+    ctx = wl.ctx if wl.ctx_min is None else (wl.ctx + wl.ctx_min) // 2
+    return wl.num_seqs * ctx * wl.num_kv_heads * per_tok
+
+
+# ------------------------------------------------------------------------- CPU --
+def _oracle_setup(workload: str, seed: int, kv_heads=None):
+    """The oracle's cache of sequence 0 of the workload; rows of the given kv heads."""
+    import oracle
+    inp = synth.make(workload, seed)
+    wl = inp.wl
+    c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
+                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+    k, v = inp.kv_seq(0)
+    pt = inp.page_table[:1]
+    sl = np.array(inp.seq_lens[:1], np.int32)
+    rc = c.append(k[None], v[None], pt, np.zeros(1, np.int32), valid=sl)
+    assert rc == 0
+    q = inp.q()[:1]
+    heads = range(wl.num_kv_heads) if kv_heads is None else kv_heads
+    mask = np.zeros((1, wl.num_queries, wl.num_q_heads), np.uint8)
+    for h in heads:
+        mask[:, :, h * wl.group:(h + 1) * wl.group] = 1
+    return inp, c, q, pt, sl, mask.reshape(-1), len(list(heads))
+
+
+def cpu_baseline(workload: str, seed: int, seconds: float):
+    """The oracle's decode (fp64 attention + bound over the quantized cache), single
+    thread, on whole sequences of the workload until about `seconds` of CPU work."""
+    inp, c, q, pt, sl, mask, nh = _oracle_setup(workload, seed)
+    wl = inp.wl
+    th = int(sl.sum()) * nh
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        c.decode(q, pt, sl, tau=wl.tau, row_mask=mask)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 1000:
+            break
+    return {"value": th * reps / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"sequence 0 of {wl.name} ({int(sl[0])} tokens x {wl.num_kv_heads} kv "
+                      f"heads x {wl.num_q_heads} q heads), decode + bound, {reps} repeat(s), "
+                      f"{el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = synth.WORKLOADS[args.workload]
+    inp, c, q, pt, sl, mask, nh = _oracle_setup(args.workload, args.seed, [0])
+    th = int(sl.sum()) * nh
+    for _ in range(args.warmup):
+        c.decode(q, pt, sl, tau=wl.tau, row_mask=mask)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        c.decode(q, pt, sl, tau=wl.tau, row_mask=mask)
+    el = time.perf_counter() - t0
+    ms = el * 1e3 / max(1, args.steps)
+    value = th / (ms * 1e-3)
+    res = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64 (attention, bound), f32 (codec)",
+        "data": "synthetic",
+        "config": {"workload": _workload_desc(wl),
+                   "sample": f"each step: kv head 0 of sequence 0 ({int(sl[0])} tokens, "
+                             f"{wl.group * wl.num_queries} query rows) of the workload"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "kv head 0 of sequence 0 of the workload per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,194 @@
+/*
+ * kvq.h -- C ABI of the B200 quantized-KV decode-attention library (libkvq.so).
+ *
+ * The operations follow the tiered, runtime-certified quantized attention of
+ * "Runtime-Certified Bounded-Error Quantized Attention":
+ *   - Methodology 1 (Tiered storage): Tier 1 in GPU memory holds INT8 (or
+ *     INT4) key codes and per-group INT4 value codes with scale/offset
+ *     metadata and a per-block error annotation eta_b; Tier 2 in pinned host
+ *     memory holds the unquantized originals.
+ *   - Methodology 2 (Two-term error decomposition): per query, a bound
+ *     E_key + E_val on the error of the quantized attention output, computed
+ *     online from the quantization scales, the query norms and the value
+ *     range, without touching the originals.
+ *   - Methodology 1 (Fallback) / 3 (ladder, per-head rung): a query whose
+ *     bound exceeds tau is recomputed as exact dense attention from Tier 2.
+ * and the rotated-key codec of "Statistical Inference and Quality Measures of
+ * KV Cache Quantisations Inspired by TurboQuant" (Quantisation schemes, KQV:
+ * Walsh-Hadamard transform before scalar quantization of K).
+ *
+ * Conventions
+ *   - Every pointer is caller-owned; the library never allocates or frees
+ *     memory and keeps no state between calls except a cache of TMA
+ *     descriptors and of device properties.  "device" = CUDA device memory
+ *     (or managed), "host" = host memory, "pinned" = page-locked host memory.
+ *   - Every call validates its arguments before launching anything and
+ *     returns a kvq_status (0 = KVQ_OK); no exception crosses the ABI.
+ *     kvq_last_error() gives a message for the last failure on this thread.
+ *   - All calls are asynchronous on the given stream except
+ *     kvq_fallback_exact and kvq_device_error, which wait (with a deadline).
+ *   - Calls on distinct streams with distinct output/workspace buffers are
+ *     independent.  Only devices of compute capability 10.0 (sm_100a) run
+ *     the kernels.
+ *
+ * Quantized cache layout (one block per physical page and kv head, 16 tokens;
+ * nb = head_dim/32):
+ *   [K codes 16*head_dim*k_bits/8 B][V codes 16*head_dim/2 B]
+ *   [K scales fp16 [16][head_dim/k_group]][V (scale, zero) fp16 [16][nb][2]]
+ *   K code of channel c (b = c/32, w = c%32, s = w/8, i = w%8) in a token row:
+ *     8 bit: byte s*8*nb + 8*b + i (int8);
+ *     4 bit: byte s*4*nb + 4*b + i/2, low nibble for even c (4-bit two's complement).
+ *   V code of channel c (g = c/32, w = c%32): byte (w/4)*2*nb + 2*g + (w%4)/2,
+ *     low nibble for even c (unsigned).
+ *   Key codec per token and k_group channels: s = fp16 rounded up of
+ *   max|x|/Q (Q = 127 or 7), code = rint(x/s) in [-Q, Q].  Value codec per
+ *   token and 32 channels: z = fp16 rounded down of min x, s = fp16 rounded up
+ *   of (max x - z)/15, code = rint((x - z)/s) in [0, 15].
+ *   eta[page][kv_head] = max over the block's tokens of |v - fmaf(code, s, z)|,
+ *   rounded up by one fp32 ulp.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* kvq_stream_t;
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = -1, /* null pointer, bad size, layout or stride */
+  KVQ_ERR_UNSUPPORTED = -2, /* valid but unsupported shape (head_dim, group, rows) */
+  KVQ_ERR_RANGE = -3,       /* non-finite input or fp16-overflowing scale/zero */
+  KVQ_ERR_CUDA = -4,        /* a CUDA runtime call failed */
+  KVQ_ERR_TIMEOUT = -5,     /* a bounded host wait gave up */
+  KVQ_ERR_DEVICE = -6       /* a kernel reported an error (see kvq_device_error) */
+} kvq_status;
+
+typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
+
+#define KVQ_PAGE_SIZE 16
+
+typedef struct kvq_cache {
+  int32_t num_kv_heads;    /* Hkv >= 1 */
+  int32_t head_dim;        /* d: 64 or 128 */
+  int32_t page_size;       /* tokens per page: must be 16 */
+  int32_t num_pages;       /* physical pages in the pool */
+  int32_t k_bits;          /* 8 or 4 */
+  int32_t k_group;         /* 32, 64 or 128, divides head_dim */
+  int32_t k_rotate;        /* 1: keys (and queries) get the randomized Hadamard rotation */
+  int32_t v_bits;          /* must be 4 */
+  int32_t v_group;         /* must be 32 */
+  void* pool;              /* device, kvq_pool_bytes() bytes, 16-byte aligned */
+  float* v_eta;            /* device, [num_pages][num_kv_heads]; zero before a page's first append */
+  const int8_t* rot_signs; /* device, head_dim entries of +1/-1; required iff k_rotate */
+  int32_t* error_word;     /* device, one int32 kernels set to a kvq_status on error; may be NULL */
+} kvq_cache;
+
+/* Bytes of one (page, kv head) block, and of the whole pool; 0 if the cache
+ * description is invalid or unsupported. */
+KVQ_API size_t kvq_block_bytes(const kvq_cache* cache);
+KVQ_API size_t kvq_pool_bytes(const kvq_cache* cache);
+
+/* Quantize-on-append (Methodology 1, Tier 1).
+ * Token t < valid_tokens[s] (or < num_tokens when valid_tokens is NULL) of
+ * sequence s is written at logical position start_pos[s] + t, i.e. into
+ * physical page page_table[s*max_pages_per_seq + pos/16], slot pos%16, of
+ * every kv head.  k, v (device, in_dtype) element (s, h, t, c) is at
+ * s*seq_stride + h*head_stride + t*token_stride + c (strides in elements;
+ * channels contiguous).  page_table, start_pos, valid_tokens: device int32.
+ * eta of the touched blocks is raised with an atomic max, so eta of a reused
+ * page must be zeroed by the caller first.  A non-finite input or an
+ * fp16-overflowing scale writes zero codes and scale for that group and sets
+ * *error_word = KVQ_ERR_RANGE; a page index outside [0, num_pages) skips the
+ * token and sets KVQ_ERR_INVALID_ARG.  Asynchronous on `stream`. */
+KVQ_API int kvq_quantize_append(const kvq_cache* cache, const void* k, const void* v, int in_dtype,
+                        int64_t seq_stride, int64_t head_stride, int64_t token_stride,
+                        int32_t num_seqs, int32_t num_tokens, const int32_t* valid_tokens,
+                        const int32_t* start_pos, const int32_t* page_table,
+                        int32_t max_pages_per_seq, kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attention / kvq_error_bound need for this shape
+ * on the current device (split-K partials and per-(sequence, kv head)
+ * counters).  The workspace must be zero-filled once before its first use;
+ * every call leaves its counters at zero again.  Returns 0 on invalid input. */
+KVQ_API size_t kvq_workspace_size(const kvq_cache* cache, int32_t num_seqs, int32_t num_queries,
+                          int32_t num_q_heads, int32_t max_pages_per_seq);
+
+/* Quantized decode attention with the certified bound (Methodology 2).
+ * q (device, q_dtype) [num_seqs][num_queries][num_q_heads][head_dim]; q head h
+ * attends kv head h / (num_q_heads/num_kv_heads) over tokens [0, seq_lens[s])
+ * of its sequence (no mask inside the context).  num_queries *
+ * (num_q_heads/num_kv_heads) must be <= 4.  softmax_scale <= 0 selects
+ * 1/sqrt(head_dim).  Writes (device) out fp32 [..][head_dim] (quantized-path
+ * attention), bound fp32 [num_seqs][num_queries][num_q_heads] (a certified
+ * upper bound on max_c |o_exact - out| against exact attention over the
+ * originals) and flags uint8 (bound > tau; tau = INFINITY never flags).
+ * An empty context gives out = 0, bound = 0, flag = 0.  page_table and
+ * seq_lens: device int32.  Page indices outside the pool set
+ * *error_word = KVQ_ERR_INVALID_ARG and that page is skipped.  workspace:
+ * device, >= kvq_workspace_size() bytes, 16-byte aligned.  Asynchronous. */
+KVQ_API int kvq_decode_attention(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
+                         int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
+                         int32_t max_pages_per_seq, const int32_t* seq_lens,
+                         float softmax_scale, float tau, float* out, float* bound,
+                         uint8_t* flags, void* workspace, size_t workspace_bytes,
+                         kvq_stream_t stream);
+
+/* The certified bound and flags alone: the same pass as
+ * kvq_decode_attention without writing attention outputs. */
+KVQ_API int kvq_error_bound(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
+                    int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
+                    int32_t max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
+                    float tau, float* bound, uint8_t* flags, void* workspace,
+                    size_t workspace_bytes, kvq_stream_t stream);
+
+/* Staging bytes kvq_fallback_exact needs to recompute one (sequence, kv head)
+ * of up to max_ctx tokens (the minimum; more lets it batch several). */
+KVQ_API size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype, int32_t max_ctx);
+
+/* Exact recomputation from Tier 2 (Methodology 1, Fallback; per-head rung of
+ * the ladder, applied per query).  Waits on `main` for the decode that wrote
+ * `flags` (device uint8, same shape as bound), copies them to flags_host
+ * (pinned, num_seqs*num_queries*num_q_heads bytes) on `side`, and polls with
+ * a deadline of timeout_ms (KVQ_ERR_TIMEOUT when it passes; 0 times out at
+ * once).  For every (sequence, kv head) with a flagged query it copies the
+ * originals k_orig_host, v_orig_host (pinned, orig_dtype, element (s, h, t, c)
+ * at s*orig_seq_stride + h*orig_head_stride + t*head_dim + c) for tokens
+ * [0, seq_lens_host[s]) into `staging` (device) with cudaMemcpyAsync on
+ * `side`, and overwrites out rows of the flagged queries with exact fp32
+ * softmax attention (softmax_scale as in decode).  q as in decode.  `main`
+ * then waits for `side`.  *num_fallback (host) = number of recomputed
+ * queries.  On any error out is left unmodified for the rows not yet
+ * recomputed.  Blocks the calling thread until the flags are on the host. */
+KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const void* v_orig_host,
+                       int orig_dtype, int64_t orig_seq_stride, int64_t orig_head_stride,
+                       const void* q, int q_dtype, int32_t num_seqs, int32_t num_queries,
+                       int32_t num_q_heads, const int32_t* seq_lens_host, float softmax_scale,
+                       const uint8_t* flags, uint8_t* flags_host, float* out, void* staging,
+                       size_t staging_bytes, kvq_stream_t main_stream,
+                       kvq_stream_t side_stream, int32_t timeout_ms, int32_t* num_fallback);
+
+/* Waits for `stream`, reads *cache->error_word into *code (KVQ_OK when no
+ * kernel reported an error) and resets it to KVQ_OK. */
+KVQ_API int kvq_device_error(const kvq_cache* cache, kvq_stream_t stream, int32_t* code);
+
+KVQ_API const char* kvq_status_string(int status);
+KVQ_API const char* kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

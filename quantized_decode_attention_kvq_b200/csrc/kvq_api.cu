@@ -1,0 +1,561 @@
+// kvq_api.cu -- the C ABI (include/kvq.h): argument validation, status codes,
+// launch planning (split-K sizing against the SM count and occupancy), TMA
+// descriptor encoding, and the host orchestration of the exact fallback
+// (flag read-back with a bounded wait, Tier-2 page-in with cudaMemcpyAsync on
+// a side stream, recomputation kernel, stream hand-back).
+#include <cudaTypedefs.h>
+
+#include <chrono>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <thread>
+#include <tuple>
+#include <vector>
+
+#include "kvq_internal.cuh"
+
+using namespace kvq;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return status;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_cache(const kvq_cache* c) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+  if (c->page_size != KVQ_PAGE_SIZE) return fail(KVQ_ERR_UNSUPPORTED, "page_size must be 16");
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", c->head_dim);
+  if (c->k_bits != 8 && c->k_bits != 4)
+    return fail(KVQ_ERR_UNSUPPORTED, "k_bits %d unsupported (8 or 4)", c->k_bits);
+  if (c->k_group != 32 && c->k_group != 64 && c->k_group != 128)
+    return fail(KVQ_ERR_UNSUPPORTED, "k_group %d unsupported (32, 64, 128)", c->k_group);
+  if (c->head_dim % c->k_group)
+    return fail(KVQ_ERR_UNSUPPORTED, "k_group %d does not divide head_dim %d", c->k_group,
+                c->head_dim);
+  if (c->v_bits != 4 || c->v_group != 32)
+    return fail(KVQ_ERR_UNSUPPORTED, "values must be 4-bit with group 32");
+  if (c->num_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "num_kv_heads < 1");
+  if (c->num_pages < 0) return fail(KVQ_ERR_INVALID_ARG, "num_pages < 0");
+  if (c->k_rotate != 0 && c->k_rotate != 1) return fail(KVQ_ERR_INVALID_ARG, "k_rotate not 0/1");
+  if (c->k_rotate && !c->rot_signs) return fail(KVQ_ERR_INVALID_ARG, "k_rotate needs rot_signs");
+  if (!c->pool || !c->v_eta) return fail(KVQ_ERR_INVALID_ARG, "pool or v_eta is NULL");
+  if (!aligned16(c->pool)) return fail(KVQ_ERR_INVALID_ARG, "pool not 16-byte aligned");
+  return KVQ_OK;
+}
+
+BlockLayout layout_of(const kvq_cache* c) { return BlockLayout{c->head_dim, c->k_bits, c->k_group}; }
+
+float rot_constant(int d) { return (float)(1.0 / std::sqrt((double)d)); }
+
+struct DeviceInfo {
+  int sms = 0, major = 0, max_smem = 0;
+};
+
+int device_info(DeviceInfo* out, int* dev_out) {
+  static std::mutex mu;
+  static std::map<int, DeviceInfo> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(dev);
+  if (it == cache.end()) {
+    DeviceInfo di;
+    if ((e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    if ((e = cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev)) !=
+        cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    if ((e = cudaDeviceGetAttribute(&di.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                    dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    it = cache.emplace(dev, di).first;
+  }
+  *out = it->second;
+  if (dev_out) *dev_out = dev;
+  if (out->major != 10)
+    return fail(KVQ_ERR_UNSUPPORTED, "device %d has compute capability %d.x; sm_100a required",
+                dev, out->major);
+  return KVQ_OK;
+}
+
+// blocks of the decode kernel resident per SM (after opting into its shared memory)
+int decode_occupancy(const DecodeVariant& v, int* occ) {
+  static std::mutex mu;
+  static std::map<std::pair<int, void*>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto key = std::make_pair(dev, reinterpret_cast<void*>(v.kernel));
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(v.kernel),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reinterpret_cast<const void*>(v.kernel),
+                                                      decode_threads(), v.smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (n < 1) n = 1;
+    it = cache.emplace(key, n).first;
+  }
+  *occ = it->second;
+  return KVQ_OK;
+}
+
+struct Plan {
+  int splits = 1, pps = 1;
+  size_t part_bytes = 0, counter_bytes = 0;
+  size_t total() const { return counter_bytes + part_bytes; }
+};
+
+constexpr int kMaxPagesPerSplit = 128;
+
+// Split-K sizing: fill every SM's resident slots once with (sequence, kv head,
+// split) CTAs; long contexts cap the pages of one split so a ragged batch
+// spreads over several waves.
+int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
+  DecodeVariant v = select_decode_kernel(c->head_dim, c->k_bits, c->k_group);
+  if (!v.kernel) return fail(KVQ_ERR_UNSUPPORTED, "no decode kernel for this codec");
+  DeviceInfo di;
+  int rc = device_info(&di, nullptr);
+  if (rc) return rc;
+  int occ = 1;
+  if ((rc = decode_occupancy(v, &occ))) return rc;
+  const int64_t units = (int64_t)num_seqs * c->num_kv_heads;
+  const int64_t slots = (int64_t)di.sms * occ;
+  int64_t splits = units > 0 ? std::max<int64_t>(1, slots / units) : 1;
+  int64_t pps = (max_pages + splits - 1) / splits;
+  if (pps > kMaxPagesPerSplit) pps = kMaxPagesPerSplit;
+  // KVQ_PAGES_PER_SPLIT overrides the split size (tuning and tests)
+  if (const char* env = std::getenv("KVQ_PAGES_PER_SPLIT")) {
+    const long o = std::strtol(env, nullptr, 10);
+    if (o > 0) pps = o;
+  }
+  if (pps < 1) pps = 1;
+  splits = (max_pages + pps - 1) / pps;
+  if (splits < 1) splits = 1;
+  p->splits = (int)splits;
+  p->pps = (int)pps;
+  p->counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
+  p->part_bytes = (size_t)units * splits * v.record * sizeof(float);
+  return KVQ_OK;
+}
+
+// TMA descriptor of the K-code tiles: 3-D {row bytes, 16 rows, page x kv head}.
+int key_tensor_map(const kvq_cache* c, CUtensorMap* out) {
+  static std::mutex mu;
+  static std::map<std::tuple<void*, int, int, int, int, int>, CUtensorMap> cache;
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  const BlockLayout L = layout_of(c);
+  std::lock_guard<std::mutex> lk(mu);
+  auto key = std::make_tuple(c->pool, c->num_pages, c->num_kv_heads, c->head_dim, c->k_bits,
+                             c->k_group);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *out = it->second;
+    return KVQ_OK;
+  }
+  if (!encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+      return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  CUtensorMap m;
+  const int row = L.k_row();
+  cuuint64_t dims[3] = {(cuuint64_t)row, (cuuint64_t)kPage,
+                        (cuuint64_t)c->num_pages * (cuuint64_t)c->num_kv_heads};
+  cuuint64_t strides[2] = {(cuuint64_t)row, (cuuint64_t)L.bytes()};
+  cuuint32_t box[3] = {(cuuint32_t)row, (cuuint32_t)kPage, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, c->pool, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  cache.emplace(key, m);
+  *out = m;
+  return KVQ_OK;
+}
+
+int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
+                int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
+                int32_t max_pages, const int32_t* seq_lens, float softmax_scale, float tau,
+                float* out, float* bound, uint8_t* flags, void* ws, size_t ws_bytes,
+                cudaStream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (num_seqs < 0 || num_queries < 1 || num_q_heads < 1 || max_pages < 1)
+    return fail(KVQ_ERR_INVALID_ARG, "bad sizes (num_seqs %d, num_queries %d, num_q_heads %d, "
+                "max_pages_per_seq %d)", num_seqs, num_queries, num_q_heads, max_pages);
+  if (num_q_heads % cache->num_kv_heads)
+    return fail(KVQ_ERR_INVALID_ARG, "num_q_heads %d not a multiple of num_kv_heads %d",
+                num_q_heads, cache->num_kv_heads);
+  const int G = num_q_heads / cache->num_kv_heads;
+  if ((int64_t)num_queries * G > 4)
+    return fail(KVQ_ERR_UNSUPPORTED, "num_queries * (num_q_heads/num_kv_heads) = %d > 4",
+                num_queries * G);
+  if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad q_dtype");
+  if (num_seqs == 0) return KVQ_OK;
+  if (!q || !page_table || !seq_lens || !bound || !flags)
+    return fail(KVQ_ERR_INVALID_ARG, "NULL q, page_table, seq_lens, bound or flags");
+  if (std::isnan(tau)) return fail(KVQ_ERR_INVALID_ARG, "tau is NaN");
+  Plan plan;
+  if ((rc = make_plan(cache, num_seqs, max_pages, &plan))) return rc;
+  if (!ws || ws_bytes < plan.total())
+    return fail(KVQ_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", ws_bytes,
+                plan.total());
+  if (!aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");
+  DecodeVariant v = select_decode_kernel(cache->head_dim, cache->k_bits, cache->k_group);
+  CUtensorMap kmap;
+  if ((rc = key_tensor_map(cache, &kmap))) return rc;
+  DecodeArgs a;
+  a.pool = static_cast<const uint8_t*>(cache->pool);
+  a.eta = cache->v_eta;
+  a.signs = cache->k_rotate ? cache->rot_signs : nullptr;
+  a.err = cache->error_word;
+  a.q = q;
+  a.q_bf16 = q_dtype == KVQ_BF16;
+  a.page_table = page_table;
+  a.max_pages = max_pages;
+  a.seq_lens = seq_lens;
+  a.num_seqs = num_seqs;
+  a.nq = num_queries;
+  a.hq = num_q_heads;
+  a.hkv = cache->num_kv_heads;
+  a.G = G;
+  a.R = num_queries * G;
+  a.num_pages = cache->num_pages;
+  a.pps = plan.pps;
+  a.s_att = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)cache->head_dim));
+  a.tau = tau;
+  a.rot_c = rot_constant(cache->head_dim);
+  a.out = out;
+  a.bound = bound;
+  a.flags = flags;
+  a.counters = static_cast<int*>(ws);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.counter_bytes);
+  dim3 grid(plan.splits, cache->num_kv_heads, num_seqs);
+  if (grid.y > 65535 || grid.z > 65535)
+    return fail(KVQ_ERR_UNSUPPORTED, "grid too large (kv heads %d, sequences %d)", grid.y, grid.z);
+  v.kernel<<<grid, decode_threads(), v.smem, stream>>>(a, kmap);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  return KVQ_OK;
+}
+
+bool fault_injected(const char* what) {
+  const char* f = std::getenv("KVQ_FAULT");
+  return f && std::strcmp(f, what) == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_status_string(int s) {
+  switch (s) {
+    case KVQ_OK: return "KVQ_OK";
+    case KVQ_ERR_INVALID_ARG: return "KVQ_ERR_INVALID_ARG";
+    case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
+    case KVQ_ERR_RANGE: return "KVQ_ERR_RANGE";
+    case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+    case KVQ_ERR_TIMEOUT: return "KVQ_ERR_TIMEOUT";
+    case KVQ_ERR_DEVICE: return "KVQ_ERR_DEVICE";
+    default: return "KVQ_UNKNOWN_STATUS";
+  }
+}
+
+const char* kvq_last_error(void) { return g_last_error.c_str(); }
+
+size_t kvq_block_bytes(const kvq_cache* cache) {
+  if (!cache || cache->page_size != KVQ_PAGE_SIZE) return 0;
+  if ((cache->head_dim != 64 && cache->head_dim != 128) || (cache->k_bits != 8 && cache->k_bits != 4))
+    return 0;
+  if (cache->k_group != 32 && cache->k_group != 64 && cache->k_group != 128) return 0;
+  if (cache->head_dim % cache->k_group || cache->v_bits != 4 || cache->v_group != 32) return 0;
+  return (size_t)layout_of(cache).bytes();
+}
+
+size_t kvq_pool_bytes(const kvq_cache* cache) {
+  const size_t bb = kvq_block_bytes(cache);
+  if (!bb || cache->num_pages < 0 || cache->num_kv_heads < 1) return 0;
+  return bb * (size_t)cache->num_pages * (size_t)cache->num_kv_heads;
+}
+
+int kvq_quantize_append(const kvq_cache* cache, const void* k, const void* v, int in_dtype,
+                        int64_t seq_stride, int64_t head_stride, int64_t token_stride,
+                        int32_t num_seqs, int32_t num_tokens, const int32_t* valid_tokens,
+                        const int32_t* start_pos, const int32_t* page_table,
+                        int32_t max_pages_per_seq, kvq_stream_t stream) {
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad in_dtype");
+  if (num_seqs < 0 || num_tokens < 0 || max_pages_per_seq < 1)
+    return fail(KVQ_ERR_INVALID_ARG, "bad sizes");
+  if (num_seqs == 0 || num_tokens == 0) return KVQ_OK;
+  if (!k || !v || !start_pos || !page_table)
+    return fail(KVQ_ERR_INVALID_ARG, "NULL k, v, start_pos or page_table");
+  if (seq_stride < 0 || head_stride < 0 || token_stride < 0)
+    return fail(KVQ_ERR_INVALID_ARG, "negative stride");
+  DeviceInfo di;
+  if ((rc = device_info(&di, nullptr))) return rc;
+  AppendArgs a;
+  a.pool = static_cast<uint8_t*>(cache->pool);
+  a.eta = cache->v_eta;
+  a.signs = cache->k_rotate ? cache->rot_signs : nullptr;
+  a.err = cache->error_word;
+  a.k = k;
+  a.v = v;
+  a.in_bf16 = in_dtype == KVQ_BF16;
+  a.seq_stride = seq_stride;
+  a.head_stride = head_stride;
+  a.tok_stride = token_stride;
+  a.num_seqs = num_seqs;
+  a.num_tokens = num_tokens;
+  a.hkv = cache->num_kv_heads;
+  a.num_pages = cache->num_pages;
+  a.max_pages = max_pages_per_seq;
+  a.valid = valid_tokens;
+  a.start_pos = start_pos;
+  a.page_table = page_table;
+  a.rot_c = rot_constant(cache->head_dim);
+  cudaError_t e = launch_append(a, cache->head_dim, cache->k_bits, cache->k_group,
+                                reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+  return KVQ_OK;
+}
+
+size_t kvq_workspace_size(const kvq_cache* cache, int32_t num_seqs, int32_t num_queries,
+                          int32_t num_q_heads, int32_t max_pages_per_seq) {
+  if (check_cache(cache) || num_seqs < 0 || num_queries < 1 || num_q_heads < 1 ||
+      max_pages_per_seq < 1)
+    return 0;
+  Plan p;
+  if (make_plan(cache, num_seqs, max_pages_per_seq, &p)) return 0;
+  return p.total();
+}
+
+int kvq_decode_attention(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
+                         int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
+                         int32_t max_pages_per_seq, const int32_t* seq_lens,
+                         float softmax_scale, float tau, float* out, float* bound,
+                         uint8_t* flags, void* workspace, size_t workspace_bytes,
+                         kvq_stream_t stream) {
+  if (!out && num_seqs > 0) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+  return decode_impl(cache, q, q_dtype, num_seqs, num_queries, num_q_heads, page_table,
+                     max_pages_per_seq, seq_lens, softmax_scale, tau, out, bound, flags,
+                     workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int kvq_error_bound(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
+                    int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
+                    int32_t max_pages_per_seq, const int32_t* seq_lens, float softmax_scale,
+                    float tau, float* bound, uint8_t* flags, void* workspace,
+                    size_t workspace_bytes, kvq_stream_t stream) {
+  return decode_impl(cache, q, q_dtype, num_seqs, num_queries, num_q_heads, page_table,
+                     max_pages_per_seq, seq_lens, softmax_scale, tau, nullptr, bound, flags,
+                     workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype, int32_t max_ctx) {
+  if (!cache || (cache->head_dim != 64 && cache->head_dim != 128) || max_ctx < 0) return 0;
+  if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return 0;
+  const size_t es = orig_dtype == KVQ_BF16 ? 2 : 4;
+  const size_t one = ((size_t)max_ctx * cache->head_dim * es + 255) / 256 * 256;
+  return 2 * (one > 0 ? one : 256);
+}
+
+int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const void* v_orig_host,
+                       int orig_dtype, int64_t orig_seq_stride, int64_t orig_head_stride,
+                       const void* q, int q_dtype, int32_t num_seqs, int32_t num_queries,
+                       int32_t num_q_heads, const int32_t* seq_lens_host, float softmax_scale,
+                       const uint8_t* flags, uint8_t* flags_host, float* out, void* staging,
+                       size_t staging_bytes, kvq_stream_t main_stream, kvq_stream_t side_stream,
+                       int32_t timeout_ms, int32_t* num_fallback) {
+  if (num_fallback) *num_fallback = 0;
+  if (!cache) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->head_dim != 64 && cache->head_dim != 128)
+    return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d unsupported", cache->head_dim);
+  if (cache->num_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "num_kv_heads < 1");
+  if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad orig_dtype");
+  if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad q_dtype");
+  if (num_seqs < 0 || num_queries < 1 || num_q_heads < 1 || num_q_heads % cache->num_kv_heads)
+    return fail(KVQ_ERR_INVALID_ARG, "bad sizes");
+  if (num_seqs == 0) return KVQ_OK;
+  if (!k_orig_host || !v_orig_host || !q || !seq_lens_host || !flags || !flags_host || !out ||
+      !staging || !num_fallback)
+    return fail(KVQ_ERR_INVALID_ARG, "NULL argument");
+  if (orig_seq_stride < 0 || orig_head_stride < 0) return fail(KVQ_ERR_INVALID_ARG, "negative stride");
+  DeviceInfo di;
+  int rc = device_info(&di, nullptr);
+  if (rc) return rc;
+  const int D = cache->head_dim, hkv = cache->num_kv_heads, G = num_q_heads / hkv;
+  const size_t es = orig_dtype == KVQ_BF16 ? 2 : 4;
+  int32_t max_n = 0;
+  for (int s = 0; s < num_seqs; ++s) {
+    if (seq_lens_host[s] < 0) return fail(KVQ_ERR_INVALID_ARG, "negative seq_len");
+    max_n = std::max(max_n, seq_lens_host[s]);
+  }
+  if (staging_bytes < kvq_fallback_staging_size(cache, orig_dtype, max_n))
+    return fail(KVQ_ERR_INVALID_ARG, "staging %zu bytes < %zu required", staging_bytes,
+                kvq_fallback_staging_size(cache, orig_dtype, max_n));
+  cudaStream_t ms = reinterpret_cast<cudaStream_t>(main_stream);
+  cudaStream_t ss = reinterpret_cast<cudaStream_t>(side_stream);
+  const size_t rows = (size_t)num_seqs * num_queries * num_q_heads;
+
+  cudaEvent_t ev_dec = nullptr, ev_flags = nullptr, ev_done = nullptr;
+  auto cleanup = [&]() {
+    if (ev_dec) cudaEventDestroy(ev_dec);
+    if (ev_flags) cudaEventDestroy(ev_flags);
+    if (ev_done) cudaEventDestroy(ev_done);
+  };
+  cudaError_t e;
+  if ((e = cudaEventCreateWithFlags(&ev_dec, cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&ev_flags, cudaEventDisableTiming)) != cudaSuccess ||
+      (e = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming)) != cudaSuccess) {
+    cleanup();
+    return cuda_fail(e, "cudaEventCreate");
+  }
+  // flags -> host on the side stream, after the decode on the main stream
+  if ((e = cudaEventRecord(ev_dec, ms)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(ss, ev_dec, 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(flags_host, flags, rows, cudaMemcpyDeviceToHost, ss)) != cudaSuccess ||
+      (e = cudaEventRecord(ev_flags, ss)) != cudaSuccess) {
+    cleanup();
+    return cuda_fail(e, "flag read-back");
+  }
+  // bounded wait for the flags
+  {
+    const auto t0 = std::chrono::steady_clock::now();
+    for (;;) {
+      const double ms_el =
+          std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
+      if (ms_el >= (double)timeout_ms) {
+        cleanup();
+        return fail(KVQ_ERR_TIMEOUT, "flags not ready after %d ms", timeout_ms);
+      }
+      e = cudaEventQuery(ev_flags);
+      if (e == cudaSuccess) break;
+      if (e != cudaErrorNotReady) {
+        cleanup();
+        return cuda_fail(e, "cudaEventQuery");
+      }
+      std::this_thread::sleep_for(std::chrono::microseconds(20));
+    }
+  }
+  // page in and recompute, batching (sequence, kv head) units into the staging buffer
+  FbArgs fa;
+  std::memset(&fa, 0, sizeof(fa));
+  fa.staging = static_cast<const uint8_t*>(staging);
+  fa.q = q;
+  fa.q_bf16 = q_dtype == KVQ_BF16;
+  fa.kv_bf16 = orig_dtype == KVQ_BF16;
+  fa.s_att = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)D));
+  fa.out = out;
+  size_t used = 0;
+  int32_t count = 0;
+  auto flush = [&]() -> int {
+    if (fa.num_items == 0) return KVQ_OK;
+    cudaError_t le = launch_fallback(fa, D, ss);
+    if (le != cudaSuccess) return cuda_fail(le, "fallback kernel launch");
+    fa.num_items = 0;
+    used = 0;
+    return KVQ_OK;
+  };
+  for (int s = 0; s < num_seqs; ++s) {
+    for (int h = 0; h < hkv; ++h) {
+      std::vector<int64_t> rws;
+      for (int i = 0; i < num_queries; ++i)
+        for (int gq = 0; gq < G; ++gq) {
+          const int64_t row = ((int64_t)s * num_queries + i) * num_q_heads + h * G + gq;
+          if (flags_host[row]) rws.push_back(row);
+        }
+      if (rws.empty()) continue;
+      const int n = seq_lens_host[s];
+      const size_t one = ((size_t)n * D * es + 255) / 256 * 256;
+      if (used + 2 * one > staging_bytes || fa.num_items + (int)rws.size() > kFbMaxItems)
+        if ((rc = flush())) { cleanup(); return rc; }
+      const int64_t koff = (int64_t)used, voff = (int64_t)(used + one);
+      if (n > 0) {
+        if (fault_injected("memcpy")) {
+          cleanup();
+          return fail(KVQ_ERR_CUDA, "cudaMemcpyAsync failed (injected fault)");
+        }
+        const uint8_t* kh = static_cast<const uint8_t*>(k_orig_host) +
+                            ((int64_t)s * orig_seq_stride + (int64_t)h * orig_head_stride) * es;
+        const uint8_t* vh = static_cast<const uint8_t*>(v_orig_host) +
+                            ((int64_t)s * orig_seq_stride + (int64_t)h * orig_head_stride) * es;
+        if ((e = cudaMemcpyAsync(static_cast<uint8_t*>(staging) + koff, kh, (size_t)n * D * es,
+                                 cudaMemcpyHostToDevice, ss)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(static_cast<uint8_t*>(staging) + voff, vh, (size_t)n * D * es,
+                                 cudaMemcpyHostToDevice, ss)) != cudaSuccess) {
+          cleanup();
+          return cuda_fail(e, "cudaMemcpyAsync (Tier-2 page-in)");
+        }
+      }
+      used += 2 * one;
+      for (int64_t row : rws) {
+        FbItem& it = fa.items[fa.num_items++];
+        it.k_off = koff;
+        it.v_off = voff;
+        it.q_row = row;
+        it.n = n;
+        ++count;
+      }
+    }
+  }
+  if ((rc = flush())) { cleanup(); return rc; }
+  if ((e = cudaEventRecord(ev_done, ss)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(ms, ev_done, 0)) != cudaSuccess) {
+    cleanup();
+    return cuda_fail(e, "stream hand-back");
+  }
+  cleanup();
+  *num_fallback = count;
+  return KVQ_OK;
+}
+
+int kvq_device_error(const kvq_cache* cache, kvq_stream_t stream, int32_t* code) {
+  if (!cache || !code) return fail(KVQ_ERR_INVALID_ARG, "NULL argument");
+  *code = KVQ_OK;
+  if (!cache->error_word) return KVQ_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int32_t v = 0;
+  if ((e = cudaMemcpyAsync(&v, cache->error_word, sizeof(v), cudaMemcpyDeviceToHost, s)) !=
+          cudaSuccess ||
+      (e = cudaMemsetAsync(cache->error_word, 0, sizeof(v), s)) != cudaSuccess ||
+      (e = cudaStreamSynchronize(s)) != cudaSuccess)
+    return cuda_fail(e, "error word read-back");
+  *code = v;
+  return KVQ_OK;
+}
+
+}  // extern "C"

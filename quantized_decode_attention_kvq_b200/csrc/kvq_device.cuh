@@ -1,0 +1,185 @@
+// kvq_device.cuh -- device-side building blocks shared by the kvq kernels:
+// layout constants, mbarrier / bulk-copy / TMA wrappers with bounded waits,
+// legacy-warp MMA wrappers, the warp Walsh-Hadamard rotation and the
+// device error word.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+constexpr int kPage = 16;
+// slack factor on the certified bound and on Delta (absorbs the fp32 rounding
+// of the quantizer, of the dequantization and of the rotation)
+constexpr float kKappa = 1.0f + 1.0f / 1024.0f;
+// relative size of the fp32 rotation error allowance (see the bound's Delta)
+constexpr float kRotSlack = 1.0f / 65536.0f;
+constexpr float kLog2e = 1.4426950408889634f;
+// iteration limit of every spin on an mbarrier (each try_wait already
+// suspends for a hardware-defined time, so this is on the order of seconds)
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+// Byte layout of one (page, kv head) block of the quantized pool.
+struct BlockLayout {
+  int d, kbits, kgroup;
+  __host__ __device__ int ngk() const { return d / kgroup; }
+  __host__ __device__ int nb() const { return d / 32; }
+  __host__ __device__ int k_row() const { return d * kbits / 8; }
+  __host__ __device__ int v_row() const { return d / 2; }
+  __host__ __device__ int k_bytes() const { return kPage * k_row(); }
+  __host__ __device__ int v_bytes() const { return kPage * v_row(); }
+  __host__ __device__ int ks_bytes() const { return kPage * ngk() * 2; }
+  __host__ __device__ int vm_bytes() const { return kPage * nb() * 4; }
+  __host__ __device__ int v_off() const { return k_bytes(); }
+  __host__ __device__ int ks_off() const { return k_bytes() + v_bytes(); }
+  __host__ __device__ int vm_off() const { return ks_off() + ks_bytes(); }
+  __host__ __device__ int bytes() const { return vm_off() + vm_bytes(); }
+};
+
+__device__ __forceinline__ void set_error(int32_t* word, int code) {
+  if (word) atomicCAS(word, 0, code);
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---- mbarrier --------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for phase `parity` of `bar`; false if the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// ---- bulk copies (global -> shared, completion on an mbarrier) -------------
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+// 3-D tiled TMA load (no multicast) of box {x0.., y0.., z0} of `map`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---- warp-level MMA (fragment layouts of the PTX m16n8k32 / m16n8k16 shapes) --
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                       uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t x, uint32_t m, uint32_t o) {
+  return (x & m) | o;
+}
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
+  return *reinterpret_cast<__half2*>(&u);
+}
+
+// ---- randomized Walsh-Hadamard rotation of one vector held by a warp ------
+// Lane l holds elements [l*E, l*E + E) of a d = 32*E vector.  Computes
+// y = c * H_d * (sigma o x) with butterflies in the fixed order stride 1, 2,
+// ..., d/2 (pair (a, b) at (j, j+stride) -> (a+b, a-b)), then the product by
+// c = fp32(1/sqrt(d)); every operation is a single fp32 add, sub or mul, so
+// the result does not depend on how the butterflies are distributed.
+template <int E>
+__device__ __forceinline__ void warp_rotate(float (&x)[E], const int8_t* sigma, int lane,
+                                            float c) {
+#pragma unroll
+  for (int e = 0; e < E; ++e)
+    if (sigma[lane * E + e] < 0) x[e] = -x[e];
+#pragma unroll
+  for (int h = 1; h < E; h *= 2) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if ((e & h) == 0) {
+        float a = x[e], b = x[e + h];
+        x[e] = __fadd_rn(a, b);
+        x[e + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int hl = 1; hl < 32; hl *= 2) {
+    const bool upper = (lane & hl) != 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float other = __shfl_xor_sync(0xffffffffu, x[e], hl);
+      // lower element a (index j), upper element b (index j + stride)
+      x[e] = upper ? __fsub_rn(other, x[e]) : __fadd_rn(x[e], other);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) x[e] = __fmul_rn(x[e], c);
+}
+
+__device__ __forceinline__ float load_elem(const void* p, int is_bf16, int64_t i) {
+  if (is_bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  return reinterpret_cast<const float*>(p)[i];
+}
+
+}  // namespace kvq

@@ -206,7 +206,7 @@ class Inputs:
         if self.outlier_channels.shape[1]:
             for h in range(wl.num_kv_heads):
                 k[h][:, self.outlier_channels[h]] *= np.float32(wl.outlier_scale)
-        if b in self.spike_seqs:
+        if b in self.spike_seqs and n > 0:
             gs = _rng(self.seed, wl.name, _S_SPIKE, 1 + b)
             nt = max(1, int(round(wl.spike_token_frac * n)))
             for h in range(wl.num_kv_heads):

@@ -1,0 +1,168 @@
+"""GPU parity: the CUDA path (through the C ABI) against the oracle on the same
+seeded inputs.  Codes, scales, eta and flags bit-exact; outputs within max-abs
+2e-3 and relative L2 1e-3; the bound within 1e-4 relative and never below the
+observed error against exact attention."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_cases import (TOL_BOUND_REL, TOL_MAXABS, TOL_RELL2, compare_flags, compare_outputs,
+                       gpu_cache, oracle_pool, run_gpu, to_torch)
+from oracle_cases import SMALL, max_err, small
+from quantized_decode_attention_kvq_b200 import inputs as synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("the GPU tests need a CUDA device")
+    from quantized_decode_attention_kvq_b200 import build
+    build.build()
+
+
+def _check_decode(inp, g, o_hat, bound, flags, tau):
+    emax, rel = compare_outputs(g["out"], o_hat)
+    assert emax <= TOL_MAXABS and rel <= TOL_RELL2, (emax, rel)
+    brel = np.abs(g["bound"] - bound) / np.maximum(bound, 1e-30)
+    assert brel.max() <= TOL_BOUND_REL, brel.max()
+    bad, tie = compare_flags(g["flags"], flags, bound, tau)
+    assert bad == 0, (bad, tie)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("seed", [0, 1])
+def test_append_bit_exact(name, seed):
+    inp = small(name, seed)
+    k, v = inp.kv()
+    g = run_gpu(inp, k, v)
+    oc = oracle_pool(inp, k, v)
+    assert g["err"] == 0
+    pool = g["cache"].pool.cpu().numpy()
+    assert np.array_equal(pool, oc.pool), np.flatnonzero(pool != oc.pool)[:10]
+    eta = g["cache"].eta.cpu().numpy()
+    assert np.array_equal(eta.view(np.uint32), oc.eta.view(np.uint32))
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_decode_matches_oracle(name, seed):
+    inp = small(name, seed)
+    k, v = inp.kv()
+    q = inp.q()
+    g = run_gpu(inp, k, v, q)
+    oc = oracle_pool(inp, k, v)
+    o_hat, bound, flags, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=inp.wl.tau)
+    assert g["err"] == 0
+    _check_decode(inp, g, o_hat, bound, flags, inp.wl.tau)
+    # certified: the GPU's own output is within its bound of exact attention
+    o_dense = oracle.dense(q, k, v, inp.seq_lens)
+    assert (g["bound"] >= max_err(o_dense, g["out"])).all()
+
+
+@pytest.mark.parametrize("name", ["llama8b", "serving"])
+def test_flags_with_finite_tau(name):
+    """Flags bit-exact at a tau inside the bound distribution (about half flagged)."""
+    inp = small(name, 4)
+    k, v = inp.kv()
+    q = inp.q()
+    oc = oracle_pool(inp, k, v)
+    _, bound, _, _ = oc.decode(q, inp.page_table, inp.seq_lens)
+    tau = float(np.float32(np.median(bound)))
+    o_hat, bound, flags, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=tau)
+    g = run_gpu(inp, k, v, q, tau=tau)
+    assert 0 < flags.sum() < flags.size
+    _check_decode(inp, g, o_hat, bound, flags, tau)
+
+
+def test_bound_only_entry_point_matches():
+    inp = small("llama8b", 0)
+    k, v = inp.kv()
+    a = run_gpu(inp, k, v, tau=5.0)
+    b = run_gpu(inp, k, v, tau=5.0, bound_only=True)
+    assert np.array_equal(a["bound"], b["bound"]) and np.array_equal(a["flags"], b["flags"])
+
+
+def test_page_permutation_invariance():
+    """Outputs depend on logical order only: another physical permutation of the
+    same pages gives bit-identical results."""
+    inp = small("llama8b", 1)
+    k, v = inp.kv()
+    q = inp.q()
+    a = run_gpu(inp, k, v, q)
+    rng = np.random.default_rng(123)
+    perm = rng.permutation(inp.num_pages).astype(np.int32)
+    pt2 = np.where(inp.page_table >= 0, perm[np.maximum(inp.page_table, 0)], -1).astype(np.int32)
+    b = run_gpu(inp, k, v, q, page_table=pt2)
+    assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["bound"], b["bound"])
+
+
+@pytest.mark.parametrize("pps", [1, 3, 7])
+def test_split_count_invariance(monkeypatch, pps):
+    """Split-K with other split sizes agrees with the single-pass oracle."""
+    monkeypatch.setenv("KVQ_PAGES_PER_SPLIT", str(pps))
+    inp = small("long128k", 0)
+    k, v = inp.kv()
+    q = inp.q()
+    g = run_gpu(inp, k, v, q)
+    oc = oracle_pool(inp, k, v)
+    o_hat, bound, flags, _ = oc.decode(q, inp.page_table, inp.seq_lens)
+    _check_decode(inp, g, o_hat, bound, flags, math.inf)
+
+
+def test_ragged_and_empty_contexts():
+    inp = synth.make("serving", 7, num_seqs=5, num_q_heads=8, num_kv_heads=2, ctx=70, ctx_min=1)
+    inp.seq_lens[2] = 0          # an empty context
+    inp.seq_lens[3] = 16         # exactly one page
+    k, v = inp.kv()
+    q = inp.q()
+    g = run_gpu(inp, k, v, q, tau=math.inf)
+    oc = oracle_pool(inp, k, v)
+    o_hat, bound, flags, _ = oc.decode(q, inp.page_table, inp.seq_lens)
+    _check_decode(inp, g, o_hat, bound, flags, math.inf)
+    rows = slice(2 * 8, 3 * 8)
+    assert (g["out"][rows] == 0).all() and (g["bound"][rows] == 0).all()
+
+
+def test_device_errors_are_reported():
+    inp = small("llama8b", 0)
+    k, v = inp.kv()
+    c = gpu_cache(inp)
+    kd, vd = to_torch(k), to_torch(v)
+    pt = inp.page_table.copy()
+    pt[0, 1] = inp.num_pages + 5                       # outside the pool
+    ptd = torch.from_numpy(pt).cuda()
+    sp = torch.zeros(inp.wl.num_seqs, dtype=torch.int32, device="cuda")
+    sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
+    c.append(kd, vd, ptd, sp, sl)
+    from quantized_decode_attention_kvq_b200 import kvq
+    assert c.device_error() == kvq.KVQ_ERR_INVALID_ARG
+    assert c.device_error() == 0                        # cleared
+    ws = c.workspace(inp.wl.num_seqs, 1, inp.wl.num_q_heads, pt.shape[1])
+    c.decode(to_torch(inp.q()), ptd, sl, ws)
+    assert c.device_error() == kvq.KVQ_ERR_INVALID_ARG
+    # non-finite input
+    kn = k.copy()
+    kn[0, 0, 3, 5] = 0x7FC0                            # bf16 NaN
+    c2 = gpu_cache(inp)
+    c2.append(to_torch(kn), vd, torch.from_numpy(inp.page_table).cuda(), sp, sl)
+    assert c2.device_error() == kvq.KVQ_ERR_RANGE
+
+
+@pytest.mark.parametrize("name", ["llama8b", "long128k", "rotated"])
+def test_full_size_parity(name):
+    """The workloads at full size, every output element against the oracle."""
+    inp = synth.make(name, 0)
+    k, v = inp.kv()
+    q = inp.q()
+    g = run_gpu(inp, k, v, q)
+    assert g["err"] == 0
+    oc = oracle_pool(inp, k, v)
+    assert np.array_equal(g["cache"].pool.cpu().numpy(), oc.pool)
+    o_hat, bound, flags, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=inp.wl.tau)
+    _check_decode(inp, g, o_hat, bound, flags, inp.wl.tau)
