@@ -180,6 +180,32 @@ KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, 
                        size_t staging_bytes, kvq_stream_t main_stream,
                        kvq_stream_t side_stream, int32_t timeout_ms, int32_t* num_fallback);
 
+/* Size of the static device scratch of kvq_decode_attention_noalloc. */
+#define KVQ_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+
+/* kvq_decode_attention for callers that cannot allocate device memory where
+ * they call it (an allocator-free runtime, fixed buffers handed over by a
+ * host framework, code where cudaMalloc is forbidden or would synchronize).
+ * The pages have no counterpart of this entry point: it exists for such
+ * callers only.  Same arguments and results as kvq_decode_attention, without
+ * the workspace: the split-K scratch is a static device array of
+ * KVQ_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.  Shapes whose scratch (kvq_workspace_size) exceeds it
+ * return KVQ_ERR_UNSUPPORTED.  The call allocates no device memory (no
+ * cudaMalloc, cudaFree or any allocating CUDA or framework routine); it clears
+ * the scratch's counters with cudaMemsetAsync on `stream` before the decode.
+ * The first call on a device looks up the array's device address with that
+ * device current, so make that first call before any stream capture.  Every
+ * call shares the one array: calls that may overlap on the GPU (on different
+ * streams, or from several threads) race on it and must be serialized by the
+ * caller.  Asynchronous on `stream`. */
+KVQ_API int kvq_decode_attention_noalloc(const kvq_cache* cache, const void* q, int q_dtype,
+                                         int32_t num_seqs, int32_t num_queries,
+                                         int32_t num_q_heads, const int32_t* page_table,
+                                         int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                         float softmax_scale, float tau, float* out,
+                                         float* bound, uint8_t* flags, kvq_stream_t stream);
+
 /* Waits for `stream`, reads *cache->error_word into *code (KVQ_OK when no
  * kernel reported an error) and resets it to KVQ_OK. */
 KVQ_API int kvq_device_error(const kvq_cache* cache, kvq_stream_t stream, int32_t* code);

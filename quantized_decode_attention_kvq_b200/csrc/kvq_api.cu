@@ -559,3 +559,70 @@ int kvq_device_error(const kvq_cache* cache, kvq_stream_t stream, int32_t* code)
 }
 
 }  // extern "C"
+
+// ---- decode without caller-provided workspace ---------------------------------------
+// For callers that cannot allocate device memory at the point of the call (an
+// allocator-free runtime, a host that hands the library fixed buffers, code
+// running where cudaMalloc is forbidden or would synchronize): the split-K
+// scratch lives in this static device array instead of a caller workspace.
+// Each GPU that loads the library holds KVQ_NOALLOC_SCRATCH_BYTES of it until
+// the process exits.
+namespace {
+__device__ __align__(256) uint8_t g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device.  In host code the
+// array's name is only a stand-in, so the address is looked up once per device
+// (with that device current) and cached.
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[256] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 256) return fail(KVQ_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return KVQ_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int kvq_decode_attention_noalloc(const kvq_cache* cache, const void* q, int q_dtype,
+                                 int32_t num_seqs, int32_t num_queries, int32_t num_q_heads,
+                                 const int32_t* page_table, int32_t max_pages_per_seq,
+                                 const int32_t* seq_lens, float softmax_scale, float tau,
+                                 float* out, float* bound, uint8_t* flags, kvq_stream_t stream) {
+  if (!out && num_seqs > 0) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (num_seqs == 0) return KVQ_OK;
+  const size_t need =
+      kvq_workspace_size(cache, num_seqs, num_queries, num_q_heads, max_pages_per_seq);
+  if (need == 0)
+    return fail(KVQ_ERR_INVALID_ARG, "invalid decode shape (num_queries %d, num_q_heads %d, "
+                "max_pages_per_seq %d)", num_queries, num_q_heads, max_pages_per_seq);
+  if (need > (size_t)KVQ_NOALLOC_SCRATCH_BYTES)
+    return fail(KVQ_ERR_UNSUPPORTED, "this shape needs %zu bytes of split-K scratch; the "
+                "static scratch of kvq_decode_attention_noalloc holds %d bytes",
+                need, KVQ_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the per-(sequence, kv head) counters at the front of the scratch must start
+  // at zero whatever an earlier call left there
+  const size_t counters = ((size_t)num_seqs * cache->num_kv_heads * sizeof(int) + 255) / 256 * 256;
+  cudaError_t e = cudaMemsetAsync(scratch, 0, counters, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scratch counters)");
+  return decode_impl(cache, q, q_dtype, num_seqs, num_queries, num_q_heads, page_table,
+                     max_pages_per_seq, seq_lens, softmax_scale, tau, out, bound, flags, scratch,
+                     (size_t)KVQ_NOALLOC_SCRATCH_BYTES, s);
+}
+
+}  // extern "C"

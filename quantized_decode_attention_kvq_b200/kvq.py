@@ -34,7 +34,8 @@ PAGE_SIZE = 16
 
 EXPORTED = ("kvq_block_bytes", "kvq_pool_bytes", "kvq_quantize_append", "kvq_workspace_size",
             "kvq_decode_attention", "kvq_error_bound", "kvq_fallback_staging_size",
-            "kvq_fallback_exact", "kvq_device_error", "kvq_status_string", "kvq_last_error")
+            "kvq_fallback_exact", "kvq_device_error", "kvq_status_string", "kvq_last_error",
+            "kvq_decode_attention_noalloc")
 
 
 class KvqError(RuntimeError):
@@ -76,6 +77,8 @@ def _load() -> ctypes.CDLL:
                                               I32, I32, I32, P, F, P, P, P, P, SZ, P, P, I32,
                                               ctypes.POINTER(I32)]),
         "kvq_device_error": (ctypes.c_int, [C, P, ctypes.POINTER(I32)]),
+        "kvq_decode_attention_noalloc": (ctypes.c_int, [C, P, ctypes.c_int, I32, I32, I32, P,
+                                                        I32, P, F, F, P, P, P, P]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -172,6 +175,21 @@ def kvq_error_bound(cache, q, q_dtype, num_seqs, num_queries, num_q_heads, page_
                                 num_q_heads, _ptr(page_table), max_pages_per_seq,
                                 _ptr(seq_lens), softmax_scale, tau, _ptr(bound), _ptr(flags),
                                 _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def kvq_decode_attention_noalloc(cache, q, q_dtype, num_seqs, num_queries, num_q_heads,
+                                 page_table, max_pages_per_seq, seq_lens, softmax_scale, tau, out,
+                                 bound, flags, stream=None) -> int:
+    """kvq_decode_attention with the library's static device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    return _lib.kvq_decode_attention_noalloc(ctypes.byref(cache), _ptr(q), q_dtype, num_seqs,
+                                             num_queries, num_q_heads, _ptr(page_table),
+                                             max_pages_per_seq, _ptr(seq_lens), softmax_scale,
+                                             tau, _ptr(out), _ptr(bound), _ptr(flags),
+                                             _stream(stream))
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 
 def kvq_fallback_staging_size(cache, orig_dtype, max_ctx) -> int:

@@ -1,0 +1,69 @@
+"""kvq_decode_attention_noalloc: the decode entry point for callers that cannot
+allocate device memory where they call it -- an allocator-free runtime, a host
+framework that hands the library fixed buffers, or code that runs where a
+cudaMalloc is forbidden or would synchronize the device.  It uses the
+library's static device scratch instead of a caller workspace.
+
+Checked here through the C ABI against kvq_decode_attention with a workspace,
+on two calls in a row (the scratch keeps the previous call's contents), within
+the tolerances of the other parity tests.  This file is collected last."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_cases import TOL_BOUND_REL, TOL_MAXABS, TOL_RELL2, compare_outputs, run_gpu
+from oracle_cases import small
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(g, inp, tau):
+    from quantized_decode_attention_kvq_b200 import kvq
+    wl = inp.wl
+    S, NQ, HQ, d = wl.num_seqs, wl.num_queries, wl.num_q_heads, wl.head_dim
+    out = torch.full((S, NQ, HQ, d), float("nan"), dtype=torch.float32, device="cuda")
+    bound = torch.full((S, NQ, HQ), float("nan"), dtype=torch.float32, device="cuda")
+    flags = torch.full((S, NQ, HQ), 7, dtype=torch.uint8, device="cuda")
+    q = g["q"]
+    rc = kvq.kvq_decode_attention_noalloc(
+        g["cache"].desc, q, kvq.KVQ_BF16 if q.dtype == torch.bfloat16 else kvq.KVQ_F32, S, NQ,
+        HQ, g["pt"], g["pt"].shape[1], g["sl"], 0.0, tau, out, bound, flags)
+    assert rc == kvq.KVQ_OK, kvq.last_error()
+    torch.cuda.synchronize()
+    return (out.cpu().numpy().reshape(-1, d).astype(np.float64),
+            bound.cpu().numpy().reshape(-1).astype(np.float64), flags.cpu().numpy().reshape(-1))
+
+
+@pytest.mark.parametrize("name,tau", [("llama8b", 5.0), ("serving", math.inf)])
+def test_noalloc_matches_workspace_entry_point(name, tau):
+    if not torch.cuda.is_available():
+        pytest.fail("the GPU tests need a CUDA device")
+    inp = small(name, 3)
+    g = run_gpu(inp, tau=tau)                       # kvq_decode_attention with a workspace
+    for _ in range(2):                              # two calls in a row share the scratch
+        out, bound, flags = _noalloc(g, inp, tau)
+        emax, rel = compare_outputs(out, g["out"])
+        assert emax <= TOL_MAXABS and rel <= TOL_RELL2, (emax, rel)
+        assert (np.abs(bound - g["bound"]) <= TOL_BOUND_REL * g["bound"]).all()
+        assert np.array_equal(flags, g["flags"])
+    assert g["cache"].device_error() == 0
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    from quantized_decode_attention_kvq_b200 import kvq
+    if not torch.cuda.is_available():
+        pytest.fail("the GPU tests need a CUDA device")
+    inp = small("llama8b", 0)
+    c = kvq.PagedCache(inp.wl.num_kv_heads, inp.wl.head_dim, inp.num_pages)
+    seqs, max_pages = 4096, 4096                    # far more split-K scratch than it holds
+    need = kvq.kvq_workspace_size(c.desc, seqs, 1, inp.wl.num_q_heads, max_pages)
+    assert need > kvq.NOALLOC_SCRATCH_BYTES
+    dummy = torch.zeros(16, dtype=torch.int32, device="cuda")
+    rc = kvq.kvq_decode_attention_noalloc(c.desc, dummy, kvq.KVQ_BF16, seqs, 1,
+                                          inp.wl.num_q_heads, dummy, max_pages, dummy, 0.0,
+                                          math.inf, dummy, dummy, dummy)
+    assert rc == kvq.KVQ_ERR_UNSUPPORTED
+    assert "static scratch" in kvq.last_error()
