@@ -64,11 +64,14 @@ struct DecodeCfg {
   static constexpr int SZ_RS = kWarps * S * REST;
   static constexpr int OFF_BAR = (OFF_RS + SZ_RS + 15) / 16 * 16;
   static constexpr int OFF_PG = OFF_BAR + kWarps * S * 8;
-  static constexpr int OFF_Q = (OFF_PG + kWarps * S * 4 + 15) / 16 * 16;   // int qfix[4][D]
-  static constexpr int OFF_QF = OFF_Q + kRows * D * 4;                      // float q'[4][D]
+  static constexpr int OFF_Q = (OFF_PG + kWarps * S * 4 + 15) / 16 * 16;   // int8 qdig[4][4][D]
+  static constexpr int OFF_QB = OFF_Q + kRows * 4 * D;                      // int qsum[4][NGK][4]
+  static constexpr int OFF_QF = OFF_QB + kRows * NGK * 4 * 4;               // float q'[4][D]
   static constexpr int OFF_RC = OFF_QF + kRows * D * 4;                     // row constants
   static constexpr int RC_FLOATS = kRows * (2 + NGK);                       // zs, cb, cg[NGK]
-  static constexpr int OFF_FLAG = OFF_RC + RC_FLOATS * 4;
+  static constexpr int META_FLOATS = kPage * NB + kPage * NGK;              // per warp
+  static constexpr int OFF_META = (OFF_RC + RC_FLOATS * 4 + 15) / 16 * 16;
+  static constexpr int OFF_FLAG = OFF_META + kWarps * META_FLOATS * 4;
   static constexpr int END = OFF_FLAG + 16;
   // merge area (aliases the stage buffers once the page loop is over)
   static constexpr int MW_FLOATS = kRows * D + kRows * 8 + kRows * NB + 2 * NB + 1;
@@ -77,45 +80,12 @@ struct DecodeCfg {
   static_assert(MERGE_BYTES <= OFF_BAR, "merge area must fit in the stage buffers");
 };
 
-__device__ __forceinline__ int q_digit(int v, int i) {
-  int d0 = (int)(int8_t)(v & 0xFF);
-  if (i == 0) return d0;
-  v = (v - d0) >> 8;
-  int d1 = (int)(int8_t)(v & 0xFF);
-  if (i == 1) return d1;
-  v = (v - d1) >> 8;
-  int d2 = (int)(int8_t)(v & 0xFF);
-  if (i == 2) return d2;
-  return (v - d2) >> 8;
-}
-
-template <int D>
-__device__ __forceinline__ void finalize_row(const DecodeArgs& a, int b, int kvh, int r,
-                                             float l, float A, float B, float E, float dmax,
-                                             float range, float etamax, const float* o_row,
-                                             int c0, int cstep, bool write_stats) {
-  if (r >= a.R) return;
-  const int qi = r / a.G, h = kvh * a.G + r % a.G;
-  const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + h;
-  if (a.out) {
-    const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-    for (int c = c0; c < D; c += cstep) a.out[row * D + c] = o_row[c] * inv_l;
-  }
-  if (write_stats) {
-    float bd = 0.f;
-    if (l > 0.f) {
-      const float tv = fminf(tanhf(0.5f * dmax), A / B);
-      const float ekey = tv * (range + 2.0f * etamax);
-      const float evl = E / l;
-      bd = kKappa * (ekey + evl);
-    }
-    a.bound[row] = bd;
-    a.flags[row] = bd > a.tau ? 1 : 0;
-  }
-}
+// resident CTAs per SM the register budget is sized for (4 = 128 registers)
+template <int D, int KB, int KG>
+constexpr int min_ctas() { return (KB == 4 && KG == 32) ? 3 : 4; }
 
 template <int D, int KB, int KG, int S>
-__global__ void __launch_bounds__(kWarps * 32, 3)
+__global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     decode_mma_kernel(const __grid_constant__ DecodeArgs a,
                       const __grid_constant__ CUtensorMap kmap) {
   using C = DecodeCfg<D, KB, KG, S>;
@@ -157,9 +127,23 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
   uint8_t* rest = sm + C::OFF_RS + warp * S * C::REST;
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + warp * S;
   int* spage = reinterpret_cast<int*>(sm + C::OFF_PG) + warp * S;
-  int* qfix = reinterpret_cast<int*>(sm + C::OFF_Q);
+  int8_t* qdig = reinterpret_cast<int8_t*>(sm + C::OFF_Q);
+  int* qsum = reinterpret_cast<int*>(sm + C::OFF_QB);
   float* qf = reinterpret_cast<float*>(sm + C::OFF_QF);
   float* rc = reinterpret_cast<float*>(sm + C::OFF_RC);
+
+  // the query rows go first, ahead of the page copies in the memory queues
+  constexpr int QPT = kRows * D / (kWarps * 32);   // query elements per thread
+  float qreg[QPT];
+#pragma unroll
+  for (int k = 0; k < QPT; ++k) {
+    const int i = tid + k * kWarps * 32, r = i / D, c = i % D;
+    qreg[k] = 0.f;
+    if (r < a.R) {
+      const int qi = r / a.G, h = kvh * a.G + r % a.G;
+      qreg[k] = load_elem(a.q, a.q_bf16, (((int64_t)b * a.nq + qi) * a.hq + h) * D + c);
+    }
+  }
 
   // ---- pipeline start: page indices, barriers, first S copies --------------
   const int first = p0 + warp;
@@ -203,17 +187,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
   };
   for (int j = 0; j < S && j < nloc; ++j) issue(j);
 
-  // ---- query rows: load, rotate, fixed point, norms -------------------------
-  for (int i = tid; i < kRows * D; i += blockDim.x) {
-    const int r = i / D, c = i % D;
-    float x = 0.f;
-    if (r < a.R) {
-      const int qi = r / a.G, h = kvh * a.G + r % a.G;
-      const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + h;
-      x = load_elem(a.q, a.q_bf16, row * D + c);
-    }
-    qf[i] = x;
-  }
+  // ---- query rows: rotate, fixed point, norms (loaded before the copies) -----
+#pragma unroll
+  for (int k = 0; k < QPT; ++k) qf[tid + k * kWarps * 32] = qreg[k];
   __syncthreads();
   if (warp < kRows) {
     const int r = warp;
@@ -242,8 +218,35 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     if (am > 0.f) frexpf(am, &ex);
     int F = am > 0.f ? 30 - ex : 0;
     F = min(F, 100);
+    // q' * 2^F in int32, split into four signed base-256 digits, stored in the
+    // order the MMA B fragments read them: for 4-bit keys, position
+    // 32b + 8s + 4(i%2) + i/2 holds channel 32b + 8s + i (even/odd nibbles)
+    int ds[4] = {0, 0, 0, 0};  // digit sums over this lane's channels (one key group)
 #pragma unroll
-    for (int e = 0; e < E; ++e) qfix[r * D + lane * E + e] = __float2int_rn(ldexpf(x[e], F));
+    for (int e = 0; e < E; ++e) {
+      const int c = lane * E + e;
+      int v = __float2int_rn(ldexpf(x[e], F));
+      const int i8 = c % 8;
+      const int pos = KB == 8 ? c : (c - i8) + 4 * (i8 % 2) + i8 / 2;
+#pragma unroll
+      for (int d = 0; d < 4; ++d) {
+        const int dg = d < 3 ? (int)(int8_t)(v & 0xFF) : v;
+        v = (v - dg) >> 8;
+        qdig[(r * 4 + d) * D + pos] = (int8_t)dg;
+        ds[d] += dg;
+      }
+    }
+    if (KB == 4) {  // sum of every digit over each key group (bias of code + 8)
+#pragma unroll
+      for (int d = 0; d < 4; ++d)
+#pragma unroll
+        for (int o = 1; o < KG / E; o *= 2) ds[d] += __shfl_xor_sync(0xffffffffu, ds[d], o);
+      if ((lane * E) % KG == 0) {
+        const int g = (lane * E) / KG;
+#pragma unroll
+        for (int d = 0; d < 4; ++d) qsum[(r * NGK + g) * 4 + d] = ds[d];
+      }
+    }
     if (lane == 0) {
       rc[r] = ldexpf(a.s_att * kLog2e, -F);                      // zs: score scale, log2 units
       rc[kRows + r] = a.signs ? kKappa * a.s_att * kRotSlack * sqrtf((float)D) * (float)Q *
@@ -265,18 +268,12 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
 #pragma unroll
     for (int ks = 0; ks < NB; ++ks)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          uint32_t w = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int ch = KB == 8 ? 32 * ks + 8 * c4 + 4 * jj + e : 32 * ks + 8 * c4 + 2 * e + jj;
-            const int dg = q_digit(qfix[r * D + ch], 2 * nt + dl);
-            w |= (uint32_t)(dg & 0xFF) << (8 * e);
-          }
-          qb[ks][nt][jj] = w;
-        }
+      for (int nt = 0; nt < 2; ++nt) {
+        const uint2 w2 = *reinterpret_cast<const uint2*>(qdig + (r * 4 + 2 * nt + dl) * D + 32 * ks +
+                                                         8 * c4);
+        qb[ks][nt][0] = w2.x;
+        qb[ks][nt][1] = w2.y;
+      }
   }
   // initial accumulators: 4-bit key codes enter as code + 8
   int cinit[NGK][2][2];
@@ -285,12 +282,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int dd = 0; dd < 2; ++dd) {
-        int s = 0;
-        if (KB == 4)
-          for (int c = g * KG; c < (g + 1) * KG; ++c) s += q_digit(qfix[c4 * D + c], 2 * nt + dd);
-        cinit[g][nt][dd] = -8 * s;
-      }
+      for (int dd = 0; dd < 2; ++dd)
+        cinit[g][nt][dd] = KB == 4 ? -8 * qsum[(c4 * NGK + g) * 4 + 2 * nt + dd] : 0;
   const float zs = rc[c4];
   const float cb = rc[kRows + c4];
   float cg[NGK];
@@ -299,17 +292,34 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
 
   // ---- accumulators ------------------------------------------------------------
   float m2 = -INFINITY, lsum = 0.f, Asum = 0.f, Bsum = 0.f, Esum = 0.f, dmax = 0.f;
-  float zacc[NB];
+  // PV accumulators: m-tile 2g holds the low-nibble channels of group g (codes
+  // entered as fp16 subnormals c*2^-24), m-tile 2g+1 the high-nibble channels
+  // (16c*2^-24); the power-of-two factors are removed after the loop.
   float opv[2 * NB][4];
-#pragma unroll
-  for (int g = 0; g < NB; ++g) zacc[g] = 0.f;
+  float zmv[4];  // zero-point MMA: rows = groups, columns = (row, hi/lo part)
 #pragma unroll
   for (int t = 0; t < 2 * NB; ++t)
 #pragma unroll
     for (int e = 0; e < 4; ++e) opv[t][e] = 0.f;
-  float vhi = -INFINITY, vlo = INFINITY, etamax = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) zmv[e] = 0.f;
+  constexpr int EPL = NB / 2;  // V metadata entries converted per lane and page
+  float vhi[EPL], vlo[EPL], etamax = 0.f;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    vhi[i] = -INFINITY;
+    vlo[i] = INFINITY;
+  }
   const int hP = g8 & 3;
   const bool lo_part = g8 >= 4;
+  float* vs32 = reinterpret_cast<float*>(sm + C::OFF_META) + warp * C::META_FLOATS;
+  float* ks32 = vs32 + kPage * NB;
+  // hi part of a value: its top 11 significant bits (exact in fp16); lo lanes
+  // take the remainder, so hi + lo reproduces the fp32 value to ~2^-22
+  auto hilo = [&](float v) {
+    const float t = __int_as_float(__float_as_int(v) & 0xFFFFE000);
+    return lo_part ? v - t : t;
+  };
 
   const float* eta_kv = a.eta + kvh;
   float eta_next = 0.f;
@@ -340,6 +350,33 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
       const int tok0 = (first + j * kWarps) * kPage;
       const int nval = min(kPage, n - tok0);
       etamax = fmaxf(etamax, eta_cur);
+      const uint32_t* vm = reinterpret_cast<const uint32_t*>(rs + C::VB + C::KSB);
+      const __half* ksc = reinterpret_cast<const __half*>(rs + C::VB);
+
+      // --- page metadata to fp32 once for the warp; value range per group -------
+      {
+        uint32_t mw[EPL];
+        if constexpr (EPL == 2) {
+          const uint2 v2 = reinterpret_cast<const uint2*>(vm)[lane];
+          mw[0] = v2.x;
+          mw[1] = v2.y;
+        } else {
+          mw[0] = vm[lane];
+        }
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+          const int e = lane * EPL + i;  // token e / NB, group e % NB
+          const __half2 sz = u32_as_h2(mw[i]);
+          const float s = __low2float(sz), z = __high2float(sz);
+          const bool in = e / NB < nval;
+          vs32[e] = in ? s : 0.f;
+          if (in) {
+            vhi[i] = fmaxf(vhi[i], __fmaf_rn(15.0f, s, z));
+            vlo[i] = fminf(vlo[i], z);
+          }
+        }
+        for (int e = lane; e < kPage * NGK; e += 32) ks32[e] = __half2float(ksc[e]);
+      }
 
       // --- K codes of rows g8, g8+8 (this lane's stripe) -> QK^T on int8 MMA ---
       constexpr int KW = C::KSTR / 4;    // 32-bit words per stripe
@@ -393,9 +430,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) mma_s8(acc[g][nt], a0, a1, a2, a3, qb[ks][nt][0], qb[ks][nt][1]);
       }
+      __syncwarp();  // the fp32 metadata table is complete
 
       // --- scores (log2 units) and Delta for tokens g8, g8+8 of row c4 -------------
-      const __half* ksc = reinterpret_cast<const __half*>(rs + C::VB);
       float zt[2], dl[2];
       bool vt[2];
 #pragma unroll
@@ -405,10 +442,11 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
         float dot = 0.f, dsum = 0.f, smax = 0.f;
 #pragma unroll
         for (int g = 0; g < NGK; ++g) {
-          const float s = __half2float(ksc[tok * NGK + g]);
-          const float d0 = (float)acc[g][0][2 * sl], d1 = (float)acc[g][0][2 * sl + 1];
-          const float d2 = (float)acc[g][1][2 * sl], d3 = (float)acc[g][1][2 * sl + 1];
-          const float raw = fmaf(d3, 16777216.f, fmaf(d2, 65536.f, fmaf(d1, 256.f, d0)));
+          const float s = ks32[tok * NGK + g];
+          // digits 0,1 and 2,3 recombined exactly in int32, then once in fp32
+          const int lo = acc[g][0][2 * sl] + acc[g][0][2 * sl + 1] * 256;
+          const int hi = acc[g][1][2 * sl] + acc[g][1][2 * sl + 1] * 256;
+          const float raw = fmaf((float)hi, 65536.f, (float)lo);
           dot = fmaf(raw, s, dot);
           dsum = fmaf(cg[g], s, dsum);
           smax = fmaxf(smax, s);
@@ -431,10 +469,17 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
       for (int sl = 0; sl < 2; ++sl) {
         if (vt[sl]) {
           const float w = sl ? w1 : w0;
-          ta = fmaf(w, expm1f(dl[sl]), ta);
-          tb = fmaf(w, expf(-dl[sl]), tb);
+          const float d = dl[sl];
+          const float ep = exp2f(d * kLog2e), en = exp2f(-d * kLog2e);
+          // e^d - 1: Taylor to d^5 below 1/16 (no cancellation), else from e^d
+          const float em1 =
+              d < 0.0625f
+                  ? d * fmaf(d, fmaf(d, fmaf(d, fmaf(d, 1.0f / 120, 1.0f / 24), 1.0f / 6), 0.5f), 1.0f)
+                  : ep - 1.0f;
+          ta = fmaf(w, em1, ta);
+          tb = fmaf(w, en, tb);
           tw += w;
-          dmax = fmaxf(dmax, dl[sl]);
+          dmax = fmaxf(dmax, d);
         }
       }
       lsum = fmaf(lsum, alpha, tw);
@@ -442,26 +487,11 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
       Bsum = fmaf(Bsum, alpha, tb);
       Esum = fmaf(Esum, alpha, tw * eta_cur);
 
-      // --- value range of group c4 over tokens g8, g8+8 --------------------------
-      const uint32_t* vm = reinterpret_cast<const uint32_t*>(rs + C::VB + C::KSB);
-      if (c4 < NB) {
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          if (vt[sl]) {
-            const __half2 sz = u32_as_h2(vm[(g8 + 8 * sl) * NB + c4]);
-            const float s = __low2float(sz), z = __high2float(sz);
-            vhi = fmaxf(vhi, __fmaf_rn(15.0f, s, z));
-            vlo = fminf(vlo, z);
-          }
-        }
-      }
-
       // --- rescale the PV state when a row max moved --------------------------------
       if (__any_sync(0xffffffffu, alpha != 1.0f)) {
         const int base = lane & ~3;
         const float a0 = __shfl_sync(0xffffffffu, alpha, base | (2 * (c4 & 1)));
         const float a1 = __shfl_sync(0xffffffffu, alpha, base | (2 * (c4 & 1) + 1));
-        const float az = __shfl_sync(0xffffffffu, alpha, base | hP);
 #pragma unroll
         for (int t = 0; t < 2 * NB; ++t) {
           opv[t][0] *= a0;
@@ -469,21 +499,32 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
           opv[t][2] *= a0;
           opv[t][3] *= a1;
         }
-#pragma unroll
-        for (int g = 0; g < NB; ++g) zacc[g] *= az;
+        zmv[0] *= a0;
+        zmv[1] *= a1;
       }
 
-      // --- P' = w * sV for tokens c4 + 4k, row hP (hi or lo half) -----------------
+      // --- weights w of tokens c4 + 4k for row hP (the MMA B layout) --------------
       float x[4];
       x[0] = __shfl_sync(0xffffffffu, w0, 4 * c4 + hP);
       x[1] = __shfl_sync(0xffffffffu, w0, 4 * c4 + 16 + hP);
       x[2] = __shfl_sync(0xffffffffu, w1, 4 * c4 + hP);
       x[3] = __shfl_sync(0xffffffffu, w1, 4 * c4 + 16 + hP);
-      bool vx[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) vx[k] = c4 + 4 * k < nval;
 
-      // V code stripes (row g8) of tokens c4 + 4k
+      // --- zero points: sum_j w_j zV_{j,g} on one MMA (rows = groups) -------------
+      {
+        uint32_t zw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int tok = c4 + 4 * k;
+          const uint32_t wv = vm[tok * NB + (g8 < NB ? g8 : 0)];
+          zw[k] = (g8 < NB && tok < nval) ? wv : 0u;
+        }
+        const uint32_t bz0 = h2_as_u32(__floats2half2_rn(hilo(x[0]), hilo(x[1])));
+        const uint32_t bz1 = h2_as_u32(__floats2half2_rn(hilo(x[2]), hilo(x[3])));
+        mma_f16(zmv, prmt(zw[0], zw[1], 0x7632u), 0u, prmt(zw[2], zw[3], 0x7632u), 0u, bz0, bz1);
+      }
+
+      // --- PV: V code stripes (row g8) of tokens c4 + 4k ---------------------------
       uint32_t vw[4][C::VSTR / 4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -496,42 +537,36 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
           vw[k][0] = *reinterpret_cast<const uint32_t*>(p);
         }
       }
+      float sv[4][NB];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if constexpr (NB == 4) {
+          const float4 f = *reinterpret_cast<const float4*>(vs32 + (c4 + 4 * k) * NB);
+          sv[k][0] = f.x;
+          sv[k][1] = f.y;
+          sv[k][2] = f.z;
+          sv[k][3] = f.w;
+        } else {
+          const float2 f = *reinterpret_cast<const float2*>(vs32 + (c4 + 4 * k) * NB);
+          sv[k][0] = f.x;
+          sv[k][1] = f.y;
+        }
+      }
 #pragma unroll
       for (int g = 0; g < NB; ++g) {
-        float P[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const __half2 sz = u32_as_h2(vm[(c4 + 4 * k) * NB + g]);
-          const float s = __low2float(sz), z = __high2float(sz);
-          P[k] = vx[k] ? x[k] * s : 0.f;
-          zacc[g] = vx[k] ? fmaf(x[k], z, zacc[g]) : zacc[g];
-        }
-        uint32_t bf[2];
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          const __half2 hi = __floats2half2_rn(P[2 * pr], P[2 * pr + 1]);
-          const float2 hf = __half22float2(hi);
-          const __half2 lo = __floats2half2_rn(P[2 * pr] - hf.x, P[2 * pr + 1] - hf.y);
-          bf[pr] = lo_part ? h2_as_u32(lo) : h2_as_u32(hi);
-        }
-        // A fragments for m-tiles 2g (low nibbles) and 2g+1 (high nibbles)
-        const int wsel = (2 * g) / 4;            // word of the stripe holding group g
+        // P' = w * sV (zero outside the context), as fp16 hi or lo part
+        const uint32_t b01 = h2_as_u32(__floats2half2_rn(hilo(x[0] * sv[0][g]), hilo(x[1] * sv[1][g])));
+        const uint32_t b23 = h2_as_u32(__floats2half2_rn(hilo(x[2] * sv[2][g]), hilo(x[3] * sv[3][g])));
+        const int wsel = (2 * g) / 4;            // stripe word holding group g
         const int p = (2 * g) % 4;               // byte offset of group g in that word
         const uint32_t sel = (uint32_t)(p | ((p + 1) << 4) | ((4 + p) << 8) | ((5 + p) << 12));
         const uint32_t r01 = prmt(vw[0][wsel], vw[1][wsel], sel);   // tokens c4, c4+4
         const uint32_t r23 = prmt(vw[2][wsel], vw[3][wsel], sel);   // tokens c4+8, c4+12
         const uint32_t r01s = r01 >> 8, r23s = r23 >> 8;
-        const __half2 k1024 = __float2half2_rn(1024.f);
-        const __half2 k16inv = __float2half2_rn(0.0625f);
-        const __half2 km64 = __float2half2_rn(-64.f);
-        auto lo_n = [&](uint32_t r) {
-          return h2_as_u32(__hsub2(u32_as_h2((r & 0x000F000Fu) | 0x64006400u), k1024));
-        };
-        auto hi_n = [&](uint32_t r) {
-          return h2_as_u32(__hfma2(u32_as_h2((r & 0x00F000F0u) | 0x64006400u), k16inv, km64));
-        };
-        mma_f16(opv[2 * g], lo_n(r01), lo_n(r01s), lo_n(r23), lo_n(r23s), bf[0], bf[1]);
-        mma_f16(opv[2 * g + 1], hi_n(r01), hi_n(r01s), hi_n(r23), hi_n(r23s), bf[0], bf[1]);
+        mma_f16(opv[2 * g], r01 & 0x000F000Fu, r01s & 0x000F000Fu, r23 & 0x000F000Fu,
+                r23s & 0x000F000Fu, b01, b23);
+        mma_f16(opv[2 * g + 1], r01 & 0x00F000F0u, r01s & 0x00F000F0u, r23 & 0x00F000F0u,
+                r23s & 0x00F000F0u, b01, b23);
       }
     }
     __syncwarp();
@@ -546,18 +581,20 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     Bsum += __shfl_xor_sync(0xffffffffu, Bsum, o);
     Esum += __shfl_xor_sync(0xffffffffu, Esum, o);
     dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
-    vhi = fmaxf(vhi, __shfl_xor_sync(0xffffffffu, vhi, o));
-    vlo = fminf(vlo, __shfl_xor_sync(0xffffffffu, vlo, o));
   }
 #pragma unroll
-  for (int g = 0; g < NB; ++g) {
-    zacc[g] += __shfl_xor_sync(0xffffffffu, zacc[g], 1);
-    zacc[g] += __shfl_xor_sync(0xffffffffu, zacc[g], 2);
-  }
+  for (int o = 2; o < 32; o *= 2)
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      vhi[i] = fmaxf(vhi[i], __shfl_xor_sync(0xffffffffu, vhi[i], o));
+      vlo[i] = fminf(vlo[i], __shfl_xor_sync(0xffffffffu, vlo[i], o));
+    }
 #pragma unroll
   for (int t = 0; t < 2 * NB; ++t)
 #pragma unroll
     for (int e = 0; e < 4; ++e) opv[t][e] += __shfl_xor_sync(0xffffffffu, opv[t][e], 2);
+#pragma unroll
+  for (int e = 0; e < 2; ++e) zmv[e] += __shfl_xor_sync(0xffffffffu, zmv[e], 2);
 
   __syncthreads();  // every warp is done with its stage buffers
   // merge area: per warp w: o[4][D], st[4][8], z[4][NB], vhi[NB], vlo[NB], eta
@@ -571,13 +608,18 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     for (int g = 0; g < NB; ++g)
 #pragma unroll
       for (int hn = 0; hn < 2; ++hn) {
+        const float f = hn ? 1048576.0f : 16777216.0f;   // 2^20, 2^24
         const int chR = 32 * g + 4 * g8 + hn, chR8 = chR + 2;
         const int h0 = 2 * c4, h1 = 2 * c4 + 1;
-        mo[h0 * D + chR] = opv[2 * g + hn][0];
-        mo[h1 * D + chR] = opv[2 * g + hn][1];
-        mo[h0 * D + chR8] = opv[2 * g + hn][2];
-        mo[h1 * D + chR8] = opv[2 * g + hn][3];
+        mo[h0 * D + chR] = opv[2 * g + hn][0] * f;
+        mo[h1 * D + chR] = opv[2 * g + hn][1] * f;
+        mo[h0 * D + chR8] = opv[2 * g + hn][2] * f;
+        mo[h1 * D + chR8] = opv[2 * g + hn][3] * f;
       }
+    if (g8 < NB) {
+      mz[(2 * c4) * NB + g8] = zmv[0];
+      mz[(2 * c4 + 1) * NB + g8] = zmv[1];
+    }
   }
   if (g8 == 0) {  // lanes 0..3 hold row c4's statistics
     mst[c4 * 8 + 0] = m2;
@@ -586,103 +628,108 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     mst[c4 * 8 + 3] = Bsum;
     mst[c4 * 8 + 4] = Esum;
     mst[c4 * 8 + 5] = dmax;
-    if (c4 < NB) {
-      mr[c4] = vhi;
-      mr[NB + c4] = vlo;
-    }
   }
-  if (c4 == 0 && g8 < 4) {
+  if (lane < 2) {  // lane parity selects the groups of the range entries
 #pragma unroll
-    for (int g = 0; g < NB; ++g) mz[g8 * NB + g] = zacc[g];
+    for (int i = 0; i < EPL; ++i) {
+      const int g = (lane * EPL + i) % NB;
+      mr[g] = vhi[i];
+      mr[NB + g] = vlo[i];
+    }
   }
   if (lane == 0) mr[2 * NB] = etamax;
   __syncthreads();
 
-  // ---- CTA merge: all warps -> one record in shared memory ----------------------
-  float* cm = reinterpret_cast<float*>(sm) + kWarps * C::MW_FLOATS;   // merged record
-  float* cst = cm + kRows * D;
-  float* cr = cst + kRows * 8;
-  if (tid < kRows) {
-    const int r = tid;
-    float M = -INFINITY;
-    for (int w = 0; w < kWarps; ++w)
-      M = fmaxf(M, reinterpret_cast<float*>(sm)[w * C::MW_FLOATS + kRows * D + r * 8]);
-    float L = 0.f, A = 0.f, Bv = 0.f, Ev = 0.f, Dm = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const float* s = reinterpret_cast<float*>(sm) + w * C::MW_FLOATS + kRows * D + r * 8;
-      const float f = s[0] == -INFINITY ? 0.f : exp2f(s[0] - M);
-      L = fmaf(f, s[1], L);
-      A = fmaf(f, s[2], A);
-      Bv = fmaf(f, s[3], Bv);
-      Ev = fmaf(f, s[4], Ev);
-      Dm = fmaxf(Dm, s[5]);
+  // ---- merges: warp r owns query row r ----------------------------------------
+  // (1) the CTA's warps -> one record; (2) the last CTA of (b, kvh) merges the
+  // records of all splits.  Lane l owns channels [l*CPL, l*CPL + CPL).
+  constexpr int CPL = D / 32;
+  constexpr int RF = record_floats(D);
+  const int r = warp;
+  const float* wa = reinterpret_cast<const float*>(sm);   // per-warp areas, MW_FLOATS each
+  float mW = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) mW = fmaxf(mW, wa[w * C::MW_FLOATS + kRows * D + r * 8]);
+  float st5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};   // l, A, B, E (rescaled), max Delta
+  float o[CPL];
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) o[e] = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float* mwp = wa + w * C::MW_FLOATS;
+    const float* stw = mwp + kRows * D + r * 8;
+    const float f = stw[0] == -INFINITY ? 0.f : exp2f(stw[0] - mW);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) st5[t] = fmaf(f, stw[1 + t], st5[t]);
+    st5[4] = fmaxf(st5[4], stw[5]);
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) {
+      const int c = lane * CPL + e;
+      o[e] = fmaf(f, mwp[r * D + c] + mwp[kRows * D + kRows * 8 + r * NB + c / 32], o[e]);
     }
-    cst[r * 8 + 0] = M;
-    cst[r * 8 + 1] = L;
-    cst[r * 8 + 2] = A;
-    cst[r * 8 + 3] = Bv;
-    cst[r * 8 + 4] = Ev;
-    cst[r * 8 + 5] = Dm;
-  } else if (tid == kRows) {
-    float hi[NB], lo[NB], et = 0.f;
-    for (int g = 0; g < NB; ++g) {
-      hi[g] = -INFINITY;
-      lo[g] = INFINITY;
-    }
-    for (int w = 0; w < kWarps; ++w) {
-      const float* r = reinterpret_cast<float*>(sm) + w * C::MW_FLOATS + kRows * D + kRows * 8 +
-                       kRows * NB;
-      for (int g = 0; g < NB; ++g) {
-        hi[g] = fmaxf(hi[g], r[g]);
-        lo[g] = fminf(lo[g], r[NB + g]);
-      }
-      et = fmaxf(et, r[2 * NB]);
-    }
-    for (int g = 0; g < NB; ++g) {
-      cr[g] = hi[g];
-      cr[NB + g] = lo[g];
-    }
-    cr[2 * NB] = et;
   }
-  __syncthreads();
-  for (int i = tid; i < kRows * D; i += blockDim.x) {
-    const int r = i / D, c = i % D;
-    const float M = cst[r * 8];
-    float o = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const float* mwp = reinterpret_cast<float*>(sm) + w * C::MW_FLOATS;
-      const float mwr = mwp[kRows * D + r * 8];
-      if (mwr == -INFINITY) continue;
-      const float f = exp2f(mwr - M);
-      o = fmaf(f, mwp[i] + mwp[kRows * D + kRows * 8 + r * NB + c / 32], o);
-    }
-    cm[i] = o;
+  float rg[2 * NB + 1];   // group maxima, group minima, eta
+#pragma unroll
+  for (int g = 0; g < NB; ++g) {
+    rg[g] = -INFINITY;
+    rg[NB + g] = INFINITY;
   }
-  __syncthreads();
+  rg[2 * NB] = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float* rw = wa + w * C::MW_FLOATS + kRows * D + kRows * 8 + kRows * NB;
+#pragma unroll
+    for (int g = 0; g < NB; ++g) {
+      rg[g] = fmaxf(rg[g], rw[g]);
+      rg[NB + g] = fminf(rg[NB + g], rw[NB + g]);
+    }
+    rg[2 * NB] = fmaxf(rg[2 * NB], rw[2 * NB]);
+  }
 
-  auto range_of = [&](const float* r) {
-    float rg = 0.f;
-    for (int g = 0; g < NB; ++g) rg = fmaxf(rg, r[g] - r[NB + g]);
-    return rg;
+  auto finalize = [&](float l, float A, float Bv, float E, float dm,
+                      const float (&rgv)[2 * NB + 1], const float (&ov)[CPL]) {
+    if (r >= a.R) return;
+    const int qi = r / a.G, h = kvh * a.G + r % a.G;
+    const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + h;
+    if (a.out) {
+      const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) a.out[row * D + lane * CPL + e] = ov[e] * inv_l;
+    }
+    if (lane == 0) {
+      float bd = 0.f;
+      if (l > 0.f) {
+        float range = 0.f;
+#pragma unroll
+        for (int g = 0; g < NB; ++g) range = fmaxf(range, rgv[g] - rgv[NB + g]);
+        const float tv = fminf(tanhf(0.5f * dm), A / Bv);
+        bd = kKappa * (tv * (range + 2.0f * rgv[2 * NB]) + E / l);
+      }
+      a.bound[row] = bd;
+      a.flags[row] = bd > a.tau ? 1 : 0;
+    }
   };
 
   if (active == 1) {  // the only split: finish here
-    for (int r = 0; r < kRows; ++r) {
-      const float* s = cst + r * 8;
-      finalize_row<D>(a, b, kvh, r, s[1], s[2], s[3], s[4], s[5], range_of(cr), cr[2 * NB],
-                      cm + r * D, tid, blockDim.x, tid == 0);
-    }
+    finalize(st5[0], st5[1], st5[2], st5[3], st5[4], rg, o);
     return;
   }
 
   // ---- write this split's record; the last CTA of (b, kvh) merges all --------------
   const int64_t unit = (int64_t)b * a.hkv + kvh;
   const int splits = gridDim.x;
-  float* rec = a.part + (unit * splits + split) * record_floats(D);
-  for (int i = tid; i < 2 * NB + 1; i += blockDim.x) rec[1 + i] = cr[i];
-  for (int i = tid; i < kRows * 8; i += blockDim.x) rec[kHdr + (i / 8) * (8 + D) + i % 8] = cst[i];
-  for (int i = tid; i < kRows * D; i += blockDim.x)
-    rec[kHdr + (i / D) * (8 + D) + 8 + i % D] = cm[i];
+  float* rec = a.part + (unit * splits + split) * RF;
+  if (r == 0 && lane == 0) {
+#pragma unroll
+    for (int i = 0; i < 2 * NB + 1; ++i) rec[1 + i] = rg[i];
+  }
+  if (lane == 0) {
+    rec[kHdr + r * (8 + D) + 0] = mW;
+#pragma unroll
+    for (int t = 0; t < 5; ++t) rec[kHdr + r * (8 + D) + 1 + t] = st5[t];
+  }
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) rec[kHdr + r * (8 + D) + 8 + lane * CPL + e] = o[e];
   __threadfence();
   __syncthreads();
   int* flag = reinterpret_cast<int*>(sm + C::OFF_FLAG);
@@ -693,64 +740,74 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
   __syncthreads();
   if (!*flag) return;
   __threadfence();
-  const float* recs = a.part + unit * splits * record_floats(D);
-  // statistics per row (every thread recomputes what it needs; reads hit L2)
-  float* fst = cst;   // reuse: merged stats of all splits
-  if (tid < kRows) {
-    const int r = tid;
-    float M = -INFINITY;
-    for (int s = 0; s < active; ++s)
-      M = fmaxf(M, __ldcg(recs + s * record_floats(D) + kHdr + r * (8 + D)));
-    float L = 0.f, A = 0.f, Bv = 0.f, Ev = 0.f, Dm = 0.f;
-    for (int s = 0; s < active; ++s) {
-      const float* st = recs + s * record_floats(D) + kHdr + r * (8 + D);
-      const float ms = __ldcg(st);
-      const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
-      L = fmaf(f, __ldcg(st + 1), L);
-      A = fmaf(f, __ldcg(st + 2), A);
-      Bv = fmaf(f, __ldcg(st + 3), Bv);
-      Ev = fmaf(f, __ldcg(st + 4), Ev);
-      Dm = fmaxf(Dm, __ldcg(st + 5));
-    }
-    fst[r * 8 + 0] = M;
-    fst[r * 8 + 1] = L;
-    fst[r * 8 + 2] = A;
-    fst[r * 8 + 3] = Bv;
-    fst[r * 8 + 4] = Ev;
-    fst[r * 8 + 5] = Dm;
-  } else if (tid == kRows) {
+  const float* recs = a.part + unit * splits * RF;
+  // statistics of row r over all splits, lanes striding over the splits
+  float M = -INFINITY;
+  for (int sp = lane; sp < active; sp += 32) M = fmaxf(M, __ldcg(recs + (int64_t)sp * RF + kHdr + r * (8 + D)));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float t5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int g = 0; g < NB; ++g) {
+    rg[g] = -INFINITY;
+    rg[NB + g] = INFINITY;
+  }
+  rg[2 * NB] = 0.f;
+  for (int sp = lane; sp < active; sp += 32) {
+    const float* rp = recs + (int64_t)sp * RF;
+    const float* st = rp + kHdr + r * (8 + D);
+    const float ms = __ldcg(st);
+    const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) t5[t] = fmaf(f, __ldcg(st + 1 + t), t5[t]);
+    t5[4] = fmaxf(t5[4], __ldcg(st + 5));
+#pragma unroll
     for (int g = 0; g < NB; ++g) {
-      float hi = -INFINITY, lo = INFINITY;
-      for (int s = 0; s < active; ++s) {
-        hi = fmaxf(hi, __ldcg(recs + s * record_floats(D) + 1 + g));
-        lo = fminf(lo, __ldcg(recs + s * record_floats(D) + 1 + NB + g));
+      rg[g] = fmaxf(rg[g], __ldcg(rp + 1 + g));
+      rg[NB + g] = fminf(rg[NB + g], __ldcg(rp + 1 + NB + g));
+    }
+    rg[2 * NB] = fmaxf(rg[2 * NB], __ldcg(rp + 1 + 2 * NB));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+    for (int t = 0; t < 4; ++t) t5[t] += __shfl_xor_sync(0xffffffffu, t5[t], off);
+    t5[4] = fmaxf(t5[4], __shfl_xor_sync(0xffffffffu, t5[4], off));
+#pragma unroll
+    for (int g = 0; g < NB; ++g) {
+      rg[g] = fmaxf(rg[g], __shfl_xor_sync(0xffffffffu, rg[g], off));
+      rg[NB + g] = fminf(rg[NB + g], __shfl_xor_sync(0xffffffffu, rg[NB + g], off));
+    }
+    rg[2 * NB] = fmaxf(rg[2 * NB], __shfl_xor_sync(0xffffffffu, rg[2 * NB], off));
+  }
+  // outputs: chunks of 32 splits, the weights broadcast from lane sp % 32
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) o[e] = 0.f;
+  for (int c0 = 0; c0 < active; c0 += 32) {
+    const int ns = min(32, active - c0);
+    float fl = 0.f;
+    if (lane < ns) {
+      const float ms = __ldcg(recs + (int64_t)(c0 + lane) * RF + kHdr + r * (8 + D));
+      fl = ms == -INFINITY ? 0.f : exp2f(ms - M);
+    }
+#pragma unroll 4
+    for (int i = 0; i < ns; ++i) {
+      const float f = __shfl_sync(0xffffffffu, fl, i);
+      const float* op = recs + (int64_t)(c0 + i) * RF + kHdr + r * (8 + D) + 8 + lane * CPL;
+      if constexpr (CPL == 4) {
+        const float4 v4 = __ldcg(reinterpret_cast<const float4*>(op));
+        o[0] = fmaf(f, v4.x, o[0]);
+        o[1] = fmaf(f, v4.y, o[1]);
+        o[2] = fmaf(f, v4.z, o[2]);
+        o[3] = fmaf(f, v4.w, o[3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) o[e] = fmaf(f, __ldcg(op + e), o[e]);
       }
-      cr[g] = hi;
-      cr[NB + g] = lo;
     }
-    float et = 0.f;
-    for (int s = 0; s < active; ++s) et = fmaxf(et, __ldcg(recs + s * record_floats(D) + 1 + 2 * NB));
-    cr[2 * NB] = et;
   }
+  finalize(t5[0], t5[1], t5[2], t5[3], t5[4], rg, o);
   __syncthreads();
-  for (int i = tid; i < kRows * D; i += blockDim.x) {
-    const int r = i / D, c = i % D;
-    const float M = fst[r * 8];
-    float o = 0.f;
-    for (int s = 0; s < active; ++s) {
-      const float* st = recs + s * record_floats(D) + kHdr + r * (8 + D);
-      const float ms = __ldcg(st);
-      if (ms == -INFINITY) continue;
-      o = fmaf(exp2f(ms - M), __ldcg(st + 8 + c), o);
-    }
-    cm[i] = o;
-  }
-  __syncthreads();
-  for (int r = 0; r < kRows; ++r) {
-    const float* s = fst + r * 8;
-    finalize_row<D>(a, b, kvh, r, s[1], s[2], s[3], s[4], s[5], range_of(cr), cr[2 * NB],
-                    cm + r * D, tid, blockDim.x, tid == 0);
-  }
   if (tid == 0) a.counters[unit] = 0;  // leave the workspace ready for the next call
 }
 
