@@ -92,13 +92,33 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   constexpr int NB = C::NB, NGK = C::NGK;
   constexpr int Q = KB == 8 ? 127 : 7;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~(uintptr_t)1023);
+  // 1024-byte aligned base (swizzled TMA tiles); pointer arithmetic on the
+  // __shared__ array keeps every access below in the shared address space
+  uint8_t* sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c4 = lane & 3, g8 = lane >> 2;
 
+  // The context length, the query rows and this warp's first 32 page indices
+  // are loaded together: none of these addresses depends on the others.
+  const int p0 = split * a.pps;
+  const int first = p0 + warp;
+  const int32_t* ptab = a.page_table + (int64_t)b * a.max_pages;
   int n = a.seq_lens[b];
+  const int pt_first = first + lane * kWarps < min(p0 + a.pps, a.max_pages)
+                           ? __ldg(ptab + first + lane * kWarps) : -1;
+  constexpr int QPT = kRows * D / (kWarps * 32);   // query elements per thread
+  float qreg[QPT];
+#pragma unroll
+  for (int k = 0; k < QPT; ++k) {
+    const int i = tid + k * kWarps * 32, r = i / D, c = i % D;
+    qreg[k] = 0.f;
+    if (r < a.R) {
+      const int qi = r / a.G, h = kvh * a.G + r % a.G;
+      qreg[k] = load_elem(a.q, a.q_bf16, (((int64_t)b * a.nq + qi) * a.hq + h) * D + c);
+    }
+  }
+
   if (n < 0) n = 0;
   if (n > a.max_pages * kPage) {
     if (tid == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
@@ -120,7 +140,6 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     }
     return;
   }
-  const int p0 = split * a.pps;
   const int p1 = min(p0 + a.pps, npages);
 
   uint8_t* ktile = sm + C::OFF_KT + warp * S * C::KT;
@@ -132,28 +151,13 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   float* qf = reinterpret_cast<float*>(sm + C::OFF_QF);
   float* rc = reinterpret_cast<float*>(sm + C::OFF_RC);
 
-  // the query rows go first, ahead of the page copies in the memory queues
-  constexpr int QPT = kRows * D / (kWarps * 32);   // query elements per thread
-  float qreg[QPT];
-#pragma unroll
-  for (int k = 0; k < QPT; ++k) {
-    const int i = tid + k * kWarps * 32, r = i / D, c = i % D;
-    qreg[k] = 0.f;
-    if (r < a.R) {
-      const int qi = r / a.G, h = kvh * a.G + r % a.G;
-      qreg[k] = load_elem(a.q, a.q_bf16, (((int64_t)b * a.nq + qi) * a.hq + h) * D + c);
-    }
-  }
-
   // ---- pipeline start: page indices, barriers, first S copies --------------
-  const int first = p0 + warp;
   const int nloc = first < p1 ? (p1 - first + kWarps - 1) / kWarps : 0;
-  const int32_t* ptab = a.page_table + (int64_t)b * a.max_pages;
   auto fetch_chunk = [&](int c) -> int {
     const int j = c * 32 + lane;
     return j < nloc ? __ldg(ptab + first + j * kWarps) : -1;
   };
-  int pt_chunk = -1, pt_val = -1, pt_next = fetch_chunk(0);
+  int pt_chunk = -1, pt_val = -1, pt_next = lane < nloc ? pt_first : -1;
   if (lane == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
     mbar_fence_init();
@@ -161,7 +165,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   if (tid == 0) prefetch_tensormap(&kmap);
   __syncwarp();
 
-  auto issue = [&](int j) {  // whole warp calls; lane 0 issues the copies of local page j
+  auto issue = [&](int j, int st) {  // whole warp; lane 0 issues local page j into stage st
     const int c = j >> 5;
     if (c != pt_chunk) {
       pt_val = (c == pt_chunk + 1) ? pt_next : fetch_chunk(c);
@@ -169,7 +173,6 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       pt_chunk = c;
     }
     const int page = __shfl_sync(0xffffffffu, pt_val, j & 31);
-    const int st = j % S;
     if (lane == 0) {
       const bool ok = page >= 0 && page < a.num_pages;
       spage[st] = ok ? page : -1;
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     }
     __syncwarp();  // publish spage[st] to the warp
   };
-  for (int j = 0; j < S && j < nloc; ++j) issue(j);
+  for (int j = 0; j < S && j < nloc; ++j) issue(j, j);
 
   // ---- query rows: rotate, fixed point, norms (loaded before the copies) -----
 #pragma unroll
@@ -316,9 +319,14 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   float* ks32 = vs32 + kPage * NB;
   // hi part of a value: its top 11 significant bits (exact in fp16); lo lanes
   // take the remainder, so hi + lo reproduces the fp32 value to ~2^-22
-  auto hilo = [&](float v) {
-    const float t = __int_as_float(__float_as_int(v) & 0xFFFFE000);
-    return lo_part ? v - t : t;
+  // (two at a time: v = K1*t + K2*x with (K1, K2) = (1, 0) or (-1, 1))
+  const float2 K1 = lo_part ? make_float2(-1.f, -1.f) : make_float2(1.f, 1.f);
+  const float2 K2 = lo_part ? make_float2(1.f, 1.f) : make_float2(0.f, 0.f);
+  auto hilo2 = [&](float2 v) -> uint32_t {
+    const float2 t = make_float2(__int_as_float(__float_as_int(v.x) & 0xFFFFE000),
+                                 __int_as_float(__float_as_int(v.y) & 0xFFFFE000));
+    const float2 r = fma2(t, K1, mul2(v, K2));
+    return h2_as_u32(__floats2half2_rn(r.x, r.y));
   };
 
   const float* eta_kv = a.eta + kvh;
@@ -328,27 +336,43 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     const int pg = spage[0];
     eta_next = pg >= 0 ? __ldg(eta_kv + (int64_t)pg * a.hkv) : 0.f;
   }
+  // this lane's fixed offsets inside a stage
+  constexpr int KW = C::KSTR / 4;                        // 32-bit words per key stripe
+  constexpr int KCH = C::KSTR >= 16 ? C::KSTR / 16 : 1;  // 16-byte chunks per key stripe
+  int koff[KCH];                                         // row g8; row g8+8 is +8 rows
+#pragma unroll
+  for (int hh = 0; hh < KCH; ++hh) {
+    if constexpr (C::KSTR >= 16) {
+      int chunk = (c4 * C::KSTR) / 16 + hh;
+      if (C::SWZ) chunk ^= (g8 & 7);
+      koff[hh] = g8 * C::KRB + chunk * 16;
+    } else {
+      koff[hh] = g8 * C::KRB + c4 * C::KSTR;
+    }
+  }
+  const int voff = c4 * C::VRB + g8 * C::VSTR;           // V stripe of token c4 (+4 rows per k)
+  const int zgrp = g8 < NB ? g8 : 0;
 
   // ---- page loop ---------------------------------------------------------------
+  int st = 0;
+  uint32_t par = 0;
   for (int j = 0; j < nloc; ++j) {
-    const int st = j % S;
-    const uint32_t par = (uint32_t)((j / S) & 1);
     bool ok = mbar_wait(&bar[st], par);
     if (!__all_sync(0xffffffffu, ok)) {
       if (lane == 0) set_error(a.err, KVQ_ERR_TIMEOUT);
       break;
     }
+    const int stn = st + 1 == S ? 0 : st + 1;
     const int page = spage[st];
     const float eta_cur = eta_next;
     if (j + 1 < nloc) {
-      const int pn = spage[(j + 1) % S];
+      const int pn = spage[stn];
       eta_next = pn >= 0 ? __ldg(eta_kv + (int64_t)pn * a.hkv) : 0.f;
     }
     if (page >= 0) {
       const uint8_t* kt = ktile + st * C::KT;
       const uint8_t* rs = rest + st * C::REST;
-      const int tok0 = (first + j * kWarps) * kPage;
-      const int nval = min(kPage, n - tok0);
+      const int nval = min(kPage, n - (first + j * kWarps) * kPage);
       etamax = fmaxf(etamax, eta_cur);
       const uint32_t* vm = reinterpret_cast<const uint32_t*>(rs + C::VB + C::KSB);
       const __half* ksc = reinterpret_cast<const __half*>(rs + C::VB);
@@ -366,37 +390,32 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
           const int e = lane * EPL + i;  // token e / NB, group e % NB
-          const __half2 sz = u32_as_h2(mw[i]);
-          const float s = __low2float(sz), z = __high2float(sz);
+          const float2 sz = __half22float2(u32_as_h2(mw[i]));
           const bool in = e / NB < nval;
-          vs32[e] = in ? s : 0.f;
-          if (in) {
-            vhi[i] = fmaxf(vhi[i], __fmaf_rn(15.0f, s, z));
-            vlo[i] = fminf(vlo[i], z);
-          }
+          const int tok = e / NB, gg = e % NB;   // table [group][token % 4][token / 4]
+          vs32[gg * kPage + (tok % 4) * 4 + tok / 4] = in ? sz.x : 0.f;
+          vhi[i] = in ? fmaxf(vhi[i], __fmaf_rn(15.0f, sz.x, sz.y)) : vhi[i];
+          vlo[i] = in ? fminf(vlo[i], sz.y) : vlo[i];
         }
         for (int e = lane; e < kPage * NGK; e += 32) ks32[e] = __half2float(ksc[e]);
       }
 
       // --- K codes of rows g8, g8+8 (this lane's stripe) -> QK^T on int8 MMA ---
-      constexpr int KW = C::KSTR / 4;    // 32-bit words per stripe
       uint32_t wk[2][KW];
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
-        const int row = g8 + 8 * rr;
+        const uint8_t* kr = kt + rr * 8 * C::KRB;
         if constexpr (C::KSTR >= 16) {
 #pragma unroll
-          for (int hh = 0; hh < C::KSTR / 16; ++hh) {
-            int chunk = (c4 * C::KSTR) / 16 + hh;
-            if (C::SWZ) chunk ^= (row & 7);
-            const uint4 v4 = *reinterpret_cast<const uint4*>(kt + row * C::KRB + chunk * 16);
+          for (int hh = 0; hh < KCH; ++hh) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(kr + koff[hh]);
             wk[rr][4 * hh + 0] = v4.x;
             wk[rr][4 * hh + 1] = v4.y;
             wk[rr][4 * hh + 2] = v4.z;
             wk[rr][4 * hh + 3] = v4.w;
           }
         } else {
-          const uint2 v2 = *reinterpret_cast<const uint2*>(kt + row * C::KRB + c4 * C::KSTR);
+          const uint2 v2 = *reinterpret_cast<const uint2*>(kr + koff[0]);
           wk[rr][0] = v2.x;
           wk[rr][1] = v2.y;
         }
@@ -434,25 +453,34 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 
       // --- scores (log2 units) and Delta for tokens g8, g8+8 of row c4 -------------
       float zt[2], dl[2];
-      bool vt[2];
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
         const int tok = g8 + 8 * sl;
-        vt[sl] = tok < nval;
+        const bool vt = tok < nval;
         float dot = 0.f, dsum = 0.f, smax = 0.f;
+        float sg[NGK];
+        if constexpr (NGK == 4) {
+          const float4 f4 = *reinterpret_cast<const float4*>(ks32 + tok * 4);
+          sg[0] = f4.x;
+          sg[1] = f4.y;
+          sg[2] = f4.z;
+          sg[3] = f4.w;
+        } else {
+#pragma unroll
+          for (int g = 0; g < NGK; ++g) sg[g] = ks32[tok * NGK + g];
+        }
 #pragma unroll
         for (int g = 0; g < NGK; ++g) {
-          const float s = ks32[tok * NGK + g];
           // digits 0,1 and 2,3 recombined exactly in int32, then once in fp32
-          const int lo = acc[g][0][2 * sl] + acc[g][0][2 * sl + 1] * 256;
-          const int hi = acc[g][1][2 * sl] + acc[g][1][2 * sl + 1] * 256;
+          const int lo = acc[g][0][2 * sl] + (acc[g][0][2 * sl + 1] << 8);
+          const int hi = acc[g][1][2 * sl] + (acc[g][1][2 * sl + 1] << 8);
           const float raw = fmaf((float)hi, 65536.f, (float)lo);
-          dot = fmaf(raw, s, dot);
-          dsum = fmaf(cg[g], s, dsum);
-          smax = fmaxf(smax, s);
+          dot = fmaf(raw, sg[g], dot);
+          dsum = fmaf(cg[g], sg[g], dsum);
+          smax = fmaxf(smax, sg[g]);
         }
-        zt[sl] = vt[sl] ? dot * zs : -INFINITY;
-        dl[sl] = fmaf(cb, smax, dsum);
+        zt[sl] = vt ? dot * zs : -INFINITY;
+        dl[sl] = vt ? fmaf(cb, smax, dsum) : 0.f;
       }
 
       // --- online softmax and bound sums (row c4) -------------------------------
@@ -460,28 +488,30 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float mnew = fmaxf(m2, mx);
-      const float alpha = exp2f(m2 - mnew);
-      m2 = mnew;
-      const float w0 = exp2f(zt[0] - mnew), w1 = exp2f(zt[1] - mnew);
-      float ta = 0.f, tb = 0.f, tw = 0.f;
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        if (vt[sl]) {
-          const float w = sl ? w1 : w0;
-          const float d = dl[sl];
-          const float ep = exp2f(d * kLog2e), en = exp2f(-d * kLog2e);
-          // e^d - 1: Taylor to d^5 below 1/16 (no cancellation), else from e^d
-          const float em1 =
-              d < 0.0625f
-                  ? d * fmaf(d, fmaf(d, fmaf(d, fmaf(d, 1.0f / 120, 1.0f / 24), 1.0f / 6), 0.5f), 1.0f)
-                  : ep - 1.0f;
-          ta = fmaf(w, em1, ta);
-          tb = fmaf(w, en, tb);
-          tw += w;
-          dmax = fmaxf(dmax, d);
-        }
-      }
+      // The reference max moves only when the page max exceeds it by more than
+      // 2 (log2 units): weights stay <= 4, so w * sV fits fp16 for any finite
+      // value scale, and the accumulators are rescaled on few pages.
+      const float mref = mx > m2 + 2.0f ? mx : m2;
+      const float alpha = exp2f(m2 - mref);
+      m2 = mref;
+      const float w0 = exp2f(zt[0] - mref), w1 = exp2f(zt[1] - mref);
+      // tokens outside the context have w = 0 and Delta = 0
+      const float2 d2 = make_float2(dl[0], dl[1]);
+      const float2 e2 = mul2(d2, make_float2(kLog2e, kLog2e));
+      const float2 ep = make_float2(exp2f(e2.x), exp2f(e2.y));
+      const float2 en = make_float2(exp2f(-e2.x), exp2f(-e2.y));
+      // e^d - 1: Taylor to d^5 below 1/16 (no cancellation), else from e^d
+      float2 pl = fma2(d2, make_float2(1.0f / 120, 1.0f / 120), make_float2(1.0f / 24, 1.0f / 24));
+      pl = fma2(d2, pl, make_float2(1.0f / 6, 1.0f / 6));
+      pl = fma2(d2, pl, make_float2(0.5f, 0.5f));
+      pl = fma2(d2, pl, make_float2(1.0f, 1.0f));
+      pl = mul2(d2, pl);
+      const float em0 = d2.x < 0.0625f ? pl.x : ep.x - 1.0f;
+      const float em1 = d2.y < 0.0625f ? pl.y : ep.y - 1.0f;
+      const float ta = fmaf(w1, em1, w0 * em0);
+      const float tb = fmaf(w1, en.y, w0 * en.x);
+      dmax = fmaxf(dmax, fmaxf(d2.x, d2.y));
+      const float tw = w0 + w1;
       lsum = fmaf(lsum, alpha, tw);
       Asum = fmaf(Asum, alpha, ta);
       Bsum = fmaf(Bsum, alpha, tb);
@@ -516,11 +546,11 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int tok = c4 + 4 * k;
-          const uint32_t wv = vm[tok * NB + (g8 < NB ? g8 : 0)];
+          const uint32_t wv = vm[tok * NB + zgrp];
           zw[k] = (g8 < NB && tok < nval) ? wv : 0u;
         }
-        const uint32_t bz0 = h2_as_u32(__floats2half2_rn(hilo(x[0]), hilo(x[1])));
-        const uint32_t bz1 = h2_as_u32(__floats2half2_rn(hilo(x[2]), hilo(x[3])));
+        const uint32_t bz0 = hilo2(make_float2(x[0], x[1]));
+        const uint32_t bz1 = hilo2(make_float2(x[2], x[3]));
         mma_f16(zmv, prmt(zw[0], zw[1], 0x7632u), 0u, prmt(zw[2], zw[3], 0x7632u), 0u, bz0, bz1);
       }
 
@@ -528,7 +558,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       uint32_t vw[4][C::VSTR / 4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint8_t* p = rs + (c4 + 4 * k) * C::VRB + g8 * C::VSTR;
+        const uint8_t* p = rs + voff + 4 * k * C::VRB;
         if constexpr (C::VSTR == 8) {
           const uint2 v2 = *reinterpret_cast<const uint2*>(p);
           vw[k][0] = v2.x;
@@ -537,26 +567,12 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
           vw[k][0] = *reinterpret_cast<const uint32_t*>(p);
         }
       }
-      float sv[4][NB];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if constexpr (NB == 4) {
-          const float4 f = *reinterpret_cast<const float4*>(vs32 + (c4 + 4 * k) * NB);
-          sv[k][0] = f.x;
-          sv[k][1] = f.y;
-          sv[k][2] = f.z;
-          sv[k][3] = f.w;
-        } else {
-          const float2 f = *reinterpret_cast<const float2*>(vs32 + (c4 + 4 * k) * NB);
-          sv[k][0] = f.x;
-          sv[k][1] = f.y;
-        }
-      }
 #pragma unroll
       for (int g = 0; g < NB; ++g) {
-        // P' = w * sV (zero outside the context), as fp16 hi or lo part
-        const uint32_t b01 = h2_as_u32(__floats2half2_rn(hilo(x[0] * sv[0][g]), hilo(x[1] * sv[1][g])));
-        const uint32_t b23 = h2_as_u32(__floats2half2_rn(hilo(x[2] * sv[2][g]), hilo(x[3] * sv[3][g])));
+        // P' = w * sV of tokens c4 + 4k (zero outside the context), fp16 hi or lo part
+        const float4 sv = *reinterpret_cast<const float4*>(vs32 + g * kPage + c4 * 4);
+        const uint32_t b01 = hilo2(mul2(make_float2(x[0], x[1]), make_float2(sv.x, sv.y)));
+        const uint32_t b23 = hilo2(mul2(make_float2(x[2], x[3]), make_float2(sv.z, sv.w)));
         const int wsel = (2 * g) / 4;            // stripe word holding group g
         const int p = (2 * g) % 4;               // byte offset of group g in that word
         const uint32_t sel = (uint32_t)(p | ((p + 1) << 4) | ((4 + p) << 8) | ((5 + p) << 12));
@@ -570,7 +586,9 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       }
     }
     __syncwarp();
-    if (j + S < nloc) issue(j + S);
+    if (j + S < nloc) issue(j + S, st);
+    st = stn;
+    par ^= (stn == 0) ? 1u : 0u;
   }
 
   // ---- warp reductions ----------------------------------------------------------

@@ -140,6 +140,24 @@ __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
   return *reinterpret_cast<__half2*>(&u);
 }
 
+// ---- packed fp32x2 arithmetic (one instruction for two IEEE fp32 lanes) ------
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+      "mul.rn.f32x2 pd, pa, pb;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 pa, pb, pc, pd;\n\tmov.b64 pa, {%2, %3};\n\tmov.b64 pb, {%4, %5};\n\t"
+      "mov.b64 pc, {%6, %7};\n\tfma.rn.f32x2 pd, pa, pb, pc;\n\tmov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
 // ---- randomized Walsh-Hadamard rotation of one vector held by a warp ------
 // Lane l holds elements [l*E, l*E + E) of a d = 32*E vector.  Computes
 // y = c * H_d * (sigma o x) with butterflies in the fixed order stride 1, 2,
