@@ -81,10 +81,20 @@ def _traffic_record():
         return None
 
 
+def _smi_time(stamp: str):
+    """nvidia-smi timestamp ('YYYY/MM/DD HH:MM:SS.mmm', local time) -> epoch seconds."""
+    try:
+        base, _, frac = stamp.strip().partition(".")
+        t = time.mktime(time.strptime(base, "%Y/%m/%d %H:%M:%S"))
+        return t + (float("0." + frac) if frac.isdigit() else 0.0)
+    except ValueError:
+        return None
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled during the timed region."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -97,7 +107,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -108,10 +118,11 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
+    def stop(self, window=None):
+        """Median clocks of the samples taken inside `window` (host epoch seconds)."""
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -124,6 +135,10 @@ class ClockSampler:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
+            if window is not None:
+                t = _smi_time(f[0])
+                if t is None or not (window[0] - 0.02 <= t <= window[1] + 0.02):
+                    continue
             try:
                 sm.append(float(f[1]))
                 mx.append(float(f[2]))
@@ -221,7 +236,8 @@ class GpuStep:
         self.out = torch.empty((B, NQ, HQ, d), dtype=torch.float32, device="cuda")
         self.bound = torch.empty((B, NQ, HQ), dtype=torch.float32, device="cuda")
         self.flags = torch.empty((B, NQ, HQ), dtype=torch.uint8, device="cuda")
-        self.stream = torch.cuda.current_stream()
+        # one dedicated stream: the eager steps and the captured graph use it
+        self.stream = torch.cuda.Stream()
         s = self.stream.cuda_stream
         L = kvq.lib()
         self.L = L
@@ -266,14 +282,26 @@ def run_gpu(args):
     reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl))))
     reps = min(reps, 8)
     st = GpuStep(args.workload, args.seed, reps)
-    for i in range(args.warmup):
-        st.step(i)
+    # setup: one untimed call per cache replica (library-side descriptors and
+    # occupancy are cached by the first call), then the W warm-up steps
+    with torch.cuda.stream(st.stream):
+        for r in range(reps):
+            st.step(r)
+        for i in range(args.warmup):
+            st.step(i)
     torch.cuda.synchronize()
     err = st.caches[0].device_error()
     if err:
         raise RuntimeError(f"device error {err} during warm-up")
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    # the K timed steps are captured into one CUDA graph (kernels, and timing
+    # events around every decode launch); the timed region is its replay
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=st.stream):
+        for i in range(args.steps):
+            st.step(args.warmup + i, evs[i])
+    torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local) if rank == 0 else None
@@ -282,12 +310,16 @@ def run_gpu(args):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    t0.record()
-    for i in range(args.steps):
-        st.step(args.warmup + i, evs[i])
-    t1.record()
+    w0 = time.time()
+    with torch.cuda.stream(st.stream):
+        t0.record(st.stream)
+        graph.replay()
+        t1.record(st.stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop() if sampler else None
+    w1 = time.time()
+    clocks = sampler.stop((w0, w1)) if sampler else None
+    if clocks is None and sampler:
+        clocks = {"sm_mhz": None, "note": "timed region shorter than the 20 ms sampling period"}
     _barrier(world)
     ms_total = t0.elapsed_time(t1)
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
@@ -310,16 +342,17 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(e_steps):
-        st.qd.copy_(q_h, non_blocking=True)
-        st.k_new.copy_(kn_h, non_blocking=True)
-        st.v_new.copy_(vn_h, non_blocking=True)
-        st.step(i)
-        out_h.copy_(st.out, non_blocking=True)
-        bound_h.copy_(st.bound, non_blocking=True)
-        flags_h.copy_(st.flags, non_blocking=True)
-    e1.record()
+    with torch.cuda.stream(st.stream):
+        e0.record(st.stream)
+        for i in range(e_steps):
+            st.qd.copy_(q_h, non_blocking=True)
+            st.k_new.copy_(kn_h, non_blocking=True)
+            st.v_new.copy_(vn_h, non_blocking=True)
+            st.step(i)
+            out_h.copy_(st.out, non_blocking=True)
+            bound_h.copy_(st.bound, non_blocking=True)
+            flags_h.copy_(st.flags, non_blocking=True)
+        e1.record(st.stream)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e_steps, world)
 
@@ -452,7 +485,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--seed", type=int, default=0)
