@@ -26,12 +26,14 @@
 //         value range [min z, max fmaf(15, s, z)] per group.
 //   PV    fp16 tensor cores: V codes are exact in fp16; the per-token group
 //         scale is folded into P' = w * sV (split hi + lo, both fp16, so the
-//         product keeps ~22 bits) and the zero point is added as
-//         sum_j w_j zV_{j,g} on CUDA cores.
+//         product keeps ~22 bits); the zero point adds sum_j w_j zV_{j,g}
+//         through one more MMA per page (rows = groups).
 // Warps merge in shared memory; splits merge in the last CTA of each
 // (sequence, kv head) to finish: o = O/l, TV = min(tanh(maxDelta/2), A/B),
 // E_key = TV*(range + 2 max eta), E_val = E/l, bound = kappa*(E_key+E_val),
 // flag = bound > tau.
+#include <type_traits>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -98,6 +100,14 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c4 = lane & 3, g8 = lane >> 2;
+  // The key-tile descriptor and this warp's ring barriers need nothing from
+  // memory: start them first, so their latency overlaps the loads below.
+  if (tid == 0) prefetch_tensormap(&kmap);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + warp * S;
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
+    mbar_fence_init();
+  }
 
   // The context length, the query rows and this warp's first 32 page indices
   // are loaded together: none of these addresses depends on the others.
@@ -144,7 +154,6 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 
   uint8_t* ktile = sm + C::OFF_KT + warp * S * C::KT;
   uint8_t* rest = sm + C::OFF_RS + warp * S * C::REST;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + warp * S;
   int* spage = reinterpret_cast<int*>(sm + C::OFF_PG) + warp * S;
   int8_t* qdig = reinterpret_cast<int8_t*>(sm + C::OFF_Q);
   int* qsum = reinterpret_cast<int*>(sm + C::OFF_QB);
@@ -158,11 +167,6 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     return j < nloc ? __ldg(ptab + first + j * kWarps) : -1;
   };
   int pt_chunk = -1, pt_val = -1, pt_next = lane < nloc ? pt_first : -1;
-  if (lane == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
-    mbar_fence_init();
-  }
-  if (tid == 0) prefetch_tensormap(&kmap);
   __syncwarp();
 
   auto issue = [&](int j, int st) {  // whole warp; lane 0 issues local page j into stage st
@@ -748,22 +752,29 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   }
 #pragma unroll
   for (int e = 0; e < CPL; ++e) rec[kHdr + r * (8 + D) + 8 + lane * CPL + e] = o[e];
-  __threadfence();
+  // The barrier orders every thread's record stores before thread 0's ticket;
+  // the ticket's release publishes them at GPU scope and, for the last CTA,
+  // its acquire makes every other CTA's records visible to the whole CTA
+  // (through the second barrier).
   __syncthreads();
   int* flag = reinterpret_cast<int*>(sm + C::OFF_FLAG);
   if (tid == 0) {
-    const int prev = atomicAdd(a.counters + unit, 1);
+    const int prev = atomic_add_acq_rel(a.counters + unit, 1);
     *flag = prev == active - 1;
   }
   __syncthreads();
   if (!*flag) return;
-  __threadfence();
+
+  // ---- last CTA: merge the records of all active splits, row r per warp -------------
+  // Splits are taken in chunks of 32 * KS: lane l reads the statistics of splits
+  // c0 + l + 32k together, the chunk's running maximum rescales what came before,
+  // and the outputs are read 16 splits at a time (lane l owns CPL channels), each
+  // split's weight broadcast from the lane that read its statistics.
+  using VT = typename std::conditional<CPL == 4, float4, float2>::type;
+  constexpr int KS = 4;
+  constexpr int SUB = 16;
   const float* recs = a.part + unit * splits * RF;
-  // statistics of row r over all splits, lanes striding over the splits
-  float M = -INFINITY;
-  for (int sp = lane; sp < active; sp += 32) M = fmaxf(M, __ldcg(recs + (int64_t)sp * RF + kHdr + r * (8 + D)));
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float Mr = -INFINITY;
   float t5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int g = 0; g < NB; ++g) {
@@ -771,58 +782,108 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     rg[NB + g] = INFINITY;
   }
   rg[2 * NB] = 0.f;
-  for (int sp = lane; sp < active; sp += 32) {
-    const float* rp = recs + (int64_t)sp * RF;
-    const float* st = rp + kHdr + r * (8 + D);
-    const float ms = __ldcg(st);
-    const float f = ms == -INFINITY ? 0.f : exp2f(ms - M);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) t5[t] = fmaf(f, __ldcg(st + 1 + t), t5[t]);
-    t5[4] = fmaxf(t5[4], __ldcg(st + 5));
+  for (int e = 0; e < CPL; ++e) o[e] = 0.f;
+  auto out_of = [&](int sp) -> const VT* {
+    return reinterpret_cast<const VT*>(recs + (int64_t)sp * RF + kHdr + r * (8 + D) + 8 +
+                                       lane * CPL);
+  };
+  for (int c0 = 0; c0 < active; c0 += 32 * KS) {
+    float4 sa[KS];  // (m, l, A, B) of split c0 + 32k + lane
+    float2 sb[KS];  // (E, max Delta)
 #pragma unroll
-    for (int g = 0; g < NB; ++g) {
-      rg[g] = fmaxf(rg[g], __ldcg(rp + 1 + g));
-      rg[NB + g] = fminf(rg[NB + g], __ldcg(rp + 1 + NB + g));
+    for (int k = 0; k < KS; ++k) {
+      const int sp = c0 + 32 * k + lane;
+      sa[k] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+      sb[k] = make_float2(0.f, 0.f);
+      if (sp < active) {
+        const float* st = recs + (int64_t)sp * RF + kHdr + r * (8 + D);
+        sa[k] = __ldcg(reinterpret_cast<const float4*>(st));
+        sb[k] = __ldcg(reinterpret_cast<const float2*>(st + 4));
+        const float* rp = recs + (int64_t)sp * RF + 1;
+#pragma unroll
+        for (int g = 0; g < NB; ++g) {
+          rg[g] = fmaxf(rg[g], __ldcg(rp + g));
+          rg[NB + g] = fminf(rg[NB + g], __ldcg(rp + NB + g));
+        }
+        rg[2 * NB] = fmaxf(rg[2 * NB], __ldcg(rp + 2 * NB));
+      }
     }
-    rg[2 * NB] = fmaxf(rg[2 * NB], __ldcg(rp + 1 + 2 * NB));
+    // the first outputs of the chunk are read together with its statistics
+    VT v0[SUB];
+#pragma unroll
+    for (int i = 0; i < SUB; ++i) {
+      const int sp = c0 + i;
+      v0[i] = sp < active ? __ldcg(out_of(sp)) : VT{};
+    }
+    float Mc = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KS; ++k) Mc = fmaxf(Mc, sa[k].x);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
+    const float Mn = fmaxf(Mr, Mc);
+    const float sc = Mr == -INFINITY ? 0.f : exp2f(Mr - Mn);
+    Mr = Mn;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) t5[t] *= sc;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) o[e] *= sc;
+    float f[KS], p5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      f[k] = sa[k].x == -INFINITY ? 0.f : exp2f(sa[k].x - Mn);
+      p5[0] = fmaf(f[k], sa[k].y, p5[0]);
+      p5[1] = fmaf(f[k], sa[k].z, p5[1]);
+      p5[2] = fmaf(f[k], sa[k].w, p5[2]);
+      p5[3] = fmaf(f[k], sb[k].x, p5[3]);
+      p5[4] = fmaxf(p5[4], sb[k].y);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) p5[t] += __shfl_xor_sync(0xffffffffu, p5[t], off);
+      p5[4] = fmaxf(p5[4], __shfl_xor_sync(0xffffffffu, p5[4], off));
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) t5[t] += p5[t];
+    t5[4] = fmaxf(t5[4], p5[4]);
+    auto accumulate = [&](int ib, const VT (&v)[SUB]) {
+#pragma unroll
+      for (int i = 0; i < SUB; ++i) {
+        const float fs = __shfl_sync(0xffffffffu, f[(ib + i) / 32], (ib + i) % 32);
+        if constexpr (CPL == 4) {
+          o[0] = fmaf(fs, v[i].x, o[0]);
+          o[1] = fmaf(fs, v[i].y, o[1]);
+          o[2] = fmaf(fs, v[i].z, o[2]);
+          o[3] = fmaf(fs, v[i].w, o[3]);
+        } else {
+          o[0] = fmaf(fs, v[i].x, o[0]);
+          o[1] = fmaf(fs, v[i].y, o[1]);
+        }
+      }
+    };
+    accumulate(0, v0);
+#pragma unroll
+    for (int ib = SUB; ib < 32 * KS; ib += SUB) {
+      if (c0 + ib < active) {  // warp-uniform
+        VT v[SUB];
+#pragma unroll
+        for (int i = 0; i < SUB; ++i) {
+          const int sp = c0 + ib + i;
+          v[i] = sp < active ? __ldcg(out_of(sp)) : VT{};
+        }
+        accumulate(ib, v);
+      }
+    }
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) t5[t] += __shfl_xor_sync(0xffffffffu, t5[t], off);
-    t5[4] = fmaxf(t5[4], __shfl_xor_sync(0xffffffffu, t5[4], off));
 #pragma unroll
     for (int g = 0; g < NB; ++g) {
       rg[g] = fmaxf(rg[g], __shfl_xor_sync(0xffffffffu, rg[g], off));
       rg[NB + g] = fminf(rg[NB + g], __shfl_xor_sync(0xffffffffu, rg[NB + g], off));
     }
     rg[2 * NB] = fmaxf(rg[2 * NB], __shfl_xor_sync(0xffffffffu, rg[2 * NB], off));
-  }
-  // outputs: chunks of 32 splits, the weights broadcast from lane sp % 32
-#pragma unroll
-  for (int e = 0; e < CPL; ++e) o[e] = 0.f;
-  for (int c0 = 0; c0 < active; c0 += 32) {
-    const int ns = min(32, active - c0);
-    float fl = 0.f;
-    if (lane < ns) {
-      const float ms = __ldcg(recs + (int64_t)(c0 + lane) * RF + kHdr + r * (8 + D));
-      fl = ms == -INFINITY ? 0.f : exp2f(ms - M);
-    }
-#pragma unroll 4
-    for (int i = 0; i < ns; ++i) {
-      const float f = __shfl_sync(0xffffffffu, fl, i);
-      const float* op = recs + (int64_t)(c0 + i) * RF + kHdr + r * (8 + D) + 8 + lane * CPL;
-      if constexpr (CPL == 4) {
-        const float4 v4 = __ldcg(reinterpret_cast<const float4*>(op));
-        o[0] = fmaf(f, v4.x, o[0]);
-        o[1] = fmaf(f, v4.y, o[1]);
-        o[2] = fmaf(f, v4.z, o[2]);
-        o[3] = fmaf(f, v4.w, o[3]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) o[e] = fmaf(f, __ldcg(op + e), o[e]);
-      }
-    }
   }
   finalize(t5[0], t5[1], t5[2], t5[3], t5[4], rg, o);
   __syncthreads();
