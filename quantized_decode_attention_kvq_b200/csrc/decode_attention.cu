@@ -358,15 +358,19 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   const int zgrp = g8 < NB ? g8 : 0;
 
   // ---- page loop ---------------------------------------------------------------
-  int st = 0;
-  uint32_t par = 0;
-  for (int j = 0; j < nloc; ++j) {
-    bool ok = mbar_wait(&bar[st], par);
+  // One step per local page j, in ring stage j % S.  The stage is a template
+  // constant (the loop is unrolled by S), so every shared-memory address below is
+  // a fixed offset; FULL pages (all 16 tokens inside the context, every page but
+  // possibly a sequence's last) skip the per-token context masks.
+  auto page_step = [&](auto st_c, auto full_c, int j, uint32_t par) -> bool {
+    constexpr int st = decltype(st_c)::value;
+    constexpr bool FULL = decltype(full_c)::value;
+    constexpr int stn = st + 1 == S ? 0 : st + 1;
+    const bool ok = mbar_wait(&bar[st], par);
     if (!__all_sync(0xffffffffu, ok)) {
       if (lane == 0) set_error(a.err, KVQ_ERR_TIMEOUT);
-      break;
+      return false;
     }
-    const int stn = st + 1 == S ? 0 : st + 1;
     const int page = spage[st];
     const float eta_cur = eta_next;
     if (j + 1 < nloc) {
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     if (page >= 0) {
       const uint8_t* kt = ktile + st * C::KT;
       const uint8_t* rs = rest + st * C::REST;
-      const int nval = min(kPage, n - (first + j * kWarps) * kPage);
+      const int nval = FULL ? kPage : min(kPage, n - (first + j * kWarps) * kPage);
       etamax = fmaxf(etamax, eta_cur);
       const uint32_t* vm = reinterpret_cast<const uint32_t*>(rs + C::VB + C::KSB);
       const __half* ksc = reinterpret_cast<const __half*>(rs + C::VB);
@@ -591,8 +595,20 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     }
     __syncwarp();
     if (j + S < nloc) issue(j + S, st);
-    st = stn;
-    par ^= (stn == 0) ? 1u : 0u;
+    return true;
+  };
+  const int last_page = npages - 1;
+  uint32_t par = 0;
+  bool going = true;
+  for (int j0 = 0; j0 < nloc && going; j0 += S) {
+    static_for<0, S>([&](auto u_c) {
+      const int j = j0 + decltype(u_c)::value;
+      if (!going || j >= nloc) return;
+      const bool full = first + j * kWarps < last_page || n % kPage == 0;
+      going = full ? page_step(u_c, std::true_type{}, j, par)
+                   : page_step(u_c, std::false_type{}, j, par);
+    });
+    par ^= 1u;
   }
 
   // ---- warp reductions ----------------------------------------------------------
