@@ -171,13 +171,29 @@ def _dist_setup(n_gpus):
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """The maximum of a per-rank number over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def _rank_times(ms_total: float, dec_ms: float, e2e_ms: float, steps: int, world: int):
+    """Per-step, per-decode and end-to-end times of the job: the slowest rank's."""
+    ms_total = _max_over_ranks(ms_total, world)
+    dec_ms = _max_over_ranks(dec_ms, world)
+    e2e_ms = _max_over_ranks(e2e_ms, world)
+    return ms_total / max(1, steps), dec_ms, e2e_ms
+
+
+def _job_value(token_heads_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of all ranks (independent replicas, one per
+    rank) over the slowest rank's time per step."""
+    return token_heads_per_rank * world / (ms_per_step * 1e-3)
 
 
 def _barrier(world):
@@ -260,6 +276,39 @@ class GpuStep:
         self.cache_bytes = inp.num_pages * wl.num_kv_heads * bb
         self.replicas = replicas
         self.launches_per_step = 2
+        # finite tau: flagged rows are recomputed exactly from pinned host originals
+        self.fallback = None
+        if math.isfinite(wl.tau):
+            kh = (torch.from_numpy(k.view(np.int16)).view(torch.bfloat16) if k.dtype == np.uint16
+                  else torch.from_numpy(k)).pin_memory()
+            vh = (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
+                  else torch.from_numpy(v)).pin_memory()
+            fb_bytes = kvq.kvq_fallback_staging_size(base.desc, dt, max(inp.seq_lens)) * 8
+            self.fallback = dict(
+                kh=kh, vh=vh, dt=dt, qdt=qdt, T=T, side=torch.cuda.Stream(),
+                flags_h=torch.zeros(self.flags.numel(), dtype=torch.uint8).pin_memory(),
+                sl_h=np.array(inp.seq_lens, np.int32),
+                staging=torch.empty(fb_bytes, dtype=torch.uint8, device="cuda"), rows=0, calls=0,
+                h2d=0)
+
+    def fallback_exact(self, r=0):
+        """The exact fallback of the rows the last decode flagged (host-synchronous)."""
+        fb, wl, kvq = self.fallback, self.wl, self.kvq
+        B, NQ, HQ, d = self.out.shape
+        rc, n = kvq.kvq_fallback_exact(
+            self.caches[r].desc, fb["kh"], fb["vh"], fb["dt"], wl.num_kv_heads * fb["T"] * d,
+            fb["T"] * d, self.qd, fb["qdt"], B, NQ, HQ, fb["sl_h"].ctypes.data, 0.0, self.flags,
+            fb["flags_h"], self.out, fb["staging"], fb["staging"].numel(), self.stream,
+            fb["side"], 60000)
+        if rc:
+            raise RuntimeError(kvq.last_error())
+        fl = fb["flags_h"].numpy().reshape(B, NQ, HQ).any(axis=1)     # (seq, q head)
+        pairs = fl.reshape(B, wl.num_kv_heads, -1).any(axis=2)
+        es = 2 if fb["dt"] == kvq.KVQ_BF16 else 4
+        fb["h2d"] += int(2 * es * d * (pairs * fb["sl_h"][:, None]).sum())
+        fb["rows"] += n
+        fb["calls"] += 1
+        return n
 
     def step(self, i, ev=None):
         r = i % self.replicas
@@ -323,9 +372,6 @@ def run_gpu(args):
     _barrier(world)
     ms_total = t0.elapsed_time(t1)
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
-    ms_total = _max_over_ranks(ms_total, world)
-    dec_ms = _max_over_ranks(dec_ms, world)
-    ms_step = ms_total / args.steps
 
     # end to end through the public API with host buffers: H2D of the step's inputs
     # (q and the new K/V token) from pinned memory, the two calls, D2H of the results
@@ -337,7 +383,9 @@ def run_gpu(args):
     flags_h = torch.empty(st.flags.shape, dtype=torch.uint8).pin_memory()
     h2d = q_h.numel() * q_h.element_size() + 2 * kn_h.numel() * kn_h.element_size()
     d2h = out_h.numel() * 4 + bound_h.numel() * 4 + flags_h.numel()
-    e_steps = max(1, args.steps)
+    # with a finite tau the step ends with the host-synchronous exact fallback of the
+    # flagged rows, which pages in their originals: a few steps suffice
+    e_steps = max(1, args.steps) if st.fallback is None else max(1, min(args.steps, 5))
     _barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -349,19 +397,22 @@ def run_gpu(args):
             st.k_new.copy_(kn_h, non_blocking=True)
             st.v_new.copy_(vn_h, non_blocking=True)
             st.step(i)
+            if st.fallback is not None:
+                st.fallback_exact(i % st.replicas)
             out_h.copy_(st.out, non_blocking=True)
             bound_h.copy_(st.bound, non_blocking=True)
             flags_h.copy_(st.flags, non_blocking=True)
         e1.record(st.stream)
     torch.cuda.synchronize()
-    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / e_steps, world)
+    ms_step, dec_ms, e2e_ms = _rank_times(ms_total, dec_ms, e0.elapsed_time(e1) / e_steps,
+                                          args.steps, world)
 
     peak, peak_kind = _peaks()
     achieved = st.decode_bytes / (dec_ms * 1e-3) / 1e9
     traffic = _traffic_record()
     res = {
         "metric": METRIC,
-        "value": st.token_heads * world / (ms_step * 1e-3),
+        "value": _job_value(st.token_heads, world, ms_step),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -382,11 +433,21 @@ def run_gpu(args):
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "kernel": "decode_mma_kernel", "kernel_ms": dec_ms},
-        "e2e": {"value": st.token_heads * world / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": _job_value(st.token_heads, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": st.launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if st.fallback is not None:
+        fb = st.fallback
+        rows_per_step = fb["rows"] / max(1, fb["calls"])
+        res["fallback"] = {
+            "tau": wl.tau, "rate": rows_per_step / st.out.shape[0] / st.out.shape[1] /
+            st.out.shape[2], "rows_per_step": rows_per_step,
+            "h2d_bytes_per_step": fb["h2d"] / max(1, fb["calls"]),
+            "note": "value times append + decode (graph); e2e adds the exact fallback of the "
+                    "flagged rows (H2D of their originals + fp32 attention)"}
+        res["e2e"]["h2d_bytes_per_step"] = int(h2d + fb["h2d"] / max(1, fb["calls"]))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(args.workload, args.seed, args.cpu_seconds)
     if world > 1:
