@@ -107,8 +107,10 @@ KVQ_API size_t kvq_pool_bytes(const kvq_cache* cache);
  * physical page page_table[s*max_pages_per_seq + pos/16], slot pos%16, of
  * every kv head.  k, v (device, in_dtype) element (s, h, t, c) is at
  * s*seq_stride + h*head_stride + t*token_stride + c (strides in elements;
- * channels contiguous).  page_table, start_pos, valid_tokens: device int32.
- * eta of the touched blocks is raised with an atomic max, so eta of a reused
+ * channels contiguous); every element with t < num_tokens must be readable,
+ * also for tokens at or past valid_tokens[s] (they are loaded before the
+ * valid count is known, and ignored).  page_table, start_pos, valid_tokens:
+ * device int32.  eta of the touched blocks is raised with an atomic max, so eta of a reused
  * page must be zeroed by the caller first.  A non-finite input or an
  * fp16-overflowing scale writes zero codes and scale for that group and sets
  * *error_word = KVQ_ERR_RANGE; a page index outside [0, num_pages) skips the

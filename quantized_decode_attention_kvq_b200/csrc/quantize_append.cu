@@ -32,6 +32,16 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const AppendArgs a
   const int h = (int)(item % a.hkv);
   const int t = (int)((item / a.hkv) % a.num_tokens);
   const int s = (int)(item / ((int64_t)a.hkv * a.num_tokens));
+  // The token's k and v (always inside the caller's [num_seqs][num_tokens]
+  // input) are loaded first: they do not depend on where the token goes, so
+  // their latency overlaps the position -> page-table lookups below.
+  const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
+  float xk[E], xv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    xk[e] = load_elem(a.k, a.in_bf16, base + lane * E + e);
+    xv[e] = load_elem(a.v, a.in_bf16, base + lane * E + e);
+  }
   if (a.valid && t >= a.valid[s]) return;
   const int pos = a.start_pos[s] + t;
   const int lp = pos / kPage;
@@ -46,14 +56,6 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const AppendArgs a
   }
   const int slot = pos % kPage;
   uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
-  const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
-
-  float xk[E], xv[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    xk[e] = load_elem(a.k, a.in_bf16, base + lane * E + e);
-    xv[e] = load_elem(a.v, a.in_bf16, base + lane * E + e);
-  }
   if (a.signs) warp_rotate<E>(xk, a.signs, lane, a.rot_c);
 
   // ---------------- keys: symmetric, per token and KG channels --------------
