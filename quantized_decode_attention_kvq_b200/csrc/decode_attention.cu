@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       for (int sl = 0; sl < 2; ++sl) {
         const int tok = g8 + 8 * sl;
         const bool vt = tok < nval;
-        float dot = 0.f, dsum = 0.f, smax = 0.f;
+        float dot = 0.f, dsum = 0.f;
         float sg[NGK];
         if constexpr (NGK == 4) {
           const float4 f4 = *reinterpret_cast<const float4*>(ks32 + tok * 4);
@@ -485,8 +485,10 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
           const float raw = fmaf((float)hi, 65536.f, (float)lo);
           dot = fmaf(raw, sg[g], dot);
           dsum = fmaf(cg[g], sg[g], dsum);
-          smax = fmaxf(smax, sg[g]);
         }
+        float smax = sg[0];   // scales are >= 0
+#pragma unroll
+        for (int g = 1; g < NGK; ++g) smax = fmaxf(smax, sg[g]);
         zt[sl] = vt ? dot * zs : -INFINITY;
         dl[sl] = vt ? fmaf(cb, smax, dsum) : 0.f;
       }
@@ -500,22 +502,21 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       // 2 (log2 units): weights stay <= 4, so w * sV fits fp16 for any finite
       // value scale, and the accumulators are rescaled on few pages.
       const float mref = mx > m2 + 2.0f ? mx : m2;
-      const float alpha = exp2f(m2 - mref);
+      const float alpha = ex2(m2 - mref);
       m2 = mref;
-      const float w0 = exp2f(zt[0] - mref), w1 = exp2f(zt[1] - mref);
+      const float w0 = ex2(zt[0] - mref), w1 = ex2(zt[1] - mref);
       // tokens outside the context have w = 0 and Delta = 0
       const float2 d2 = make_float2(dl[0], dl[1]);
       const float2 e2 = mul2(d2, make_float2(kLog2e, kLog2e));
-      const float2 ep = make_float2(exp2f(e2.x), exp2f(e2.y));
-      const float2 en = make_float2(exp2f(-e2.x), exp2f(-e2.y));
-      // e^d - 1: Taylor to d^5 below 1/16 (no cancellation), else from e^d
-      float2 pl = fma2(d2, make_float2(1.0f / 120, 1.0f / 120), make_float2(1.0f / 24, 1.0f / 24));
-      pl = fma2(d2, pl, make_float2(1.0f / 6, 1.0f / 6));
-      pl = fma2(d2, pl, make_float2(0.5f, 0.5f));
+      const float2 ep = make_float2(ex2(e2.x), ex2(e2.y));
+      const float2 en = make_float2(ex2(-e2.x), ex2(-e2.y));
+      // e^d - 1: below 2^-6 the Taylor series to d^3 (truncation < 2e-7 relative);
+      // above it e^d - 1 directly (relative error < 2^-22 * e^d / (e^d - 1) < 2e-5)
+      float2 pl = fma2(d2, make_float2(1.0f / 6, 1.0f / 6), make_float2(0.5f, 0.5f));
       pl = fma2(d2, pl, make_float2(1.0f, 1.0f));
       pl = mul2(d2, pl);
-      const float em0 = d2.x < 0.0625f ? pl.x : ep.x - 1.0f;
-      const float em1 = d2.y < 0.0625f ? pl.y : ep.y - 1.0f;
+      const float em0 = d2.x < 0.015625f ? pl.x : ep.x - 1.0f;
+      const float em1 = d2.y < 0.015625f ? pl.y : ep.y - 1.0f;
       const float ta = fmaf(w1, em1, w0 * em0);
       const float tb = fmaf(w1, en.y, w0 * en.x);
       dmax = fmaxf(dmax, fmaxf(d2.x, d2.y));
@@ -555,7 +556,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
         for (int k = 0; k < 4; ++k) {
           const int tok = c4 + 4 * k;
           const uint32_t wv = vm[tok * NB + zgrp];
-          zw[k] = (g8 < NB && tok < nval) ? wv : 0u;
+          // rows g8 >= NB of this MMA are padding (never read): no mask on FULL pages
+          zw[k] = FULL || (g8 < NB && tok < nval) ? wv : 0u;
         }
         const uint32_t bz0 = hilo2(make_float2(x[0], x[1]));
         const uint32_t bz1 = hilo2(make_float2(x[2], x[3]));
@@ -696,7 +698,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   for (int w = 0; w < kWarps; ++w) {
     const float* mwp = wa + w * C::MW_FLOATS;
     const float* stw = mwp + kRows * D + r * 8;
-    const float f = stw[0] == -INFINITY ? 0.f : exp2f(stw[0] - mW);
+    const float f = stw[0] == -INFINITY ? 0.f : ex2(stw[0] - mW);
 #pragma unroll
     for (int t = 0; t < 4; ++t) st5[t] = fmaf(f, stw[1 + t], st5[t]);
     st5[4] = fmaxf(st5[4], stw[5]);
@@ -838,7 +840,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
     const float Mn = fmaxf(Mr, Mc);
-    const float sc = Mr == -INFINITY ? 0.f : exp2f(Mr - Mn);
+    const float sc = Mr == -INFINITY ? 0.f : ex2(Mr - Mn);
     Mr = Mn;
 #pragma unroll
     for (int t = 0; t < 4; ++t) t5[t] *= sc;
@@ -847,7 +849,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     float f[KS], p5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < KS; ++k) {
-      f[k] = sa[k].x == -INFINITY ? 0.f : exp2f(sa[k].x - Mn);
+      f[k] = sa[k].x == -INFINITY ? 0.f : ex2(sa[k].x - Mn);
       p5[0] = fmaf(f[k], sa[k].y, p5[0]);
       p5[1] = fmaf(f[k], sa[k].z, p5[1]);
       p5[2] = fmaf(f[k], sa[k].w, p5[2]);

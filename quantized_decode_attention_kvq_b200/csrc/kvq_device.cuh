@@ -108,6 +108,15 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ---- 2^x by the hardware approximation (PTX ex2.approx.ftz.f32) -------------
+// Relative error about 2^-22; results below the normal range flush to +0 and
+// 2^-inf = +0.  Softmax weights and the bound's exponentials need no more.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---- compile-time loop: f(std::integral_constant<int, I>) for I in [B, E) -----
 template <int B, int E, class F>
 __device__ __forceinline__ void static_for(F&& f) {
