@@ -36,7 +36,9 @@
  *   [K codes 16*head_dim*k_bits/8 B][V codes 16*head_dim/2 B]
  *   [K scales fp16 [16][head_dim/k_group]][V (scale, zero) fp16 [16][nb][2]]
  *   K code of channel c (b = c/32, w = c%32, s = w/8, i = w%8) in a token row:
- *     8 bit: byte s*8*nb + 8*b + i (int8);
+ *     8 bit: byte s*8*nb + 8*b + i (int8); for head_dim 128 (128-byte rows)
+ *            that byte's 16-byte chunk index is XORed with slot % 8, slot =
+ *            the token's row in the page;
  *     4 bit: byte s*4*nb + 4*b + i/2, low nibble for even c (4-bit two's complement).
  *   V code of channel c (g = c/32, w = c%32): byte (w/4)*2*nb + 2*g + (w%4)/2,
  *     low nibble for even c (unsigned).

@@ -7,10 +7,10 @@
 // norms and the value range only).
 //
 // Grid (split, kv head, sequence); 4 warps per CTA.  Each warp streams its
-// own pages of the split through an S-stage ring in shared memory: one TMA
-// tiled load brings the page's K codes (128B-swizzled when rows are 128 B),
-// one bulk copy brings V codes + K scales + V scale/zero; completion on an
-// mbarrier per stage, every wait bounded.
+// own pages of the split through an S-stage ring in shared memory: one bulk
+// copy (cp.async.bulk) brings the page's whole block -- K codes (stored with
+// their 16-byte chunks pre-permuted for conflict-free reads), V codes, K
+// scales, V scale/zero; completion on an mbarrier per stage, every wait bounded.
 //
 // Per page (16 tokens x up to 4 query rows of one GQA group):
 //   QK^T  int8 tensor cores, exact: q' (rotated if the cache is) is held in
@@ -59,12 +59,11 @@ struct DecodeCfg {
   static constexpr bool SWZ = KRB == 128;
   static constexpr int KSTR = KRB / 4;            // K stripe bytes per lane
   static constexpr int VSTR = VRB / 8;            // V stripe bytes per lane
-  // shared memory carve-up (offsets from a 1024-aligned base)
-  static constexpr int OFF_KT = 0;
-  static constexpr int SZ_KT = kWarps * S * KT;
-  static constexpr int OFF_RS = OFF_KT + SZ_KT;
-  static constexpr int SZ_RS = kWarps * S * REST;
-  static constexpr int OFF_BAR = (OFF_RS + SZ_RS + 15) / 16 * 16;
+  // shared memory carve-up (offsets from a 128-aligned base): per warp S stages
+  // of one whole block each (K codes, then V codes and metadata)
+  static constexpr int OFF_ST = 0;
+  static constexpr int SZ_ST = kWarps * S * BLOCK;
+  static constexpr int OFF_BAR = (OFF_ST + SZ_ST + 15) / 16 * 16;
   static constexpr int OFF_PG = OFF_BAR + kWarps * S * 8;
   static constexpr int OFF_Q = (OFF_PG + kWarps * S * 4 + 15) / 16 * 16;   // int8 qdig[4][4][D]
   static constexpr int OFF_QB = OFF_Q + kRows * 4 * D;                      // int qsum[4][NGK][4]
@@ -78,7 +77,7 @@ struct DecodeCfg {
   // merge area (aliases the stage buffers once the page loop is over)
   static constexpr int MW_FLOATS = kRows * D + kRows * 8 + kRows * NB + 2 * NB + 1;
   static constexpr int MERGE_BYTES = (kWarps + 1) * MW_FLOATS * 4;
-  static constexpr int SMEM = 1024 + (END > MERGE_BYTES ? END : MERGE_BYTES);
+  static constexpr int SMEM = 128 + (END > MERGE_BYTES ? END : MERGE_BYTES);
   static_assert(MERGE_BYTES <= OFF_BAR, "merge area must fit in the stage buffers");
 };
 
@@ -88,21 +87,18 @@ constexpr int min_ctas() { return (KB == 4 && KG == 32) ? 3 : 4; }
 
 template <int D, int KB, int KG, int S>
 __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
-    decode_mma_kernel(const __grid_constant__ DecodeArgs a,
-                      const __grid_constant__ CUtensorMap kmap) {
+    decode_mma_kernel(const __grid_constant__ DecodeArgs a) {
   using C = DecodeCfg<D, KB, KG, S>;
   constexpr int NB = C::NB, NGK = C::NGK;
   constexpr int Q = KB == 8 ? 127 : 7;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base (swizzled TMA tiles); pointer arithmetic on the
-  // __shared__ array keeps every access below in the shared address space
-  uint8_t* sm = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  // 128-byte aligned base; pointer arithmetic on the __shared__ array keeps
+  // every access below in the shared address space
+  uint8_t* sm = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c4 = lane & 3, g8 = lane >> 2;
-  // The key-tile descriptor and this warp's ring barriers need nothing from
-  // memory: start them first, so their latency overlaps the loads below.
-  if (tid == 0) prefetch_tensormap(&kmap);
+  // This warp's ring barriers need nothing from memory: set them up first.
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + warp * S;
   if (lane == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
@@ -152,8 +148,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   }
   const int p1 = min(p0 + a.pps, npages);
 
-  uint8_t* ktile = sm + C::OFF_KT + warp * S * C::KT;
-  uint8_t* rest = sm + C::OFF_RS + warp * S * C::REST;
+  uint8_t* stage0 = sm + C::OFF_ST + warp * S * C::BLOCK;
   int* spage = reinterpret_cast<int*>(sm + C::OFF_PG) + warp * S;
   int8_t* qdig = reinterpret_cast<int8_t*>(sm + C::OFF_Q);
   int* qsum = reinterpret_cast<int*>(sm + C::OFF_QB);
@@ -183,8 +178,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       if (ok) {
         const int64_t blk = (int64_t)page * a.hkv + kvh;
         mbar_arrive_expect_tx(&bar[st], C::BLOCK);
-        tma_load_3d(ktile + st * C::KT, &kmap, 0, 0, (int)blk, &bar[st]);
-        bulk_g2s(rest + st * C::REST, a.pool + blk * C::BLOCK + C::KT, C::REST, &bar[st]);
+        bulk_g2s(stage0 + st * C::BLOCK, a.pool + blk * C::BLOCK, C::BLOCK, &bar[st]);
       } else {
         set_error(a.err, KVQ_ERR_INVALID_ARG);
         mbar_arrive(&bar[st]);
@@ -378,8 +372,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       eta_next = pn >= 0 ? __ldg(eta_kv + (int64_t)pn * a.hkv) : 0.f;
     }
     if (page >= 0) {
-      const uint8_t* kt = ktile + st * C::KT;
-      const uint8_t* rs = rest + st * C::REST;
+      const uint8_t* kt = stage0 + st * C::BLOCK;
+      const uint8_t* rs = kt + C::KT;
       const int nval = FULL ? kPage : min(kPage, n - (first + j * kWarps) * kPage);
       etamax = fmaxf(etamax, eta_cur);
       const uint32_t* vm = reinterpret_cast<const uint32_t*>(rs + C::VB + C::KSB);

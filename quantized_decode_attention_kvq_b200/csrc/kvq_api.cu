@@ -3,7 +3,6 @@
 // descriptor encoding, and the host orchestration of the exact fallback
 // (flag read-back with a bounded wait, Tier-2 page-in with cudaMemcpyAsync on
 // a side stream, recomputation kernel, stream hand-back).
-#include <cudaTypedefs.h>
 
 #include <chrono>
 #include <cstdarg>
@@ -164,45 +163,6 @@ int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
   return KVQ_OK;
 }
 
-// TMA descriptor of the K-code tiles: 3-D {row bytes, 16 rows, page x kv head}.
-int key_tensor_map(const kvq_cache* c, CUtensorMap* out) {
-  static std::mutex mu;
-  static std::map<std::tuple<void*, int, int, int, int, int>, CUtensorMap> cache;
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  const BlockLayout L = layout_of(c);
-  std::lock_guard<std::mutex> lk(mu);
-  auto key = std::make_tuple(c->pool, c->num_pages, c->num_kv_heads, c->head_dim, c->k_bits,
-                             c->k_group);
-  auto it = cache.find(key);
-  if (it != cache.end()) {
-    *out = it->second;
-    return KVQ_OK;
-  }
-  if (!encode) {
-    cudaDriverEntryPointQueryResult q;
-    void* fn = nullptr;
-    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
-      return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
-  CUtensorMap m;
-  const int row = L.k_row();
-  cuuint64_t dims[3] = {(cuuint64_t)row, (cuuint64_t)kPage,
-                        (cuuint64_t)c->num_pages * (cuuint64_t)c->num_kv_heads};
-  cuuint64_t strides[2] = {(cuuint64_t)row, (cuuint64_t)L.bytes()};
-  cuuint32_t box[3] = {(cuuint32_t)row, (cuuint32_t)kPage, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, c->pool, dims, strides, box, estr,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE,
-                      row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-  cache.emplace(key, m);
-  *out = m;
-  return KVQ_OK;
-}
-
 int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
                 int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
                 int32_t max_pages, const int32_t* seq_lens, float softmax_scale, float tau,
@@ -232,8 +192,6 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
                 plan.total());
   if (!aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");
   DecodeVariant v = select_decode_kernel(cache->head_dim, cache->k_bits, cache->k_group);
-  CUtensorMap kmap;
-  if ((rc = key_tensor_map(cache, &kmap))) return rc;
   DecodeArgs a;
   a.pool = static_cast<const uint8_t*>(cache->pool);
   a.eta = cache->v_eta;
@@ -263,7 +221,7 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
   dim3 grid(plan.splits, cache->num_kv_heads, num_seqs);
   if (grid.y > 65535 || grid.z > 65535)
     return fail(KVQ_ERR_UNSUPPORTED, "grid too large (kv heads %d, sequences %d)", grid.y, grid.z);
-  v.kernel<<<grid, decode_threads(), v.smem, stream>>>(a, kmap);
+  v.kernel<<<grid, decode_threads(), v.smem, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   return KVQ_OK;

@@ -42,7 +42,7 @@ struct DecodeArgs {
   int* counters;
 };
 
-using DecodeKernel = void (*)(const DecodeArgs, const CUtensorMap);
+using DecodeKernel = void (*)(const DecodeArgs);
 struct DecodeVariant {
   DecodeKernel kernel;
   int smem;    // dynamic shared memory bytes

@@ -95,7 +95,10 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const AppendArgs a
       const int c = lane * E + e;            // even channel of the pair
       const int b = c / 32, w = c % 32;
       if (KB == 8) {
-        const int byte = (w / 8) * (8 * NB) + 8 * b + (w % 8);
+        int byte = (w / 8) * (8 * NB) + 8 * b + (w % 8);
+        // 128-byte rows: 16-byte chunk index XOR slot % 8 (bank-conflict-free
+        // reads of the page's 16 rows without any swizzle on the copy)
+        if (D == 128) byte = (((byte >> 4) ^ (slot & 7)) << 4) | (byte & 15);
         row[byte] = (uint8_t)(int8_t)code[e];
         row[byte + 1] = (uint8_t)(int8_t)code[e + 1];
       } else {
