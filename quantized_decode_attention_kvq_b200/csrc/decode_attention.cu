@@ -83,7 +83,7 @@ struct DecodeCfg {
 
 // resident CTAs per SM the register budget is sized for (4 = 128 registers)
 template <int D, int KB, int KG>
-constexpr int min_ctas() { return (KB == 4 && KG == 32) ? 3 : 4; }
+constexpr int min_ctas() { return 4; }
 
 template <int D, int KB, int KG, int S>
 __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
@@ -276,15 +276,16 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
         qb[ks][nt][1] = w2.y;
       }
   }
-  // initial accumulators: 4-bit key codes enter as code + 8
-  int cinit[NGK][2][2];
+  // 4-bit key codes enter as code + 8: per key group, the bias -8 * (sum of each
+  // digit of row c4 over the group), recombined like the accumulators
+  // (digits 0 + 256 * 1 -> blo, digits 2 + 256 * 3 -> bhi)
+  int blo[NGK], bhi[NGK];
 #pragma unroll
-  for (int g = 0; g < NGK; ++g)
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int dd = 0; dd < 2; ++dd)
-        cinit[g][nt][dd] = KB == 4 ? -8 * qsum[(c4 * NGK + g) * 4 + 2 * nt + dd] : 0;
+  for (int g = 0; g < NGK; ++g) {
+    const int* qs = qsum + (c4 * NGK + g) * 4;
+    blo[g] = KB == 4 ? -8 * (qs[0] + 256 * qs[1]) : 0;
+    bhi[g] = KB == 4 ? -8 * (qs[2] + 256 * qs[3]) : 0;
+  }
   const float zs = rc[c4];
   const float cb = rc[kRows + c4];
   float cg[NGK];
@@ -422,69 +423,67 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
           wk[rr][1] = v2.y;
         }
       }
-      int acc[NGK][2][4];
-#pragma unroll
-      for (int g = 0; g < NGK; ++g)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          acc[g][nt][0] = cinit[g][nt][0];
-          acc[g][nt][1] = cinit[g][nt][1];
-          acc[g][nt][2] = cinit[g][nt][0];
-          acc[g][nt][3] = cinit[g][nt][1];
-        }
-#pragma unroll
-      for (int ks = 0; ks < NB; ++ks) {
-        const int g = (32 * ks) / KG;
-        uint32_t a0, a1, a2, a3;
-        if (KB == 8) {
-          a0 = wk[0][2 * ks];
-          a1 = wk[1][2 * ks];
-          a2 = wk[0][2 * ks + 1];
-          a3 = wk[1][2 * ks + 1];
-        } else {
-          const uint32_t x0 = wk[0][ks], x1 = wk[1][ks];
-          a0 = (x0 & 0x0F0F0F0Fu) ^ 0x08080808u;
-          a2 = ((x0 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-          a1 = (x1 & 0x0F0F0F0Fu) ^ 0x08080808u;
-          a3 = ((x1 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) mma_s8(acc[g][nt], a0, a1, a2, a3, qb[ks][nt][0], qb[ks][nt][1]);
-      }
       __syncwarp();  // the fp32 metadata table is complete
 
       // --- scores (log2 units) and Delta for tokens g8, g8+8 of row c4 -------------
-      float zt[2], dl[2];
+      // Each key group's int32 accumulators are folded into the fp32 score as
+      // soon as its k-steps are done, so one group's accumulators are live at a time.
+      float sg[2][NGK];
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
         const int tok = g8 + 8 * sl;
-        const bool vt = tok < nval;
-        float dot = 0.f, dsum = 0.f;
-        float sg[NGK];
         if constexpr (NGK == 4) {
           const float4 f4 = *reinterpret_cast<const float4*>(ks32 + tok * 4);
-          sg[0] = f4.x;
-          sg[1] = f4.y;
-          sg[2] = f4.z;
-          sg[3] = f4.w;
+          sg[sl][0] = f4.x;
+          sg[sl][1] = f4.y;
+          sg[sl][2] = f4.z;
+          sg[sl][3] = f4.w;
         } else {
 #pragma unroll
-          for (int g = 0; g < NGK; ++g) sg[g] = ks32[tok * NGK + g];
+          for (int g = 0; g < NGK; ++g) sg[sl][g] = ks32[tok * NGK + g];
+        }
+      }
+      float dot[2] = {0.f, 0.f}, dsum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int g = 0; g < NGK; ++g) {
+        int acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+#pragma unroll
+        for (int ks = g * (KG / 32); ks < (g + 1) * (KG / 32); ++ks) {
+          uint32_t a0, a1, a2, a3;
+          if (KB == 8) {
+            a0 = wk[0][2 * ks];
+            a1 = wk[1][2 * ks];
+            a2 = wk[0][2 * ks + 1];
+            a3 = wk[1][2 * ks + 1];
+          } else {
+            const uint32_t x0 = wk[0][ks], x1 = wk[1][ks];
+            a0 = (x0 & 0x0F0F0F0Fu) ^ 0x08080808u;
+            a2 = ((x0 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+            a1 = (x1 & 0x0F0F0F0Fu) ^ 0x08080808u;
+            a3 = ((x1 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+          }
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) mma_s8(acc[nt], a0, a1, a2, a3, qb[ks][nt][0], qb[ks][nt][1]);
         }
 #pragma unroll
-        for (int g = 0; g < NGK; ++g) {
+        for (int sl = 0; sl < 2; ++sl) {
           // digits 0,1 and 2,3 recombined exactly in int32, then once in fp32
-          const int lo = acc[g][0][2 * sl] + (acc[g][0][2 * sl + 1] << 8);
-          const int hi = acc[g][1][2 * sl] + (acc[g][1][2 * sl + 1] << 8);
+          const int lo = acc[0][2 * sl] + acc[0][2 * sl + 1] * 256 + blo[g];
+          const int hi = acc[1][2 * sl] + acc[1][2 * sl + 1] * 256 + bhi[g];
           const float raw = fmaf((float)hi, 65536.f, (float)lo);
-          dot = fmaf(raw, sg[g], dot);
-          dsum = fmaf(cg[g], sg[g], dsum);
+          dot[sl] = fmaf(raw, sg[sl][g], dot[sl]);
+          dsum[sl] = fmaf(cg[g], sg[sl][g], dsum[sl]);
         }
-        float smax = sg[0];   // scales are >= 0
+      }
+      float zt[2], dl[2];
 #pragma unroll
-        for (int g = 1; g < NGK; ++g) smax = fmaxf(smax, sg[g]);
-        zt[sl] = vt ? dot * zs : -INFINITY;
-        dl[sl] = vt ? fmaf(cb, smax, dsum) : 0.f;
+      for (int sl = 0; sl < 2; ++sl) {
+        const bool vt = g8 + 8 * sl < nval;
+        float smax = sg[sl][0];   // scales are >= 0
+#pragma unroll
+        for (int g = 1; g < NGK; ++g) smax = fmaxf(smax, sg[sl][g]);
+        zt[sl] = vt ? dot[sl] * zs : -INFINITY;
+        dl[sl] = vt ? fmaf(cb, smax, dsum[sl]) : 0.f;
       }
 
       // --- online softmax and bound sums (row c4) -------------------------------
