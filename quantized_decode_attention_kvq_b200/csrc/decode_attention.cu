@@ -89,6 +89,7 @@ template <int D, int KB, int KG, int S>
 __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     decode_mma_kernel(const __grid_constant__ DecodeArgs a) {
   using C = DecodeCfg<D, KB, KG, S>;
+  static_assert(S < 32, "the issue side must stay within one 32-page chunk of the loop");
   constexpr int NB = C::NB, NGK = C::NGK;
   constexpr int Q = KB == 8 ? 127 : 7;
   extern __shared__ uint8_t smem_raw[];
@@ -162,6 +163,12 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     return j < nloc ? __ldg(ptab + first + j * kWarps) : -1;
   };
   int pt_chunk = -1, pt_val = -1, pt_next = lane < nloc ? pt_first : -1;
+  // eta of the pages: lane l holds eta of local page 32c + l of the chunk c being
+  // issued (eta_iss) and of the chunk being processed (eta_proc).  Each is loaded
+  // when the issue side enters its chunk, S pages before the first of them is
+  // processed, and read by a shuffle -- no per-page load on the loop's path.
+  const float* eta_kv = a.eta + kvh;
+  float eta_iss = 0.f, eta_proc = 0.f;
   __syncwarp();
 
   auto issue = [&](int j, int st) {  // whole warp; lane 0 issues local page j into stage st
@@ -170,6 +177,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       pt_val = (c == pt_chunk + 1) ? pt_next : fetch_chunk(c);
       pt_next = fetch_chunk(c + 1);
       pt_chunk = c;
+      eta_iss = (unsigned)pt_val < (unsigned)a.num_pages ? __ldg(eta_kv + (int64_t)pt_val * a.hkv)
+                                                        : 0.f;
     }
     const int page = __shfl_sync(0xffffffffu, pt_val, j & 31);
     if (lane == 0) {
@@ -328,13 +337,6 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     return h2_as_u32(__floats2half2_rn(r.x, r.y));
   };
 
-  const float* eta_kv = a.eta + kvh;
-  float eta_next = 0.f;
-  if (nloc > 0) {
-    __syncwarp();
-    const int pg = spage[0];
-    eta_next = pg >= 0 ? __ldg(eta_kv + (int64_t)pg * a.hkv) : 0.f;
-  }
   // this lane's fixed offsets inside a stage
   constexpr int KW = C::KSTR / 4;                        // 32-bit words per key stripe
   constexpr int KCH = C::KSTR >= 16 ? C::KSTR / 16 : 1;  // 16-byte chunks per key stripe
@@ -360,18 +362,14 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   auto page_step = [&](auto st_c, auto full_c, int j, uint32_t par) -> bool {
     constexpr int st = decltype(st_c)::value;
     constexpr bool FULL = decltype(full_c)::value;
-    constexpr int stn = st + 1 == S ? 0 : st + 1;
     const bool ok = mbar_wait(&bar[st], par);
     if (!__all_sync(0xffffffffu, ok)) {
       if (lane == 0) set_error(a.err, KVQ_ERR_TIMEOUT);
       return false;
     }
     const int page = spage[st];
-    const float eta_cur = eta_next;
-    if (j + 1 < nloc) {
-      const int pn = spage[stn];
-      eta_next = pn >= 0 ? __ldg(eta_kv + (int64_t)pn * a.hkv) : 0.f;
-    }
+    if ((j & 31) == 0) eta_proc = eta_iss;   // the issue side is S < 32 pages ahead
+    const float eta_cur = __shfl_sync(0xffffffffu, eta_proc, j & 31);
     if (page >= 0) {
       const uint8_t* kt = stage0 + st * C::BLOCK;
       const uint8_t* rs = kt + C::KT;
