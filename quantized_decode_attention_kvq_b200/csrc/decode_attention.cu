@@ -85,6 +85,18 @@ struct DecodeCfg {
 template <int D, int KB, int KG>
 constexpr int min_ctas() { return 4; }
 
+// First page of split s when npages pages are shared by n splits in decreasing
+// sizes (split i weighs 10(n-1) - i, so the first is 10/9 of the last): the
+// grid puts the split index in its slow dimension, later splits are launched
+// later, and with fewer pages the splits of a (sequence, kv head) end together.
+__device__ __forceinline__ int split_start(int s, int n, int npages) {
+  if (n <= 1) return s <= 0 ? 0 : npages;
+  const int64_t k = 10LL * (n - 1);
+  const int64_t w = s * k - (int64_t)s * (s - 1) / 2;
+  const int64_t wn = n * k - (int64_t)n * (n - 1) / 2;
+  return (int)((int64_t)npages * w / wn);
+}
+
 template <int D, int KB, int KG, int S>
 __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     decode_mma_kernel(const __grid_constant__ DecodeArgs a) {
@@ -96,7 +108,9 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   // 128-byte aligned base; pointer arithmetic on the __shared__ array keeps
   // every access below in the shared address space
   uint8_t* sm = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  // grid (unit, split): the unit = (sequence, kv head) index runs fastest, so
+  // every unit's first split is launched before any unit's second one
+  const int split = blockIdx.y, kvh = blockIdx.x % a.hkv, b = blockIdx.x / a.hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c4 = lane & 3, g8 = lane >> 2;
   // This warp's ring barriers need nothing from memory: set them up first.
@@ -107,13 +121,15 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   }
 
   // The context length, the query rows and this warp's first 32 page indices
-  // are loaded together: none of these addresses depends on the others.
-  const int p0 = split * a.pps;
-  const int first = p0 + warp;
+  // are loaded together: none of these addresses depends on the others (the
+  // page indices assume a full-length context and are reloaded otherwise).
+  const int nsp = gridDim.y;
+  const int p0_spec = split_start(split, nsp, a.max_pages);
+  const int p1_spec = split_start(split + 1, nsp, a.max_pages);
   const int32_t* ptab = a.page_table + (int64_t)b * a.max_pages;
   int n = a.seq_lens[b];
-  const int pt_first = first + lane * kWarps < min(p0 + a.pps, a.max_pages)
-                           ? __ldg(ptab + first + lane * kWarps) : -1;
+  int pt_first = p0_spec + warp + lane * kWarps < p1_spec
+                     ? __ldg(ptab + p0_spec + warp + lane * kWarps) : -1;
   constexpr int QPT = kRows * D / (kWarps * 32);   // query elements per thread
   float qreg[QPT];
 #pragma unroll
@@ -147,7 +163,11 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     }
     return;
   }
-  const int p1 = min(p0 + a.pps, npages);
+  const int p0 = split_start(split, active, npages);
+  const int p1 = split_start(split + 1, active, npages);
+  const int first = p0 + warp;
+  if (p0 != p0_spec || p1 != p1_spec)
+    pt_first = first + lane * kWarps < p1 ? __ldg(ptab + first + lane * kWarps) : -1;
 
   uint8_t* stage0 = sm + C::OFF_ST + warp * S * C::BLOCK;
   int* spage = reinterpret_cast<int*>(sm + C::OFF_PG) + warp * S;
@@ -748,7 +768,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 
   // ---- write this split's record; the last CTA of (b, kvh) merges all --------------
   const int64_t unit = (int64_t)b * a.hkv + kvh;
-  const int splits = gridDim.x;
+  const int splits = gridDim.y;
   float* rec = a.part + (unit * splits + split) * RF;
   if (r == 0 && lane == 0) {
 #pragma unroll

@@ -218,9 +218,12 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
   a.flags = flags;
   a.counters = static_cast<int*>(ws);
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.counter_bytes);
-  dim3 grid(plan.splits, cache->num_kv_heads, num_seqs);
-  if (grid.y > 65535 || grid.z > 65535)
-    return fail(KVQ_ERR_UNSUPPORTED, "grid too large (kv heads %d, sequences %d)", grid.y, grid.z);
+  // (sequence x kv head, split): the split index in the slow dimension
+  const int64_t units = (int64_t)num_seqs * cache->num_kv_heads;
+  if (units > 0x7fffffffLL || plan.splits > 65535)
+    return fail(KVQ_ERR_UNSUPPORTED, "grid too large (%lld units, %d splits)", (long long)units,
+                plan.splits);
+  dim3 grid((unsigned)units, (unsigned)plan.splits, 1);
   v.kernel<<<grid, decode_threads(), v.smem, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
