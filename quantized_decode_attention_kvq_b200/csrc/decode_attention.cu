@@ -89,12 +89,16 @@ constexpr int min_ctas() { return 4; }
 // sizes (split i weighs 10(n-1) - i, so the first is 10/9 of the last): the
 // grid puts the split index in its slow dimension, later splits are launched
 // later, and with fewer pages the splits of a (sequence, kv head) end together.
+// (fp32 arithmetic: no 64-bit division on the kernel's start path; every CTA
+// evaluates the same expression, so neighbouring splits agree on their border,
+// and the result is monotone in s with split_start(0) = 0, split_start(n) = npages)
 __device__ __forceinline__ int split_start(int s, int n, int npages) {
-  if (n <= 1) return s <= 0 ? 0 : npages;
-  const int64_t k = 10LL * (n - 1);
-  const int64_t w = s * k - (int64_t)s * (s - 1) / 2;
-  const int64_t wn = n * k - (int64_t)n * (n - 1) / 2;
-  return (int)((int64_t)npages * w / wn);
+  if (s <= 0) return 0;
+  if (s >= n) return npages;
+  const float k = 10.0f * (float)(n - 1);
+  const float w = (float)s * k - 0.5f * (float)s * (float)(s - 1);
+  const float wn = (float)n * k - 0.5f * (float)n * (float)(n - 1);
+  return min(npages, (int)__fmul_rn((float)npages, __fdiv_rn(w, wn)));
 }
 
 template <int D, int KB, int KG, int S>
