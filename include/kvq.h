@@ -19,8 +19,9 @@
  *
  * Conventions
  *   - Every pointer is caller-owned; the library never allocates or frees
- *     memory and keeps no state between calls except a cache of TMA
- *     descriptors and of device properties.  "device" = CUDA device memory
+ *     memory on the decode path and keeps no state between calls except a
+ *     cache of device properties (and the static scratch of
+ *     kvq_decode_attention_noalloc).  "device" = CUDA device memory
  *     (or managed), "host" = host memory, "pinned" = page-locked host memory.
  *   - Every call validates its arguments before launching anything and
  *     returns a kvq_status (0 = KVQ_OK); no exception crosses the ABI.

@@ -1,6 +1,6 @@
 // kvq_api.cu -- the C ABI (include/kvq.h): argument validation, status codes,
-// launch planning (split-K sizing against the SM count and occupancy), TMA
-// descriptor encoding, and the host orchestration of the exact fallback
+// launch planning (split-K sizing against the SM count and occupancy), and the
+// host orchestration of the exact fallback
 // (flag read-back with a bounded wait, Tier-2 page-in with cudaMemcpyAsync on
 // a side stream, recomputation kernel, stream hand-back).
 

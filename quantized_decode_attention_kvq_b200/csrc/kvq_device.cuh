@@ -1,7 +1,7 @@
 // kvq_device.cuh -- device-side building blocks shared by the kvq kernels:
-// layout constants, mbarrier / bulk-copy / TMA wrappers with bounded waits,
-// legacy-warp MMA wrappers, the warp Walsh-Hadamard rotation and the
-// device error word.
+// layout constants, mbarrier / bulk-copy wrappers with bounded waits, warp
+// MMA wrappers, packed fp32x2 arithmetic, the hardware 2^x, the warp
+// Walsh-Hadamard rotation and the device error word.
 #pragma once
 
 #include <type_traits>
