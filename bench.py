@@ -4,6 +4,9 @@ A step is one pass of the whole hot path over one batch: quantize-on-append of
 the step's new K/V token of every sequence into the paged cache, then the fused
 split-K decode attention with its per-query bound and flags over the full
 context (and, when tau is finite and a query is flagged, the exact fallback).
+By default the append runs inside the decode launch (kvq_decode_attention_append,
+one launch per step); --two-calls times kvq_quantize_append followed by
+kvq_decode_attention instead.
 The metric is KV token-heads processed per second (sum of context lengths x kv
 heads per step) and the achieved HBM bandwidth of the decode kernel against the
 measured peak.
@@ -205,7 +208,7 @@ def _barrier(world):
 class GpuStep:
     """Device-resident workload and the raw C-ABI calls of one step."""
 
-    def __init__(self, wl_name: str, seed: int, replicas: int):
+    def __init__(self, wl_name: str, seed: int, replicas: int, two_calls: bool = False):
         import ctypes
 
         import torch
@@ -269,13 +272,24 @@ class GpuStep:
              self.pt.shape[1], self.sl.data_ptr(), 0.0, wl.tau, self.out.data_ptr(),
              self.bound.data_ptr(), self.flags.data_ptr(), w.data_ptr(), w.numel(), s)
             for c, w in zip(self.caches, self.ws)]
+        # the fused step: the new token appended inside the decode launch
+        self.fused_args = [
+            (ctypes.byref(c.desc), kn.data_ptr(), vn.data_ptr(), dt, kn.stride(0), kn.stride(1),
+             self.qd.data_ptr(), qdt, B, NQ, HQ, self.pt.data_ptr(), self.pt.shape[1],
+             self.sl.data_ptr(), 0.0, wl.tau, self.out.data_ptr(), self.bound.data_ptr(),
+             self.flags.data_ptr(), w.data_ptr(), w.numel(), s)
+            for c, w in zip(self.caches, self.ws)]
+        self.two_calls = two_calls
         self.token_heads = int(sum(inp.seq_lens)) * wl.num_kv_heads
         bb = base.block_bytes
         self.decode_bytes = (sum(inp.seq_lens) * wl.num_kv_heads * bb // 16
                              + sum(inp.pages_per_seq) * wl.num_kv_heads * 4)
+        if not two_calls:   # plus the new token in (k and v) and its codes out
+            es = 2 if dt == kvq.KVQ_BF16 else 4
+            self.decode_bytes += wl.num_seqs * wl.num_kv_heads * (2 * wl.head_dim * es + bb // 16)
         self.cache_bytes = inp.num_pages * wl.num_kv_heads * bb
         self.replicas = replicas
-        self.launches_per_step = 2
+        self.launches_per_step = 2 if two_calls else 1
         # finite tau: flagged rows are recomputed exactly from pinned host originals
         self.fallback = None
         if math.isfinite(wl.tau):
@@ -312,6 +326,15 @@ class GpuStep:
 
     def step(self, i, ev=None):
         r = i % self.replicas
+        if not self.two_calls:
+            if ev is not None:
+                ev[0].record(self.stream)
+            rc = self.L.kvq_decode_attention_append(*self.fused_args[r])
+            if rc:
+                raise RuntimeError(self.kvq.last_error())
+            if ev is not None:
+                ev[1].record(self.stream)
+            return
         rc = self.L.kvq_quantize_append(*self.append_args[r])
         if rc:
             raise RuntimeError(self.kvq.last_error())
@@ -330,7 +353,7 @@ def run_gpu(args):
     wl = synth.WORKLOADS[args.workload]
     reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl))))
     reps = min(reps, 8)
-    st = GpuStep(args.workload, args.seed, reps)
+    st = GpuStep(args.workload, args.seed, reps, two_calls=args.two_calls)
     # setup: one untimed call per cache replica (library-side descriptors and
     # occupancy are cached by the first call), then the W warm-up steps
     with torch.cuda.stream(st.stream):
@@ -427,12 +450,16 @@ def run_gpu(args):
                    "l2": f"inputs larger than L2: {reps} cache replicas of "
                          f"{st.cache_bytes / 1e6:.1f} MB rotated per step",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "step": ("kvq_quantize_append + kvq_decode_attention" if st.two_calls else
+                            "kvq_decode_attention_append (append fused into the decode)"),
                    "token_heads_per_step": st.token_heads,
                    "decode_bytes_per_launch": st.decode_bytes},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy bandwidth",
-                     "kernel": "decode_mma_kernel", "kernel_ms": dec_ms},
+                     "kernel": "decode_mma_kernel" + ("" if st.two_calls else
+                                                       " (append fused)"),
+                     "kernel_ms": dec_ms},
         "e2e": {"value": _job_value(st.token_heads, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": st.launches_per_step * args.steps,
@@ -553,6 +580,9 @@ def main():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--two-calls", action="store_true",
+                    help="step = kvq_quantize_append + kvq_decode_attention (default: the fused "
+                         "kvq_decode_attention_append)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -159,6 +159,31 @@ KVQ_API int kvq_error_bound(const kvq_cache* cache, const void* q, int q_dtype, 
                     float tau, float* bound, uint8_t* flags, void* workspace,
                     size_t workspace_bytes, kvq_stream_t stream);
 
+/* One decode step in one launch: kvq_quantize_append of the step's new token
+ * fused into kvq_decode_attention.  For every sequence s with seq_lens[s] >= 1
+ * the new token -- k_new / v_new (device, in_dtype) element (s, h, c) at
+ * s*new_seq_stride + h*new_head_stride + c -- is quantized exactly as
+ * kvq_quantize_append would (same codes, scales and eta) into logical
+ * position seq_lens[s] - 1, i.e. physical page
+ * page_table[s*max_pages_per_seq + (seq_lens[s]-1)/16], and the attention over
+ * seq_lens[s] tokens includes it.  Equivalent to kvq_quantize_append
+ * (num_tokens = 1, start_pos = seq_lens - 1) followed by kvq_decode_attention,
+ * with the same results, minus one launch and its dependent round trips; the
+ * warp of the decode that reads the sequence's last page writes the token
+ * into it first.  Sequences with seq_lens[s] == 0 append nothing.  Errors as
+ * for the two calls.  Not the "Runtime-Certified..." pages' own interface: a
+ * fusion of two of its calls. */
+KVQ_API int kvq_decode_attention_append(const kvq_cache* cache, const void* k_new,
+                                        const void* v_new, int in_dtype,
+                                        int64_t new_seq_stride, int64_t new_head_stride,
+                                        const void* q, int q_dtype, int32_t num_seqs,
+                                        int32_t num_queries, int32_t num_q_heads,
+                                        const int32_t* page_table, int32_t max_pages_per_seq,
+                                        const int32_t* seq_lens, float softmax_scale, float tau,
+                                        float* out, float* bound, uint8_t* flags,
+                                        void* workspace, size_t workspace_bytes,
+                                        kvq_stream_t stream);
+
 /* Staging bytes kvq_fallback_exact needs to recompute one (sequence, kv head)
  * of up to max_ctx tokens (the minimum; more lets it batch several). */
 KVQ_API size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype, int32_t max_ctx);

@@ -35,6 +35,7 @@
 #include <type_traits>
 
 #include "kvq_internal.cuh"
+#include "quantize_token.cuh"
 
 namespace kvq {
 
@@ -81,6 +82,10 @@ struct DecodeCfg {
   static_assert(MERGE_BYTES <= OFF_BAR, "merge area must fit in the stage buffers");
 };
 
+// weight of the last split when the append is fused (its appending warp spends
+// about two pages' time on the new token before starting on its pages)
+constexpr float kAppendLastSplit = 0.85f;
+
 // resident CTAs per SM the register budget is sized for (4 = 128 registers)
 template <int D, int KB, int KG>
 constexpr int min_ctas() { return 4; }
@@ -91,17 +96,51 @@ constexpr int min_ctas() { return 4; }
 // later, and with fewer pages the splits of a (sequence, kv head) end together.
 // (fp32 arithmetic: no 64-bit division on the kernel's start path; every CTA
 // evaluates the same expression, so neighbouring splits agree on their border,
-// and the result is monotone in s with split_start(0) = 0, split_start(n) = npages)
-__device__ __forceinline__ int split_start(int s, int n, int npages) {
+// and the result is monotone in s with split_start(0) = 0, split_start(n) = npages).
+// last_w scales the last split's weight (the fused append gives its warp extra
+// work before its pages).
+__device__ __forceinline__ int split_start(int s, int n, int npages, float last_w) {
   if (s <= 0) return 0;
   if (s >= n) return npages;
   const float k = 10.0f * (float)(n - 1);
   const float w = (float)s * k - 0.5f * (float)s * (float)(s - 1);
-  const float wn = (float)n * k - 0.5f * (float)n * (float)(n - 1);
+  const float wn = (float)(n - 1) * k - 0.5f * (float)(n - 1) * (float)(n - 2) +
+                   last_w * (k - (float)(n - 1));
   return min(npages, (int)__fmul_rn((float)npages, __fdiv_rn(w, wn)));
 }
 
-template <int D, int KB, int KG, int S>
+// The step's new token of (b, kvh) into slot (n - 1) % 16 of physical page pg
+// (kvq_decode_attention_append); returns the token's eta contribution.  Not
+// inlined: its registers stay out of the decode's allocation.
+template <int D, int KB, int KG>
+__device__ __noinline__ float fused_append(const DecodeArgs& a, int b, int kvh, int n, int pg,
+                                           int lane) {
+  constexpr int E = D / 32;
+  float xk[E], xv[E];
+  const int64_t base = b * a.app_seq_stride + kvh * a.app_head_stride + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    xk[e] = load_elem(a.app_k, a.app_bf16, base + e);
+    xv[e] = load_elem(a.app_v, a.app_bf16, base + e);
+  }
+  float eu = 0.f;
+  if ((unsigned)pg < (unsigned)a.num_pages) {
+    const BlockLayout L{D, KB, KG};
+    uint8_t* blk = const_cast<uint8_t*>(a.pool) + ((int64_t)pg * a.hkv + kvh) * L.bytes();
+    eu = quantize_token_warp<D, KB, KG>(xk, xv, blk, (n - 1) % kPage,
+                                        const_cast<float*>(a.eta) + (int64_t)pg * a.hkv + kvh,
+                                        a.signs, a.rot_c, a.err, lane);
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  } else if (lane == 0) {
+    set_error(a.err, KVQ_ERR_INVALID_ARG);
+  }
+  __syncwarp();
+  return eu;
+}
+
+// APPEND: the fused step (kvq_decode_attention_append); a separate
+// instantiation, so the plain decode carries none of its code or registers.
+template <int D, int KB, int KG, int S, bool APPEND>
 __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     decode_mma_kernel(const __grid_constant__ DecodeArgs a) {
   using C = DecodeCfg<D, KB, KG, S>;
@@ -128,12 +167,26 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   // are loaded together: none of these addresses depends on the others (the
   // page indices assume a full-length context and are reloaded otherwise).
   const int nsp = gridDim.y;
-  const int p0_spec = split_start(split, nsp, a.max_pages);
-  const int p1_spec = split_start(split + 1, nsp, a.max_pages);
+  constexpr float kLastW = APPEND ? kAppendLastSplit : 1.0f;
+  const int p0_spec = split_start(split, nsp, a.max_pages, kLastW);
+  const int p1_spec = split_start(split + 1, nsp, a.max_pages, kLastW);
   const int32_t* ptab = a.page_table + (int64_t)b * a.max_pages;
   int n = a.seq_lens[b];
   int pt_first = p0_spec + warp + lane * kWarps < p1_spec
                      ? __ldg(ptab + p0_spec + warp + lane * kWarps) : -1;
+  constexpr int E = D / 32;
+  if constexpr (APPEND) {
+    // the warp that appends when the context is full-length (the usual case):
+    // start pulling the step's new token toward L2 now
+    const int lp = a.max_pages - 1;
+    if (lp >= p0_spec && lp < p1_spec && (lp - p0_spec) % kWarps == warp && lane < 2) {
+      const int esz = a.app_bf16 ? 2 : 4;
+      const char* src = static_cast<const char*>(lane == 0 ? a.app_k : a.app_v) +
+                        (b * a.app_seq_stride + kvh * a.app_head_stride) * esz;
+      for (int off = 0; off < D * esz; off += 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(src + off));
+    }
+  }
   constexpr int QPT = kRows * D / (kWarps * 32);   // query elements per thread
   float qreg[QPT];
 #pragma unroll
@@ -167,11 +220,25 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     }
     return;
   }
-  const int p0 = split_start(split, active, npages);
-  const int p1 = split_start(split + 1, active, npages);
+  const int p0 = split_start(split, active, npages, kLastW);
+  const int p1 = split_start(split + 1, active, npages, kLastW);
   const int first = p0 + warp;
   if (p0 != p0_spec || p1 != p1_spec)
     pt_first = first + lane * kWarps < p1 ? __ldg(ptab + first + lane * kWarps) : -1;
+  // The fused append is done by the warp whose local pages include the
+  // sequence's last page, before that page's copy: codes and metadata go to
+  // global memory through the generic proxy, and the proxy fence orders them
+  // before the bulk copy (async proxy) that reads the page back.  When the last
+  // page is among the warp's first S it runs here; otherwise just before the
+  // page loop, so the rest of the CTA does not wait for it at the prologue's
+  // barriers.  Returns the token's eta contribution (0 if the page is invalid).
+  const bool app_here =
+      APPEND && npages - 1 >= p0 && npages - 1 < p1 && (npages - 1 - p0) % kWarps == warp;
+  const int j_last = (npages - 1 - first) / kWarps;   // local index of the last page
+  auto do_append = [&]() -> float {
+    return fused_append<D, KB, KG>(a, b, kvh, n, ptab[npages - 1], lane);
+  };
+  if (app_here && j_last < S) (void)do_append();
 
   uint8_t* stage0 = sm + C::OFF_ST + warp * S * C::BLOCK;
   int* spage = reinterpret_cast<int*>(sm + C::OFF_PG) + warp * S;
@@ -201,8 +268,11 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       pt_val = (c == pt_chunk + 1) ? pt_next : fetch_chunk(c);
       pt_next = fetch_chunk(c + 1);
       pt_chunk = c;
-      eta_iss = (unsigned)pt_val < (unsigned)a.num_pages ? __ldg(eta_kv + (int64_t)pt_val * a.hkv)
-                                                        : 0.f;
+      // (the fused append raises eta in this kernel: read it from L2, not L1)
+      eta_iss = (unsigned)pt_val < (unsigned)a.num_pages
+                    ? (APPEND ? __ldcg(eta_kv + (int64_t)pt_val * a.hkv)
+                              : __ldg(eta_kv + (int64_t)pt_val * a.hkv))
+                    : 0.f;
     }
     const int page = __shfl_sync(0xffffffffu, pt_val, j & 31);
     if (lane == 0) {
@@ -377,6 +447,14 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   }
   const int voff = c4 * C::VRB + g8 * C::VSTR;           // V stripe of token c4 (+4 rows per k)
   const int zgrp = g8 < NB ? g8 : 0;
+
+  // the fused append when the last page comes later: after the q prologue, so
+  // only this warp (whose split is the shortest) starts its pages later
+  if (app_here && j_last >= S) {
+    const float eu = do_append();
+    // the last page's eta, if its chunk was already loaded, gets the token too
+    if ((j_last >> 5) == pt_chunk && lane == (j_last & 31)) eta_iss = fmaxf(eta_iss, eu);
+  }
 
   // ---- page loop ---------------------------------------------------------------
   // One step per local page j, in ring stage j % S.  The stage is a template
@@ -927,8 +1005,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 template <int D, int KB, int KG>
 DecodeVariant make_variant() {
   constexpr int S = 3;
-  return DecodeVariant{decode_mma_kernel<D, KB, KG, S>, DecodeCfg<D, KB, KG, S>::SMEM,
-                       record_floats(D)};
+  return DecodeVariant{decode_mma_kernel<D, KB, KG, S, false>, decode_mma_kernel<D, KB, KG, S, true>,
+                       DecodeCfg<D, KB, KG, S>::SMEM, record_floats(D)};
 }
 
 DecodeVariant select_decode_kernel(int d, int kbits, int kgroup) {
@@ -945,7 +1023,7 @@ DecodeVariant select_decode_kernel(int d, int kbits, int kgroup) {
   KVQ_DECODE_CASE(64, 4, 64)
   KVQ_DECODE_CASE(64, 4, 32)
 #undef KVQ_DECODE_CASE
-  return DecodeVariant{nullptr, 0, 0};
+  return DecodeVariant{nullptr, nullptr, 0, 0};
 }
 
 int decode_threads() { return kWarps * 32; }

@@ -112,6 +112,9 @@ int decode_occupancy(const DecodeVariant& v, int* occ) {
   if (it == cache.end()) {
     cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void*>(v.kernel),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(v.kernel_append),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, v.smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     int n = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reinterpret_cast<const void*>(v.kernel),
@@ -163,11 +166,19 @@ int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
   return KVQ_OK;
 }
 
+// The step's new token for kvq_decode_attention_append (NULL: plain decode).
+struct NewToken {
+  const void* k;
+  const void* v;
+  int bf16;
+  int64_t seq_stride, head_stride;
+};
+
 int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
                 int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
                 int32_t max_pages, const int32_t* seq_lens, float softmax_scale, float tau,
                 float* out, float* bound, uint8_t* flags, void* ws, size_t ws_bytes,
-                cudaStream_t stream) {
+                cudaStream_t stream, const NewToken* nt = nullptr) {
   int rc = check_cache(cache);
   if (rc) return rc;
   if (num_seqs < 0 || num_queries < 1 || num_q_heads < 1 || max_pages < 1)
@@ -218,13 +229,18 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
   a.flags = flags;
   a.counters = static_cast<int*>(ws);
   a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plan.counter_bytes);
+  a.app_k = nt ? nt->k : nullptr;
+  a.app_v = nt ? nt->v : nullptr;
+  a.app_bf16 = nt ? nt->bf16 : 0;
+  a.app_seq_stride = nt ? nt->seq_stride : 0;
+  a.app_head_stride = nt ? nt->head_stride : 0;
   // (sequence x kv head, split): the split index in the slow dimension
   const int64_t units = (int64_t)num_seqs * cache->num_kv_heads;
   if (units > 0x7fffffffLL || plan.splits > 65535)
     return fail(KVQ_ERR_UNSUPPORTED, "grid too large (%lld units, %d splits)", (long long)units,
                 plan.splits);
   dim3 grid((unsigned)units, (unsigned)plan.splits, 1);
-  v.kernel<<<grid, decode_threads(), v.smem, stream>>>(a);
+  (nt ? v.kernel_append : v.kernel)<<<grid, decode_threads(), v.smem, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   return KVQ_OK;
@@ -342,6 +358,25 @@ int kvq_error_bound(const kvq_cache* cache, const void* q, int q_dtype, int32_t 
   return decode_impl(cache, q, q_dtype, num_seqs, num_queries, num_q_heads, page_table,
                      max_pages_per_seq, seq_lens, softmax_scale, tau, nullptr, bound, flags,
                      workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int kvq_decode_attention_append(const kvq_cache* cache, const void* k_new, const void* v_new,
+                                int in_dtype, int64_t new_seq_stride, int64_t new_head_stride,
+                                const void* q, int q_dtype, int32_t num_seqs, int32_t num_queries,
+                                int32_t num_q_heads, const int32_t* page_table,
+                                int32_t max_pages_per_seq, const int32_t* seq_lens,
+                                float softmax_scale, float tau, float* out, float* bound,
+                                uint8_t* flags, void* workspace, size_t workspace_bytes,
+                                kvq_stream_t stream) {
+  if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad in_dtype");
+  if (new_seq_stride < 0 || new_head_stride < 0)
+    return fail(KVQ_ERR_INVALID_ARG, "negative stride");
+  if (num_seqs > 0 && (!k_new || !v_new)) return fail(KVQ_ERR_INVALID_ARG, "NULL k_new or v_new");
+  if (!out && num_seqs > 0) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+  const NewToken nt{k_new, v_new, in_dtype == KVQ_BF16, new_seq_stride, new_head_stride};
+  return decode_impl(cache, q, q_dtype, num_seqs, num_queries, num_q_heads, page_table,
+                     max_pages_per_seq, seq_lens, softmax_scale, tau, out, bound, flags, workspace,
+                     workspace_bytes, reinterpret_cast<cudaStream_t>(stream), &nt);
 }
 
 size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype, int32_t max_ctx) {

@@ -40,11 +40,19 @@ struct DecodeArgs {
   uint8_t* flags;
   float* part;
   int* counters;
+  // fused append (NULL app_k: none): the new token of sequence s, kv head h at
+  // element s * app_seq_stride + h * app_head_stride, written at position
+  // seq_lens[s] - 1 before the decode reads the page
+  const void* app_k;
+  const void* app_v;
+  int app_bf16;
+  int64_t app_seq_stride, app_head_stride;
 };
 
 using DecodeKernel = void (*)(const DecodeArgs);
 struct DecodeVariant {
   DecodeKernel kernel;
+  DecodeKernel kernel_append;  // the same with the step's append fused in
   int smem;    // dynamic shared memory bytes
   int record;  // floats per split record
 };

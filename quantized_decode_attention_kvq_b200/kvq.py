@@ -35,7 +35,7 @@ PAGE_SIZE = 16
 EXPORTED = ("kvq_block_bytes", "kvq_pool_bytes", "kvq_quantize_append", "kvq_workspace_size",
             "kvq_decode_attention", "kvq_error_bound", "kvq_fallback_staging_size",
             "kvq_fallback_exact", "kvq_device_error", "kvq_status_string", "kvq_last_error",
-            "kvq_decode_attention_noalloc")
+            "kvq_decode_attention_noalloc", "kvq_decode_attention_append")
 
 
 class KvqError(RuntimeError):
@@ -79,6 +79,9 @@ def _load() -> ctypes.CDLL:
         "kvq_device_error": (ctypes.c_int, [C, P, ctypes.POINTER(I32)]),
         "kvq_decode_attention_noalloc": (ctypes.c_int, [C, P, ctypes.c_int, I32, I32, I32, P,
                                                         I32, P, F, F, P, P, P, P]),
+        "kvq_decode_attention_append": (ctypes.c_int, [C, P, P, ctypes.c_int, I64, I64, P,
+                                                       ctypes.c_int, I32, I32, I32, P, I32, P, F,
+                                                       F, P, P, P, P, SZ, P]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -190,6 +193,21 @@ def kvq_decode_attention_noalloc(cache, q, q_dtype, num_seqs, num_queries, num_q
 
 
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def kvq_decode_attention_append(cache, k_new, v_new, in_dtype, new_seq_stride, new_head_stride,
+                                q, q_dtype, num_seqs, num_queries, num_q_heads, page_table,
+                                max_pages_per_seq, seq_lens, softmax_scale, tau, out, bound,
+                                flags, workspace, workspace_bytes, stream=None) -> int:
+    """One decode step in one launch: the new token of every sequence is appended
+    at position seq_lens - 1, then the decode runs over seq_lens tokens."""
+    return _lib.kvq_decode_attention_append(ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
+                                            in_dtype, new_seq_stride, new_head_stride, _ptr(q),
+                                            q_dtype, num_seqs, num_queries, num_q_heads,
+                                            _ptr(page_table), max_pages_per_seq, _ptr(seq_lens),
+                                            softmax_scale, tau, _ptr(out), _ptr(bound),
+                                            _ptr(flags), _ptr(workspace), workspace_bytes,
+                                            _stream(stream))
 
 
 def kvq_fallback_staging_size(cache, orig_dtype, max_ctx) -> int:
