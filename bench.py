@@ -205,6 +205,24 @@ def _barrier(world):
         dist.barrier()
 
 
+def _packed(tensors):
+    """One device byte buffer holding copies of `tensors` (256-byte aligned parts)
+    and the views of it that replace them."""
+    import torch
+    sizes = [t.numel() * t.element_size() for t in tensors]
+    offs, total = [], 0
+    for n in sizes:
+        offs.append(total)
+        total += (n + 255) // 256 * 256
+    buf = torch.empty(total, dtype=torch.uint8, device=tensors[0].device)
+    views = []
+    for t, o, n in zip(tensors, offs, sizes):
+        v = buf[o:o + n].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+    return buf, views
+
+
 class GpuStep:
     """Device-resident workload and the raw C-ABI calls of one step."""
 
@@ -252,9 +270,13 @@ class GpuStep:
         self.ws = [c.workspace(wl.num_seqs, wl.num_queries, wl.num_q_heads, self.pt.shape[1])
                    for c in self.caches]
         B, NQ, HQ, d = q.shape
-        self.out = torch.empty((B, NQ, HQ, d), dtype=torch.float32, device="cuda")
-        self.bound = torch.empty((B, NQ, HQ), dtype=torch.float32, device="cuda")
-        self.flags = torch.empty((B, NQ, HQ), dtype=torch.uint8, device="cuda")
+        # the step's inputs (q, new k, new v) and results (out, bound, flags) each
+        # live in one device buffer, so a step moves them with one copy each way
+        self.io_in, (self.qd, self.k_new, self.v_new) = _packed([self.qd, self.k_new, self.v_new])
+        self.io_out, (self.out, self.bound, self.flags) = _packed(
+            [torch.empty((B, NQ, HQ, d), dtype=torch.float32, device="cuda"),
+             torch.empty((B, NQ, HQ), dtype=torch.float32, device="cuda"),
+             torch.empty((B, NQ, HQ), dtype=torch.uint8, device="cuda")])
         # one dedicated stream: the eager steps and the captured graph use it
         self.stream = torch.cuda.Stream()
         s = self.stream.cuda_stream
@@ -397,15 +419,12 @@ def run_gpu(args):
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
 
     # end to end through the public API with host buffers: H2D of the step's inputs
-    # (q and the new K/V token) from pinned memory, the two calls, D2H of the results
-    q_h = st.qd.cpu().pin_memory()
-    kn_h = st.k_new.cpu().pin_memory()
-    vn_h = st.v_new.cpu().pin_memory()
-    out_h = torch.empty(st.out.shape, dtype=torch.float32).pin_memory()
-    bound_h = torch.empty(st.bound.shape, dtype=torch.float32).pin_memory()
-    flags_h = torch.empty(st.flags.shape, dtype=torch.uint8).pin_memory()
-    h2d = q_h.numel() * q_h.element_size() + 2 * kn_h.numel() * kn_h.element_size()
-    d2h = out_h.numel() * 4 + bound_h.numel() * 4 + flags_h.numel()
+    # (q and the new K/V token, packed) from pinned memory, the step's call(s), D2H
+    # of the results (out, bound, flags, packed)
+    in_h = st.io_in.cpu().pin_memory()
+    out_h = torch.empty(st.io_out.shape, dtype=torch.uint8).pin_memory()
+    h2d = st.qd.numel() * st.qd.element_size() + 2 * st.k_new.numel() * st.k_new.element_size()
+    d2h = st.out.numel() * 4 + st.bound.numel() * 4 + st.flags.numel()
     # with a finite tau the step ends with the host-synchronous exact fallback of the
     # flagged rows, which pages in their originals: a few steps suffice
     e_steps = max(1, args.steps) if st.fallback is None else max(1, min(args.steps, 5))
@@ -416,15 +435,11 @@ def run_gpu(args):
     with torch.cuda.stream(st.stream):
         e0.record(st.stream)
         for i in range(e_steps):
-            st.qd.copy_(q_h, non_blocking=True)
-            st.k_new.copy_(kn_h, non_blocking=True)
-            st.v_new.copy_(vn_h, non_blocking=True)
+            st.io_in.copy_(in_h, non_blocking=True)
             st.step(i)
             if st.fallback is not None:
                 st.fallback_exact(i % st.replicas)
-            out_h.copy_(st.out, non_blocking=True)
-            bound_h.copy_(st.bound, non_blocking=True)
-            flags_h.copy_(st.flags, non_blocking=True)
+            out_h.copy_(st.io_out, non_blocking=True)
         e1.record(st.stream)
     torch.cuda.synchronize()
     ms_step, dec_ms, e2e_ms = _rank_times(ms_total, dec_ms, e0.elapsed_time(e1) / e_steps,
