@@ -185,7 +185,12 @@ KVQ_API int kvq_decode_attention_append(const kvq_cache* cache, const void* k_ne
                                         kvq_stream_t stream);
 
 /* Staging bytes kvq_fallback_exact needs to recompute one (sequence, kv head)
- * of up to max_ctx tokens (the minimum; more lets it batch several). */
+ * of up to max_ctx tokens: a merge scratch (48 items x 8 rows x (head_dim
+ * + 2) floats, rounded up to 256 B) plus K and V of max_ctx tokens (each
+ * rounded up to 256 B).  This is the minimum; with room for two such K/V
+ * pairs beyond the scratch, the call splits the buffer in two halves and the
+ * copies into one overlap the recomputation from the other.  0 for an
+ * unsupported head_dim or dtype. */
 KVQ_API size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype, int32_t max_ctx);
 
 /* Exact recomputation from Tier 2 (Methodology 1, Fallback; per-head rung of
@@ -196,10 +201,14 @@ KVQ_API size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype,
  * once).  For every (sequence, kv head) with a flagged query it copies the
  * originals k_orig_host, v_orig_host (pinned, orig_dtype, element (s, h, t, c)
  * at s*orig_seq_stride + h*orig_head_stride + t*head_dim + c) for tokens
- * [0, seq_lens_host[s]) into `staging` (device) with cudaMemcpyAsync on
- * `side`, and overwrites out rows of the flagged queries with exact fp32
- * softmax attention (softmax_scale as in decode).  q as in decode.  `main`
- * then waits for `side`.  *num_fallback (host) = number of recomputed
+ * [0, seq_lens_host[s]) into `staging` (device, 16-byte aligned, at least
+ * kvq_fallback_staging_size bytes) with cudaMemcpyAsync on `side`, and
+ * overwrites out rows of the flagged queries with exact fp32 softmax
+ * attention (softmax_scale as in decode).  q as in decode.  The recompute
+ * kernels run on `main`, each after the copies it reads (events), so `main`
+ * is ordered after all of this call's work when it returns; the copies into
+ * a staging half that is being reused wait (on `side`) for the recompute
+ * that read it before.  *num_fallback (host) = number of recomputed
  * queries.  On any error out is left unmodified for the rows not yet
  * recomputed.  Blocks the calling thread until the flags are on the host. */
 KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const void* v_orig_host,

@@ -384,7 +384,7 @@ size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype, int32_t
   if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return 0;
   const size_t es = orig_dtype == KVQ_BF16 ? 2 : 4;
   const size_t one = ((size_t)max_ctx * cache->head_dim * es + 255) / 256 * 256;
-  return 2 * (one > 0 ? one : 256);
+  return fallback_scratch_bytes(cache->head_dim) + 2 * one;
 }
 
 int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const void* v_orig_host,
@@ -425,19 +425,25 @@ int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const vo
   cudaStream_t ss = reinterpret_cast<cudaStream_t>(side_stream);
   const size_t rows = (size_t)num_seqs * num_queries * num_q_heads;
 
-  cudaEvent_t ev_dec = nullptr, ev_flags = nullptr, ev_done = nullptr;
+  if (reinterpret_cast<uintptr_t>(staging) % 16)
+    return fail(KVQ_ERR_INVALID_ARG, "staging is not 16-byte aligned");
+  // the decode, the flags on the host, the copies of the open batch, and the
+  // last recompute that read each staging half
+  cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  cudaEvent_t& ev_dec = ev[0];
+  cudaEvent_t& ev_flags = ev[1];
+  cudaEvent_t& ev_copied = ev[2];
+  cudaEvent_t* ev_half = ev + 3;
   auto cleanup = [&]() {
-    if (ev_dec) cudaEventDestroy(ev_dec);
-    if (ev_flags) cudaEventDestroy(ev_flags);
-    if (ev_done) cudaEventDestroy(ev_done);
+    for (cudaEvent_t& x : ev)
+      if (x) cudaEventDestroy(x);
   };
   cudaError_t e;
-  if ((e = cudaEventCreateWithFlags(&ev_dec, cudaEventDisableTiming)) != cudaSuccess ||
-      (e = cudaEventCreateWithFlags(&ev_flags, cudaEventDisableTiming)) != cudaSuccess ||
-      (e = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming)) != cudaSuccess) {
-    cleanup();
-    return cuda_fail(e, "cudaEventCreate");
-  }
+  for (cudaEvent_t& x : ev)
+    if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) {
+      cleanup();
+      return cuda_fail(e, "cudaEventCreate");
+    }
   // flags -> host on the side stream, after the decode on the main stream
   if ((e = cudaEventRecord(ev_dec, ms)) != cudaSuccess ||
       (e = cudaStreamWaitEvent(ss, ev_dec, 0)) != cudaSuccess ||
@@ -465,28 +471,56 @@ int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const vo
       std::this_thread::sleep_for(std::chrono::microseconds(20));
     }
   }
-  // page in and recompute, batching (sequence, kv head) units into the staging buffer
+  // Page in and recompute.  The staging buffer holds the merge scratch, then
+  // two halves when there is room for the longest (sequence, kv head) in each,
+  // else one region.  The originals go in on `side`; a batch's recompute runs
+  // on `main` after its copies, and the next copies into the same half wait
+  // for that recompute, so one half is being filled while the other is read.
+  const size_t scratch = fallback_scratch_bytes(D);
+  const size_t pair_max = 2 * (((size_t)max_n * D * es + 255) / 256 * 256);
+  const size_t region = staging_bytes - scratch;
+  const int halves = pair_max > 0 && region >= 2 * pair_max ? 2 : 1;
+  const size_t half_bytes = halves == 2 ? region / 2 / 256 * 256 : region;
   FbArgs fa;
   std::memset(&fa, 0, sizeof(fa));
   fa.staging = static_cast<const uint8_t*>(staging);
   fa.q = q;
+  fa.out = out;
+  fa.scratch = static_cast<float*>(staging);
   fa.q_bf16 = q_dtype == KVQ_BF16;
   fa.kv_bf16 = orig_dtype == KVQ_BF16;
   fa.s_att = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)D));
-  fa.out = out;
+  int half = 0;
+  bool half_read[2] = {false, false};
   size_t used = 0;
   int32_t count = 0;
-  auto flush = [&]() -> int {
+  // the recompute of the items gathered so far, after every copy issued so far
+  auto launch = [&]() -> int {
     if (fa.num_items == 0) return KVQ_OK;
-    cudaError_t le = launch_fallback(fa, D, ss);
-    if (le != cudaSuccess) return cuda_fail(le, "fallback kernel launch");
+    if ((e = cudaEventRecord(ev_copied, ss)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(ms, ev_copied, 0)) != cudaSuccess)
+      return cuda_fail(e, "copy hand-off");
+    if ((e = launch_fallback(fa, D, ms)) != cudaSuccess) return cuda_fail(e, "fallback kernel launch");
     fa.num_items = 0;
-    used = 0;
+    fa.any_split = 0;
     return KVQ_OK;
   };
+  // close the batch in the current half and open the other one
+  auto next_half = [&]() -> int {
+    int r = launch();
+    if (r) return r;
+    if ((e = cudaEventRecord(ev_half[half], ms)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    half_read[half] = true;
+    half = (half + 1) % halves;
+    used = 0;
+    if (half_read[half] && (e = cudaStreamWaitEvent(ss, ev_half[half], 0)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamWaitEvent");
+    return KVQ_OK;
+  };
+  std::vector<int64_t> rws;
   for (int s = 0; s < num_seqs; ++s) {
     for (int h = 0; h < hkv; ++h) {
-      std::vector<int64_t> rws;
+      rws.clear();
       for (int i = 0; i < num_queries; ++i)
         for (int gq = 0; gq < G; ++gq) {
           const int64_t row = ((int64_t)s * num_queries + i) * num_q_heads + h * G + gq;
@@ -495,9 +529,10 @@ int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const vo
       if (rws.empty()) continue;
       const int n = seq_lens_host[s];
       const size_t one = ((size_t)n * D * es + 255) / 256 * 256;
-      if (used + 2 * one > staging_bytes || fa.num_items + (int)rws.size() > kFbMaxItems)
-        if ((rc = flush())) { cleanup(); return rc; }
-      const int64_t koff = (int64_t)used, voff = (int64_t)(used + one);
+      if (used + 2 * one > half_bytes)
+        if ((rc = next_half())) { cleanup(); return rc; }
+      const int64_t koff = (int64_t)(scratch + half * half_bytes + used);
+      const int64_t voff = koff + (int64_t)one;
       if (n > 0) {
         if (fault_injected("memcpy")) {
           cleanup();
@@ -516,22 +551,31 @@ int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const vo
         }
       }
       used += 2 * one;
-      for (int64_t row : rws) {
-        FbItem& it = fa.items[fa.num_items++];
-        it.k_off = koff;
-        it.v_off = voff;
-        it.q_row = row;
-        it.n = n;
-        ++count;
+      // items: row groups of up to kFbRows, each cut into nchunk token ranges
+      const int nchunk = n <= kFbMinChunk ? 1 : std::min(kFbMaxChunks, (n + kFbMinChunk - 1) / kFbMinChunk);
+      const int clen = (n + nchunk - 1) / nchunk;
+      for (size_t g0 = 0; g0 < rws.size(); g0 += kFbRows) {
+        const int nrw = (int)std::min<size_t>(kFbRows, rws.size() - g0);
+        if (fa.num_items + nchunk > kFbMaxItems)
+          if ((rc = launch())) { cleanup(); return rc; }
+        for (int c = 0; c < nchunk; ++c) {
+          FbItem& it = fa.items[fa.num_items++];
+          it.k_off = koff;
+          it.v_off = voff;
+          it.row0 = rws[g0];
+          it.t0 = c * clen;
+          it.t1 = std::min(n, (c + 1) * clen);
+          for (int r = 0; r < kFbRows; ++r) it.roff[r] = r < nrw ? (int32_t)(rws[g0 + r] - rws[g0]) : 0;
+          it.nrows = (int16_t)nrw;
+          it.chunk = (int16_t)c;
+          it.nchunk = (int16_t)nchunk;
+        }
+        if (nchunk > 1) fa.any_split = 1;
+        count += nrw;
       }
     }
   }
-  if ((rc = flush())) { cleanup(); return rc; }
-  if ((e = cudaEventRecord(ev_done, ss)) != cudaSuccess ||
-      (e = cudaStreamWaitEvent(ms, ev_done, 0)) != cudaSuccess) {
-    cleanup();
-    return cuda_fail(e, "stream hand-back");
-  }
+  if ((rc = launch())) { cleanup(); return rc; }
   cleanup();
   *num_fallback = count;
   return KVQ_OK;

@@ -57,27 +57,44 @@ struct DecodeVariant {
   int record;  // floats per split record
 };
 
-constexpr int kFbMaxItems = 64;
+// Exact fallback work items.  One item = one CTA: up to kFbRows flagged query
+// rows of one (sequence, kv head) over the token range [t0, t1) of its staged
+// originals.  A (sequence, kv head) longer than kFbMinChunk tokens is cut into
+// up to kFbMaxChunks ranges (consecutive items, chunk 0..nchunk-1) whose
+// partial softmax states go to the scratch and are merged by a second kernel.
+constexpr int kFbRows = 8;
+constexpr int kFbMaxItems = 48;     // items per launch (the argument block stays < 4 KB)
+constexpr int kFbMaxChunks = 8;
+constexpr int kFbMinChunk = 128;    // tokens
 struct FbItem {
-  int64_t k_off;  // bytes into staging
+  int64_t k_off;             // bytes into staging: K [n][D], then V at v_off
   int64_t v_off;
-  int64_t q_row;  // flattened (sequence, query, q head)
-  int n;
-  int pad;
+  int64_t row0;              // flattened (sequence, query, q head) index of row offset 0
+  int32_t t0, t1;            // token range of this item
+  int32_t roff[kFbRows];     // row = row0 + roff[r], r < nrows
+  int16_t nrows, chunk, nchunk, pad;
 };
 struct FbArgs {
   const uint8_t* staging;
   const void* q;
+  float* out;
+  float* scratch;            // [kFbMaxItems][kFbRows][D + 2]: o (unnormalised), m, l
   int q_bf16, kv_bf16;
   float s_att;
-  float* out;
   int num_items;
+  int any_split;             // some item has nchunk > 1: the merge kernel runs
+  int pad;
   FbItem items[kFbMaxItems];
 };
+// bytes of the merge scratch at the start of the staging buffer
+inline size_t fallback_scratch_bytes(int d) {
+  return ((size_t)kFbMaxItems * kFbRows * (d + 2) * sizeof(float) + 255) / 256 * 256;
+}
 
 cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, cudaStream_t s);
 DecodeVariant select_decode_kernel(int d, int kbits, int kgroup);
 int decode_threads();
+// the recompute (and, when an item was split, the merge) on `stream`
 cudaError_t launch_fallback(const FbArgs& a, int d, cudaStream_t stream);
 
 }  // namespace kvq

@@ -107,9 +107,11 @@ def test_validation_before_any_cuda_call(kvq):
 
 def test_fallback_validation_and_staging_size(kvq):
     d = _desc(kvq)
-    assert kvq.kvq_fallback_staging_size(d, kvq.KVQ_BF16, 1000) == 2 * 1000 * 128 * 2
-    assert kvq.kvq_fallback_staging_size(d, kvq.KVQ_F32, 3) == 2 * 1536 // 256 * 256 + 512 * 0 \
-        or kvq.kvq_fallback_staging_size(d, kvq.KVQ_F32, 3) == 2 * 1536
+    scratch = 48 * 8 * (128 + 2) * 4                  # merge scratch, a multiple of 256 B
+    assert kvq.kvq_fallback_staging_size(d, kvq.KVQ_BF16, 1000) == scratch + 2 * 1000 * 128 * 2
+    assert kvq.kvq_fallback_staging_size(d, kvq.KVQ_F32, 3) == scratch + 2 * 1536
+    assert kvq.kvq_fallback_staging_size(d, kvq.KVQ_F32, 0) == scratch
+    assert kvq.kvq_fallback_staging_size(d, 9, 10) == 0
     rc, n = kvq.kvq_fallback_exact(d, None, None, kvq.KVQ_BF16, 0, 0, 0x10, kvq.KVQ_BF16, 1, 1,
                                    32, None, 0.0, 0x20, 0x30, 0x40, 0x50, 1 << 20, 0, 0, 100)
     assert rc == kvq.KVQ_ERR_INVALID_ARG and n == 0

@@ -1,7 +1,10 @@
 """Certified fallback: flagged queries are recomputed exactly from the pinned
 host originals (side stream, cudaMemcpyAsync); the others keep the quantized
-output.  Host-side failures (deadline, injected copy failure) leave out as it
-was and return a clean status; no GPU fault is provoked."""
+output.  The staging layouts (one region; two halves; two halves that each
+carry several launches), row groups of more than 8 queries per (sequence,
+kv head), token ranges split into merged chunks, and fp32 / d=64 originals
+are covered.  Host-side failures (deadline, injected copy failure) leave out
+as it was and return a clean status; no GPU fault is provoked."""
 
 import numpy as np
 import pytest
@@ -26,7 +29,7 @@ def _host(x: np.ndarray) -> torch.Tensor:
     return t.contiguous().pin_memory()
 
 
-def _fallback(inp, g, k, v, timeout_ms=10000):
+def _fallback(inp, g, k, v, timeout_ms=10000, mult=3):
     from quantized_decode_attention_kvq_b200 import kvq
     wl = inp.wl
     kh, vh = _host(k), _host(v)
@@ -36,7 +39,7 @@ def _fallback(inp, g, k, v, timeout_ms=10000):
     flags_host = torch.zeros(g["flags"].size, dtype=torch.uint8).pin_memory()
     T = k.shape[2]
     dt = kvq.KVQ_BF16 if k.dtype == np.uint16 else kvq.KVQ_F32
-    st_bytes = kvq.kvq_fallback_staging_size(g["cache"].desc, dt, max(inp.seq_lens)) * 3
+    st_bytes = kvq.kvq_fallback_staging_size(g["cache"].desc, dt, max(inp.seq_lens)) * mult
     staging = torch.empty(st_bytes, dtype=torch.uint8, device="cuda")
     side = torch.cuda.Stream()
     sl_host = np.array(inp.seq_lens, np.int32)
@@ -102,3 +105,45 @@ def test_fallback_injected_copy_failure(monkeypatch):
     assert rc == kvq.KVQ_ERR_CUDA and n == 0
     assert "injected" in kvq.last_error()
     assert np.array_equal(out, g["out"])
+
+
+def _check_recovered(inp, g, out, q, k, v):
+    o_dense = oracle.dense(q, k, v, inp.seq_lens)
+    flagged = g["flags"].astype(bool)
+    assert flagged.any()
+    assert compare_outputs(out[flagged], o_dense[flagged])[0] <= 1e-4
+    assert np.array_equal(out[~flagged], g["out"][~flagged])
+
+
+@pytest.mark.parametrize("mult", [1, 3, 40])
+def test_fallback_staging_layouts_and_row_groups(mult):
+    # 30 sequences x 2 kv heads with 12 q heads each: up to 12 flagged rows per
+    # (sequence, kv head), so two row groups; lengths above 128 split in two
+    # chunks.  The flags are seeded (the fallback reads only q, flags and out;
+    # the decode takes at most 4 rows per kv head).  mult 1: one staging
+    # region (each batch's copies wait for the previous recompute); 3: two
+    # halves; 40: two halves, each holding more items than one launch takes.
+    from gpu_cases import gpu_cache, to_torch
+    inp = small("serving", 4, num_seqs=30, num_q_heads=24, num_kv_heads=2)
+    k, v = inp.kv()
+    q = inp.q()
+    rng = np.random.default_rng(40 + mult)
+    flags = (rng.random(q.shape[:3]) < 0.7).astype(np.uint8).reshape(-1)
+    flags[:12] = 1                                         # one full pair of 12 rows
+    g = dict(cache=gpu_cache(inp), q=to_torch(q), flags=flags,
+             out=rng.standard_normal((flags.size, inp.wl.head_dim)).astype(np.float32))
+    rc, n, out, fh = _fallback(inp, g, k, v, mult=mult)
+    assert rc == 0 and n == int(flags.sum())
+    assert np.array_equal(fh, flags)
+    _check_recovered(inp, g, out, q, k, v)
+
+
+def test_fallback_fp32_head_dim_64():
+    inp = small("tiny", 5)                                  # fp32 originals, d=64, 4 queries
+    k, v = inp.kv()
+    q = inp.q()
+    g = run_gpu(inp, k, v, q, tau=0.0)                      # every row flagged
+    assert g["flags"].all()
+    rc, n, out, _ = _fallback(inp, g, k, v, mult=1)
+    assert rc == 0 and n == g["flags"].size
+    _check_recovered(inp, g, out, q, k, v)
