@@ -162,6 +162,25 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
     mbar_fence_init();
   }
+  // Launched with programmatic serialization, the CTA may start while the
+  // previous grid in the stream is still running.  Until pdl_wait it only
+  // prefetches into L2 the pages its warps will copy first, at the indices the
+  // page table holds now for a full-length context: these are hints (clamped
+  // to the pool, and a prefetch changes no memory), so nothing computed below
+  // depends on what the previous grid writes.  Every load that does comes
+  // after the wait.
+  {
+    const int sp0 = split_start(split, gridDim.y, a.max_pages, APPEND ? kAppendLastSplit : 1.0f);
+    const int sp1 = split_start(split + 1, gridDim.y, a.max_pages, APPEND ? kAppendLastSplit : 1.0f);
+    const int lp = sp0 + warp + lane * kWarps;
+    if (lane < S && lp < sp1) {
+      const int pg = __ldcg(a.page_table + (int64_t)b * a.max_pages + lp);
+      if (pg >= 0 && pg < a.num_pages)
+        bulk_prefetch_l2(a.pool + ((int64_t)pg * a.hkv + kvh) * C::BLOCK, C::BLOCK);
+    }
+  }
+  pdl_wait();
+  pdl_release();
 
   // The context length, the query rows and this warp's first 32 page indices
   // are loaded together: none of these addresses depends on the others (the
@@ -188,15 +207,19 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     }
   }
   constexpr int QPT = kRows * D / (kWarps * 32);   // query elements per thread
-  float qreg[QPT];
+  // raw element bits, all loads issued before any is used (the bf16 -> fp32
+  // conversion waits until the rows are written to shared memory)
+  uint32_t qraw[QPT];
+  const bool qb16 = a.q_bf16;
 #pragma unroll
   for (int k = 0; k < QPT; ++k) {
     const int i = tid + k * kWarps * 32, r = i / D, c = i % D;
-    qreg[k] = 0.f;
-    if (r < a.R) {
-      const int qi = r / a.G, h = kvh * a.G + r % a.G;
-      qreg[k] = load_elem(a.q, a.q_bf16, (((int64_t)b * a.nq + qi) * a.hq + h) * D + c);
-    }
+    const int qi = r / a.G, h = kvh * a.G + r % a.G;
+    const int64_t e = (((int64_t)b * a.nq + qi) * a.hq + h) * D + c;
+    const int64_t eo = r < a.R ? e : 0;   // an in-range address for padding rows
+    qraw[k] = qb16 ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(a.q) + eo)
+                   : __float_as_uint(__ldg(reinterpret_cast<const float*>(a.q) + eo));
+    if (r >= a.R) qraw[k] = 0u;
   }
 
   if (n < 0) n = 0;
@@ -281,7 +304,9 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       if (ok) {
         const int64_t blk = (int64_t)page * a.hkv + kvh;
         mbar_arrive_expect_tx(&bar[st], C::BLOCK);
-        bulk_g2s(stage0 + st * C::BLOCK, a.pool + blk * C::BLOCK, C::BLOCK, &bar[st]);
+        // a launch reads each cache page once: its lines are evicted first
+        bulk_g2s_hint(stage0 + st * C::BLOCK, a.pool + blk * C::BLOCK, C::BLOCK, &bar[st],
+                      l2_evict_first_policy());
       } else {
         set_error(a.err, KVQ_ERR_INVALID_ARG);
         mbar_arrive(&bar[st]);
@@ -293,7 +318,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 
   // ---- query rows: rotate, fixed point, norms (loaded before the copies) -----
 #pragma unroll
-  for (int k = 0; k < QPT; ++k) qf[tid + k * kWarps * 32] = qreg[k];
+  for (int k = 0; k < QPT; ++k)
+    qf[tid + k * kWarps * 32] = qb16 ? __uint_as_float(qraw[k] << 16) : __uint_as_float(qraw[k]);
   __syncthreads();
   if (warp < kRows) {
     const int r = warp;

@@ -240,8 +240,8 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
     return fail(KVQ_ERR_UNSUPPORTED, "grid too large (%lld units, %d splits)", (long long)units,
                 plan.splits);
   dim3 grid((unsigned)units, (unsigned)plan.splits, 1);
-  (nt ? v.kernel_append : v.kernel)<<<grid, decode_threads(), v.smem, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(nt ? v.kernel_append : v.kernel, grid, dim3(decode_threads()),
+                             (size_t)v.smem, stream, a);
   if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
   return KVQ_OK;
 }

@@ -95,6 +95,43 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// L2 policy for data read once: its lines are the first evicted, so a stream of
+// them leaves the small inputs every launch re-reads (context lengths, page
+// table, queries, eta, split records) resident in L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// bulk_g2s with an L2 cache policy (l2_evict_first_policy for streamed data)
+__device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// Programmatic dependent launch.  A grid launched with programmatic stream
+// serialization may start while the grid before it in the stream is still
+// finishing; griddepcontrol.wait holds the thread until that grid has
+// completed and its writes are visible (a no-op for an ordinary launch).
+// launch_dependents lets the next such grid begin launching; it starts once
+// every CTA of this grid has run (or passed) that point, so its CTAs take only
+// SM slots this grid has left.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Bring [src, src + bytes) into L2 (16-byte aligned address and size); no
+// destination, no completion, no effect on memory contents.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---- 2^x by the hardware approximation (PTX ex2.approx.ftz.f32) -------------
 // Relative error about 2^-22; results below the normal range flush to +0 and
 // 2^-inf = +0.  Softmax weights and the bound's exponentials need no more.

@@ -91,6 +91,25 @@ inline size_t fallback_scratch_bytes(int d) {
   return ((size_t)kFbMaxItems * kFbRows * (d + 2) * sizeof(float) + 255) / 256 * 256;
 }
 
+// Launch with programmatic stream serialization (the kernel calls pdl_wait
+// before any access that depends on earlier work in the stream): its launch
+// and its first prefetches overlap the end of the grid before it.
+template <typename Arg>
+cudaError_t launch_pdl(void (*kernel)(Arg), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       const Arg& arg) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, arg);
+}
+
 cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, cudaStream_t s);
 DecodeVariant select_decode_kernel(int d, int kbits, int kgroup);
 int decode_threads();
