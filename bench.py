@@ -205,6 +205,31 @@ def _barrier(world):
         dist.barrier()
 
 
+def _cudart():
+    """The CUDA runtime torch loaded, for the end-to-end loop's copies and events
+    (thin calls: the loop issues about ten per step)."""
+    import ctypes
+    import glob
+
+    import torch
+    here = os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib")
+    for c in sorted(glob.glob(os.path.join(here, "libcudart.so*"))) + ["libcudart.so.12"]:
+        try:
+            rt = ctypes.CDLL(c)
+            break
+        except OSError:
+            continue
+    else:
+        raise RuntimeError("libcudart not found")
+    vp = ctypes.c_void_p
+    rt.cudaMemcpyAsync.argtypes = [vp, vp, ctypes.c_size_t, ctypes.c_int, vp]
+    rt.cudaEventRecord.argtypes = [vp, vp]
+    rt.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+    rt.cudaEventCreateWithFlags.argtypes = [ctypes.POINTER(vp), ctypes.c_uint]
+    rt.cudaEventDestroy.argtypes = [vp]
+    return rt
+
+
 def _packed(tensors):
     """One device byte buffer holding copies of `tensors` (256-byte aligned parts)
     and the views of it that replace them."""
@@ -270,13 +295,6 @@ class GpuStep:
         self.ws = [c.workspace(wl.num_seqs, wl.num_queries, wl.num_q_heads, self.pt.shape[1])
                    for c in self.caches]
         B, NQ, HQ, d = q.shape
-        # the step's inputs (q, new k, new v) and results (out, bound, flags) each
-        # live in one device buffer, so a step moves them with one copy each way
-        self.io_in, (self.qd, self.k_new, self.v_new) = _packed([self.qd, self.k_new, self.v_new])
-        self.io_out, (self.out, self.bound, self.flags) = _packed(
-            [torch.empty((B, NQ, HQ, d), dtype=torch.float32, device="cuda"),
-             torch.empty((B, NQ, HQ), dtype=torch.float32, device="cuda"),
-             torch.empty((B, NQ, HQ), dtype=torch.uint8, device="cuda")])
         # one dedicated stream: the eager steps and the captured graph use it
         self.stream = torch.cuda.Stream()
         s = self.stream.cuda_stream
@@ -284,23 +302,45 @@ class GpuStep:
         self.L = L
         dt = kvq.KVQ_BF16 if self.kd.dtype == torch.bfloat16 else kvq.KVQ_F32
         qdt = kvq.KVQ_BF16 if self.qd.dtype == torch.bfloat16 else kvq.KVQ_F32
-        kn, vn = self.k_new, self.v_new
-        self.append_args = [
-            (ctypes.byref(c.desc), kn.data_ptr(), vn.data_ptr(), dt, kn.stride(0), kn.stride(1),
-             kn.stride(2), wl.num_seqs, 1, None, self.new_pos.data_ptr(), self.pt.data_ptr(),
-             self.pt.shape[1], s) for c in self.caches]
-        self.decode_args = [
-            (ctypes.byref(c.desc), self.qd.data_ptr(), qdt, B, NQ, HQ, self.pt.data_ptr(),
-             self.pt.shape[1], self.sl.data_ptr(), 0.0, wl.tau, self.out.data_ptr(),
-             self.bound.data_ptr(), self.flags.data_ptr(), w.data_ptr(), w.numel(), s)
-            for c, w in zip(self.caches, self.ws)]
-        # the fused step: the new token appended inside the decode launch
-        self.fused_args = [
-            (ctypes.byref(c.desc), kn.data_ptr(), vn.data_ptr(), dt, kn.stride(0), kn.stride(1),
-             self.qd.data_ptr(), qdt, B, NQ, HQ, self.pt.data_ptr(), self.pt.shape[1],
-             self.sl.data_ptr(), 0.0, wl.tau, self.out.data_ptr(), self.bound.data_ptr(),
-             self.flags.data_ptr(), w.data_ptr(), w.numel(), s)
-            for c, w in zip(self.caches, self.ws)]
+        q0, kn0, vn0 = self.qd, self.k_new, self.v_new
+
+        def io_set():
+            """The step's inputs (q, new k, new v) and results (out, bound, flags),
+            each group in one device buffer (one copy each way per step), and the
+            pre-marshalled C-ABI arguments of the step's calls on them."""
+            io_in, (qd, kn, vn) = _packed([q0, kn0, vn0])
+            io_out, (out, bound, flags) = _packed(
+                [torch.empty((B, NQ, HQ, d), dtype=torch.float32, device="cuda"),
+                 torch.empty((B, NQ, HQ), dtype=torch.float32, device="cuda"),
+                 torch.empty((B, NQ, HQ), dtype=torch.uint8, device="cuda")])
+            append_args = [
+                (ctypes.byref(c.desc), kn.data_ptr(), vn.data_ptr(), dt, kn.stride(0),
+                 kn.stride(1), kn.stride(2), wl.num_seqs, 1, None, self.new_pos.data_ptr(),
+                 self.pt.data_ptr(), self.pt.shape[1], s) for c in self.caches]
+            decode_args = [
+                (ctypes.byref(c.desc), qd.data_ptr(), qdt, B, NQ, HQ, self.pt.data_ptr(),
+                 self.pt.shape[1], self.sl.data_ptr(), 0.0, wl.tau, out.data_ptr(),
+                 bound.data_ptr(), flags.data_ptr(), w.data_ptr(), w.numel(), s)
+                for c, w in zip(self.caches, self.ws)]
+            # the fused step: the new token appended inside the decode launch
+            fused_args = [
+                (ctypes.byref(c.desc), kn.data_ptr(), vn.data_ptr(), dt, kn.stride(0),
+                 kn.stride(1), qd.data_ptr(), qdt, B, NQ, HQ, self.pt.data_ptr(),
+                 self.pt.shape[1], self.sl.data_ptr(), 0.0, wl.tau, out.data_ptr(),
+                 bound.data_ptr(), flags.data_ptr(), w.data_ptr(), w.numel(), s)
+                for c, w in zip(self.caches, self.ws)]
+            return dict(io_in=io_in, qd=qd, k_new=kn, v_new=vn, io_out=io_out, out=out,
+                        bound=bound, flags=flags, append_args=append_args,
+                        decode_args=decode_args, fused_args=fused_args)
+
+        # two sets: the end-to-end loop copies one step's inputs and the previous
+        # step's results while the other set's step runs; the timed graph uses set 0
+        self.io = [io_set(), io_set()]
+        io0 = self.io[0]
+        self.io_in, self.qd, self.k_new, self.v_new = io0["io_in"], io0["qd"], io0["k_new"], \
+            io0["v_new"]
+        self.io_out, self.out, self.bound, self.flags = io0["io_out"], io0["out"], \
+            io0["bound"], io0["flags"]
         self.two_calls = two_calls
         self.token_heads = int(sum(inp.seq_lens)) * wl.num_kv_heads
         bb = base.block_bytes
@@ -346,23 +386,24 @@ class GpuStep:
         fb["calls"] += 1
         return n
 
-    def step(self, i, ev=None):
+    def step(self, i, ev=None, io=0):
         r = i % self.replicas
+        st = self.io[io]
         if not self.two_calls:
             if ev is not None:
                 ev[0].record(self.stream)
-            rc = self.L.kvq_decode_attention_append(*self.fused_args[r])
+            rc = self.L.kvq_decode_attention_append(*st["fused_args"][r])
             if rc:
                 raise RuntimeError(self.kvq.last_error())
             if ev is not None:
                 ev[1].record(self.stream)
             return
-        rc = self.L.kvq_quantize_append(*self.append_args[r])
+        rc = self.L.kvq_quantize_append(*st["append_args"][r])
         if rc:
             raise RuntimeError(self.kvq.last_error())
         if ev is not None:
             ev[0].record(self.stream)
-        rc = self.L.kvq_decode_attention(*self.decode_args[r])
+        rc = self.L.kvq_decode_attention(*st["decode_args"][r])
         if rc:
             raise RuntimeError(self.kvq.last_error())
         if ev is not None:
@@ -426,8 +467,8 @@ def run_gpu(args):
     # end to end through the public API with host buffers: H2D of the step's inputs
     # (q and the new K/V token, packed) from pinned memory, the step's call(s), D2H
     # of the results (out, bound, flags, packed)
-    in_h = st.io_in.cpu().pin_memory()
-    out_h = torch.empty(st.io_out.shape, dtype=torch.uint8).pin_memory()
+    in_h = [st.io[k]["io_in"].cpu().pin_memory() for k in (0, 1)]
+    out_h = [torch.empty(st.io_out.shape, dtype=torch.uint8).pin_memory() for _ in (0, 1)]
     h2d = st.qd.numel() * st.qd.element_size() + 2 * st.k_new.numel() * st.k_new.element_size()
     d2h = st.out.numel() * 4 + st.bound.numel() * 4 + st.flags.numel()
     # with a finite tau the step ends with the host-synchronous exact fallback of the
@@ -437,15 +478,65 @@ def run_gpu(args):
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(st.stream):
+    if st.fallback is None:
+        # Pipelined over the two buffer sets: step i's inputs go in on one copy
+        # stream while step i-1 runs, and step i-1's results come back on another
+        # while step i runs.  A set's inputs are overwritten only after the step
+        # that read them ran, and its results only after they were copied out.
+        import ctypes
+        rt = _cudart()
+        H2D, D2H, NO_TIMING = 1, 2, 2
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        sm, si, so = st.stream.cuda_stream, s_in.cuda_stream, s_out.cuda_stream
+        evs = [[ctypes.c_void_p() for _ in (0, 1)] for _ in range(3)]
+        for e in sum(evs, []):
+            if rt.cudaEventCreateWithFlags(ctypes.byref(e), NO_TIMING):
+                raise RuntimeError("cudaEventCreateWithFlags failed")
+        ev_in, ev_ran, ev_out = evs
+        d_in = [st.io[k]["io_in"].data_ptr() for k in (0, 1)]
+        d_out = [st.io[k]["io_out"].data_ptr() for k in (0, 1)]
+        h_in = [t.data_ptr() for t in in_h]
+        h_out = [t.data_ptr() for t in out_h]
+        n_in, n_out = st.io_in.numel(), st.io_out.numel()
+        err = 0
         e0.record(st.stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
         for i in range(e_steps):
-            st.io_in.copy_(in_h, non_blocking=True)
-            st.step(i)
-            if st.fallback is not None:
-                st.fallback_exact(i % st.replicas)
-            out_h.copy_(st.io_out, non_blocking=True)
+            k = i & 1
+            if i >= 2:
+                err |= rt.cudaStreamWaitEvent(si, ev_ran[k], 0)
+            err |= rt.cudaMemcpyAsync(d_in[k], h_in[k], n_in, H2D, si)
+            err |= rt.cudaEventRecord(ev_in[k], si)
+            err |= rt.cudaStreamWaitEvent(sm, ev_in[k], 0)
+            if i >= 2:
+                err |= rt.cudaStreamWaitEvent(sm, ev_out[k], 0)
+            st.step(i, io=k)
+            err |= rt.cudaEventRecord(ev_ran[k], sm)
+            err |= rt.cudaStreamWaitEvent(so, ev_ran[k], 0)
+            err |= rt.cudaMemcpyAsync(h_out[k], d_out[k], n_out, D2H, so)
+            err |= rt.cudaEventRecord(ev_out[k], so)
+        st.stream.wait_stream(s_out)
         e1.record(st.stream)
+        torch.cuda.synchronize()
+        for e in sum(evs, []):
+            rt.cudaEventDestroy(e)
+        if err:
+            raise RuntimeError("a CUDA runtime call of the end-to-end loop failed")
+        # every step computes the same batch: the results read back through either
+        # set are the device results of the timed steps
+        ref = st.io_out.cpu()
+        if not all(torch.equal(t, ref) for t in out_h[:min(2, e_steps)]):
+            raise RuntimeError("end-to-end results differ from the device results")
+    else:
+        with torch.cuda.stream(st.stream):
+            e0.record(st.stream)
+            for i in range(e_steps):
+                st.io_in.copy_(in_h[0], non_blocking=True)
+                st.step(i)
+                st.fallback_exact(i % st.replicas)
+                out_h[0].copy_(st.io_out, non_blocking=True)
+            e1.record(st.stream)
     torch.cuda.synchronize()
     ms_step, dec_ms, e2e_ms = _rank_times(ms_total, dec_ms, e0.elapsed_time(e1) / e_steps,
                                           args.steps, world)
@@ -483,7 +574,11 @@ def run_gpu(args):
                      "timing": ("events around every decode launch" if st.two_calls else
                                 "events around the replay of K back-to-back launches, / K")},
         "e2e": {"value": _job_value(st.token_heads, world, e2e_ms), "unit": UNIT,
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "note": ("each step: H2D of its packed inputs from pinned memory, the step's "
+                         "call, D2H of its packed results; without a fallback the copies of "
+                         "one step overlap the neighbouring steps' kernels (two buffer sets, "
+                         "two copy streams)")},
         "gpu_launches": st.launches_per_step * args.steps,
         "clocks": clocks,
     }
