@@ -166,3 +166,50 @@ def test_full_size_parity(name):
     assert np.array_equal(g["cache"].pool.cpu().numpy(), oc.pool)
     o_hat, bound, flags, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=inp.wl.tau)
     _check_decode(inp, g, o_hat, bound, flags, inp.wl.tau)
+
+
+@pytest.mark.parametrize("name,seed", [("llama8b", 0), ("llama8b", 1), ("long128k", 0)])
+def test_fused_step_full_size(name, seed):
+    """The configuration the benchmark times, at full size: the context up to the
+    last token appended, then one kvq_decode_attention_append launch that encodes
+    the last token of every sequence and decodes.  The pool and eta must equal the
+    oracle's full append bit for bit; every output, bound and flag is checked
+    against the oracle's decode."""
+    from quantized_decode_attention_kvq_b200 import kvq
+    inp = synth.make(name, seed)
+    wl = inp.wl
+    k, v = inp.kv()
+    q = inp.q()
+    kd, vd, qd = to_torch(k), to_torch(v), to_torch(q)
+    pt = torch.from_numpy(inp.page_table).cuda()
+    lens = np.array(inp.seq_lens, np.int32)
+    sl = torch.from_numpy(lens).cuda()
+    before = torch.from_numpy(np.maximum(lens - 1, 0)).cuda()
+    zeros = torch.zeros(wl.num_seqs, dtype=torch.int32, device="cuda")
+    last = torch.from_numpy(np.maximum(lens - 1, 0).astype(np.int64)).cuda()
+    idx = last.view(-1, 1, 1, 1).expand(-1, wl.num_kv_heads, 1, wl.head_dim)
+    k_new = torch.gather(kd, 2, idx).contiguous()
+    v_new = torch.gather(vd, 2, idx).contiguous()
+    c = gpu_cache(inp)
+    c.append(kd, vd, pt, zeros, before)
+    S, NQ, HQ, d = q.shape
+    ws = c.workspace(S, NQ, HQ, pt.shape[1])
+    out = torch.full((S, NQ, HQ, d), float("nan"), dtype=torch.float32, device="cuda")
+    bound = torch.full((S, NQ, HQ), float("nan"), dtype=torch.float32, device="cuda")
+    flags = torch.full((S, NQ, HQ), 7, dtype=torch.uint8, device="cuda")
+    dt = kvq.KVQ_BF16 if kd.dtype == torch.bfloat16 else kvq.KVQ_F32
+    rc = kvq.kvq_decode_attention_append(
+        c.desc, k_new, v_new, dt, k_new.stride(0), k_new.stride(1), qd,
+        kvq.KVQ_BF16 if qd.dtype == torch.bfloat16 else kvq.KVQ_F32, S, NQ, HQ, pt,
+        pt.shape[1], sl, 0.0, wl.tau, out, bound, flags, ws, ws.numel())
+    assert rc == kvq.KVQ_OK, kvq.last_error()
+    torch.cuda.synchronize()
+    assert c.device_error() == 0
+    oc = oracle_pool(inp, k, v)
+    assert np.array_equal(c.pool.cpu().numpy(), oc.pool)
+    assert np.array_equal(c.eta.cpu().numpy().view(np.uint32), oc.eta.view(np.uint32))
+    o_hat, ob, of, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=wl.tau)
+    g = dict(out=out.cpu().numpy().reshape(-1, d).astype(np.float64),
+             bound=bound.cpu().numpy().reshape(-1).astype(np.float64),
+             flags=flags.cpu().numpy().reshape(-1))
+    _check_decode(inp, g, o_hat, ob, of, wl.tau)
