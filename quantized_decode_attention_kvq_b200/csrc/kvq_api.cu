@@ -133,7 +133,7 @@ struct Plan {
   size_t total() const { return counter_bytes + part_bytes; }
 };
 
-constexpr int kMaxPagesPerSplit = 128;
+constexpr int kMaxPagesPerSplit = 256;
 
 // Split-K sizing: fill every SM's resident slots once with (sequence, kv head,
 // split) CTAs; long contexts cap the pages of one split so a ragged batch
