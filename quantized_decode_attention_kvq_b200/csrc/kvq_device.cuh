@@ -86,15 +86,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // ---- bulk copies (global -> shared, completion on an mbarrier) -------------
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
 // L2 policy for data read once: its lines are the first evicted, so a stream of
 // them leaves the small inputs every launch re-reads (context lengths, page
 // table, queries, eta, split records) resident in L2.
@@ -104,7 +95,9 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   return p;
 }
 
-// bulk_g2s with an L2 cache policy (l2_evict_first_policy for streamed data)
+// One bulk copy of `bytes` (16-byte aligned addresses and size) into this
+// CTA's shared memory; its bytes complete the transaction count of `bar`.
+// `policy` is an L2 cache policy (l2_evict_first_policy for streamed data).
 __device__ __forceinline__ void bulk_g2s_hint(void* dst, const void* src, uint32_t bytes,
                                               uint64_t* bar, uint64_t policy) {
   asm volatile(
