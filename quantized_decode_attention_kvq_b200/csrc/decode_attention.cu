@@ -878,9 +878,21 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   const int64_t unit = (int64_t)b * a.hkv + kvh;
   const int splits = gridDim.y;
   float* rec = a.part + (unit * splits + split) * RF;
-  if (r == 0 && lane == 0) {
+  // header: the value range per group and eta at floats 4..(4 + 2 NB), 16-byte
+  // aligned so the merging CTA reads them as whole vectors (the rest is zero)
+  constexpr int HV = (2 * NB + 1 + 3) / 4;   // float4 vectors of the header
+  static_assert(4 + 4 * HV <= kHdr, "the record header holds the range and eta");
+  if (r == 0 && lane < HV) {
+    float hv[4];
 #pragma unroll
-    for (int i = 0; i < 2 * NB + 1; ++i) rec[1 + i] = rg[i];
+    for (int i = 0; i < 4; ++i) {
+      const int idx = 4 * lane + i;
+      hv[i] = 0.f;
+#pragma unroll
+      for (int t = 0; t < 2 * NB + 1; ++t)
+        if (t == idx) hv[i] = rg[t];
+    }
+    reinterpret_cast<float4*>(rec + 4)[lane] = make_float4(hv[0], hv[1], hv[2], hv[3]);
   }
   if (lane == 0) {
     rec[kHdr + r * (8 + D) + 0] = mW;
@@ -937,13 +949,24 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
         const float* st = recs + (int64_t)sp * RF + kHdr + r * (8 + D);
         sa[k] = __ldcg(reinterpret_cast<const float4*>(st));
         sb[k] = __ldcg(reinterpret_cast<const float2*>(st + 4));
-        const float* rp = recs + (int64_t)sp * RF + 1;
+        if (r == 0) {   // the header is the same for every row: warp 0 reads it
+          const float4* rp = reinterpret_cast<const float4*>(recs + (int64_t)sp * RF + 4);
+          float hv[4 * HV];
 #pragma unroll
-        for (int g = 0; g < NB; ++g) {
-          rg[g] = fmaxf(rg[g], __ldcg(rp + g));
-          rg[NB + g] = fminf(rg[NB + g], __ldcg(rp + NB + g));
+          for (int c = 0; c < HV; ++c) {
+            const float4 x = __ldcg(rp + c);
+            hv[4 * c] = x.x;
+            hv[4 * c + 1] = x.y;
+            hv[4 * c + 2] = x.z;
+            hv[4 * c + 3] = x.w;
+          }
+#pragma unroll
+          for (int g = 0; g < NB; ++g) {
+            rg[g] = fmaxf(rg[g], hv[g]);
+            rg[NB + g] = fminf(rg[NB + g], hv[NB + g]);
+          }
+          rg[2 * NB] = fmaxf(rg[2 * NB], hv[2 * NB]);
         }
-        rg[2 * NB] = fmaxf(rg[2 * NB], __ldcg(rp + 2 * NB));
       }
     }
     // the first outputs of the chunk are read together with its statistics
@@ -1021,6 +1044,16 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       rg[NB + g] = fminf(rg[NB + g], __shfl_xor_sync(0xffffffffu, rg[NB + g], off));
     }
     rg[2 * NB] = fmaxf(rg[2 * NB], __shfl_xor_sync(0xffffffffu, rg[2 * NB], off));
+  }
+  {  // warp 0's header merge to every warp (the stage buffers are free by now)
+    float* rgs = reinterpret_cast<float*>(sm + C::OFF_ST);
+    if (r == 0 && lane == 0) {
+#pragma unroll
+      for (int i = 0; i < 2 * NB + 1; ++i) rgs[i] = rg[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 2 * NB + 1; ++i) rg[i] = rgs[i];
   }
   finalize(t5[0], t5[1], t5[2], t5[3], t5[4], rg, o);
   __syncthreads();
