@@ -877,7 +877,13 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   // ---- write this split's record; the last CTA of (b, kvh) merges all --------------
   const int64_t unit = (int64_t)b * a.hkv + kvh;
   const int splits = gridDim.y;
-  float* rec = a.part + (unit * splits + split) * RF;
+  // A unit's records (splits x RF floats) are grouped by kind so the merging CTA
+  // reads each kind with neighbouring lanes on neighbouring addresses: headers
+  // [split][kHdr], row statistics [row][split][8], outputs [split][row][D].
+  float* ubase = a.part + unit * splits * RF;
+  float* rec = ubase + (int64_t)split * kHdr;
+  float* rst = ubase + (int64_t)splits * kHdr + ((int64_t)r * splits + split) * 8;
+  float* rout = ubase + (int64_t)splits * (kHdr + kRows * 8) + ((int64_t)split * kRows + r) * D;
   // header: the value range per group and eta at floats 4..(4 + 2 NB), 16-byte
   // aligned so the merging CTA reads them as whole vectors (the rest is zero)
   constexpr int HV = (2 * NB + 1 + 3) / 4;   // float4 vectors of the header
@@ -895,12 +901,12 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     reinterpret_cast<float4*>(rec + 4)[lane] = make_float4(hv[0], hv[1], hv[2], hv[3]);
   }
   if (lane == 0) {
-    rec[kHdr + r * (8 + D) + 0] = mW;
+    rst[0] = mW;
 #pragma unroll
-    for (int t = 0; t < 5; ++t) rec[kHdr + r * (8 + D) + 1 + t] = st5[t];
+    for (int t = 0; t < 5; ++t) rst[1 + t] = st5[t];
   }
 #pragma unroll
-  for (int e = 0; e < CPL; ++e) rec[kHdr + r * (8 + D) + 8 + lane * CPL + e] = o[e];
+  for (int e = 0; e < CPL; ++e) rout[lane * CPL + e] = o[e];
   // The barrier orders every thread's record stores before thread 0's ticket;
   // the ticket's release publishes them at GPU scope and, for the last CTA,
   // its acquire makes every other CTA's records visible to the whole CTA
@@ -934,8 +940,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 #pragma unroll
   for (int e = 0; e < CPL; ++e) o[e] = 0.f;
   auto out_of = [&](int sp) -> const VT* {
-    return reinterpret_cast<const VT*>(recs + (int64_t)sp * RF + kHdr + r * (8 + D) + 8 +
-                                       lane * CPL);
+    return reinterpret_cast<const VT*>(recs + (int64_t)splits * (kHdr + kRows * 8) +
+                                       ((int64_t)sp * kRows + r) * D + lane * CPL);
   };
   for (int c0 = 0; c0 < active; c0 += 32 * KS) {
     float4 sa[KS];  // (m, l, A, B) of split c0 + 32k + lane
@@ -946,11 +952,11 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       sa[k] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
       sb[k] = make_float2(0.f, 0.f);
       if (sp < active) {
-        const float* st = recs + (int64_t)sp * RF + kHdr + r * (8 + D);
+        const float* st = recs + (int64_t)splits * kHdr + ((int64_t)r * splits + sp) * 8;
         sa[k] = __ldcg(reinterpret_cast<const float4*>(st));
         sb[k] = __ldcg(reinterpret_cast<const float2*>(st + 4));
         if (r == 0) {   // the header is the same for every row: warp 0 reads it
-          const float4* rp = reinterpret_cast<const float4*>(recs + (int64_t)sp * RF + 4);
+          const float4* rp = reinterpret_cast<const float4*>(recs + (int64_t)sp * kHdr + 4);
           float hv[4 * HV];
 #pragma unroll
           for (int c = 0; c < HV; ++c) {
