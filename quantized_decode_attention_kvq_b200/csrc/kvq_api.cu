@@ -408,9 +408,8 @@ int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const vo
       !staging || !num_fallback)
     return fail(KVQ_ERR_INVALID_ARG, "NULL argument");
   if (orig_seq_stride < 0 || orig_head_stride < 0) return fail(KVQ_ERR_INVALID_ARG, "negative stride");
-  DeviceInfo di;
-  int rc = device_info(&di, nullptr);
-  if (rc) return rc;
+  if (reinterpret_cast<uintptr_t>(staging) % 16)
+    return fail(KVQ_ERR_INVALID_ARG, "staging is not 16-byte aligned");
   const int D = cache->head_dim, hkv = cache->num_kv_heads, G = num_q_heads / hkv;
   const size_t es = orig_dtype == KVQ_BF16 ? 2 : 4;
   int32_t max_n = 0;
@@ -421,12 +420,13 @@ int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const vo
   if (staging_bytes < kvq_fallback_staging_size(cache, orig_dtype, max_n))
     return fail(KVQ_ERR_INVALID_ARG, "staging %zu bytes < %zu required", staging_bytes,
                 kvq_fallback_staging_size(cache, orig_dtype, max_n));
+  DeviceInfo di;
+  int rc = device_info(&di, nullptr);
+  if (rc) return rc;
   cudaStream_t ms = reinterpret_cast<cudaStream_t>(main_stream);
   cudaStream_t ss = reinterpret_cast<cudaStream_t>(side_stream);
   const size_t rows = (size_t)num_seqs * num_queries * num_q_heads;
 
-  if (reinterpret_cast<uintptr_t>(staging) % 16)
-    return fail(KVQ_ERR_INVALID_ARG, "staging is not 16-byte aligned");
   // the decode, the flags on the host, the copies of the open batch, and the
   // last recompute that read each staging half
   cudaEvent_t ev[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};

@@ -6,6 +6,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -118,3 +119,22 @@ def test_fallback_validation_and_staging_size(kvq):
     rc, n = kvq.kvq_fallback_exact(d, 0x1, 0x1, 9, 0, 0, 0x10, kvq.KVQ_BF16, 1, 1, 32, 0x1,
                                    0.0, 0x20, 0x30, 0x40, 0x50, 1 << 20, 0, 0, 100)
     assert rc == kvq.KVQ_ERR_INVALID_ARG
+
+
+def test_fallback_staging_checks_come_before_any_device_call(kvq):
+    # (no GPU here: each call must fail on its arguments, not on the device)
+    d = _desc(kvq)
+    sl = np.array([10, 20], np.int32)
+    need = kvq.kvq_fallback_staging_size(d, kvq.KVQ_BF16, 20)
+
+    def call(lens, staging, nbytes):
+        return kvq.kvq_fallback_exact(d, 0x100, 0x100, kvq.KVQ_BF16, 0, 0, 0x100, kvq.KVQ_BF16,
+                                      2, 1, 32, lens.ctypes.data, 0.0, 0x100, 0x100, 0x100,
+                                      staging, nbytes, 0, 0, 100)
+
+    rc, n = call(sl, 0x108, need)
+    assert rc == kvq.KVQ_ERR_INVALID_ARG and n == 0 and "aligned" in kvq.last_error()
+    rc, n = call(sl, 0x100, need - 1)
+    assert rc == kvq.KVQ_ERR_INVALID_ARG and "required" in kvq.last_error()
+    rc, n = call(np.array([10, -1], np.int32), 0x100, need)
+    assert rc == kvq.KVQ_ERR_INVALID_ARG and "seq_len" in kvq.last_error()
