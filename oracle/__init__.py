@@ -57,7 +57,7 @@ def lib() -> ctypes.CDLL:
         L.oc_f16_round.argtypes = [ctypes.c_float, ctypes.c_int]
         L.oc_block_bytes.restype = ctypes.c_int64
         for name in ("oc_quantize_sym", "oc_quantize_asym", "oc_append", "oc_decode",
-                     "oc_dense", "oc_f16_round_n"):
+                     "oc_decode_promote_values", "oc_dense", "oc_f16_round_n"):
             getattr(L, name).restype = ctypes.c_int
     return _lib
 
@@ -182,6 +182,39 @@ class Cache:
             raise ValueError(f"oracle decode failed: {rc}")
         return out, bound, flags, diag
 
+
+    def decode_promote_values(self, q, page_table, seq_lens, v_orig, v_tol, scale=None,
+                              tau=math.inf, row_mask=None):
+        """Decode with rung 2 of the fallback ladder: blocks whose estimated share of
+        E_val (mass x eta) exceeds v_tol take the original values v_orig
+        [num_seqs][Hkv][T][d] (fp32, or bf16 bits as uint16).  Returns
+        (o f64 [rows][d], bound f64 [rows], flags u8 [rows], promoted blocks i32
+        [rows], diag [rows][8] with E_val of the blocks not promoted)."""
+        q = np.ascontiguousarray(q)
+        v_orig = np.ascontiguousarray(v_orig)
+        B, NQ, HQ, d = q.shape
+        _, H, T, dv = v_orig.shape
+        assert dv == d and H == self.cfg.hkv
+        rows = B * NQ * HQ
+        scale = default_scale(d) if scale is None else np.float32(scale)
+        out = np.zeros((rows, d), dtype=np.float64)
+        bound = np.zeros(rows, dtype=np.float64)
+        flags = np.zeros(rows, dtype=np.uint8)
+        promoted = np.zeros(rows, dtype=np.int32)
+        diag = np.zeros((rows, 8), dtype=np.float64)
+        pt = _c(page_table, np.int32)
+        sl = _c(seq_lens, np.int32)
+        rm = None if row_mask is None else _c(row_mask, np.uint8)
+        rc = lib().oc_decode_promote_values(
+            ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(q),
+            int(q.dtype == np.float32), B, NQ, HQ, _p(pt), pt.shape[1], _p(sl),
+            ctypes.c_float(scale), ctypes.c_float(tau), _p(self.signs), _p(v_orig),
+            int(v_orig.dtype == np.float32), ctypes.c_int64(H * T * d), ctypes.c_int64(T * d),
+            ctypes.c_int64(d), ctypes.c_double(v_tol), _p(out), _p(bound), _p(flags),
+            _p(promoted), _p(diag), _p(rm))
+        if rc != OK:
+            raise ValueError(f"oracle promoted decode failed: {rc}")
+        return out, bound, flags, promoted, diag
 
     def decode_terms(self, q, page_table, n, b, i, h, scale=None):
         """Per-token (z_hat, Delta) of one query row over the first n tokens."""

@@ -595,6 +595,114 @@ int oc_decode_terms(const oc_cfg* c, const uint8_t* pool, const float* eta, cons
   return OC_OK;
 }
 
+/* Value promotion: rung 2 of the fallback ladder ("Runtime-Certified
+ * Bounded-Error Quantized Attention", Methodology 3: page in full-precision
+ * values for the blocks whose estimated value-error contribution exceeds a
+ * threshold).  A block is one page of one kv head.  Per query row, with z^,
+ * p^, Delta, E_key as in oc_decode:
+ *   M_b    = sum_{j in b} p^_j          (the block's estimated attention mass)
+ *   c_b    = M_b * eta_b                (its share of E_val)
+ *   promoted blocks: c_b > v_tol
+ *   o'     = sum_j p^_j v~_j,  v~_j = the original v_j in a promoted block,
+ *                              else v^_j
+ *   E_val' = sum of c_b over the blocks not promoted
+ *   bound' = kappa * (E_key + E_val');  flag' = bound' > tau.
+ * E_key is unchanged: a promoted value lies within eta_b of its code's value,
+ * which the 2 * max eta of E_key's range term already covers.
+ * v_orig element (b, h, t, ch) at b*seq_stride + h*head_stride + t*tok_stride
+ * + ch (fp32, or bf16 bits when v_is_f32 is 0).  promoted (optional) gets per
+ * row the number of promoted blocks; diag as in oc_decode, with E_val'. */
+int oc_decode_promote_values(const oc_cfg* c, const uint8_t* pool, const float* eta,
+                             const void* q, int q_is_f32, int num_seqs, int nq, int hq,
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             float scale, float tau, const int8_t* sigma, const void* v_orig,
+                             int v_is_f32, int64_t seq_stride, int64_t head_stride,
+                             int64_t tok_stride, double v_tol, double* out, double* bound,
+                             uint8_t* flags, int32_t* promoted, double* diag,
+                             const uint8_t* row_mask) {
+  if (!oc_cfg_ok(c) || hq % c->hkv || (c->krotate && !sigma) || !v_orig) return OC_ERR_ARG;
+  int d = c->d, G = hq / c->hkv;
+  int64_t bb = oc_block_bytes(c);
+  double sc = (double)scale;
+  for (int b = 0; b < num_seqs; ++b) {
+    int n = seq_lens[b];
+    int npg = (n + OC_PAGE - 1) / OC_PAGE;
+    double* z = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* dl = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* et = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* mass = npg ? (double*)malloc(sizeof(double) * npg) : NULL;
+    uint8_t* prom = npg ? (uint8_t*)malloc(npg) : NULL;
+    for (int i = 0; i < nq; ++i)
+      for (int h = 0; h < hq; ++h) {
+        int64_t row = ((int64_t)b * nq + i) * hq + h;
+        if (row_mask && !row_mask[row]) continue;
+        int kv = h / G;
+        double* o = out + row * d;
+        for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+        if (n == 0) {
+          bound[row] = 0.0;
+          flags[row] = 0;
+          if (promoted) promoted[row] = 0;
+          if (diag) for (int t = 0; t < 8; ++t) diag[row * 8 + t] = 0.0;
+          continue;
+        }
+        float qf[128], qr[128], vf[128];
+        const float* qp = oc_row_query(c, q, q_is_f32, row, sigma, qf, qr);
+        double range, eta_max;
+        oc_row_terms(c, pool, eta, qp, b, kv, n, page_table, max_pages, sc, z, dl, et, &range,
+                     &eta_max);
+        double m = -INFINITY;
+        for (int j = 0; j < n; ++j) if (z[j] > m) m = z[j];
+        double l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        for (int lp = 0; lp < npg; ++lp) mass[lp] = 0.0;
+        for (int j = 0; j < n; ++j) mass[j / OC_PAGE] += exp(z[j] - m) / l;
+        int np_ = 0;
+        for (int lp = 0; lp < npg; ++lp) {
+          prom[lp] = mass[lp] * et[lp * OC_PAGE] > v_tol ? 1 : 0;
+          np_ += prom[lp];
+        }
+        double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
+        double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+        for (int j = 0; j < n; ++j) {
+          double p = exp(z[j] - m) / l;
+          if (prom[j / OC_PAGE]) {
+            oc_load_vec(v_orig, v_is_f32, b * seq_stride + kv * head_stride + j * tok_stride, d,
+                        vf);
+            for (int ch = 0; ch < d; ++ch) o[ch] += p * (double)vf[ch];
+          } else {
+            int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
+            const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+            oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+            for (int ch = 0; ch < d; ++ch) o[ch] += p * vhat[ch];
+            Ev += p * et[j];
+          }
+          A += p * expm1(dl[j]);
+          B += p * exp(-dl[j]);
+          if (dl[j] > dmax) dmax = dl[j];
+        }
+        double tv = tanh(dmax / 2.0);
+        if (A / B < tv) tv = A / B;
+        double ekey = tv * (range + 2.0 * eta_max);
+        double bd = OC_KAPPA * (ekey + Ev);
+        bound[row] = bd;
+        flags[row] = bd > (double)tau ? 1 : 0;
+        if (promoted) promoted[row] = np_;
+        if (diag) {
+          double* dg = diag + row * 8;
+          dg[0] = tv; dg[1] = ekey; dg[2] = Ev; dg[3] = dmax;
+          dg[4] = A; dg[5] = B; dg[6] = range; dg[7] = eta_max;
+        }
+      }
+    free(z);
+    free(dl);
+    free(et);
+    free(mass);
+    free(prom);
+  }
+  return OC_OK;
+}
+
 /* Exact dense attention on the originals (the fallback's ground truth):
  * o = softmax(scale * q . k_j) v, fp64, no quantization, no rotation.
  * k, v element (b, h, t, ch) at b*seq_stride + h*head_stride + t*tok_stride + ch. */
