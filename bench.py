@@ -64,9 +64,11 @@ def _peaks():
     return 6650.0, "fallback"
 
 
-def _traffic_record():
+def _traffic_record(workload: str, two_calls: bool):
     """dram bytes per decode launch from the committed ncu summary, if it was taken
-    on the current kernel source."""
+    on the current kernel source, for this workload and launch (the fused step)."""
+    if workload != "llama8b" or two_calls:
+        return None
     p = os.path.join(ROOT, "profiles", "decode_attention_llama8b_traffic.md")
     if not os.path.exists(p):
         return None
@@ -543,7 +545,7 @@ def run_gpu(args):
 
     peak, peak_kind = _peaks()
     achieved = st.decode_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = _traffic_record()
+    traffic = _traffic_record(args.workload, st.two_calls)
     res = {
         "metric": METRIC,
         "value": _job_value(st.token_heads, world, ms_step),
