@@ -31,6 +31,12 @@
  *   - Calls on distinct streams with distinct output/workspace buffers are
  *     independent.  Only devices of compute capability 10.0 (sm_100a) run
  *     the kernels.
+ *   - The decode entry points launch with programmatic stream serialization:
+ *     their CTAs may start while the previous kernel in the stream is
+ *     finishing, but before griddepcontrol.wait they only set up shared
+ *     memory and prefetch cache pages into L2 (which changes no memory), so
+ *     every result is the same as after a plain stream-ordered launch,
+ *     whatever that kernel writes.
  *
  * Quantized cache layout (one block per physical page and kv head, 16 tokens;
  * nb = head_dim/32):
