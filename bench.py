@@ -650,6 +650,28 @@ def _oracle_worker(job):
     return _oracle_decode_loop(*job)
 
 
+def _oracle_codec_and_dense(workload: str, seed: int):
+    """Single-thread rates of the oracle's other two stages on sequence 0 of the
+    workload, all kv heads: the codec (append of every token) and the exact
+    dense attention the fallback computes (every query row), in KV
+    token-heads/s."""
+    import oracle
+    inp = synth.make(workload, seed)
+    wl = inp.wl
+    c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
+                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+    k, v = inp.kv_seq(0)
+    sl = np.array(inp.seq_lens[:1], np.int32)
+    th = int(sl[0]) * wl.num_kv_heads
+    t0 = time.perf_counter()
+    rc = c.append(k[None], v[None], inp.page_table[:1], np.zeros(1, np.int32), valid=sl)
+    t1 = time.perf_counter()
+    assert rc == 0
+    oracle.dense(inp.q()[:1], k[None], v[None], sl)
+    t2 = time.perf_counter()
+    return th / (t1 - t0), th / (t2 - t1)
+
+
 def cpu_baseline(workload: str, seed: int, seconds: float):
     """The oracle's decode (fp64 attention + bound over the quantized cache) on whole
     sequences of the workload: one process per kv head of sequence 0 on the host's
@@ -662,9 +684,11 @@ def cpu_baseline(workload: str, seed: int, seconds: float):
         res = pool.map(_oracle_worker, [(workload, seed, [h], seconds) for h in range(n)])
     value = sum(r[0] for r in res) / max(r[1] for r in res)
     th1, el1, reps1 = _oracle_decode_loop(workload, seed, None, seconds)
+    codec, dense = _oracle_codec_and_dense(workload, seed)
     inp = synth.make(workload, seed)
     return {"value": value, "unit": UNIT, "cores": n, "kind": "oracle",
             "single_core_value": th1 / el1,
+            "single_core_codec_value": codec, "single_core_dense_value": dense,
             "sample": f"sequence 0 of {wl.name} ({int(inp.seq_lens[0])} tokens x "
                       f"{wl.num_q_heads // wl.num_kv_heads} q heads per kv head), decode + "
                       f"bound: {n} processes, one kv head each, about {seconds:.0f} s each; "

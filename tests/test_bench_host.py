@@ -28,4 +28,5 @@ def test_cpu_baseline_reports_its_sample():
     assert r["kind"] == "oracle" and r["unit"] == bench.UNIT
     assert r["cores"] == 1                       # one kv head: one process
     assert r["value"] > 0 and r["single_core_value"] > 0
+    assert r["single_core_codec_value"] > 0 and r["single_core_dense_value"] > 0
     assert "tiny" in r["sample"]
