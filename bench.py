@@ -42,6 +42,7 @@ METRIC = ("quantized-KV decode attention: KV tokens·heads/s and achieved HBM GB
           "vs peak")
 UNIT = "KV token-heads/s"
 L2_BYTES = 126 * 2 ** 20
+SPEC_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (context for frac_vs_spec)
 DECODE_SRC = os.path.join(ROOT, "quantized_decode_attention_kvq_b200", "csrc",
                           "decode_attention.cu")
 
@@ -64,26 +65,25 @@ def _peaks():
     return 6650.0, "fallback"
 
 
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "decode_attention_traffic.json")
+
+
 def _traffic_record(workload: str, two_calls: bool):
-    """dram bytes per decode launch from the committed ncu summary, if it was taken
-    on the current kernel source, for this workload and launch (the fused step)."""
-    if workload != "llama8b" or two_calls:
-        return None
-    p = os.path.join(ROOT, "profiles", "decode_attention_llama8b_traffic.md")
-    if not os.path.exists(p):
+    """DRAM bytes per decode launch from the committed ncu record
+    (profiles/decode_attention_traffic.json) for this workload and the fused
+    step's launch, if it was taken on the current decode kernel source."""
+    if two_calls or not os.path.exists(TRAFFIC_JSON):
         return None
     src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
-    rec = {}
-    for line in open(p):
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            rec[k.strip()] = v.strip()
-    if rec.get("decode_source_sha256_16") != src_hash:
-        return None
-    try:
-        return float(rec["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
-        return None
+    with open(TRAFFIC_JSON) as f:
+        recs = json.load(f).get("records", [])
+    for r in recs:
+        if r.get("workload") == workload and r.get("decode_source_sha256_16") == src_hash:
+            try:
+                return float(r["dram_bytes_per_launch"])
+            except (KeyError, TypeError, ValueError):
+                return None
+    return None
 
 
 def _smi_time(stamp: str):
@@ -412,17 +412,15 @@ class GpuStep:
             ev[1].record(self.stream)
 
 
-def run_gpu(args):
+def _timed_replay(st, args, world, rank, local):
+    """W eager warm-up steps, the K timed steps captured into one CUDA graph,
+    untimed replays of that graph (the first pays the graph's upload; the
+    rest, about 0.2 s of them, put the GPU under the load the clocks are
+    sampled in), then the timed replay between two events.  Returns (device
+    ms of the K steps, mean decode-launch ms, clocks)."""
     import torch
-    rank, world, local = _dist_setup(args.gpus)
-    wl = synth.WORKLOADS[args.workload]
-    reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl))))
-    reps = min(reps, 8)
-    st = GpuStep(args.workload, args.seed, reps, two_calls=args.two_calls)
-    # setup: one untimed call per cache replica (library-side descriptors and
-    # occupancy are cached by the first call), then the W warm-up steps
     with torch.cuda.stream(st.stream):
-        for r in range(reps):
+        for r in range(st.replicas):      # setup: library descriptors and occupancy
             st.step(r)
         for i in range(args.warmup):
             st.step(i)
@@ -430,11 +428,10 @@ def run_gpu(args):
     err = st.caches[0].device_error()
     if err:
         raise RuntimeError(f"device error {err} during warm-up")
-    # the K timed steps are captured into one CUDA graph; the timed region is its
-    # replay.  The default step is one launch, so the graph holds those launches
-    # alone and a launch's duration is the region's time / K (an event pair
-    # around every launch would add its own nodes to each step).  With
-    # --two-calls, events around every decode launch separate it from the append.
+    # The default step is one launch, so the graph holds those launches alone and
+    # a launch's duration is the region's time / K (an event pair around every
+    # launch would add its own nodes to each step).  With --two-calls, events
+    # around every decode launch separate it from the append.
     evs = [(torch.cuda.Event(enable_timing=True, external=True),
             torch.cuda.Event(enable_timing=True, external=True)) for _ in range(args.steps)] \
         if st.two_calls else [None] * args.steps
@@ -445,6 +442,14 @@ def run_gpu(args):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(st.stream):
+        t0.record(st.stream)
+        graph.replay()                    # untimed: uploads the graph
+        t1.record(st.stream)
+    torch.cuda.synchronize()
+    one = max(1e-3, t0.elapsed_time(t1))
+    pre = max(1, min(2000, int(200.0 / one)))
+    pre = int(_max_over_ranks(float(pre), world))     # the same count on every rank
     sampler = ClockSampler(local) if rank == 0 else None
     _barrier(world)
     torch.cuda.synchronize()
@@ -453,22 +458,34 @@ def run_gpu(args):
         time.sleep(0.3)
     w0 = time.time()
     with torch.cuda.stream(st.stream):
+        for _ in range(pre):
+            graph.replay()
         t0.record(st.stream)
         graph.replay()
         t1.record(st.stream)
     torch.cuda.synchronize()
     w1 = time.time()
     clocks = sampler.stop((w0, w1)) if sampler else None
-    if clocks is None and sampler:
-        clocks = {"sm_mhz": None, "note": "timed region shorter than the 20 ms sampling period"}
+    if clocks is not None:
+        clocks["window"] = (f"{pre} untimed replays of the same graph directly before the "
+                            f"timed one, and the timed one")
+    elif sampler:
+        clocks = {"sm_mhz": None, "note": "no nvidia-smi sample inside the window"}
     _barrier(world)
     ms_total = t0.elapsed_time(t1)
     dec_ms = (float(np.mean([a.elapsed_time(b) for a, b in evs])) if st.two_calls
               else ms_total / max(1, args.steps))
+    del graph
+    return ms_total, dec_ms, clocks
 
-    # end to end through the public API with host buffers: H2D of the step's inputs
-    # (q and the new K/V token, packed) from pinned memory, the step's call(s), D2H
-    # of the results (out, bound, flags, packed)
+
+def _e2e(st, args, world):
+    """The same steps end to end through the C ABI with host buffers: per step the
+    H2D of its packed inputs (q and the new K/V token) from pinned memory, the
+    step's call(s), the D2H of its packed results (out, bound, flags); with a
+    finite tau, also the host-synchronous exact fallback of the flagged rows.
+    Returns (ms per step, h2d bytes per step, d2h bytes per step)."""
+    import torch
     in_h = [st.io[k]["io_in"].cpu().pin_memory() for k in (0, 1)]
     out_h = [torch.empty(st.io_out.shape, dtype=torch.uint8).pin_memory() for _ in (0, 1)]
     h2d = st.qd.numel() * st.qd.element_size() + 2 * st.k_new.numel() * st.k_new.element_size()
@@ -540,38 +557,40 @@ def run_gpu(args):
                 out_h[0].copy_(st.io_out, non_blocking=True)
             e1.record(st.stream)
     torch.cuda.synchronize()
-    ms_step, dec_ms, e2e_ms = _rank_times(ms_total, dec_ms, e0.elapsed_time(e1) / e_steps,
-                                          args.steps, world)
+    return e0.elapsed_time(e1) / e_steps, h2d, d2h
 
+
+def measure_workload(name, args, world, rank, local):
+    """One workload's measurement on this rank: the device-timed value and the
+    decode kernel's roofline, the clocks, and the end-to-end number."""
+    import torch
+    wl = synth.WORKLOADS[name]
+    reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl))))
+    reps = min(reps, 8)
+    st = GpuStep(name, args.seed, reps, two_calls=args.two_calls)
+    ms_total, dec_ms, clocks = _timed_replay(st, args, world, rank, local)
+    e2e_ms, h2d, d2h = _e2e(st, args, world)
+    ms_step, dec_ms, e2e_ms = _rank_times(ms_total, dec_ms, e2e_ms, args.steps, world)
     peak, peak_kind = _peaks()
     achieved = st.decode_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = _traffic_record(args.workload, st.two_calls)
-    res = {
-        "metric": METRIC,
+    rec = {
         "value": _job_value(st.token_heads, world, ms_step),
         "unit": UNIT,
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": ms_step,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "s8xs8->s32 (QK), f16xf16->f32 (PV), f32 softmax/bound",
-        "data": "synthetic (seeded N(0,1) bf16 + outlier channels, as the workload states)",
+        "steps": args.steps,
         "config": {"workload": _workload_desc(wl),
                    "l2": f"inputs larger than L2: {reps} cache replicas of "
                          f"{st.cache_bytes / 1e6:.1f} MB rotated per step",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "step": ("kvq_quantize_append + kvq_decode_attention" if st.two_calls else
                             "kvq_decode_attention_append (append fused into the decode)"),
                    "token_heads_per_step": st.token_heads,
                    "decode_bytes_per_launch": st.decode_bytes},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
+                     "frac": achieved / peak, "traffic": _traffic_record(name, st.two_calls),
                      "peak_kind": f"{peak_kind} copy bandwidth",
-                     "kernel": "decode_mma_kernel" + ("" if st.two_calls else
-                                                       " (append fused)"),
+                     "frac_vs_spec": achieved / SPEC_HBM_GBS,
+                     "spec_peak": SPEC_HBM_GBS,
+                     "kernel": "decode_mma_kernel" + ("" if st.two_calls else " (append fused)"),
                      "kernel_ms": dec_ms,
                      "timing": ("events around every decode launch" if st.two_calls else
                                 "events around the replay of K back-to-back launches, / K")},
@@ -587,13 +606,47 @@ def run_gpu(args):
     if st.fallback is not None:
         fb = st.fallback
         rows_per_step = fb["rows"] / max(1, fb["calls"])
-        res["fallback"] = {
-            "tau": wl.tau, "rate": rows_per_step / st.out.shape[0] / st.out.shape[1] /
-            st.out.shape[2], "rows_per_step": rows_per_step,
-            "h2d_bytes_per_step": fb["h2d"] / max(1, fb["calls"]),
+        rows = st.out.shape[0] * st.out.shape[1] * st.out.shape[2]
+        rec["fallback"] = {
+            "tau": wl.tau, "rate": rows_per_step / rows, "rows_per_step": rows_per_step,
+            "rows": rows, "h2d_bytes_per_step": fb["h2d"] / max(1, fb["calls"]),
             "note": "value times append + decode (graph); e2e adds the exact fallback of the "
                     "flagged rows (H2D of their originals + fp32 attention)"}
-        res["e2e"]["h2d_bytes_per_step"] = int(h2d + fb["h2d"] / max(1, fb["calls"]))
+        rec["e2e"]["h2d_bytes_per_step"] = int(h2d + fb["h2d"] / max(1, fb["calls"]))
+    del st
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_gpu(args):
+    rank, world, local = _dist_setup(args.gpus)
+    main = measure_workload(args.workload, args, world, rank, local)
+    also = [w for w in args.also.split(",") if w and w != "none" and w != args.workload]
+    subs = {w: measure_workload(w, args, world, rank, local) for w in also}
+    res = {
+        "metric": METRIC,
+        "value": main["value"],
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": main["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "s8xs8->s32 (QK), f16xf16->f32 (PV), f32 softmax/bound",
+        "data": "synthetic (seeded N(0,1) bf16 + outlier channels, as the workload states)",
+        "config": dict(main["config"],
+                       parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+        "roofline": main["roofline"],
+        "e2e": main["e2e"],
+        "gpu_launches": main["gpu_launches"],
+        "clocks": main["clocks"],
+    }
+    if "fallback" in main:
+        res["fallback"] = main["fallback"]
+    if subs:
+        res["workloads"] = subs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(args.workload, args.seed, args.cpu_seconds)
     if world > 1:
@@ -745,12 +798,17 @@ def main():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--also", default=None,
+                    help="comma-separated workloads measured in the same run and reported "
+                         "under 'workloads' (default: long128k,serving with llama8b; 'none')")
     ap.add_argument("--two-calls", action="store_true",
                     help="step = kvq_quantize_append + kvq_decode_attention (default: the fused "
                          "kvq_decode_attention_append)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.also is None:
+        args.also = "long128k,serving" if args.workload == "llama8b" else "none"
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -82,7 +82,9 @@ typedef enum {
   KVQ_ERR_RANGE = -3,       /* non-finite input or fp16-overflowing scale/zero */
   KVQ_ERR_CUDA = -4,        /* a CUDA runtime call failed */
   KVQ_ERR_TIMEOUT = -5,     /* a bounded host wait gave up */
-  KVQ_ERR_DEVICE = -6       /* a kernel reported an error (see kvq_device_error) */
+  KVQ_ERR_DEVICE = -6       /* reserved; no call returns it.  Kernels report their errors
+                               (KVQ_ERR_INVALID_ARG, KVQ_ERR_RANGE, KVQ_ERR_TIMEOUT) in
+                               the cache's error word, read by kvq_device_error */
 } kvq_status;
 
 typedef enum { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
@@ -147,9 +149,15 @@ KVQ_API size_t kvq_workspace_size(const kvq_cache* cache, int32_t num_seqs, int3
  * upper bound on max_c |o_exact - out| against exact attention over the
  * originals) and flags uint8 (bound > tau; tau = INFINITY never flags).
  * An empty context gives out = 0, bound = 0, flag = 0.  page_table and
- * seq_lens: device int32.  Page indices outside the pool set
- * *error_word = KVQ_ERR_INVALID_ARG and that page is skipped.  workspace:
- * device, >= kvq_workspace_size() bytes, 16-byte aligned.  Asynchronous. */
+ * seq_lens: device int32.  A page that cannot be read leaves its (sequence,
+ * kv head) without a certified bound: a page index outside the pool (never
+ * copied; *error_word = KVQ_ERR_INVALID_ARG), a bounded wait for a page copy
+ * that ran out (KVQ_ERR_TIMEOUT) or seq_lens[s] > 16*max_pages_per_seq (the
+ * context is cut to the page table; KVQ_ERR_INVALID_ARG).  Every query row of
+ * that (sequence, kv head) then gets bound = +INFINITY and flag = 1 whatever
+ * tau is, so kvq_fallback_exact recomputes it; out holds attention over the
+ * pages that were read.  workspace: device, >= kvq_workspace_size() bytes,
+ * 16-byte aligned.  Asynchronous. */
 KVQ_API int kvq_decode_attention(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
                          int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
                          int32_t max_pages_per_seq, const int32_t* seq_lens,
@@ -216,7 +224,12 @@ KVQ_API size_t kvq_fallback_staging_size(const kvq_cache* cache, int orig_dtype,
  * a staging half that is being reused wait (on `side`) for the recompute
  * that read it before.  *num_fallback (host) = number of recomputed
  * queries.  On any error out is left unmodified for the rows not yet
- * recomputed.  Blocks the calling thread until the flags are on the host. */
+ * recomputed.  Blocks the calling thread until the flags are on the host.
+ * After an error return (KVQ_ERR_TIMEOUT included) copies and kernels this
+ * call queued may still be pending on main_stream and side_stream: the flag
+ * read-back into flags_host, page-ins into staging and recomputes into out.
+ * Synchronize both streams (or order later work after them) before reusing
+ * flags_host, staging or out. */
 KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const void* v_orig_host,
                        int orig_dtype, int64_t orig_seq_stride, int64_t orig_head_stride,
                        const void* q, int q_dtype, int32_t num_seqs, int32_t num_queries,
@@ -239,8 +252,11 @@ KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, 
  * return KVQ_ERR_UNSUPPORTED.  The call allocates no device memory (no
  * cudaMalloc, cudaFree or any allocating CUDA or framework routine); it clears
  * the scratch's counters with cudaMemsetAsync on `stream` before the decode.
- * The first call on a device looks up the array's device address with that
- * device current, so make that first call before any stream capture.  Every
+ * Each call made outside a stream capture looks up the array's device address
+ * on the current device (so a device reset, which may move it, is followed);
+ * a call while `stream` is capturing uses the address the last uncaptured call
+ * on that device found, so make one call on the device before any capture
+ * (without one, the captured call returns KVQ_ERR_INVALID_ARG).  Every
  * call shares the one array: calls that may overlap on the GPU (on different
  * streams, or from several threads) race on it and must be serialized by the
  * caller.  Asynchronous on `stream`. */

@@ -15,6 +15,7 @@ magnitude against the pages is unpinned: the pages print no worked bound.
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -46,20 +47,53 @@ def build(force: bool = False) -> str:
 _lib: Optional[ctypes.CDLL] = None
 
 
+def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
+    L.oc_f16_value.restype = ctypes.c_double
+    L.oc_f16_value.argtypes = [ctypes.c_uint16]
+    L.oc_f16_round.restype = ctypes.c_uint16
+    L.oc_f16_round.argtypes = [ctypes.c_float, ctypes.c_int]
+    L.oc_block_bytes.restype = ctypes.c_int64
+    for name in ("oc_quantize_sym", "oc_quantize_asym", "oc_append", "oc_decode",
+                 "oc_decode_promote_values", "oc_dense", "oc_f16_round_n"):
+        getattr(L, name).restype = ctypes.c_int
+    return L
+
+
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
-        L = _lib
-        L.oc_f16_value.restype = ctypes.c_double
-        L.oc_f16_value.argtypes = [ctypes.c_uint16]
-        L.oc_f16_round.restype = ctypes.c_uint16
-        L.oc_f16_round.argtypes = [ctypes.c_float, ctypes.c_int]
-        L.oc_block_bytes.restype = ctypes.c_int64
-        for name in ("oc_quantize_sym", "oc_quantize_asym", "oc_append", "oc_decode",
-                     "oc_decode_promote_values", "oc_dense", "oc_f16_round_n"):
-            getattr(L, name).restype = ctypes.c_int
+        _lib = _configure(ctypes.CDLL(build()))
     return _lib
+
+
+@contextlib.contextmanager
+def library_override(path: str):
+    """Route every oracle call through another build of kvq_oracle.c while the
+    block runs.  Test hook only: the tests that plant a mistake in a copy of
+    the oracle use it to check that the pins catch that mistake."""
+    global _lib
+    saved = lib()
+    _lib = _configure(ctypes.CDLL(os.path.abspath(path)))
+    try:
+        yield _lib
+    finally:
+        _lib = saved
+
+
+def compile_variant(src_text: str, out_dir: str, name: str) -> str:
+    """Compile C source text with the oracle's flags into out_dir/name.so."""
+    src = os.path.join(out_dir, name + ".c")
+    with open(src, "w") as f:
+        f.write(src_text)
+    so = os.path.join(out_dir, name + ".so")
+    subprocess.check_call(["gcc", *CFLAGS, "-o", so, src, "-lm"])
+    return so
+
+
+def source_text() -> str:
+    """The oracle's C source (for the planted-mistake tests)."""
+    with open(_SRC) as f:
+        return f.read()
 
 
 class OcCfg(ctypes.Structure):

@@ -223,7 +223,10 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   }
 
   if (n < 0) n = 0;
-  if (n > a.max_pages * kPage) {
+  // A context longer than the page table is cut to it; the pages past the cut
+  // are never read, so the unit's results are marked uncertified (below).
+  const bool clamped = n > a.max_pages * kPage;
+  if (clamped) {
     if (tid == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
     n = a.max_pages * kPage;
   }
@@ -435,7 +438,11 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
 #pragma unroll
   for (int e = 0; e < 4; ++e) zmv[e] = 0.f;
   constexpr int EPL = NB / 2;  // V metadata entries converted per lane and page
-  float vhi[EPL], vlo[EPL], etamax = 0.f;
+  // etamax = +inf marks a unit with a page that was not read (an index outside
+  // the pool, a wait that ran out, a context cut to the page table): every
+  // merge below takes maxima, so the mark reaches the finish, which then
+  // reports bound = +inf and flag = 1 instead of a bound over the pages read.
+  float vhi[EPL], vlo[EPL], etamax = clamped ? INFINITY : 0.f;
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     vhi[i] = -INFINITY;
@@ -493,6 +500,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     const bool ok = mbar_wait(&bar[st], par);
     if (!__all_sync(0xffffffffu, ok)) {
       if (lane == 0) set_error(a.err, KVQ_ERR_TIMEOUT);
+      etamax = INFINITY;
       return false;
     }
     const int page = spage[st];
@@ -713,6 +721,8 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
         mma_f16(opv[2 * g + 1], r01 & 0x00F000F0u, r01s & 0x00F000F0u, r23 & 0x00F000F0u,
                 r23s & 0x00F000F0u, b01, b23);
       }
+    } else {
+      etamax = INFINITY;   // the page was not read
     }
     __syncwarp();
     if (j + S < nloc) issue(j + S, st);
@@ -856,8 +866,10 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       for (int e = 0; e < CPL; ++e) a.out[row * D + lane * CPL + e] = ov[e] * inv_l;
     }
     if (lane == 0) {
-      float bd = 0.f;
-      if (l > 0.f) {
+      // a page of the unit was not read: no certified bound
+      const bool skipped = rgv[2 * NB] == INFINITY;
+      float bd = skipped ? INFINITY : 0.f;
+      if (!skipped && l > 0.f) {
         float range = 0.f;
 #pragma unroll
         for (int g = 0; g < NB; ++g) range = fmaxf(range, rgv[g] - rgv[NB + g]);
@@ -865,7 +877,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
         bd = kKappa * (tv * (range + 2.0f * rgv[2 * NB]) + E / l);
       }
       a.bound[row] = bd;
-      a.flags[row] = bd > a.tau ? 1 : 0;
+      a.flags[row] = skipped || bd > a.tau ? 1 : 0;
     }
   };
 

@@ -611,21 +611,30 @@ namespace {
 __device__ __align__(256) uint8_t g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
-// array's name is only a stand-in, so the address is looked up once per device
-// (with that device current) and cached.
-int noalloc_scratch(void** out) {
+// array's name is only a stand-in, so the address is looked up with that device
+// current.  It is looked up again on every call made outside a stream capture
+// (a device reset reloads the module, and the array may move); while `stream`
+// is capturing, the runtime cannot be asked, so the address cached by the last
+// call outside a capture on this device is used.
+int noalloc_scratch(cudaStream_t stream, void** out) {
   static std::mutex mu;
   static void* addr[256] = {nullptr};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 256) return fail(KVQ_ERR_UNSUPPORTED, "device index %d", dev);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if ((e = cudaStreamIsCapturing(stream, &cap)) != cudaSuccess)
+    return cuda_fail(e, "cudaStreamIsCapturing");
   std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
     addr[dev] = p;
+  } else if (!addr[dev]) {
+    return fail(KVQ_ERR_INVALID_ARG, "the first kvq_decode_attention_noalloc call on device %d "
+                "must come before any stream capture", dev);
   }
   *out = addr[dev];
   return KVQ_OK;
@@ -652,9 +661,9 @@ int kvq_decode_attention_noalloc(const kvq_cache* cache, const void* q, int q_dt
     return fail(KVQ_ERR_UNSUPPORTED, "this shape needs %zu bytes of split-K scratch; the "
                 "static scratch of kvq_decode_attention_noalloc holds %d bytes",
                 need, KVQ_NOALLOC_SCRATCH_BYTES);
-  void* scratch = nullptr;
-  if ((rc = noalloc_scratch(&scratch))) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(s, &scratch))) return rc;
   // the per-(sequence, kv head) counters at the front of the scratch must start
   // at zero whatever an earlier call left there
   const size_t counters = ((size_t)num_seqs * cache->num_kv_heads * sizeof(int) + 255) / 256 * 256;

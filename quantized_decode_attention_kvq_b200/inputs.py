@@ -38,6 +38,8 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from typing import Dict, List, Optional
 
 import numpy as np
@@ -106,9 +108,11 @@ def _rng(seed: int, cfg: str, stream: int, index: int = 0) -> np.random.Generato
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 to the nearest bf16 (ties to even); returns uint16 bits."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    r = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    """Round finite fp32 to the nearest bf16 (ties to even); returns uint16 bits.
+    (For a finite value the 32-bit sum below cannot wrap: the largest finite
+    pattern 0xFF7FFFFF plus 0x8000 stays under 2^32.)"""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return r.astype(np.uint16)
 
 
@@ -191,10 +195,11 @@ class Inputs:
                               dtype=np.float32)
         return self._cast(x)
 
-    def kv_seq(self, b: int, ctx_stride: Optional[int] = None):
+    def kv_seq(self, b: int, ctx_stride: Optional[int] = None, out=None):
         """(k, v) of sequence b as [Hkv][ctx_stride][d] (bf16 bits or fp32).
 
-        Tokens at positions >= seq_lens[b] are zero."""
+        Tokens at positions >= seq_lens[b] are zero.  With `out` = (k, v)
+        arrays of that shape, they are filled in place and returned."""
         wl = self.wl
         n = self.seq_lens[b]
         T = ctx_stride if ctx_stride is not None else n
@@ -216,23 +221,37 @@ class Inputs:
                     sg = np.where(gs.integers(0, 2, size=nt) == 1, 1.0, -1.0)
                     arr[h, toks, ch] = (sg * wl.spike_value).astype(np.float32)
         kc, vc = self._cast(k), self._cast(v)
-        if T == n:
-            return kc, vc
-        ko = np.zeros((wl.num_kv_heads, T, wl.head_dim), dtype=kc.dtype)
-        vo = np.zeros_like(ko)
+        if out is None:
+            if T == n:
+                return kc, vc
+            out = (np.zeros((wl.num_kv_heads, T, wl.head_dim), dtype=kc.dtype),
+                   np.zeros((wl.num_kv_heads, T, wl.head_dim), dtype=kc.dtype))
+        ko, vo = out
         ko[:, :n] = kc
         vo[:, :n] = vc
+        ko[:, n:] = 0
+        vo[:, n:] = 0
         return ko, vo
 
-    def kv(self, ctx_stride: Optional[int] = None):
-        """(k, v) of all sequences as [num_seqs][Hkv][ctx_stride][d]."""
+    def kv(self, ctx_stride: Optional[int] = None, threads: Optional[int] = None):
+        """(k, v) of all sequences as [num_seqs][Hkv][ctx_stride][d].
+
+        Sequences are drawn from their own streams, so they are filled in
+        parallel threads (numpy releases the interpreter lock while it fills
+        large arrays) with values independent of the thread count."""
+        wl = self.wl
         T = ctx_stride if ctx_stride is not None else max(self.seq_lens)
-        ks, vs = [], []
-        for b in range(self.wl.num_seqs):
-            k, v = self.kv_seq(b, T)
-            ks.append(k)
-            vs.append(v)
-        return np.stack(ks), np.stack(vs)
+        dt = np.float32 if wl.dtype == "fp32" else np.uint16
+        shape = (wl.num_seqs, wl.num_kv_heads, T, wl.head_dim)
+        k, v = np.empty(shape, dtype=dt), np.empty(shape, dtype=dt)
+        n = threads or min(wl.num_seqs, os.cpu_count() or 1, 16)
+        if n <= 1:
+            for b in range(wl.num_seqs):
+                self.kv_seq(b, T, out=(k[b], v[b]))
+        else:
+            with ThreadPoolExecutor(max_workers=n) as ex:
+                list(ex.map(lambda b: self.kv_seq(b, T, out=(k[b], v[b])), range(wl.num_seqs)))
+        return k, v
 
     def as_f32(self, x: np.ndarray) -> np.ndarray:
         return x if x.dtype == np.float32 else bf16_bits_to_f32(x)

@@ -213,3 +213,45 @@ def test_fused_step_full_size(name, seed):
              bound=bound.cpu().numpy().reshape(-1).astype(np.float64),
              flags=flags.cpu().numpy().reshape(-1))
     _check_decode(inp, g, o_hat, ob, of, wl.tau)
+
+
+@pytest.mark.parametrize("pages_per_split", [None, "64"])
+def test_unread_page_leaves_no_certified_bound(monkeypatch, pages_per_split):
+    """A page index outside the pool is never copied: the error word is set and
+    every row of that (sequence, kv head) gets bound = +inf and flag = 1, even
+    with tau = inf, so the exact fallback recomputes it.  A context longer than
+    the page table does the same.  Other units are untouched."""
+    from quantized_decode_attention_kvq_b200 import kvq
+    if pages_per_split:
+        monkeypatch.setenv("KVQ_PAGES_PER_SPLIT", pages_per_split)
+    inp = small("llama8b", 0)
+    wl = inp.wl
+    g = run_gpu(inp)
+    assert g["err"] == 0
+    G = wl.num_q_heads // wl.num_kv_heads
+    # sequence 1, logical page 5 -> an index one past the pool (kv head 0 and 1)
+    pt = inp.page_table.copy()
+    pt[1, 5] = inp.num_pages
+    ptd = torch.from_numpy(pt).cuda()
+    ws = g["cache"].workspace(wl.num_seqs, wl.num_queries, wl.num_q_heads, pt.shape[1])
+    out, bound, flags = g["cache"].decode(g["q"], ptd, g["sl"], ws, tau=math.inf)
+    torch.cuda.synchronize()
+    assert g["cache"].device_error() == kvq.KVQ_ERR_INVALID_ARG
+    b = bound.cpu().numpy().reshape(wl.num_seqs, -1)
+    f = flags.cpu().numpy().reshape(wl.num_seqs, -1)
+    assert np.isinf(b[1]).all() and (f[1] == 1).all()
+    ref_b = g["bound"].reshape(wl.num_seqs, -1)
+    assert np.array_equal(b[0], ref_b[0].astype(np.float32)) and (f[0] == 0).all()
+    ref_o = g["out"].reshape(wl.num_seqs, -1)
+    assert np.array_equal(out.cpu().numpy().reshape(wl.num_seqs, -1)[0], ref_o[0].astype(np.float32))
+    # a context longer than the page table: sequence 0 is cut, marked uncertified
+    sl = g["sl"].clone()
+    sl[0] = pt.shape[1] * 16 + 1
+    out, bound, flags = g["cache"].decode(g["q"], g["pt"], sl, ws, tau=math.inf)
+    torch.cuda.synchronize()
+    assert g["cache"].device_error() == kvq.KVQ_ERR_INVALID_ARG
+    b = bound.cpu().numpy().reshape(wl.num_seqs, -1)
+    f = flags.cpu().numpy().reshape(wl.num_seqs, -1)
+    assert np.isinf(b[0]).all() and (f[0] == 1).all()
+    assert np.isfinite(b[1]).all() and (f[1] == 0).all()
+    assert G == 4

@@ -20,21 +20,42 @@ from oracle_cases import small
 pytestmark = pytest.mark.gpu
 
 
-def _noalloc(g, inp, tau):
+def _buffers(inp):
+    wl = inp.wl
+    S, NQ, HQ, d = wl.num_seqs, wl.num_queries, wl.num_q_heads, wl.head_dim
+    return (torch.empty((S, NQ, HQ, d), dtype=torch.float32, device="cuda"),
+            torch.empty((S, NQ, HQ), dtype=torch.float32, device="cuda"),
+            torch.empty((S, NQ, HQ), dtype=torch.uint8, device="cuda"))
+
+
+def _noalloc(g, inp, tau, bufs, stream=None):
+    """One call into caller-owned buffers (poisoned first); no torch allocation
+    happens between the poisoning and the read-back."""
     from quantized_decode_attention_kvq_b200 import kvq
     wl = inp.wl
     S, NQ, HQ, d = wl.num_seqs, wl.num_queries, wl.num_q_heads, wl.head_dim
-    out = torch.full((S, NQ, HQ, d), float("nan"), dtype=torch.float32, device="cuda")
-    bound = torch.full((S, NQ, HQ), float("nan"), dtype=torch.float32, device="cuda")
-    flags = torch.full((S, NQ, HQ), 7, dtype=torch.uint8, device="cuda")
-    q = g["q"]
-    rc = kvq.kvq_decode_attention_noalloc(
-        g["cache"].desc, q, kvq.KVQ_BF16 if q.dtype == torch.bfloat16 else kvq.KVQ_F32, S, NQ,
-        HQ, g["pt"], g["pt"].shape[1], g["sl"], 0.0, tau, out, bound, flags)
+    out, bound, flags = bufs
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        out.fill_(float("nan"))
+        bound.fill_(float("nan"))
+        flags.fill_(7)
+        q = g["q"]
+        rc = kvq.kvq_decode_attention_noalloc(
+            g["cache"].desc, q, kvq.KVQ_BF16 if q.dtype == torch.bfloat16 else kvq.KVQ_F32, S,
+            NQ, HQ, g["pt"], g["pt"].shape[1], g["sl"], 0.0, tau, out, bound, flags, s)
     assert rc == kvq.KVQ_OK, kvq.last_error()
     torch.cuda.synchronize()
     return (out.cpu().numpy().reshape(-1, d).astype(np.float64),
             bound.cpu().numpy().reshape(-1).astype(np.float64), flags.cpu().numpy().reshape(-1))
+
+
+def _check(res, g):
+    out, bound, flags = res
+    emax, rel = compare_outputs(out, g["out"])
+    assert emax <= TOL_MAXABS and rel <= TOL_RELL2, (emax, rel)
+    assert (np.abs(bound - g["bound"]) <= TOL_BOUND_REL * g["bound"]).all()
+    assert np.array_equal(flags, g["flags"])
 
 
 @pytest.mark.parametrize("name,tau", [("llama8b", 5.0), ("serving", math.inf)])
@@ -43,13 +64,30 @@ def test_noalloc_matches_workspace_entry_point(name, tau):
         pytest.fail("the GPU tests need a CUDA device")
     inp = small(name, 3)
     g = run_gpu(inp, tau=tau)                       # kvq_decode_attention with a workspace
+    bufs = _buffers(inp)
     for _ in range(2):                              # two calls in a row share the scratch
-        out, bound, flags = _noalloc(g, inp, tau)
-        emax, rel = compare_outputs(out, g["out"])
-        assert emax <= TOL_MAXABS and rel <= TOL_RELL2, (emax, rel)
-        assert (np.abs(bound - g["bound"]) <= TOL_BOUND_REL * g["bound"]).all()
-        assert np.array_equal(flags, g["flags"])
+        _check(_noalloc(g, inp, tau, bufs), g)
     assert g["cache"].device_error() == 0
+
+
+def test_noalloc_allocates_nothing_and_runs_on_any_stream():
+    """After a first call (which may load the library's device code), further
+    calls leave the device's free memory unchanged, on the default stream and on
+    a stream of the caller's."""
+    if not torch.cuda.is_available():
+        pytest.fail("the GPU tests need a CUDA device")
+    inp = small("llama8b", 5)
+    g = run_gpu(inp, tau=5.0)
+    bufs = _buffers(inp)
+    side = torch.cuda.Stream()
+    _check(_noalloc(g, inp, 5.0, bufs), g)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    _check(_noalloc(g, inp, 5.0, bufs), g)
+    _check(_noalloc(g, inp, 5.0, bufs, stream=side), g)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
