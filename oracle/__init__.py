@@ -250,6 +250,46 @@ class Cache:
             raise ValueError(f"oracle promoted decode failed: {rc}")
         return out, bound, flags, promoted, diag
 
+    def decode_adaptive(self, q, page_table, seq_lens, k_orig, v_orig, tau_cov, v_tol=math.inf,
+                        rank_tol=0.0, scale=None, tau=math.inf, row_mask=None):
+        """Adaptive precision ("Runtime-Certified...", Methodology 3): per row the
+        top-K* blocks covering tau_cov of the estimated mass take the original
+        keys, blocks whose new mass x eta exceeds v_tol take the original values,
+        and the ranking-consistency check over the key-promoted blocks (log-mass
+        slack rank_tol) flags the row when it fails.  k_orig, v_orig
+        [num_seqs][Hkv][T][d] (fp32, or bf16 bits as uint16).  Returns a dict:
+        out f64 [rows][d], bound, flags, kprom/vprom u8 [rows][max_pages], nkey,
+        nval, rank_fail per row, diag [rows][8]."""
+        q = np.ascontiguousarray(q)
+        k_orig = np.ascontiguousarray(k_orig)
+        v_orig = np.ascontiguousarray(v_orig)
+        assert k_orig.shape == v_orig.shape and k_orig.dtype == v_orig.dtype
+        B, NQ, HQ, d = q.shape
+        _, H, T, dv = v_orig.shape
+        assert dv == d and H == self.cfg.hkv
+        rows = B * NQ * HQ
+        pt = _c(page_table, np.int32)
+        mp = pt.shape[1]
+        scale = default_scale(d) if scale is None else np.float32(scale)
+        r = dict(out=np.zeros((rows, d)), bound=np.zeros(rows), flags=np.zeros(rows, np.uint8),
+                 kprom=np.zeros((rows, mp), np.uint8), vprom=np.zeros((rows, mp), np.uint8),
+                 nkey=np.zeros(rows, np.int32), nval=np.zeros(rows, np.int32),
+                 rank_fail=np.zeros(rows, np.uint8), diag=np.zeros((rows, 8)))
+        sl = _c(seq_lens, np.int32)
+        rm = None if row_mask is None else _c(row_mask, np.uint8)
+        rc = lib().oc_decode_adaptive(
+            ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(q),
+            int(q.dtype == np.float32), B, NQ, HQ, _p(pt), mp, _p(sl), ctypes.c_float(scale),
+            ctypes.c_float(tau), _p(self.signs), _p(k_orig), _p(v_orig),
+            int(v_orig.dtype == np.float32), ctypes.c_int64(H * T * d), ctypes.c_int64(T * d),
+            ctypes.c_int64(d), ctypes.c_double(tau_cov), ctypes.c_double(v_tol),
+            ctypes.c_double(rank_tol), _p(r["out"]), _p(r["bound"]), _p(r["flags"]),
+            _p(r["kprom"]), _p(r["vprom"]), _p(r["nkey"]), _p(r["nval"]), _p(r["rank_fail"]),
+            _p(r["diag"]), _p(rm))
+        if rc != OK:
+            raise ValueError(f"oracle adaptive decode failed: {rc}")
+        return r
+
     def decode_terms(self, q, page_table, n, b, i, h, scale=None):
         """Per-token (z_hat, Delta) of one query row over the first n tokens."""
         q = np.ascontiguousarray(q)

@@ -754,3 +754,191 @@ void oc_certified_output(const double* ohat, const double* odense, const uint8_t
     for (int ch = 0; ch < d; ++ch)
       out[r * d + ch] = flags[r] ? odense[r * d + ch] : ohat[r * d + ch];
 }
+
+/* ------------------------------------------------------------------------ */
+/* Adaptive precision and the first rungs of the fallback ladder             */
+/* ("Runtime-Certified Bounded-Error Quantized Attention", Methodology 3:    */
+/* adaptive top-K* block selection from a light scoring pass with the       */
+/* quantized keys, promotion of those blocks to full-precision keys, the    */
+/* ranking-consistency check, and value promotion).  A block is one page of */
+/* one kv head.  Per query row (sequence b, query i, q head h; kv head      */
+/* h / (Hq/Hkv)), with z^, p^, Delta as in oc_decode:                       */
+/*   M^_b   = sum_{j in b} p^_j     (estimated mass of the block)             */
+/*   order  = blocks by M^_b descending, ties by lower block index            */
+/*   K*     = the smallest k whose first k blocks in that order have mass     */
+/*            >= tau_cov (every block if none does); they are key-promoted    */
+/*   z~_j   = scale * q . k_j from the originals (q unrotated) in a          */
+/*            key-promoted block, else z^_j                                   */
+/*   Delta~ = kappa * scale * 2^-16 * |q|_2 * |k_j|_2 in a key-promoted block */
+/*            (allowance for an fp32 dot product of the originals), else      */
+/*            Delta_j                                                         */
+/*   p~     = softmax(z~),  M~_b = sum_{j in b} p~_j                          */
+/*   value-promoted blocks: M~_b * eta_b > v_tol (rung 2 on the new masses)   */
+/*   o~     = sum_j p~_j v~_j, v~_j = the original v_j in a value-promoted    */
+/*            block, else v^_j                                                */
+/*   A = sum p~ (e^Delta~ - 1), B = sum p~ e^-Delta~, TV = min(tanh(max      */
+/*   Delta~ / 2), A/B); E_key = TV (range + 2 max eta) with range and eta as */
+/*   in oc_decode; E_val = sum of p~_j eta_{block(j)} over the blocks whose   */
+/*   values are not promoted; bound = kappa (E_key + E_val)                   */
+/*   ranking check: L_b = log sum_{j in b} e^{z~_j} over the key-promoted     */
+/*   blocks in their selection order; the ranking is inconsistent when a     */
+/*   later block's L exceeds an earlier block's L by more than rank_tol       */
+/*   flag   = inconsistent || bound > tau.                                    */
+/* kprom, vprom (optional): [rows][max_pages] 1 for a promoted block;        */
+/* nkey, nval, rank_fail (optional): per row.  row_mask as in oc_decode.     */
+/* k_orig / v_orig element (b, h, t, ch) at b*seq_stride + h*head_stride +   */
+/* t*tok_stride + ch (fp32, or bf16 bits when kv_is_f32 is 0).               */
+/* ------------------------------------------------------------------------ */
+typedef struct { double m; int b; } oc_blk;
+
+static int oc_blk_cmp(const void* x, const void* y) {
+  const oc_blk* a = (const oc_blk*)x;
+  const oc_blk* b = (const oc_blk*)y;
+  if (a->m > b->m) return -1;
+  if (a->m < b->m) return 1;
+  return (a->b > b->b) - (a->b < b->b);
+}
+
+int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, const void* q,
+                       int q_is_f32, int num_seqs, int nq, int hq, const int32_t* page_table,
+                       int max_pages, const int32_t* seq_lens, float scale, float tau,
+                       const int8_t* sigma, const void* k_orig, const void* v_orig,
+                       int kv_is_f32, int64_t seq_stride, int64_t head_stride,
+                       int64_t tok_stride, double tau_cov, double v_tol, double rank_tol,
+                       double* out, double* bound, uint8_t* flags, uint8_t* kprom,
+                       uint8_t* vprom, int32_t* nkey, int32_t* nval, uint8_t* rank_fail,
+                       double* diag, const uint8_t* row_mask) {
+  if (!oc_cfg_ok(c) || hq % c->hkv || (c->krotate && !sigma) || !k_orig || !v_orig)
+    return OC_ERR_ARG;
+  int d = c->d, G = hq / c->hkv;
+  int64_t bb = oc_block_bytes(c);
+  double sc = (double)scale;
+  for (int b = 0; b < num_seqs; ++b) {
+    int n = seq_lens[b];
+    int npg = (n + OC_PAGE - 1) / OC_PAGE;
+    double* z = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* dl = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* et = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* p = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    oc_blk* ord = npg ? (oc_blk*)malloc(sizeof(oc_blk) * npg) : NULL;
+    uint8_t* kp = npg ? (uint8_t*)malloc(npg) : NULL;
+    uint8_t* vp = npg ? (uint8_t*)malloc(npg) : NULL;
+    double* mass = npg ? (double*)malloc(sizeof(double) * npg) : NULL;
+    for (int i = 0; i < nq; ++i)
+      for (int h = 0; h < hq; ++h) {
+        int64_t row = ((int64_t)b * nq + i) * hq + h;
+        if (row_mask && !row_mask[row]) continue;
+        int kv = h / G;
+        double* o = out + row * d;
+        for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+        if (kprom) memset(kprom + row * max_pages, 0, max_pages);
+        if (vprom) memset(vprom + row * max_pages, 0, max_pages);
+        if (nkey) nkey[row] = 0;
+        if (nval) nval[row] = 0;
+        if (rank_fail) rank_fail[row] = 0;
+        if (n == 0) {
+          bound[row] = 0.0;
+          flags[row] = 0;
+          if (diag) for (int t = 0; t < 8; ++t) diag[row * 8 + t] = 0.0;
+          continue;
+        }
+        float qf[128], qr[128], kf[128], vf[128];
+        const float* qp = oc_row_query(c, q, q_is_f32, row, sigma, qf, qr);
+        double range, eta_max;
+        oc_row_terms(c, pool, eta, qp, b, kv, n, page_table, max_pages, sc, z, dl, et, &range,
+                     &eta_max);
+        /* scoring pass: estimated block masses under the quantized softmax */
+        double m = -INFINITY;
+        for (int j = 0; j < n; ++j) if (z[j] > m) m = z[j];
+        double l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        for (int lp = 0; lp < npg; ++lp) { ord[lp].m = 0.0; ord[lp].b = lp; }
+        for (int j = 0; j < n; ++j) ord[j / OC_PAGE].m += exp(z[j] - m) / l;
+        /* top-K* blocks covering tau_cov of the estimated mass */
+        qsort(ord, npg, sizeof(oc_blk), oc_blk_cmp);
+        int kstar = 0;
+        double cum = 0.0;
+        while (kstar < npg && cum < tau_cov) cum += ord[kstar++].m;
+        for (int lp = 0; lp < npg; ++lp) kp[lp] = 0;
+        for (int k = 0; k < kstar; ++k) kp[ord[k].b] = 1;
+        /* mixed scores: originals in the key-promoted blocks */
+        double qn2 = 0.0;
+        for (int ch = 0; ch < d; ++ch) qn2 += (double)qf[ch] * (double)qf[ch];
+        qn2 = sqrt(qn2);
+        for (int j = 0; j < n; ++j) {
+          if (!kp[j / OC_PAGE]) continue;
+          oc_load_vec(k_orig, kv_is_f32, b * seq_stride + kv * head_stride + j * tok_stride, d,
+                      kf);
+          double dot = 0.0, kn2 = 0.0;
+          for (int ch = 0; ch < d; ++ch) {
+            dot += (double)qf[ch] * (double)kf[ch];
+            kn2 += (double)kf[ch] * (double)kf[ch];
+          }
+          z[j] = sc * dot;
+          dl[j] = OC_KAPPA * sc * OC_ROT_SLACK * qn2 * sqrt(kn2);
+        }
+        m = -INFINITY;
+        for (int j = 0; j < n; ++j) if (z[j] > m) m = z[j];
+        l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        for (int j = 0; j < n; ++j) p[j] = exp(z[j] - m) / l;
+        /* value promotion on the new masses */
+        for (int lp = 0; lp < npg; ++lp) mass[lp] = 0.0;
+        for (int j = 0; j < n; ++j) mass[j / OC_PAGE] += p[j];
+        int nv = 0;
+        for (int lp = 0; lp < npg; ++lp) {
+          vp[lp] = mass[lp] * et[lp * OC_PAGE] > v_tol ? 1 : 0;
+          nv += vp[lp];
+        }
+        /* output and bound */
+        double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
+        double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+        for (int j = 0; j < n; ++j) {
+          if (vp[j / OC_PAGE]) {
+            oc_load_vec(v_orig, kv_is_f32, b * seq_stride + kv * head_stride + j * tok_stride,
+                        d, vf);
+            for (int ch = 0; ch < d; ++ch) o[ch] += p[j] * (double)vf[ch];
+          } else {
+            int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
+            const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+            oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+            for (int ch = 0; ch < d; ++ch) o[ch] += p[j] * vhat[ch];
+            Ev += p[j] * et[j];
+          }
+          A += p[j] * expm1(dl[j]);
+          B += p[j] * exp(-dl[j]);
+          if (dl[j] > dmax) dmax = dl[j];
+        }
+        double tv = tanh(dmax / 2.0);
+        if (A / B < tv) tv = A / B;
+        double ekey = tv * (range + 2.0 * eta_max);
+        double bd = OC_KAPPA * (ekey + Ev);
+        /* ranking check over the key-promoted blocks, in selection order */
+        int fail = 0;
+        double lmin = INFINITY;
+        for (int k = 0; k < kstar; ++k) {
+          int lp = ord[k].b;
+          int j0 = lp * OC_PAGE, j1 = j0 + OC_PAGE < n ? j0 + OC_PAGE : n;
+          double s = 0.0;
+          for (int j = j0; j < j1; ++j) s += exp(z[j] - m);
+          double L = log(s) + m;
+          if (L - lmin > rank_tol) fail = 1;
+          if (L < lmin) lmin = L;
+        }
+        bound[row] = bd;
+        flags[row] = (fail || bd > (double)tau) ? 1 : 0;
+        if (kprom) for (int lp = 0; lp < npg; ++lp) kprom[row * max_pages + lp] = kp[lp];
+        if (vprom) for (int lp = 0; lp < npg; ++lp) vprom[row * max_pages + lp] = vp[lp];
+        if (nkey) nkey[row] = kstar;
+        if (nval) nval[row] = nv;
+        if (rank_fail) rank_fail[row] = (uint8_t)fail;
+        if (diag) {
+          double* dg = diag + row * 8;
+          dg[0] = tv; dg[1] = ekey; dg[2] = Ev; dg[3] = dmax;
+          dg[4] = A; dg[5] = B; dg[6] = range; dg[7] = eta_max;
+        }
+      }
+    free(z); free(dl); free(et); free(p); free(ord); free(kp); free(vp); free(mass);
+  }
+  return OC_OK;
+}
