@@ -238,6 +238,70 @@ KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, 
                        size_t staging_bytes, kvq_stream_t main_stream,
                        kvq_stream_t side_stream, int32_t timeout_ms, int32_t* num_fallback);
 
+/* Adaptive precision and the first rungs of the fallback ladder ("Runtime-
+ * Certified Bounded-Error Quantized Attention", Methodology 3: adaptive top-K*
+ * selection from a light scoring pass with the quantized keys, the
+ * ranking-consistency check, rung 2 value promotion), for the rows a decode
+ * flagged.  A block is one 16-token page of one kv head.  Per flagged query
+ * row (sequence, query, q head; kv head h / (num_q_heads/num_kv_heads)):
+ *   M^_b  = the block's mass under the softmax of the quantized scores
+ *   keys  : the blocks in order of M^_b (descending; ties by lower page) up
+ *           to the fewest whose mass reaches tau_cov (none if tau_cov <= 0)
+ *           take the original keys: exact scores s*q.k (q unrotated) with
+ *           Delta_j = kappa*s*2^-16*|q|_2*|k_j|_2 (an allowance for the fp32
+ *           dot product) instead of the quantized Delta_j
+ *   values: blocks with M^_b * eta_b > v_tol take the original values and
+ *           leave E_val
+ *   out, bound: attention and the certified bound of kvq_decode_attention
+ *           recomputed with these scores, Delta and values
+ *   ranking check: along the key-promoted blocks in order of M^_b, a block
+ *           whose exact log-mass log sum_{j in b} e^{z_j} exceeds an earlier
+ *           block's by more than rank_tol makes the ranking inconsistent
+ *   flag  = inconsistent || bound > tau (|| a page could not be read)
+ * Waits on `main_stream` for the decode that wrote `flags`, reads them into
+ * flags_host (pinned, num_seqs*num_queries*num_q_heads bytes) on
+ * `side_stream` with a deadline of timeout_ms for the whole call
+ * (KVQ_ERR_TIMEOUT when it passes), scores and selects on `main_stream`,
+ * reads back the union of promoted blocks per (sequence, kv head), copies
+ * only those blocks' originals (k_orig_host, v_orig_host: pinned, layout as
+ * for kvq_fallback_exact) into `staging` with cudaMemcpyAsync on
+ * `side_stream`, and recomputes the flagged rows on `main_stream`,
+ * overwriting their out, bound and flags (device, as written by the decode);
+ * rows not flagged are left as they are.  promoted_keys / promoted_values
+ * (device, [rows][max_pages_per_seq] uint8, or NULL) get the flagged rows'
+ * promotion maps.  work: device, >= kvq_adaptive_work_size() bytes; host_work:
+ * pinned, >= kvq_adaptive_host_size() bytes; staging: device, at least
+ * kvq_adaptive_staging_size() bytes (the promoted blocks of one (sequence, kv
+ * head)); all 16-byte aligned.  max_pages_per_seq <= 8192.  On return
+ * *num_rows = the rows that ran through the ladder and *num_flagged = the
+ * rows flagged afterwards (flags_host holds the new flags); `main_stream` is
+ * ordered after all of this call's work.  After an error return, queued work
+ * may still be pending on both streams (synchronize them before reusing the
+ * buffers).  KVQ_FAULT=memcpy makes the page-in fail (KVQ_ERR_CUDA) for
+ * tests.  Blocks the calling thread on the bounded waits. */
+KVQ_API size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs,
+                                      int32_t num_queries, int32_t num_q_heads,
+                                      int32_t max_pages_per_seq);
+KVQ_API size_t kvq_adaptive_host_size(const kvq_cache* cache, int32_t num_seqs,
+                                      int32_t max_pages_per_seq);
+KVQ_API size_t kvq_adaptive_staging_size(const kvq_cache* cache, int orig_dtype,
+                                         int32_t max_pages_per_seq);
+KVQ_API int kvq_adaptive_precision(const kvq_cache* cache, const void* k_orig_host,
+                                   const void* v_orig_host, int orig_dtype,
+                                   int64_t orig_seq_stride, int64_t orig_head_stride,
+                                   const void* q, int q_dtype, int32_t num_seqs,
+                                   int32_t num_queries, int32_t num_q_heads,
+                                   const int32_t* page_table, int32_t max_pages_per_seq,
+                                   const int32_t* seq_lens, const int32_t* seq_lens_host,
+                                   float softmax_scale, float tau, float tau_cov, float v_tol,
+                                   float rank_tol, uint8_t* flags, uint8_t* flags_host,
+                                   float* out, float* bound, uint8_t* promoted_keys,
+                                   uint8_t* promoted_values, void* work, size_t work_bytes,
+                                   void* host_work, size_t host_work_bytes, void* staging,
+                                   size_t staging_bytes, kvq_stream_t main_stream,
+                                   kvq_stream_t side_stream, int32_t timeout_ms,
+                                   int32_t* num_rows, int32_t* num_flagged);
+
 /* Size of the static device scratch of kvq_decode_attention_noalloc. */
 #define KVQ_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
 

@@ -254,7 +254,7 @@ class Cache:
                         rank_tol=0.0, scale=None, tau=math.inf, row_mask=None):
         """Adaptive precision ("Runtime-Certified...", Methodology 3): per row the
         top-K* blocks covering tau_cov of the estimated mass take the original
-        keys, blocks whose new mass x eta exceeds v_tol take the original values,
+        keys, blocks whose estimated mass x eta exceeds v_tol take the original values,
         and the ranking-consistency check over the key-promoted blocks (log-mass
         slack rank_tol) flags the row when it fails.  k_orig, v_orig
         [num_seqs][Hkv][T][d] (fp32, or bf16 bits as uint16).  Returns a dict:

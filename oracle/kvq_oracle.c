@@ -772,8 +772,9 @@ void oc_certified_output(const double* ohat, const double* odense, const uint8_t
 /*   Delta~ = kappa * scale * 2^-16 * |q|_2 * |k_j|_2 in a key-promoted block */
 /*            (allowance for an fp32 dot product of the originals), else      */
 /*            Delta_j                                                         */
-/*   p~     = softmax(z~),  M~_b = sum_{j in b} p~_j                          */
-/*   value-promoted blocks: M~_b * eta_b > v_tol (rung 2 on the new masses)   */
+/*   p~     = softmax(z~)                                                     */
+/*   value-promoted blocks: M^_b * eta_b > v_tol (rung 2: the block's         */
+/*            estimated share of E_val, from the same scoring pass)            */
 /*   o~     = sum_j p~_j v~_j, v~_j = the original v_j in a value-promoted    */
 /*            block, else v^_j                                                */
 /*   A = sum p~ (e^Delta~ - 1), B = sum p~ e^-Delta~, TV = min(tanh(max      */
@@ -823,7 +824,6 @@ int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, c
     oc_blk* ord = npg ? (oc_blk*)malloc(sizeof(oc_blk) * npg) : NULL;
     uint8_t* kp = npg ? (uint8_t*)malloc(npg) : NULL;
     uint8_t* vp = npg ? (uint8_t*)malloc(npg) : NULL;
-    double* mass = npg ? (double*)malloc(sizeof(double) * npg) : NULL;
     for (int i = 0; i < nq; ++i)
       for (int h = 0; h < hq; ++h) {
         int64_t row = ((int64_t)b * nq + i) * hq + h;
@@ -854,6 +854,12 @@ int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, c
         for (int j = 0; j < n; ++j) l += exp(z[j] - m);
         for (int lp = 0; lp < npg; ++lp) { ord[lp].m = 0.0; ord[lp].b = lp; }
         for (int j = 0; j < n; ++j) ord[j / OC_PAGE].m += exp(z[j] - m) / l;
+        /* value promotion on the estimated masses (before the sort reorders them) */
+        int nv = 0;
+        for (int lp = 0; lp < npg; ++lp) {
+          vp[lp] = ord[lp].m * et[lp * OC_PAGE] > v_tol ? 1 : 0;
+          nv += vp[lp];
+        }
         /* top-K* blocks covering tau_cov of the estimated mass */
         qsort(ord, npg, sizeof(oc_blk), oc_blk_cmp);
         int kstar = 0;
@@ -882,14 +888,6 @@ int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, c
         l = 0.0;
         for (int j = 0; j < n; ++j) l += exp(z[j] - m);
         for (int j = 0; j < n; ++j) p[j] = exp(z[j] - m) / l;
-        /* value promotion on the new masses */
-        for (int lp = 0; lp < npg; ++lp) mass[lp] = 0.0;
-        for (int j = 0; j < n; ++j) mass[j / OC_PAGE] += p[j];
-        int nv = 0;
-        for (int lp = 0; lp < npg; ++lp) {
-          vp[lp] = mass[lp] * et[lp * OC_PAGE] > v_tol ? 1 : 0;
-          nv += vp[lp];
-        }
         /* output and bound */
         double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
         double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
@@ -938,7 +936,7 @@ int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, c
           dg[4] = A; dg[5] = B; dg[6] = range; dg[7] = eta_max;
         }
       }
-    free(z); free(dl); free(et); free(p); free(ord); free(kp); free(vp); free(mass);
+    free(z); free(dl); free(et); free(p); free(ord); free(kp); free(vp);
   }
   return OC_OK;
 }

@@ -581,6 +581,374 @@ int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, const vo
   return KVQ_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Work-buffer layout of kvq_adaptive_precision for at most `units` flagged
+// (sequence, kv head) units, `slots` flagged rows and `mp` pages per sequence.
+struct AdLayout {
+  size_t units, items, kp, vp, korder, blse, nkey, nval, rank_fail, um, smap, part, total;
+};
+constexpr int kAdMaxChunks = 8;      // page ranges per unit in the correction
+constexpr int kAdMinChunkPages = 16;
+constexpr int kAdMaxPages = 8192;    // the selection sorts one row's pages in shared memory
+
+AdLayout ad_layout(int64_t units, int64_t slots, int64_t mp, int d) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  AdLayout L;
+  size_t o = 0;
+  L.units = o; o += up(units * sizeof(AdUnit));
+  L.items = o; o += up(units * kAdMaxChunks * sizeof(AdItem));
+  L.kp = o; o += up(slots * mp);
+  L.vp = o; o += up(slots * mp);
+  L.korder = o; o += up(slots * mp * 4);
+  L.blse = o; o += up(slots * mp * 4);
+  L.nkey = o; o += up(slots * 4);
+  L.nval = o; o += up(slots * 4);
+  L.rank_fail = o; o += up(slots);
+  L.um = o; o += up(units * mp);
+  L.smap = o; o += up(units * mp * 4);
+  L.part = o; o += up(units * kAdMaxChunks * adaptive_part_floats(d) * sizeof(float));
+  L.total = o;
+  return L;
+}
+
+// Pinned host scratch: the units, the union of promoted pages per unit and
+// the staged-page maps, each written once per call.
+size_t ad_host_bytes(int64_t units, int64_t mp) {
+  return ((size_t)units * sizeof(AdUnit) + 255) / 256 * 256 + (size_t)units * mp +
+         (size_t)units * mp * 4 + 256;
+}
+
+// Polls `ev` until it completes or the deadline passes (a deadline already
+// passed times out at once, as a timeout of 0 ms does).
+int wait_event_until(cudaEvent_t ev, std::chrono::steady_clock::time_point deadline,
+                     const char* what) {
+  for (;;) {
+    if (std::chrono::steady_clock::now() >= deadline)
+      return fail(KVQ_ERR_TIMEOUT, "%s: not complete before the deadline", what);
+    cudaError_t e = cudaEventQuery(ev);
+    if (e == cudaSuccess) return KVQ_OK;
+    if (e != cudaErrorNotReady) return cuda_fail(e, what);
+    std::this_thread::sleep_for(std::chrono::microseconds(20));
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs, int32_t num_queries,
+                              int32_t num_q_heads, int32_t max_pages_per_seq) {
+  if (check_cache(cache) || num_seqs < 0 || num_queries < 1 || num_q_heads < 1 ||
+      max_pages_per_seq < 1 || max_pages_per_seq > kAdMaxPages)
+    return 0;
+  const int64_t units = (int64_t)num_seqs * cache->num_kv_heads;
+  const int64_t slots = (int64_t)num_seqs * num_queries * num_q_heads;
+  return ad_layout(units, slots, max_pages_per_seq, cache->head_dim).total;
+}
+
+size_t kvq_adaptive_host_size(const kvq_cache* cache, int32_t num_seqs,
+                              int32_t max_pages_per_seq) {
+  if (!cache || cache->num_kv_heads < 1 || num_seqs < 0 || max_pages_per_seq < 1) return 0;
+  return ad_host_bytes((int64_t)num_seqs * cache->num_kv_heads, max_pages_per_seq);
+}
+
+size_t kvq_adaptive_staging_size(const kvq_cache* cache, int orig_dtype,
+                                 int32_t max_pages_per_seq) {
+  if (!cache || (cache->head_dim != 64 && cache->head_dim != 128) || max_pages_per_seq < 1)
+    return 0;
+  if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return 0;
+  const size_t es = orig_dtype == KVQ_BF16 ? 2 : 4;
+  return 2 * (size_t)max_pages_per_seq * KVQ_PAGE_SIZE * cache->head_dim * es;
+}
+
+int kvq_adaptive_precision(const kvq_cache* cache, const void* k_orig_host,
+                           const void* v_orig_host, int orig_dtype, int64_t orig_seq_stride,
+                           int64_t orig_head_stride, const void* q, int q_dtype,
+                           int32_t num_seqs, int32_t num_queries, int32_t num_q_heads,
+                           const int32_t* page_table, int32_t max_pages_per_seq,
+                           const int32_t* seq_lens, const int32_t* seq_lens_host,
+                           float softmax_scale, float tau, float tau_cov, float v_tol,
+                           float rank_tol, uint8_t* flags, uint8_t* flags_host, float* out,
+                           float* bound, uint8_t* promoted_keys, uint8_t* promoted_values,
+                           void* work, size_t work_bytes, void* host_work,
+                           size_t host_work_bytes, void* staging, size_t staging_bytes,
+                           kvq_stream_t main_stream, kvq_stream_t side_stream,
+                           int32_t timeout_ms, int32_t* num_rows, int32_t* num_flagged) {
+  if (num_rows) *num_rows = 0;
+  if (num_flagged) *num_flagged = 0;
+  int rc = check_cache(cache);
+  if (rc) return rc;
+  if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad orig_dtype");
+  if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad q_dtype");
+  if (num_seqs < 0 || num_queries < 1 || num_q_heads < 1 || max_pages_per_seq < 1 ||
+      num_q_heads % cache->num_kv_heads)
+    return fail(KVQ_ERR_INVALID_ARG, "bad sizes");
+  const int D = cache->head_dim, hkv = cache->num_kv_heads, G = num_q_heads / hkv;
+  if ((int64_t)num_queries * G > 4)
+    return fail(KVQ_ERR_UNSUPPORTED, "num_queries * (num_q_heads/num_kv_heads) = %d > 4",
+                num_queries * G);
+  if (max_pages_per_seq > kAdMaxPages)
+    return fail(KVQ_ERR_UNSUPPORTED, "max_pages_per_seq %d > %d", max_pages_per_seq, kAdMaxPages);
+  if (std::isnan(tau) || std::isnan(tau_cov) || std::isnan(v_tol) || std::isnan(rank_tol))
+    return fail(KVQ_ERR_INVALID_ARG, "NaN threshold");
+  if (num_seqs == 0) return KVQ_OK;
+  if (!k_orig_host || !v_orig_host || !q || !page_table || !seq_lens || !seq_lens_host ||
+      !flags || !flags_host || !out || !bound || !work || !host_work || !staging ||
+      !num_rows || !num_flagged)
+    return fail(KVQ_ERR_INVALID_ARG, "NULL argument");
+  if (orig_seq_stride < 0 || orig_head_stride < 0) return fail(KVQ_ERR_INVALID_ARG, "negative stride");
+  if (!aligned16(work) || !aligned16(staging) || !aligned16(host_work))
+    return fail(KVQ_ERR_INVALID_ARG, "work, host_work or staging not 16-byte aligned");
+  const int mp = max_pages_per_seq;
+  const int64_t units_max = (int64_t)num_seqs * hkv;
+  const int64_t rows = (int64_t)num_seqs * num_queries * num_q_heads;
+  const AdLayout WL = ad_layout(units_max, rows, mp, D);
+  if (work_bytes < WL.total)
+    return fail(KVQ_ERR_INVALID_ARG, "work %zu bytes < %zu required", work_bytes, WL.total);
+  if (host_work_bytes < ad_host_bytes(units_max, mp))
+    return fail(KVQ_ERR_INVALID_ARG, "host_work %zu bytes < %zu required", host_work_bytes,
+                ad_host_bytes(units_max, mp));
+  const size_t es = orig_dtype == KVQ_BF16 ? 2 : 4;
+  const size_t page_bytes = (size_t)KVQ_PAGE_SIZE * D * es;
+  for (int s = 0; s < num_seqs; ++s)
+    if (seq_lens_host[s] < 0 || seq_lens_host[s] > mp * KVQ_PAGE_SIZE)
+      return fail(KVQ_ERR_INVALID_ARG, "seq_lens_host[%d] = %d outside [0, %d]", s,
+                  seq_lens_host[s], mp * KVQ_PAGE_SIZE);
+  DeviceInfo di;
+  if ((rc = device_info(&di, nullptr))) return rc;
+  const int smem = adaptive_select_smem(mp, D);
+  if (smem > di.max_smem)
+    return fail(KVQ_ERR_UNSUPPORTED, "selection needs %d bytes of shared memory", smem);
+  cudaStream_t ms = reinterpret_cast<cudaStream_t>(main_stream);
+  cudaStream_t ss = reinterpret_cast<cudaStream_t>(side_stream);
+  const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
+
+  cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+  auto cleanup = [&]() {
+    for (cudaEvent_t& x : ev)
+      if (x) cudaEventDestroy(x);
+  };
+  cudaError_t e;
+  for (cudaEvent_t& x : ev)
+    if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) {
+      cleanup();
+      return cuda_fail(e, "cudaEventCreate");
+    }
+  auto bail = [&](int code) { cleanup(); return code; };
+  // 1. the decode's flags on the host (side stream, after the decode on main)
+  if ((e = cudaEventRecord(ev[0], ms)) != cudaSuccess ||
+      (e = cudaStreamWaitEvent(ss, ev[0], 0)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(flags_host, flags, rows, cudaMemcpyDeviceToHost, ss)) != cudaSuccess ||
+      (e = cudaEventRecord(ev[1], ss)) != cudaSuccess)
+    return bail(cuda_fail(e, "flag read-back"));
+  if ((rc = wait_event_until(ev[1], deadline, "flag read-back"))) return bail(rc);
+
+  // 2. flagged units and their rows (row slots are the flagged rows, in order)
+  uint8_t* hw = static_cast<uint8_t*>(host_work);
+  AdUnit* hunits = reinterpret_cast<AdUnit*>(hw);
+  uint8_t* hum = hw + ((size_t)units_max * sizeof(AdUnit) + 255) / 256 * 256;
+  int32_t* hsmap = reinterpret_cast<int32_t*>(hum + (size_t)units_max * mp);
+  hsmap = reinterpret_cast<int32_t*>((reinterpret_cast<uintptr_t>(hsmap) + 15) / 16 * 16);
+  int nu = 0, nslots = 0;
+  for (int s = 0; s < num_seqs; ++s)
+    for (int h = 0; h < hkv; ++h) {
+      AdUnit un;
+      std::memset(&un, 0, sizeof(un));
+      un.seq = s;
+      un.kvh = h;
+      un.rslot = nslots;
+      for (int i = 0; i < num_queries; ++i)
+        for (int gq = 0; gq < G; ++gq) {
+          const int64_t row = ((int64_t)s * num_queries + i) * num_q_heads + h * G + gq;
+          if (flags_host[row]) un.rows[un.nrows++] = (int32_t)row;
+        }
+      if (un.nrows == 0) continue;
+      nslots += un.nrows;
+      hunits[nu++] = un;
+    }
+  *num_rows = nslots;
+  if (nu == 0) return bail(KVQ_OK);
+
+  uint8_t* wb = static_cast<uint8_t*>(work);
+  AdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.pool = static_cast<const uint8_t*>(cache->pool);
+  a.eta = cache->v_eta;
+  a.signs = cache->k_rotate ? cache->rot_signs : nullptr;
+  a.err = cache->error_word;
+  a.q = q;
+  a.q_bf16 = q_dtype == KVQ_BF16;
+  a.kv_bf16 = orig_dtype == KVQ_BF16;
+  a.page_table = page_table;
+  a.max_pages = mp;
+  a.seq_lens = seq_lens;
+  a.nq = num_queries;
+  a.hq = num_q_heads;
+  a.hkv = hkv;
+  a.G = G;
+  a.num_pages = cache->num_pages;
+  a.s_att = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)D));
+  a.rot_c = rot_constant(D);
+  a.tau = tau;
+  a.tau_cov = tau_cov;
+  a.v_tol = v_tol;
+  a.rank_tol = rank_tol;
+  a.kp = wb + WL.kp;
+  a.vp = wb + WL.vp;
+  a.korder = reinterpret_cast<int32_t*>(wb + WL.korder);
+  a.blse = reinterpret_cast<float*>(wb + WL.blse);
+  a.nkey = reinterpret_cast<int32_t*>(wb + WL.nkey);
+  a.nval = reinterpret_cast<int32_t*>(wb + WL.nval);
+  a.rank_fail = wb + WL.rank_fail;
+  a.out = out;
+  a.bound = bound;
+  a.flags = flags;
+  a.staging = static_cast<const uint8_t*>(staging);
+  AdUnit* d_units = reinterpret_cast<AdUnit*>(wb + WL.units);
+  AdItem* d_items = reinterpret_cast<AdItem*>(wb + WL.items);
+  uint8_t* d_um = wb + WL.um;
+  int32_t* d_smap = reinterpret_cast<int32_t*>(wb + WL.smap);
+
+  // 3. scoring pass and selection for every flagged unit; the union of promoted
+  //    pages per unit back to the host
+  if ((e = cudaMemcpyAsync(d_units, hunits, (size_t)nu * sizeof(AdUnit), cudaMemcpyHostToDevice,
+                           ms)) != cudaSuccess)
+    return bail(cuda_fail(e, "unit list H2D"));
+  a.units = d_units;
+  a.num_units = nu;
+  a.um = d_um;
+  if ((e = launch_adaptive_select(a, D, cache->k_bits, cache->k_group, smem, ms)) != cudaSuccess)
+    return bail(cuda_fail(e, "selection kernel launch"));
+  if ((e = cudaMemcpyAsync(hum, d_um, (size_t)nu * mp, cudaMemcpyDeviceToHost, ms)) != cudaSuccess ||
+      (e = cudaEventRecord(ev[2], ms)) != cudaSuccess)
+    return bail(cuda_fail(e, "promoted-page read-back"));
+  if ((rc = wait_event_until(ev[2], deadline, "promoted-page read-back"))) return bail(rc);
+
+  // 4. staged-page maps; batches of units whose promoted pages fit the staging
+  std::vector<int64_t> stage_bytes(nu);
+  for (int iu = 0; iu < nu; ++iu) {
+    const uint8_t* um = hum + (size_t)iu * mp;
+    int32_t* sm = hsmap + (size_t)iu * mp;
+    int k = 0;
+    for (int b = 0; b < mp; ++b) sm[b] = um[b] ? k++ : -1;
+    hunits[iu].nstaged = k;
+    stage_bytes[iu] = 2 * (int64_t)k * (int64_t)page_bytes;
+    if (stage_bytes[iu] > (int64_t)staging_bytes)
+      return bail(fail(KVQ_ERR_INVALID_ARG, "staging %zu bytes < %lld needed by one (sequence, "
+                       "kv head)", staging_bytes, (long long)stage_bytes[iu]));
+  }
+  if ((e = cudaMemcpyAsync(d_smap, hsmap, (size_t)nu * mp * 4, cudaMemcpyHostToDevice, ms)) !=
+      cudaSuccess)
+    return bail(cuda_fail(e, "page map H2D"));
+  bool staging_read = false;   // ev[3]: the last correction that read the staging
+  std::vector<AdItem> items;
+  for (int b0 = 0; b0 < nu;) {
+    // the batch [b0, b1)
+    int64_t used = 0;
+    int b1 = b0;
+    while (b1 < nu && used + stage_bytes[b1] <= (int64_t)staging_bytes) used += stage_bytes[b1++];
+    items.clear();
+    int64_t off = 0;
+    for (int iu = b0; iu < b1; ++iu) {
+      hunits[iu].stage_off = off;
+      off += stage_bytes[iu];
+      const int n = seq_lens_host[hunits[iu].seq];
+      const int npg = (n + KVQ_PAGE_SIZE - 1) / KVQ_PAGE_SIZE;
+      const int nch = std::max(1, std::min(kAdMaxChunks, (npg + kAdMinChunkPages - 1) / kAdMinChunkPages));
+      const int per = (npg + nch - 1) / nch;
+      const int first = (int)items.size();
+      for (int c = 0; c < nch; ++c) {
+        AdItem it;
+        it.unit = iu - b0;
+        it.p0 = std::min(npg, c * per);
+        it.p1 = std::min(npg, (c + 1) * per);
+        it.chunk = c;
+        it.nchunk = nch;
+        it.first = first;
+        items.push_back(it);
+      }
+    }
+    // the batch's unit records (stage offsets) and items
+    if ((e = cudaMemcpyAsync(d_units + b0, hunits + b0, (size_t)(b1 - b0) * sizeof(AdUnit),
+                             cudaMemcpyHostToDevice, ms)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(d_items, items.data(), items.size() * sizeof(AdItem),
+                             cudaMemcpyHostToDevice, ms)) != cudaSuccess)
+      return bail(cuda_fail(e, "batch H2D"));
+    // page-in on the side stream, after the correction that last read the staging
+    if (staging_read && (e = cudaStreamWaitEvent(ss, ev[3], 0)) != cudaSuccess)
+      return bail(cuda_fail(e, "cudaStreamWaitEvent"));
+    for (int iu = b0; iu < b1; ++iu) {
+      const AdUnit& un = hunits[iu];
+      const int n = seq_lens_host[un.seq];
+      const uint8_t* um = hum + (size_t)iu * mp;
+      const int32_t* sm = hsmap + (size_t)iu * mp;
+      const int64_t src0 = ((int64_t)un.seq * orig_seq_stride + (int64_t)un.kvh * orig_head_stride) * es;
+      uint8_t* dk = static_cast<uint8_t*>(staging) + un.stage_off;
+      uint8_t* dv = dk + (size_t)un.nstaged * page_bytes;
+      for (int b = 0; b < mp;) {
+        if (!um[b]) { ++b; continue; }
+        int e2 = b;
+        while (e2 < mp && um[e2]) ++e2;
+        const int64_t t0 = (int64_t)b * KVQ_PAGE_SIZE;
+        const int64_t t1 = std::min<int64_t>((int64_t)e2 * KVQ_PAGE_SIZE, n);
+        if (t1 > t0) {
+          if (fault_injected("memcpy")) return bail(fail(KVQ_ERR_CUDA, "cudaMemcpyAsync failed (injected fault)"));
+          const size_t bytes = (size_t)(t1 - t0) * D * es;
+          const size_t soff = (size_t)sm[b] * page_bytes;
+          const uint8_t* kh = static_cast<const uint8_t*>(k_orig_host) + src0 + t0 * D * es;
+          const uint8_t* vh = static_cast<const uint8_t*>(v_orig_host) + src0 + t0 * D * es;
+          if ((e = cudaMemcpyAsync(dk + soff, kh, bytes, cudaMemcpyHostToDevice, ss)) != cudaSuccess ||
+              (e = cudaMemcpyAsync(dv + soff, vh, bytes, cudaMemcpyHostToDevice, ss)) != cudaSuccess)
+            return bail(cuda_fail(e, "cudaMemcpyAsync (Tier-2 page-in)"));
+        }
+        b = e2;
+      }
+    }
+    // correction and finish on main, after the copies
+    AdArgs ab = a;
+    ab.units = d_units + b0;
+    ab.num_units = b1 - b0;
+    ab.items = d_items;
+    ab.num_items = (int)items.size();
+    ab.smap = d_smap + (size_t)b0 * mp;
+    ab.part = reinterpret_cast<float*>(wb + WL.part);
+    if ((e = cudaEventRecord(ev[0], ss)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(ms, ev[0], 0)) != cudaSuccess)
+      return bail(cuda_fail(e, "copy hand-off"));
+    if ((e = launch_adaptive_correct(ab, D, cache->k_bits, cache->k_group, ms)) != cudaSuccess ||
+        (e = launch_adaptive_finish(ab, D, ms)) != cudaSuccess)
+      return bail(cuda_fail(e, "correction kernel launch"));
+    if ((e = cudaEventRecord(ev[3], ms)) != cudaSuccess) return bail(cuda_fail(e, "cudaEventRecord"));
+    staging_read = true;
+    // the items and unit records of the next batch overwrite these: wait (bounded)
+    if (b1 < nu && (rc = wait_event_until(ev[3], deadline, "correction batch"))) return bail(rc);
+    b0 = b1;
+  }
+  // 5. per-row promotion maps for the caller; the new flags on the host
+  for (int iu = 0; iu < nu && (promoted_keys || promoted_values); ++iu)
+    for (int r = 0; r < hunits[iu].nrows; ++r) {
+      const int64_t row = hunits[iu].rows[r];
+      const size_t so = (size_t)(hunits[iu].rslot + r) * mp;
+      if (promoted_keys &&
+          (e = cudaMemcpyAsync(promoted_keys + row * mp, a.kp + so, mp, cudaMemcpyDeviceToDevice, ms)) != cudaSuccess)
+        return bail(cuda_fail(e, "promotion map copy"));
+      if (promoted_values &&
+          (e = cudaMemcpyAsync(promoted_values + row * mp, a.vp + so, mp, cudaMemcpyDeviceToDevice, ms)) != cudaSuccess)
+        return bail(cuda_fail(e, "promotion map copy"));
+    }
+  if ((e = cudaMemcpyAsync(flags_host, flags, rows, cudaMemcpyDeviceToHost, ms)) != cudaSuccess ||
+      (e = cudaEventRecord(ev[2], ms)) != cudaSuccess)
+    return bail(cuda_fail(e, "flag read-back"));
+  if ((rc = wait_event_until(ev[2], deadline, "final flag read-back"))) return bail(rc);
+  int cnt = 0;
+  for (int64_t r = 0; r < rows; ++r) cnt += flags_host[r] != 0;
+  *num_flagged = cnt;
+  return bail(KVQ_OK);
+}
+
 int kvq_device_error(const kvq_cache* cache, kvq_stream_t stream, int32_t* code) {
   if (!cache || !code) return fail(KVQ_ERR_INVALID_ARG, "NULL argument");
   *code = KVQ_OK;

@@ -110,6 +110,59 @@ cudaError_t launch_pdl(void (*kernel)(Arg), dim3 grid, dim3 block, size_t smem, 
   return cudaLaunchKernelEx(&cfg, kernel, arg);
 }
 
+// ---- adaptive precision (adaptive.cu) ------------------------------------------
+// One flagged (sequence, kv head) with its flagged query rows (at most 4).
+struct AdUnit {
+  int32_t seq, kvh, nrows, rslot;   // rslot: this unit's first row slot
+  int32_t rows[4];                  // flattened (sequence, query, q head) row indices
+  int64_t stage_off;                // bytes into staging: its promoted pages' K, then V
+  int32_t nstaged, pad;             // pages staged
+};
+// One correction item: pages [p0, p1) of unit `unit`.
+struct AdItem {
+  int32_t unit, p0, p1, chunk, nchunk, first;   // first: the unit's first item
+};
+struct AdArgs {
+  const uint8_t* pool;
+  const float* eta;
+  const int8_t* signs;
+  int32_t* err;
+  const void* q;
+  int q_bf16, kv_bf16;
+  const int32_t* page_table;
+  int max_pages;
+  const int32_t* seq_lens;
+  int nq, hq, hkv, G, num_pages;
+  float s_att, rot_c, tau, tau_cov, v_tol, rank_tol;
+  const AdUnit* units;
+  int num_units;
+  const AdItem* items;
+  int num_items;
+  // per row slot, [slots][max_pages]: key / value promotion, the key-promoted
+  // pages in selection order, exact block log-masses; per slot counts
+  uint8_t* kp;
+  uint8_t* vp;
+  int32_t* korder;
+  float* blse;
+  int32_t* nkey;
+  int32_t* nval;
+  uint8_t* um;                 // [units][max_pages]: kp | vp over the unit's rows
+  const int32_t* smap;         // [units][max_pages]: staged index of a page, or -1
+  const uint8_t* staging;
+  float* part;                 // [items][4 rows][D + 8] and [items][2 NB + 1]
+  float* out;
+  float* bound;
+  uint8_t* flags;
+  uint8_t* rank_fail;          // per row slot
+};
+// bytes of the per-item partial records
+__host__ __device__ inline size_t adaptive_part_floats(int d) { return 4 * (size_t)(d + 8) + 2 * (d / 32) + 4; }
+cudaError_t launch_adaptive_select(const AdArgs& a, int d, int kbits, int kgroup, int smem,
+                                   cudaStream_t s);
+cudaError_t launch_adaptive_correct(const AdArgs& a, int d, int kbits, int kgroup, cudaStream_t s);
+cudaError_t launch_adaptive_finish(const AdArgs& a, int d, cudaStream_t s);
+int adaptive_select_smem(int max_pages, int d);
+
 cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, cudaStream_t s);
 DecodeVariant select_decode_kernel(int d, int kbits, int kgroup);
 int decode_threads();

@@ -35,7 +35,9 @@ PAGE_SIZE = 16
 EXPORTED = ("kvq_block_bytes", "kvq_pool_bytes", "kvq_quantize_append", "kvq_workspace_size",
             "kvq_decode_attention", "kvq_error_bound", "kvq_fallback_staging_size",
             "kvq_fallback_exact", "kvq_device_error", "kvq_status_string", "kvq_last_error",
-            "kvq_decode_attention_noalloc", "kvq_decode_attention_append")
+            "kvq_decode_attention_noalloc", "kvq_decode_attention_append",
+            "kvq_adaptive_work_size", "kvq_adaptive_host_size", "kvq_adaptive_staging_size",
+            "kvq_adaptive_precision")
 
 
 class KvqError(RuntimeError):
@@ -82,6 +84,14 @@ def _load() -> ctypes.CDLL:
         "kvq_decode_attention_append": (ctypes.c_int, [C, P, P, ctypes.c_int, I64, I64, P,
                                                        ctypes.c_int, I32, I32, I32, P, I32, P, F,
                                                        F, P, P, P, P, SZ, P]),
+        "kvq_adaptive_work_size": (SZ, [C, I32, I32, I32, I32]),
+        "kvq_adaptive_host_size": (SZ, [C, I32, I32]),
+        "kvq_adaptive_staging_size": (SZ, [C, ctypes.c_int, I32]),
+        "kvq_adaptive_precision": (ctypes.c_int, [C, P, P, ctypes.c_int, I64, I64, P,
+                                                  ctypes.c_int, I32, I32, I32, P, I32, P, P, F,
+                                                  F, F, F, F, P, P, P, P, P, P, P, SZ, P, SZ, P,
+                                                  SZ, P, P, I32, ctypes.POINTER(I32),
+                                                  ctypes.POINTER(I32)]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
@@ -227,6 +237,39 @@ def kvq_fallback_exact(cache, k_orig_host, v_orig_host, orig_dtype, orig_seq_str
                                  _ptr(staging), staging_bytes, _stream(main_stream),
                                  _stream(side_stream), timeout_ms, ctypes.byref(nfb))
     return rc, nfb.value
+
+
+def kvq_adaptive_work_size(cache, num_seqs, num_queries, num_q_heads, max_pages_per_seq) -> int:
+    return _lib.kvq_adaptive_work_size(ctypes.byref(cache), num_seqs, num_queries, num_q_heads,
+                                       max_pages_per_seq)
+
+
+def kvq_adaptive_host_size(cache, num_seqs, max_pages_per_seq) -> int:
+    return _lib.kvq_adaptive_host_size(ctypes.byref(cache), num_seqs, max_pages_per_seq)
+
+
+def kvq_adaptive_staging_size(cache, orig_dtype, max_pages_per_seq) -> int:
+    return _lib.kvq_adaptive_staging_size(ctypes.byref(cache), orig_dtype, max_pages_per_seq)
+
+
+def kvq_adaptive_precision(cache, k_orig_host, v_orig_host, orig_dtype, orig_seq_stride,
+                           orig_head_stride, q, q_dtype, num_seqs, num_queries, num_q_heads,
+                           page_table, max_pages_per_seq, seq_lens, seq_lens_host, softmax_scale,
+                           tau, tau_cov, v_tol, rank_tol, flags, flags_host, out, bound,
+                           promoted_keys, promoted_values, work, work_bytes, host_work,
+                           host_work_bytes, staging, staging_bytes, main_stream=None,
+                           side_stream=None, timeout_ms=10000):
+    """Returns (status, rows that ran through the ladder, rows flagged afterwards)."""
+    nr, nf = ctypes.c_int32(0), ctypes.c_int32(0)
+    rc = _lib.kvq_adaptive_precision(
+        ctypes.byref(cache), _ptr(k_orig_host), _ptr(v_orig_host), orig_dtype, orig_seq_stride,
+        orig_head_stride, _ptr(q), q_dtype, num_seqs, num_queries, num_q_heads, _ptr(page_table),
+        max_pages_per_seq, _ptr(seq_lens), _ptr(seq_lens_host), softmax_scale, tau, tau_cov,
+        v_tol, rank_tol, _ptr(flags), _ptr(flags_host), _ptr(out), _ptr(bound),
+        _ptr(promoted_keys), _ptr(promoted_values), _ptr(work), work_bytes, _ptr(host_work),
+        host_work_bytes, _ptr(staging), staging_bytes, _stream(main_stream), _stream(side_stream),
+        timeout_ms, ctypes.byref(nr), ctypes.byref(nf))
+    return rc, nr.value, nf.value
 
 
 def kvq_device_error(cache, stream=None):

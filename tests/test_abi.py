@@ -31,7 +31,7 @@ def test_header_declares_the_four_calls():
     for fn in ("kvq_quantize_append", "kvq_decode_attention", "kvq_error_bound",
                "kvq_fallback_exact"):
         assert fn in names
-    assert len(names) == 13
+    assert len(names) == 17
 
 
 def test_library_exports_every_declared_symbol(kvq):
