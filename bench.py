@@ -43,6 +43,11 @@ METRIC = ("quantized-KV decode attention: KV tokens·heads/s and achieved HBM GB
 UNIT = "KV token-heads/s"
 L2_BYTES = 126 * 2 ** 20
 SPEC_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (context for frac_vs_spec)
+# adaptive-precision ladder of the serving line: the pages' example coverage
+# (99.5% of the estimated mass on full-precision keys), value promotion of
+# blocks whose estimated share of the value error exceeds 1e-4, and a ranking
+# check that tolerates exact log-mass inversions up to 0.1
+LADDER = {"tau_cov": 0.995, "v_tol": 1e-4, "rank_tol": 0.1}
 DECODE_SRC = os.path.join(ROOT, "quantized_decode_attention_kvq_b200", "csrc",
                           "decode_attention.cu")
 
@@ -368,6 +373,17 @@ class GpuStep:
                 sl_h=np.array(inp.seq_lens, np.int32),
                 staging=torch.empty(fb_bytes, dtype=torch.uint8, device="cuda"), rows=0, calls=0,
                 h2d=0)
+            # the adaptive-precision ladder run before the exact fallback
+            mp = self.pt.shape[1]
+            rows = self.flags.numel()
+            ad_host = kvq.kvq_adaptive_host_size(base.desc, B, mp)
+            self.ladder = dict(
+                work=torch.zeros(kvq.kvq_adaptive_work_size(base.desc, B, NQ, HQ, mp),
+                                 dtype=torch.uint8, device="cuda"),
+                host=torch.zeros(ad_host, dtype=torch.uint8).pin_memory(),
+                kp=torch.zeros((rows, mp), dtype=torch.uint8, device="cuda"),
+                vp=torch.zeros((rows, mp), dtype=torch.uint8, device="cuda"),
+                rows_in=0, rows_after=0, calls=0, h2d=0)
 
     def fallback_exact(self, r=0):
         """The exact fallback of the rows the last decode flagged (host-synchronous)."""
@@ -387,6 +403,39 @@ class GpuStep:
         fb["rows"] += n
         fb["calls"] += 1
         return n
+
+    def adaptive(self, r=0):
+        """The adaptive-precision ladder on the rows the last decode flagged
+        (host-synchronous): top-K* key promotion (tau_cov), value promotion
+        (v_tol) and the ranking check (rank_tol); flags are rewritten for the
+        exact fallback that follows."""
+        fb, ad, wl, kvq = self.fallback, self.ladder, self.wl, self.kvq
+        B, NQ, HQ, d = self.out.shape
+        mp = self.pt.shape[1]
+        rc, n_in, n_after = kvq.kvq_adaptive_precision(
+            self.caches[r].desc, fb["kh"], fb["vh"], fb["dt"], wl.num_kv_heads * fb["T"] * d,
+            fb["T"] * d, self.qd, fb["qdt"], B, NQ, HQ, self.pt, mp, self.sl,
+            fb["sl_h"].ctypes.data, 0.0, wl.tau, LADDER["tau_cov"], LADDER["v_tol"],
+            LADDER["rank_tol"], self.flags, fb["flags_h"], self.out, self.bound, ad["kp"],
+            ad["vp"], ad["work"], ad["work"].numel(), ad["host"], ad["host"].numel(),
+            fb["staging"], fb["staging"].numel(), self.stream, fb["side"], 60000)
+        if rc:
+            raise RuntimeError(kvq.last_error())
+        # bytes paged in: the union of promoted pages per (sequence, kv head), K and V
+        if n_in:
+            fl = fb["flags_h"]
+            um = (ad["kp"] | ad["vp"]).view(B, NQ, wl.num_kv_heads, -1, mp).amax(dim=(1, 3))
+            es = 2 if fb["dt"] == kvq.KVQ_BF16 else 4
+            th = self.torch
+            sl = th.tensor(fb["sl_h"], dtype=th.int64, device=um.device)
+            tok = th.clamp(sl[:, None, None] - 16 * th.arange(mp, device=um.device), 0, 16)
+            ad["h2d"] += int((um.to(th.int64) * tok).sum().item()) * 2 * d * es
+            ad["kp"].zero_()
+            ad["vp"].zero_()
+        ad["rows_in"] += n_in
+        ad["rows_after"] += n_after
+        ad["calls"] += 1
+        return n_in, n_after
 
     def step(self, i, ev=None, io=0):
         r = i % self.replicas
@@ -479,7 +528,7 @@ def _timed_replay(st, args, world, rank, local):
     return ms_total, dec_ms, clocks
 
 
-def _e2e(st, args, world):
+def _e2e(st, args, world, ladder=False):
     """The same steps end to end through the C ABI with host buffers: per step the
     H2D of its packed inputs (q and the new K/V token) from pinned memory, the
     step's call(s), the D2H of its packed results (out, bound, flags); with a
@@ -553,6 +602,8 @@ def _e2e(st, args, world):
             for i in range(e_steps):
                 st.io_in.copy_(in_h[0], non_blocking=True)
                 st.step(i)
+                if ladder:
+                    st.adaptive(i % st.replicas)
                 st.fallback_exact(i % st.replicas)
                 out_h[0].copy_(st.io_out, non_blocking=True)
             e1.record(st.stream)
@@ -570,6 +621,14 @@ def measure_workload(name, args, world, rank, local):
     st = GpuStep(name, args.seed, reps, two_calls=args.two_calls)
     ms_total, dec_ms, clocks = _timed_replay(st, args, world, rank, local)
     e2e_ms, h2d, d2h = _e2e(st, args, world)
+    lad_ms = None
+    if st.fallback is not None:
+        fb_rows, fb_calls, fb_h2d = st.fallback["rows"], st.fallback["calls"], st.fallback["h2d"]
+        lad_ms, _, _ = _e2e(st, args, world, ladder=True)
+        lad_ms = _max_over_ranks(lad_ms, world)
+        lad_fb = (st.fallback["rows"] - fb_rows, st.fallback["calls"] - fb_calls,
+                  st.fallback["h2d"] - fb_h2d)
+        st.fallback["rows"], st.fallback["calls"], st.fallback["h2d"] = fb_rows, fb_calls, fb_h2d
     ms_step, dec_ms, e2e_ms = _rank_times(ms_total, dec_ms, e2e_ms, args.steps, world)
     peak, peak_kind = _peaks()
     achieved = st.decode_bytes / (dec_ms * 1e-3) / 1e9
@@ -613,6 +672,23 @@ def measure_workload(name, args, world, rank, local):
             "note": "value times append + decode (graph); e2e adds the exact fallback of the "
                     "flagged rows (H2D of their originals + fp32 attention)"}
         rec["e2e"]["h2d_bytes_per_step"] = int(h2d + fb["h2d"] / max(1, fb["calls"]))
+        ad = st.ladder
+        calls = max(1, ad["calls"])
+        rec["ladder"] = {
+            "what": "kvq_adaptive_precision on the decode's flagged rows (top-K* key promotion, "
+                    "value promotion, ranking check), then kvq_fallback_exact on the rows "
+                    "still flagged",
+            **LADDER,
+            "rows_in_per_step": ad["rows_in"] / calls,
+            "rows_flagged_after_ladder_per_step": ad["rows_after"] / calls,
+            "fallback_rate": ad["rows_after"] / calls / rows,
+            "promoted_h2d_bytes_per_step": ad["h2d"] / calls,
+            "fallback_h2d_bytes_per_step": lad_fb[2] / max(1, lad_fb[1]),
+            "e2e": {"value": _job_value(st.token_heads, world, lad_ms), "unit": UNIT,
+                    "ms_per_step": lad_ms,
+                    "h2d_bytes_per_step": int(h2d + ad["h2d"] / calls +
+                                              lad_fb[2] / max(1, lad_fb[1])),
+                    "d2h_bytes_per_step": int(d2h)}}
     del st
     torch.cuda.empty_cache()
     return rec

@@ -85,52 +85,59 @@ def run_adaptive(inp, k, v, q, tau, tau_cov, v_tol, rank_tol, staging_bytes=None
     return res
 
 
-def _oracle_row_decisions(inp, c, q, k, r, tau_cov, v_tol, rank_tol, tau):
+def ambiguous_rows(c, q, k, page_table, seq_lens, group, ref, tau_cov, v_tol, rank_tol, tau,
+                   as_f32, row_mask=None):
     """Rows whose integer decisions lie within BAND of a threshold, judged on the
-    oracle's fp64 values."""
-    wl = inp.wl
-    amb = np.zeros(r["bound"].size, bool)
-    s_att = float(oracle.default_scale(wl.head_dim))
-    for b in range(wl.num_seqs):
-        n = inp.seq_lens[b]
+    oracle's fp64 values (q, k of the sequences the oracle cache holds)."""
+    B, NQ, HQ, d = q.shape
+    amb = np.zeros(B * NQ * HQ, bool)
+    s_att = float(oracle.default_scale(d))
+    for b in range(B):
+        n = int(seq_lens[b])
         if n == 0:
             continue
         npg = (n + 15) // 16
-        for i in range(wl.num_queries):
-            for h in range(wl.num_q_heads):
-                row = (b * wl.num_queries + i) * wl.num_q_heads + h
-                z, _ = c.decode_terms(q, inp.page_table, n, b, i, h)
+        for i in range(NQ):
+            for h in range(HQ):
+                row = (b * NQ + i) * HQ + h
+                if row_mask is not None and not row_mask[row]:
+                    continue
+                z, _ = c.decode_terms(q, page_table, n, b, i, h)
                 p = np.exp(z - z.max())
                 p /= p.sum()
-                m = np.array([p[16 * x:16 * x + 16].sum() for x in range(npg)])
+                m = np.add.reduceat(p, np.arange(0, n, 16))
                 order = sorted(range(npg), key=lambda x: (-m[x], x))
                 cum = np.cumsum(m[order])
-                K = int(r["nkey"][row])
+                K = int(ref["nkey"][row])
                 if tau_cov > 0:
-                    if K >= 1 and abs(cum[K - 1] - tau_cov) <= BAND * max(tau_cov, 1e-30):
+                    if K >= 1 and abs(cum[K - 1] - tau_cov) <= BAND * tau_cov:
                         amb[row] = True
-                    if K >= 2 and abs(cum[K - 2] - tau_cov) <= BAND * max(tau_cov, 1e-30):
+                    if K >= 2 and abs(cum[K - 2] - tau_cov) <= BAND * tau_cov:
                         amb[row] = True
                     if 1 <= K < npg and abs(m[order[K - 1]] - m[order[K]]) <= BAND * m[order[K - 1]]:
                         amb[row] = True
-                eta = np.array([c.eta[inp.page_table[b, x], h // wl.group] for x in range(npg)],
-                               np.float64)
+                kv = h // group
+                eta = c.eta[page_table[b, :npg], kv].astype(np.float64)
                 if np.isfinite(v_tol) and (np.abs(m * eta - v_tol) <= BAND * abs(v_tol)).any():
                     amb[row] = True
                 blocks = order[:K]
-                if blocks:
-                    kv = h // wl.group
-                    qf = inp.as_f32(q[b, i, h]).astype(np.float64)
-                    kf = inp.as_f32(k[b, kv, :n]).astype(np.float64)
+                if len(blocks) > 1:
+                    qf = as_f32(q[b, i, h]).astype(np.float64)
+                    kf = as_f32(k[b, kv, :n]).astype(np.float64)
                     zz = s_att * (kf @ qf)
-                    L = [np.log(np.exp(zz[16 * x:16 * x + 16] - zz.max()).sum()) + zz.max()
-                         for x in blocks]
-                    for y in range(1, len(L)):
-                        if abs(L[y] - min(L[:y]) - rank_tol) <= BAND:
-                            amb[row] = True
-                if math.isfinite(tau) and abs(r["bound"][row] - tau) <= 1e-4 * abs(tau):
+                    e = np.exp(zz - zz.max())
+                    L = np.log(np.add.reduceat(e, np.arange(0, n, 16)))[blocks] + zz.max()
+                    gap = L[1:] - np.minimum.accumulate(L)[:-1]
+                    if (np.abs(gap - rank_tol) <= BAND).any():
+                        amb[row] = True
+                if math.isfinite(tau) and abs(ref["bound"][row] - tau) <= 1e-4 * abs(tau):
                     amb[row] = True
     return amb
+
+
+def _oracle_row_decisions(inp, c, q, k, r, tau_cov, v_tol, rank_tol, tau):
+    return ambiguous_rows(c, q, k, inp.page_table, inp.seq_lens, inp.wl.group, r, tau_cov,
+                          v_tol, rank_tol, tau, inp.as_f32)
 
 
 def _check(inp, res, ref, amb, flagged):
@@ -234,3 +241,32 @@ def test_timeout_and_injected_copy_failure(monkeypatch):
     monkeypatch.setenv("KVQ_FAULT", "memcpy")
     res = run_adaptive(inp, k, v, q, 0.0, 0.9, math.inf, 0.0)
     assert res["rc"] == kvq.KVQ_ERR_CUDA and "injected" in res["msg"]
+
+
+@pytest.mark.parametrize("name,seed,v_tol", [("llama8b", 0, 1e-3), ("serving", 1, 1e-3),
+                                             ("rotated", 2, 3e-3)])
+def test_value_promotion_matches_its_oracle(name, seed, v_tol):
+    """Rung 2 alone (tau_cov = 0): outputs, bounds, promoted counts and flags
+    against oc_decode_promote_values."""
+    inp = small(name, seed)
+    k, v = inp.kv()
+    q = inp.q()
+    tau = 0.0
+    res = run_adaptive(inp, k, v, q, tau, 0.0, v_tol, 0.0)
+    assert res["rc"] == 0, res.get("msg")
+    oc = oracle_cache(inp)
+    assert oc.append(k, v, inp.page_table, np.zeros(inp.wl.num_seqs, np.int32),
+                     valid=np.array(inp.seq_lens, np.int32)) == 0
+    o, b, f, npro, _ = oc.decode_promote_values(q, inp.page_table, inp.seq_lens, v, v_tol,
+                                                tau=tau)
+    ref = dict(nkey=np.zeros_like(npro), bound=b)
+    amb = ambiguous_rows(oc, q, k, inp.page_table, inp.seq_lens, inp.wl.group, ref, 0.0, v_tol,
+                         0.0, tau, inp.as_f32)
+    ok = ~amb
+    assert ok.sum() == ok.size
+    assert np.array_equal(res["vp"].sum(axis=1)[ok], npro[ok])
+    assert not res["kp"].any()
+    emax = np.abs(res["out"][ok] - o[ok]).max()
+    assert emax <= TOL_MAXABS, emax
+    assert (np.abs(res["bound"][ok] - b[ok]) <= TOL_BOUND_REL * b[ok]).all()
+    assert np.array_equal(res["flags"][ok], f[ok])
