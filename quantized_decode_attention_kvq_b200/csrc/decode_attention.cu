@@ -731,6 +731,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   const int last_page = npages - 1;
   uint32_t par = 0;
   bool going = true;
+  int jstop = nloc;   // the page whose wait ran out, if one did
   for (int j0 = 0; j0 < nloc && going; j0 += S) {
     static_for<0, S>([&](auto u_c) {
       const int j = j0 + decltype(u_c)::value;
@@ -738,8 +739,20 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
       const bool full = first + j * kWarps < last_page || n % kPage == 0;
       going = full ? page_step(u_c, std::true_type{}, j, par)
                    : page_step(u_c, std::false_type{}, j, par);
+      if (!going) jstop = j;
     });
     par ^= 1u;
+  }
+  // After a wait that ran out, the copies still in flight (pages jstop ..
+  // min(jstop + S, nloc) - 1, issued but not consumed) are waited for, each
+  // with the same bounded wait, before their stages become the merge area.
+  if (!going) {
+    for (int j = jstop; j < nloc && j < jstop + S; ++j) {
+      static_for<0, S>([&](auto u_c) {
+        constexpr int u = decltype(u_c)::value;
+        if (j % S == u) (void)mbar_wait(&bar[u], (uint32_t)((j / S) & 1));
+      });
+    }
   }
 
   // ---- warp reductions ----------------------------------------------------------

@@ -1,7 +1,9 @@
 """Helpers of the GPU parity tests: run the library through the C ABI on a seeded
 workload, and the oracle on the same bytes.  Test helper only."""
 
+import json
 import math
+import os
 
 import numpy as np
 import torch
@@ -72,6 +74,23 @@ def compare_outputs(out, ref):
     err = np.abs(out - ref)
     rel = np.linalg.norm(out - ref) / max(np.linalg.norm(ref), 1e-300)
     return float(err.max()), float(rel)
+
+
+def record_margin(label, out, ref, **extra):
+    """Append the observed output margin against the oracle (max-abs, relative
+    L2, the worst row and its largest |output|) to the JSON-lines file named
+    by KVQ_MARGIN_LOG, when that variable is set."""
+    path = os.environ.get("KVQ_MARGIN_LOG")
+    if not path:
+        return
+    err = np.abs(out - ref).max(axis=-1)
+    row = int(err.argmax())
+    rec = dict(label=label, max_abs=float(err.max()),
+               rel_l2=float(np.linalg.norm(out - ref) / max(np.linalg.norm(ref), 1e-300)),
+               worst_row=row, worst_row_max_abs_out=float(np.abs(ref[row]).max()),
+               rows=int(err.size), **extra)
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
 
 
 def compare_flags(gflags, oflags, obound, tau):

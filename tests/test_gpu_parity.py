@@ -11,6 +11,7 @@ import torch
 
 import oracle
 from gpu_cases import (TOL_BOUND_REL, TOL_MAXABS, TOL_RELL2, compare_flags, compare_outputs,
+                       record_margin,
                        gpu_cache, oracle_pool, run_gpu, to_torch)
 from oracle_cases import SMALL, max_err, small
 from quantized_decode_attention_kvq_b200 import inputs as synth
@@ -27,6 +28,10 @@ def _cuda():
 
 
 def _check_decode(inp, g, o_hat, bound, flags, tau):
+    wl = inp.wl
+    record_margin(f"{wl.name} B={wl.num_seqs} ctx<={max(inp.seq_lens)} seed={inp.seed}",
+                  g["out"], o_hat, spike_seqs=list(inp.spike_seqs),
+                  rows_per_seq=wl.num_queries * wl.num_q_heads)
     emax, rel = compare_outputs(g["out"], o_hat)
     assert emax <= TOL_MAXABS and rel <= TOL_RELL2, (emax, rel)
     brel = np.abs(g["bound"] - bound) / np.maximum(bound, 1e-30)
