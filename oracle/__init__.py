@@ -52,6 +52,9 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oc_f16_value.argtypes = [ctypes.c_uint16]
     L.oc_f16_round.restype = ctypes.c_uint16
     L.oc_f16_round.argtypes = [ctypes.c_float, ctypes.c_int]
+    L.oc_f16_rn.restype = ctypes.c_uint16
+    L.oc_f16_rn.argtypes = [ctypes.c_float]
+    L.oc_med3_chunk.restype = ctypes.c_int
     L.oc_block_bytes.restype = ctypes.c_int64
     for name in ("oc_quantize_sym", "oc_quantize_asym", "oc_append", "oc_decode",
                  "oc_decode_promote_values", "oc_dense", "oc_f16_round_n"):
@@ -98,7 +101,8 @@ def source_text() -> str:
 
 class OcCfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("d", "hkv", "kbits", "kgroup", "krotate", "vbits", "vgroup", "num_pages")]
+                ("d", "hkv", "kbits", "kgroup", "krotate", "vbits", "vgroup", "num_pages",
+                 "outliers")]
 
 
 def _p(a: Optional[np.ndarray]):
@@ -120,6 +124,18 @@ def f16_round(x, up: bool) -> np.ndarray:
     out = np.empty(x.shape, dtype=np.uint16)
     lib().oc_f16_round_n(_p(x), ctypes.c_int64(x.size), int(bool(up)), _p(out))
     return out
+
+
+def f16_rn(x) -> np.ndarray:
+    """Round fp32 to the nearest binary16 (ties to even): bits."""
+    x = _c(x, np.float32).ravel()
+    return np.array([lib().oc_f16_rn(ctypes.c_float(v)) for v in x], dtype=np.uint16)
+
+
+def med3_chunk(x) -> int:
+    """Med3x outlier chunk of one vector (index of 4-element chunk, or -1)."""
+    x = _c(x, np.float32).ravel()
+    return int(lib().oc_med3_chunk(_p(x), x.size))
 
 
 def f16_value(h) -> np.ndarray:
@@ -164,9 +180,9 @@ class Cache:
     """The oracle's own paged Tier-1 cache (same byte format as the library's)."""
 
     def __init__(self, head_dim, num_kv_heads, num_pages, k_bits=8, k_group=128,
-                 k_rotate=False, v_bits=4, v_group=32, rot_signs=None):
+                 k_rotate=False, v_bits=4, v_group=32, rot_signs=None, outliers=False):
         self.cfg = OcCfg(head_dim, num_kv_heads, k_bits, k_group, int(bool(k_rotate)),
-                         v_bits, v_group, num_pages)
+                         v_bits, v_group, num_pages, int(bool(outliers)))
         bb = lib().oc_block_bytes(ctypes.byref(self.cfg))
         if bb < 0:
             raise ValueError("unsupported cache configuration")

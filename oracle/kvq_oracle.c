@@ -188,6 +188,31 @@ int oc_quantize_sym(const float* x, int n, int Q, uint16_t* scale_bits, int8_t* 
   return OC_OK;
 }
 
+/* The same two quantizers with the channels [skip0, skip1) of the group left
+ * out (an extracted outlier chunk): they take no part in the scale, the zero
+ * or the error, and get code 0.  skip0 = skip1 is the plain quantizer. */
+static int oc_quantize_sym_skip(const float* x, int n, int Q, int skip0, int skip1,
+                                uint16_t* scale_bits, int8_t* codes) {
+  float y[128];
+  for (int c = 0; c < n; ++c) y[c] = (c >= skip0 && c < skip1) ? 0.0f : x[c];
+  return oc_quantize_sym(y, n, Q, scale_bits, codes);   /* 0 leaves max|x| unchanged */
+}
+
+int oc_quantize_asym(const float* x, int n, uint16_t* scale_bits, uint16_t* zero_bits,
+                     uint8_t* codes, float* max_err);
+
+static int oc_quantize_asym_skip(const float* x, int n, int skip0, int skip1,
+                                 uint16_t* scale_bits, uint16_t* zero_bits, uint8_t* codes,
+                                 float* max_err) {
+  if (skip0 >= skip1) return oc_quantize_asym(x, n, scale_bits, zero_bits, codes, max_err);
+  float y[128];
+  int first = skip0 > 0 ? 0 : skip1;   /* a channel of the group that is kept */
+  for (int c = 0; c < n; ++c) y[c] = (c >= skip0 && c < skip1) ? x[first] : x[c];
+  int rc = oc_quantize_asym(y, n, scale_bits, zero_bits, codes, max_err);
+  for (int c = skip0; c < skip1; ++c) codes[c] = 0;
+  return rc;   /* max_err: the kept channels' (the copies add no new error) */
+}
+
 /* Asymmetric 4-bit group quantizer for values.
  * z = fp16_down(min x); s = fp16_up((max x - z) / 15);
  * code = clamp(rint((x - z) / s), 0, 15) (s = 0 -> 0);
@@ -247,16 +272,24 @@ range:
 /* V codes: per token d/2 bytes; channel c (group g = c/32, w = c%32) sits in */
 /*   byte (w/4)*(2*nb) + 2*g + (w%4)/2, low nibble for even c, unsigned.     */
 /* eta is a separate fp32 array [num_pages][Hkv].                             */
+/* With outlier extraction (outliers = 1) the block ends in an outlier       */
+/* section: [K chunk index u8 [16]][V chunk index u8 [16]]                   */
+/* [K chunk values fp16 [16][4]][V chunk values fp16 [16][4]]; index 0xFF =  */
+/* no outlier in that token.                                                  */
 /* ------------------------------------------------------------------------ */
 typedef struct {
-  int32_t d, hkv, kbits, kgroup, krotate, vbits, vgroup, num_pages;
+  int32_t d, hkv, kbits, kgroup, krotate, vbits, vgroup, num_pages, outliers;
 } oc_cfg;
+
+#define OC_NO_OUTLIER 0xFFu
+#define OC_OUT_BYTES (2 * OC_PAGE + 2 * OC_PAGE * 4 * 2)
 
 static int oc_cfg_ok(const oc_cfg* c) {
   if (!c || (c->d != 64 && c->d != 128) || c->hkv <= 0 || c->num_pages < 0) return 0;
   if (c->kbits != 8 && c->kbits != 4) return 0;
   if (c->kgroup <= 0 || c->kgroup % 32 || c->d % c->kgroup) return 0;
   if (c->vbits != 4 || c->vgroup != 32) return 0;
+  if (c->outliers != 0 && c->outliers != 1) return 0;
   return 1;
 }
 
@@ -265,9 +298,61 @@ static int64_t oc_vcode_bytes(const oc_cfg* c) { return (int64_t)OC_PAGE * c->d 
 static int64_t oc_kscale_bytes(const oc_cfg* c) { return (int64_t)OC_PAGE * (c->d / c->kgroup) * 2; }
 static int64_t oc_vmeta_bytes(const oc_cfg* c) { return (int64_t)OC_PAGE * (c->d / 32) * 4; }
 
+static int64_t oc_out_off(const oc_cfg* c) {
+  return oc_kcode_bytes(c) + oc_vcode_bytes(c) + oc_kscale_bytes(c) + oc_vmeta_bytes(c);
+}
+
 int64_t oc_block_bytes(const oc_cfg* c) {
   if (!oc_cfg_ok(c)) return -1;
-  return oc_kcode_bytes(c) + oc_vcode_bytes(c) + oc_kscale_bytes(c) + oc_vmeta_bytes(c);
+  return oc_out_off(c) + (c->outliers ? OC_OUT_BYTES : 0);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Median-multiplier outlier extraction (Med3x; "Hurwitz Quaternion          */
+/* Multiplicative Quantization for KV Cache Compression", Method 3): a      */
+/* vector is cut into 4-element chunks; a chunk whose norm exceeds 3x the    */
+/* median chunk norm is an outlier, kept in fp16 with a flag, and the bulk   */
+/* codec quantizes the rest.  Readings: the median is taken over the chunks */
+/* of one token's vector (K after rotation, or V); chunk norm =              */
+/* sqrt((x0*x0 + x1*x1) + (x2*x2 + x3*x3)) in fp32, each product rounded;    */
+/* the median of the even count of norms is the mean of the two middle       */
+/* ones, 0.5f * (a + b); at most one chunk per vector is extracted: the      */
+/* largest norm above 3.0f * median (ties: the lower chunk index).           */
+/* Returns the chunk index, or -1.                                            */
+/* ------------------------------------------------------------------------ */
+int oc_med3_chunk(const float* x, int d) {
+  int nc = d / 4;
+  float r[32], srt[32];
+  for (int i = 0; i < nc; ++i) {
+    float a = x[4 * i] * x[4 * i], b = x[4 * i + 1] * x[4 * i + 1];
+    float e = x[4 * i + 2] * x[4 * i + 2], f = x[4 * i + 3] * x[4 * i + 3];
+    r[i] = sqrtf((a + b) + (e + f));
+    if (isnan(r[i])) return -1;   /* a NaN input: no extraction (the bulk codec flags it) */
+    srt[i] = r[i];
+  }
+  for (int i = 1; i < nc; ++i)   /* insertion sort, ascending */
+    for (int j = i; j > 0 && srt[j - 1] > srt[j]; --j) {
+      float t = srt[j]; srt[j] = srt[j - 1]; srt[j - 1] = t;
+    }
+  float med = 0.5f * (srt[nc / 2 - 1] + srt[nc / 2]);
+  float thr = 3.0f * med;
+  int best = -1;
+  for (int i = 0; i < nc; ++i)
+    if (r[i] > thr && (best < 0 || r[i] > r[best])) best = i;
+  return best;
+}
+
+/* binary16 round-to-nearest, ties to the even pattern (the directed
+ * neighbours from oc_f16_round, then the nearer one). */
+uint16_t oc_f16_rn(float xf) {
+  uint16_t dn = oc_f16_round(xf, 0), up = oc_f16_round(xf, 1);
+  if (dn == up) return dn;
+  double x = (double)xf, vd = oc_f16_value(dn), vu = oc_f16_value(up);
+  if (isinf(vu) || isinf(vd)) return isinf(vu) ? dn : up;
+  double ed = x - vd, eu = vu - x;
+  if (ed < eu) return dn;
+  if (eu < ed) return up;
+  return (dn & 1u) == 0 ? dn : up;
 }
 
 static int64_t oc_k8_byte(int d, int slot, int ch) {
@@ -298,12 +383,53 @@ static void oc_wr16(uint8_t* p, uint16_t v) { p[0] = (uint8_t)(v & 0xFF); p[1] =
 
 /* Quantize one token of one kv head into slot `slot` of block `blk`.
  * x_k, x_v: fp32 [d]; returns the token's fp32 max value error through *verr. */
+/* Channels [skip0, skip1) of the group [g0, g0 + n) that lie in the chunk
+ * [4*chunk, 4*chunk + 4) (an empty range when chunk < 0 or no overlap). */
+static void oc_chunk_in_group(int chunk, int g0, int n, int* skip0, int* skip1) {
+  *skip0 = *skip1 = 0;
+  if (chunk < 0) return;
+  int a = 4 * chunk - g0, b = a + 4;
+  if (a < 0) a = 0;
+  if (b > n) b = n;
+  if (a < b) { *skip0 = a; *skip1 = b; }
+}
+
 static int oc_quantize_token(const oc_cfg* c, uint8_t* blk, int slot, const float* xk_in,
                              const float* xv, const int8_t* sigma, float* verr) {
   int d = c->d, rc = OC_OK;
   float xk_rot[128];
   const float* xk = xk_in;
   if (c->krotate) { oc_rotate(xk_in, sigma, d, xk_rot); xk = xk_rot; }
+  /* outlier chunks (Med3x), at most one per vector, kept in fp16 */
+  int ck = -1, cv = -1;
+  float out_err = 0.0f;
+  if (c->outliers) {
+    ck = oc_med3_chunk(xk, d);
+    cv = oc_med3_chunk(xv, d);
+    uint8_t* os = blk + oc_out_off(c);
+    os[slot] = ck < 0 ? OC_NO_OUTLIER : (uint8_t)ck;
+    os[OC_PAGE + slot] = cv < 0 ? OC_NO_OUTLIER : (uint8_t)cv;
+    for (int i = 0; i < 4; ++i) {
+      uint16_t hk = 0, hv = 0;
+      if (ck >= 0) {
+        float x = xk[4 * ck + i];
+        if (!isfinite(x) || fabsf(x) > 65504.0f) rc = OC_ERR_RANGE;
+        else hk = oc_f16_rn(x);
+      }
+      if (cv >= 0) {
+        float x = xv[4 * cv + i];
+        if (!isfinite(x) || fabsf(x) > 65504.0f) {
+          rc = OC_ERR_RANGE;
+        } else {
+          hv = oc_f16_rn(x);
+          float err = fabsf(x - (float)oc_f16_value(hv));
+          if (err > out_err) out_err = err;
+        }
+      }
+      oc_wr16(os + 2 * OC_PAGE + (slot * 4 + i) * 2, hk);
+      oc_wr16(os + 2 * OC_PAGE + OC_PAGE * 8 + (slot * 4 + i) * 2, hv);
+    }
+  }
   /* keys */
   int Q = c->kbits == 8 ? 127 : 7;
   uint8_t* kcodes = blk;
@@ -311,7 +437,9 @@ static int oc_quantize_token(const oc_cfg* c, uint8_t* blk, int slot, const floa
   for (int g = 0; g < d / c->kgroup; ++g) {
     int8_t codes[128];
     uint16_t sb;
-    int r = oc_quantize_sym(xk + g * c->kgroup, c->kgroup, Q, &sb, codes);
+    int s0, s1;
+    oc_chunk_in_group(ck, g * c->kgroup, c->kgroup, &s0, &s1);
+    int r = oc_quantize_sym_skip(xk + g * c->kgroup, c->kgroup, Q, s0, s1, &sb, codes);
     if (r != OC_OK) rc = r;
     oc_wr16(kscales + ((int64_t)slot * (d / c->kgroup) + g) * 2, sb);
     for (int i = 0; i < c->kgroup; ++i) {
@@ -327,12 +455,14 @@ static int oc_quantize_token(const oc_cfg* c, uint8_t* blk, int slot, const floa
   /* values */
   uint8_t* vrow = blk + oc_kcode_bytes(c) + (int64_t)slot * (d / 2);
   uint8_t* vmeta = blk + oc_kcode_bytes(c) + oc_vcode_bytes(c) + oc_kscale_bytes(c);
-  float e = 0.0f;
+  float e = out_err;
   for (int g = 0; g < d / 32; ++g) {
     uint8_t codes[32];
     uint16_t sb, zb;
     float ge;
-    int r = oc_quantize_asym(xv + g * 32, 32, &sb, &zb, codes, &ge);
+    int s0, s1;
+    oc_chunk_in_group(cv, g * 32, 32, &s0, &s1);
+    int r = oc_quantize_asym_skip(xv + g * 32, 32, s0, s1, &sb, &zb, codes, &ge);
     if (r != OC_OK) rc = r;
     oc_wr16(vmeta + ((int64_t)slot * (d / 32) + g) * 4, sb);
     oc_wr16(vmeta + ((int64_t)slot * (d / 32) + g) * 4 + 2, zb);
@@ -392,7 +522,7 @@ int oc_append(const oc_cfg* c, uint8_t* pool, float* eta, const void* k, const v
 /* Dequantized view of one token of one kv head, read back from the layout. */
 static void oc_read_token(const oc_cfg* c, const uint8_t* blk, int slot, double* khat,
                           double* kscale, double* vhat, double* vs, double* vz,
-                          double* vtop) {
+                          double* vtop, int* kchunk, int* vchunk) {
   int d = c->d, ngk = d / c->kgroup;
   const uint8_t* kcodes = blk;
   const uint8_t* vrow = blk + oc_kcode_bytes(c) + (int64_t)slot * (d / 2);
@@ -420,6 +550,21 @@ static void oc_read_token(const oc_cfg* c, const uint8_t* blk, int slot, double*
   for (int ch = 0; ch < d; ++ch) {
     unsigned code = oc_get_nibble(vrow, oc_v4_byte(d, ch), ch);
     vhat[ch] = vs[ch / 32] * (double)code + vz[ch / 32];   /* exact in fp64 */
+  }
+  *kchunk = *vchunk = -1;
+  if (c->outliers) {   /* the fp16 outlier chunks, in place of their codes */
+    const uint8_t* os = blk + oc_out_off(c);
+    if (os[slot] != OC_NO_OUTLIER) {
+      *kchunk = os[slot];
+      for (int i = 0; i < 4; ++i)
+        khat[4 * *kchunk + i] = oc_f16_value(oc_rd16(os + 2 * OC_PAGE + (slot * 4 + i) * 2));
+    }
+    if (os[OC_PAGE + slot] != OC_NO_OUTLIER) {
+      *vchunk = os[OC_PAGE + slot];
+      for (int i = 0; i < 4; ++i)
+        vhat[4 * *vchunk + i] =
+            oc_f16_value(oc_rd16(os + 2 * OC_PAGE + OC_PAGE * 8 + (slot * 4 + i) * 2));
+    }
   }
 }
 
@@ -459,24 +604,41 @@ static void oc_row_terms(const oc_cfg* c, const uint8_t* pool, const float* eta,
   double vtop_max[4], vz_min[4], eta_max = 0.0;
   for (int g = 0; g < ngv; ++g) { vtop_max[g] = -INFINITY; vz_min[g] = INFINITY; }
   double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+  int kc, vc;
   for (int j = 0; j < n; ++j) {
     int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
     const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
-    oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+    oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop, &kc, &vc);
     double dot = 0.0, smax = 0.0, qs = 0.0;
     for (int ch = 0; ch < d; ++ch) dot += (double)qp[ch] * khat[ch];
     for (int g = 0; g < ngk; ++g) {
       qs += qn1[g] * ks[g] / 2.0;
       if (ks[g] > smax) smax = ks[g];
     }
+    /* an fp16 outlier chunk: |k - k^| <= 2^-11 |k^| + 2^-25 per channel (half an
+     * fp16 ulp), and, for rotated keys, its norm joins the rotation allowance */
+    double qo = 0.0, kon = 0.0;
+    if (kc >= 0)
+      for (int i = 0; i < 4; ++i) {
+        double kx = khat[4 * kc + i];
+        qo += fabs((double)qp[4 * kc + i]) * (ldexp(fabs(kx), -11) + ldexp(1.0, -25));
+        kon += kx * kx;
+      }
     z[j] = sc * dot;
-    dl[j] = OC_KAPPA * sc * (qs + rot * smax);
+    dl[j] = OC_KAPPA * sc * (qs + rot * smax + qo +
+                             (c->krotate ? OC_ROT_SLACK * qn2 * sqrt(kon) : 0.0));
     et[j] = (double)eta[(int64_t)page * c->hkv + kv];
     if (et[j] > eta_max) eta_max = et[j];
     for (int g = 0; g < ngv; ++g) {
       if (vtop[g] > vtop_max[g]) vtop_max[g] = vtop[g];
       if (vz[g] < vz_min[g]) vz_min[g] = vz[g];
     }
+    if (vc >= 0)   /* the stored outlier values lie outside [z, z + 15 s] */
+      for (int i = 0; i < 4; ++i) {
+        int g = (4 * vc + i) / 32;
+        if (vhat[4 * vc + i] > vtop_max[g]) vtop_max[g] = vhat[4 * vc + i];
+        if (vhat[4 * vc + i] < vz_min[g]) vz_min[g] = vhat[4 * vc + i];
+      }
   }
   double range = 0.0;
   for (int g = 0; g < ngv; ++g)
@@ -547,11 +709,12 @@ int oc_decode(const oc_cfg* c, const uint8_t* pool, const float* eta, const void
         for (int j = 0; j < n; ++j) l += exp(z[j] - m);
         double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
         double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+        int kc, vc;
         for (int j = 0; j < n; ++j) {
           double p = exp(z[j] - m) / l;
           int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
           const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
-          oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+          oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop, &kc, &vc);
           for (int ch = 0; ch < d; ++ch) o[ch] += p * vhat[ch];
           A += p * expm1(dl[j]);
           B += p * exp(-dl[j]);
@@ -664,6 +827,7 @@ int oc_decode_promote_values(const oc_cfg* c, const uint8_t* pool, const float* 
         }
         double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
         double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+        int kc, vc;
         for (int j = 0; j < n; ++j) {
           double p = exp(z[j] - m) / l;
           if (prom[j / OC_PAGE]) {
@@ -673,7 +837,7 @@ int oc_decode_promote_values(const oc_cfg* c, const uint8_t* pool, const float* 
           } else {
             int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
             const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
-            oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+            oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop, &kc, &vc);
             for (int ch = 0; ch < d; ++ch) o[ch] += p * vhat[ch];
             Ev += p * et[j];
           }
@@ -891,6 +1055,7 @@ int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, c
         /* output and bound */
         double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
         double khat[128], ks[4], vhat[128], vs[4], vz[4], vtop[4];
+        int kc, vc;
         for (int j = 0; j < n; ++j) {
           if (vp[j / OC_PAGE]) {
             oc_load_vec(v_orig, kv_is_f32, b * seq_stride + kv * head_stride + j * tok_stride,
@@ -899,7 +1064,7 @@ int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, c
           } else {
             int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
             const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
-            oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop);
+            oc_read_token(c, blk, j % OC_PAGE, khat, ks, vhat, vs, vz, vtop, &kc, &vc);
             for (int ch = 0; ch < d; ++ch) o[ch] += p[j] * vhat[ch];
             Ev += p[j] * et[j];
           }

@@ -128,8 +128,8 @@ def test_bound_terms_match_hand_worked(oracle_lib, case):
 # the bound's derivation; every replacement must change the source.
 MUTANTS = [
     ("delta_without_half", "qs += qn1[g] * ks[g] / 2.0;", "qs += qn1[g] * ks[g];"),
-    ("delta_without_kappa", "dl[j] = OC_KAPPA * sc * (qs + rot * smax);",
-     "dl[j] = sc * (qs + rot * smax);"),
+    ("delta_without_kappa", "dl[j] = OC_KAPPA * sc * (qs + rot * smax + qo +",
+     "dl[j] = sc * (qs + rot * smax + qo +"),
     ("bound_without_kappa", "double bd = OC_KAPPA * (ekey + Ev);", "double bd = ekey + Ev;"),
     ("ekey_single_eta", "double ekey = tv * (range + 2.0 * eta_max);",
      "double ekey = tv * (range + eta_max);"),
