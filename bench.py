@@ -48,8 +48,9 @@ SPEC_HBM_GBS = 8000.0     # nominal B200 HBM3e bandwidth (context for frac_vs_sp
 # blocks whose estimated share of the value error exceeds 1e-4, and a ranking
 # check that tolerates exact log-mass inversions up to 0.1
 LADDER = {"tau_cov": 0.995, "v_tol": 1e-4, "rank_tol": 0.1}
-DECODE_SRC = os.path.join(ROOT, "quantized_decode_attention_kvq_b200", "csrc",
-                          "decode_attention.cu")
+# the sources of the decode kernel (and of the token codec its fused append runs)
+DECODE_SRCS = [os.path.join(ROOT, "quantized_decode_attention_kvq_b200", "csrc", f)
+               for f in ("decode_kernel.cuh", "quantize_token.cuh", "kvq_device.cuh")]
 
 
 def _workload_desc(wl) -> str:
@@ -73,13 +74,22 @@ def _peaks():
 TRAFFIC_JSON = os.path.join(ROOT, "profiles", "decode_attention_traffic.json")
 
 
+def decode_source_hash() -> str:
+    """First 16 hex digits of the sha256 of the decode kernel's sources."""
+    h = hashlib.sha256()
+    for p in DECODE_SRCS:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def _traffic_record(workload: str, two_calls: bool):
     """DRAM bytes per decode launch from the committed ncu record
     (profiles/decode_attention_traffic.json) for this workload and the fused
     step's launch, if it was taken on the current decode kernel source."""
     if two_calls or not os.path.exists(TRAFFIC_JSON):
         return None
-    src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
+    src_hash = decode_source_hash()
     with open(TRAFFIC_JSON) as f:
         recs = json.load(f).get("records", [])
     for r in recs:

@@ -55,6 +55,23 @@
  *   of (max x - z)/15, code = rint((x - z)/s) in [0, 15].
  *   eta[page][kv_head] = max over the block's tokens of |v - fmaf(code, s, z)|,
  *   rounded up by one fp32 ulp.
+ *
+ * Outlier extraction (outliers = 1; the median-multiplier rule of "Hurwitz
+ * Quaternion Multiplicative Quantization for KV Cache Compression", Method 3):
+ *   a token's vector (K after the rotation, if any, and V) is cut into
+ *   4-channel chunks; the chunk with the largest norm
+ *   sqrt((x0*x0 + x1*x1) + (x2*x2 + x3*x3)) (fp32, each operation rounded)
+ *   above 3 * median of the vector's chunk norms (the median of the even
+ *   count is 0.5 * (a + b) of the two middle norms) is kept in fp16 (round to
+ *   nearest; ties: the lower chunk index; no extraction if a norm is NaN).
+ *   Its channels get code 0 and take no part in their group's scale, zero or
+ *   error; eta also covers the fp16 rounding of the extracted values.  The
+ *   block then ends in a 288-byte outlier section:
+ *     [K chunk index u8 [16]][V chunk index u8 [16]]
+ *     [K chunk values fp16 [16][4]][V chunk values fp16 [16][4]]
+ *   index 0xFF = no extraction in that token (its values are then 0).
+ *   An extracted value that is not finite or above 65504 in magnitude is
+ *   stored as 0 and sets KVQ_ERR_RANGE.
  */
 #ifndef KVQ_H_
 #define KVQ_H_
@@ -105,6 +122,7 @@ typedef struct kvq_cache {
   float* v_eta;            /* device, [num_pages][num_kv_heads]; zero before a page's first append */
   const int8_t* rot_signs; /* device, head_dim entries of +1/-1; required iff k_rotate */
   int32_t* error_word;     /* device, one int32 kernels set to a kvq_status on error; may be NULL */
+  int32_t outliers;        /* 1: outlier extraction (see the layout above); 0: none */
 } kvq_cache;
 
 /* Bytes of one (page, kv head) block, and of the whole pool; 0 if the cache

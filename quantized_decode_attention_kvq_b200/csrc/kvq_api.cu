@@ -59,12 +59,15 @@ int check_cache(const kvq_cache* c) {
   if (c->num_pages < 0) return fail(KVQ_ERR_INVALID_ARG, "num_pages < 0");
   if (c->k_rotate != 0 && c->k_rotate != 1) return fail(KVQ_ERR_INVALID_ARG, "k_rotate not 0/1");
   if (c->k_rotate && !c->rot_signs) return fail(KVQ_ERR_INVALID_ARG, "k_rotate needs rot_signs");
+  if (c->outliers != 0 && c->outliers != 1) return fail(KVQ_ERR_INVALID_ARG, "outliers not 0/1");
   if (!c->pool || !c->v_eta) return fail(KVQ_ERR_INVALID_ARG, "pool or v_eta is NULL");
   if (!aligned16(c->pool)) return fail(KVQ_ERR_INVALID_ARG, "pool not 16-byte aligned");
   return KVQ_OK;
 }
 
-BlockLayout layout_of(const kvq_cache* c) { return BlockLayout{c->head_dim, c->k_bits, c->k_group}; }
+BlockLayout layout_of(const kvq_cache* c) {
+  return BlockLayout{c->head_dim, c->k_bits, c->k_group, c->outliers};
+}
 
 float rot_constant(int d) { return (float)(1.0 / std::sqrt((double)d)); }
 
@@ -139,7 +142,7 @@ constexpr int kMaxPagesPerSplit = 256;
 // split) CTAs; long contexts cap the pages of one split so a ragged batch
 // spreads over several waves.
 int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
-  DecodeVariant v = select_decode_kernel(c->head_dim, c->k_bits, c->k_group);
+  DecodeVariant v = select_decode_kernel(c->head_dim, c->k_bits, c->k_group, c->outliers);
   if (!v.kernel) return fail(KVQ_ERR_UNSUPPORTED, "no decode kernel for this codec");
   DeviceInfo di;
   int rc = device_info(&di, nullptr);
@@ -202,7 +205,8 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
     return fail(KVQ_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", ws_bytes,
                 plan.total());
   if (!aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");
-  DecodeVariant v = select_decode_kernel(cache->head_dim, cache->k_bits, cache->k_group);
+  DecodeVariant v = select_decode_kernel(cache->head_dim, cache->k_bits, cache->k_group,
+                                         cache->outliers);
   DecodeArgs a;
   a.pool = static_cast<const uint8_t*>(cache->pool);
   a.eta = cache->v_eta;
@@ -276,6 +280,7 @@ size_t kvq_block_bytes(const kvq_cache* cache) {
     return 0;
   if (cache->k_group != 32 && cache->k_group != 64 && cache->k_group != 128) return 0;
   if (cache->head_dim % cache->k_group || cache->v_bits != 4 || cache->v_group != 32) return 0;
+  if (cache->outliers != 0 && cache->outliers != 1) return 0;
   return (size_t)layout_of(cache).bytes();
 }
 
@@ -322,7 +327,7 @@ int kvq_quantize_append(const kvq_cache* cache, const void* k, const void* v, in
   a.start_pos = start_pos;
   a.page_table = page_table;
   a.rot_c = rot_constant(cache->head_dim);
-  cudaError_t e = launch_append(a, cache->head_dim, cache->k_bits, cache->k_group,
+  cudaError_t e = launch_append(a, cache->head_dim, cache->k_bits, cache->k_group, cache->outliers,
                                 reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
   return KVQ_OK;
@@ -641,8 +646,8 @@ extern "C" {
 
 size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs, int32_t num_queries,
                               int32_t num_q_heads, int32_t max_pages_per_seq) {
-  if (check_cache(cache) || num_seqs < 0 || num_queries < 1 || num_q_heads < 1 ||
-      max_pages_per_seq < 1 || max_pages_per_seq > kAdMaxPages)
+  if (check_cache(cache) || cache->outliers || num_seqs < 0 || num_queries < 1 ||
+      num_q_heads < 1 || max_pages_per_seq < 1 || max_pages_per_seq > kAdMaxPages)
     return 0;
   const int64_t units = (int64_t)num_seqs * cache->num_kv_heads;
   const int64_t slots = (int64_t)num_seqs * num_queries * num_q_heads;
@@ -681,6 +686,9 @@ int kvq_adaptive_precision(const kvq_cache* cache, const void* k_orig_host,
   if (num_flagged) *num_flagged = 0;
   int rc = check_cache(cache);
   if (rc) return rc;
+  if (cache->outliers)
+    return fail(KVQ_ERR_UNSUPPORTED, "the adaptive-precision ladder reads caches without "
+                "outlier extraction only");
   if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad orig_dtype");
   if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad q_dtype");
   if (num_seqs < 0 || num_queries < 1 || num_q_heads < 1 || max_pages_per_seq < 1 ||

@@ -25,9 +25,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 // suspends for a hardware-defined time, so this is on the order of seconds)
 constexpr uint32_t kSpinLimit = 1u << 22;
 
+// Outlier section of a block (outlier extraction): chunk indices of K and V,
+// then the chunks' fp16 values, [16][4] each.
+constexpr int kOutBytes = 2 * kPage + 2 * kPage * 4 * 2;
+constexpr uint8_t kNoOutlier = 0xFF;
+
 // Byte layout of one (page, kv head) block of the quantized pool.
 struct BlockLayout {
   int d, kbits, kgroup;
+  int out = 0;  // 1: the block ends in the outlier section
   __host__ __device__ int ngk() const { return d / kgroup; }
   __host__ __device__ int nb() const { return d / 32; }
   __host__ __device__ int k_row() const { return d * kbits / 8; }
@@ -39,7 +45,8 @@ struct BlockLayout {
   __host__ __device__ int v_off() const { return k_bytes(); }
   __host__ __device__ int ks_off() const { return k_bytes() + v_bytes(); }
   __host__ __device__ int vm_off() const { return ks_off() + ks_bytes(); }
-  __host__ __device__ int bytes() const { return vm_off() + vm_bytes(); }
+  __host__ __device__ int out_off() const { return vm_off() + vm_bytes(); }
+  __host__ __device__ int bytes() const { return out_off() + (out ? kOutBytes : 0); }
 };
 
 __device__ __forceinline__ void set_error(int32_t* word, int code) {

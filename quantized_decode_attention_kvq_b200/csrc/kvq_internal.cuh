@@ -163,8 +163,11 @@ cudaError_t launch_adaptive_correct(const AdArgs& a, int d, int kbits, int kgrou
 cudaError_t launch_adaptive_finish(const AdArgs& a, int d, cudaStream_t s);
 int adaptive_select_smem(int max_pages, int d);
 
-cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, cudaStream_t s);
-DecodeVariant select_decode_kernel(int d, int kbits, int kgroup);
+cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, int out,
+                          cudaStream_t s);
+// out: the cache's outlier extraction (0 or 1)
+DecodeVariant select_decode_kernel(int d, int kbits, int kgroup, int out);
+DecodeVariant select_decode_kernel_med3(int d, int kbits, int kgroup);
 int decode_threads();
 // the recompute (and, when an item was split, the merge) on `stream`
 cudaError_t launch_fallback(const FbArgs& a, int d, cudaStream_t stream);

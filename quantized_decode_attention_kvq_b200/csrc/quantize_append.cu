@@ -9,16 +9,19 @@
 // E_val) raised as each token lands in its block.
 //
 // One warp quantizes one (token, kv head) with quantize_token_warp
-// (quantize_token.cuh), after finding the token's page through the page table.
+// (quantize_token.cuh), after finding the token's page through the page table;
+// with outlier extraction, the median-multiplier chunk of K and of V goes to
+// the block's outlier section first ("Hurwitz Quaternion Multiplicative
+// Quantization for KV Cache Compression", Method 3).
 #include "kvq_internal.cuh"
 #include "quantize_token.cuh"
 
 namespace kvq {
 
-template <int D, int KB, int KG>
+template <int D, int KB, int KG, bool OUT>
 __global__ void __launch_bounds__(256) quantize_append_kernel(const AppendArgs a) {
   constexpr int E = D / 32;             // channels per lane
-  const BlockLayout L{D, KB, KG};
+  const BlockLayout L{D, KB, KG, OUT ? 1 : 0};
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int64_t total = (int64_t)a.num_seqs * a.num_tokens * a.hkv;
@@ -50,15 +53,17 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(const AppendArgs a
   }
   const int slot = pos % kPage;
   uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
-  quantize_token_warp<D, KB, KG>(xk, xv, blk, slot, a.eta + (int64_t)page * a.hkv + h, a.signs,
+  quantize_token_warp<D, KB, KG, OUT>(xk, xv, blk, slot, a.eta + (int64_t)page * a.hkv + h, a.signs,
                                  a.rot_c, a.err, lane);
 }
 
 using AppendKernel = void (*)(const AppendArgs);
 
-AppendKernel select_append_kernel(int d, int kbits, int kgroup) {
-#define KVQ_APPEND_CASE(D_, KB_, KG_) \
-  if (d == D_ && kbits == KB_ && kgroup == KG_) return quantize_append_kernel<D_, KB_, KG_>;
+AppendKernel select_append_kernel(int d, int kbits, int kgroup, int out) {
+#define KVQ_APPEND_CASE(D_, KB_, KG_)                                                \
+  if (d == D_ && kbits == KB_ && kgroup == KG_)                                      \
+    return out ? quantize_append_kernel<D_, KB_, KG_, true>                          \
+               : quantize_append_kernel<D_, KB_, KG_, false>;
   KVQ_APPEND_CASE(128, 8, 128)
   KVQ_APPEND_CASE(128, 8, 64)
   KVQ_APPEND_CASE(128, 8, 32)
@@ -73,9 +78,9 @@ AppendKernel select_append_kernel(int d, int kbits, int kgroup) {
   return nullptr;
 }
 
-cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup,
+cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, int out,
                           cudaStream_t stream) {
-  AppendKernel k = select_append_kernel(d, kbits, kgroup);
+  AppendKernel k = select_append_kernel(d, kbits, kgroup, out);
   if (!k) return cudaErrorInvalidValue;
   const int64_t items = (int64_t)a.num_seqs * a.num_tokens * a.hkv;
   if (items == 0) return cudaSuccess;

@@ -53,7 +53,7 @@ class kvq_cache(ctypes.Structure):
                 ("k_rotate", ctypes.c_int32), ("v_bits", ctypes.c_int32),
                 ("v_group", ctypes.c_int32), ("pool", ctypes.c_void_p),
                 ("v_eta", ctypes.c_void_p), ("rot_signs", ctypes.c_void_p),
-                ("error_word", ctypes.c_void_p)]
+                ("error_word", ctypes.c_void_p), ("outliers", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -284,9 +284,10 @@ class PagedCache:
 
     def __init__(self, num_kv_heads: int, head_dim: int, num_pages: int, k_bits: int = 8,
                  k_group: int = 128, k_rotate: bool = False, rot_signs=None, v_bits: int = 4,
-                 v_group: int = 32, device="cuda"):
+                 v_group: int = 32, outliers: bool = False, device="cuda"):
         self.desc = kvq_cache(num_kv_heads, head_dim, PAGE_SIZE, num_pages, k_bits, k_group,
-                              int(bool(k_rotate)), v_bits, v_group, None, None, None, None)
+                              int(bool(k_rotate)), v_bits, v_group, None, None, None, None,
+                              int(bool(outliers)))
         bb = kvq_block_bytes(self.desc)
         if bb == 0:
             raise KvqError(KVQ_ERR_UNSUPPORTED, "kvq_block_bytes")

@@ -27,15 +27,16 @@ def to_torch(x: np.ndarray, device="cuda") -> torch.Tensor:
     return t.to(device)
 
 
-def gpu_cache(inp, num_pages=None):
+def gpu_cache(inp, num_pages=None, outliers=False):
     from quantized_decode_attention_kvq_b200 import kvq
     wl = inp.wl
     return kvq.PagedCache(wl.num_kv_heads, wl.head_dim, num_pages or inp.num_pages,
                           k_bits=wl.k_bits, k_group=wl.k_group, k_rotate=wl.k_rotate,
-                          rot_signs=inp.rot_signs)
+                          rot_signs=inp.rot_signs, outliers=outliers)
 
 
-def run_gpu(inp, k=None, v=None, q=None, tau=None, page_table=None, bound_only=False):
+def run_gpu(inp, k=None, v=None, q=None, tau=None, page_table=None, bound_only=False,
+            outliers=False):
     """Append the whole context and decode every row on the GPU."""
     wl = inp.wl
     if k is None:
@@ -43,7 +44,7 @@ def run_gpu(inp, k=None, v=None, q=None, tau=None, page_table=None, bound_only=F
     if q is None:
         q = inp.q()
     pt = inp.page_table if page_table is None else page_table
-    c = gpu_cache(inp)
+    c = gpu_cache(inp, outliers=outliers)
     kd, vd = to_torch(k), to_torch(v)
     ptd = torch.from_numpy(pt).cuda()
     sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
@@ -61,9 +62,9 @@ def run_gpu(inp, k=None, v=None, q=None, tau=None, page_table=None, bound_only=F
     return res
 
 
-def oracle_pool(inp, k, v):
+def oracle_pool(inp, k, v, outliers=False):
     wl = inp.wl
-    c = oracle_cache(inp)
+    c = oracle_cache(inp, outliers=outliers)
     rc = c.append(k, v, inp.page_table, np.zeros(wl.num_seqs, np.int32),
                   valid=np.array(inp.seq_lens, np.int32))
     assert rc == 0

@@ -26,10 +26,11 @@ def small(name, seed=0, **kw):
     return synth.make(name, seed, **ov)
 
 
-def oracle_cache(inp):
+def oracle_cache(inp, outliers=False):
     wl = inp.wl
     return oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
-                        k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+                        k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
+                        outliers=outliers)
 
 
 def run_oracle(inp, tau=None):

@@ -63,6 +63,18 @@ def test_block_bytes_match_the_layout(kvq):
     assert kvq.kvq_block_bytes(_desc(kvq, k_group=48)) == 0
 
 
+def test_outlier_section_size_and_checks(kvq):
+    # the outlier section: 16 + 16 chunk indices, 16 x 4 fp16 values for K and for V
+    for kw in ({}, dict(k_bits=4, k_group=32), dict(head_dim=64, k_group=32)):
+        plain = kvq.kvq_block_bytes(_desc(kvq, **kw))
+        ext = kvq.kvq_block_bytes(_desc(kvq, outliers=1, **kw))
+        assert ext == plain + 288 and ext % 16 == 0
+    assert kvq.kvq_block_bytes(_desc(kvq, outliers=2)) == 0
+    # the adaptive-precision ladder reads caches without extraction only
+    assert kvq.kvq_adaptive_work_size(_desc(kvq), 2, 1, 32, 4) > 0
+    assert kvq.kvq_adaptive_work_size(_desc(kvq, outliers=1), 2, 1, 32, 4) == 0
+
+
 def test_status_strings(kvq):
     assert kvq.status_string(0) == "KVQ_OK"
     assert kvq.status_string(-5) == "KVQ_ERR_TIMEOUT"
