@@ -53,6 +53,22 @@ DECODE_SRCS = [os.path.join(ROOT, "quantized_decode_attention_kvq_b200", "csrc",
                for f in ("decode_kernel.cuh", "quantize_token.cuh", "kvq_device.cuh")]
 
 
+def _variant(name: str):
+    """'llama8b' -> ('llama8b', False); 'llama8b+med3' -> ('llama8b', True): the
+    workload with Med3x outlier extraction in the cache."""
+    base, _, ext = name.partition("+")
+    if base not in synth.WORKLOADS or ext not in ("", "med3"):
+        raise SystemExit(f"unknown workload {name}")
+    return base, ext == "med3"
+
+
+def _describe(name: str) -> str:
+    base, outliers = _variant(name)
+    return _workload_desc(synth.WORKLOADS[base]) + (
+        ", Med3x outlier extraction (one 4-channel chunk of K and of V per token in fp16)"
+        if outliers else "")
+
+
 def _workload_desc(wl) -> str:
     ctx = f"ctx {wl.ctx}" if wl.ctx_min is None else f"ctx U[{wl.ctx_min},{wl.ctx}]"
     rot = "Hadamard-rotated " if wl.k_rotate else ""
@@ -268,7 +284,8 @@ def _packed(tensors):
 class GpuStep:
     """Device-resident workload and the raw C-ABI calls of one step."""
 
-    def __init__(self, wl_name: str, seed: int, replicas: int, two_calls: bool = False):
+    def __init__(self, wl_name: str, seed: int, replicas: int, two_calls: bool = False,
+                 outliers: bool = False):
         import ctypes
 
         import torch
@@ -292,7 +309,8 @@ class GpuStep:
         self.pt = torch.from_numpy(inp.page_table).cuda()
         self.sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
         base = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, k_bits=wl.k_bits,
-                              k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+                              k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
+                              outliers=outliers)
         zeros = torch.zeros(wl.num_seqs, dtype=torch.int32, device="cuda")
         base.append(self.kd, self.vd, self.pt, zeros, self.sl)
         torch.cuda.synchronize()
@@ -305,7 +323,8 @@ class GpuStep:
         self.caches = [base]
         for _ in range(replicas - 1):
             c = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, k_bits=wl.k_bits,
-                               k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+                               k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
+                               outliers=outliers)
             c.pool.copy_(base.pool)
             c.eta.copy_(base.eta)
             self.caches.append(c)
@@ -371,6 +390,7 @@ class GpuStep:
         self.launches_per_step = 2 if two_calls else 1
         # finite tau: flagged rows are recomputed exactly from pinned host originals
         self.fallback = None
+        self.ladder = None
         if math.isfinite(wl.tau):
             kh = (torch.from_numpy(k.view(np.int16)).view(torch.bfloat16) if k.dtype == np.uint16
                   else torch.from_numpy(k)).pin_memory()
@@ -383,7 +403,9 @@ class GpuStep:
                 sl_h=np.array(inp.seq_lens, np.int32),
                 staging=torch.empty(fb_bytes, dtype=torch.uint8, device="cuda"), rows=0, calls=0,
                 h2d=0)
-            # the adaptive-precision ladder run before the exact fallback
+        if self.fallback is not None and not outliers:
+            # the adaptive-precision ladder run before the exact fallback (it reads
+            # caches without outlier extraction)
             mp = self.pt.shape[1]
             rows = self.flags.numel()
             ad_host = kvq.kvq_adaptive_host_size(base.desc, B, mp)
@@ -623,16 +645,18 @@ def _e2e(st, args, world, ladder=False):
 
 def measure_workload(name, args, world, rank, local):
     """One workload's measurement on this rank: the device-timed value and the
-    decode kernel's roofline, the clocks, and the end-to-end number."""
+    decode kernel's roofline, the clocks, and the end-to-end number.  A name
+    ending in "+med3" is the workload with outlier extraction in the cache."""
     import torch
-    wl = synth.WORKLOADS[name]
-    reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl))))
+    base, outliers = _variant(name)
+    wl = synth.WORKLOADS[base]
+    reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl, outliers))))
     reps = min(reps, 8)
-    st = GpuStep(name, args.seed, reps, two_calls=args.two_calls)
+    st = GpuStep(base, args.seed, reps, two_calls=args.two_calls, outliers=outliers)
     ms_total, dec_ms, clocks = _timed_replay(st, args, world, rank, local)
     e2e_ms, h2d, d2h = _e2e(st, args, world)
     lad_ms = None
-    if st.fallback is not None:
+    if st.ladder is not None:
         fb_rows, fb_calls, fb_h2d = st.fallback["rows"], st.fallback["calls"], st.fallback["h2d"]
         lad_ms, _, _ = _e2e(st, args, world, ladder=True)
         lad_ms = _max_over_ranks(lad_ms, world)
@@ -647,7 +671,7 @@ def measure_workload(name, args, world, rank, local):
         "unit": UNIT,
         "ms_per_step": ms_step,
         "steps": args.steps,
-        "config": {"workload": _workload_desc(wl),
+        "config": {"workload": _describe(name),
                    "l2": f"inputs larger than L2: {reps} cache replicas of "
                          f"{st.cache_bytes / 1e6:.1f} MB rotated per step",
                    "step": ("kvq_quantize_append + kvq_decode_attention" if st.two_calls else
@@ -682,6 +706,7 @@ def measure_workload(name, args, world, rank, local):
             "note": "value times append + decode (graph); e2e adds the exact fallback of the "
                     "flagged rows (H2D of their originals + fp32 attention)"}
         rec["e2e"]["h2d_bytes_per_step"] = int(h2d + fb["h2d"] / max(1, fb["calls"]))
+    if st.ladder is not None:
         ad = st.ladder
         calls = max(1, ad["calls"])
         rec["ladder"] = {
@@ -742,9 +767,9 @@ def run_gpu(args):
         print(json.dumps(res), flush=True)
 
 
-def _cache_bytes_estimate(wl) -> int:
+def _cache_bytes_estimate(wl, outliers=False) -> int:
     per_tok = wl.head_dim * wl.k_bits // 8 + wl.head_dim // 2 + 2 * wl.head_dim // wl.k_group \
-        + 4 * wl.head_dim // 32
+        + 4 * wl.head_dim // 32 + (18 if outliers else 0)
     ctx = wl.ctx if wl.ctx_min is None else (wl.ctx + wl.ctx_min) // 2
     return wl.num_seqs * ctx * wl.num_kv_heads * per_tok
 
@@ -753,10 +778,12 @@ def _cache_bytes_estimate(wl) -> int:
 def _oracle_setup(workload: str, seed: int, kv_heads=None):
     """The oracle's cache of sequence 0 of the workload; rows of the given kv heads."""
     import oracle
-    inp = synth.make(workload, seed)
+    base, outliers = _variant(workload)
+    inp = synth.make(base, seed)
     wl = inp.wl
     c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
-                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
+                     outliers=outliers)
     k, v = inp.kv_seq(0)
     pt = inp.page_table[:1]
     sl = np.array(inp.seq_lens[:1], np.int32)
@@ -795,10 +822,12 @@ def _oracle_codec_and_dense(workload: str, seed: int):
     dense attention the fallback computes (every query row), in KV
     token-heads/s."""
     import oracle
-    inp = synth.make(workload, seed)
+    base, outliers = _variant(workload)
+    inp = synth.make(base, seed)
     wl = inp.wl
     c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
-                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs)
+                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
+                     outliers=outliers)
     k, v = inp.kv_seq(0)
     sl = np.array(inp.seq_lens[:1], np.int32)
     th = int(sl[0]) * wl.num_kv_heads
@@ -817,14 +846,14 @@ def cpu_baseline(workload: str, seed: int, seconds: float):
     cores (spawned, so no CUDA state is inherited), each for about `seconds`, and
     the same single-threaded on all kv heads."""
     import multiprocessing
-    wl = synth.WORKLOADS[workload]
+    wl = synth.WORKLOADS[_variant(workload)[0]]
     n = max(1, min(os.cpu_count() or 1, wl.num_kv_heads))
     with multiprocessing.get_context("spawn").Pool(n) as pool:
         res = pool.map(_oracle_worker, [(workload, seed, [h], seconds) for h in range(n)])
     value = sum(r[0] for r in res) / max(r[1] for r in res)
     th1, el1, reps1 = _oracle_decode_loop(workload, seed, None, seconds)
     codec, dense = _oracle_codec_and_dense(workload, seed)
-    inp = synth.make(workload, seed)
+    inp = synth.make(_variant(workload)[0], seed)
     return {"value": value, "unit": UNIT, "cores": n, "kind": "oracle",
             "single_core_value": th1 / el1,
             "single_core_codec_value": codec, "single_core_dense_value": dense,
@@ -839,7 +868,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = synth.WORKLOADS[args.workload]
+    wl = synth.WORKLOADS[_variant(args.workload)[0]]
     inp, c, q, pt, sl, mask, nh = _oracle_setup(args.workload, args.seed, [0])
     th = int(sl.sum()) * nh
     for _ in range(args.warmup):
@@ -864,7 +893,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64 (attention, bound), f32 (codec)",
         "data": "synthetic",
-        "config": {"workload": _workload_desc(wl),
+        "config": {"workload": _describe(args.workload),
                    "sample": f"each step: kv head 0 of sequence 0 ({int(sl[0])} tokens, "
                              f"{wl.group * wl.num_queries} query rows) of the workload"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -879,14 +908,16 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="llama8b",
+                    choices=sorted(synth.WORKLOADS) + [w + "+med3" for w in sorted(synth.WORKLOADS)])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--also", default=None,
                     help="comma-separated workloads measured in the same run and reported "
-                         "under 'workloads' (default: long128k,serving with llama8b; 'none')")
+                         "under 'workloads'; a '+med3' suffix adds outlier extraction to the "
+                         "cache (default: long128k,serving,llama8b+med3 with llama8b; 'none')")
     ap.add_argument("--two-calls", action="store_true",
                     help="step = kvq_quantize_append + kvq_decode_attention (default: the fused "
                          "kvq_decode_attention_append)")
@@ -894,7 +925,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.also is None:
-        args.also = "long128k,serving" if args.workload == "llama8b" else "none"
+        args.also = "long128k,serving,llama8b+med3" if args.workload == "llama8b" else "none"
     if args.impl == "reference":
         run_reference(args)
     else:

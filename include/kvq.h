@@ -174,8 +174,14 @@ KVQ_API size_t kvq_workspace_size(const kvq_cache* cache, int32_t num_seqs, int3
  * context is cut to the page table; KVQ_ERR_INVALID_ARG).  Every query row of
  * that (sequence, kv head) then gets bound = +INFINITY and flag = 1 whatever
  * tau is, so kvq_fallback_exact recomputes it; out holds attention over the
- * pages that were read.  workspace: device, >= kvq_workspace_size() bytes,
- * 16-byte aligned.  Asynchronous. */
+ * pages that were read.  With outlier extraction (cache->outliers = 1) the
+ * scores use the extracted key chunks' fp16 values (against q' in fp32) and
+ * Delta_j adds, per extracted channel, |q'_c| (2^-11 |k16_c| + 2^-25) (half
+ * an fp16 ulp; for rotated keys also s*2^-16*|q'|_2 times the chunk's norm,
+ * all times kappa * softmax scale); the outputs use the extracted value
+ * chunks' fp16 values, and the value range of each group widens to them.
+ * workspace: device, >= kvq_workspace_size() bytes, 16-byte aligned.
+ * Asynchronous. */
 KVQ_API int kvq_decode_attention(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_seqs,
                          int32_t num_queries, int32_t num_q_heads, const int32_t* page_table,
                          int32_t max_pages_per_seq, const int32_t* seq_lens,
@@ -296,7 +302,9 @@ KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, 
  * ordered after all of this call's work.  After an error return, queued work
  * may still be pending on both streams (synchronize them before reusing the
  * buffers).  KVQ_FAULT=memcpy makes the page-in fail (KVQ_ERR_CUDA) for
- * tests.  Blocks the calling thread on the bounded waits. */
+ * tests.  Blocks the calling thread on the bounded waits.  A cache with
+ * outlier extraction returns KVQ_ERR_UNSUPPORTED (and kvq_adaptive_work_size
+ * 0): the ladder reads caches without extraction only. */
 KVQ_API size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs,
                                       int32_t num_queries, int32_t num_q_heads,
                                       int32_t max_pages_per_seq);

@@ -656,13 +656,18 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
             const float4 q4 = *reinterpret_cast<const float4*>(qf + c4 * D + 4 * ck);
             const float d4 = fmaf(q4.w, k23.y, fmaf(q4.z, k23.x, fmaf(q4.y, k01.y, q4.x * k01.x)));
             zt[sl] = fmaf(d4, a.s_att * kLog2e, zt[sl]);
-            float u = fabsf(q4.x) * fmaf(fabsf(k01.x), 0x1p-11f, 0x1p-25f);
-            u = fmaf(fabsf(q4.y), fmaf(fabsf(k01.y), 0x1p-11f, 0x1p-25f), u);
-            u = fmaf(fabsf(q4.z), fmaf(fabsf(k23.x), 0x1p-11f, 0x1p-25f), u);
-            u = fmaf(fabsf(q4.w), fmaf(fabsf(k23.y), 0x1p-11f, 0x1p-25f), u);
-            const float kn = fmaf(k23.y, k23.y, fmaf(k23.x, k23.x, fmaf(k01.y, k01.y, k01.x * k01.x)));
-            const float cr = rc[(2 + NGK) * kRows + c4];
-            dl[sl] = fmaf(cr, sqrtf(kn), fmaf(kKappa * a.s_att, u, dl[sl]));
+            // sum |q_i| (2^-11 |k_i| + 2^-25) = 2^-11 sum |q_i k_i| + 2^-25 sum |q_i|
+            const float qk = fmaf(fabsf(q4.w), fabsf(k23.y),
+                                  fmaf(fabsf(q4.z), fabsf(k23.x),
+                                       fmaf(fabsf(q4.y), fabsf(k01.y), fabsf(q4.x) * fabsf(k01.x))));
+            const float q1 = (fabsf(q4.x) + fabsf(q4.y)) + (fabsf(q4.z) + fabsf(q4.w));
+            dl[sl] = fmaf(kKappa * a.s_att, fmaf(qk, 0x1p-11f, q1 * 0x1p-25f), dl[sl]);
+            if (a.signs) {   // rotated keys: the chunk's norm (a few ulps of it are in kappa)
+              const float kn =
+                  fmaf(k23.y, k23.y, fmaf(k23.x, k23.x, fmaf(k01.y, k01.y, k01.x * k01.x)));
+              const float cr = rc[(2 + NGK) * kRows + c4];
+              dl[sl] = fmaf(cr, kn > 0.f ? kn * rsqrtf(kn) : 0.f, dl[sl]);
+            }
           }
         }
       }

@@ -19,8 +19,20 @@ def test_traffic_record_only_for_its_capture(monkeypatch):
     assert v is None or v > 110e6
     # once the kernel source changes (here: another file hashed in its place),
     # the record is no longer used
-    monkeypatch.setattr(bench, "DECODE_SRC", os.path.join(ROOT, "bench.py"))
+    monkeypatch.setattr(bench, "DECODE_SRCS", [os.path.join(ROOT, "bench.py")])
     assert bench._traffic_record("llama8b", False) is None
+
+
+def test_workload_variants():
+    assert bench._variant("llama8b") == ("llama8b", False)
+    assert bench._variant("llama8b+med3") == ("llama8b", True)
+    assert "Med3x" in bench._describe("serving+med3")
+    for bad in ("llama8b+x", "nosuch", "nosuch+med3"):
+        try:
+            bench._variant(bad)
+        except SystemExit:
+            continue
+        raise AssertionError(bad)
 
 
 def test_cpu_baseline_reports_its_sample():
