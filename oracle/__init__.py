@@ -9,8 +9,8 @@ with gcc, fp32 codec arithmetic in a fixed order and fp64 attention.
 Every function cites the page passage it follows; see ``kvq_oracle.c``.
 Pinned by ``tests/test_oracle_*.py`` against hand-worked cases, closed forms,
 library routines (scipy's Hadamard matrix, numpy's float16, torch's fp64
-scaled-dot-product attention) and brute force.  Parity of the bound's
-magnitude against the pages is unpinned: the pages print no worked bound.
+scaled-dot-product attention) and brute force; the bound's magnitude by
+hand-worked cases (``tests/golden/bound_hand_worked.txt``).
 """
 
 from __future__ import annotations
@@ -56,6 +56,10 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     L.oc_f16_rn.argtypes = [ctypes.c_float]
     L.oc_med3_chunk.restype = ctypes.c_int
     L.oc_block_bytes.restype = ctypes.c_int64
+    if hasattr(L, "oq_block_bytes"):
+        L.oq_block_bytes.restype = ctypes.c_int64
+        for name in ("oq_lloyd_max", "oq_tables", "oq_append", "oq_decode"):
+            getattr(L, name).restype = ctypes.c_int
     for name in ("oc_quantize_sym", "oc_quantize_asym", "oc_append", "oc_decode",
                  "oc_decode_promote_values", "oc_dense", "oc_f16_round_n"):
         getattr(L, name).restype = ctypes.c_int
@@ -351,3 +355,93 @@ def dense(q, k, v, seq_lens, scale=None, row_mask=None) -> np.ndarray:
 def certified(o_hat, o_dense, flags) -> np.ndarray:
     """Final output: exact dense attention for flagged rows, else o_hat."""
     return np.where(np.asarray(flags, bool)[:, None], o_dense, o_hat)
+
+
+# ------------------------------------------------------------------ KQV ----
+class OqCfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("d", "hkv", "num_pages")]
+
+
+KQV_KBITS, KQV_VBITS = 4, 3
+
+
+def lloyd_max(bits):
+    """Lloyd-Max centroids of N(0, 1) with 2^bits levels (fp64, ascending)."""
+    c = np.zeros(1 << bits, dtype=np.float64)
+    it = lib().oq_lloyd_max(bits, _p(c))
+    if it < 0:
+        raise ValueError("bad bit count")
+    return c
+
+
+def kqv_tables(bits, d):
+    """(centroids, thresholds) fp32 for unit vectors in dimension d."""
+    cent = np.zeros(1 << bits, dtype=np.float32)
+    thr = np.zeros((1 << bits) - 1, dtype=np.float32)
+    if lib().oq_tables(bits, d, _p(cent), _p(thr)) != OK:
+        raise ValueError("bad bit count")
+    return cent, thr
+
+
+def qjl(r, S):
+    """The QJL sketch bits (packed, d/8 bytes) of r and sum_i S_ic b_i."""
+    r = _c(r, np.float32)
+    S = _c(S, np.float32)
+    d = r.size
+    bits = np.zeros(d // 8, dtype=np.uint8)
+    rsum = np.zeros(d, dtype=np.float32)
+    lib().oq_qjl(_p(r), _p(S), d, _p(bits), _p(rsum))
+    return bits, rsum
+
+
+class KqvCache:
+    """The oracle's paged cache of the KQV codec ("Statistical Inference and
+    Quality Measures of KV Cache Quantisations Inspired by TurboQuant",
+    Quantisation schemes: KQV): rotated K in 4-bit Lloyd-Max codes, rotated V
+    in 3-bit codes plus the 1-bit QJL sketch of the residual."""
+
+    def __init__(self, head_dim, num_kv_heads, num_pages, rot_signs, qjl_matrix):
+        self.cfg = OqCfg(head_dim, num_kv_heads, num_pages)
+        bb = lib().oq_block_bytes(ctypes.byref(self.cfg))
+        if bb < 0:
+            raise ValueError("unsupported cache configuration")
+        self.block_bytes = int(bb)
+        self.pool = np.zeros(num_pages * num_kv_heads * self.block_bytes, dtype=np.uint8)
+        self.eta = np.zeros((num_pages, num_kv_heads), dtype=np.float32)
+        self.signs = _c(rot_signs, np.int8)
+        self.S = _c(qjl_matrix, np.float32)
+        assert self.S.shape == (head_dim, head_dim)
+
+    def append(self, k, v, page_table, start_pos, valid=None):
+        k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v)
+        assert k.shape == v.shape and k.dtype == v.dtype and k.ndim == 4
+        B, H, T, d = k.shape
+        pt = _c(page_table, np.int32)
+        sp = _c(start_pos, np.int32)
+        vl = None if valid is None else _c(valid, np.int32)
+        return lib().oq_append(ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(k),
+                               _p(v), int(k.dtype == np.float32), ctypes.c_int64(H * T * d),
+                               ctypes.c_int64(T * d), ctypes.c_int64(d), B, T, _p(vl), _p(pt),
+                               pt.shape[1], _p(sp), _p(self.signs), _p(self.S))
+
+    def decode(self, q, page_table, seq_lens, scale=None, tau=math.inf, row_mask=None):
+        """Returns (o_hat f64 [rows][d], bound f64 [rows], flags u8 [rows], diag [rows][8])."""
+        q = np.ascontiguousarray(q)
+        B, NQ, HQ, d = q.shape
+        rows = B * NQ * HQ
+        scale = default_scale(d) if scale is None else np.float32(scale)
+        out = np.zeros((rows, d), dtype=np.float64)
+        bound = np.zeros(rows, dtype=np.float64)
+        flags = np.zeros(rows, dtype=np.uint8)
+        diag = np.zeros((rows, 8), dtype=np.float64)
+        pt = _c(page_table, np.int32)
+        sl = _c(seq_lens, np.int32)
+        rm = None if row_mask is None else _c(row_mask, np.uint8)
+        rc = lib().oq_decode(ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(q),
+                             int(q.dtype == np.float32), B, NQ, HQ, _p(pt), pt.shape[1], _p(sl),
+                             ctypes.c_float(scale), ctypes.c_float(tau), _p(self.signs),
+                             _p(self.S), _p(out), _p(bound), _p(flags), _p(diag), _p(rm))
+        if rc != OK:
+            raise ValueError(f"oracle decode failed: {rc}")
+        return out, bound, flags, diag

@@ -1105,3 +1105,376 @@ int oc_decode_adaptive(const oc_cfg* c, const uint8_t* pool, const float* eta, c
   }
   return OC_OK;
 }
+
+/* ======================================================================== */
+/* KQV codec ("Statistical Inference and Quality Measures of KV Cache       */
+/* Quantisations Inspired by TurboQuant", Quantisation schemes: KQV).       */
+/* K and V both get the randomized Walsh-Hadamard rotation (oc_rotate, one  */
+/* sign vector sigma).  K takes the n-bit scalar MSE (Lloyd-Max) quantizer  */
+/* of the rotated unit vector's coordinates; V takes the (n-1)-bit one plus */
+/* the 1-bit QJL sketch of its residual.  Here n = 4.                       */
+/* Readings (the pages give the scheme, not its arithmetic):                */
+/*  - the coordinates of a rotated unit vector follow the page's             */
+/*    Beta((d-1)/2, (d-1)/2) marginal on [-1, 1], which tends to N(0, 1/d);  */
+/*    the codebook is the Lloyd-Max quantizer of N(0, 1) scaled by 1/sqrt(d) */
+/*    (centroids c_i / sqrt(d), thresholds (c_i + c_{i+1}) / (2 sqrt(d)),    */
+/*    computed in fp64 and rounded once to fp32);                            */
+/*  - a vector's Euclidean norm |x'| is kept in fp32, u = x' / |x'| (u = 0   */
+/*    for a zero vector); code = the number of thresholds strictly below u; */
+/*  - QJL: S is a d x d matrix of N(0, 1) entries (an input, drawn from the  */
+/*    seed); r = u - c_code; bit i = [sum_c S_ic r_c >= 0] (1 = +1, 0 = -1); */
+/*    r~ = sqrt(pi/2)/d * |r| * S^T b, so v^' = |v'| (c_code + r~);          */
+/*  - every dot product and squared norm is a sequential fmaf chain over     */
+/*    c = 0 .. d-1 (the decisions of codes and bits depend on its rounding); */
+/*  - the certified bound keeps the structure of oc_decode: Delta_j =        */
+/*    kappa*s*(|q'|_1 eps_j + 2^-16 |q'|_2 |k_j|) with eps_j the token's     */
+/*    largest |k' - k^'| (fp32, one ulp up); eta_b = the block's largest      */
+/*    |v - v^| in the unrotated domain plus 2^-16 |v| (fp32 reconstruction   */
+/*    allowance), one ulp up; the value range per 32-channel group from a   */
+/*    per-block max / min of v^ that starts at 0 (a zeroed block).           */
+/* Block of one (page, kv head), 16 tokens:                                   */
+/*   [K codes u4 [16][d/2]][V codes u4 (3-bit) [16][d/2]][V sketch [16][d/8]] */
+/*   [|k'| f32 [16]][eps f32 [16]][|v'| f32 [16]][|r| f32 [16]]              */
+/*   [v^ max, min f32 [d/32][2]]                                             */
+/* nibble of channel c in byte c/2, low nibble for even c; sketch bit i in   */
+/* byte i/8, bit i%8 (least significant first).                              */
+/* ======================================================================== */
+typedef struct {
+  int32_t d, hkv, num_pages;
+} oq_cfg;
+
+#define OQ_KBITS 4
+#define OQ_VBITS 3
+#define OQ_PI 3.14159265358979323846
+
+static int oq_ok(const oq_cfg* c) {
+  return c && (c->d == 64 || c->d == 128) && c->hkv > 0 && c->num_pages >= 0;
+}
+static int64_t oq_off_vc(const oq_cfg* c) { return (int64_t)OC_PAGE * c->d / 2; }
+static int64_t oq_off_vs(const oq_cfg* c) { return (int64_t)OC_PAGE * c->d; }
+static int64_t oq_off_kn(const oq_cfg* c) { return (int64_t)OC_PAGE * c->d + OC_PAGE * c->d / 8; }
+static int64_t oq_off_ke(const oq_cfg* c) { return oq_off_kn(c) + 4 * OC_PAGE; }
+static int64_t oq_off_vn(const oq_cfg* c) { return oq_off_kn(c) + 8 * OC_PAGE; }
+static int64_t oq_off_vr(const oq_cfg* c) { return oq_off_kn(c) + 12 * OC_PAGE; }
+static int64_t oq_off_rg(const oq_cfg* c) { return oq_off_kn(c) + 16 * OC_PAGE; }
+
+int64_t oq_block_bytes(const oq_cfg* c) {
+  if (!oq_ok(c)) return -1;
+  return oq_off_rg(c) + (int64_t)(c->d / 32) * 2 * 4;
+}
+
+/* Lloyd-Max quantizer of N(0, 1) with 2^bits levels (ascending centroids
+ * into c): Lloyd's iteration from evenly spaced positive centroids, using
+ * the symmetric half.  A cell [a, b] (a >= 0) has centroid
+ * (phi(a) - phi(b)) / (Q(a) - Q(b)), phi the density and Q(x) = P(X > x) =
+ * erfc(x / sqrt 2) / 2; thresholds are midpoints, 0 in the middle.  Stops
+ * when no centroid moves by more than 2^-52 of the largest.  Returns the
+ * iterations taken. */
+static double oq_phi(double x) { return isinf(x) ? 0.0 : exp(-0.5 * x * x) / sqrt(2.0 * OQ_PI); }
+static double oq_tail(double x) { return isinf(x) ? 0.0 : 0.5 * erfc(x / sqrt(2.0)); }
+
+int oq_lloyd_max(int bits, double* c) {
+  if (bits < 1 || bits > 6) return OC_ERR_ARG;
+  int n = (1 << bits) / 2;
+  double p[32], t[33];
+  for (int i = 0; i < n; ++i) p[i] = 3.0 * (i + 0.5) / n;
+  int it;
+  for (it = 1; it <= 1000000; ++it) {
+    t[0] = 0.0;
+    for (int i = 1; i < n; ++i) t[i] = 0.5 * (p[i - 1] + p[i]);
+    t[n] = INFINITY;
+    double move = 0.0;
+    for (int i = 0; i < n; ++i) {
+      double np = (oq_phi(t[i]) - oq_phi(t[i + 1])) / (oq_tail(t[i]) - oq_tail(t[i + 1]));
+      if (fabs(np - p[i]) > move) move = fabs(np - p[i]);
+      p[i] = np;
+    }
+    if (move <= ldexp(p[n - 1], -52)) break;
+  }
+  for (int i = 0; i < n; ++i) {
+    c[n + i] = p[i];
+    c[n - 1 - i] = -p[i];
+  }
+  return it;
+}
+
+/* fp32 tables for unit vectors in dimension d: cent[i] = c_i / sqrt(d),
+ * thr[i] = (c_i + c_{i+1}) / (2 sqrt(d)) (i < 2^bits - 1). */
+int oq_tables(int bits, int d, float* cent, float* thr) {
+  double c[64];
+  int r = oq_lloyd_max(bits, c);
+  if (r < 0) return r;
+  int L = 1 << bits;
+  double sd = sqrt((double)d);
+  for (int i = 0; i < L; ++i) cent[i] = (float)(c[i] / sd);
+  for (int i = 0; i + 1 < L; ++i) thr[i] = (float)((c[i] + c[i + 1]) / (2.0 * sd));
+  return OC_OK;
+}
+
+static float oq_dot(const float* a, const float* b, int n) {
+  float s = 0.0f;
+  for (int i = 0; i < n; ++i) s = fmaf(a[i], b[i], s);
+  return s;
+}
+
+static int oq_code(float u, const float* thr, int L) {
+  int k = 0;
+  for (int i = 0; i + 1 < L; ++i) k += thr[i] < u;
+  return k;
+}
+
+/* The QJL sketch of r (bits, d/8 bytes) and its estimate r~ (without the
+ * |r| * sqrt(pi/2)/d factor when unit_scale is 0: sum_i S_ic b_i). */
+void oq_qjl(const float* r, const float* S, int d, uint8_t* bits, float* rsum) {
+  memset(bits, 0, (size_t)d / 8);
+  for (int i = 0; i < d; ++i)
+    if (oq_dot(S + (int64_t)i * d, r, d) >= 0.0f) bits[i / 8] |= (uint8_t)(1u << (i % 8));
+  for (int ch = 0; ch < d; ++ch) {
+    float acc = 0.0f;
+    for (int i = 0; i < d; ++i) {
+      float b = (bits[i / 8] >> (i % 8)) & 1u ? 1.0f : -1.0f;
+      acc = fmaf(S[(int64_t)i * d + ch], b, acc);
+    }
+    rsum[ch] = acc;
+  }
+}
+
+static void oq_wrf(uint8_t* p, float x) { memcpy(p, &x, 4); }
+static float oq_rdf(const uint8_t* p) { float x; memcpy(&x, p, 4); return x; }
+
+/* Quantize one token of one kv head into slot `slot`; returns its eta
+ * contribution (one ulp up) and raises the block's v^ range. */
+static int oq_quantize_token(const oq_cfg* c, uint8_t* blk, int slot, const float* k,
+                             const float* v, const int8_t* sigma, const float* S,
+                             const float* kcent, const float* kthr, const float* vcent,
+                             const float* vthr, float* eta_out) {
+  int d = c->d, rc = OC_OK;
+  int LK = 1 << OQ_KBITS, LV = 1 << OQ_VBITS;
+  float kr[128], vr[128], u[128], r[128], rs[128], vh[128], tmp[128];
+  int8_t ones[128];
+  for (int i = 0; i < d; ++i) ones[i] = 1;
+  /* keys */
+  oc_rotate(k, sigma, d, kr);
+  float nk = sqrtf(oq_dot(kr, kr, d));
+  if (!isfinite(nk)) { rc = OC_ERR_RANGE; nk = 0.0f; }
+  float eps = 0.0f;
+  uint8_t* kc = blk + (int64_t)slot * (d / 2);
+  for (int ch = 0; ch < d; ++ch) {
+    float uu = nk > 0.0f ? kr[ch] / nk : 0.0f;
+    int code = oq_code(uu, kthr, LK);
+    oc_put_nibble(kc, ch / 2, ch, (unsigned)code);
+    float kh = nk * kcent[code];
+    float e = fabsf(kr[ch] - kh);
+    if (nk > 0.0f && e > eps) eps = e;
+  }
+  oq_wrf(blk + oq_off_kn(c) + 4 * slot, nk);
+  oq_wrf(blk + oq_off_ke(c) + 4 * slot, nextafterf(eps, INFINITY));
+  /* values */
+  oc_rotate(v, sigma, d, vr);
+  float nv = sqrtf(oq_dot(vr, vr, d));
+  if (!isfinite(nv)) { rc = OC_ERR_RANGE; nv = 0.0f; }
+  uint8_t* vc = blk + oq_off_vc(c) + (int64_t)slot * (d / 2);
+  int code[128];
+  for (int ch = 0; ch < d; ++ch) {
+    u[ch] = nv > 0.0f ? vr[ch] / nv : 0.0f;
+    code[ch] = oq_code(u[ch], vthr, LV);
+    oc_put_nibble(vc, ch / 2, ch, (unsigned)code[ch]);
+    r[ch] = u[ch] - vcent[code[ch]];
+  }
+  float rn = sqrtf(oq_dot(r, r, d));
+  uint8_t* bits = blk + oq_off_vs(c) + (int64_t)slot * (d / 8);
+  oq_qjl(r, S, d, bits, rs);
+  oq_wrf(blk + oq_off_vn(c) + 4 * slot, nv);
+  oq_wrf(blk + oq_off_vr(c) + 4 * slot, rn);
+  /* reconstruction in the unrotated domain: v^ = sigma o (c H v^') */
+  float rho = (float)(sqrt(OQ_PI / 2.0) / d) * rn;
+  for (int ch = 0; ch < d; ++ch) tmp[ch] = nv * (vcent[code[ch]] + rho * rs[ch]);
+  oc_rotate(tmp, ones, d, vh);
+  float err = 0.0f;
+  for (int ch = 0; ch < d; ++ch) {
+    if (sigma[ch] < 0) vh[ch] = -vh[ch];
+    float e = fabsf(v[ch] - vh[ch]);
+    if (e > err) err = e;
+  }
+  if (rc != OC_OK) err = 0.0f;
+  *eta_out = nextafterf(fmaf(1.0f / 65536.0f, nv, err), INFINITY);
+  uint8_t* rg = blk + oq_off_rg(c);
+  for (int g = 0; g < d / 32; ++g) {
+    float hi = oq_rdf(rg + 8 * g), lo = oq_rdf(rg + 8 * g + 4);
+    for (int ch = 32 * g; ch < 32 * g + 32; ++ch) {
+      if (vh[ch] > hi) hi = vh[ch];
+      if (vh[ch] < lo) lo = vh[ch];
+    }
+    oq_wrf(rg + 8 * g, hi);
+    oq_wrf(rg + 8 * g + 4, lo);
+  }
+  return rc;
+}
+
+/* Quantize-on-append for the KQV codec; arguments as oc_append, plus the
+ * QJL matrix S (fp32 [d][d], row i = projection i). */
+int oq_append(const oq_cfg* c, uint8_t* pool, float* eta, const void* k, const void* v,
+              int in_is_f32, int64_t seq_stride, int64_t head_stride, int64_t tok_stride,
+              int num_seqs, int num_tokens, const int32_t* valid, const int32_t* page_table,
+              int max_pages, const int32_t* start_pos, const int8_t* sigma, const float* S) {
+  if (!oq_ok(c) || !sigma || !S) return OC_ERR_ARG;
+  float kcent[16], kthr[15], vcent[8], vthr[7];
+  oq_tables(OQ_KBITS, c->d, kcent, kthr);
+  oq_tables(OQ_VBITS, c->d, vcent, vthr);
+  int64_t bb = oq_block_bytes(c);
+  int rc = OC_OK;
+  float xk[128], xv[128];
+  for (int b = 0; b < num_seqs; ++b) {
+    int nt = valid ? valid[b] : num_tokens;
+    for (int t = 0; t < nt; ++t) {
+      int pos = start_pos[b] + t;
+      int lp = pos / OC_PAGE;
+      if (lp >= max_pages) return OC_ERR_ARG;
+      int page = page_table[(int64_t)b * max_pages + lp];
+      if (page < 0 || page >= c->num_pages) return OC_ERR_ARG;
+      for (int h = 0; h < c->hkv; ++h) {
+        int64_t off = b * seq_stride + h * head_stride + t * tok_stride;
+        oc_load_vec(k, in_is_f32, off, c->d, xk);
+        oc_load_vec(v, in_is_f32, off, c->d, xv);
+        int bad = 0;
+        for (int i = 0; i < c->d; ++i) bad |= !isfinite(xk[i]) || !isfinite(xv[i]);
+        uint8_t* blk = pool + ((int64_t)page * c->hkv + h) * bb;
+        float e;
+        int r = oq_quantize_token(c, blk, pos % OC_PAGE, xk, xv, sigma, S, kcent, kthr, vcent,
+                                  vthr, &e);
+        if (r != OC_OK || bad) rc = OC_ERR_RANGE;
+        float* ep = eta + (int64_t)page * c->hkv + h;
+        if (e > *ep) *ep = e;
+      }
+    }
+  }
+  return rc;
+}
+
+/* Decode attention and its certified bound over a KQV cache, for every query
+ * row (sequence b, query i, q head h; kv head h / (Hq/Hkv)), in fp64:
+ *   q' = rotated q;  k^'_jc = |k_j| * cent4[code] (the fp32 product the
+ *   append used);  z^_j = scale * q' . k^'_j
+ *   v^'_jc = |v_j| (cent3[code] + sqrt(pi/2)/d |r_j| sum_i S_ic b_ji)
+ *   o^ = sigma o (H sum_j p^_j v^'_j) / sqrt(d)      (unrotated)
+ *   Delta_j = kappa*scale*(|q'|_1 eps_j + 2^-16 |q'|_2 |k_j|)
+ *   A, B, TV as in oc_decode; range = max_g (max_b hi_{b,g} - min_b lo_{b,g})
+ *   over the context's blocks; E_key = TV (range + 2 max eta); E_val =
+ *   sum_j p^_j eta_{block(j)}; bound = kappa (E_key + E_val).
+ * diag (optional) as in oc_decode. */
+int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void* q,
+              int q_is_f32, int num_seqs, int nq, int hq, const int32_t* page_table,
+              int max_pages, const int32_t* seq_lens, float scale, float tau,
+              const int8_t* sigma, const float* S, double* out, double* bound, uint8_t* flags,
+              double* diag, const uint8_t* row_mask) {
+  if (!oq_ok(c) || hq % c->hkv || !sigma || !S) return OC_ERR_ARG;
+  int d = c->d, G = hq / c->hkv, NG = d / 32;
+  float kcent[16], kthr[15], vcent[8], vthr[7];
+  oq_tables(OQ_KBITS, d, kcent, kthr);
+  oq_tables(OQ_VBITS, d, vcent, vthr);
+  int64_t bb = oq_block_bytes(c);
+  double sc = (double)scale, sd = sqrt((double)d);
+  for (int b = 0; b < num_seqs; ++b) {
+    int n = seq_lens[b];
+    double* z = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* dl = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    for (int i = 0; i < nq; ++i)
+      for (int h = 0; h < hq; ++h) {
+        int64_t row = ((int64_t)b * nq + i) * hq + h;
+        if (row_mask && !row_mask[row]) continue;
+        int kv = h / G;
+        double* o = out + row * d;
+        for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+        if (n == 0) {
+          bound[row] = 0.0;
+          flags[row] = 0;
+          if (diag) for (int t = 0; t < 8; ++t) diag[row * 8 + t] = 0.0;
+          continue;
+        }
+        float qf[128], qr[128];
+        oc_load_vec(q, q_is_f32, row * d, d, qf);
+        oc_rotate(qf, sigma, d, qr);
+        double qn1 = 0.0, qn2 = 0.0;
+        for (int ch = 0; ch < d; ++ch) {
+          qn1 += fabs((double)qr[ch]);
+          qn2 += (double)qr[ch] * (double)qr[ch];
+        }
+        qn2 = sqrt(qn2);
+        double hi[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        double lo[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+        double eta_max = 0.0, m = -INFINITY;
+        for (int j = 0; j < n; ++j) {
+          int page = page_table[(int64_t)b * max_pages + j / OC_PAGE], slot = j % OC_PAGE;
+          const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+          float nk = oq_rdf(blk + oq_off_kn(c) + 4 * slot);
+          double dot = 0.0;
+          for (int ch = 0; ch < d; ++ch) {
+            unsigned code = oc_get_nibble(blk + (int64_t)slot * (d / 2), ch / 2, ch);
+            dot += (double)qr[ch] * (double)(nk * kcent[code]);
+          }
+          z[j] = sc * dot;
+          dl[j] = OC_KAPPA * sc * (qn1 * (double)oq_rdf(blk + oq_off_ke(c) + 4 * slot) +
+                                   OC_ROT_SLACK * qn2 * (double)nk);
+          if (z[j] > m) m = z[j];
+          if (slot == 0 || j == 0) {   /* each block of the context once */
+            const uint8_t* rg = blk + oq_off_rg(c);
+            for (int g = 0; g < NG; ++g) {
+              if (oq_rdf(rg + 8 * g) > hi[g]) hi[g] = oq_rdf(rg + 8 * g);
+              if (oq_rdf(rg + 8 * g + 4) < lo[g]) lo[g] = oq_rdf(rg + 8 * g + 4);
+            }
+            double e = (double)eta[(int64_t)page * c->hkv + kv];
+            if (e > eta_max) eta_max = e;
+          }
+        }
+        double l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0, op[128];
+        for (int ch = 0; ch < d; ++ch) op[ch] = 0.0;
+        for (int j = 0; j < n; ++j) {
+          double p = exp(z[j] - m) / l;
+          int page = page_table[(int64_t)b * max_pages + j / OC_PAGE], slot = j % OC_PAGE;
+          const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+          double nv = oq_rdf(blk + oq_off_vn(c) + 4 * slot);
+          double rho = sqrt(OQ_PI / 2.0) / d * (double)oq_rdf(blk + oq_off_vr(c) + 4 * slot);
+          const uint8_t* bits = blk + oq_off_vs(c) + (int64_t)slot * (d / 8);
+          for (int ch = 0; ch < d; ++ch) {
+            unsigned code = oc_get_nibble(blk + oq_off_vc(c) + (int64_t)slot * (d / 2), ch / 2, ch);
+            double s = 0.0;
+            for (int ii = 0; ii < d; ++ii)
+              s += ((bits[ii / 8] >> (ii % 8)) & 1u ? 1.0 : -1.0) * (double)S[(int64_t)ii * d + ch];
+            op[ch] += p * nv * ((double)vcent[code] + rho * s);
+          }
+          A += p * expm1(dl[j]);
+          B += p * exp(-dl[j]);
+          Ev += p * (double)eta[(int64_t)page * c->hkv + kv];
+          if (dl[j] > dmax) dmax = dl[j];
+        }
+        /* o = sigma o (H op) / sqrt(d), fp64 butterflies */
+        for (int hh = 1; hh < d; hh *= 2)
+          for (int i0 = 0; i0 < d; i0 += 2 * hh)
+            for (int jj = i0; jj < i0 + hh; ++jj) {
+              double a = op[jj], bq = op[jj + hh];
+              op[jj] = a + bq;
+              op[jj + hh] = a - bq;
+            }
+        for (int ch = 0; ch < d; ++ch) o[ch] = (sigma[ch] < 0 ? -op[ch] : op[ch]) / sd;
+        double range = 0.0;
+        for (int g = 0; g < NG; ++g)
+          if (hi[g] - lo[g] > range) range = hi[g] - lo[g];
+        double tv = tanh(dmax / 2.0);
+        if (A / B < tv) tv = A / B;
+        double ekey = tv * (range + 2.0 * eta_max);
+        double bd = OC_KAPPA * (ekey + Ev);
+        bound[row] = bd;
+        flags[row] = bd > (double)tau ? 1 : 0;
+        if (diag) {
+          double* dg = diag + row * 8;
+          dg[0] = tv; dg[1] = ekey; dg[2] = Ev; dg[3] = dmax;
+          dg[4] = A; dg[5] = B; dg[6] = range; dg[7] = eta_max;
+        }
+      }
+    free(z);
+    free(dl);
+  }
+  return OC_OK;
+}

@@ -47,8 +47,8 @@ import numpy as np
 PAGE_SIZE = 16
 
 # stream ids (fixed order: Q, K, V, outlier channels, spikes, Hadamard signs,
-# page permutation, context lengths)
-_S_Q, _S_K, _S_V, _S_OUTLIER, _S_SPIKE, _S_SIGNS, _S_PERM, _S_LEN = range(8)
+# page permutation, context lengths, the KQV codec's QJL projections)
+_S_Q, _S_K, _S_V, _S_OUTLIER, _S_SPIKE, _S_SIGNS, _S_PERM, _S_LEN, _S_QJL = range(9)
 
 _CONFIG_IDS = {"tiny": 1, "llama8b": 2, "long128k": 3, "rotated": 4, "serving": 5}
 
@@ -175,11 +175,19 @@ class Inputs:
         return sorted(int(x) for x in g.choice(wl.num_seqs, size=n, replace=False))
 
     def _signs(self) -> Optional[np.ndarray]:
-        wl = self.wl
-        if not wl.k_rotate:
-            return None
-        g = _rng(self.seed, wl.name, _S_SIGNS)
-        return np.where(g.integers(0, 2, size=wl.head_dim) == 1, 1, -1).astype(np.int8)
+        return self.rotation_signs() if self.wl.k_rotate else None
+
+    def rotation_signs(self) -> np.ndarray:
+        """The Hadamard sign vector of the seed (drawn whether or not the
+        workload's own codec rotates; the KQV codec always does)."""
+        g = _rng(self.seed, self.wl.name, _S_SIGNS)
+        return np.where(g.integers(0, 2, size=self.wl.head_dim) == 1, 1, -1).astype(np.int8)
+
+    def qjl_matrix(self) -> np.ndarray:
+        """The KQV codec's QJL projections: fp32 [d][d], i.i.d. N(0, 1)."""
+        g = _rng(self.seed, self.wl.name, _S_QJL)
+        d = self.wl.head_dim
+        return g.standard_normal((d, d), dtype=np.float32)
 
     # -- tensors ------------------------------------------------------------
     def _cast(self, x32: np.ndarray) -> np.ndarray:
