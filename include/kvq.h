@@ -123,7 +123,47 @@ typedef struct kvq_cache {
   const int8_t* rot_signs; /* device, head_dim entries of +1/-1; required iff k_rotate */
   int32_t* error_word;     /* device, one int32 kernels set to a kvq_status on error; may be NULL */
   int32_t outliers;        /* 1: outlier extraction (see the layout above); 0: none */
+  int32_t codec;           /* KVQ_CODEC_INT (0: the layout above) or KVQ_CODEC_KQV (1) */
+  const float* qjl;        /* device, KVQ_CODEC_KQV: the QJL projections S, fp32
+                              [head_dim][head_dim] row-major (row i = projection i) */
 } kvq_cache;
+
+#define KVQ_CODEC_INT 0
+#define KVQ_CODEC_KQV 1
+
+/* The KQV codec ("Statistical Inference and Quality Measures of KV Cache
+ * Quantisations Inspired by TurboQuant", Quantisation schemes: KQV), codec =
+ * KVQ_CODEC_KQV: K and V rotated by the randomized Walsh-Hadamard transform
+ * (rot_signs, required; k_rotate must be 1), K coded by the 4-bit Lloyd-Max
+ * quantizer of the rotated unit vector's coordinates, V by the 3-bit one
+ * plus the 1-bit QJL sketch of its residual (k_bits 4, v_bits 3, k_group =
+ * v_group = head_dim, outliers 0):
+ *   x' = rotation of x; n = |x'|_2 (fp32, a sequential fmaf chain over the
+ *   channels); u = x' / n (0 when n = 0); code = the number of thresholds
+ *   below u (kvq_kqv_codebook); k^' = n * centroid[code];
+ *   V: r = u - centroid3[code]; bit i = [sum_c S_ic r_c >= 0] (sequential
+ *   fmaf chain); v^' = n_v (centroid3[code] + sqrt(pi/2)/d |r| S^T b);
+ *   v^ = sigma o (H v^') / sqrt(d).
+ * Block of one (page, kv head), 16 tokens (d = head_dim):
+ *   [K codes 4-bit [16][d/2]][V codes 3-bit in nibbles [16][d/2]]
+ *   [V sketch bits [16][d/8]][|k'| f32 [16]][eps f32 [16]][|v'| f32 [16]]
+ *   [|r| f32 [16]][v^ max, min f32 [d/32][2]]
+ * nibble of channel c in byte c/2 (low nibble for even c); sketch bit i in
+ * byte i/8, bit i%8.  eps = max_c |k'_c - k^'_c| one ulp up; eta[page][h] =
+ * max over the block of (max_c |v_c - v^_c| + 2^-16 n_v) one ulp up; the
+ * range of each 32-channel group starts at [0, 0] in a zeroed block and
+ * widens to every v^ appended.  The decode's bound uses Delta_j =
+ * kappa*s*(|q'|_1 eps_j + 2^-16 |q'|_2 n_kj) and E_key = TV (max_g range_g +
+ * 2 max eta).  kvq_decode_attention_append and kvq_adaptive_precision return
+ * KVQ_ERR_UNSUPPORTED for this codec. */
+
+/* Centroids (2^bits) and decision thresholds (2^bits - 1) of the KQV codec's
+ * scalar quantizer for unit vectors in dimension head_dim: the Lloyd-Max
+ * quantizer of N(0, 1) (the Gaussian limit of the Beta((d-1)/2, (d-1)/2)
+ * coordinate marginal) divided by sqrt(head_dim), computed in fp64 and
+ * rounded to fp32.  bits 1..6; host memory; returns a kvq_status. */
+KVQ_API int kvq_kqv_codebook(int32_t bits, int32_t head_dim, float* centroids,
+                             float* thresholds);
 
 /* Bytes of one (page, kv head) block, and of the whole pool; 0 if the cache
  * description is invalid or unsupported. */

@@ -1378,8 +1378,10 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
     int n = seq_lens[b];
     double* z = n ? (double*)malloc(sizeof(double) * n) : NULL;
     double* dl = n ? (double*)malloc(sizeof(double) * n) : NULL;
-    for (int i = 0; i < nq; ++i)
-      for (int h = 0; h < hq; ++h) {
+    double* vh = n ? (double*)malloc(sizeof(double) * n * d) : NULL;
+    int vh_kv = -1;
+    for (int h = 0; h < hq; ++h)     /* q heads outermost: the rows of one kv head together */
+      for (int i = 0; i < nq; ++i) {
         int64_t row = ((int64_t)b * nq + i) * hq + h;
         if (row_mask && !row_mask[row]) continue;
         int kv = h / G;
@@ -1428,22 +1430,31 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
         }
         double l = 0.0;
         for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        /* the rotated reconstructions v^'_j of this (sequence, kv head), once for
+         * the rows that share them */
+        if (kv != vh_kv) {
+          for (int j = 0; j < n; ++j) {
+            int page = page_table[(int64_t)b * max_pages + j / OC_PAGE], slot = j % OC_PAGE;
+            const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+            double nv = oq_rdf(blk + oq_off_vn(c) + 4 * slot);
+            double rho = sqrt(OQ_PI / 2.0) / d * (double)oq_rdf(blk + oq_off_vr(c) + 4 * slot);
+            const uint8_t* bits = blk + oq_off_vs(c) + (int64_t)slot * (d / 8);
+            for (int ch = 0; ch < d; ++ch) {
+              unsigned code = oc_get_nibble(blk + oq_off_vc(c) + (int64_t)slot * (d / 2), ch / 2, ch);
+              double s = 0.0;
+              for (int ii = 0; ii < d; ++ii)
+                s += ((bits[ii / 8] >> (ii % 8)) & 1u ? 1.0 : -1.0) * (double)S[(int64_t)ii * d + ch];
+              vh[(int64_t)j * d + ch] = nv * ((double)vcent[code] + rho * s);
+            }
+          }
+          vh_kv = kv;
+        }
         double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0, op[128];
         for (int ch = 0; ch < d; ++ch) op[ch] = 0.0;
         for (int j = 0; j < n; ++j) {
           double p = exp(z[j] - m) / l;
-          int page = page_table[(int64_t)b * max_pages + j / OC_PAGE], slot = j % OC_PAGE;
-          const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
-          double nv = oq_rdf(blk + oq_off_vn(c) + 4 * slot);
-          double rho = sqrt(OQ_PI / 2.0) / d * (double)oq_rdf(blk + oq_off_vr(c) + 4 * slot);
-          const uint8_t* bits = blk + oq_off_vs(c) + (int64_t)slot * (d / 8);
-          for (int ch = 0; ch < d; ++ch) {
-            unsigned code = oc_get_nibble(blk + oq_off_vc(c) + (int64_t)slot * (d / 2), ch / 2, ch);
-            double s = 0.0;
-            for (int ii = 0; ii < d; ++ii)
-              s += ((bits[ii / 8] >> (ii % 8)) & 1u ? 1.0 : -1.0) * (double)S[(int64_t)ii * d + ch];
-            op[ch] += p * nv * ((double)vcent[code] + rho * s);
-          }
+          int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
+          for (int ch = 0; ch < d; ++ch) op[ch] += p * vh[(int64_t)j * d + ch];
           A += p * expm1(dl[j]);
           B += p * exp(-dl[j]);
           Ev += p * (double)eta[(int64_t)page * c->hkv + kv];
@@ -1475,6 +1486,7 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
       }
     free(z);
     free(dl);
+    free(vh);
   }
   return OC_OK;
 }

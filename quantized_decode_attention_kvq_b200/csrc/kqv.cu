@@ -1,0 +1,803 @@
+// kqv.cu -- the KQV codec of "Statistical Inference and Quality Measures of KV
+// Cache Quantisations Inspired by TurboQuant" (Quantisation schemes: KQV):
+// K and V rotated by the randomized Walsh-Hadamard transform, K coded by the
+// 4-bit scalar MSE (Lloyd-Max) quantizer of the rotated unit vector's
+// coordinates, V by the 3-bit one plus the 1-bit QJL sketch of its residual,
+// with the certified bound of "Runtime-Certified Bounded-Error Quantized
+// Attention" (Methodology 2) carried over to this codec.
+//
+//   kvq_kqv_codebook      host: the Lloyd-Max quantizer of N(0, 1) by
+//                         Lloyd's iteration on the decision thresholds, the
+//                         Gaussian limit of the page's Beta coordinate
+//                         marginal, scaled by 1/sqrt(d)
+//   kqv_append_kernel     one warp per (token, kv head): rotation, norms,
+//                         codes, the sketch (S r, one projection per lane
+//                         and pass), the reconstruction for eta and the value
+//                         range
+//   kqv_partial_kernel    grid (sequence x kv head, split), 4 warps, each warp
+//                         streaming its pages through a 2-stage bulk-copy
+//                         ring: scores on the CUDA cores (lane = 4 channels,
+//                         codebook lookups from a bank-replicated shared
+//                         table, a reduce-scatter of the 8 tokens x 4 rows
+//                         partial sums), online softmax, the bound's sums,
+//                         PV as two accumulations per channel (the codebook
+//                         part and the sketch part, the latter indexed by
+//                         projection)
+//   kqv_merge_kernel      per (sequence, kv head): the split records' merge,
+//                         the sketch part through S^T, the inverse rotation,
+//                         the bound and the flag
+// Every dot product or squared norm whose rounding decides a code or a
+// sketch bit is the sequential fmaf chain over the channels that the codec's
+// definition fixes, so codes, bits, norms and eta are bit-identical to a
+// sequential implementation.
+#include <cmath>
+#include <map>
+#include <mutex>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+// ================================================================ codebook ====
+namespace {
+
+constexpr double kPi = 3.14159265358979323846;
+
+double normal_pdf(double x) { return std::isinf(x) ? 0.0 : std::exp(-0.5 * x * x) / std::sqrt(2.0 * kPi); }
+// P(X > x) for X ~ N(0, 1)
+double normal_sf(double x) { return std::isinf(x) ? 0.0 : 0.5 * std::erfc(x / std::sqrt(2.0)); }
+
+// Lloyd's iteration on the positive decision thresholds of the symmetric
+// quantizer with L = 2^bits levels: the centroids of the cells they bound
+// (conditional means, closed form for the normal density), then the
+// midpoints of neighbouring centroids as the new thresholds, until no
+// threshold moves by more than 2^-52 of the largest centroid.  Writes the L
+// centroids, ascending and exactly antisymmetric.
+void lloyd_max_normal(int bits, double* cent) {
+  const int L = 1 << bits, half = L / 2;
+  double thr[33];                        // thr[0] = 0 < thr[1] < ... ; thr[half] = +inf
+  double c[32];
+  for (int i = 0; i <= half; ++i) thr[i] = i == half ? INFINITY : 3.0 * i / half;
+  for (int it = 0; it < 1000000; ++it) {
+    for (int i = 0; i < half; ++i)
+      c[i] = (normal_pdf(thr[i]) - normal_pdf(thr[i + 1])) /
+             (normal_sf(thr[i]) - normal_sf(thr[i + 1]));
+    double moved = 0.0;
+    for (int i = 1; i < half; ++i) {
+      const double t = 0.5 * (c[i - 1] + c[i]);
+      moved = std::fmax(moved, std::fabs(t - thr[i]));
+      thr[i] = t;
+    }
+    if (moved <= std::ldexp(c[half - 1], -52)) {
+      for (int i = 0; i < half; ++i)   // the centroids of the final thresholds
+        c[i] = (normal_pdf(thr[i]) - normal_pdf(thr[i + 1])) /
+               (normal_sf(thr[i]) - normal_sf(thr[i + 1]));
+      break;
+    }
+  }
+  for (int i = 0; i < half; ++i) {
+    cent[half + i] = c[i];
+    cent[half - 1 - i] = -c[i];
+  }
+}
+
+int codebook_f32(int bits, int d, float* cent, float* thr) {
+  double c[64];
+  lloyd_max_normal(bits, c);
+  const int L = 1 << bits;
+  const double sd = std::sqrt((double)d);
+  for (int i = 0; i < L; ++i) cent[i] = (float)(c[i] / sd);
+  for (int i = 0; i + 1 < L; ++i) thr[i] = (float)((c[i] + c[i + 1]) / (2.0 * sd));
+  return KVQ_OK;
+}
+
+}  // namespace
+
+int kqv_tables(int d, KqvTables* t) {
+  static std::mutex mu;
+  static std::map<int, KqvTables> cache;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(d);
+  if (it == cache.end()) {
+    KqvTables x;
+    codebook_f32(4, d, x.kcent, x.kthr);
+    codebook_f32(3, d, x.vcent, x.vthr);
+    it = cache.emplace(d, x).first;
+  }
+  *t = it->second;
+  return KVQ_OK;
+}
+
+// ================================================================ append =====
+template <int L>
+__device__ __forceinline__ int kqv_code(float u, const float* thr) {
+  int k = 0;
+#pragma unroll
+  for (int i = 0; i + 1 < L; ++i) k += thr[i] < u;
+  return k;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) kqv_append_kernel(const KqvAppendArgs ka) {
+  constexpr int E = D / 32;
+  constexpr int LPG = 32 / E;           // lanes per 32-channel group
+  const AppendArgs& a = ka.a;
+  const KqvLayout L{D};
+  __shared__ float sh[8][2][D];         // per warp: the rotated vector, the residual
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t item = (int64_t)blockIdx.x * 8 + w;
+  const int64_t total = (int64_t)a.num_seqs * a.num_tokens * a.hkv;
+  if (item >= total) return;   // warp-uniform
+  const int h = (int)(item % a.hkv);
+  const int t = (int)((item / a.hkv) % a.num_tokens);
+  const int s = (int)(item / ((int64_t)a.hkv * a.num_tokens));
+  const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
+  float xk[E], xv[E], vin[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    xk[e] = load_elem(a.k, a.in_bf16, base + lane * E + e);
+    xv[e] = vin[e] = load_elem(a.v, a.in_bf16, base + lane * E + e);
+  }
+  if (a.valid && t >= a.valid[s]) return;
+  const int pos = a.start_pos[s] + t;
+  const int lp = pos / kPage;
+  if (pos < 0 || lp >= a.max_pages) {
+    if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+    return;
+  }
+  const int page = a.page_table[(int64_t)s * a.max_pages + lp];
+  if (page < 0 || page >= a.num_pages) {
+    if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+    return;
+  }
+  const int slot = pos % kPage;
+  uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
+  float* xs = sh[w][0];
+  float* rs = sh[w][1];
+
+  // ---- keys: rotate, norm, codes, eps ----
+  warp_rotate<E>(xk, a.signs, lane, a.rot_c);
+#pragma unroll
+  for (int e = 0; e < E; ++e) xs[lane * E + e] = xk[e];
+  __syncwarp();
+  float nk = 0.f;
+  for (int c = 0; c < D; ++c) nk = __fmaf_rn(xs[c], xs[c], nk);
+  nk = __fsqrt_rn(nk);
+  const bool okk = isfinite(nk);
+  if (!okk) nk = 0.f;
+  int code[E];
+  float eps = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float u = nk > 0.f ? __fdiv_rn(xk[e], nk) : 0.f;
+    code[e] = kqv_code<16>(u, ka.t.kthr);
+    const float kh = __fmul_rn(nk, ka.t.kcent[code[e]]);
+    if (nk > 0.f) eps = fmaxf(eps, fabsf(__fsub_rn(xk[e], kh)));
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o *= 2) eps = fmaxf(eps, __shfl_xor_sync(0xffffffffu, eps, o));
+  {
+    uint8_t* kc = blk + slot * (D / 2) + lane * (E / 2);
+#pragma unroll
+    for (int e = 0; e < E; e += 2) kc[e / 2] = (uint8_t)(code[e] | (code[e + 1] << 4));
+  }
+  __syncwarp();   // every lane has read xs
+
+  // ---- values: rotate, norm, codes, residual, its norm ----
+  warp_rotate<E>(xv, a.signs, lane, a.rot_c);
+#pragma unroll
+  for (int e = 0; e < E; ++e) xs[lane * E + e] = xv[e];
+  __syncwarp();
+  float nv = 0.f;
+  for (int c = 0; c < D; ++c) nv = __fmaf_rn(xs[c], xs[c], nv);
+  nv = __fsqrt_rn(nv);
+  const bool okv = isfinite(nv);
+  if (!okv) nv = 0.f;
+  int vcode[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const float u = nv > 0.f ? __fdiv_rn(xv[e], nv) : 0.f;
+    vcode[e] = kqv_code<8>(u, ka.t.vthr);
+    rs[lane * E + e] = __fsub_rn(u, ka.t.vcent[vcode[e]]);
+  }
+  __syncwarp();
+  float rn = 0.f;
+  for (int c = 0; c < D; ++c) rn = __fmaf_rn(rs[c], rs[c], rn);
+  rn = __fsqrt_rn(rn);
+
+  // ---- the QJL sketch: projection i = lane + 32 m, a sequential chain over c ----
+  uint32_t word[E];
+#pragma unroll
+  for (int m = 0; m < E; ++m) {
+    const float* Si = ka.qjl + (int64_t)(lane + 32 * m) * D;
+    float acc = 0.f;
+    for (int c = 0; c < D; ++c) acc = __fmaf_rn(__ldg(Si + c), rs[c], acc);
+    word[m] = __ballot_sync(0xffffffffu, acc >= 0.f);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int m = 0; m < E; ++m)
+      reinterpret_cast<uint32_t*>(blk + L.vs() + slot * (D / 8))[m] = word[m];
+    reinterpret_cast<float*>(blk + L.kn())[slot] = nk;
+    reinterpret_cast<float*>(blk + L.ke())[slot] = nextafterf(eps, INFINITY);
+    reinterpret_cast<float*>(blk + L.vn())[slot] = nv;
+    reinterpret_cast<float*>(blk + L.vr())[slot] = rn;
+  }
+  {
+    uint8_t* vc = blk + L.vc() + slot * (D / 2) + lane * (E / 2);
+#pragma unroll
+    for (int e = 0; e < E; e += 2) vc[e / 2] = (uint8_t)(vcode[e] | (vcode[e + 1] << 4));
+  }
+
+  // ---- reconstruction: v^' = nv (c3 + rho S^T b), v^ = sigma o (c H v^') ----
+  const float rho = __fmul_rn(ka.qjl_c, rn);
+  float vh[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int c = lane * E + e;
+    float acc = 0.f;
+#pragma unroll
+    for (int m = 0; m < E; ++m)
+      for (int b = 0; b < 32; ++b) {
+        const float sgn = (word[m] >> b) & 1u ? 1.f : -1.f;
+        acc = __fmaf_rn(__ldg(ka.qjl + (int64_t)(32 * m + b) * D + c), sgn, acc);
+      }
+    vh[e] = __fmul_rn(nv, __fadd_rn(ka.t.vcent[vcode[e]], __fmul_rn(rho, acc)));
+  }
+  warp_hadamard<E>(vh, lane, a.rot_c);
+  float err = 0.f, hi = 0.f, lo = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if (a.signs[lane * E + e] < 0) vh[e] = -vh[e];
+    err = fmaxf(err, fabsf(__fsub_rn(vin[e], vh[e])));
+    hi = fmaxf(hi, vh[e]);
+    lo = fminf(lo, vh[e]);
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o *= 2) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, o));
+#pragma unroll
+  for (int o = 1; o < LPG; o *= 2) {
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+  }
+  if (!okk || !okv) err = 0.f;
+  if (lane == 0) {
+    if (!okk || !okv) set_error(a.err, KVQ_ERR_RANGE);
+    const float eu = nextafterf(__fmaf_rn(0x1p-16f, nv, err), INFINITY);
+    atomicMax(reinterpret_cast<int*>(a.eta + (int64_t)page * a.hkv + h), __float_as_int(eu));
+  }
+  if (lane % LPG == 0) {
+    // the block's range starts at [0, 0]: a maximum >= 0 orders like its int
+    // bits, a minimum <= 0 (sign bit set) like its unsigned bits, reversed
+    float* rg = reinterpret_cast<float*>(blk + L.rg()) + 2 * (lane / LPG);
+    if (hi > 0.f) atomicMax(reinterpret_cast<int*>(rg), __float_as_int(hi));
+    if (lo < 0.f) atomicMax(reinterpret_cast<unsigned int*>(rg + 1), __float_as_uint(lo));
+  }
+}
+
+cudaError_t launch_kqv_append(const KqvAppendArgs& a, int d, cudaStream_t stream) {
+  const int64_t items = (int64_t)a.a.num_seqs * a.a.num_tokens * a.a.hkv;
+  if (items == 0) return cudaSuccess;
+  const int64_t blocks = (items + 7) / 8;
+  if (d == 128) kqv_append_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  else if (d == 64) kqv_append_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(a);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+// ================================================================ decode =====
+constexpr int kKqWarps = 4;
+constexpr int kKqRows = 4;
+constexpr int kKqStages = 2;
+constexpr int kKqHdr = 16;   // floats: range max [NB], range min [NB], eta max
+__host__ __device__ constexpr int kqv_rec_floats(int d) { return kKqHdr + kKqRows * 8 + 2 * kKqRows * d; }
+
+template <int D>
+struct KqCfg {
+  // KqvLayout{D}.bytes(): codes, sketch, four fp32 per token, the range
+  static constexpr int BLOCK = kPage * D + kPage * D / 8 + 16 * kPage + (D / 32) * 8;
+  static constexpr int OFF_ST = 0;                                           // [warp][stage][BLOCK]
+  static constexpr int OFF_W = OFF_ST + kKqWarps * kKqStages * BLOCK;        // [warp][2][16][4] f32
+  static constexpr int OFF_LUT = OFF_W + kKqWarps * 2 * kPage * kKqRows * 4; // [16 + 8][32] f32
+  static constexpr int OFF_Q = OFF_LUT + 24 * 32 * 4;                       // q' [4][D] f32
+  static constexpr int OFF_QN = OFF_Q + kKqRows * D * 4;                    // |q'|_1, |q'|_2 [4][2]
+  static constexpr int OFF_BAR = (OFF_QN + 32 + 15) / 16 * 16;              // [warp][stage] u64
+  static constexpr int OFF_PG = OFF_BAR + kKqWarps * kKqStages * 8;          // [warp][stage] i32
+  static constexpr int END = OFF_PG + kKqWarps * kKqStages * 4;
+  // merge of the CTA's warps (aliases the stages): per warp [4][D] x 2, [4][8], header
+  static constexpr int MW = 2 * kKqRows * D + kKqRows * 8 + kKqHdr;
+  static constexpr int MERGE = kKqWarps * MW * 4;
+  static constexpr int SMEM = 128 + (END > MERGE ? END : MERGE);
+  static_assert(MERGE <= OFF_BAR, "the merge area must not reach the barriers");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDecodeArgs ka) {
+  using C = KqCfg<D>;
+  constexpr int E = D / 32, NB = D / 32;
+  const DecodeArgs& a = ka.a;
+  const KqvLayout L{D};
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
+  const int split = blockIdx.y, kvh = blockIdx.x % a.hkv, b = blockIdx.x / a.hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + warp * kKqStages;
+  int* spage = reinterpret_cast<int*>(sm + C::OFF_PG) + warp * kKqStages;
+  if (lane == 0) {
+    for (int s = 0; s < kKqStages; ++s) mbar_init(&bar[s], 1);
+    mbar_fence_init();
+  }
+  int n = a.seq_lens[b];
+  if (n < 0) n = 0;
+  const bool clamped = n > a.max_pages * kPage;
+  if (clamped) {
+    if (tid == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+    n = a.max_pages * kPage;
+  }
+  const int npages = (n + kPage - 1) / kPage;
+  const int p0 = split * a.pps;
+  if (p0 >= npages) return;   // inactive split (the merge reads active splits only)
+  const int p1 = min(npages, p0 + a.pps);
+
+  // ---- tables and query rows ----
+  float* lut = reinterpret_cast<float*>(sm + C::OFF_LUT);   // [24][32]: 16 key, 8 value entries
+  for (int i = tid; i < 24 * 32; i += blockDim.x) {
+    const int k = i / 32;
+    lut[i] = k < 16 ? ka.t.kcent[k] : ka.t.vcent[k - 16];
+  }
+  float* qs = reinterpret_cast<float*>(sm + C::OFF_Q);
+  float* qn = reinterpret_cast<float*>(sm + C::OFF_QN);
+  {
+    const int r = warp;   // 4 warps, 4 rows
+    float x[E];
+    if (r < a.R) {
+      const int qi = r / a.G, hq = kvh * a.G + r % a.G;
+      const int64_t e0 = (((int64_t)b * a.nq + qi) * a.hq + hq) * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = load_elem(a.q, a.q_bf16, e0 + e);
+      warp_rotate<E>(x, a.signs, lane, a.rot_c);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = 0.f;
+    }
+    float l1 = 0.f, l2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      qs[r * D + lane * E + e] = x[e];
+      l1 += fabsf(x[e]);
+      l2 = fmaf(x[e], x[e], l2);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o *= 2) {
+      l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      l2 += __shfl_xor_sync(0xffffffffu, l2, o);
+    }
+    if (lane == 0) {
+      qn[2 * r] = l1;
+      qn[2 * r + 1] = sqrtf(l2);
+    }
+  }
+  __syncthreads();
+  float qreg[kKqRows][E];
+#pragma unroll
+  for (int r = 0; r < kKqRows; ++r)
+#pragma unroll
+    for (int e = 0; e < E; ++e) qreg[r][e] = qs[r * D + lane * E + e];
+  const int myr = lane & 3;               // the row of this lane's scores
+  const float cq1 = kKappa * a.s_att * qn[2 * myr];
+  const float cq2 = kKappa * a.s_att * kRotSlack * qn[2 * myr + 1];
+  const float zsc = a.s_att * kLog2e;
+
+  // ---- pages of this warp: p0 + warp, p0 + warp + 4, ... ----
+  const int first = p0 + warp;
+  const int nloc = first < p1 ? (p1 - first + kKqWarps - 1) / kKqWarps : 0;
+  uint8_t* stage0 = sm + C::OFF_ST + warp * kKqStages * C::BLOCK;
+  const int32_t* ptab = a.page_table + (int64_t)b * a.max_pages;
+  auto issue = [&](int j, int st) {
+    if (lane == 0) {
+      const int pg = ptab[first + j * kKqWarps];
+      const bool ok = pg >= 0 && pg < a.num_pages;
+      spage[st] = ok ? pg : -1;
+      if (ok) {
+        mbar_arrive_expect_tx(&bar[st], C::BLOCK);
+        bulk_g2s_hint(stage0 + st * C::BLOCK, a.pool + ((int64_t)pg * a.hkv + kvh) * C::BLOCK,
+                      C::BLOCK, &bar[st], l2_evict_first_policy());
+      } else {
+        set_error(a.err, KVQ_ERR_INVALID_ARG);
+        mbar_arrive(&bar[st]);
+      }
+    }
+    __syncwarp();
+  };
+  for (int j = 0; j < kKqStages && j < nloc; ++j) issue(j, j);
+
+  float acc1[kKqRows][E], acc2[kKqRows][E];
+#pragma unroll
+  for (int r = 0; r < kKqRows; ++r)
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc1[r][e] = acc2[r][e] = 0.f;
+  float m2 = -INFINITY, lsum = 0.f, Asum = 0.f, Bsum = 0.f, Esum = 0.f, dmax = 0.f;
+  float rhi[NB], rlo[NB], etamax = clamped ? INFINITY : 0.f;
+#pragma unroll
+  for (int g = 0; g < NB; ++g) {
+    rhi[g] = -INFINITY;
+    rlo[g] = INFINITY;
+  }
+  float* wts = reinterpret_cast<float*>(sm + C::OFF_W) + warp * 2 * kPage * kKqRows;
+  int jstop = nloc;
+  for (int j = 0; j < nloc; ++j) {
+    const int st = j % kKqStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar[st], (uint32_t)((j / kKqStages) & 1)))) {
+      if (lane == 0) set_error(a.err, KVQ_ERR_TIMEOUT);
+      etamax = INFINITY;
+      jstop = j;
+      break;
+    }
+    const int pg = spage[st];
+    if (pg < 0) {
+      etamax = INFINITY;   // the page was not read
+    } else {
+      const uint8_t* blk = stage0 + st * C::BLOCK;
+      const float* fk = reinterpret_cast<const float*>(blk + L.kn());
+      const float* fe = reinterpret_cast<const float*>(blk + L.ke());
+      const float* fv = reinterpret_cast<const float*>(blk + L.vn());
+      const float* fr = reinterpret_cast<const float*>(blk + L.vr());
+      const float* frg = reinterpret_cast<const float*>(blk + L.rg());
+      const int nval = min(kPage, n - (first + j * kKqWarps) * kPage);
+      const float eta_pg = __ldg(a.eta + (int64_t)pg * a.hkv + kvh);
+      etamax = fmaxf(etamax, eta_pg);
+#pragma unroll
+      for (int g = 0; g < NB; ++g) {
+        rhi[g] = fmaxf(rhi[g], frg[2 * g]);
+        rlo[g] = fminf(rlo[g], frg[2 * g + 1]);
+      }
+      // ---- scores of tokens t0 = lane / 4 and t0 + 8 for row lane % 4 ----
+      float zs2[2];
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        // partial scores of tokens 8 hf + tl, rows r: index tl * 4 + r
+        float part[32];
+#pragma unroll
+        for (int tl = 0; tl < 8; ++tl) {
+          const int t = 8 * hf + tl;
+          const uint8_t* kc = blk + t * (D / 2) + lane * (E / 2);
+          float cv[E];
+#pragma unroll
+          for (int e = 0; e < E; e += 2) {
+            const unsigned byte = kc[e / 2];
+            cv[e] = lut[(byte & 15u) * 32 + lane];
+            cv[e + 1] = lut[(byte >> 4) * 32 + lane];
+          }
+#pragma unroll
+          for (int r = 0; r < kKqRows; ++r) {
+            float s = qreg[r][0] * cv[0];
+#pragma unroll
+            for (int e = 1; e < E; ++e) s = fmaf(qreg[r][e], cv[e], s);
+            part[tl * 4 + r] = s;
+          }
+        }
+        // reduce-scatter over the warp: lane l ends with the sum of index l
+#pragma unroll
+        for (int o = 16, cnt = 32; o >= 1; o >>= 1, cnt >>= 1) {
+          const bool up = (lane & o) != 0;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            if (k < cnt / 2) {
+              const float send = up ? part[k] : part[cnt / 2 + k];
+              const float keep = up ? part[cnt / 2 + k] : part[k];
+              part[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+          }
+        }
+        zs2[hf] = part[0];
+      }
+      // ---- online softmax and the bound's sums, once per page ----
+      float zt[2], dl[2];
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int t = 8 * hf + (lane >> 2);
+        const bool vt = t < nval;
+        const float nk = fk[t];
+        zt[hf] = vt ? zs2[hf] * nk * zsc : -INFINITY;
+        dl[hf] = vt ? fmaf(cq1, fe[t], cq2 * nk) : 0.f;
+      }
+      float mx = fmaxf(zt[0], zt[1]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mref = mx > m2 + 2.0f ? mx : m2;
+      const float alpha = ex2(m2 - mref);
+      m2 = mref;
+      float tl_ = 0.f, ta = 0.f, tb = 0.f;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int t = 8 * hf + (lane >> 2);
+        const bool vt = t < nval;
+        const float wv = ex2(zt[hf] - mref);
+        const float d = dl[hf];
+        const float ed = ex2(d * kLog2e), en = ex2(-d * kLog2e);
+        const float em = d < 0.015625f ? d * fmaf(d, fmaf(d, 1.0f / 6, 0.5f), 1.0f) : ed - 1.0f;
+        tl_ += wv;
+        ta = fmaf(wv, em, ta);
+        tb = fmaf(wv, en, tb);
+        dmax = fmaxf(dmax, d);
+        // weights of the PV accumulations (0 outside the context: the slots
+        // past it may hold another sequence's norms)
+        const float wa = vt ? wv * fv[t] : 0.f;
+        wts[t * 4 + (lane & 3)] = wa;
+        wts[kPage * 4 + t * 4 + (lane & 3)] = vt ? wa * fr[t] : 0.f;
+      }
+      lsum = fmaf(lsum, alpha, tl_);
+      Asum = fmaf(Asum, alpha, ta);
+      Bsum = fmaf(Bsum, alpha, tb);
+      Esum = fmaf(Esum, alpha, tl_ * eta_pg);
+      if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+        for (int r = 0; r < kKqRows; ++r) {
+          const float ar = __shfl_sync(0xffffffffu, alpha, r);
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            acc1[r][e] *= ar;
+            acc2[r][e] *= ar;
+          }
+        }
+      }
+      __syncwarp();
+      // ---- PV: lane l owns channels (and projections) [l E, l E + E) ----
+#pragma unroll 4
+      for (int t = 0; t < kPage; ++t) {
+        const float4 wa4 = reinterpret_cast<const float4*>(wts)[t];
+        const float4 wb4 = reinterpret_cast<const float4*>(wts + kPage * 4)[t];
+        const uint8_t* vc = blk + L.vc() + t * (D / 2) + lane * (E / 2);
+        const unsigned sb = blk[L.vs() + t * (D / 8) + (lane * E) / 8] >> ((lane * E) % 8);
+        float cv[E], sg[E];
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          const unsigned byte = vc[e / 2];
+          cv[e] = lut[(16 + (byte & 15u)) * 32 + lane];
+          cv[e + 1] = lut[(16 + (byte >> 4)) * 32 + lane];
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) sg[e] = (sb >> e) & 1u ? 1.f : -1.f;
+        const float war[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
+        const float wbr[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
+#pragma unroll
+        for (int r = 0; r < kKqRows; ++r)
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            acc1[r][e] = fmaf(war[r], cv[e], acc1[r][e]);
+            acc2[r][e] = fmaf(wbr[r], sg[e], acc2[r][e]);
+          }
+      }
+    }
+    __syncwarp();
+    if (j + kKqStages < nloc) issue(j + kKqStages, st);
+  }
+  // after a wait that ran out, the copies still in flight are waited for
+  // (bounded) before the stages become the merge area
+  if (jstop < nloc)
+    for (int j = jstop; j < nloc && j < jstop + kKqStages; ++j)
+      (void)mbar_wait(&bar[j % kKqStages], (uint32_t)((j / kKqStages) & 1));
+
+  // ---- per-warp sums over the lanes of each row ----
+#pragma unroll
+  for (int o = 4; o < 32; o *= 2) {
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    Asum += __shfl_xor_sync(0xffffffffu, Asum, o);
+    Bsum += __shfl_xor_sync(0xffffffffu, Bsum, o);
+    Esum += __shfl_xor_sync(0xffffffffu, Esum, o);
+    dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+  }
+  __syncthreads();   // every warp is done with its stages
+  float* mw = reinterpret_cast<float*>(sm) + warp * C::MW;
+#pragma unroll
+  for (int r = 0; r < kKqRows; ++r)
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      mw[r * D + lane * E + e] = acc1[r][e];
+      mw[kKqRows * D + r * D + lane * E + e] = acc2[r][e];
+    }
+  if (lane < 4) {
+    float* stt = mw + 2 * kKqRows * D + lane * 8;
+    stt[0] = m2;
+    stt[1] = lsum;
+    stt[2] = Asum;
+    stt[3] = Bsum;
+    stt[4] = Esum;
+    stt[5] = dmax;
+  }
+  if (lane == 0) {
+    float* hd = mw + 2 * kKqRows * D + kKqRows * 8;
+#pragma unroll
+    for (int g = 0; g < NB; ++g) {
+      hd[g] = rhi[g];
+      hd[NB + g] = rlo[g];
+    }
+    hd[2 * NB] = etamax;
+  }
+  __syncthreads();
+  // ---- warp r merges row r of the 4 warps into this split's record ----
+  const int r = warp;
+  float* rec = a.part + ((int64_t)blockIdx.x * gridDim.y + split) * kqv_rec_floats(D);
+  float mW = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kKqWarps; ++w) mW = fmaxf(mW, reinterpret_cast<float*>(sm)[w * C::MW + 2 * kKqRows * D + r * 8]);
+  float st5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+  float o1[E], o2[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) o1[e] = o2[e] = 0.f;
+#pragma unroll
+  for (int w = 0; w < kKqWarps; ++w) {
+    const float* mwp = reinterpret_cast<float*>(sm) + w * C::MW;
+    const float* stw = mwp + 2 * kKqRows * D + r * 8;
+    const float f = stw[0] == -INFINITY ? 0.f : ex2(stw[0] - mW);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) st5[k] = fmaf(f, stw[1 + k], st5[k]);
+    st5[4] = fmaxf(st5[4], stw[5]);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      o1[e] = fmaf(f, mwp[r * D + lane * E + e], o1[e]);
+      o2[e] = fmaf(f, mwp[kKqRows * D + r * D + lane * E + e], o2[e]);
+    }
+  }
+  if (r == 0 && lane < kKqHdr) {
+    float hv = 0.f;
+    if (lane < 2 * NB + 1) {
+      hv = lane < NB ? -INFINITY : (lane < 2 * NB ? INFINITY : 0.f);
+#pragma unroll
+      for (int w = 0; w < kKqWarps; ++w) {
+        const float x = reinterpret_cast<float*>(sm)[w * C::MW + 2 * kKqRows * D + kKqRows * 8 + lane];
+        hv = lane < NB ? fmaxf(hv, x) : (lane < 2 * NB ? fminf(hv, x) : fmaxf(hv, x));
+      }
+    }
+    rec[lane] = hv;
+  }
+  if (lane == 0) {
+    float* rs = rec + kKqHdr + r * 8;
+    rs[0] = mW;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) rs[1 + k] = st5[k];
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    rec[kKqHdr + kKqRows * 8 + r * D + lane * E + e] = o1[e];
+    rec[kKqHdr + kKqRows * 8 + kKqRows * D + r * D + lane * E + e] = o2[e];
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kKqWarps * 32) kqv_merge_kernel(const KqvDecodeArgs ka) {
+  constexpr int E = D / 32, NB = D / 32;
+  constexpr int RF = kqv_rec_floats(D);
+  const DecodeArgs& a = ka.a;
+  __shared__ float sB[kKqWarps][D];
+  __shared__ float shd[kKqHdr];
+  const int unit = blockIdx.x, kvh = unit % a.hkv, b = unit / a.hkv;
+  const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n = a.seq_lens[b];
+  if (n < 0) n = 0;
+  if (n > a.max_pages * kPage) n = a.max_pages * kPage;
+  const int npages = (n + kPage - 1) / kPage;
+  const int active = (npages + a.pps - 1) / a.pps;
+  const int qi = r / a.G, hq = kvh * a.G + r % a.G;
+  const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + hq;
+  if (npages == 0) {   // empty context: zero output, zero bound (uniform over the CTA)
+    if (r < a.R) {
+      if (a.out)
+        for (int c = lane; c < D; c += 32) a.out[row * D + c] = 0.f;
+      if (lane == 0) {
+        a.bound[row] = 0.f;
+        a.flags[row] = 0;
+      }
+    }
+    return;
+  }
+  const float* ubase = a.part + (int64_t)unit * ka.nsp * RF;
+  if (r == 0 && lane < 2 * NB + 1) {
+    float hv = lane < NB ? -INFINITY : (lane < 2 * NB ? INFINITY : 0.f);
+    for (int sp = 0; sp < active; ++sp) {
+      const float x = __ldcg(ubase + (int64_t)sp * RF + lane);
+      hv = lane < NB ? fmaxf(hv, x) : (lane < 2 * NB ? fminf(hv, x) : fmaxf(hv, x));
+    }
+    shd[lane] = hv;
+  }
+  float M = -INFINITY, l = 0.f, A = 0.f, Bv = 0.f, Ev = 0.f, dm = 0.f;
+  float o1[E], o2[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) o1[e] = o2[e] = 0.f;
+  for (int sp = 0; sp < active; ++sp) {
+    const float* rec = ubase + (int64_t)sp * RF;
+    const float* st = rec + kKqHdr + r * 8;
+    const float ms = __ldcg(st);
+    if (ms == -INFINITY) continue;   // a split whose pages were all outside the row's context
+    const float Mn = fmaxf(M, ms);
+    const float fo = M == -INFINITY ? 0.f : ex2(M - Mn);
+    const float fs = ex2(ms - Mn);
+    l = fmaf(l, fo, fs * __ldcg(st + 1));
+    A = fmaf(A, fo, fs * __ldcg(st + 2));
+    Bv = fmaf(Bv, fo, fs * __ldcg(st + 3));
+    Ev = fmaf(Ev, fo, fs * __ldcg(st + 4));
+    dm = fmaxf(dm, __ldcg(st + 5));
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int c = lane * E + e;
+      o1[e] = fmaf(o1[e], fo, fs * __ldcg(rec + kKqHdr + kKqRows * 8 + r * D + c));
+      o2[e] = fmaf(o2[e], fo, fs * __ldcg(rec + kKqHdr + kKqRows * 8 + kKqRows * D + r * D + c));
+    }
+    M = Mn;
+  }
+  const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) sB[r][lane * E + e] = o2[e] * inv_l;
+  __syncthreads();   // sB of every warp and the merged header
+  // o' = o1 / l + sqrt(pi/2)/d * S^T (o2 / l), then o = sigma o (c H o')
+  float x[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int c = lane * E + e;
+    float acc = 0.f;
+    for (int i = 0; i < D; ++i) acc = fmaf(__ldg(ka.qjl + (int64_t)i * D + c), sB[r][i], acc);
+    x[e] = fmaf(ka.qjl_c, acc, o1[e] * inv_l);
+  }
+  warp_hadamard<E>(x, lane, a.rot_c);
+  if (r >= a.R) return;
+  if (a.out) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int c = lane * E + e;
+      a.out[row * D + c] = a.signs[c] < 0 ? -x[e] : x[e];
+    }
+  }
+  if (lane == 0) {
+    const bool skipped = shd[2 * NB] == INFINITY;   // a page of the unit was not read
+    float bd = skipped ? INFINITY : 0.f;
+    if (!skipped && l > 0.f) {
+      float range = 0.f;
+#pragma unroll
+      for (int g = 0; g < NB; ++g) range = fmaxf(range, shd[g] - shd[NB + g]);
+      const float tv = fminf(tanhf(0.5f * dm), A / Bv);
+      bd = kKappa * (tv * (range + 2.0f * shd[2 * NB]) + Ev / l);
+    }
+    a.bound[row] = bd;
+    a.flags[row] = skipped || bd > a.tau ? 1 : 0;
+  }
+}
+
+const void* kqv_partial_kernel(int d) {
+  if (d == 128) return reinterpret_cast<const void*>(kqv_partial_kernel<128>);
+  if (d == 64) return reinterpret_cast<const void*>(kqv_partial_kernel<64>);
+  return nullptr;
+}
+int kqv_partial_smem(int d) { return d == 128 ? KqCfg<128>::SMEM : KqCfg<64>::SMEM; }
+int kqv_record_floats(int d) { return kqv_rec_floats(d); }
+int kqv_threads() { return kKqWarps * 32; }
+
+cudaError_t launch_kqv_decode(const KqvDecodeArgs& a, int d, int units, int splits,
+                              cudaStream_t stream) {
+  if (units == 0) return cudaSuccess;
+  const dim3 grid((unsigned)units, (unsigned)splits, 1);
+  if (d == 128) {
+    kqv_partial_kernel<128><<<grid, kKqWarps * 32, KqCfg<128>::SMEM, stream>>>(a);
+    kqv_merge_kernel<128><<<units, kKqWarps * 32, 0, stream>>>(a);
+  } else if (d == 64) {
+    kqv_partial_kernel<64><<<grid, kKqWarps * 32, KqCfg<64>::SMEM, stream>>>(a);
+    kqv_merge_kernel<64><<<units, kKqWarps * 32, 0, stream>>>(a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvq
+
+extern "C" int kvq_kqv_codebook(int32_t bits, int32_t head_dim, float* centroids,
+                                float* thresholds) {
+  if (bits < 1 || bits > 6 || head_dim < 1 || !centroids || !thresholds) return KVQ_ERR_INVALID_ARG;
+  double c[64];
+  kvq::lloyd_max_normal(bits, c);
+  const int L = 1 << bits;
+  const double sd = std::sqrt((double)head_dim);
+  for (int i = 0; i < L; ++i) centroids[i] = (float)(c[i] / sd);
+  for (int i = 0; i + 1 < L; ++i) thresholds[i] = (float)((c[i] + c[i + 1]) / (2.0 * sd));
+  return KVQ_OK;
+}

@@ -41,11 +41,31 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+int check_kqv(const kvq_cache* c) {
+  if (c->k_bits != 4 || c->v_bits != 3 || c->k_group != c->head_dim || c->v_group != c->head_dim)
+    return fail(KVQ_ERR_UNSUPPORTED, "the KQV codec takes k_bits 4, v_bits 3 and groups of head_dim");
+  if (c->k_rotate != 1 || !c->rot_signs)
+    return fail(KVQ_ERR_INVALID_ARG, "the KQV codec needs k_rotate 1 and rot_signs");
+  if (!c->qjl) return fail(KVQ_ERR_INVALID_ARG, "the KQV codec needs the QJL matrix");
+  if (c->outliers != 0) return fail(KVQ_ERR_UNSUPPORTED, "the KQV codec has no outlier extraction");
+  return KVQ_OK;
+}
+
 int check_cache(const kvq_cache* c) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
   if (c->page_size != KVQ_PAGE_SIZE) return fail(KVQ_ERR_UNSUPPORTED, "page_size must be 16");
   if (c->head_dim != 64 && c->head_dim != 128)
     return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", c->head_dim);
+  if (c->codec != KVQ_CODEC_INT && c->codec != KVQ_CODEC_KQV)
+    return fail(KVQ_ERR_INVALID_ARG, "codec %d unknown", c->codec);
+  if (c->codec == KVQ_CODEC_KQV) {
+    if (int rc = check_kqv(c)) return rc;
+    if (c->num_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "num_kv_heads < 1");
+    if (c->num_pages < 0) return fail(KVQ_ERR_INVALID_ARG, "num_pages < 0");
+    if (!c->pool || !c->v_eta) return fail(KVQ_ERR_INVALID_ARG, "pool or v_eta is NULL");
+    if (!aligned16(c->pool)) return fail(KVQ_ERR_INVALID_ARG, "pool not 16-byte aligned");
+    return KVQ_OK;
+  }
   if (c->k_bits != 8 && c->k_bits != 4)
     return fail(KVQ_ERR_UNSUPPORTED, "k_bits %d unsupported (8 or 4)", c->k_bits);
   if (c->k_group != 32 && c->k_group != 64 && c->k_group != 128)
@@ -70,6 +90,8 @@ BlockLayout layout_of(const kvq_cache* c) {
 }
 
 float rot_constant(int d) { return (float)(1.0 / std::sqrt((double)d)); }
+// fp32(sqrt(pi/2) / d): the QJL estimate's scale per unit of |r|
+float kqv_qjl_constant(int d) { return (float)(std::sqrt(3.14159265358979323846 / 2.0) / d); }
 
 struct DeviceInfo {
   int sms = 0, major = 0, max_smem = 0;
@@ -141,14 +163,41 @@ constexpr int kMaxPagesPerSplit = 256;
 // Split-K sizing: fill every SM's resident slots once with (sequence, kv head,
 // split) CTAs; long contexts cap the pages of one split so a ragged batch
 // spreads over several waves.
+// blocks of the KQV codec's partial decode kernel resident per SM
+int kqv_occupancy(int d, int* occ) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto key = std::make_pair(dev, d);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    const void* k = kqv_partial_kernel(d);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kqv_partial_smem(d));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kqv_threads(), kqv_partial_smem(d));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    it = cache.emplace(key, n < 1 ? 1 : n).first;
+  }
+  *occ = it->second;
+  return KVQ_OK;
+}
+
 int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
-  DecodeVariant v = select_decode_kernel(c->head_dim, c->k_bits, c->k_group, c->outliers);
-  if (!v.kernel) return fail(KVQ_ERR_UNSUPPORTED, "no decode kernel for this codec");
+  const bool kqv = c->codec == KVQ_CODEC_KQV;
+  DecodeVariant v{nullptr, nullptr, 0, 0};
+  if (!kqv) {
+    v = select_decode_kernel(c->head_dim, c->k_bits, c->k_group, c->outliers);
+    if (!v.kernel) return fail(KVQ_ERR_UNSUPPORTED, "no decode kernel for this codec");
+  }
   DeviceInfo di;
   int rc = device_info(&di, nullptr);
   if (rc) return rc;
   int occ = 1;
-  if ((rc = decode_occupancy(v, &occ))) return rc;
+  if ((rc = kqv ? kqv_occupancy(c->head_dim, &occ) : decode_occupancy(v, &occ))) return rc;
   const int64_t units = (int64_t)num_seqs * c->num_kv_heads;
   const int64_t slots = (int64_t)di.sms * occ;
   int64_t splits = units > 0 ? std::max<int64_t>(1, slots / units) : 1;
@@ -165,7 +214,8 @@ int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
   p->splits = (int)splits;
   p->pps = (int)pps;
   p->counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
-  p->part_bytes = (size_t)units * splits * v.record * sizeof(float);
+  p->part_bytes = (size_t)units * splits * (kqv ? kqv_record_floats(c->head_dim) : v.record) *
+                  sizeof(float);
   return KVQ_OK;
 }
 
@@ -205,8 +255,11 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
     return fail(KVQ_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", ws_bytes,
                 plan.total());
   if (!aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");
-  DecodeVariant v = select_decode_kernel(cache->head_dim, cache->k_bits, cache->k_group,
-                                         cache->outliers);
+  const bool kqv = cache->codec == KVQ_CODEC_KQV;
+  if (kqv && nt) return fail(KVQ_ERR_UNSUPPORTED, "the KQV codec has no fused append");
+  DecodeVariant v{nullptr, nullptr, 0, 0};
+  if (!kqv)
+    v = select_decode_kernel(cache->head_dim, cache->k_bits, cache->k_group, cache->outliers);
   DecodeArgs a;
   a.pool = static_cast<const uint8_t*>(cache->pool);
   a.eta = cache->v_eta;
@@ -243,6 +296,17 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
   if (units > 0x7fffffffLL || plan.splits > 65535)
     return fail(KVQ_ERR_UNSUPPORTED, "grid too large (%lld units, %d splits)", (long long)units,
                 plan.splits);
+  if (kqv) {
+    KqvDecodeArgs ka;
+    ka.a = a;
+    ka.qjl = cache->qjl;
+    ka.qjl_c = kqv_qjl_constant(cache->head_dim);
+    ka.nsp = plan.splits;
+    kqv_tables(cache->head_dim, &ka.t);
+    cudaError_t e = launch_kqv_decode(ka, cache->head_dim, (int)units, plan.splits, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "KQV decode launch");
+    return KVQ_OK;
+  }
   dim3 grid((unsigned)units, (unsigned)plan.splits, 1);
   cudaError_t e = launch_pdl(nt ? v.kernel_append : v.kernel, grid, dim3(decode_threads()),
                              (size_t)v.smem, stream, a);
@@ -276,8 +340,14 @@ const char* kvq_last_error(void) { return g_last_error.c_str(); }
 
 size_t kvq_block_bytes(const kvq_cache* cache) {
   if (!cache || cache->page_size != KVQ_PAGE_SIZE) return 0;
-  if ((cache->head_dim != 64 && cache->head_dim != 128) || (cache->k_bits != 8 && cache->k_bits != 4))
-    return 0;
+  if (cache->head_dim != 64 && cache->head_dim != 128) return 0;
+  if (cache->codec == KVQ_CODEC_KQV) {
+    if (cache->k_bits != 4 || cache->v_bits != 3 || cache->k_group != cache->head_dim ||
+        cache->v_group != cache->head_dim || cache->outliers != 0)
+      return 0;
+    return (size_t)KqvLayout{cache->head_dim}.bytes();
+  }
+  if (cache->codec != KVQ_CODEC_INT || (cache->k_bits != 8 && cache->k_bits != 4)) return 0;
   if (cache->k_group != 32 && cache->k_group != 64 && cache->k_group != 128) return 0;
   if (cache->head_dim % cache->k_group || cache->v_bits != 4 || cache->v_group != 32) return 0;
   if (cache->outliers != 0 && cache->outliers != 1) return 0;
@@ -327,6 +397,16 @@ int kvq_quantize_append(const kvq_cache* cache, const void* k, const void* v, in
   a.start_pos = start_pos;
   a.page_table = page_table;
   a.rot_c = rot_constant(cache->head_dim);
+  if (cache->codec == KVQ_CODEC_KQV) {
+    KqvAppendArgs ka;
+    ka.a = a;
+    ka.qjl = cache->qjl;
+    ka.qjl_c = kqv_qjl_constant(cache->head_dim);
+    kqv_tables(cache->head_dim, &ka.t);
+    cudaError_t e = launch_kqv_append(ka, cache->head_dim, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "KQV append kernel launch");
+    return KVQ_OK;
+  }
   cudaError_t e = launch_append(a, cache->head_dim, cache->k_bits, cache->k_group, cache->outliers,
                                 reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
@@ -646,7 +726,8 @@ extern "C" {
 
 size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs, int32_t num_queries,
                               int32_t num_q_heads, int32_t max_pages_per_seq) {
-  if (check_cache(cache) || cache->outliers || num_seqs < 0 || num_queries < 1 ||
+  if (check_cache(cache) || cache->outliers || cache->codec != KVQ_CODEC_INT || num_seqs < 0 ||
+      num_queries < 1 ||
       num_q_heads < 1 || max_pages_per_seq < 1 || max_pages_per_seq > kAdMaxPages)
     return 0;
   const int64_t units = (int64_t)num_seqs * cache->num_kv_heads;
@@ -686,9 +767,9 @@ int kvq_adaptive_precision(const kvq_cache* cache, const void* k_orig_host,
   if (num_flagged) *num_flagged = 0;
   int rc = check_cache(cache);
   if (rc) return rc;
-  if (cache->outliers)
-    return fail(KVQ_ERR_UNSUPPORTED, "the adaptive-precision ladder reads caches without "
-                "outlier extraction only");
+  if (cache->outliers || cache->codec != KVQ_CODEC_INT)
+    return fail(KVQ_ERR_UNSUPPORTED, "the adaptive-precision ladder reads Tier-1 caches "
+                "without outlier extraction only");
   if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad orig_dtype");
   if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad q_dtype");
   if (num_seqs < 0 || num_queries < 1 || num_q_heads < 1 || max_pages_per_seq < 1 ||

@@ -218,11 +218,19 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 // c = fp32(1/sqrt(d)); every operation is a single fp32 add, sub or mul, so
 // the result does not depend on how the butterflies are distributed.
 template <int E>
+__device__ __forceinline__ void warp_hadamard(float (&x)[E], int lane, float c);
+template <int E>
 __device__ __forceinline__ void warp_rotate(float (&x)[E], const int8_t* sigma, int lane,
                                             float c) {
 #pragma unroll
   for (int e = 0; e < E; ++e)
     if (sigma[lane * E + e] < 0) x[e] = -x[e];
+  warp_hadamard<E>(x, lane, c);
+}
+// The butterflies and the product by c of warp_rotate, without the signs:
+// y = c * H_d * x (its own inverse, since (c H_d)^2 = I).
+template <int E>
+__device__ __forceinline__ void warp_hadamard(float (&x)[E], int lane, float c) {
 #pragma unroll
   for (int h = 1; h < E; h *= 2) {
 #pragma unroll

@@ -163,6 +163,48 @@ cudaError_t launch_adaptive_correct(const AdArgs& a, int d, int kbits, int kgrou
 cudaError_t launch_adaptive_finish(const AdArgs& a, int d, cudaStream_t s);
 int adaptive_select_smem(int max_pages, int d);
 
+// ---- the KQV codec (kqv.cu) -------------------------------------------------
+// Byte layout of one (page, kv head) block: K codes (nibbles), V codes
+// (3-bit in nibbles), V sketch bits, then per token |k'|, eps, |v'|, |r|
+// (fp32), then the block's v^ max / min per 32-channel group.
+struct KqvLayout {
+  int d;
+  __host__ __device__ int vc() const { return kPage * d / 2; }
+  __host__ __device__ int vs() const { return kPage * d; }
+  __host__ __device__ int kn() const { return kPage * d + kPage * d / 8; }
+  __host__ __device__ int ke() const { return kn() + 4 * kPage; }
+  __host__ __device__ int vn() const { return kn() + 8 * kPage; }
+  __host__ __device__ int vr() const { return kn() + 12 * kPage; }
+  __host__ __device__ int rg() const { return kn() + 16 * kPage; }
+  __host__ __device__ int bytes() const { return rg() + (d / 32) * 8; }
+};
+// fp32 codebooks: 4-bit keys, 3-bit values
+struct KqvTables {
+  float kcent[16], kthr[15], vcent[8], vthr[7];
+};
+struct KqvAppendArgs {
+  AppendArgs a;
+  const float* qjl;   // S [d][d]
+  float qjl_c;        // fp32(sqrt(pi/2) / d)
+  KqvTables t;
+};
+struct KqvDecodeArgs {
+  DecodeArgs a;       // out, bound, flags, part as for the Tier-1 decode; no fused append
+  const float* qjl;
+  float qjl_c;
+  int nsp;            // splits of the partial grid (records per unit)
+  KqvTables t;
+};
+int kqv_tables(int d, KqvTables* t);   // host; cached per head_dim
+cudaError_t launch_kqv_append(const KqvAppendArgs& a, int d, cudaStream_t s);
+// the partial kernel over (unit, split), then the merge per unit
+cudaError_t launch_kqv_decode(const KqvDecodeArgs& a, int d, int units, int splits,
+                              cudaStream_t s);
+const void* kqv_partial_kernel(int d);
+int kqv_partial_smem(int d);
+int kqv_record_floats(int d);
+int kqv_threads();
+
 cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, int out,
                           cudaStream_t s);
 // out: the cache's outlier extraction (0 or 1)

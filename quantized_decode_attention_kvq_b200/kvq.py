@@ -30,6 +30,8 @@ KVQ_ERR_TIMEOUT = -5
 KVQ_ERR_DEVICE = -6
 KVQ_F32 = 0
 KVQ_BF16 = 1
+KVQ_CODEC_INT = 0
+KVQ_CODEC_KQV = 1
 PAGE_SIZE = 16
 
 EXPORTED = ("kvq_block_bytes", "kvq_pool_bytes", "kvq_quantize_append", "kvq_workspace_size",
@@ -37,7 +39,7 @@ EXPORTED = ("kvq_block_bytes", "kvq_pool_bytes", "kvq_quantize_append", "kvq_wor
             "kvq_fallback_exact", "kvq_device_error", "kvq_status_string", "kvq_last_error",
             "kvq_decode_attention_noalloc", "kvq_decode_attention_append",
             "kvq_adaptive_work_size", "kvq_adaptive_host_size", "kvq_adaptive_staging_size",
-            "kvq_adaptive_precision")
+            "kvq_adaptive_precision", "kvq_kqv_codebook")
 
 
 class KvqError(RuntimeError):
@@ -53,7 +55,8 @@ class kvq_cache(ctypes.Structure):
                 ("k_rotate", ctypes.c_int32), ("v_bits", ctypes.c_int32),
                 ("v_group", ctypes.c_int32), ("pool", ctypes.c_void_p),
                 ("v_eta", ctypes.c_void_p), ("rot_signs", ctypes.c_void_p),
-                ("error_word", ctypes.c_void_p), ("outliers", ctypes.c_int32)]
+                ("error_word", ctypes.c_void_p), ("outliers", ctypes.c_int32),
+                ("codec", ctypes.c_int32), ("qjl", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -93,6 +96,7 @@ def _load() -> ctypes.CDLL:
                                                   SZ, P, P, I32, ctypes.POINTER(I32),
                                                   ctypes.POINTER(I32)]),
         "kvq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "kvq_kqv_codebook": (ctypes.c_int, [I32, I32, P, P]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
@@ -284,10 +288,17 @@ class PagedCache:
 
     def __init__(self, num_kv_heads: int, head_dim: int, num_pages: int, k_bits: int = 8,
                  k_group: int = 128, k_rotate: bool = False, rot_signs=None, v_bits: int = 4,
-                 v_group: int = 32, outliers: bool = False, device="cuda"):
+                 v_group: int = 32, outliers: bool = False, codec: str = "int", qjl_matrix=None,
+                 device="cuda"):
+        """codec "int": the Tier-1 INT8/INT4 codec (k_bits, k_group, k_rotate,
+        outliers apply); codec "kqv": the KQV codec (rotation with rot_signs, 4-bit
+        Lloyd-Max keys, 3-bit values plus the QJL sketch with qjl_matrix [d][d])."""
+        if codec == "kqv":
+            k_bits, v_bits, k_group, v_group, k_rotate = 4, 3, head_dim, head_dim, True
         self.desc = kvq_cache(num_kv_heads, head_dim, PAGE_SIZE, num_pages, k_bits, k_group,
                               int(bool(k_rotate)), v_bits, v_group, None, None, None, None,
-                              int(bool(outliers)))
+                              int(bool(outliers)),
+                              KVQ_CODEC_KQV if codec == "kqv" else KVQ_CODEC_INT, None)
         bb = kvq_block_bytes(self.desc)
         if bb == 0:
             raise KvqError(KVQ_ERR_UNSUPPORTED, "kvq_block_bytes")
@@ -304,6 +315,10 @@ class PagedCache:
         self.desc.v_eta = self.eta.data_ptr()
         self.desc.rot_signs = None if self.signs is None else self.signs.data_ptr()
         self.desc.error_word = self.error_word.data_ptr()
+        self.qjl = None
+        if codec == "kqv":
+            self.qjl = torch.as_tensor(qjl_matrix, dtype=torch.float32).to(device).contiguous()
+            self.desc.qjl = self.qjl.data_ptr()
 
     @property
     def head_dim(self) -> int:
@@ -359,3 +374,13 @@ class PagedCache:
         rc, code = kvq_device_error(self.desc, stream)
         _check(rc, "kvq_device_error")
         return code
+
+
+def kqv_codebook(bits: int, head_dim: int):
+    """The KQV codec's fp32 centroids and thresholds (kvq_kqv_codebook)."""
+    import numpy as np
+    cent = np.zeros(1 << bits, dtype=np.float32)
+    thr = np.zeros((1 << bits) - 1, dtype=np.float32)
+    _check(lib().kvq_kqv_codebook(bits, head_dim, cent.ctypes.data, thr.ctypes.data),
+           "kvq_kqv_codebook")
+    return cent, thr

@@ -31,7 +31,7 @@ def test_header_declares_the_four_calls():
     for fn in ("kvq_quantize_append", "kvq_decode_attention", "kvq_error_bound",
                "kvq_fallback_exact"):
         assert fn in names
-    assert len(names) == 17
+    assert len(names) == 18
 
 
 def test_library_exports_every_declared_symbol(kvq):
@@ -73,6 +73,18 @@ def test_outlier_section_size_and_checks(kvq):
     # the adaptive-precision ladder reads caches without extraction only
     assert kvq.kvq_adaptive_work_size(_desc(kvq), 2, 1, 32, 4) > 0
     assert kvq.kvq_adaptive_work_size(_desc(kvq, outliers=1), 2, 1, 32, 4) == 0
+
+
+def test_kqv_block_size_and_checks(kvq):
+    kqv = dict(codec=kvq.KVQ_CODEC_KQV, k_bits=4, v_bits=3, k_rotate=1, rot_signs=0x3000,
+               qjl=0x4000)
+    # codes 16 x d/2 + 16 x d/2, sketch 16 x d/8, four fp32 per token, the range
+    assert kvq.kvq_block_bytes(_desc(kvq, k_group=128, v_group=128, **kqv)) == 2592
+    assert kvq.kvq_block_bytes(_desc(kvq, head_dim=64, k_group=64, v_group=64, **kqv)) == 1424
+    assert kvq.kvq_block_bytes(_desc(kvq, k_group=32, v_group=128, **kqv)) == 0
+    assert kvq.kvq_block_bytes(_desc(kvq, k_group=128, v_group=128, codec=7)) == 0
+    d = _desc(kvq, k_group=128, v_group=128, **kqv)
+    assert kvq.kvq_adaptive_work_size(d, 2, 1, 32, 4) == 0
 
 
 def test_status_strings(kvq):
