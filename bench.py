@@ -54,19 +54,27 @@ DECODE_SRCS = [os.path.join(ROOT, "quantized_decode_attention_kvq_b200", "csrc",
 
 
 def _variant(name: str):
-    """'llama8b' -> ('llama8b', False); 'llama8b+med3' -> ('llama8b', True): the
-    workload with Med3x outlier extraction in the cache."""
+    """'llama8b' -> ('llama8b', ''); 'llama8b+med3' -> ('llama8b', 'med3'): the
+    workload with Med3x outlier extraction in the cache; 'llama8b+kqv': the
+    workload's data and shapes in a cache of the KQV codec."""
     base, _, ext = name.partition("+")
-    if base not in synth.WORKLOADS or ext not in ("", "med3"):
+    if base not in synth.WORKLOADS or ext not in ("", "med3", "kqv"):
         raise SystemExit(f"unknown workload {name}")
-    return base, ext == "med3"
+    return base, ext
 
 
 def _describe(name: str) -> str:
-    base, outliers = _variant(name)
-    return _workload_desc(synth.WORKLOADS[base]) + (
+    base, ext = _variant(name)
+    wl = synth.WORKLOADS[base]
+    if ext == "kqv":
+        ctx = f"ctx {wl.ctx}" if wl.ctx_min is None else f"ctx U[{wl.ctx_min},{wl.ctx}]"
+        return (f"{wl.name} data and shapes: B={wl.num_seqs}, Hq={wl.num_q_heads}, "
+                f"Hkv={wl.num_kv_heads}, d={wl.head_dim}, {ctx}, KQV codec (Hadamard-rotated "
+                f"K and V; K 4-bit Lloyd-Max, V 3-bit Lloyd-Max + 1-bit QJL sketch; fp32 "
+                f"norms), 16-token pages (seeded permutation), tau={wl.tau}")
+    return _workload_desc(wl) + (
         ", Med3x outlier extraction (one 4-channel chunk of K and of V per token in fp16)"
-        if outliers else "")
+        if ext == "med3" else "")
 
 
 def _workload_desc(wl) -> str:
@@ -285,7 +293,7 @@ class GpuStep:
     """Device-resident workload and the raw C-ABI calls of one step."""
 
     def __init__(self, wl_name: str, seed: int, replicas: int, two_calls: bool = False,
-                 outliers: bool = False):
+                 outliers: bool = False, codec: str = "int"):
         import ctypes
 
         import torch
@@ -308,9 +316,11 @@ class GpuStep:
         self.kd, self.vd, self.qd = dev(k), dev(v), dev(q)
         self.pt = torch.from_numpy(inp.page_table).cuda()
         self.sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
-        base = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, k_bits=wl.k_bits,
-                              k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
-                              outliers=outliers)
+        ckw = dict(k_bits=wl.k_bits, k_group=wl.k_group, k_rotate=wl.k_rotate,
+                   rot_signs=inp.rot_signs, outliers=outliers)
+        if codec == "kqv":
+            ckw = dict(codec="kqv", rot_signs=inp.rotation_signs(), qjl_matrix=inp.qjl_matrix())
+        base = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, **ckw)
         zeros = torch.zeros(wl.num_seqs, dtype=torch.int32, device="cuda")
         base.append(self.kd, self.vd, self.pt, zeros, self.sl)
         torch.cuda.synchronize()
@@ -322,9 +332,7 @@ class GpuStep:
         self.v_new = torch.gather(self.vd, 2, idx).contiguous()
         self.caches = [base]
         for _ in range(replicas - 1):
-            c = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, k_bits=wl.k_bits,
-                               k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
-                               outliers=outliers)
+            c = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, **ckw)
             c.pool.copy_(base.pool)
             c.eta.copy_(base.eta)
             self.caches.append(c)
@@ -387,7 +395,7 @@ class GpuStep:
             self.decode_bytes += wl.num_seqs * wl.num_kv_heads * (2 * wl.head_dim * es + bb // 16)
         self.cache_bytes = inp.num_pages * wl.num_kv_heads * bb
         self.replicas = replicas
-        self.launches_per_step = 2 if two_calls else 1
+        self.launches_per_step = (3 if codec == "kqv" else 2) if two_calls else 1
         # finite tau: flagged rows are recomputed exactly from pinned host originals
         self.fallback = None
         self.ladder = None
@@ -403,7 +411,7 @@ class GpuStep:
                 sl_h=np.array(inp.seq_lens, np.int32),
                 staging=torch.empty(fb_bytes, dtype=torch.uint8, device="cuda"), rows=0, calls=0,
                 h2d=0)
-        if self.fallback is not None and not outliers:
+        if self.fallback is not None and not outliers and codec == "int":
             # the adaptive-precision ladder run before the exact fallback (it reads
             # caches without outlier extraction)
             mp = self.pt.shape[1]
@@ -648,11 +656,14 @@ def measure_workload(name, args, world, rank, local):
     decode kernel's roofline, the clocks, and the end-to-end number.  A name
     ending in "+med3" is the workload with outlier extraction in the cache."""
     import torch
-    base, outliers = _variant(name)
+    base, ext = _variant(name)
     wl = synth.WORKLOADS[base]
-    reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl, outliers))))
+    reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl, ext))))
     reps = min(reps, 8)
-    st = GpuStep(base, args.seed, reps, two_calls=args.two_calls, outliers=outliers)
+    # the KQV codec has no fused step: its step is the append and the decode
+    two_calls = args.two_calls or ext == "kqv"
+    st = GpuStep(base, args.seed, reps, two_calls=two_calls, outliers=ext == "med3",
+                 codec="kqv" if ext == "kqv" else "int")
     ms_total, dec_ms, clocks = _timed_replay(st, args, world, rank, local)
     e2e_ms, h2d, d2h = _e2e(st, args, world)
     lad_ms = None
@@ -683,7 +694,8 @@ def measure_workload(name, args, world, rank, local):
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "frac_vs_spec": achieved / SPEC_HBM_GBS,
                      "spec_peak": SPEC_HBM_GBS,
-                     "kernel": "decode_mma_kernel" + ("" if st.two_calls else " (append fused)"),
+                     "kernel": ("kqv_partial_kernel + kqv_merge_kernel" if ext == "kqv" else
+                                "decode_mma_kernel" + ("" if st.two_calls else " (append fused)")),
                      "kernel_ms": dec_ms,
                      "timing": ("events around every decode launch" if st.two_calls else
                                 "events around the replay of K back-to-back launches, / K")},
@@ -767,23 +779,36 @@ def run_gpu(args):
         print(json.dumps(res), flush=True)
 
 
-def _cache_bytes_estimate(wl, outliers=False) -> int:
+def _cache_bytes_estimate(wl, ext="") -> int:
     per_tok = wl.head_dim * wl.k_bits // 8 + wl.head_dim // 2 + 2 * wl.head_dim // wl.k_group \
-        + 4 * wl.head_dim // 32 + (18 if outliers else 0)
+        + 4 * wl.head_dim // 32 + (18 if ext == "med3" else 0)
+    if ext == "kqv":
+        per_tok = wl.head_dim + wl.head_dim // 8 + 16 + wl.head_dim // 64
     ctx = wl.ctx if wl.ctx_min is None else (wl.ctx + wl.ctx_min) // 2
     return wl.num_seqs * ctx * wl.num_kv_heads * per_tok
 
 
 # ------------------------------------------------------------------------- CPU --
-def _oracle_setup(workload: str, seed: int, kv_heads=None):
-    """The oracle's cache of sequence 0 of the workload; rows of the given kv heads."""
+def _oracle_cache(workload: str, seed: int):
+    """The workload's inputs and an empty oracle cache of its codec."""
     import oracle
-    base, outliers = _variant(workload)
+    base, ext = _variant(workload)
     inp = synth.make(base, seed)
     wl = inp.wl
-    c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
-                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
-                     outliers=outliers)
+    if ext == "kqv":
+        c = oracle.KqvCache(wl.head_dim, wl.num_kv_heads, inp.num_pages, inp.rotation_signs(),
+                            inp.qjl_matrix())
+    else:
+        c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
+                         k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
+                         outliers=ext == "med3")
+    return inp, c
+
+
+def _oracle_setup(workload: str, seed: int, kv_heads=None):
+    """The oracle's cache of sequence 0 of the workload; rows of the given kv heads."""
+    inp, c = _oracle_cache(workload, seed)
+    wl = inp.wl
     k, v = inp.kv_seq(0)
     pt = inp.page_table[:1]
     sl = np.array(inp.seq_lens[:1], np.int32)
@@ -822,12 +847,8 @@ def _oracle_codec_and_dense(workload: str, seed: int):
     dense attention the fallback computes (every query row), in KV
     token-heads/s."""
     import oracle
-    base, outliers = _variant(workload)
-    inp = synth.make(base, seed)
+    inp, c = _oracle_cache(workload, seed)
     wl = inp.wl
-    c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
-                     k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
-                     outliers=outliers)
     k, v = inp.kv_seq(0)
     sl = np.array(inp.seq_lens[:1], np.int32)
     th = int(sl[0]) * wl.num_kv_heads
@@ -909,7 +930,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--workload", default="llama8b",
-                    choices=sorted(synth.WORKLOADS) + [w + "+med3" for w in sorted(synth.WORKLOADS)])
+                    choices=sorted(synth.WORKLOADS) + [w + x for x in ("+med3", "+kqv")
+                                                        for w in sorted(synth.WORKLOADS)])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -917,7 +939,8 @@ def main():
     ap.add_argument("--also", default=None,
                     help="comma-separated workloads measured in the same run and reported "
                          "under 'workloads'; a '+med3' suffix adds outlier extraction to the "
-                         "cache (default: long128k,serving,llama8b+med3 with llama8b; 'none')")
+                         "cache, '+kqv' uses the KQV codec (default: "
+                         "long128k,serving,llama8b+med3,llama8b+kqv with llama8b; 'none')")
     ap.add_argument("--two-calls", action="store_true",
                     help="step = kvq_quantize_append + kvq_decode_attention (default: the fused "
                          "kvq_decode_attention_append)")
@@ -925,7 +948,8 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.also is None:
-        args.also = "long128k,serving,llama8b+med3" if args.workload == "llama8b" else "none"
+        args.also = ("long128k,serving,llama8b+med3,llama8b+kqv" if args.workload == "llama8b"
+                     else "none")
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -30,6 +30,7 @@
 // sketch bit is the sequential fmaf chain over the channels that the codec's
 // definition fixes, so codes, bits, norms and eta are bit-identical to a
 // sequential implementation.
+#include <algorithm>
 #include <cmath>
 #include <map>
 #include <mutex>
@@ -117,172 +118,223 @@ __device__ __forceinline__ int kqv_code(float u, const float* thr) {
   return k;
 }
 
+// One warp per (token, kv head), 8 warps per CTA looping over the items; the
+// CTA first stages S in shared memory with rows padded to D + 1 floats, so the
+// lanes' reads of a column (the sketch) and of a row (the reconstruction)
+// fall in distinct banks.
+constexpr int kKqAppendWarps = 8;
 template <int D>
-__global__ void __launch_bounds__(256) kqv_append_kernel(const KqvAppendArgs ka) {
+constexpr int kqv_append_smem() { return (D * (D + 1) + kKqAppendWarps * 3 * D) * 4; }
+
+template <int D>
+__global__ void __launch_bounds__(kKqAppendWarps * 32) kqv_append_kernel(const KqvAppendArgs ka) {
   constexpr int E = D / 32;
   constexpr int LPG = 32 / E;           // lanes per 32-channel group
+  constexpr int SP = D + 1;             // padded row of S
   const AppendArgs& a = ka.a;
   const KqvLayout L{D};
-  __shared__ float sh[8][2][D];         // per warp: the rotated vector, the residual
+  extern __shared__ float smf[];
+  float* Ss = smf;                                        // S [D][D + 1]
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int64_t item = (int64_t)blockIdx.x * 8 + w;
+  float* xs = smf + D * SP + w * 3 * D;                   // per warp: rotated vector,
+  float* rs = xs + D;                                     // residual,
+  float* ts = rs + D;                                     // reconstruction
+  for (int idx = threadIdx.x; idx < D * D; idx += blockDim.x)
+    Ss[(idx / D) * SP + idx % D] = __ldg(ka.qjl + idx);
+  __syncthreads();
   const int64_t total = (int64_t)a.num_seqs * a.num_tokens * a.hkv;
-  if (item >= total) return;   // warp-uniform
-  const int h = (int)(item % a.hkv);
-  const int t = (int)((item / a.hkv) % a.num_tokens);
-  const int s = (int)(item / ((int64_t)a.hkv * a.num_tokens));
-  const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
-  float xk[E], xv[E], vin[E];
+  for (int64_t item = (int64_t)blockIdx.x * kKqAppendWarps + w; item < total;
+       item += (int64_t)gridDim.x * kKqAppendWarps) {
+    const int h = (int)(item % a.hkv);
+    const int t = (int)((item / a.hkv) % a.num_tokens);
+    const int s = (int)(item / ((int64_t)a.hkv * a.num_tokens));
+    const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
+    float xk[E], xv[E], vin[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    xk[e] = load_elem(a.k, a.in_bf16, base + lane * E + e);
-    xv[e] = vin[e] = load_elem(a.v, a.in_bf16, base + lane * E + e);
-  }
-  if (a.valid && t >= a.valid[s]) return;
-  const int pos = a.start_pos[s] + t;
-  const int lp = pos / kPage;
-  if (pos < 0 || lp >= a.max_pages) {
-    if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
-    return;
-  }
-  const int page = a.page_table[(int64_t)s * a.max_pages + lp];
-  if (page < 0 || page >= a.num_pages) {
-    if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
-    return;
-  }
-  const int slot = pos % kPage;
-  uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
-  float* xs = sh[w][0];
-  float* rs = sh[w][1];
+    for (int e = 0; e < E; ++e) {
+      xk[e] = load_elem(a.k, a.in_bf16, base + lane * E + e);
+      xv[e] = vin[e] = load_elem(a.v, a.in_bf16, base + lane * E + e);
+    }
+    if (a.valid && t >= a.valid[s]) continue;
+    const int pos = a.start_pos[s] + t;
+    const int lp = pos / kPage;
+    if (pos < 0 || lp >= a.max_pages) {
+      if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+      continue;
+    }
+    const int page = a.page_table[(int64_t)s * a.max_pages + lp];
+    if (page < 0 || page >= a.num_pages) {
+      if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+      continue;
+    }
+    const int slot = pos % kPage;
+    uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
 
-  // ---- keys: rotate, norm, codes, eps ----
-  warp_rotate<E>(xk, a.signs, lane, a.rot_c);
+    // ---- keys: rotate, norm, codes, eps ----
+    warp_rotate<E>(xk, a.signs, lane, a.rot_c);
+    __syncwarp();   // the previous item's reads of xs are done
 #pragma unroll
-  for (int e = 0; e < E; ++e) xs[lane * E + e] = xk[e];
-  __syncwarp();
-  float nk = 0.f;
-  for (int c = 0; c < D; ++c) nk = __fmaf_rn(xs[c], xs[c], nk);
-  nk = __fsqrt_rn(nk);
-  const bool okk = isfinite(nk);
-  if (!okk) nk = 0.f;
-  int code[E];
-  float eps = 0.f;
+    for (int e = 0; e < E; ++e) xs[lane * E + e] = xk[e];
+    __syncwarp();
+    float nk = 0.f;
+    for (int c = 0; c < D; ++c) nk = __fmaf_rn(xs[c], xs[c], nk);
+    nk = __fsqrt_rn(nk);
+    const bool okk = isfinite(nk);
+    if (!okk) nk = 0.f;
+    int code[E];
+    float eps = 0.f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const float u = nk > 0.f ? __fdiv_rn(xk[e], nk) : 0.f;
-    code[e] = kqv_code<16>(u, ka.t.kthr);
-    const float kh = __fmul_rn(nk, ka.t.kcent[code[e]]);
-    if (nk > 0.f) eps = fmaxf(eps, fabsf(__fsub_rn(xk[e], kh)));
-  }
+    for (int e = 0; e < E; ++e) {
+      const float u = nk > 0.f ? __fdiv_rn(xk[e], nk) : 0.f;
+      code[e] = kqv_code<16>(u, ka.t.kthr);
+      const float kh = __fmul_rn(nk, ka.t.kcent[code[e]]);
+      if (nk > 0.f) eps = fmaxf(eps, fabsf(__fsub_rn(xk[e], kh)));
+    }
 #pragma unroll
-  for (int o = 1; o < 32; o *= 2) eps = fmaxf(eps, __shfl_xor_sync(0xffffffffu, eps, o));
-  {
-    uint8_t* kc = blk + slot * (D / 2) + lane * (E / 2);
+    for (int o = 1; o < 32; o *= 2) eps = fmaxf(eps, __shfl_xor_sync(0xffffffffu, eps, o));
+    {
+      uint8_t* kc = blk + slot * (D / 2) + lane * (E / 2);
 #pragma unroll
-    for (int e = 0; e < E; e += 2) kc[e / 2] = (uint8_t)(code[e] | (code[e + 1] << 4));
-  }
-  __syncwarp();   // every lane has read xs
+      for (int e = 0; e < E; e += 2) kc[e / 2] = (uint8_t)(code[e] | (code[e + 1] << 4));
+    }
+    __syncwarp();   // every lane has read xs
 
-  // ---- values: rotate, norm, codes, residual, its norm ----
-  warp_rotate<E>(xv, a.signs, lane, a.rot_c);
+    // ---- values: rotate, norm, codes, residual, its norm ----
+    warp_rotate<E>(xv, a.signs, lane, a.rot_c);
 #pragma unroll
-  for (int e = 0; e < E; ++e) xs[lane * E + e] = xv[e];
-  __syncwarp();
-  float nv = 0.f;
-  for (int c = 0; c < D; ++c) nv = __fmaf_rn(xs[c], xs[c], nv);
-  nv = __fsqrt_rn(nv);
-  const bool okv = isfinite(nv);
-  if (!okv) nv = 0.f;
-  int vcode[E];
+    for (int e = 0; e < E; ++e) xs[lane * E + e] = xv[e];
+    __syncwarp();
+    float nv = 0.f;
+    for (int c = 0; c < D; ++c) nv = __fmaf_rn(xs[c], xs[c], nv);
+    nv = __fsqrt_rn(nv);
+    const bool okv = isfinite(nv);
+    if (!okv) nv = 0.f;
+    int vcode[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const float u = nv > 0.f ? __fdiv_rn(xv[e], nv) : 0.f;
-    vcode[e] = kqv_code<8>(u, ka.t.vthr);
-    rs[lane * E + e] = __fsub_rn(u, ka.t.vcent[vcode[e]]);
-  }
-  __syncwarp();
-  float rn = 0.f;
-  for (int c = 0; c < D; ++c) rn = __fmaf_rn(rs[c], rs[c], rn);
-  rn = __fsqrt_rn(rn);
+    for (int e = 0; e < E; ++e) {
+      const float u = nv > 0.f ? __fdiv_rn(xv[e], nv) : 0.f;
+      vcode[e] = kqv_code<8>(u, ka.t.vthr);
+      rs[lane * E + e] = __fsub_rn(u, ka.t.vcent[vcode[e]]);
+    }
+    __syncwarp();
+    float rn = 0.f;
+    for (int c = 0; c < D; ++c) rn = __fmaf_rn(rs[c], rs[c], rn);
+    rn = __fsqrt_rn(rn);
 
-  // ---- the QJL sketch: projection i = lane + 32 m, a sequential chain over c ----
-  uint32_t word[E];
+    // ---- the QJL sketch: projection i = lane + 32 m, a sequential chain over c
+    // (E independent chains per lane) ----
+    float acc[E];
 #pragma unroll
-  for (int m = 0; m < E; ++m) {
-    const float* Si = ka.qjl + (int64_t)(lane + 32 * m) * D;
-    float acc = 0.f;
-    for (int c = 0; c < D; ++c) acc = __fmaf_rn(__ldg(Si + c), rs[c], acc);
-    word[m] = __ballot_sync(0xffffffffu, acc >= 0.f);
-  }
-  if (lane == 0) {
+    for (int m = 0; m < E; ++m) acc[m] = 0.f;
+    for (int c = 0; c < D; ++c) {
+      const float rc = rs[c];
 #pragma unroll
-    for (int m = 0; m < E; ++m)
-      reinterpret_cast<uint32_t*>(blk + L.vs() + slot * (D / 8))[m] = word[m];
-    reinterpret_cast<float*>(blk + L.kn())[slot] = nk;
-    reinterpret_cast<float*>(blk + L.ke())[slot] = nextafterf(eps, INFINITY);
-    reinterpret_cast<float*>(blk + L.vn())[slot] = nv;
-    reinterpret_cast<float*>(blk + L.vr())[slot] = rn;
-  }
-  {
-    uint8_t* vc = blk + L.vc() + slot * (D / 2) + lane * (E / 2);
+      for (int m = 0; m < E; ++m) acc[m] = __fmaf_rn(Ss[(lane + 32 * m) * SP + c], rc, acc[m]);
+    }
+    uint32_t word[E];
 #pragma unroll
-    for (int e = 0; e < E; e += 2) vc[e / 2] = (uint8_t)(vcode[e] | (vcode[e + 1] << 4));
-  }
+    for (int m = 0; m < E; ++m) word[m] = __ballot_sync(0xffffffffu, acc[m] >= 0.f);
+    if (lane == 0) {
+#pragma unroll
+      for (int m = 0; m < E; ++m)
+        reinterpret_cast<uint32_t*>(blk + L.vs() + slot * (D / 8))[m] = word[m];
+      reinterpret_cast<float*>(blk + L.kn())[slot] = nk;
+      reinterpret_cast<float*>(blk + L.ke())[slot] = nextafterf(eps, INFINITY);
+      reinterpret_cast<float*>(blk + L.vn())[slot] = nv;
+      reinterpret_cast<float*>(blk + L.vr())[slot] = rn;
+    }
+    {
+      uint8_t* vc = blk + L.vc() + slot * (D / 2) + lane * (E / 2);
+#pragma unroll
+      for (int e = 0; e < E; e += 2) vc[e / 2] = (uint8_t)(vcode[e] | (vcode[e + 1] << 4));
+    }
 
-  // ---- reconstruction: v^' = nv (c3 + rho S^T b), v^ = sigma o (c H v^') ----
-  const float rho = __fmul_rn(ka.qjl_c, rn);
-  float vh[E];
+    // ---- reconstruction: sum_i S_ic b_i for channels c = lane + 32 m (a
+    // sequential chain over i each), then v^' = nv (c3 + rho sum) ----
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int c = lane * E + e;
-    float acc = 0.f;
+    for (int m = 0; m < E; ++m) acc[m] = 0.f;
 #pragma unroll
-    for (int m = 0; m < E; ++m)
-      for (int b = 0; b < 32; ++b) {
-        const float sgn = (word[m] >> b) & 1u ? 1.f : -1.f;
-        acc = __fmaf_rn(__ldg(ka.qjl + (int64_t)(32 * m + b) * D + c), sgn, acc);
+    for (int mw = 0; mw < E; ++mw)
+      for (int bi = 0; bi < 32; ++bi) {
+        const float sgn = (word[mw] >> bi) & 1u ? 1.f : -1.f;
+        const float* row = Ss + (32 * mw + bi) * SP + lane;
+#pragma unroll
+        for (int m = 0; m < E; ++m) acc[m] = __fmaf_rn(row[32 * m], sgn, acc[m]);
       }
-    vh[e] = __fmul_rn(nv, __fadd_rn(ka.t.vcent[vcode[e]], __fmul_rn(rho, acc)));
-  }
-  warp_hadamard<E>(vh, lane, a.rot_c);
-  float err = 0.f, hi = 0.f, lo = 0.f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    if (a.signs[lane * E + e] < 0) vh[e] = -vh[e];
-    err = fmaxf(err, fabsf(__fsub_rn(vin[e], vh[e])));
-    hi = fmaxf(hi, vh[e]);
-    lo = fminf(lo, vh[e]);
-  }
+    for (int m = 0; m < E; ++m) ts[lane + 32 * m] = acc[m];
+    __syncwarp();
+    const float rho = __fmul_rn(ka.qjl_c, rn);
+    float vh[E];
 #pragma unroll
-  for (int o = 1; o < 32; o *= 2) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, o));
+    for (int e = 0; e < E; ++e)
+      vh[e] = __fmul_rn(nv, __fadd_rn(ka.t.vcent[vcode[e]], __fmul_rn(rho, ts[lane * E + e])));
+    warp_hadamard<E>(vh, lane, a.rot_c);
+    float err = 0.f, hi = 0.f, lo = 0.f;
 #pragma unroll
-  for (int o = 1; o < LPG; o *= 2) {
-    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    for (int e = 0; e < E; ++e) {
+      if (a.signs[lane * E + e] < 0) vh[e] = -vh[e];
+      err = fmaxf(err, fabsf(__fsub_rn(vin[e], vh[e])));
+      hi = fmaxf(hi, vh[e]);
+      lo = fminf(lo, vh[e]);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o *= 2) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, o));
+#pragma unroll
+    for (int o = 1; o < LPG; o *= 2) {
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    }
+    if (!okk || !okv) err = 0.f;
+    if (lane == 0) {
+      if (!okk || !okv) set_error(a.err, KVQ_ERR_RANGE);
+      const float eu = nextafterf(__fmaf_rn(0x1p-16f, nv, err), INFINITY);
+      atomicMax(reinterpret_cast<int*>(a.eta + (int64_t)page * a.hkv + h), __float_as_int(eu));
+    }
+    if (lane % LPG == 0) {
+      // the block's range starts at [0, 0]: a maximum >= 0 orders like its int
+      // bits, a minimum <= 0 (sign bit set) like its unsigned bits, reversed
+      float* rg = reinterpret_cast<float*>(blk + L.rg()) + 2 * (lane / LPG);
+      if (hi > 0.f) atomicMax(reinterpret_cast<int*>(rg), __float_as_int(hi));
+      if (lo < 0.f) atomicMax(reinterpret_cast<unsigned int*>(rg + 1), __float_as_uint(lo));
+    }
   }
-  if (!okk || !okv) err = 0.f;
-  if (lane == 0) {
-    if (!okk || !okv) set_error(a.err, KVQ_ERR_RANGE);
-    const float eu = nextafterf(__fmaf_rn(0x1p-16f, nv, err), INFINITY);
-    atomicMax(reinterpret_cast<int*>(a.eta + (int64_t)page * a.hkv + h), __float_as_int(eu));
+}
+
+template <int D>
+cudaError_t launch_kqv_append_d(const KqvAppendArgs& a, cudaStream_t stream) {
+  // opt in to the staged S's shared memory once per device
+  static std::mutex mu;
+  static std::map<int, int> sms_of;
+  constexpr int smem = kqv_append_smem<D>();
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = sms_of.find(dev);
+    if (it == sms_of.end()) {
+      if ((e = cudaFuncSetAttribute(kqv_append_kernel<D>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+              cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+      it = sms_of.emplace(dev, sms).first;
+    }
+    sms = it->second;
   }
-  if (lane % LPG == 0) {
-    // the block's range starts at [0, 0]: a maximum >= 0 orders like its int
-    // bits, a minimum <= 0 (sign bit set) like its unsigned bits, reversed
-    float* rg = reinterpret_cast<float*>(blk + L.rg()) + 2 * (lane / LPG);
-    if (hi > 0.f) atomicMax(reinterpret_cast<int*>(rg), __float_as_int(hi));
-    if (lo < 0.f) atomicMax(reinterpret_cast<unsigned int*>(rg + 1), __float_as_uint(lo));
-  }
+  const int64_t items = (int64_t)a.a.num_seqs * a.a.num_tokens * a.a.hkv;
+  const int64_t blocks = std::min<int64_t>((items + kKqAppendWarps - 1) / kKqAppendWarps, 2 * sms);
+  kqv_append_kernel<D><<<(unsigned)blocks, kKqAppendWarps * 32, smem, stream>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_kqv_append(const KqvAppendArgs& a, int d, cudaStream_t stream) {
   const int64_t items = (int64_t)a.a.num_seqs * a.a.num_tokens * a.a.hkv;
   if (items == 0) return cudaSuccess;
-  const int64_t blocks = (items + 7) / 8;
-  if (d == 128) kqv_append_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(a);
-  else if (d == 64) kqv_append_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(a);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (d == 128) return launch_kqv_append_d<128>(a, stream);
+  if (d == 64) return launch_kqv_append_d<64>(a, stream);
+  return cudaErrorInvalidValue;
 }
 
 // ================================================================ decode =====
@@ -393,9 +445,18 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
   const int nloc = first < p1 ? (p1 - first + kKqWarps - 1) / kKqWarps : 0;
   uint8_t* stage0 = sm + C::OFF_ST + warp * kKqStages * C::BLOCK;
   const int32_t* ptab = a.page_table + (int64_t)b * a.max_pages;
+  // lane l holds the page index of local page 32 c + l of chunk c (loaded a
+  // chunk at a time, so no issue waits on a page-table load of its own)
+  int pt_chunk = -1, pt_val = -1;
   auto issue = [&](int j, int st) {
+    if ((j >> 5) != pt_chunk) {
+      pt_chunk = j >> 5;
+      const int jl = 32 * pt_chunk + lane;
+      pt_val = jl < nloc ? __ldg(ptab + first + jl * kKqWarps) : -1;
+    }
+    const int pgv = __shfl_sync(0xffffffffu, pt_val, j & 31);
     if (lane == 0) {
-      const int pg = ptab[first + j * kKqWarps];
+      const int pg = pgv;
       const bool ok = pg >= 0 && pg < a.num_pages;
       spage[st] = ok ? pg : -1;
       if (ok) {
@@ -671,6 +732,7 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_merge_kernel(const KqvDecod
   constexpr int RF = kqv_rec_floats(D);
   const DecodeArgs& a = ka.a;
   __shared__ float sB[kKqWarps][D];
+  __shared__ float sO[kKqWarps][D];
   __shared__ float shd[kKqHdr];
   const int unit = blockIdx.x, kvh = unit % a.hkv, b = unit / a.hkv;
   const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -728,17 +790,30 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_merge_kernel(const KqvDecod
   }
   const float inv_l = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) sB[r][lane * E + e] = o2[e] * inv_l;
-  __syncthreads();   // sB of every warp and the merged header
-  // o' = o1 / l + sqrt(pi/2)/d * S^T (o2 / l), then o = sigma o (c H o')
+  for (int e = 0; e < E; ++e) {
+    sB[r][lane * E + e] = o2[e] * inv_l;
+    sO[r][lane * E + e] = o1[e] * inv_l;
+  }
+  __syncthreads();   // sB, sO of every warp and the merged header
+  // o' = o1 / l + sqrt(pi/2)/d * S^T (o2 / l): thread c < D takes channel c of
+  // the 4 rows (coalesced reads of S, one pass for the CTA)
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float acc[kKqRows] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) {
+      const float sv = __ldg(ka.qjl + (int64_t)i * D + c);
+#pragma unroll
+      for (int rr = 0; rr < kKqRows; ++rr) acc[rr] = fmaf(sv, sB[rr][i], acc[rr]);
+    }
+#pragma unroll
+    for (int rr = 0; rr < kKqRows; ++rr) sO[rr][c] = fmaf(ka.qjl_c, acc[rr], sO[rr][c]);
+  }
+  __syncthreads();
+  // then o = sigma o (c H o')
   float x[E];
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const int c = lane * E + e;
-    float acc = 0.f;
-    for (int i = 0; i < D; ++i) acc = fmaf(__ldg(ka.qjl + (int64_t)i * D + c), sB[r][i], acc);
-    x[e] = fmaf(ka.qjl_c, acc, o1[e] * inv_l);
-  }
+  for (int e = 0; e < E; ++e) x[e] = sO[r][lane * E + e];
   warp_hadamard<E>(x, lane, a.rot_c);
   if (r >= a.R) return;
   if (a.out) {

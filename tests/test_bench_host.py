@@ -24,9 +24,11 @@ def test_traffic_record_only_for_its_capture(monkeypatch):
 
 
 def test_workload_variants():
-    assert bench._variant("llama8b") == ("llama8b", False)
-    assert bench._variant("llama8b+med3") == ("llama8b", True)
+    assert bench._variant("llama8b") == ("llama8b", "")
+    assert bench._variant("llama8b+med3") == ("llama8b", "med3")
+    assert bench._variant("llama8b+kqv") == ("llama8b", "kqv")
     assert "Med3x" in bench._describe("serving+med3")
+    assert "KQV" in bench._describe("llama8b+kqv")
     for bad in ("llama8b+x", "nosuch", "nosuch+med3"):
         try:
             bench._variant(bad)
