@@ -85,7 +85,10 @@ struct DecodeCfg {
   static constexpr int META_FLOATS = kPage * NB + kPage * NGK;              // per warp
   static constexpr int OFF_META = (OFF_RC + RC_FLOATS * 4 + 15) / 16 * 16;
   static constexpr int OFF_FLAG = OFF_META + kWarps * META_FLOATS * 4;
-  static constexpr int END = OFF_FLAG + 16;
+  // OUT: q' chunk-major, [chunk][row][4] fp32 (the 4 rows of one chunk are
+  // neighbouring 16-byte vectors: conflict-free reads by the lanes of a token)
+  static constexpr int OFF_QC = OFF_FLAG + 16;
+  static constexpr int END = OFF_QC + (OUT ? kRows * D * 4 : 0);
   // merge area (aliases the stage buffers once the page loop is over)
   static constexpr int MW_FLOATS = kRows * D + kRows * 8 + kRows * NB + 2 * NB + 1;
   static constexpr int MERGE_BYTES = (kWarps + 1) * MW_FLOATS * 4;
@@ -406,8 +409,12 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
     }
     // the extracted key chunks are scored against q' in fp32
     if constexpr (OUT) {
+      float* qc = reinterpret_cast<float*>(sm + C::OFF_QC);
 #pragma unroll
-      for (int e = 0; e < E; ++e) qf[r * D + lane * E + e] = x[e];
+      for (int e = 0; e < E; ++e) {
+        const int c = lane * E + e;
+        qc[((c / 4) * kRows + r) * 4 + c % 4] = x[e];
+      }
     }
   }
   __syncthreads();
@@ -653,7 +660,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
             const uint2 kw = *reinterpret_cast<const uint2*>(os + 2 * kPage + tok * 8);
             const float2 k01 = __half22float2(u32_as_h2(kw.x));
             const float2 k23 = __half22float2(u32_as_h2(kw.y));
-            const float4 q4 = *reinterpret_cast<const float4*>(qf + c4 * D + 4 * ck);
+            const float4 q4 = reinterpret_cast<const float4*>(sm + C::OFF_QC)[ck * kRows + c4];
             const float d4 = fmaf(q4.w, k23.y, fmaf(q4.z, k23.x, fmaf(q4.y, k01.y, q4.x * k01.x)));
             zt[sl] = fmaf(d4, a.s_att * kLog2e, zt[sl]);
             // sum |q_i| (2^-11 |k_i| + 2^-25) = 2^-11 sum |q_i k_i| + 2^-25 sum |q_i|
