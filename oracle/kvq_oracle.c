@@ -264,9 +264,10 @@ range:
 /*   [K codes][V codes][K scales fp16 [16][d/gk]][V scale,zero fp16 [16][d/32][2]] */
 /* K codes, per token d*bits/8 bytes in 4 stripes; channel c (block          */
 /*   b = c/32, w = c%32, stripe s = w/8, i = w%8) sits in                     */
-/*   8 bit: byte s*(8*nb) + 8*b + i, int8 two's complement; when a row is    */
-/*          128 bytes (d = 128) the 16-byte chunk index of that byte is XORed */
-/*          with slot % 8 (slot = the token's row in the page);               */
+/*   8 bit: byte s*(8*nb) + 8*b + i, int8 two's complement (the library's    */
+/*          device layout also permutes the 16-byte chunks of 128-byte rows  */
+/*          by the token's slot; that is a byte permutation the tests apply  */
+/*          to this logical order before comparing pools);                   */
 /*   4 bit: byte s*(4*nb) + 4*b + i/2, low nibble for even c, 4-bit two's    */
 /*          complement;  nb = d/32.                                           */
 /* V codes: per token d/2 bytes; channel c (group g = c/32, w = c%32) sits in */
@@ -355,11 +356,9 @@ uint16_t oc_f16_rn(float xf) {
   return (dn & 1u) == 0 ? dn : up;
 }
 
-static int64_t oc_k8_byte(int d, int slot, int ch) {
+static int64_t oc_k8_byte(int d, int ch) {
   int nb = d / 32, b = ch / 32, w = ch % 32;
-  int64_t p = (int64_t)(w / 8) * (8 * nb) + 8 * b + w % 8;
-  if (d == 128) p = (((p >> 4) ^ (slot & 7)) << 4) | (p & 15);
-  return p;
+  return (int64_t)(w / 8) * (8 * nb) + 8 * b + w % 8;
 }
 static int64_t oc_k4_byte(int d, int ch) {
   int nb = d / 32, b = ch / 32, w = ch % 32;
@@ -445,7 +444,7 @@ static int oc_quantize_token(const oc_cfg* c, uint8_t* blk, int slot, const floa
     for (int i = 0; i < c->kgroup; ++i) {
       int ch = g * c->kgroup + i;
       if (c->kbits == 8) {
-        kcodes[(int64_t)slot * d + oc_k8_byte(d, slot, ch)] = (uint8_t)codes[i];
+        kcodes[(int64_t)slot * d + oc_k8_byte(d, ch)] = (uint8_t)codes[i];
       } else {
         uint8_t* row = kcodes + (int64_t)slot * (d / 2);
         oc_put_nibble(row, oc_k4_byte(d, ch), ch, (unsigned)(codes[i] & 0xF));
@@ -532,7 +531,7 @@ static void oc_read_token(const oc_cfg* c, const uint8_t* blk, int slot, double*
     kscale[g] = oc_f16_value(oc_rd16(kscales + ((int64_t)slot * ngk + g) * 2));
   for (int ch = 0; ch < d; ++ch) {
     int code;
-    if (c->kbits == 8) code = (int8_t)kcodes[(int64_t)slot * d + oc_k8_byte(d, slot, ch)];
+    if (c->kbits == 8) code = (int8_t)kcodes[(int64_t)slot * d + oc_k8_byte(d, ch)];
     else {
       unsigned nib = oc_get_nibble(kcodes + (int64_t)slot * (d / 2), oc_k4_byte(d, ch), ch);
       code = nib >= 8 ? (int)nib - 16 : (int)nib;

@@ -33,6 +33,23 @@ def oracle_cache(inp, outliers=False):
                         outliers=outliers)
 
 
+def device_pool(c):
+    """The oracle cache's pool (logical stripe order) in the library's device
+    layout, as include/kvq.h documents it: with d = 128 and 8-bit keys, the
+    16-byte chunk q of the 128-byte key row of token slot s sits at chunk
+    q ^ (s % 8).  Every other layout is the same in both."""
+    pool = np.asarray(c.pool)
+    if not (c.cfg.d == 128 and c.cfg.kbits == 8):
+        return pool
+    blocks = pool.reshape(-1, c.block_bytes).copy()
+    k = blocks[:, :16 * 128].reshape(-1, 16, 8, 16)
+    out = np.empty_like(k)
+    for s in range(16):
+        out[:, s, [q ^ (s % 8) for q in range(8)], :] = k[:, s, :, :]
+    blocks[:, :16 * 128] = out.reshape(-1, 16 * 128)
+    return blocks.reshape(-1)
+
+
 def run_oracle(inp, tau=None):
     """Append the whole context, decode every row, and compute dense attention."""
     wl = inp.wl

@@ -15,7 +15,7 @@ import torch
 import oracle
 from gpu_cases import (TOL_BOUND_REL, TOL_MAXABS, TOL_RELL2, compare_flags, compare_outputs,
                        gpu_cache, oracle_pool, record_margin, run_gpu, to_torch)
-from oracle_cases import SMALL, max_err, small
+from oracle_cases import SMALL, device_pool, max_err, small
 from quantized_decode_attention_kvq_b200 import inputs as synth
 
 pytestmark = pytest.mark.gpu
@@ -58,8 +58,9 @@ def test_append_bit_exact_with_extraction(name, seed):
     oc = oracle_pool(inp, k, v, outliers=True)
     assert g["err"] == 0
     pool = g["cache"].pool.cpu().numpy()
-    assert pool.size == oc.pool.size
-    assert np.array_equal(pool, oc.pool), np.flatnonzero(pool != oc.pool)[:10]
+    opool = device_pool(oc)
+    assert pool.size == opool.size
+    assert np.array_equal(pool, opool), np.flatnonzero(pool != opool)[:10]
     eta = g["cache"].eta.cpu().numpy()
     assert np.array_equal(eta.view(np.uint32), oc.eta.view(np.uint32))
     # the case exercises the extraction: some keys and some values have a chunk out
@@ -123,7 +124,7 @@ def test_hand_worked_spike_token_on_gpu():
     oc = oracle.Cache(d, 1, 1, k_bits=8, k_group=d, outliers=True)
     assert oc.append(k.reshape(1, 1, 1, d), v.reshape(1, 1, 1, d), np.zeros((1, 1), np.int32),
                      np.zeros(1, np.int32)) == 0
-    assert np.array_equal(blk, oc.pool)
+    assert np.array_equal(blk, device_pool(oc))
     out = 16 * d + 16 * d // 2 + 16 * 2 + 16 * (d // 32) * 4
     assert blk[out] == 15 and blk[out + 16] == 2
     assert list(blk[out + 32:out + 40].view(np.float16).astype(np.float64)) == [40, 1, 1, 1]
@@ -156,7 +157,7 @@ def test_extracted_value_out_of_fp16_range_is_reported():
     rc = oc.append(k, v, inp.page_table, np.zeros(wl.num_seqs, np.int32),
                    valid=np.array(inp.seq_lens, np.int32))
     assert rc == oracle.ERR_RANGE
-    assert np.array_equal(c.pool.cpu().numpy(), oc.pool)
+    assert np.array_equal(c.pool.cpu().numpy(), device_pool(oc))
 
 
 def _fused_step(inp, k, v, q, outliers):
@@ -201,7 +202,7 @@ def test_fused_step_with_extraction(name):
     q = inp.q()
     c, g = _fused_step(inp, k, v, q, True)
     oc = oracle_pool(inp, k, v, outliers=True)
-    assert np.array_equal(c.pool.cpu().numpy(), oc.pool)
+    assert np.array_equal(c.pool.cpu().numpy(), device_pool(oc))
     assert np.array_equal(c.eta.cpu().numpy().view(np.uint32), oc.eta.view(np.uint32))
     o_hat, ob, of, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=inp.wl.tau)
     _check(inp, g, o_hat, ob, of, inp.wl.tau, f"med3 fused {name}")
@@ -216,7 +217,7 @@ def test_fused_step_full_size_with_extraction():
     q = inp.q()
     c, g = _fused_step(inp, k, v, q, True)
     oc = oracle_pool(inp, k, v, outliers=True)
-    assert np.array_equal(c.pool.cpu().numpy(), oc.pool)
+    assert np.array_equal(c.pool.cpu().numpy(), device_pool(oc))
     assert np.array_equal(c.eta.cpu().numpy().view(np.uint32), oc.eta.view(np.uint32))
     o_hat, ob, of, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=inp.wl.tau)
     _check(inp, g, o_hat, ob, of, inp.wl.tau, "med3 llama8b full size")

@@ -13,7 +13,7 @@ import oracle
 from gpu_cases import (TOL_BOUND_REL, TOL_MAXABS, TOL_RELL2, compare_flags, compare_outputs,
                        record_margin,
                        gpu_cache, oracle_pool, run_gpu, to_torch)
-from oracle_cases import SMALL, max_err, small
+from oracle_cases import SMALL, device_pool, max_err, small
 from quantized_decode_attention_kvq_b200 import inputs as synth
 
 pytestmark = pytest.mark.gpu
@@ -49,7 +49,8 @@ def test_append_bit_exact(name, seed):
     oc = oracle_pool(inp, k, v)
     assert g["err"] == 0
     pool = g["cache"].pool.cpu().numpy()
-    assert np.array_equal(pool, oc.pool), np.flatnonzero(pool != oc.pool)[:10]
+    opool = device_pool(oc)
+    assert np.array_equal(pool, opool), np.flatnonzero(pool != opool)[:10]
     eta = g["cache"].eta.cpu().numpy()
     assert np.array_equal(eta.view(np.uint32), oc.eta.view(np.uint32))
 
@@ -168,7 +169,7 @@ def test_full_size_parity(name):
     g = run_gpu(inp, k, v, q)
     assert g["err"] == 0
     oc = oracle_pool(inp, k, v)
-    assert np.array_equal(g["cache"].pool.cpu().numpy(), oc.pool)
+    assert np.array_equal(g["cache"].pool.cpu().numpy(), device_pool(oc))
     o_hat, bound, flags, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=inp.wl.tau)
     _check_decode(inp, g, o_hat, bound, flags, inp.wl.tau)
 
@@ -211,7 +212,7 @@ def test_fused_step_full_size(name, seed):
     torch.cuda.synchronize()
     assert c.device_error() == 0
     oc = oracle_pool(inp, k, v)
-    assert np.array_equal(c.pool.cpu().numpy(), oc.pool)
+    assert np.array_equal(c.pool.cpu().numpy(), device_pool(oc))
     assert np.array_equal(c.eta.cpu().numpy().view(np.uint32), oc.eta.view(np.uint32))
     o_hat, ob, of, _ = oc.decode(q, inp.page_table, inp.seq_lens, tau=wl.tau)
     g = dict(out=out.cpu().numpy().reshape(-1, d).astype(np.float64),

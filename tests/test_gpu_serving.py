@@ -15,7 +15,7 @@ import torch
 import oracle
 from gpu_cases import (TOL_BOUND_REL, TOL_MAXABS, TOL_RELL2, compare_flags, compare_outputs,
                        run_gpu)
-from oracle_cases import max_err, oracle_cache
+from oracle_cases import device_pool, max_err, oracle_cache
 from quantized_decode_attention_kvq_b200 import inputs as synth
 
 pytestmark = pytest.mark.gpu
@@ -49,7 +49,7 @@ def test_serving_full_size_sampled_sequences():
     pages = np.concatenate([pt[i, :inp.pages_per_seq[s]] for i, s in enumerate(sel)])
     bb = oc.block_bytes
     gpool = g["cache"].pool.cpu().numpy().reshape(inp.num_pages, wl.num_kv_heads, bb)
-    opool = oc.pool.reshape(inp.num_pages, wl.num_kv_heads, bb)
+    opool = device_pool(oc).reshape(inp.num_pages, wl.num_kv_heads, bb)
     assert np.array_equal(gpool[pages], opool[pages])
     assert np.array_equal(g["cache"].eta.cpu().numpy()[pages], oc.eta[pages])
 

@@ -187,9 +187,13 @@ def _u16(buf, off):
     return int(buf[off]) | (int(buf[off + 1]) << 8)
 
 
-def _k8_byte(d, ch, slot=0):   # documented layout (8-bit keys)
+def _k8_byte(d, ch):   # documented stripe order (8-bit keys), the oracle's pool
     nb, b, w = d // 32, ch // 32, ch % 32
-    p = (w // 8) * (8 * nb) + 8 * b + w % 8
+    return (w // 8) * (8 * nb) + 8 * b + w % 8
+
+
+def _k8_device_byte(d, ch, slot):   # the library's device layout of the same byte
+    p = _k8_byte(d, ch)
     if d == 128:   # 128-byte rows: the 16-byte chunk index is XORed with slot % 8
         p = (((p >> 4) ^ (slot % 8)) << 4) | (p & 15)
     return p
@@ -210,15 +214,38 @@ def test_nibble_layouts_are_bijections(d):
     for f in (_k4_byte, _v4_byte):
         slots = {(f(d, c), c % 2) for c in range(d)}
         assert len(slots) == d and max(b for b, _ in slots) == d // 2 - 1
+    assert sorted(_k8_byte(d, c) for c in range(d)) == list(range(d))
     for slot in range(16):
-        assert sorted(_k8_byte(d, c, slot) for c in range(d)) == list(range(d))
+        assert sorted(_k8_device_byte(d, c, slot) for c in range(d)) == list(range(d))
     # a thread of the decode kernel reads one contiguous stripe per token
     assert [_v4_byte(128, c) for c in (0, 1, 2, 3, 32, 34, 4)] == [0, 0, 1, 1, 2, 3, 8]
     assert [_k4_byte(128, c) for c in (0, 2, 6, 8, 32, 40)] == [0, 1, 3, 16, 4, 20]
     assert [_k8_byte(128, c) for c in (0, 7, 8, 32, 39, 40, 127)] == [0, 7, 32, 8, 15, 40, 127]
     # slot 3 of a 128-byte row: chunk q of the stripe order lands in chunk q ^ 3
-    assert [_k8_byte(128, c, 3) for c in (0, 7, 8, 32, 39, 40, 127)] == [48, 55, 16, 56, 63, 24, 79]
-    assert [_k8_byte(64, c, 3) for c in (0, 8, 32)] == [0, 16, 8]   # 64-byte rows: unchanged
+    assert [_k8_device_byte(128, c, 3) for c in (0, 7, 8, 32, 39, 40, 127)] == \
+        [48, 55, 16, 56, 63, 24, 79]
+    assert [_k8_device_byte(64, c, 3) for c in (0, 8, 32)] == [0, 16, 8]   # 64-byte rows
+
+
+def test_device_permutation_helper(oracle_lib):
+    """device_pool (the test-side conversion of the oracle's logical pool into
+    the library's documented device layout) moves each key code to the byte
+    the documented formula gives, and nothing else."""
+    from oracle_cases import device_pool
+    rng = np.random.default_rng(11)
+    d, H = 128, 2
+    k = rng.standard_normal((1, H, 20, d)).astype(np.float32)
+    v = rng.standard_normal((1, H, 20, d)).astype(np.float32)
+    c = oracle.Cache(d, H, 2, k_bits=8, k_group=128)
+    assert c.append(k, v, np.array([[1, 0]], np.int32), [0]) == 0
+    dev = device_pool(c)
+    bb = c.block_bytes
+    for blk in range(2 * H):
+        lo, do = c.pool[blk * bb:(blk + 1) * bb], dev[blk * bb:(blk + 1) * bb]
+        assert np.array_equal(lo[16 * d:], do[16 * d:])
+        for slot in range(16):
+            for ch in range(d):
+                assert do[slot * d + _k8_device_byte(d, ch, slot)] == lo[slot * d + _k8_byte(d, ch)]
 
 
 @pytest.mark.parametrize("kbits,kgroup,d", [(8, 128, 128), (4, 32, 128), (8, 32, 64)])
@@ -245,7 +272,7 @@ def test_pack_roundtrip_through_pool(oracle_lib, kbits, kgroup, d):
                 for i, cd in enumerate(codes):
                     ch = g * kgroup + i
                     if kbits == 8:
-                        assert np.int8(blk[slot * d + _k8_byte(d, ch, slot)]) == cd
+                        assert np.int8(blk[slot * d + _k8_byte(d, ch)]) == cd
                     else:
                         byte = int(blk[slot * d // 2 + _k4_byte(d, ch)])
                         nib = (byte >> 4) if ch % 2 else (byte & 15)
