@@ -16,13 +16,13 @@
 //                         range
 //   kqv_partial_kernel    grid (sequence x kv head, split), 4 warps, each warp
 //                         streaming its pages through a 2-stage bulk-copy
-//                         ring: scores on the CUDA cores (lane = 4 channels,
-//                         codebook lookups from a bank-replicated shared
-//                         table, a reduce-scatter of the 8 tokens x 4 rows
-//                         partial sums), online softmax, the bound's sums,
-//                         PV as two accumulations per channel (the codebook
-//                         part and the sketch part, the latter indexed by
-//                         projection)
+//                         ring: scores on fp16 tensor cores (one byte of
+//                         codes = one A register, looked up as the centroids'
+//                         fp16 hi and lo parts from a bank-replicated shared
+//                         table; q' as hi and lo B columns), online softmax,
+//                         the bound's sums, PV on the CUDA cores as two
+//                         accumulations per lane (the codebook part per
+//                         channel, the sketch part per projection)
 //   kqv_merge_kernel      per (sequence, kv head): the split records' merge,
 //                         the sketch part through S^T, the inverse rotation,
 //                         the bound and the flag
@@ -392,10 +392,21 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
   const int p1 = min(npages, p0 + a.pps);
 
   // ---- tables and query rows ----
-  float* lut = reinterpret_cast<float*>(sm + C::OFF_LUT);   // [24][32]: 16 key, 8 value entries
+  // [24][32]: rows 0..15 the key centroids as packed fp16 (hi, lo) with
+  // hi + lo = the fp32 centroid to ~2^-22; rows 16..23 the value centroids
+  // (fp32); every entry replicated per lane, so lookups never conflict
+  float* lut = reinterpret_cast<float*>(sm + C::OFF_LUT);
+  uint32_t* lutk = reinterpret_cast<uint32_t*>(lut);
   for (int i = tid; i < 24 * 32; i += blockDim.x) {
     const int k = i / 32;
-    lut[i] = k < 16 ? ka.t.kcent[k] : ka.t.vcent[k - 16];
+    if (k < 16) {
+      const float c = ka.t.kcent[k];
+      const __half hi = __float2half_rn(c);
+      const __half lo = __float2half_rn(c - __half2float(hi));
+      lutk[i] = h2_as_u32(__halves2half2(hi, lo));
+    } else {
+      lut[i] = ka.t.vcent[k - 16];
+    }
   }
   float* qs = reinterpret_cast<float*>(sm + C::OFF_Q);
   float* qn = reinterpret_cast<float*>(sm + C::OFF_QN);
@@ -430,14 +441,35 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
     }
   }
   __syncthreads();
-  float qreg[kKqRows][E];
+  // B fragments of the QK^T MMA (m16n8k16, k = 16 channels per step): column
+  // n = g8 holds row n % 4 of q', its fp16 hi part (n < 4) or the remainder
+  // (n >= 4); k pairs (2 c4, 2 c4 + 1) and (2 c4 + 8, 2 c4 + 9)
+  constexpr int KS = D / 16;
+  const int g8 = lane >> 2, c4 = lane & 3;
+  uint32_t qb[KS][2];
+  {
+    const int qr = g8 & 3;
+    const bool lo_part = g8 >= 4;
+    auto part = [&](float v) -> __half {
+      const __half hi = __float2half_rn(v);
+      return lo_part ? __float2half_rn(v - __half2float(hi)) : hi;
+    };
 #pragma unroll
-  for (int r = 0; r < kKqRows; ++r)
+    for (int kk = 0; kk < KS; ++kk)
 #pragma unroll
-    for (int e = 0; e < E; ++e) qreg[r][e] = qs[r * D + lane * E + e];
-  const int myr = lane & 3;               // the row of this lane's scores
-  const float cq1 = kKappa * a.s_att * qn[2 * myr];
-  const float cq2 = kKappa * a.s_att * kRotSlack * qn[2 * myr + 1];
+      for (int h = 0; h < 2; ++h) {
+        const int c = 16 * kk + 8 * h + 2 * c4;
+        qb[kk][h] = h2_as_u32(__halves2half2(part(qs[qr * D + c]), part(qs[qr * D + c + 1])));
+      }
+  }
+  // this lane's scores: token g8 (c4 < 2) or g8 + 8 (c4 >= 2), rows r0, r0 + 1
+  const int r0 = 2 * (c4 & 1);
+  float cq1[2], cq2[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    cq1[k] = kKappa * a.s_att * qn[2 * (r0 + k)];
+    cq2[k] = kKappa * a.s_att * kRotSlack * qn[2 * (r0 + k) + 1];
+  }
   const float zsc = a.s_att * kLog2e;
 
   // ---- pages of this warp: p0 + warp, p0 + warp + 4, ... ----
@@ -477,7 +509,8 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
   for (int r = 0; r < kKqRows; ++r)
 #pragma unroll
     for (int e = 0; e < E; ++e) acc1[r][e] = acc2[r][e] = 0.f;
-  float m2 = -INFINITY, lsum = 0.f, Asum = 0.f, Bsum = 0.f, Esum = 0.f, dmax = 0.f;
+  float m2[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f}, Asum[2] = {0.f, 0.f},
+        Bsum[2] = {0.f, 0.f}, Esum[2] = {0.f, 0.f}, dmax[2] = {0.f, 0.f};
   float rhi[NB], rlo[NB], etamax = clamped ? INFINITY : 0.f;
 #pragma unroll
   for (int g = 0; g < NB; ++g) {
@@ -512,90 +545,89 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
         rhi[g] = fmaxf(rhi[g], frg[2 * g]);
         rlo[g] = fminf(rlo[g], frg[2 * g + 1]);
       }
-      // ---- scores of tokens t0 = lane / 4 and t0 + 8 for row lane % 4 ----
-      float zs2[2];
+      // ---- QK^T on fp16 tensor cores: tokens = M, channels = K ----
+      // One byte of a token's codes is one A register (two channels); the
+      // lane needs byte c4 of every 4-byte word of rows g8 and g8 + 8.
+      float sc4[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        uint32_t wr[2][D / 8];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        // partial scores of tokens 8 hf + tl, rows r: index tl * 4 + r
-        float part[32];
+        for (int h = 0; h < 2; ++h) {
+          const uint4* rowp = reinterpret_cast<const uint4*>(blk + (g8 + 8 * h) * (D / 2));
 #pragma unroll
-        for (int tl = 0; tl < 8; ++tl) {
-          const int t = 8 * hf + tl;
-          const uint8_t* kc = blk + t * (D / 2) + lane * (E / 2);
-          float cv[E];
-#pragma unroll
-          for (int e = 0; e < E; e += 2) {
-            const unsigned byte = kc[e / 2];
-            cv[e] = lut[(byte & 15u) * 32 + lane];
-            cv[e + 1] = lut[(byte >> 4) * 32 + lane];
-          }
-#pragma unroll
-          for (int r = 0; r < kKqRows; ++r) {
-            float s = qreg[r][0] * cv[0];
-#pragma unroll
-            for (int e = 1; e < E; ++e) s = fmaf(qreg[r][e], cv[e], s);
-            part[tl * 4 + r] = s;
+          for (int q = 0; q < D / 32; ++q) {
+            const uint4 v4 = rowp[q];
+            wr[h][4 * q] = v4.x;
+            wr[h][4 * q + 1] = v4.y;
+            wr[h][4 * q + 2] = v4.z;
+            wr[h][4 * q + 3] = v4.w;
           }
         }
-        // reduce-scatter over the warp: lane l ends with the sum of index l
+        const uint32_t bsel = 0x4440u | (uint32_t)c4;   // byte c4, zero-extended
+        auto afrag = [&](uint32_t word, uint32_t& ahi, uint32_t& alo) {
+          const uint32_t byte = prmt(word, 0u, bsel);
+          const uint32_t v0 = lutk[(byte & 15u) * 32 + lane];
+          const uint32_t v1 = lutk[(byte >> 4) * 32 + lane];
+          ahi = prmt(v0, v1, 0x5410u);
+          alo = prmt(v0, v1, 0x7632u);
+        };
 #pragma unroll
-        for (int o = 16, cnt = 32; o >= 1; o >>= 1, cnt >>= 1) {
-          const bool up = (lane & o) != 0;
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            if (k < cnt / 2) {
-              const float send = up ? part[k] : part[cnt / 2 + k];
-              const float keep = up ? part[cnt / 2 + k] : part[k];
-              part[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-            }
-          }
+        for (int kk = 0; kk < KS; ++kk) {
+          uint32_t h0, l0, h1, l1, h2, l2, h3, l3;
+          afrag(wr[0][2 * kk], h0, l0);       // token g8, channels 16 kk + 2 c4, +1
+          afrag(wr[1][2 * kk], h1, l1);       // token g8 + 8
+          afrag(wr[0][2 * kk + 1], h2, l2);   // token g8, channels 16 kk + 8 + 2 c4, +1
+          afrag(wr[1][2 * kk + 1], h3, l3);
+          mma_f16(sc4, h0, h1, h2, h3, qb[kk][0], qb[kk][1]);
+          mma_f16(sc4, l0, l1, l2, l3, qb[kk][0], qb[kk][1]);
         }
-        zs2[hf] = part[0];
       }
-      // ---- online softmax and the bound's sums, once per page ----
+      // columns 2 c4, 2 c4 + 1: the hi (c4 < 2) or lo part of rows r0, r0 + 1
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sc4[k] += __shfl_xor_sync(0xffffffffu, sc4[k], 2);
+      const int t = g8 + 8 * (c4 >> 1);
+      const bool vt = t < nval;
+      const float nk = fk[t];
       float zt[2], dl[2];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int t = 8 * hf + (lane >> 2);
-        const bool vt = t < nval;
-        const float nk = fk[t];
-        zt[hf] = vt ? zs2[hf] * nk * zsc : -INFINITY;
-        dl[hf] = vt ? fmaf(cq1, fe[t], cq2 * nk) : 0.f;
+      for (int k = 0; k < 2; ++k) {
+        const float sraw = c4 < 2 ? sc4[k] : sc4[2 + k];
+        zt[k] = vt ? sraw * nk * zsc : -INFINITY;
+        dl[k] = vt ? fmaf(cq1[k], fe[t], cq2[k] * nk) : 0.f;
       }
-      float mx = fmaxf(zt[0], zt[1]);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float mref = mx > m2 + 2.0f ? mx : m2;
-      const float alpha = ex2(m2 - mref);
-      m2 = mref;
-      float tl_ = 0.f, ta = 0.f, tb = 0.f;
+      // ---- online softmax and the bound's sums, rows r0 + k, once per page ----
+      float alpha[2];
+      const float wvn = vt ? fv[t] : 0.f, wrn = vt ? fr[t] : 0.f;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int t = 8 * hf + (lane >> 2);
-        const bool vt = t < nval;
-        const float wv = ex2(zt[hf] - mref);
-        const float d = dl[hf];
+      for (int k = 0; k < 2; ++k) {
+        float mx = zt[k];
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float mref = mx > m2[k] + 2.0f ? mx : m2[k];
+        alpha[k] = ex2(m2[k] - mref);
+        m2[k] = mref;
+        const float wv = ex2(zt[k] - mref);
+        const float d = dl[k];
         const float ed = ex2(d * kLog2e), en = ex2(-d * kLog2e);
         const float em = d < 0.015625f ? d * fmaf(d, fmaf(d, 1.0f / 6, 0.5f), 1.0f) : ed - 1.0f;
-        tl_ += wv;
-        ta = fmaf(wv, em, ta);
-        tb = fmaf(wv, en, tb);
-        dmax = fmaxf(dmax, d);
+        lsum[k] = fmaf(lsum[k], alpha[k], wv);
+        Asum[k] = fmaf(Asum[k], alpha[k], wv * em);
+        Bsum[k] = fmaf(Bsum[k], alpha[k], wv * en);
+        Esum[k] = fmaf(Esum[k], alpha[k], wv * eta_pg);
+        dmax[k] = fmaxf(dmax[k], d);
         // weights of the PV accumulations (0 outside the context: the slots
         // past it may hold another sequence's norms)
-        const float wa = vt ? wv * fv[t] : 0.f;
-        wts[t * 4 + (lane & 3)] = wa;
-        wts[kPage * 4 + t * 4 + (lane & 3)] = vt ? wa * fr[t] : 0.f;
+        const float wa = wv * wvn;
+        wts[t * 4 + r0 + k] = wa;
+        wts[kPage * 4 + t * 4 + r0 + k] = wa * wrn;
       }
-      lsum = fmaf(lsum, alpha, tl_);
-      Asum = fmaf(Asum, alpha, ta);
-      Bsum = fmaf(Bsum, alpha, tb);
-      Esum = fmaf(Esum, alpha, tl_ * eta_pg);
-      if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+      if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
 #pragma unroll
         for (int r = 0; r < kKqRows; ++r) {
-          const float ar = __shfl_sync(0xffffffffu, alpha, r);
+          // row r's factor sits in lanes with c4 & 1 == r / 2, slot r % 2
+          const float ar = __shfl_sync(0xffffffffu, alpha[r & 1], r >> 1);
 #pragma unroll
           for (int e = 0; e < E; ++e) {
             acc1[r][e] *= ar;
@@ -640,15 +672,17 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
     for (int j = jstop; j < nloc && j < jstop + kKqStages; ++j)
       (void)mbar_wait(&bar[j % kKqStages], (uint32_t)((j / kKqStages) & 1));
 
-  // ---- per-warp sums over the lanes of each row ----
+  // ---- per-warp sums over the lanes of each row (lanes with the same c4 & 1) ----
 #pragma unroll
-  for (int o = 4; o < 32; o *= 2) {
-    lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    Asum += __shfl_xor_sync(0xffffffffu, Asum, o);
-    Bsum += __shfl_xor_sync(0xffffffffu, Bsum, o);
-    Esum += __shfl_xor_sync(0xffffffffu, Esum, o);
-    dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
-  }
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int o = 2; o < 32; o *= 2) {
+      lsum[k] += __shfl_xor_sync(0xffffffffu, lsum[k], o);
+      Asum[k] += __shfl_xor_sync(0xffffffffu, Asum[k], o);
+      Bsum[k] += __shfl_xor_sync(0xffffffffu, Bsum[k], o);
+      Esum[k] += __shfl_xor_sync(0xffffffffu, Esum[k], o);
+      dmax[k] = fmaxf(dmax[k], __shfl_xor_sync(0xffffffffu, dmax[k], o));
+    }
   __syncthreads();   // every warp is done with its stages
   float* mw = reinterpret_cast<float*>(sm) + warp * C::MW;
 #pragma unroll
@@ -658,14 +692,17 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
       mw[r * D + lane * E + e] = acc1[r][e];
       mw[kKqRows * D + r * D + lane * E + e] = acc2[r][e];
     }
-  if (lane < 4) {
-    float* stt = mw + 2 * kKqRows * D + lane * 8;
-    stt[0] = m2;
-    stt[1] = lsum;
-    stt[2] = Asum;
-    stt[3] = Bsum;
-    stt[4] = Esum;
-    stt[5] = dmax;
+  if (lane < 2) {   // lane c4 = lane holds rows 2 lane, 2 lane + 1
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      float* stt = mw + 2 * kKqRows * D + (2 * lane + k) * 8;
+      stt[0] = m2[k];
+      stt[1] = lsum[k];
+      stt[2] = Asum[k];
+      stt[3] = Bsum[k];
+      stt[4] = Esum[k];
+      stt[5] = dmax[k];
+    }
   }
   if (lane == 0) {
     float* hd = mw + 2 * kKqRows * D + kKqRows * 8;
