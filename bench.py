@@ -411,9 +411,9 @@ class GpuStep:
                 sl_h=np.array(inp.seq_lens, np.int32),
                 staging=torch.empty(fb_bytes, dtype=torch.uint8, device="cuda"), rows=0, calls=0,
                 h2d=0)
-        if self.fallback is not None and not outliers and codec == "int":
+        if self.fallback is not None and codec == "int":
             # the adaptive-precision ladder run before the exact fallback (it reads
-            # caches without outlier extraction)
+            # the Tier-1 codec's caches, with or without outlier extraction)
             mp = self.pt.shape[1]
             rows = self.flags.numel()
             ad_host = kvq.kvq_adaptive_host_size(base.desc, B, mp)
@@ -939,8 +939,8 @@ def main():
     ap.add_argument("--also", default=None,
                     help="comma-separated workloads measured in the same run and reported "
                          "under 'workloads'; a '+med3' suffix adds outlier extraction to the "
-                         "cache, '+kqv' uses the KQV codec (default: "
-                         "long128k,serving,llama8b+med3,llama8b+kqv with llama8b; 'none')")
+                         "cache, '+kqv' uses the KQV codec (default: long128k,serving,"
+                         "llama8b+med3,serving+med3,llama8b+kqv with llama8b; 'none')")
     ap.add_argument("--two-calls", action="store_true",
                     help="step = kvq_quantize_append + kvq_decode_attention (default: the fused "
                          "kvq_decode_attention_append)")
@@ -948,8 +948,8 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.also is None:
-        args.also = ("long128k,serving,llama8b+med3,llama8b+kqv" if args.workload == "llama8b"
-                     else "none")
+        args.also = ("long128k,serving,llama8b+med3,serving+med3,llama8b+kqv"
+                     if args.workload == "llama8b" else "none")
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -342,9 +342,10 @@ KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, 
  * ordered after all of this call's work.  After an error return, queued work
  * may still be pending on both streams (synchronize them before reusing the
  * buffers).  KVQ_FAULT=memcpy makes the page-in fail (KVQ_ERR_CUDA) for
- * tests.  Blocks the calling thread on the bounded waits.  A cache with
- * outlier extraction returns KVQ_ERR_UNSUPPORTED (and kvq_adaptive_work_size
- * 0): the ladder reads caches without extraction only. */
+ * tests.  Blocks the calling thread on the bounded waits.  With outlier
+ * extraction the quantized scores, values, Delta and value range include the
+ * extracted chunks exactly as kvq_decode_attention does.  A KQV cache returns
+ * KVQ_ERR_UNSUPPORTED (and kvq_adaptive_work_size 0). */
 KVQ_API size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs,
                                       int32_t num_queries, int32_t num_q_heads,
                                       int32_t max_pages_per_seq);

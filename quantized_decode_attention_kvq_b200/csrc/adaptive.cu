@@ -66,7 +66,7 @@ int adaptive_select_smem(int max_pages, int d) {
 template <int D, int KB, int KG>
 __global__ void __launch_bounds__(kAdThreads) adaptive_select_kernel(const __grid_constant__ AdArgs a) {
   constexpr int E = D / 32, NGK = D / KG;
-  const BlockLayout L{D, KB, KG};
+  const BlockLayout L{D, KB, KG, a.outliers};
   extern __shared__ __align__(16) uint8_t smem[];
   const AdUnit u = a.units[blockIdx.x];
   const int R = u.nrows, mp = a.max_pages;
@@ -120,6 +120,18 @@ __global__ void __launch_bounds__(kAdThreads) adaptive_select_kernel(const __gri
         const float sk = ad_half(blk + L.ks_off() + (slot * NGK + g) * 2);
 #pragma unroll
         for (int r = 0; r < 4; ++r) dot[r] = fmaf(acc[r], sk, dot[r]);
+      }
+      if (a.outliers) {   // an extracted key chunk: its fp16 values (its codes are 0)
+        const uint8_t* os = blk + L.out_off();
+        const int ck = os[slot];
+        if (ck < D / 4) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float kv = ad_half(os + 2 * kPage + slot * 8 + 2 * i);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) dot[r] = fmaf(qs[r * D + 4 * ck + i], kv, dot[r]);
+          }
+        }
       }
 #pragma unroll
       for (int r = 0; r < 4; ++r) z[r] = a.s_att * dot[r];
@@ -252,7 +264,8 @@ template <int D, int KB, int KG>
 __global__ void __launch_bounds__(kAdThreads) adaptive_correct_kernel(const __grid_constant__ AdArgs a) {
   constexpr int E = D / 32, NGK = D / KG, NB = D / 32;
   constexpr int Q = KB == 8 ? 127 : 7;
-  const BlockLayout L{D, KB, KG};
+  constexpr int LPC = 4 / E;   // lanes per 4-channel chunk
+  const BlockLayout L{D, KB, KG, a.outliers};
   const AdItem it = a.items[blockIdx.x];
   const AdUnit u = a.units[it.unit];
   const int R = u.nrows, mp = a.max_pages;
@@ -262,7 +275,7 @@ __global__ void __launch_bounds__(kAdThreads) adaptive_correct_kernel(const __gr
   const int es = a.kv_bf16 ? 2 : 4;
 
   // queries: original (exact scores) and rotated (scores on the codes); row constants
-  float q0[4][E], qr[4][E], cg[4][NGK], cb[4], ce[4];
+  float q0[4][E], qr[4][E], cg[4][NGK], cb[4], ce[4], cr[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const int64_t row = r < R ? u.rows[r] : 0;
@@ -292,6 +305,7 @@ __global__ void __launch_bounds__(kAdThreads) adaptive_correct_kernel(const __gr
     for (int g = 0; g < NGK; ++g) cg[r][g] = kKappa * a.s_att * 0.5f * l1[g];
     cb[r] = a.signs ? kKappa * a.s_att * kRotSlack * sqrtf((float)D) * (float)Q * sqrtf(n2) : 0.f;
     ce[r] = kKappa * a.s_att * kRotSlack * sqrtf(n0);
+    cr[r] = a.signs ? kKappa * a.s_att * kRotSlack * sqrtf(n2) : 0.f;
   }
 
   float m[4], l[4], A[4], Bs[4], Ev[4], dmax[4], o[4][E];
@@ -360,6 +374,48 @@ __global__ void __launch_bounds__(kAdThreads) adaptive_correct_kernel(const __gr
         kh[e] = ks[c / KG] * (float)ad_key_code<D, KB>(blk, slot, c);
         vh[e] = __fmaf_rn((float)ad_val_code<D>(blk + L.v_off() + slot * (D / 2), c), sv, zv);
       }
+      // extracted chunks (their codes are 0): the fp16 values; the key chunk's
+      // share of Delta per row, summed by the chunk's lanes and broadcast
+      int ck = kNoOutlier;
+      float dlo[4] = {0.f, 0.f, 0.f, 0.f};
+      if (a.outliers) {
+        const uint8_t* os = blk + L.out_off();
+        ck = os[slot];
+        const int cv = os[kPage + slot];
+        const int part = (lane % LPC) * E;   // this lane's first channel in its chunk
+        if (cv < D / 4 && lane / LPC == cv) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            vh[e] = ad_half(os + 2 * kPage + kPage * 8 + slot * 8 + 2 * (part + e));
+            vtop = fmaxf(vtop, vh[e]);
+            vzmin = fminf(vzmin, vh[e]);
+          }
+        }
+        if (ck < D / 4) {
+          float u[4] = {0.f, 0.f, 0.f, 0.f}, kn = 0.f;
+          if (lane / LPC == ck) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              kh[e] = ad_half(os + 2 * kPage + slot * 8 + 2 * (part + e));
+              kn = fmaf(kh[e], kh[e], kn);
+#pragma unroll
+              for (int r = 0; r < 4; ++r)
+                u[r] = fmaf(fabsf(qr[r][e]), fmaf(fabsf(kh[e]), 0x1p-11f, 0x1p-25f), u[r]);
+            }
+          }
+#pragma unroll
+          for (int o2 = 1; o2 < LPC; o2 *= 2) {
+            kn += __shfl_xor_sync(0xffffffffu, kn, o2);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) u[r] += __shfl_xor_sync(0xffffffffu, u[r], o2);
+          }
+          kn = __shfl_sync(0xffffffffu, kn, ck * LPC);
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            dlo[r] = fmaf(kKappa * a.s_att, __shfl_sync(0xffffffffu, u[r], ck * LPC),
+                          cr[r] * sqrtf(kn));
+        }
+      }
       // originals of a promoted page
       float kx[E], vx[E], kn2 = 0.f;
 #pragma unroll
@@ -388,7 +444,7 @@ __global__ void __launch_bounds__(kAdThreads) adaptive_correct_kernel(const __gr
         if (kpr[r]) {
           dl = ce[r] * sqrtf(kn2);
         } else {
-          dl = cb[r] * smax;
+          dl = cb[r] * smax + dlo[r];
 #pragma unroll
           for (int g = 0; g < NGK; ++g) dl = fmaf(cg[r][g], ks[g], dl);
         }

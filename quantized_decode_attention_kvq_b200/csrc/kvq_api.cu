@@ -726,7 +726,7 @@ extern "C" {
 
 size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs, int32_t num_queries,
                               int32_t num_q_heads, int32_t max_pages_per_seq) {
-  if (check_cache(cache) || cache->outliers || cache->codec != KVQ_CODEC_INT || num_seqs < 0 ||
+  if (check_cache(cache) || cache->codec != KVQ_CODEC_INT || num_seqs < 0 ||
       num_queries < 1 ||
       num_q_heads < 1 || max_pages_per_seq < 1 || max_pages_per_seq > kAdMaxPages)
     return 0;
@@ -767,9 +767,8 @@ int kvq_adaptive_precision(const kvq_cache* cache, const void* k_orig_host,
   if (num_flagged) *num_flagged = 0;
   int rc = check_cache(cache);
   if (rc) return rc;
-  if (cache->outliers || cache->codec != KVQ_CODEC_INT)
-    return fail(KVQ_ERR_UNSUPPORTED, "the adaptive-precision ladder reads Tier-1 caches "
-                "without outlier extraction only");
+  if (cache->codec != KVQ_CODEC_INT)
+    return fail(KVQ_ERR_UNSUPPORTED, "the adaptive-precision ladder reads Tier-1 caches only");
   if (orig_dtype != KVQ_F32 && orig_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad orig_dtype");
   if (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16) return fail(KVQ_ERR_INVALID_ARG, "bad q_dtype");
   if (num_seqs < 0 || num_queries < 1 || num_q_heads < 1 || max_pages_per_seq < 1 ||
@@ -879,6 +878,7 @@ int kvq_adaptive_precision(const kvq_cache* cache, const void* k_orig_host,
   a.hkv = hkv;
   a.G = G;
   a.num_pages = cache->num_pages;
+  a.outliers = cache->outliers;
   a.s_att = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)D));
   a.rot_c = rot_constant(D);
   a.tau = tau;

@@ -133,6 +133,7 @@ struct AdArgs {
   int max_pages;
   const int32_t* seq_lens;
   int nq, hq, hkv, G, num_pages;
+  int outliers;                // the cache's blocks end in the outlier section
   float s_att, rot_c, tau, tau_cov, v_tol, rank_tol;
   const AdUnit* units;
   int num_units;

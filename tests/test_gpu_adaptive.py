@@ -41,11 +41,11 @@ def _pinned(x):
 
 
 def run_adaptive(inp, k, v, q, tau, tau_cov, v_tol, rank_tol, staging_bytes=None,
-                 timeout_ms=20000):
+                 timeout_ms=20000, outliers=False):
     """Decode on the GPU, then kvq_adaptive_precision on its flagged rows."""
     from quantized_decode_attention_kvq_b200 import kvq
     wl = inp.wl
-    g = run_gpu(inp, k, v, q, tau=tau)
+    g = run_gpu(inp, k, v, q, tau=tau, outliers=outliers)
     assert g["err"] == 0
     c, qd, pt, sl = g["cache"], g["q"], g["pt"], g["sl"]
     B, NQ, HQ, d = q.shape
@@ -195,6 +195,35 @@ def test_adaptive_matches_oracle(name, seed, tau, tau_cov, v_tol, rank_tol):
     n_amb = _check(inp, res, ref, amb, flagged)
     assert n_amb == 0, f"{n_amb} rows within the decision band"
     # certified: the GPU's own output is within its bound of exact attention
+    od = oracle.dense(q, k, v, inp.seq_lens)
+    assert (res["bound"][flagged] >= max_err(od, res["out"])[flagged]).all()
+
+
+EXTRACTION_CASES = [
+    # name, seed, tau, tau_cov, v_tol, rank_tol (spikes in half the sequences)
+    ("serving", 0, 0.0, 0.995, 1e-3, 0.0),
+    ("llama8b", 2, 0.0, 0.9, 1e-3, 0.05),
+    ("rotated", 1, 0.0, 0.9, math.inf, 0.0),
+    ("tiny", 0, 0.0, 0.8, 1e-3, 0.0),
+]
+
+
+@pytest.mark.parametrize("name,seed,tau,tau_cov,v_tol,rank_tol", EXTRACTION_CASES)
+def test_adaptive_with_extraction_matches_oracle(name, seed, tau, tau_cov, v_tol, rank_tol):
+    """The ladder over a cache with Med3x outlier extraction: scores, values,
+    Delta and range include the extracted chunks, as the oracle's do."""
+    inp = small(name, seed, spike_seq_frac=0.5, spike_token_frac=0.05)
+    k, v = inp.kv()
+    q = inp.q()
+    res = run_adaptive(inp, k, v, q, tau, tau_cov, v_tol, rank_tol, outliers=True)
+    oc = oracle_cache(inp, outliers=True)
+    assert oc.append(k, v, inp.page_table, np.zeros(inp.wl.num_seqs, np.int32),
+                     valid=np.array(inp.seq_lens, np.int32)) == 0
+    flagged = res["g"]["flags"].astype(bool)
+    ref = oc.decode_adaptive(q, inp.page_table, inp.seq_lens, k, v, tau_cov, v_tol, rank_tol,
+                             tau=tau, row_mask=flagged.astype(np.uint8))
+    amb = _oracle_row_decisions(inp, oc, q, k, ref, tau_cov, v_tol, rank_tol, tau)
+    _check(inp, res, ref, amb, flagged)
     od = oracle.dense(q, k, v, inp.seq_lens)
     assert (res["bound"][flagged] >= max_err(od, res["out"])[flagged]).all()
 
