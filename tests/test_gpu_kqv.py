@@ -213,3 +213,48 @@ def test_full_size_sampled(name):
     rows, o_hat = _check(inp, r, q, wl.tau, f"kqv {name} full size")
     o_dense = oracle.dense(q[seqs], k[seqs], v[seqs], np.array(inp.seq_lens)[seqs])
     assert (max_err(o_dense, r["out"][rows]) <= r["bound"][rows]).all()
+
+
+
+def test_exact_fallback_on_a_kqv_cache():
+    """The exact fallback recomputes the flagged rows of a KQV cache from the
+    pinned originals (exact attention) and leaves the others as decoded."""
+    from quantized_decode_attention_kvq_b200 import kvq
+    inp = small("serving", 7, **SPIKES)
+    wl = inp.wl
+    k, v = inp.kv()
+    q = inp.q()
+    r = _run(inp, k, v, q)
+    tau = float(np.median(r["bound"]))
+    g = r["cache"]
+    pt = torch.from_numpy(inp.page_table).cuda()
+    sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
+    qd = to_torch(q)
+    S, NQ, HQ, d = q.shape
+    ws = g.workspace(S, NQ, HQ, pt.shape[1])
+    out, bound, flags = g.decode(qd, pt, sl, ws, tau=tau)
+    torch.cuda.synchronize()
+    fl = flags.cpu().numpy().reshape(-1).astype(bool)
+    assert 0 < fl.sum() < fl.size
+    T = k.shape[2]
+    kh = (torch.from_numpy(k.view(np.int16)).view(torch.bfloat16) if k.dtype == np.uint16
+          else torch.from_numpy(k)).pin_memory()
+    vh = (torch.from_numpy(v.view(np.int16)).view(torch.bfloat16) if v.dtype == np.uint16
+          else torch.from_numpy(v)).pin_memory()
+    dt = kvq.KVQ_BF16 if k.dtype == np.uint16 else kvq.KVQ_F32
+    qdt = kvq.KVQ_BF16 if qd.dtype == torch.bfloat16 else kvq.KVQ_F32
+    st_bytes = kvq.kvq_fallback_staging_size(g.desc, dt, max(inp.seq_lens)) * 4
+    staging = torch.empty(st_bytes, dtype=torch.uint8, device="cuda")
+    fh = torch.zeros(fl.size, dtype=torch.uint8).pin_memory()
+    sl_h = np.array(inp.seq_lens, np.int32)
+    decoded = out.cpu().numpy().reshape(-1, d).copy()
+    rc, n = kvq.kvq_fallback_exact(g.desc, kh, vh, dt, wl.num_kv_heads * T * d, T * d, qd, qdt,
+                                   S, NQ, HQ, sl_h.ctypes.data, 0.0, flags, fh, out, staging,
+                                   st_bytes, None, torch.cuda.Stream(), 20000)
+    torch.cuda.synchronize()
+    assert rc == kvq.KVQ_OK, kvq.last_error()
+    assert n == int(fl.sum())
+    res = out.cpu().numpy().reshape(-1, d).astype(np.float64)
+    od = oracle.dense(q, k, v, inp.seq_lens)
+    assert max_err(od[fl], res[fl]).max() <= 1e-4
+    assert np.array_equal(res[~fl], decoded[~fl].astype(np.float64))
