@@ -152,6 +152,11 @@ __device__ __noinline__ float fused_append(const DecodeArgs& a, int b, int kvh, 
   return eu;
 }
 
+// The ring stage of a page step: a compile-time constant, or a runtime index.
+template <int I>
+__device__ __forceinline__ constexpr int stage_index(std::integral_constant<int, I>) { return I; }
+__device__ __forceinline__ int stage_index(int st) { return st; }
+
 // APPEND: the fused step (kvq_decode_attention_append); a separate
 // instantiation, so the plain decode carries none of its code or registers.
 template <int D, int KB, int KG, int S, bool APPEND, bool OUT>
@@ -522,7 +527,7 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   // a fixed offset; FULL pages (all 16 tokens inside the context, every page but
   // possibly a sequence's last) skip the per-token context masks.
   auto page_step = [&](auto st_c, auto full_c, int j, uint32_t par) -> bool {
-    constexpr int st = decltype(st_c)::value;
+    const int st = stage_index(st_c);
     constexpr bool FULL = decltype(full_c)::value;
     const bool ok = mbar_wait(&bar[st], par);
     if (!__all_sync(0xffffffffu, ok)) {
@@ -844,16 +849,25 @@ __global__ void __launch_bounds__(kWarps * 32, min_ctas<D, KB, KG>())
   uint32_t par = 0;
   bool going = true;
   int jstop = nloc;   // the page whose wait ran out, if one did
-  for (int j0 = 0; j0 < nloc && going; j0 += S) {
+  // Full pages (every page but possibly the sequence's last) run through the
+  // mask-free step, one copy per ring stage; a partial last page, always this
+  // warp's last local page, through one masked copy with a runtime stage.
+  const bool last_partial =
+      nloc > 0 && n % kPage != 0 && first + (nloc - 1) * kWarps == last_page;
+  const int nfull = last_partial ? nloc - 1 : nloc;
+  for (int j0 = 0; j0 < nfull && going; j0 += S) {
     static_for<0, S>([&](auto u_c) {
       const int j = j0 + decltype(u_c)::value;
-      if (!going || j >= nloc) return;
-      const bool full = first + j * kWarps < last_page || n % kPage == 0;
-      going = full ? page_step(u_c, std::true_type{}, j, par)
-                   : page_step(u_c, std::false_type{}, j, par);
+      if (!going || j >= nfull) return;
+      going = page_step(u_c, std::true_type{}, j, par);
       if (!going) jstop = j;
     });
     par ^= 1u;
+  }
+  if (going && last_partial) {
+    const int j = nloc - 1;
+    going = page_step(j % S, std::false_type{}, j, (uint32_t)((j / S) & 1));
+    if (!going) jstop = j;
   }
   // After a wait that ran out, the copies still in flight (pages jstop ..
   // min(jstop + S, nloc) - 1, issued but not consumed) are waited for, each
