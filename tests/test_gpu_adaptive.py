@@ -87,7 +87,7 @@ def run_adaptive(inp, k, v, q, tau, tau_cov, v_tol, rank_tol, staging_bytes=None
 
 def ambiguous_rows(c, q, k, page_table, seq_lens, group, ref, tau_cov, v_tol, rank_tol, tau,
                    as_f32, row_mask=None):
-    """Rows whose integer decisions lie within BAND of a threshold, judged on the
+    """Rows whose integer decisions lie within BAND of a threshold, decided on the
     oracle's fp64 values (q, k of the sequences the oracle cache holds)."""
     B, NQ, HQ, d = q.shape
     amb = np.zeros(B * NQ * HQ, bool)
