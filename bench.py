@@ -939,7 +939,7 @@ def main():
     ap.add_argument("--also", default=None,
                     help="comma-separated workloads measured in the same run and reported "
                          "under 'workloads'; a '+med3' suffix adds outlier extraction to the "
-                         "cache, '+kqv' uses the KQV codec (default: long128k,serving,"
+                         "cache, '+kqv' uses the KQV codec (default: long128k,rotated,serving,"
                          "llama8b+med3,serving+med3,llama8b+kqv with llama8b; 'none')")
     ap.add_argument("--two-calls", action="store_true",
                     help="step = kvq_quantize_append + kvq_decode_attention (default: the fused "
@@ -948,7 +948,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.also is None:
-        args.also = ("long128k,serving,llama8b+med3,serving+med3,llama8b+kqv"
+        args.also = ("long128k,rotated,serving,llama8b+med3,serving+med3,llama8b+kqv"
                      if args.workload == "llama8b" else "none")
     if args.impl == "reference":
         run_reference(args)

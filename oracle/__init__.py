@@ -9,7 +9,7 @@ with gcc, fp32 codec arithmetic in a fixed order and fp64 attention.
 Every function cites the page passage it follows; see ``kvq_oracle.c``.
 Pinned by ``tests/test_oracle_*.py`` against hand-worked cases, closed forms,
 library routines (scipy's Hadamard matrix, numpy's float16, torch's fp64
-scaled-dot-product attention) and brute force; the bound's magnitude by
+scaled-dot-product attention and float8_e4m3fn cast) and brute force; the bound's magnitude by
 hand-worked cases (``tests/golden/bound_hand_worked.txt``).
 """
 
@@ -59,6 +59,14 @@ def _configure(L: ctypes.CDLL) -> ctypes.CDLL:
     if hasattr(L, "oq_block_bytes"):
         L.oq_block_bytes.restype = ctypes.c_int64
         for name in ("oq_lloyd_max", "oq_tables", "oq_append", "oq_decode"):
+            getattr(L, name).restype = ctypes.c_int
+    if hasattr(L, "oh_block_bytes"):
+        L.oh_block_bytes.restype = ctypes.c_int64
+        L.oh_e4m3_value.restype = ctypes.c_double
+        L.oh_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oh_e4m3_rn.restype = ctypes.c_uint8
+        L.oh_e4m3_rn.argtypes = [ctypes.c_float]
+        for name in ("oh_direction", "oh_append", "oh_decode"):
             getattr(L, name).restype = ctypes.c_int
     for name in ("oc_quantize_sym", "oc_quantize_asym", "oc_append", "oc_decode",
                  "oc_decode_promote_values", "oc_dense", "oc_f16_round_n"):
@@ -442,6 +450,105 @@ class KqvCache:
                              int(q.dtype == np.float32), B, NQ, HQ, _p(pt), pt.shape[1], _p(sl),
                              ctypes.c_float(scale), ctypes.c_float(tau), _p(self.signs),
                              _p(self.S), _p(out), _p(bound), _p(flags), _p(diag), _p(rm))
+        if rc != OK:
+            raise ValueError(f"oracle decode failed: {rc}")
+        return out, bound, flags, diag
+
+
+class OhCfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("d", "hkv", "num_pages", "S")]
+
+
+def hq_primary(p: int) -> np.ndarray:
+    """Unit p of the binary tetrahedral group 2T, in the oracle's order."""
+    out = np.zeros(4, dtype=np.float32)
+    lib().oh_primary(int(p), _p(out))
+    return out
+
+
+def hq_codeword(sec, i: int) -> np.ndarray:
+    """Codeword i = 24 s + p (the fp32 product q_p q_s) of a secondary set [S][4]."""
+    sec = _c(sec, np.float32)
+    out = np.zeros(4, dtype=np.float32)
+    lib().oh_codeword(_p(sec), int(i), _p(out))
+    return out
+
+
+def hq_direction(x, sec) -> int:
+    """The direction code of one 4-channel chunk x against a secondary set [S][4]."""
+    x = _c(x, np.float32)
+    sec = _c(sec, np.float32)
+    return int(lib().oh_direction(_p(x), _p(sec), int(sec.shape[0])))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().oh_e4m3_value(int(code)))
+
+
+def e4m3_rn(x) -> int:
+    return int(lib().oh_e4m3_rn(ctypes.c_float(float(x))))
+
+
+class HqCache:
+    """The oracle's paged cache of the HQMQ codec ("Hurwitz Quaternion
+    Multiplicative Quantization for KV Cache Compression", Method 1-2): every
+    4-channel chunk of K and V coded by its radius (fp8 E4M3) and the index of
+    the nearest product codeword q_p q_s (q_p in 2T, q_s from the secondary
+    set of its kv head and role)."""
+
+    def __init__(self, head_dim, num_kv_heads, num_pages, secondary):
+        sec = _c(secondary, np.float32)
+        assert sec.ndim == 4 and sec.shape[0] == num_kv_heads and sec.shape[1] == 2 \
+            and sec.shape[3] == 4
+        self.cfg = OhCfg(head_dim, num_kv_heads, num_pages, sec.shape[2])
+        bb = lib().oh_block_bytes(ctypes.byref(self.cfg))
+        if bb < 0:
+            raise ValueError("unsupported cache configuration")
+        self.block_bytes = int(bb)
+        self.pool = np.zeros(num_pages * num_kv_heads * self.block_bytes, dtype=np.uint8)
+        self.eta = np.zeros((num_pages, num_kv_heads), dtype=np.float32)
+        self.sec = sec
+
+    def append(self, k, v, page_table, start_pos, valid=None):
+        k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v)
+        assert k.shape == v.shape and k.dtype == v.dtype and k.ndim == 4
+        B, H, T, d = k.shape
+        pt = _c(page_table, np.int32)
+        sp = _c(start_pos, np.int32)
+        vl = None if valid is None else _c(valid, np.int32)
+        return lib().oh_append(ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(k),
+                               _p(v), int(k.dtype == np.float32), ctypes.c_int64(H * T * d),
+                               ctypes.c_int64(T * d), ctypes.c_int64(d), B, T, _p(vl), _p(pt),
+                               pt.shape[1], _p(sp), _p(self.sec))
+
+    def read_token(self, page: int, kv_head: int, slot: int):
+        """(k^, v^) fp32 [d] of one slot, as the append reconstructed them."""
+        d = self.cfg.d
+        blk = self.pool[(page * self.cfg.hkv + kv_head) * self.block_bytes:][:self.block_bytes]
+        kh = np.zeros(d, dtype=np.float32)
+        vh = np.zeros(d, dtype=np.float32)
+        lib().oh_read_token(ctypes.byref(self.cfg), _p(np.ascontiguousarray(blk)), int(slot),
+                            _p(np.ascontiguousarray(self.sec[kv_head])), _p(kh), _p(vh))
+        return kh, vh
+
+    def decode(self, q, page_table, seq_lens, scale=None, tau=math.inf, row_mask=None):
+        """Returns (o_hat f64 [rows][d], bound f64 [rows], flags u8 [rows], diag [rows][8])."""
+        q = np.ascontiguousarray(q)
+        B, NQ, HQ, d = q.shape
+        rows = B * NQ * HQ
+        scale = default_scale(d) if scale is None else np.float32(scale)
+        out = np.zeros((rows, d), dtype=np.float64)
+        bound = np.zeros(rows, dtype=np.float64)
+        flags = np.zeros(rows, dtype=np.uint8)
+        diag = np.zeros((rows, 8), dtype=np.float64)
+        pt = _c(page_table, np.int32)
+        sl = _c(seq_lens, np.int32)
+        rm = None if row_mask is None else _c(row_mask, np.uint8)
+        rc = lib().oh_decode(ctypes.byref(self.cfg), _p(self.pool), _p(self.eta), _p(q),
+                             int(q.dtype == np.float32), B, NQ, HQ, _p(pt), pt.shape[1], _p(sl),
+                             ctypes.c_float(scale), ctypes.c_float(tau), _p(self.sec), _p(out),
+                             _p(bound), _p(flags), _p(diag), _p(rm))
         if rc != OK:
             raise ValueError(f"oracle decode failed: {rc}")
         return out, bound, flags, diag

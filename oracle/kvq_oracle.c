@@ -20,7 +20,9 @@
  *     quantization scales, the query norms and the value range.
  * and ("Statistical Inference and Quality Measures of KV Cache Quantisations
  * Inspired by TurboQuant", Quantisation schemes, KQV): a Walsh-Hadamard
- * rotation applied to K before scalar quantization.
+ * rotation applied to K before scalar quantization, and the KQV codec (oq_*);
+ * and ("Hurwitz Quaternion Multiplicative Quantization for KV Cache
+ * Compression", Method 1-3): the HQMQ codec (oh_*) and Med3x extraction.
  *
  * Readings taken where the pages are silent (all listed in the design notes):
  *   keys per token and group, symmetric, codes in [-Q, Q] with Q = 127 (8 bit)
@@ -1485,6 +1487,389 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
       }
     free(z);
     free(dl);
+    free(vh);
+  }
+  return OC_OK;
+}
+
+/* ======================================================================== */
+/* HQMQ codec ("Hurwitz Quaternion Multiplicative Quantization for KV Cache */
+/* Compression", Method 1-2).  Every 4-channel chunk x of a K or V vector   */
+/* is a quaternion (x0 + x1 i + x2 j + x3 k) split into its radius r = |x|  */
+/* and its direction on S^3; the direction is coded by the product         */
+/* codebook C = { q_p q_s : q_p in 2T, q_s in the secondary set } (24 S    */
+/* codewords), the radius is stored in 8 bits.                              */
+/* Readings (the page gives the structure, not the arithmetic):            */
+/*  - 2T, the 24 Hurwitz units, in the order p = 0..7: +-1, +-i, +-j, +-k   */
+/*    (p = 2n + [negative], n the axis), p = 8..23: (+-1 +-i +-j +-k)/2     */
+/*    with component n negative when bit n of p - 8 is set;                 */
+/*  - the secondary set: S unit quaternions per (kv head, role), an input   */
+/*    (drawn from the seed), fp32 [hkv][2][S][4], role 0 = K, 1 = V;        */
+/*  - codeword i = 24 s + p is the Hamilton product q_p q_s in fp32: each   */
+/*    component is the 4-term signed sum of the products (exact: q_p's      */
+/*    entries are 0, +-1, +-1/2) added left to right, each add rounded;     */
+/*  - the direction's code maximizes <x, c> (equivalently <x/r, c>, r > 0). */
+/*    The inner products are taken through the group: <x, q_p q_s> =        */
+/*    <x conj(q_s), q_p>; y = x conj(q_s) has each component a sequential  */
+/*    fmaf chain over x0..x3; over the 8 axis units the best is max_n |y_n| */
+/*    (the first n on ties, sign of y_n), over the 16 half units it is      */
+/*    0.5 (((|y0| + |y1|) + |y2|) + |y3|) with the signs of y (-0 as +);    */
+/*    the half unit wins over the axis one only when strictly larger, and a */
+/*    later s only when strictly larger than every earlier candidate;       */
+/*  - r = sqrt((x0^2 + x1^2) + (x2^2 + x3^2)) in fp32 (the Med3x chunk      */
+/*    norm); stored as fp8 E4M3 (round to nearest, ties to even; above 448  */
+/*    it saturates to 448); a chunk with a non-finite norm gets code 0 and  */
+/*    radius 0 and sets the range error;                                    */
+/*  - x^ = r^ * c (fp32 products);                                           */
+/*  - per token: |k|_2 (sequential fmaf chain) and eps = |k - k^|_2 (the    */
+/*    same chain over the channels' differences) raised by 2^-16 of itself, */
+/*    one ulp up; the bound's Delta_j = kappa*s*|q|_2 (eps_j + 2^-16 |k_j|);*/
+/*  - eta_b = the block's largest max_c |v - v^| + 2^-16 |v|_2, one ulp up; */
+/*    the value range per 32-channel group starts at [0, 0] (a zeroed      */
+/*    block) and widens to every v^ appended.                                */
+/* Block of one (page, kv head), 16 tokens, d/4 chunks per vector:          */
+/*   [K codes u16 [16][d/4]][V codes u16 [16][d/4]][K radii e4m3 [16][d/4]]  */
+/*   [V radii e4m3 [16][d/4]][|k| f32 [16]][eps f32 [16]]                    */
+/*   [v^ max, min f32 [d/32][2]]                                             */
+/* u16 little-endian.                                                        */
+/* ======================================================================== */
+typedef struct {
+  int32_t d, hkv, num_pages, S;
+} oh_cfg;
+
+#define OH_MAX_S 2730   /* 24 S codewords index in 16 bits */
+
+static int oh_ok(const oh_cfg* c) {
+  return c && (c->d == 64 || c->d == 128) && c->hkv > 0 && c->num_pages >= 0 && c->S >= 1 &&
+         c->S <= OH_MAX_S;
+}
+static int64_t oh_off_vi(const oh_cfg* c) { return (int64_t)OC_PAGE * (c->d / 4) * 2; }
+static int64_t oh_off_kr(const oh_cfg* c) { return (int64_t)OC_PAGE * (c->d / 4) * 4; }
+static int64_t oh_off_vr(const oh_cfg* c) { return oh_off_kr(c) + (int64_t)OC_PAGE * (c->d / 4); }
+static int64_t oh_off_kn(const oh_cfg* c) { return oh_off_vr(c) + (int64_t)OC_PAGE * (c->d / 4); }
+static int64_t oh_off_ke(const oh_cfg* c) { return oh_off_kn(c) + 4 * OC_PAGE; }
+static int64_t oh_off_rg(const oh_cfg* c) { return oh_off_kn(c) + 8 * OC_PAGE; }
+
+int64_t oh_block_bytes(const oh_cfg* c) {
+  if (!oh_ok(c)) return -1;
+  return oh_off_rg(c) + (int64_t)(c->d / 32) * 2 * 4;
+}
+
+/* Unit p of 2T (Method 1: the 24 vertices of the 24-cell). */
+void oh_primary(int p, float* q) {
+  for (int n = 0; n < 4; ++n) q[n] = 0.0f;
+  if (p < 8) {
+    q[p / 2] = (p & 1) ? -1.0f : 1.0f;
+  } else {
+    for (int n = 0; n < 4; ++n) q[n] = ((p - 8) >> n) & 1 ? -0.5f : 0.5f;
+  }
+}
+
+/* Hamilton product a b with exact term products (a from 2T), each component
+ * summed left to right in fp32. */
+static void oh_mul(const float* a, const float* b, float* c) {
+  float t[4][4] = {
+      {a[0] * b[0], -(a[1] * b[1]), -(a[2] * b[2]), -(a[3] * b[3])},
+      {a[0] * b[1], a[1] * b[0], a[2] * b[3], -(a[3] * b[2])},
+      {a[0] * b[2], -(a[1] * b[3]), a[2] * b[0], a[3] * b[1]},
+      {a[0] * b[3], a[1] * b[2], -(a[2] * b[1]), a[3] * b[0]},
+  };
+  for (int n = 0; n < 4; ++n) c[n] = ((t[n][0] + t[n][1]) + t[n][2]) + t[n][3];
+}
+
+/* Codeword i = 24 s + p of one secondary set (sec: [S][4]). */
+void oh_codeword(const float* sec, int i, float* c) {
+  float qp[4];
+  oh_primary(i % 24, qp);
+  oh_mul(qp, sec + 4 * (i / 24), c);
+}
+
+/* The direction code of chunk x (Method 1: the codeword of largest inner
+ * product), through y = x conj(q_s) as the readings above fix. */
+int oh_direction(const float* x, const float* sec, int S) {
+  int best = 0;
+  float bv = -INFINITY;
+  for (int s = 0; s < S; ++s) {
+    const float* b = sec + 4 * s;
+    float y[4];
+    y[0] = fmaf(x[3], b[3], fmaf(x[2], b[2], fmaf(x[1], b[1], x[0] * b[0])));
+    y[1] = fmaf(x[3], b[2], fmaf(-x[2], b[3], fmaf(x[1], b[0], -x[0] * b[1])));
+    y[2] = fmaf(-x[3], b[1], fmaf(x[2], b[0], fmaf(x[1], b[3], -x[0] * b[2])));
+    y[3] = fmaf(x[3], b[0], fmaf(x[2], b[1], fmaf(-x[1], b[2], -x[0] * b[3])));
+    float a[4];
+    for (int n = 0; n < 4; ++n) a[n] = fabsf(y[n]);
+    int n0 = 0;
+    for (int n = 1; n < 4; ++n)
+      if (a[n] > a[n0]) n0 = n;
+    float v = a[n0];
+    int p = 2 * n0 + (y[n0] < 0.0f);
+    float h = 0.5f * (((a[0] + a[1]) + a[2]) + a[3]);
+    if (h > v) {
+      v = h;
+      p = 8;
+      for (int n = 0; n < 4; ++n) p += (y[n] < 0.0f) << n;
+    }
+    if (v > bv) {
+      bv = v;
+      best = 24 * s + p;
+    }
+  }
+  return best;
+}
+
+/* fp8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+ * infinities, 0x7F NaN): the value of a non-negative code, and the code of a
+ * non-negative finite x rounded to nearest, ties to the even code, saturating
+ * at 448 (0x7E). */
+double oh_e4m3_value(uint8_t code) {
+  int e = (code >> 3) & 15, m = code & 7;
+  double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+  return (code & 0x80) ? -v : v;
+}
+
+uint8_t oh_e4m3_rn(float x) {
+  double xv = (double)x;
+  if (!(xv > 0.0)) return 0;
+  if (xv >= 448.0) return 0x7E;
+  int lo = 0;
+  while (lo + 1 <= 0x7E && oh_e4m3_value((uint8_t)(lo + 1)) <= xv) ++lo;
+  if (oh_e4m3_value((uint8_t)lo) == xv) return (uint8_t)lo;
+  double dl = xv - oh_e4m3_value((uint8_t)lo), du = oh_e4m3_value((uint8_t)(lo + 1)) - xv;
+  if (dl < du) return (uint8_t)lo;
+  if (du < dl) return (uint8_t)(lo + 1);
+  return (uint8_t)((lo & 1) ? lo + 1 : lo);
+}
+
+static float oh_chunk_radius(const float* x) {
+  float a = x[0] * x[0], b = x[1] * x[1], e = x[2] * x[2], f = x[3] * x[3];
+  return sqrtf((a + b) + (e + f));
+}
+
+/* Code one d-vector x: chunk codes and radii, and the fp32 reconstruction. */
+static int oh_code_vector(const float* x, int d, const float* sec, int S, uint8_t* idx,
+                          uint8_t* rad, float* xh) {
+  int rc = OC_OK;
+  for (int ch = 0; ch < d / 4; ++ch) {
+    const float* xc = x + 4 * ch;
+    float r = oh_chunk_radius(xc);
+    int i = 0;
+    uint8_t rq = 0;
+    if (!isfinite(r)) {
+      rc = OC_ERR_RANGE;
+    } else {
+      i = oh_direction(xc, sec, S);
+      rq = oh_e4m3_rn(r);
+    }
+    oc_wr16(idx + 2 * ch, (uint16_t)i);
+    rad[ch] = rq;
+    float cw[4];
+    oh_codeword(sec, i, cw);
+    float rv = (float)oh_e4m3_value(rq);
+    for (int n = 0; n < 4; ++n) xh[4 * ch + n] = rv * cw[n];
+  }
+  return rc;
+}
+
+static float oh_chain_norm2(const float* a, int d) {
+  float s = 0.0f;
+  for (int i = 0; i < d; ++i) s = fmaf(a[i], a[i], s);
+  return s;
+}
+
+/* Quantize one token of one kv head into slot `slot` (secs: this kv head's
+ * [2][S][4]); returns its eta contribution and raises the block's range. */
+static int oh_quantize_token(const oh_cfg* c, uint8_t* blk, int slot, const float* k,
+                             const float* v, const float* secs, float* eta_out) {
+  int d = c->d, nc = d / 4, S = c->S;
+  float kh[128], vh[128], e[128];
+  int rc = oh_code_vector(k, d, secs, S, blk + (int64_t)slot * nc * 2,
+                          blk + oh_off_kr(c) + (int64_t)slot * nc, kh);
+  int rv = oh_code_vector(v, d, secs + 4 * S, S, blk + oh_off_vi(c) + (int64_t)slot * nc * 2,
+                          blk + oh_off_vr(c) + (int64_t)slot * nc, vh);
+  if (rv != OC_OK) rc = rv;
+  float nk = sqrtf(oh_chain_norm2(k, d));
+  for (int i = 0; i < d; ++i) e[i] = k[i] - kh[i];
+  float en = sqrtf(oh_chain_norm2(e, d));
+  float eps = nextafterf(fmaf(en, 1.0f / 65536.0f, en), INFINITY);
+  oq_wrf(blk + oh_off_kn(c) + 4 * slot, nk);
+  oq_wrf(blk + oh_off_ke(c) + 4 * slot, eps);
+  float err = 0.0f;
+  for (int i = 0; i < d; ++i) {
+    float ev = fabsf(v[i] - vh[i]);
+    if (ev > err) err = ev;
+  }
+  float nv = sqrtf(oh_chain_norm2(v, d));
+  *eta_out = nextafterf(fmaf(1.0f / 65536.0f, nv, err), INFINITY);
+  uint8_t* rg = blk + oh_off_rg(c);
+  for (int g = 0; g < d / 32; ++g) {
+    float hi = oq_rdf(rg + 8 * g), lo = oq_rdf(rg + 8 * g + 4);
+    for (int ch = 32 * g; ch < 32 * g + 32; ++ch) {
+      if (vh[ch] > hi) hi = vh[ch];
+      if (vh[ch] < lo) lo = vh[ch];
+    }
+    oq_wrf(rg + 8 * g, hi);
+    oq_wrf(rg + 8 * g + 4, lo);
+  }
+  return rc;
+}
+
+/* Quantize-on-append for the HQMQ codec; arguments as oc_append, plus the
+ * secondary sets sec (fp32 [hkv][2][S][4]). */
+int oh_append(const oh_cfg* c, uint8_t* pool, float* eta, const void* k, const void* v,
+              int in_is_f32, int64_t seq_stride, int64_t head_stride, int64_t tok_stride,
+              int num_seqs, int num_tokens, const int32_t* valid, const int32_t* page_table,
+              int max_pages, const int32_t* start_pos, const float* sec) {
+  if (!oh_ok(c) || !sec) return OC_ERR_ARG;
+  int64_t bb = oh_block_bytes(c);
+  int rc = OC_OK;
+  float xk[128], xv[128];
+  for (int b = 0; b < num_seqs; ++b) {
+    int nt = valid ? valid[b] : num_tokens;
+    for (int t = 0; t < nt; ++t) {
+      int pos = start_pos[b] + t;
+      int lp = pos / OC_PAGE;
+      if (lp >= max_pages) return OC_ERR_ARG;
+      int page = page_table[(int64_t)b * max_pages + lp];
+      if (page < 0 || page >= c->num_pages) return OC_ERR_ARG;
+      for (int h = 0; h < c->hkv; ++h) {
+        int64_t off = b * seq_stride + h * head_stride + t * tok_stride;
+        oc_load_vec(k, in_is_f32, off, c->d, xk);
+        oc_load_vec(v, in_is_f32, off, c->d, xv);
+        int bad = 0;
+        for (int i = 0; i < c->d; ++i) bad |= !isfinite(xk[i]) || !isfinite(xv[i]);
+        uint8_t* blk = pool + ((int64_t)page * c->hkv + h) * bb;
+        float e;
+        int r = oh_quantize_token(c, blk, pos % OC_PAGE, xk, xv, sec + (int64_t)h * 8 * c->S, &e);
+        if (r != OC_OK || bad) rc = OC_ERR_RANGE;
+        float* ep = eta + (int64_t)page * c->hkv + h;
+        if (e > *ep) *ep = e;
+      }
+    }
+  }
+  return rc;
+}
+
+/* Read back token `slot` of a block: k^ and v^ as the append reconstructed
+ * them (fp32 products r^ * c). */
+void oh_read_token(const oh_cfg* c, const uint8_t* blk, int slot, const float* secs, float* kh,
+                   float* vh) {
+  int nc = c->d / 4;
+  for (int role = 0; role < 2; ++role) {
+    const uint8_t* idx = blk + (role ? oh_off_vi(c) : 0) + (int64_t)slot * nc * 2;
+    const uint8_t* rad = blk + (role ? oh_off_vr(c) : oh_off_kr(c)) + (int64_t)slot * nc;
+    float* out = role ? vh : kh;
+    for (int ch = 0; ch < nc; ++ch) {
+      float cw[4];
+      oh_codeword(secs + role * 4 * c->S, oc_rd16(idx + 2 * ch), cw);
+      float rv = (float)oh_e4m3_value(rad[ch]);
+      for (int n = 0; n < 4; ++n) out[4 * ch + n] = rv * cw[n];
+    }
+  }
+}
+
+/* Decode attention and its certified bound over an HQMQ cache, for every
+ * query row (sequence b, query i, q head h; kv head h / (Hq/Hkv)), in fp64
+ * over the fp32 reconstructions:
+ *   z^_j = scale * q . k^_j;  o^ = sum_j p^_j v^_j
+ *   Delta_j = kappa*scale*|q|_2 (eps_j + 2^-16 |k_j|)
+ *   A, B, TV, range, E_key, E_val, bound and flag as in oq_decode.
+ * diag (optional) as in oc_decode. */
+int oh_decode(const oh_cfg* c, const uint8_t* pool, const float* eta, const void* q,
+              int q_is_f32, int num_seqs, int nq, int hq, const int32_t* page_table,
+              int max_pages, const int32_t* seq_lens, float scale, float tau, const float* sec,
+              double* out, double* bound, uint8_t* flags, double* diag,
+              const uint8_t* row_mask) {
+  if (!oh_ok(c) || hq % c->hkv || !sec) return OC_ERR_ARG;
+  int d = c->d, G = hq / c->hkv, NG = d / 32;
+  int64_t bb = oh_block_bytes(c);
+  double sc = (double)scale;
+  for (int b = 0; b < num_seqs; ++b) {
+    int n = seq_lens[b];
+    double* z = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    double* dl = n ? (double*)malloc(sizeof(double) * n) : NULL;
+    float* kh = n ? (float*)malloc(sizeof(float) * n * d) : NULL;
+    float* vh = n ? (float*)malloc(sizeof(float) * n * d) : NULL;
+    int cur_kv = -1;
+    for (int h = 0; h < hq; ++h)
+      for (int i = 0; i < nq; ++i) {
+        int64_t row = ((int64_t)b * nq + i) * hq + h;
+        if (row_mask && !row_mask[row]) continue;
+        int kv = h / G;
+        double* o = out + row * d;
+        for (int ch = 0; ch < d; ++ch) o[ch] = 0.0;
+        if (n == 0) {
+          bound[row] = 0.0;
+          flags[row] = 0;
+          if (diag) for (int t = 0; t < 8; ++t) diag[row * 8 + t] = 0.0;
+          continue;
+        }
+        if (kv != cur_kv) {   /* the reconstructions of this (sequence, kv head) */
+          for (int j = 0; j < n; ++j) {
+            int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
+            const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+            oh_read_token(c, blk, j % OC_PAGE, sec + (int64_t)kv * 8 * c->S,
+                          kh + (int64_t)j * d, vh + (int64_t)j * d);
+          }
+          cur_kv = kv;
+        }
+        float qf[128];
+        oc_load_vec(q, q_is_f32, row * d, d, qf);
+        double qn2 = 0.0;
+        for (int ch = 0; ch < d; ++ch) qn2 += (double)qf[ch] * (double)qf[ch];
+        qn2 = sqrt(qn2);
+        double hi[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        double lo[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+        double eta_max = 0.0, m = -INFINITY;
+        for (int j = 0; j < n; ++j) {
+          int page = page_table[(int64_t)b * max_pages + j / OC_PAGE], slot = j % OC_PAGE;
+          const uint8_t* blk = pool + ((int64_t)page * c->hkv + kv) * bb;
+          double dot = 0.0;
+          for (int ch = 0; ch < d; ++ch) dot += (double)qf[ch] * (double)kh[(int64_t)j * d + ch];
+          z[j] = sc * dot;
+          dl[j] = OC_KAPPA * sc * qn2 *
+                  ((double)oq_rdf(blk + oh_off_ke(c) + 4 * slot) +
+                   OC_ROT_SLACK * (double)oq_rdf(blk + oh_off_kn(c) + 4 * slot));
+          if (z[j] > m) m = z[j];
+          if (slot == 0 || j == 0) {   /* each block of the context once */
+            const uint8_t* rg = blk + oh_off_rg(c);
+            for (int g = 0; g < NG; ++g) {
+              if (oq_rdf(rg + 8 * g) > hi[g]) hi[g] = oq_rdf(rg + 8 * g);
+              if (oq_rdf(rg + 8 * g + 4) < lo[g]) lo[g] = oq_rdf(rg + 8 * g + 4);
+            }
+            double e = (double)eta[(int64_t)page * c->hkv + kv];
+            if (e > eta_max) eta_max = e;
+          }
+        }
+        double l = 0.0;
+        for (int j = 0; j < n; ++j) l += exp(z[j] - m);
+        double A = 0.0, B = 0.0, Ev = 0.0, dmax = 0.0;
+        for (int j = 0; j < n; ++j) {
+          double p = exp(z[j] - m) / l;
+          int page = page_table[(int64_t)b * max_pages + j / OC_PAGE];
+          for (int ch = 0; ch < d; ++ch) o[ch] += p * (double)vh[(int64_t)j * d + ch];
+          A += p * expm1(dl[j]);
+          B += p * exp(-dl[j]);
+          Ev += p * (double)eta[(int64_t)page * c->hkv + kv];
+          if (dl[j] > dmax) dmax = dl[j];
+        }
+        double range = 0.0;
+        for (int g = 0; g < NG; ++g)
+          if (hi[g] - lo[g] > range) range = hi[g] - lo[g];
+        double tv = tanh(dmax / 2.0);
+        if (A / B < tv) tv = A / B;
+        double ekey = tv * (range + 2.0 * eta_max);
+        double bd = OC_KAPPA * (ekey + Ev);
+        bound[row] = bd;
+        flags[row] = bd > (double)tau ? 1 : 0;
+        if (diag) {
+          double* dg = diag + row * 8;
+          dg[0] = tv; dg[1] = ekey; dg[2] = Ev; dg[3] = dmax;
+          dg[4] = A; dg[5] = B; dg[6] = range; dg[7] = eta_max;
+        }
+      }
+    free(z);
+    free(dl);
+    free(kh);
     free(vh);
   }
   return OC_OK;

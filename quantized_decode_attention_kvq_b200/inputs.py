@@ -48,7 +48,7 @@ PAGE_SIZE = 16
 
 # stream ids (fixed order: Q, K, V, outlier channels, spikes, Hadamard signs,
 # page permutation, context lengths, the KQV codec's QJL projections)
-_S_Q, _S_K, _S_V, _S_OUTLIER, _S_SPIKE, _S_SIGNS, _S_PERM, _S_LEN, _S_QJL = range(9)
+_S_Q, _S_K, _S_V, _S_OUTLIER, _S_SPIKE, _S_SIGNS, _S_PERM, _S_LEN, _S_QJL, _S_HQ = range(10)
 
 _CONFIG_IDS = {"tiny": 1, "llama8b": 2, "long128k": 3, "rotated": 4, "serving": 5}
 
@@ -188,6 +188,14 @@ class Inputs:
         g = _rng(self.seed, self.wl.name, _S_QJL)
         d = self.wl.head_dim
         return g.standard_normal((d, d), dtype=np.float32)
+
+    def hqmq_secondary(self, S: int = 64) -> np.ndarray:
+        """The HQMQ codec's secondary sets: fp32 [Hkv][2 (K, V)][S][4] random
+        unit quaternions (N(0, 1) 4-vectors normalized in fp64, then rounded
+        to fp32)."""
+        g = _rng(self.seed, self.wl.name, _S_HQ)
+        x = g.standard_normal((self.wl.num_kv_heads, 2, S, 4))
+        return (x / np.linalg.norm(x, axis=-1, keepdims=True)).astype(np.float32)
 
     # -- tensors ------------------------------------------------------------
     def _cast(self, x32: np.ndarray) -> np.ndarray:
