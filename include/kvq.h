@@ -15,7 +15,9 @@
  *     bound exceeds tau is recomputed as exact dense attention from Tier 2.
  * and the rotated-key codec of "Statistical Inference and Quality Measures of
  * KV Cache Quantisations Inspired by TurboQuant" (Quantisation schemes, KQV:
- * Walsh-Hadamard transform before scalar quantization of K).
+ * Walsh-Hadamard transform before scalar quantization of K), and two codecs of
+ * their own: that page's KQV codec and the quaternion codec of "Hurwitz
+ * Quaternion Multiplicative Quantization for KV Cache Compression" (HQMQ).
  *
  * Conventions
  *   - Every pointer is caller-owned; the library never allocates or frees
@@ -123,13 +125,20 @@ typedef struct kvq_cache {
   const int8_t* rot_signs; /* device, head_dim entries of +1/-1; required iff k_rotate */
   int32_t* error_word;     /* device, one int32 kernels set to a kvq_status on error; may be NULL */
   int32_t outliers;        /* 1: outlier extraction (see the layout above); 0: none */
-  int32_t codec;           /* KVQ_CODEC_INT (0: the layout above) or KVQ_CODEC_KQV (1) */
+  int32_t codec;           /* KVQ_CODEC_INT (0: the layout above), KVQ_CODEC_KQV (1) or
+                              KVQ_CODEC_HQMQ (2) */
   const float* qjl;        /* device, KVQ_CODEC_KQV: the QJL projections S, fp32
                               [head_dim][head_dim] row-major (row i = projection i) */
+  const float* hq_sec;     /* device, KVQ_CODEC_HQMQ: the secondary unit quaternions,
+                              fp32 [num_kv_heads][2 (K, V)][hq_s][4] */
+  int32_t hq_s;            /* KVQ_CODEC_HQMQ: secondary units per (kv head, role) S,
+                              1..64 */
 } kvq_cache;
 
 #define KVQ_CODEC_INT 0
 #define KVQ_CODEC_KQV 1
+#define KVQ_CODEC_HQMQ 2
+#define KVQ_HQMQ_MAX_S 64
 
 /* The KQV codec ("Statistical Inference and Quality Measures of KV Cache
  * Quantisations Inspired by TurboQuant", Quantisation schemes: KQV), codec =
@@ -156,6 +165,38 @@ typedef struct kvq_cache {
  * kappa*s*(|q'|_1 eps_j + 2^-16 |q'|_2 n_kj) and E_key = TV (max_g range_g +
  * 2 max eta).  kvq_decode_attention_append and kvq_adaptive_precision return
  * KVQ_ERR_UNSUPPORTED for this codec. */
+
+/* The HQMQ codec ("Hurwitz Quaternion Multiplicative Quantization for KV
+ * Cache Compression", Method 1-2), codec = KVQ_CODEC_HQMQ: every 4-channel
+ * chunk x of K and of V is a quaternion split into its radius r = |x| and
+ * its direction, coded by the product codebook {q_p q_s}: q_p one of the 24
+ * Hurwitz units (the binary tetrahedral group 2T: p = 0..7 the units +-1,
+ * +-i, +-j, +-k as p = 2 n + [negative]; p = 8..23 (+-1 +-i +-j +-k)/2 with
+ * component n negative when bit n of p - 8 is set), q_s one of the hq_s
+ * secondary units of the kv head and role (k_bits = v_bits = 6, k_group =
+ * v_group = 4, k_rotate 0, outliers 0):
+ *   code i = 24 s + p maximizing <x, q_p q_s>, evaluated as <x conj(q_s),
+ *   q_p>: y = x conj(q_s) with each component a sequential fmaf chain over
+ *   x0..x3; the best axis unit is max_n |y_n| (first n on ties), the best
+ *   half unit 0.5 (((|y0| + |y1|) + |y2|) + |y3|) with y's signs (-0 as +),
+ *   taken only when strictly larger; a later s only when strictly larger;
+ *   r = sqrt((x0^2 + x1^2) + (x2^2 + x3^2)) (fp32), stored as fp8 E4M3
+ *   (round to nearest even, saturating at 448); codeword c = q_p q_s in fp32
+ *   (exact term products summed left to right); x^ = r^ * c.
+ *   A chunk with a non-finite r gets code 0, radius 0; a token with a
+ *   non-finite value sets KVQ_ERR_RANGE and eps (K) and eta to +inf.
+ * Block of one (page, kv head), 16 tokens, n = head_dim / 4 chunks,
+ * chunk-major (token t of chunk ch at [ch][t]):
+ *   [K codes u16 [n][16]][V codes u16 [n][16]][K radii e4m3 [n][16]]
+ *   [V radii e4m3 [n][16]][|k|_2 f32 [16]][eps f32 [16]]
+ *   [v^ max, min f32 [head_dim/32][2]]
+ * eps = |k - k^|_2 (sequential fmaf chain) raised by 2^-16 of itself, one
+ * ulp up; eta[page][h] = max over the block of (max_c |v_c - v^_c| + 2^-16
+ * |v|_2) one ulp up; the range of each 32-channel group starts at [0, 0] in a
+ * zeroed block.  The decode's bound uses Delta_j = kappa*s*|q|_2 (eps_j +
+ * 2^-16 |k_j|_2) and E_key = TV (max_g range_g + 2 max eta), E_val as for
+ * the other codecs.  kvq_decode_attention_append and kvq_adaptive_precision
+ * return KVQ_ERR_UNSUPPORTED for this codec. */
 
 /* Centroids (2^bits) and decision thresholds (2^bits - 1) of the KQV codec's
  * scalar quantizer for unit vectors in dimension head_dim: the Lloyd-Max
@@ -344,8 +385,8 @@ KVQ_API int kvq_fallback_exact(const kvq_cache* cache, const void* k_orig_host, 
  * buffers).  KVQ_FAULT=memcpy makes the page-in fail (KVQ_ERR_CUDA) for
  * tests.  Blocks the calling thread on the bounded waits.  With outlier
  * extraction the quantized scores, values, Delta and value range include the
- * extracted chunks exactly as kvq_decode_attention does.  A KQV cache returns
- * KVQ_ERR_UNSUPPORTED (and kvq_adaptive_work_size 0). */
+ * extracted chunks exactly as kvq_decode_attention does.  A KQV or HQMQ cache
+ * returns KVQ_ERR_UNSUPPORTED (and kvq_adaptive_work_size 0). */
 KVQ_API size_t kvq_adaptive_work_size(const kvq_cache* cache, int32_t num_seqs,
                                       int32_t num_queries, int32_t num_q_heads,
                                       int32_t max_pages_per_seq);

@@ -1519,7 +1519,9 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
 /*  - r = sqrt((x0^2 + x1^2) + (x2^2 + x3^2)) in fp32 (the Med3x chunk      */
 /*    norm); stored as fp8 E4M3 (round to nearest, ties to even; above 448  */
 /*    it saturates to 448); a chunk with a non-finite norm gets code 0 and  */
-/*    radius 0 and sets the range error;                                    */
+/*    radius 0; a token with a non-finite K or V value sets the range error */
+/*    and gets eps = eta = +inf (K) or eta = +inf (V), so every query over  */
+/*    its block is flagged;                                                  */
 /*  - x^ = r^ * c (fp32 products);                                           */
 /*  - per token: |k|_2 (sequential fmaf chain) and eps = |k - k^|_2 (the    */
 /*    same chain over the channels' differences) raised by 2^-16 of itself, */
@@ -1527,9 +1529,10 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
 /*  - eta_b = the block's largest max_c |v - v^| + 2^-16 |v|_2, one ulp up; */
 /*    the value range per 32-channel group starts at [0, 0] (a zeroed      */
 /*    block) and widens to every v^ appended.                                */
-/* Block of one (page, kv head), 16 tokens, d/4 chunks per vector:          */
-/*   [K codes u16 [16][d/4]][V codes u16 [16][d/4]][K radii e4m3 [16][d/4]]  */
-/*   [V radii e4m3 [16][d/4]][|k| f32 [16]][eps f32 [16]]                    */
+/* Block of one (page, kv head), 16 tokens, d/4 chunks per vector, chunk-   */
+/* major (the 16 tokens of one chunk side by side):                         */
+/*   [K codes u16 [d/4][16]][V codes u16 [d/4][16]][K radii e4m3 [d/4][16]]  */
+/*   [V radii e4m3 [d/4][16]][|k| f32 [16]][eps f32 [16]]                    */
 /*   [v^ max, min f32 [d/32][2]]                                             */
 /* u16 little-endian.                                                        */
 /* ======================================================================== */
@@ -1645,7 +1648,8 @@ static float oh_chunk_radius(const float* x) {
   return sqrtf((a + b) + (e + f));
 }
 
-/* Code one d-vector x: chunk codes and radii, and the fp32 reconstruction. */
+/* Code one d-vector x: chunk codes (u16, chunk ch at idx + 2 * 16 ch) and
+ * radii (at rad + 16 ch), and the fp32 reconstruction. */
 static int oh_code_vector(const float* x, int d, const float* sec, int S, uint8_t* idx,
                           uint8_t* rad, float* xh) {
   int rc = OC_OK;
@@ -1660,8 +1664,8 @@ static int oh_code_vector(const float* x, int d, const float* sec, int S, uint8_
       i = oh_direction(xc, sec, S);
       rq = oh_e4m3_rn(r);
     }
-    oc_wr16(idx + 2 * ch, (uint16_t)i);
-    rad[ch] = rq;
+    oc_wr16(idx + 2 * OC_PAGE * ch, (uint16_t)i);
+    rad[OC_PAGE * ch] = rq;
     float cw[4];
     oh_codeword(sec, i, cw);
     float rv = (float)oh_e4m3_value(rq);
@@ -1682,15 +1686,19 @@ static int oh_quantize_token(const oh_cfg* c, uint8_t* blk, int slot, const floa
                              const float* v, const float* secs, float* eta_out) {
   int d = c->d, nc = d / 4, S = c->S;
   float kh[128], vh[128], e[128];
-  int rc = oh_code_vector(k, d, secs, S, blk + (int64_t)slot * nc * 2,
-                          blk + oh_off_kr(c) + (int64_t)slot * nc, kh);
-  int rv = oh_code_vector(v, d, secs + 4 * S, S, blk + oh_off_vi(c) + (int64_t)slot * nc * 2,
-                          blk + oh_off_vr(c) + (int64_t)slot * nc, vh);
+  int rc = oh_code_vector(k, d, secs, S, blk + 2 * slot, blk + oh_off_kr(c) + slot, kh);
+  int rv = oh_code_vector(v, d, secs + 4 * S, S, blk + oh_off_vi(c) + 2 * slot,
+                          blk + oh_off_vr(c) + slot, vh);
   if (rv != OC_OK) rc = rv;
+  int bad_k = 0, bad_v = 0;
+  for (int i = 0; i < d; ++i) {
+    bad_k |= !isfinite(k[i]);
+    bad_v |= !isfinite(v[i]);
+  }
   float nk = sqrtf(oh_chain_norm2(k, d));
   for (int i = 0; i < d; ++i) e[i] = k[i] - kh[i];
   float en = sqrtf(oh_chain_norm2(e, d));
-  float eps = nextafterf(fmaf(en, 1.0f / 65536.0f, en), INFINITY);
+  float eps = bad_k ? INFINITY : nextafterf(fmaf(en, 1.0f / 65536.0f, en), INFINITY);
   oq_wrf(blk + oh_off_kn(c) + 4 * slot, nk);
   oq_wrf(blk + oh_off_ke(c) + 4 * slot, eps);
   float err = 0.0f;
@@ -1699,7 +1707,7 @@ static int oh_quantize_token(const oh_cfg* c, uint8_t* blk, int slot, const floa
     if (ev > err) err = ev;
   }
   float nv = sqrtf(oh_chain_norm2(v, d));
-  *eta_out = nextafterf(fmaf(1.0f / 65536.0f, nv, err), INFINITY);
+  *eta_out = bad_k || bad_v ? INFINITY : nextafterf(fmaf(1.0f / 65536.0f, nv, err), INFINITY);
   uint8_t* rg = blk + oh_off_rg(c);
   for (int g = 0; g < d / 32; ++g) {
     float hi = oq_rdf(rg + 8 * g), lo = oq_rdf(rg + 8 * g + 4);
@@ -1755,13 +1763,13 @@ void oh_read_token(const oh_cfg* c, const uint8_t* blk, int slot, const float* s
                    float* vh) {
   int nc = c->d / 4;
   for (int role = 0; role < 2; ++role) {
-    const uint8_t* idx = blk + (role ? oh_off_vi(c) : 0) + (int64_t)slot * nc * 2;
-    const uint8_t* rad = blk + (role ? oh_off_vr(c) : oh_off_kr(c)) + (int64_t)slot * nc;
+    const uint8_t* idx = blk + (role ? oh_off_vi(c) : 0) + 2 * slot;
+    const uint8_t* rad = blk + (role ? oh_off_vr(c) : oh_off_kr(c)) + slot;
     float* out = role ? vh : kh;
     for (int ch = 0; ch < nc; ++ch) {
       float cw[4];
-      oh_codeword(secs + role * 4 * c->S, oc_rd16(idx + 2 * ch), cw);
-      float rv = (float)oh_e4m3_value(rad[ch]);
+      oh_codeword(secs + role * 4 * c->S, oc_rd16(idx + 2 * OC_PAGE * ch), cw);
+      float rv = (float)oh_e4m3_value(rad[OC_PAGE * ch]);
       for (int n = 0; n < 4; ++n) out[4 * ch + n] = rv * cw[n];
     }
   }

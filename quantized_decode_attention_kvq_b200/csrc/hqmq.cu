@@ -1,0 +1,767 @@
+// hqmq.cu -- the HQMQ codec of "Hurwitz Quaternion Multiplicative Quantization
+// for KV Cache Compression" (Method 1-2): every 4-channel chunk of K and V is
+// a quaternion split into its radius and its direction on S^3; the direction
+// is coded by the product codebook {q_p q_s} of the 24 Hurwitz units (the
+// binary tetrahedral group 2T) and a random secondary set per (kv head, role),
+// the radius in fp8 E4M3.  The certified bound of "Runtime-Certified
+// Bounded-Error Quantized Attention" (Methodology 2) carries over with a
+// per-token Euclidean key error.
+//
+//   hqmq_append_kernel    one warp per (token, kv head): each lane codes one
+//                         (chunk, role) pair at a time (the direction through
+//                         y = x conj(q_s) and 2T's closed-form best unit, the
+//                         radius by the fp8 conversion), then |k|, eps and
+//                         |v| as sequential chains over the channels, eta and
+//                         the value range
+//   hqmq_partial_kernel   grid (sequence x kv head, split), 4 warps, each
+//                         streaming its pages through a 2-stage bulk-copy
+//                         ring; the CTA builds its kv head's 2 x 24 S
+//                         codewords in shared memory first.  Scores with one
+//                         lane per (token, half of the chunks), PV with one
+//                         lane per chunk, online softmax and the bound's sums
+//                         as for the other codecs
+//   hqmq_merge_kernel     per (sequence, kv head): the split records' merge,
+//                         the output, the bound and the flag
+// The arithmetic that decides a code or a stored value (the chunk norm, the
+// direction's inner products, the codeword products, the error chains) is the
+// fixed-order fp32 sequence the codec's definition gives, so codes, radii,
+// norms, eps and eta are bit-identical to a sequential implementation.
+#include <cuda_fp8.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+// ---------------------------------------------------------------- codebook ---
+// unit p of 2T: p = 0..7 the axis units (+-1, +-i, +-j, +-k as 2 n + [negative]),
+// p = 8..23 the half units (component n negative when bit n of p - 8 is set)
+__device__ __forceinline__ void hq_unit(int p, float a[4]) {
+#pragma unroll
+  for (int n = 0; n < 4; ++n)
+    a[n] = p < 8 ? (n == p / 2 ? ((p & 1) ? -1.f : 1.f) : 0.f)
+                 : ((((p - 8) >> n) & 1) ? -0.5f : 0.5f);
+}
+
+// codeword i = 24 s + p: the Hamilton product q_p q_s, each component's four
+// (exact) term products added left to right
+__device__ __forceinline__ float4 hq_codeword(int i, const float4 b) {
+  float a[4];
+  hq_unit(i % 24, a);
+  const float c0 = __fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(a[0], b.x), -__fmul_rn(a[1], b.y)),
+                                       -__fmul_rn(a[2], b.z)), -__fmul_rn(a[3], b.w));
+  const float c1 = __fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(a[0], b.y), __fmul_rn(a[1], b.x)),
+                                       __fmul_rn(a[2], b.w)), -__fmul_rn(a[3], b.z));
+  const float c2 = __fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(a[0], b.z), -__fmul_rn(a[1], b.w)),
+                                       __fmul_rn(a[2], b.x)), __fmul_rn(a[3], b.y));
+  const float c3 = __fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(a[0], b.w), __fmul_rn(a[1], b.z)),
+                                       -__fmul_rn(a[2], b.y)), __fmul_rn(a[3], b.x));
+  return make_float4(c0, c1, c2, c3);
+}
+
+// The direction code of chunk x: for each secondary unit q_s, y = x conj(q_s)
+// (each component a sequential fmaf chain over x0..x3); the best axis unit
+// gives max_n |y_n| (the first n on ties), the best half unit
+// 0.5 (((|y0| + |y1|) + |y2|) + |y3|) with y's signs, taken only when strictly
+// larger; a later s wins only when strictly larger.
+__device__ __forceinline__ int hq_direction(const float x[4], const float4* sec, int S) {
+  int best = 0;
+  float bv = -INFINITY;
+  for (int s = 0; s < S; ++s) {
+    const float4 b = __ldg(sec + s);
+    const float y0 = __fmaf_rn(x[3], b.w, __fmaf_rn(x[2], b.z, __fmaf_rn(x[1], b.y, __fmul_rn(x[0], b.x))));
+    const float y1 = __fmaf_rn(x[3], b.z, __fmaf_rn(-x[2], b.w, __fmaf_rn(x[1], b.x, __fmul_rn(-x[0], b.y))));
+    const float y2 = __fmaf_rn(-x[3], b.y, __fmaf_rn(x[2], b.x, __fmaf_rn(x[1], b.w, __fmul_rn(-x[0], b.z))));
+    const float y3 = __fmaf_rn(x[3], b.x, __fmaf_rn(x[2], b.y, __fmaf_rn(-x[1], b.z, __fmul_rn(-x[0], b.w))));
+    const float a0 = fabsf(y0), a1 = fabsf(y1), a2 = fabsf(y2), a3 = fabsf(y3);
+    int n0 = 0;
+    float v = a0, yn = y0;
+    if (a1 > v) { n0 = 1; v = a1; yn = y1; }
+    if (a2 > v) { n0 = 2; v = a2; yn = y2; }
+    if (a3 > v) { n0 = 3; v = a3; yn = y3; }
+    int p = 2 * n0 + (yn < 0.f ? 1 : 0);
+    const float h = __fmul_rn(0.5f, __fadd_rn(__fadd_rn(__fadd_rn(a0, a1), a2), a3));
+    if (h > v) {
+      v = h;
+      p = 8 + (y0 < 0.f ? 1 : 0) + (y1 < 0.f ? 2 : 0) + (y2 < 0.f ? 4 : 0) + (y3 < 0.f ? 8 : 0);
+    }
+    if (v > bv) {
+      bv = v;
+      best = 24 * s + p;
+    }
+  }
+  return best;
+}
+
+// fp8 E4M3: round to nearest even, saturating at 448; and back (exact)
+__device__ __forceinline__ uint32_t e4m3_rn(float r) {
+  return (uint32_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+}  // namespace
+
+// ================================================================ append =====
+// One warp per (token, kv head), 8 warps per CTA looping over the items.  Lane
+// l codes (chunk l, K) then (chunk l, V) at d = 128, or (chunk l % 16, role
+// l / 16) at d = 64.
+constexpr int kHqAppendWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const HqAppendArgs ha) {
+  constexpr int NC = D / 4;
+  constexpr int CPL = 2 * NC / 32;   // (chunk, role) pairs per lane
+  constexpr int GL = 8;              // lanes per 32-channel group of V chunks
+  const AppendArgs& a = ha.a;
+  const HqLayout L{D};
+  const int S = ha.S;
+  __shared__ float stg[kHqAppendWarps][3][D];   // per warp: k, k - k^, v
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  float* xk = stg[w][0];
+  float* ek = stg[w][1];
+  float* xv = stg[w][2];
+  const int64_t total = (int64_t)a.num_seqs * a.num_tokens * a.hkv;
+  for (int64_t item = (int64_t)blockIdx.x * kHqAppendWarps + w; item < total;
+       item += (int64_t)gridDim.x * kHqAppendWarps) {
+    const int h = (int)(item % a.hkv);
+    const int t = (int)((item / a.hkv) % a.num_tokens);
+    const int s = (int)(item / ((int64_t)a.hkv * a.num_tokens));
+    if (a.valid && t >= a.valid[s]) continue;
+    const int pos = a.start_pos[s] + t;
+    const int lp = pos / kPage;
+    if (pos < 0 || lp >= a.max_pages) {
+      if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+      continue;
+    }
+    const int page = a.page_table[(int64_t)s * a.max_pages + lp];
+    if (page < 0 || page >= a.num_pages) {
+      if (lane == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+      continue;
+    }
+    const int slot = pos % kPage;
+    const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
+    uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
+    const float4* secs = reinterpret_cast<const float4*>(ha.sec) + (int64_t)h * 2 * S;
+    __syncwarp();   // the previous item's chains have read the staging rows
+    bool bad_k = false, bad_v = false, bad_r = false;
+    float err = 0.f, hi = 0.f, lo = 0.f;
+#pragma unroll
+    for (int u = 0; u < CPL; ++u) {
+      const int role = CPL == 2 ? u : lane / 16;
+      const int ch = CPL == 2 ? lane : lane % 16;
+      float x[4];
+#pragma unroll
+      for (int n = 0; n < 4; ++n) x[n] = load_elem(role ? a.v : a.k, a.in_bf16, base + 4 * ch + n);
+      bool fin = true;
+#pragma unroll
+      for (int n = 0; n < 4; ++n) fin = fin && isfinite(x[n]);
+      const float r = __fsqrt_rn(__fadd_rn(__fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[1], x[1])),
+                                           __fadd_rn(__fmul_rn(x[2], x[2]), __fmul_rn(x[3], x[3]))));
+      int code = 0;
+      uint32_t rq = 0;
+      if (isfinite(r)) {
+        code = hq_direction(x, secs + role * S, S);
+        rq = e4m3_rn(r);
+      } else {
+        bad_r = true;
+      }
+      reinterpret_cast<uint16_t*>(blk + (role ? L.vi() : 0))[kPage * ch + slot] = (uint16_t)code;
+      blk[(role ? L.vr() : L.kr()) + kPage * ch + slot] = (uint8_t)rq;
+      const float4 cw = hq_codeword(code, __ldg(secs + role * S + code / 24));
+      const float rv = e4m3_value(rq);
+      const float xh[4] = {__fmul_rn(rv, cw.x), __fmul_rn(rv, cw.y), __fmul_rn(rv, cw.z),
+                           __fmul_rn(rv, cw.w)};
+      if (role == 0) {
+        bad_k = bad_k || !fin;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          xk[4 * ch + n] = x[n];
+          ek[4 * ch + n] = __fsub_rn(x[n], xh[n]);
+        }
+      } else {
+        bad_v = bad_v || !fin;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          xv[4 * ch + n] = x[n];
+          err = fmaxf(err, fabsf(__fsub_rn(x[n], xh[n])));
+          hi = fmaxf(hi, xh[n]);
+          lo = fminf(lo, xh[n]);
+        }
+      }
+    }
+    bad_k = __any_sync(0xffffffffu, bad_k);
+    bad_v = __any_sync(0xffffffffu, bad_v);
+    bad_r = __any_sync(0xffffffffu, bad_r);
+#pragma unroll
+    for (int o = 1; o < 32; o *= 2) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, o));
+#pragma unroll
+    for (int o = 1; o < GL; o *= 2) {
+      hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+      lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    }
+    __syncwarp();
+    // |k|, |k - k^| and |v|: sequential chains over the channels
+    float nk2 = 0.f, e2 = 0.f, nv2 = 0.f;
+    for (int c = 0; c < D; ++c) {
+      nk2 = __fmaf_rn(xk[c], xk[c], nk2);
+      e2 = __fmaf_rn(ek[c], ek[c], e2);
+      nv2 = __fmaf_rn(xv[c], xv[c], nv2);
+    }
+    if (lane == 0) {
+      if (bad_k || bad_v || bad_r) set_error(a.err, KVQ_ERR_RANGE);
+      const float en = __fsqrt_rn(e2);
+      reinterpret_cast<float*>(blk + L.kn())[slot] = __fsqrt_rn(nk2);
+      reinterpret_cast<float*>(blk + L.ke())[slot] =
+          bad_k ? INFINITY : nextafterf(__fmaf_rn(en, 0x1p-16f, en), INFINITY);
+      const float eu = bad_k || bad_v ? INFINITY
+                                      : nextafterf(__fmaf_rn(0x1p-16f, __fsqrt_rn(nv2), err), INFINITY);
+      atomicMax(reinterpret_cast<int*>(a.eta + (int64_t)page * a.hkv + h), __float_as_int(eu));
+    }
+    // the V chunks' 32-channel groups: lanes 8 g .. 8 g + 7 (d 128), or
+    // 16 + 8 g .. (d 64); the block's range starts at [0, 0]
+    const int vlane = CPL == 2 ? lane : lane - 16;
+    if (vlane >= 0 && vlane % GL == 0) {
+      float* rg = reinterpret_cast<float*>(blk + L.rg()) + 2 * (vlane / GL);
+      if (hi > 0.f) atomicMax(reinterpret_cast<int*>(rg), __float_as_int(hi));
+      if (lo < 0.f) atomicMax(reinterpret_cast<unsigned int*>(rg + 1), __float_as_uint(lo));
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_hqmq_append_d(const HqAppendArgs& a, cudaStream_t stream) {
+  static std::mutex mu;
+  static std::map<int, int> sms_of;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = sms_of.find(dev);
+    if (it == sms_of.end()) {
+      if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+      it = sms_of.emplace(dev, sms).first;
+    }
+    sms = it->second;
+  }
+  const int64_t items = (int64_t)a.a.num_seqs * a.a.num_tokens * a.a.hkv;
+  const int64_t blocks = std::min<int64_t>((items + kHqAppendWarps - 1) / kHqAppendWarps, 4 * sms);
+  hqmq_append_kernel<D><<<(unsigned)blocks, kHqAppendWarps * 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hqmq_append(const HqAppendArgs& a, int d, cudaStream_t stream) {
+  const int64_t items = (int64_t)a.a.num_seqs * a.a.num_tokens * a.a.hkv;
+  if (items == 0) return cudaSuccess;
+  if (d == 128) return launch_hqmq_append_d<128>(a, stream);
+  if (d == 64) return launch_hqmq_append_d<64>(a, stream);
+  return cudaErrorInvalidValue;
+}
+
+// ================================================================ decode =====
+constexpr int kHqWarps = 4;
+constexpr int kHqRows = 4;
+constexpr int kHqStages = 2;
+constexpr int kHqHdr = 16;   // floats: range max [NB], range min [NB], eta max
+__host__ __device__ constexpr int hq_rec_floats(int d) { return kHqHdr + kHqRows * 8 + kHqRows * d; }
+
+template <int D>
+struct HqCfg {
+  static constexpr int NC = D / 4;
+  static constexpr int BLOCK = 24 * D + 8 * kPage + D / 4;                  // HqLayout{D}.bytes()
+  static constexpr int OFF_ST = 0;                                          // [warp][stage][BLOCK]
+  static constexpr int OFF_W = OFF_ST + kHqWarps * kHqStages * BLOCK;       // [warp][16][4] f32
+  static constexpr int OFF_Q = OFF_W + kHqWarps * kPage * kHqRows * 4;      // q [chunk][row] float4
+  static constexpr int OFF_QN = OFF_Q + NC * kHqRows * 16;                  // |q|_2 [4]
+  static constexpr int OFF_BAR = (OFF_QN + 16 + 15) / 16 * 16;              // [warp][stage] u64
+  static constexpr int OFF_PG = OFF_BAR + kHqWarps * kHqStages * 8;         // [warp][stage] i32
+  static constexpr int OFF_TAB = (OFF_PG + kHqWarps * kHqStages * 4 + 15) / 16 * 16;  // [2][24 S] float4
+  // merge of the CTA's warps (aliases the stages): per warp [4][D], [4][8], header
+  static constexpr int MW = kHqRows * D + kHqRows * 8 + kHqHdr;
+  static constexpr int MERGE = kHqWarps * MW * 4;
+  static_assert(MERGE <= OFF_W, "the merge area must stay inside the stages");
+  static_assert(BLOCK % 16 == 0, "bulk copies move multiples of 16 bytes");
+  static __host__ __device__ constexpr int smem(int S) { return 128 + OFF_TAB + 2 * 24 * S * 16; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const HqDecodeArgs ha) {
+  using C = HqCfg<D>;
+  constexpr int NC = C::NC, NB = D / 32, E = D / 32;
+  constexpr int HC = NC / 2;          // chunks per half-warp in the scores
+  constexpr int TPL = 16 * NC / 32;   // tokens per lane in PV
+  const DecodeArgs& a = ha.a;
+  const HqLayout L{D};
+  const int S = ha.S;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
+  const int split = blockIdx.y, kvh = blockIdx.x % a.hkv, b = blockIdx.x / a.hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR) + warp * kHqStages;
+  int* spage = reinterpret_cast<int*>(sm + C::OFF_PG) + warp * kHqStages;
+  if (lane == 0) {
+    for (int s = 0; s < kHqStages; ++s) mbar_init(&bar[s], 1);
+    mbar_fence_init();
+  }
+  int n = a.seq_lens[b];
+  if (n < 0) n = 0;
+  const bool clamped = n > a.max_pages * kPage;
+  if (clamped) {
+    if (tid == 0) set_error(a.err, KVQ_ERR_INVALID_ARG);
+    n = a.max_pages * kPage;
+  }
+  const int npages = (n + kPage - 1) / kPage;
+  const int p0 = split * a.pps;
+  if (p0 >= npages) return;   // inactive split (the merge reads active splits only)
+  const int p1 = min(npages, p0 + a.pps);
+
+  // ---- pages of this warp: p0 + warp, p0 + warp + 4, ...; the first copies
+  // go out before the tables are built ----
+  const int first = p0 + warp;
+  const int nloc = first < p1 ? (p1 - first + kHqWarps - 1) / kHqWarps : 0;
+  uint8_t* stage0 = sm + C::OFF_ST + warp * kHqStages * C::BLOCK;
+  const int32_t* ptab = a.page_table + (int64_t)b * a.max_pages;
+  int pt_chunk = -1, pt_val = -1;
+  auto issue = [&](int j, int st) {
+    if ((j >> 5) != pt_chunk) {
+      pt_chunk = j >> 5;
+      const int jl = 32 * pt_chunk + lane;
+      pt_val = jl < nloc ? __ldg(ptab + first + jl * kHqWarps) : -1;
+    }
+    const int pgv = __shfl_sync(0xffffffffu, pt_val, j & 31);
+    if (lane == 0) {
+      const bool ok = pgv >= 0 && pgv < a.num_pages;
+      spage[st] = ok ? pgv : -1;
+      if (ok) {
+        mbar_arrive_expect_tx(&bar[st], C::BLOCK);
+        bulk_g2s_hint(stage0 + st * C::BLOCK, a.pool + ((int64_t)pgv * a.hkv + kvh) * C::BLOCK,
+                      C::BLOCK, &bar[st], l2_evict_first_policy());
+      } else {
+        set_error(a.err, KVQ_ERR_INVALID_ARG);
+        mbar_arrive(&bar[st]);
+      }
+    }
+    __syncwarp();
+  };
+  __syncwarp();   // the barriers are initialized
+  for (int j = 0; j < kHqStages && j < nloc; ++j) issue(j, j);
+
+  // ---- the kv head's codewords, K then V: [2][24 S] ----
+  float4* tab = reinterpret_cast<float4*>(sm + C::OFF_TAB);
+  {
+    const float4* secs = reinterpret_cast<const float4*>(ha.sec) + (int64_t)kvh * 2 * S;
+    for (int i = tid; i < 48 * S; i += blockDim.x) {
+      const int role = i / (24 * S), ci = i - role * 24 * S;
+      tab[i] = hq_codeword(ci, __ldg(secs + role * S + ci / 24));
+    }
+  }
+  // ---- query rows (warp r = row r): q [chunk][row] as float4, |q|_2 ----
+  float4* qs = reinterpret_cast<float4*>(sm + C::OFF_Q);
+  float* qn = reinterpret_cast<float*>(sm + C::OFF_QN);
+  {
+    const int r = warp;
+    float x[E];
+    if (r < a.R) {
+      const int qi = r / a.G, hq = kvh * a.G + r % a.G;
+      const int64_t e0 = (((int64_t)b * a.nq + qi) * a.hq + hq) * D + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = load_elem(a.q, a.q_bf16, e0 + e);
+    } else {
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = 0.f;
+    }
+    float l2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int c = lane * E + e;
+      reinterpret_cast<float*>(qs + (c / 4) * kHqRows + r)[c % 4] = x[e];
+      l2 = fmaf(x[e], x[e], l2);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o *= 2) l2 += __shfl_xor_sync(0xffffffffu, l2, o);
+    if (lane == 0) qn[r] = sqrtf(l2);
+  }
+  __syncthreads();
+  const float4* tabK = tab;
+  const float4* tabV = tab + 24 * S;
+  // a code beyond the table (only a pool not written by this codec holds one)
+  // reads the last codeword instead of memory past the table
+  const int ncw = 24 * S;
+  // scores: lane (token t, chunk half hc) takes rows r0 = 2 hc, r0 + 1 after
+  // the halves are combined
+  const int t = lane & 15, hc = lane >> 4, r0 = 2 * hc;
+  float cq1[2], cq2[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    cq1[k] = kKappa * a.s_att * qn[r0 + k];
+    cq2[k] = kKappa * a.s_att * kRotSlack * qn[r0 + k];
+  }
+  const float zsc = a.s_att * kLog2e;
+  // PV: lane owns chunk pc for tokens t0 .. t0 + TPL - 1
+  const int pc = lane % NC, t0 = (lane / NC) * TPL;
+
+  float acc[kHqRows][4];
+#pragma unroll
+  for (int r = 0; r < kHqRows; ++r)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[r][e] = 0.f;
+  float m2[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f}, Asum[2] = {0.f, 0.f},
+        Bsum[2] = {0.f, 0.f}, Esum[2] = {0.f, 0.f}, dmax[2] = {0.f, 0.f};
+  float rhi[NB], rlo[NB], etamax = clamped ? INFINITY : 0.f;
+#pragma unroll
+  for (int g = 0; g < NB; ++g) {
+    rhi[g] = -INFINITY;
+    rlo[g] = INFINITY;
+  }
+  float* wts = reinterpret_cast<float*>(sm + C::OFF_W) + warp * kPage * kHqRows;
+  int jstop = nloc;
+  for (int j = 0; j < nloc; ++j) {
+    const int st = j % kHqStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar[st], (uint32_t)((j / kHqStages) & 1)))) {
+      if (lane == 0) set_error(a.err, KVQ_ERR_TIMEOUT);
+      etamax = INFINITY;
+      jstop = j;
+      break;
+    }
+    const int pg = spage[st];
+    if (pg < 0) {
+      etamax = INFINITY;   // the page was not read
+    } else {
+      const uint8_t* blk = stage0 + st * C::BLOCK;
+      const float* fk = reinterpret_cast<const float*>(blk + L.kn());
+      const float* fe = reinterpret_cast<const float*>(blk + L.ke());
+      const float* frg = reinterpret_cast<const float*>(blk + L.rg());
+      const int nval = min(kPage, n - (first + j * kHqWarps) * kPage);
+      const float eta_pg = __ldg(a.eta + (int64_t)pg * a.hkv + kvh);
+      etamax = fmaxf(etamax, eta_pg);
+#pragma unroll
+      for (int g = 0; g < NB; ++g) {
+        rhi[g] = fmaxf(rhi[g], frg[2 * g]);
+        rlo[g] = fminf(rlo[g], frg[2 * g + 1]);
+      }
+      // ---- scores: q . k^ of token t over half hc of the chunks (the upper
+      // half starts one chunk later, so the two halves' loads fall in
+      // different banks) ----
+      float s4[kHqRows] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const uint16_t* kidx = reinterpret_cast<const uint16_t*>(blk);
+        const uint8_t* krad = blk + L.kr();
+#pragma unroll 4
+        for (int cc = 0; cc < HC; ++cc) {
+          const int c = hc ? HC + (cc + 1) % HC : cc;
+          const int idx = min((int)kidx[kPage * c + t], ncw - 1);
+          const float rv = e4m3_value(krad[kPage * c + t]);
+          const float4 cw = tabK[idx];
+          const float k0 = __fmul_rn(rv, cw.x), k1 = __fmul_rn(rv, cw.y);
+          const float k2 = __fmul_rn(rv, cw.z), k3 = __fmul_rn(rv, cw.w);
+#pragma unroll
+          for (int r = 0; r < kHqRows; ++r) {
+            const float4 qv = qs[c * kHqRows + r];
+            s4[r] = fmaf(qv.w, k3, fmaf(qv.z, k2, fmaf(qv.y, k1, fmaf(qv.x, k0, s4[r]))));
+          }
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kHqRows; ++r) s4[r] += __shfl_xor_sync(0xffffffffu, s4[r], 16);
+      const bool vt = t < nval;
+      float zt[2], dl[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float sk = hc ? s4[2 + k] : s4[k];
+        zt[k] = vt ? sk * zsc : -INFINITY;
+        dl[k] = vt ? fmaf(cq1[k], fe[t], cq2[k] * fk[t]) : 0.f;
+      }
+      // ---- online softmax and the bound's sums, rows r0 + k ----
+      float alpha[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        float mx = zt[k];
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        const float mref = mx > m2[k] + 2.0f ? mx : m2[k];
+        alpha[k] = ex2(m2[k] - mref);
+        m2[k] = mref;
+        const float wv = ex2(zt[k] - mref);
+        const float d = dl[k];
+        const float ed = ex2(d * kLog2e), en = ex2(-d * kLog2e);
+        const float em = d < 0.015625f ? d * fmaf(d, fmaf(d, 1.0f / 6, 0.5f), 1.0f) : ed - 1.0f;
+        lsum[k] = fmaf(lsum[k], alpha[k], wv);
+        Asum[k] = fmaf(Asum[k], alpha[k], wv * em);
+        Bsum[k] = fmaf(Bsum[k], alpha[k], wv * en);
+        Esum[k] = fmaf(Esum[k], alpha[k], wv * eta_pg);
+        dmax[k] = fmaxf(dmax[k], d);
+        wts[t * 4 + r0 + k] = wv;   // 0 outside the context
+      }
+      if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
+#pragma unroll
+        for (int r = 0; r < kHqRows; ++r) {
+          // row r's factor sits in the lanes of half r / 2, slot r % 2
+          const float ar = __shfl_sync(0xffffffffu, alpha[r & 1], 16 * (r >> 1));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[r][e] *= ar;
+        }
+      }
+      __syncwarp();
+      // ---- PV: chunk pc of tokens t0 .. t0 + TPL - 1 ----
+      {
+        const uint16_t* vidx = reinterpret_cast<const uint16_t*>(blk + L.vi()) + kPage * pc + t0;
+        const uint8_t* vrad = blk + L.vr() + kPage * pc + t0;
+        uint32_t iw[TPL / 2], rw[TPL / 4];
+#pragma unroll
+        for (int i = 0; i < TPL / 8; ++i) {
+          const uint4 v4 = reinterpret_cast<const uint4*>(vidx)[i];
+          iw[4 * i] = v4.x;
+          iw[4 * i + 1] = v4.y;
+          iw[4 * i + 2] = v4.z;
+          iw[4 * i + 3] = v4.w;
+        }
+        if constexpr (TPL == 16) {
+          const uint4 r4 = *reinterpret_cast<const uint4*>(vrad);
+          rw[0] = r4.x;
+          rw[1] = r4.y;
+          rw[2] = r4.z;
+          rw[3] = r4.w;
+        } else {
+          const uint2 r2 = *reinterpret_cast<const uint2*>(vrad);
+          rw[0] = r2.x;
+          rw[1] = r2.y;
+        }
+        const float4* w4p = reinterpret_cast<const float4*>(wts) + t0;
+#pragma unroll
+        for (int tt = 0; tt < TPL; ++tt) {
+          const int idx = min((int)((iw[tt / 2] >> (16 * (tt & 1))) & 0xFFFFu), ncw - 1);
+          const float rv = e4m3_value((rw[tt / 4] >> (8 * (tt & 3))) & 0xFFu);
+          const float4 cw = tabV[idx];
+          const float v0 = __fmul_rn(rv, cw.x), v1 = __fmul_rn(rv, cw.y);
+          const float v2 = __fmul_rn(rv, cw.z), v3 = __fmul_rn(rv, cw.w);
+          const float4 w4 = w4p[tt];
+          const float wr[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int r = 0; r < kHqRows; ++r) {
+            acc[r][0] = fmaf(wr[r], v0, acc[r][0]);
+            acc[r][1] = fmaf(wr[r], v1, acc[r][1]);
+            acc[r][2] = fmaf(wr[r], v2, acc[r][2]);
+            acc[r][3] = fmaf(wr[r], v3, acc[r][3]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (j + kHqStages < nloc) issue(j + kHqStages, st);
+  }
+  // after a wait that ran out, the copies still in flight are waited for
+  // (bounded) before the stages become the merge area
+  if (jstop < nloc)
+    for (int j = jstop; j < nloc && j < jstop + kHqStages; ++j)
+      (void)mbar_wait(&bar[j % kHqStages], (uint32_t)((j / kHqStages) & 1));
+
+  // ---- per-warp sums: the rows' lanes (one half-warp each); at d = 64 the
+  // two token halves of each chunk ----
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+#pragma unroll
+    for (int o = 1; o < 16; o *= 2) {
+      lsum[k] += __shfl_xor_sync(0xffffffffu, lsum[k], o);
+      Asum[k] += __shfl_xor_sync(0xffffffffu, Asum[k], o);
+      Bsum[k] += __shfl_xor_sync(0xffffffffu, Bsum[k], o);
+      Esum[k] += __shfl_xor_sync(0xffffffffu, Esum[k], o);
+      dmax[k] = fmaxf(dmax[k], __shfl_xor_sync(0xffffffffu, dmax[k], o));
+    }
+  if constexpr (TPL < 16) {
+#pragma unroll
+    for (int r = 0; r < kHqRows; ++r)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], 16);
+  }
+  __syncthreads();   // every warp is done with its stages
+  float* mw = reinterpret_cast<float*>(sm) + warp * C::MW;
+  if (lane < NC) {
+#pragma unroll
+    for (int r = 0; r < kHqRows; ++r)
+      *reinterpret_cast<float4*>(mw + r * D + 4 * lane) =
+          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+  }
+  if (lane == 0 || lane == 16) {   // the lanes of half hc hold rows 2 hc, 2 hc + 1
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      float* stt = mw + kHqRows * D + (r0 + k) * 8;
+      stt[0] = m2[k];
+      stt[1] = lsum[k];
+      stt[2] = Asum[k];
+      stt[3] = Bsum[k];
+      stt[4] = Esum[k];
+      stt[5] = dmax[k];
+    }
+  }
+  if (lane == 0) {
+    float* hd = mw + kHqRows * D + kHqRows * 8;
+#pragma unroll
+    for (int g = 0; g < NB; ++g) {
+      hd[g] = rhi[g];
+      hd[NB + g] = rlo[g];
+    }
+    hd[2 * NB] = etamax;
+  }
+  __syncthreads();
+  // ---- warp r merges row r of the 4 warps into this split's record ----
+  const int r = warp;
+  const float* smf = reinterpret_cast<const float*>(sm);
+  float* rec = a.part + ((int64_t)blockIdx.x * gridDim.y + split) * hq_rec_floats(D);
+  float mW = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kHqWarps; ++w) mW = fmaxf(mW, smf[w * C::MW + kHqRows * D + r * 8]);
+  float st5[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+  float o1[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) o1[e] = 0.f;
+#pragma unroll
+  for (int w = 0; w < kHqWarps; ++w) {
+    const float* mwp = smf + w * C::MW;
+    const float* stw = mwp + kHqRows * D + r * 8;
+    const float f = stw[0] == -INFINITY ? 0.f : ex2(stw[0] - mW);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) st5[k] = fmaf(f, stw[1 + k], st5[k]);
+    st5[4] = fmaxf(st5[4], stw[5]);
+#pragma unroll
+    for (int e = 0; e < E; ++e) o1[e] = fmaf(f, mwp[r * D + lane * E + e], o1[e]);
+  }
+  if (r == 0 && lane < kHqHdr) {
+    float hv = 0.f;
+    if (lane < 2 * NB + 1) {
+      hv = lane < NB ? -INFINITY : (lane < 2 * NB ? INFINITY : 0.f);
+#pragma unroll
+      for (int w = 0; w < kHqWarps; ++w) {
+        const float x = smf[w * C::MW + kHqRows * D + kHqRows * 8 + lane];
+        hv = lane < NB ? fmaxf(hv, x) : (lane < 2 * NB ? fminf(hv, x) : fmaxf(hv, x));
+      }
+    }
+    rec[lane] = hv;
+  }
+  if (lane == 0) {
+    float* rs = rec + kHqHdr + r * 8;
+    rs[0] = mW;
+#pragma unroll
+    for (int k = 0; k < 5; ++k) rs[1 + k] = st5[k];
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) rec[kHqHdr + kHqRows * 8 + r * D + lane * E + e] = o1[e];
+}
+
+template <int D>
+__global__ void __launch_bounds__(kHqWarps * 32) hqmq_merge_kernel(const HqDecodeArgs ha) {
+  constexpr int E = D / 32, NB = D / 32;
+  constexpr int RF = hq_rec_floats(D);
+  const DecodeArgs& a = ha.a;
+  __shared__ float shd[kHqHdr];
+  const int unit = blockIdx.x, kvh = unit % a.hkv, b = unit / a.hkv;
+  const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n = a.seq_lens[b];
+  if (n < 0) n = 0;
+  if (n > a.max_pages * kPage) n = a.max_pages * kPage;
+  const int npages = (n + kPage - 1) / kPage;
+  const int active = (npages + a.pps - 1) / a.pps;
+  const int qi = r / a.G, hq = kvh * a.G + r % a.G;
+  const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + hq;
+  if (npages == 0) {   // empty context: zero output, zero bound (uniform over the CTA)
+    if (r < a.R) {
+      if (a.out)
+        for (int c = lane; c < D; c += 32) a.out[row * D + c] = 0.f;
+      if (lane == 0) {
+        a.bound[row] = 0.f;
+        a.flags[row] = 0;
+      }
+    }
+    return;
+  }
+  const float* ubase = a.part + (int64_t)unit * ha.nsp * RF;
+  if (r == 0 && lane < 2 * NB + 1) {
+    float hv = lane < NB ? -INFINITY : (lane < 2 * NB ? INFINITY : 0.f);
+    for (int sp = 0; sp < active; ++sp) {
+      const float x = __ldcg(ubase + (int64_t)sp * RF + lane);
+      hv = lane < NB ? fmaxf(hv, x) : (lane < 2 * NB ? fminf(hv, x) : fmaxf(hv, x));
+    }
+    shd[lane] = hv;
+  }
+  __syncthreads();
+  if (r >= a.R) return;
+  float M = -INFINITY, l = 0.f, A = 0.f, Bv = 0.f, Ev = 0.f, dm = 0.f;
+  float o1[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) o1[e] = 0.f;
+  for (int sp = 0; sp < active; ++sp) {
+    const float* rec = ubase + (int64_t)sp * RF;
+    const float* st = rec + kHqHdr + r * 8;
+    const float ms = __ldcg(st);
+    if (ms == -INFINITY) continue;   // a split whose pages were all outside the row's context
+    const float Mn = fmaxf(M, ms);
+    const float fo = M == -INFINITY ? 0.f : ex2(M - Mn);
+    const float fs = ex2(ms - Mn);
+    l = fmaf(l, fo, fs * __ldcg(st + 1));
+    A = fmaf(A, fo, fs * __ldcg(st + 2));
+    Bv = fmaf(Bv, fo, fs * __ldcg(st + 3));
+    Ev = fmaf(Ev, fo, fs * __ldcg(st + 4));
+    dm = fmaxf(dm, __ldcg(st + 5));
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+      o1[e] = fmaf(o1[e], fo, fs * __ldcg(rec + kHqHdr + kHqRows * 8 + r * D + lane * E + e));
+    M = Mn;
+  }
+  const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+  if (a.out) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) a.out[row * D + lane * E + e] = o1[e] * inv_l;
+  }
+  if (lane == 0) {
+    const bool skipped = shd[2 * NB] == INFINITY;   // a page of the unit was not read
+    float bd = skipped ? INFINITY : 0.f;
+    if (!skipped && l > 0.f) {
+      float range = 0.f;
+#pragma unroll
+      for (int g = 0; g < NB; ++g) range = fmaxf(range, shd[g] - shd[NB + g]);
+      const float tv = fminf(tanhf(0.5f * dm), A / Bv);
+      bd = kKappa * (tv * (range + 2.0f * shd[2 * NB]) + Ev / l);
+    }
+    a.bound[row] = bd;
+    a.flags[row] = skipped || bd > a.tau ? 1 : 0;
+  }
+}
+
+const void* hqmq_partial_kernel(int d) {
+  if (d == 128) return reinterpret_cast<const void*>(hqmq_partial_kernel<128>);
+  if (d == 64) return reinterpret_cast<const void*>(hqmq_partial_kernel<64>);
+  return nullptr;
+}
+int hqmq_partial_smem(int d, int S) {
+  return d == 128 ? HqCfg<128>::smem(S) : HqCfg<64>::smem(S);
+}
+int hqmq_record_floats(int d) { return hq_rec_floats(d); }
+int hqmq_threads() { return kHqWarps * 32; }
+
+cudaError_t launch_hqmq_decode(const HqDecodeArgs& a, int d, int units, int splits,
+                               cudaStream_t stream) {
+  if (units == 0) return cudaSuccess;
+  const dim3 grid((unsigned)units, (unsigned)splits, 1);
+  const size_t smem = (size_t)hqmq_partial_smem(d, a.S);
+  if (d == 128) {
+    hqmq_partial_kernel<128><<<grid, kHqWarps * 32, smem, stream>>>(a);
+    hqmq_merge_kernel<128><<<units, kHqWarps * 32, 0, stream>>>(a);
+  } else if (d == 64) {
+    hqmq_partial_kernel<64><<<grid, kHqWarps * 32, smem, stream>>>(a);
+    hqmq_merge_kernel<64><<<units, kHqWarps * 32, 0, stream>>>(a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

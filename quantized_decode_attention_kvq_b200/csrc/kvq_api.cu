@@ -15,6 +15,7 @@
 #include <string>
 #include <thread>
 #include <tuple>
+#include <tuple>
 #include <vector>
 
 #include "kvq_internal.cuh"
@@ -51,15 +52,26 @@ int check_kqv(const kvq_cache* c) {
   return KVQ_OK;
 }
 
+int check_hqmq(const kvq_cache* c) {
+  if (c->k_bits != 6 || c->v_bits != 6 || c->k_group != 4 || c->v_group != 4)
+    return fail(KVQ_ERR_UNSUPPORTED, "the HQMQ codec takes k_bits = v_bits = 6 and groups of 4");
+  if (c->k_rotate != 0) return fail(KVQ_ERR_UNSUPPORTED, "the HQMQ codec does not rotate keys");
+  if (c->outliers != 0) return fail(KVQ_ERR_UNSUPPORTED, "the HQMQ codec has no outlier extraction");
+  if (!c->hq_sec) return fail(KVQ_ERR_INVALID_ARG, "the HQMQ codec needs the secondary units");
+  if (c->hq_s < 1 || c->hq_s > KVQ_HQMQ_MAX_S)
+    return fail(KVQ_ERR_UNSUPPORTED, "hq_s %d unsupported (1..%d)", c->hq_s, KVQ_HQMQ_MAX_S);
+  return KVQ_OK;
+}
+
 int check_cache(const kvq_cache* c) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
   if (c->page_size != KVQ_PAGE_SIZE) return fail(KVQ_ERR_UNSUPPORTED, "page_size must be 16");
   if (c->head_dim != 64 && c->head_dim != 128)
     return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d unsupported (64 or 128)", c->head_dim);
-  if (c->codec != KVQ_CODEC_INT && c->codec != KVQ_CODEC_KQV)
+  if (c->codec != KVQ_CODEC_INT && c->codec != KVQ_CODEC_KQV && c->codec != KVQ_CODEC_HQMQ)
     return fail(KVQ_ERR_INVALID_ARG, "codec %d unknown", c->codec);
-  if (c->codec == KVQ_CODEC_KQV) {
-    if (int rc = check_kqv(c)) return rc;
+  if (c->codec != KVQ_CODEC_INT) {
+    if (int rc = c->codec == KVQ_CODEC_KQV ? check_kqv(c) : check_hqmq(c)) return rc;
     if (c->num_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "num_kv_heads < 1");
     if (c->num_pages < 0) return fail(KVQ_ERR_INVALID_ARG, "num_pages < 0");
     if (!c->pool || !c->v_eta) return fail(KVQ_ERR_INVALID_ARG, "pool or v_eta is NULL");
@@ -186,10 +198,35 @@ int kqv_occupancy(int d, int* occ) {
   return KVQ_OK;
 }
 
+// blocks of the HQMQ codec's partial decode kernel resident per SM (its shared
+// memory grows with the secondary set)
+int hqmq_occupancy(int d, int S, int* occ) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto key = std::make_tuple(dev, d, S);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    const void* k = hqmq_partial_kernel(d);
+    const int smem = hqmq_partial_smem(d, KVQ_HQMQ_MAX_S);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, hqmq_threads(),
+                                                      hqmq_partial_smem(d, S));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    it = cache.emplace(key, n < 1 ? 1 : n).first;
+  }
+  *occ = it->second;
+  return KVQ_OK;
+}
+
 int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
-  const bool kqv = c->codec == KVQ_CODEC_KQV;
+  const bool kqv = c->codec == KVQ_CODEC_KQV, hqmq = c->codec == KVQ_CODEC_HQMQ;
   DecodeVariant v{nullptr, nullptr, 0, 0};
-  if (!kqv) {
+  if (!kqv && !hqmq) {
     v = select_decode_kernel(c->head_dim, c->k_bits, c->k_group, c->outliers);
     if (!v.kernel) return fail(KVQ_ERR_UNSUPPORTED, "no decode kernel for this codec");
   }
@@ -197,7 +234,10 @@ int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
   int rc = device_info(&di, nullptr);
   if (rc) return rc;
   int occ = 1;
-  if ((rc = kqv ? kqv_occupancy(c->head_dim, &occ) : decode_occupancy(v, &occ))) return rc;
+  if ((rc = kqv    ? kqv_occupancy(c->head_dim, &occ)
+            : hqmq ? hqmq_occupancy(c->head_dim, c->hq_s, &occ)
+                   : decode_occupancy(v, &occ)))
+    return rc;
   const int64_t units = (int64_t)num_seqs * c->num_kv_heads;
   const int64_t slots = (int64_t)di.sms * occ;
   int64_t splits = units > 0 ? std::max<int64_t>(1, slots / units) : 1;
@@ -214,7 +254,9 @@ int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
   p->splits = (int)splits;
   p->pps = (int)pps;
   p->counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
-  p->part_bytes = (size_t)units * splits * (kqv ? kqv_record_floats(c->head_dim) : v.record) *
+  p->part_bytes = (size_t)units * splits *
+                  (kqv ? kqv_record_floats(c->head_dim)
+                       : hqmq ? hqmq_record_floats(c->head_dim) : v.record) *
                   sizeof(float);
   return KVQ_OK;
 }
@@ -255,10 +297,11 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
     return fail(KVQ_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", ws_bytes,
                 plan.total());
   if (!aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace not 16-byte aligned");
-  const bool kqv = cache->codec == KVQ_CODEC_KQV;
-  if (kqv && nt) return fail(KVQ_ERR_UNSUPPORTED, "the KQV codec has no fused append");
+  const bool kqv = cache->codec == KVQ_CODEC_KQV, hqmq = cache->codec == KVQ_CODEC_HQMQ;
+  if ((kqv || hqmq) && nt)
+    return fail(KVQ_ERR_UNSUPPORTED, "the %s codec has no fused append", kqv ? "KQV" : "HQMQ");
   DecodeVariant v{nullptr, nullptr, 0, 0};
-  if (!kqv)
+  if (!kqv && !hqmq)
     v = select_decode_kernel(cache->head_dim, cache->k_bits, cache->k_group, cache->outliers);
   DecodeArgs a;
   a.pool = static_cast<const uint8_t*>(cache->pool);
@@ -307,6 +350,16 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
     if (e != cudaSuccess) return cuda_fail(e, "KQV decode launch");
     return KVQ_OK;
   }
+  if (hqmq) {
+    HqDecodeArgs ha;
+    ha.a = a;
+    ha.sec = cache->hq_sec;
+    ha.S = cache->hq_s;
+    ha.nsp = plan.splits;
+    cudaError_t e = launch_hqmq_decode(ha, cache->head_dim, (int)units, plan.splits, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "HQMQ decode launch");
+    return KVQ_OK;
+  }
   dim3 grid((unsigned)units, (unsigned)plan.splits, 1);
   cudaError_t e = launch_pdl(nt ? v.kernel_append : v.kernel, grid, dim3(decode_threads()),
                              (size_t)v.smem, stream, a);
@@ -346,6 +399,12 @@ size_t kvq_block_bytes(const kvq_cache* cache) {
         cache->v_group != cache->head_dim || cache->outliers != 0)
       return 0;
     return (size_t)KqvLayout{cache->head_dim}.bytes();
+  }
+  if (cache->codec == KVQ_CODEC_HQMQ) {
+    if (cache->k_bits != 6 || cache->v_bits != 6 || cache->k_group != 4 || cache->v_group != 4 ||
+        cache->k_rotate != 0 || cache->outliers != 0)
+      return 0;
+    return (size_t)HqLayout{cache->head_dim}.bytes();
   }
   if (cache->codec != KVQ_CODEC_INT || (cache->k_bits != 8 && cache->k_bits != 4)) return 0;
   if (cache->k_group != 32 && cache->k_group != 64 && cache->k_group != 128) return 0;
@@ -405,6 +464,15 @@ int kvq_quantize_append(const kvq_cache* cache, const void* k, const void* v, in
     kqv_tables(cache->head_dim, &ka.t);
     cudaError_t e = launch_kqv_append(ka, cache->head_dim, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "KQV append kernel launch");
+    return KVQ_OK;
+  }
+  if (cache->codec == KVQ_CODEC_HQMQ) {
+    HqAppendArgs ha;
+    ha.a = a;
+    ha.sec = cache->hq_sec;
+    ha.S = cache->hq_s;
+    cudaError_t e = launch_hqmq_append(ha, cache->head_dim, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "HQMQ append kernel launch");
     return KVQ_OK;
   }
   cudaError_t e = launch_append(a, cache->head_dim, cache->k_bits, cache->k_group, cache->outliers,

@@ -206,6 +206,41 @@ int kqv_partial_smem(int d);
 int kqv_record_floats(int d);
 int kqv_threads();
 
+// ---- the HQMQ codec (hqmq.cu) ------------------------------------------------
+// Byte layout of one (page, kv head) block, chunk-major (token t of chunk c at
+// [c][t]): K codes u16, V codes u16, K radii e4m3, V radii e4m3, then per
+// token |k| and eps (fp32), then the block's v^ max / min per 32-channel group.
+struct HqLayout {
+  int d;
+  __host__ __device__ int nc() const { return d / 4; }
+  __host__ __device__ int vi() const { return kPage * nc() * 2; }
+  __host__ __device__ int kr() const { return kPage * nc() * 4; }
+  __host__ __device__ int vr() const { return kr() + kPage * nc(); }
+  __host__ __device__ int kn() const { return vr() + kPage * nc(); }
+  __host__ __device__ int ke() const { return kn() + 4 * kPage; }
+  __host__ __device__ int rg() const { return kn() + 8 * kPage; }
+  __host__ __device__ int bytes() const { return rg() + (d / 32) * 8; }
+};
+struct HqAppendArgs {
+  AppendArgs a;
+  const float* sec;   // [hkv][2][S][4] unit quaternions
+  int S;
+};
+struct HqDecodeArgs {
+  DecodeArgs a;       // out, bound, flags, part as for the Tier-1 decode; no fused append
+  const float* sec;
+  int S;
+  int nsp;            // splits of the partial grid (records per unit)
+};
+cudaError_t launch_hqmq_append(const HqAppendArgs& a, int d, cudaStream_t s);
+// the partial kernel over (unit, split), then the merge per unit
+cudaError_t launch_hqmq_decode(const HqDecodeArgs& a, int d, int units, int splits,
+                               cudaStream_t s);
+const void* hqmq_partial_kernel(int d);
+int hqmq_partial_smem(int d, int S);
+int hqmq_record_floats(int d);
+int hqmq_threads();
+
 cudaError_t launch_append(const AppendArgs& a, int d, int kbits, int kgroup, int out,
                           cudaStream_t s);
 // out: the cache's outlier extraction (0 or 1)

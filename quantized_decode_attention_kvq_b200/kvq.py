@@ -16,6 +16,7 @@ import math
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,6 +33,8 @@ KVQ_F32 = 0
 KVQ_BF16 = 1
 KVQ_CODEC_INT = 0
 KVQ_CODEC_KQV = 1
+KVQ_CODEC_HQMQ = 2
+KVQ_HQMQ_MAX_S = 64
 PAGE_SIZE = 16
 
 EXPORTED = ("kvq_block_bytes", "kvq_pool_bytes", "kvq_quantize_append", "kvq_workspace_size",
@@ -56,7 +59,8 @@ class kvq_cache(ctypes.Structure):
                 ("v_group", ctypes.c_int32), ("pool", ctypes.c_void_p),
                 ("v_eta", ctypes.c_void_p), ("rot_signs", ctypes.c_void_p),
                 ("error_word", ctypes.c_void_p), ("outliers", ctypes.c_int32),
-                ("codec", ctypes.c_int32), ("qjl", ctypes.c_void_p)]
+                ("codec", ctypes.c_int32), ("qjl", ctypes.c_void_p),
+                ("hq_sec", ctypes.c_void_p), ("hq_s", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -289,16 +293,24 @@ class PagedCache:
     def __init__(self, num_kv_heads: int, head_dim: int, num_pages: int, k_bits: int = 8,
                  k_group: int = 128, k_rotate: bool = False, rot_signs=None, v_bits: int = 4,
                  v_group: int = 32, outliers: bool = False, codec: str = "int", qjl_matrix=None,
-                 device="cuda"):
+                 hq_secondary=None, device="cuda"):
         """codec "int": the Tier-1 INT8/INT4 codec (k_bits, k_group, k_rotate,
         outliers apply); codec "kqv": the KQV codec (rotation with rot_signs, 4-bit
-        Lloyd-Max keys, 3-bit values plus the QJL sketch with qjl_matrix [d][d])."""
+        Lloyd-Max keys, 3-bit values plus the QJL sketch with qjl_matrix [d][d]);
+        codec "hqmq": the HQMQ codec (4-channel chunks as quaternions, the product
+        codebook of 2T and the secondary units hq_secondary [Hkv][2][S][4])."""
+        codes = {"int": KVQ_CODEC_INT, "kqv": KVQ_CODEC_KQV, "hqmq": KVQ_CODEC_HQMQ}
+        if codec not in codes:
+            raise ValueError(f"unknown codec {codec!r}")
         if codec == "kqv":
             k_bits, v_bits, k_group, v_group, k_rotate = 4, 3, head_dim, head_dim, True
+        hq_s = 0
+        if codec == "hqmq":
+            k_bits, v_bits, k_group, v_group, k_rotate = 6, 6, 4, 4, False
+            hq_s = int(np.asarray(hq_secondary).shape[2])   # S secondary units per (head, role)
         self.desc = kvq_cache(num_kv_heads, head_dim, PAGE_SIZE, num_pages, k_bits, k_group,
                               int(bool(k_rotate)), v_bits, v_group, None, None, None, None,
-                              int(bool(outliers)),
-                              KVQ_CODEC_KQV if codec == "kqv" else KVQ_CODEC_INT, None)
+                              int(bool(outliers)), codes[codec], None, None, hq_s)
         bb = kvq_block_bytes(self.desc)
         if bb == 0:
             raise KvqError(KVQ_ERR_UNSUPPORTED, "kvq_block_bytes")
@@ -319,6 +331,11 @@ class PagedCache:
         if codec == "kqv":
             self.qjl = torch.as_tensor(qjl_matrix, dtype=torch.float32).to(device).contiguous()
             self.desc.qjl = self.qjl.data_ptr()
+        self.hq_sec = None
+        if codec == "hqmq":
+            self.hq_sec = torch.as_tensor(np.asarray(hq_secondary, np.float32)).to(device).contiguous()
+            assert tuple(self.hq_sec.shape) == (num_kv_heads, 2, hq_s, 4)
+            self.desc.hq_sec = self.hq_sec.data_ptr()
 
     @property
     def head_dim(self) -> int:

@@ -87,6 +87,23 @@ def test_kqv_block_size_and_checks(kvq):
     assert kvq.kvq_adaptive_work_size(d, 2, 1, 32, 4) == 0
 
 
+def test_hqmq_block_size_and_checks(kvq):
+    hq = dict(codec=kvq.KVQ_CODEC_HQMQ, k_bits=6, v_bits=6, k_group=4, v_group=4,
+              hq_sec=0x5000, hq_s=32)
+    # u16 code + e4m3 radius per chunk for K and V (24 d per block), |k| and
+    # eps per token, the range
+    assert kvq.kvq_block_bytes(_desc(kvq, **hq)) == 24 * 128 + 128 + 32 == 3232
+    assert kvq.kvq_block_bytes(_desc(kvq, head_dim=64, **hq)) == 24 * 64 + 128 + 16 == 1680
+    assert kvq.kvq_block_bytes(_desc(kvq, **{**hq, "k_bits": 8})) == 0
+    assert kvq.kvq_block_bytes(_desc(kvq, k_rotate=1, rot_signs=0x3000, **hq)) == 0
+    d = _desc(kvq, **hq)
+    assert kvq.kvq_adaptive_work_size(d, 2, 1, 32, 4) == 0
+    # hq_s beyond the decode's shared-memory tables, or no secondary units
+    assert _decode(kvq, _desc(kvq, **{**hq, "hq_s": 65})) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _decode(kvq, _desc(kvq, **{**hq, "hq_s": 0})) == kvq.KVQ_ERR_UNSUPPORTED
+    assert _decode(kvq, _desc(kvq, **{**hq, "hq_sec": None})) == kvq.KVQ_ERR_INVALID_ARG
+
+
 def test_status_strings(kvq):
     assert kvq.status_string(0) == "KVQ_OK"
     assert kvq.status_string(-5) == "KVQ_ERR_TIMEOUT"

@@ -186,10 +186,10 @@ class _Reader:
 
     def token(self, page, kv, slot):
         nc, blk = self.nc, self.c.pool[(page * self.c.cfg.hkv + kv) * self.bb:][:self.bb]
-        ki = blk[:32 * nc].view(np.uint16).reshape(16, nc)[slot]
-        vi = blk[32 * nc:64 * nc].view(np.uint16).reshape(16, nc)[slot]
-        kr = self.E4[blk[64 * nc:80 * nc].reshape(16, nc)[slot]]
-        vr = self.E4[blk[80 * nc:96 * nc].reshape(16, nc)[slot]]
+        ki = blk[:32 * nc].view(np.uint16).reshape(nc, 16)[:, slot]
+        vi = blk[32 * nc:64 * nc].view(np.uint16).reshape(nc, 16)[:, slot]
+        kr = self.E4[blk[64 * nc:80 * nc].reshape(nc, 16)[:, slot]]
+        vr = self.E4[blk[80 * nc:96 * nc].reshape(nc, 16)[:, slot]]
         f = blk[96 * nc:].view(np.float32)
         kh = (kr[:, None] * self.books[kv][0][ki]).reshape(-1)
         vh = (vr[:, None] * self.books[kv][1][vi]).reshape(-1)
