@@ -71,8 +71,9 @@ __device__ __forceinline__ float4 hq_codeword(int i, const float4 b) {
 __device__ __forceinline__ int hq_direction(const float x[4], const float4* sec, int S) {
   int best = 0;
   float bv = -INFINITY;
+#pragma unroll 4
   for (int s = 0; s < S; ++s) {
-    const float4 b = __ldg(sec + s);
+    const float4 b = sec[s];
     const float y0 = __fmaf_rn(x[3], b.w, __fmaf_rn(x[2], b.z, __fmaf_rn(x[1], b.y, __fmul_rn(x[0], b.x))));
     const float y1 = __fmaf_rn(x[3], b.z, __fmaf_rn(-x[2], b.w, __fmaf_rn(x[1], b.x, __fmul_rn(-x[0], b.y))));
     const float y2 = __fmaf_rn(-x[3], b.y, __fmaf_rn(x[2], b.x, __fmaf_rn(x[1], b.w, __fmul_rn(-x[0], b.z))));
@@ -122,7 +123,8 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
   const AppendArgs& a = ha.a;
   const HqLayout L{D};
   const int S = ha.S;
-  __shared__ float stg[kHqAppendWarps][3][D];   // per warp: k, k - k^, v
+  __shared__ __align__(16) float stg[kHqAppendWarps][3][D];   // per warp: k, k - k^, v
+  __shared__ float4 ssec[kHqAppendWarps][2 * KVQ_HQMQ_MAX_S];  // per warp: the item's units
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   float* xk = stg[w][0];
   float* ek = stg[w][1];
@@ -148,8 +150,13 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
     const int slot = pos % kPage;
     const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
     uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
-    const float4* secs = reinterpret_cast<const float4*>(ha.sec) + (int64_t)h * 2 * S;
-    __syncwarp();   // the previous item's chains have read the staging rows
+    __syncwarp();   // the previous item's chains and searches have read the staging rows
+    {   // the kv head's secondary units, K then V, in one coalesced load
+      const float4* src = reinterpret_cast<const float4*>(ha.sec) + (int64_t)h * 2 * S;
+      for (int i = lane; i < 2 * S; i += 32) ssec[w][i] = __ldg(src + i);
+    }
+    __syncwarp();
+    const float4* secs = ssec[w];
     bool bad_k = false, bad_v = false, bad_r = false;
     float err = 0.f, hi = 0.f, lo = 0.f;
 #pragma unroll
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
       }
       reinterpret_cast<uint16_t*>(blk + (role ? L.vi() : 0))[kPage * ch + slot] = (uint16_t)code;
       blk[(role ? L.vr() : L.kr()) + kPage * ch + slot] = (uint8_t)rq;
-      const float4 cw = hq_codeword(code, __ldg(secs + role * S + code / 24));
+      const float4 cw = hq_codeword(code, secs[role * S + code / 24]);
       const float rv = e4m3_value(rq);
       const float xh[4] = {__fmul_rn(rv, cw.x), __fmul_rn(rv, cw.y), __fmul_rn(rv, cw.z),
                            __fmul_rn(rv, cw.w)};
@@ -209,10 +216,14 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
     __syncwarp();
     // |k|, |k - k^| and |v|: sequential chains over the channels
     float nk2 = 0.f, e2 = 0.f, nv2 = 0.f;
-    for (int c = 0; c < D; ++c) {
-      nk2 = __fmaf_rn(xk[c], xk[c], nk2);
-      e2 = __fmaf_rn(ek[c], ek[c], e2);
-      nv2 = __fmaf_rn(xv[c], xv[c], nv2);
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      const float4 k4 = *reinterpret_cast<const float4*>(xk + c);
+      const float4 e4 = *reinterpret_cast<const float4*>(ek + c);
+      const float4 v4 = *reinterpret_cast<const float4*>(xv + c);
+      nk2 = __fmaf_rn(k4.w, k4.w, __fmaf_rn(k4.z, k4.z, __fmaf_rn(k4.y, k4.y, __fmaf_rn(k4.x, k4.x, nk2))));
+      e2 = __fmaf_rn(e4.w, e4.w, __fmaf_rn(e4.z, e4.z, __fmaf_rn(e4.y, e4.y, __fmaf_rn(e4.x, e4.x, e2))));
+      nv2 = __fmaf_rn(v4.w, v4.w, __fmaf_rn(v4.z, v4.z, __fmaf_rn(v4.y, v4.y, __fmaf_rn(v4.x, v4.x, nv2))));
     }
     if (lane == 0) {
       if (bad_k || bad_v || bad_r) set_error(a.err, KVQ_ERR_RANGE);
@@ -320,7 +331,11 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
   }
   const int npages = (n + kPage - 1) / kPage;
   const int p0 = split * a.pps;
-  if (p0 >= npages) return;   // inactive split (the merge reads active splits only)
+  if (p0 >= npages) {   // a split past the context: an empty record for the merge
+    write_empty_record(a.part + ((int64_t)blockIdx.x * gridDim.y + split) * hq_rec_floats(D), NB,
+                       kHqHdr, kHqRows, kHqRows * D);
+    return;
+  }
   const int p1 = min(npages, p0 + a.pps);
 
   // ---- pages of this warp: p0 + warp, p0 + warp + 4, ...; the first copies
@@ -665,58 +680,37 @@ __global__ void __launch_bounds__(kHqWarps * 32) hqmq_merge_kernel(const HqDecod
   __shared__ float shd[kHqHdr];
   const int unit = blockIdx.x, kvh = unit % a.hkv, b = unit / a.hkv;
   const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int n = a.seq_lens[b];
-  if (n < 0) n = 0;
-  if (n > a.max_pages * kPage) n = a.max_pages * kPage;
-  const int npages = (n + kPage - 1) / kPage;
-  const int active = (npages + a.pps - 1) / a.pps;
-  const int qi = r / a.G, hq = kvh * a.G + r % a.G;
-  const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + hq;
-  if (npages == 0) {   // empty context: zero output, zero bound (uniform over the CTA)
-    if (r < a.R) {
-      if (a.out)
-        for (int c = lane; c < D; c += 32) a.out[row * D + c] = 0.f;
-      if (lane == 0) {
-        a.bound[row] = 0.f;
-        a.flags[row] = 0;
-      }
-    }
-    return;
-  }
-  const float* ubase = a.part + (int64_t)unit * ha.nsp * RF;
-  if (r == 0 && lane < 2 * NB + 1) {
-    float hv = lane < NB ? -INFINITY : (lane < 2 * NB ? INFINITY : 0.f);
-    for (int sp = 0; sp < active; ++sp) {
-      const float x = __ldcg(ubase + (int64_t)sp * RF + lane);
-      hv = lane < NB ? fmaxf(hv, x) : (lane < 2 * NB ? fminf(hv, x) : fmaxf(hv, x));
-    }
-    shd[lane] = hv;
-  }
-  __syncthreads();
-  if (r >= a.R) return;
-  float M = -INFINITY, l = 0.f, A = 0.f, Bv = 0.f, Ev = 0.f, dm = 0.f;
+  // every split wrote a record (an empty one when it held none of the pages),
+  // so neither the context length nor one load after another is needed: warp
+  // 0 merges the header while every warp merges its row's statistics and
+  // outputs
+  const int nsp = ha.nsp;
+  const float* ubase = a.part + (int64_t)unit * nsp * RF;
+  if (r == 0) merge_split_header<NB>(ubase, RF, nsp, lane, shd);
+  const float* st0 = ubase + kHqHdr + r * 8;
+  float m_own;
+  const SplitStats t = merge_split_stats(st0, RF, nsp, lane, &m_own);
   float o1[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) o1[e] = 0.f;
-  for (int sp = 0; sp < active; ++sp) {
-    const float* rec = ubase + (int64_t)sp * RF;
-    const float* st = rec + kHqHdr + r * 8;
-    const float ms = __ldcg(st);
-    if (ms == -INFINITY) continue;   // a split whose pages were all outside the row's context
-    const float Mn = fmaxf(M, ms);
-    const float fo = M == -INFINITY ? 0.f : ex2(M - Mn);
-    const float fs = ex2(ms - Mn);
-    l = fmaf(l, fo, fs * __ldcg(st + 1));
-    A = fmaf(A, fo, fs * __ldcg(st + 2));
-    Bv = fmaf(Bv, fo, fs * __ldcg(st + 3));
-    Ev = fmaf(Ev, fo, fs * __ldcg(st + 4));
-    dm = fmaxf(dm, __ldcg(st + 5));
+  for (int base = 0; base < nsp; base += 32) {
+    const float wl = base == 0 ? (m_own == -INFINITY ? 0.f : ex2(m_own - t.M))
+                               : split_weight(st0, RF, nsp, base, lane, t.M);
+    const int cnt = min(32, nsp - base);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      const float* orow = ubase + (int64_t)(base + k) * RF + kHqHdr + kHqRows * 8 + r * D + lane * E;
 #pragma unroll
-    for (int e = 0; e < E; ++e)
-      o1[e] = fmaf(o1[e], fo, fs * __ldcg(rec + kHqHdr + kHqRows * 8 + r * D + lane * E + e));
-    M = Mn;
+      for (int e = 0; e < E; ++e) o1[e] = fmaf(w, __ldcg(orow + e), o1[e]);
+    }
   }
-  const float inv_l = l > 0.f ? 1.0f / l : 0.f;
+  __syncthreads();   // the header
+  if (r >= a.R) return;
+  const int qi = r / a.G, hq = kvh * a.G + r % a.G;
+  const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + hq;
+  const float l = t.l;
+  const float inv_l = l > 0.f ? 1.0f / l : 0.f;   // l = 0: an empty context, output 0
   if (a.out) {
 #pragma unroll
     for (int e = 0; e < E; ++e) a.out[row * D + lane * E + e] = o1[e] * inv_l;
@@ -728,11 +722,11 @@ __global__ void __launch_bounds__(kHqWarps * 32) hqmq_merge_kernel(const HqDecod
       float range = 0.f;
 #pragma unroll
       for (int g = 0; g < NB; ++g) range = fmaxf(range, shd[g] - shd[NB + g]);
-      const float tv = fminf(tanhf(0.5f * dm), A / Bv);
-      bd = kKappa * (tv * (range + 2.0f * shd[2 * NB]) + Ev / l);
+      const float tv = fminf(tanhf(0.5f * t.dm), t.A / t.B);
+      bd = kKappa * (tv * (range + 2.0f * shd[2 * NB]) + t.E / l);
     }
     a.bound[row] = bd;
-    a.flags[row] = skipped || bd > a.tau ? 1 : 0;
+    a.flags[row] = skipped || (l > 0.f && bd > a.tau) ? 1 : 0;
   }
 }
 

@@ -388,7 +388,11 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
   }
   const int npages = (n + kPage - 1) / kPage;
   const int p0 = split * a.pps;
-  if (p0 >= npages) return;   // inactive split (the merge reads active splits only)
+  if (p0 >= npages) {   // a split past the context: an empty record for the merge
+    write_empty_record(a.part + ((int64_t)blockIdx.x * gridDim.y + split) * kqv_rec_floats(D), NB,
+                       kKqHdr, kKqRows, 2 * kKqRows * D);
+    return;
+  }
   const int p1 = min(npages, p0 + a.pps);
 
   // ---- tables and query rows ----
@@ -773,57 +777,35 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_merge_kernel(const KqvDecod
   __shared__ float shd[kKqHdr];
   const int unit = blockIdx.x, kvh = unit % a.hkv, b = unit / a.hkv;
   const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int n = a.seq_lens[b];
-  if (n < 0) n = 0;
-  if (n > a.max_pages * kPage) n = a.max_pages * kPage;
-  const int npages = (n + kPage - 1) / kPage;
-  const int active = (npages + a.pps - 1) / a.pps;
   const int qi = r / a.G, hq = kvh * a.G + r % a.G;
   const int64_t row = ((int64_t)b * a.nq + qi) * a.hq + hq;
-  if (npages == 0) {   // empty context: zero output, zero bound (uniform over the CTA)
-    if (r < a.R) {
-      if (a.out)
-        for (int c = lane; c < D; c += 32) a.out[row * D + c] = 0.f;
-      if (lane == 0) {
-        a.bound[row] = 0.f;
-        a.flags[row] = 0;
-      }
-    }
-    return;
-  }
-  const float* ubase = a.part + (int64_t)unit * ka.nsp * RF;
-  if (r == 0 && lane < 2 * NB + 1) {
-    float hv = lane < NB ? -INFINITY : (lane < 2 * NB ? INFINITY : 0.f);
-    for (int sp = 0; sp < active; ++sp) {
-      const float x = __ldcg(ubase + (int64_t)sp * RF + lane);
-      hv = lane < NB ? fmaxf(hv, x) : (lane < 2 * NB ? fminf(hv, x) : fmaxf(hv, x));
-    }
-    shd[lane] = hv;
-  }
-  float M = -INFINITY, l = 0.f, A = 0.f, Bv = 0.f, Ev = 0.f, dm = 0.f;
+  // every split wrote a record (an empty one when it held none of the pages):
+  // warp 0 merges the header while every warp merges its row's statistics and
+  // its two accumulations, the records' loads independent of one another
+  const int nsp = ka.nsp;
+  const float* ubase = a.part + (int64_t)unit * nsp * RF;
+  if (r == 0) merge_split_header<NB>(ubase, RF, nsp, lane, shd);
+  const float* st0 = ubase + kKqHdr + r * 8;
+  float m_own;
+  const SplitStats t = merge_split_stats(st0, RF, nsp, lane, &m_own);
+  const float l = t.l, A = t.A, Bv = t.B, Ev = t.E, dm = t.dm;
   float o1[E], o2[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) o1[e] = o2[e] = 0.f;
-  for (int sp = 0; sp < active; ++sp) {
-    const float* rec = ubase + (int64_t)sp * RF;
-    const float* st = rec + kKqHdr + r * 8;
-    const float ms = __ldcg(st);
-    if (ms == -INFINITY) continue;   // a split whose pages were all outside the row's context
-    const float Mn = fmaxf(M, ms);
-    const float fo = M == -INFINITY ? 0.f : ex2(M - Mn);
-    const float fs = ex2(ms - Mn);
-    l = fmaf(l, fo, fs * __ldcg(st + 1));
-    A = fmaf(A, fo, fs * __ldcg(st + 2));
-    Bv = fmaf(Bv, fo, fs * __ldcg(st + 3));
-    Ev = fmaf(Ev, fo, fs * __ldcg(st + 4));
-    dm = fmaxf(dm, __ldcg(st + 5));
+  for (int base = 0; base < nsp; base += 32) {
+    const float wl = base == 0 ? (m_own == -INFINITY ? 0.f : ex2(m_own - t.M))
+                               : split_weight(st0, RF, nsp, base, lane, t.M);
+    const int cnt = min(32, nsp - base);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+      const float w = __shfl_sync(0xffffffffu, wl, k);
+      const float* rec = ubase + (int64_t)(base + k) * RF + kKqHdr + kKqRows * 8 + r * D + lane * E;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int c = lane * E + e;
-      o1[e] = fmaf(o1[e], fo, fs * __ldcg(rec + kKqHdr + kKqRows * 8 + r * D + c));
-      o2[e] = fmaf(o2[e], fo, fs * __ldcg(rec + kKqHdr + kKqRows * 8 + kKqRows * D + r * D + c));
+      for (int e = 0; e < E; ++e) {
+        o1[e] = fmaf(w, __ldcg(rec + e), o1[e]);
+        o2[e] = fmaf(w, __ldcg(rec + kKqRows * D + e), o2[e]);
+      }
     }
-    M = Mn;
   }
   const float inv_l = l > 0.f ? 1.0f / l : 0.f;
 #pragma unroll
@@ -871,7 +853,7 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_merge_kernel(const KqvDecod
       bd = kKappa * (tv * (range + 2.0f * shd[2 * NB]) + Ev / l);
     }
     a.bound[row] = bd;
-    a.flags[row] = skipped || bd > a.tau ? 1 : 0;
+    a.flags[row] = skipped || (l > 0.f && bd > a.tau) ? 1 : 0;   // l = 0: an empty context
   }
 }
 
