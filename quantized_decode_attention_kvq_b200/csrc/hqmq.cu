@@ -33,6 +33,7 @@
 #include <mutex>
 
 #include "kvq_internal.cuh"
+#include "split_merge.cuh"
 
 namespace kvq {
 namespace {

@@ -36,6 +36,7 @@
 #include <mutex>
 
 #include "kvq_internal.cuh"
+#include "split_merge.cuh"
 
 namespace kvq {
 
