@@ -138,3 +138,36 @@ def test_noalloc_on_a_kqv_cache():
     assert g.device_error() == 0
     assert torch.equal(out, out_w.view_as(out)) and torch.equal(bound, bound_w.view_as(bound))
     assert torch.equal(flags, flags_w.view_as(flags))
+
+
+def test_noalloc_on_an_hqmq_cache():
+    """The same entry point over a cache of the HQMQ codec: bit for bit the
+    workspace decode."""
+    from quantized_decode_attention_kvq_b200 import kvq
+    from gpu_cases import to_torch
+    if not torch.cuda.is_available():
+        pytest.fail("the GPU tests need a CUDA device")
+    inp = small("serving", 8)
+    wl = inp.wl
+    k, v = inp.kv()
+    q = inp.q()
+    g = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, codec="hqmq",
+                       hq_secondary=inp.hqmq_secondary(32))
+    pt = torch.from_numpy(inp.page_table).cuda()
+    sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
+    g.append(to_torch(k), to_torch(v), pt, torch.zeros(wl.num_seqs, dtype=torch.int32,
+                                                       device="cuda"), sl)
+    qd = to_torch(q)
+    S, NQ, HQ, d = q.shape
+    ws = g.workspace(S, NQ, HQ, pt.shape[1])
+    out_w, bound_w, flags_w = g.decode(qd, pt, sl, ws, tau=20.0)
+    out, bound, flags = _buffers(inp)
+    out.fill_(float("nan"))
+    qdt = kvq.KVQ_BF16 if qd.dtype == torch.bfloat16 else kvq.KVQ_F32
+    rc = kvq.kvq_decode_attention_noalloc(g.desc, qd, qdt, S, NQ, HQ, pt, pt.shape[1], sl, 0.0,
+                                          20.0, out, bound, flags)
+    assert rc == kvq.KVQ_OK, kvq.last_error()
+    torch.cuda.synchronize()
+    assert g.device_error() == 0
+    assert torch.equal(out, out_w.view_as(out)) and torch.equal(bound, bound_w.view_as(bound))
+    assert torch.equal(flags, flags_w.view_as(flags))
