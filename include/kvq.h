@@ -182,7 +182,9 @@ typedef struct kvq_cache {
  *   taken only when strictly larger; a later s only when strictly larger;
  *   r = sqrt((x0^2 + x1^2) + (x2^2 + x3^2)) (fp32), stored as fp8 E4M3
  *   (round to nearest even, saturating at 448); codeword c = q_p q_s in fp32
- *   (exact term products summed left to right); x^ = r^ * c.
+ *   (exact term products summed left to right); x^ = r^ * c16 with c16 the
+ *   codeword rounded to fp16 per component (nearest even; the product is
+ *   exact in fp32).
  *   A chunk with a non-finite r gets code 0, radius 0; a token with a
  *   non-finite value sets KVQ_ERR_RANGE and eps (K) and eta to +inf.
  * Block of one (page, kv head), 16 tokens, n = head_dim / 4 chunks,

@@ -474,6 +474,14 @@ def hq_codeword(sec, i: int) -> np.ndarray:
     return out
 
 
+def hq_codeword16(sec, i: int) -> np.ndarray:
+    """Codeword i rounded to fp16 per component (the one the reconstruction uses)."""
+    sec = _c(sec, np.float32)
+    out = np.zeros(4, dtype=np.float32)
+    lib().oh_codeword16(_p(sec), int(i), _p(out))
+    return out
+
+
 def hq_direction(x, sec) -> int:
     """The direction code of one 4-channel chunk x against a secondary set [S][4]."""
     x = _c(x, np.float32)

@@ -1522,7 +1522,9 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
 /*    radius 0; a token with a non-finite K or V value sets the range error */
 /*    and gets eps = eta = +inf (K) or eta = +inf (V), so every query over  */
 /*    its block is flagged;                                                  */
-/*  - x^ = r^ * c (fp32 products);                                           */
+/*  - the reconstruction takes the codeword rounded to fp16 (nearest, ties  */
+/*    to even), c16: x^ = r^ * c16, exact in fp32 (4 and 11 significant    */
+/*    bits);                                                                 */
 /*  - per token: |k|_2 (sequential fmaf chain) and eps = |k - k^|_2 (the    */
 /*    same chain over the channels' differences) raised by 2^-16 of itself, */
 /*    one ulp up; the bound's Delta_j = kappa*s*|q|_2 (eps_j + 2^-16 |k_j|);*/
@@ -1585,6 +1587,12 @@ void oh_codeword(const float* sec, int i, float* c) {
   float qp[4];
   oh_primary(i % 24, qp);
   oh_mul(qp, sec + 4 * (i / 24), c);
+}
+
+/* Codeword i with every component rounded to fp16 (the reconstruction's). */
+void oh_codeword16(const float* sec, int i, float* c) {
+  oh_codeword(sec, i, c);
+  for (int n = 0; n < 4; ++n) c[n] = (float)oc_f16_value(oc_f16_rn(c[n]));
 }
 
 /* The direction code of chunk x (Method 1: the codeword of largest inner
@@ -1667,7 +1675,7 @@ static int oh_code_vector(const float* x, int d, const float* sec, int S, uint8_
     oc_wr16(idx + 2 * OC_PAGE * ch, (uint16_t)i);
     rad[OC_PAGE * ch] = rq;
     float cw[4];
-    oh_codeword(sec, i, cw);
+    oh_codeword16(sec, i, cw);
     float rv = (float)oh_e4m3_value(rq);
     for (int n = 0; n < 4; ++n) xh[4 * ch + n] = rv * cw[n];
   }
@@ -1758,7 +1766,7 @@ int oh_append(const oh_cfg* c, uint8_t* pool, float* eta, const void* k, const v
 }
 
 /* Read back token `slot` of a block: k^ and v^ as the append reconstructed
- * them (fp32 products r^ * c). */
+ * them (r^ * c16). */
 void oh_read_token(const oh_cfg* c, const uint8_t* blk, int slot, const float* secs, float* kh,
                    float* vh) {
   int nc = c->d / 4;
@@ -1768,7 +1776,7 @@ void oh_read_token(const oh_cfg* c, const uint8_t* blk, int slot, const float* s
     float* out = role ? vh : kh;
     for (int ch = 0; ch < nc; ++ch) {
       float cw[4];
-      oh_codeword(secs + role * 4 * c->S, oc_rd16(idx + 2 * OC_PAGE * ch), cw);
+      oh_codeword16(secs + role * 4 * c->S, oc_rd16(idx + 2 * OC_PAGE * ch), cw);
       float rv = (float)oh_e4m3_value(rad[OC_PAGE * ch]);
       for (int n = 0; n < 4; ++n) out[4 * ch + n] = rv * cw[n];
     }

@@ -16,7 +16,7 @@
 //   hqmq_partial_kernel   grid (sequence x kv head, split), 4 warps, each
 //                         streaming its pages through a 2-stage bulk-copy
 //                         ring; the CTA builds its kv head's 2 x 24 S
-//                         codewords in shared memory first.  Scores with one
+//                         codewords (fp16) in shared memory first.  Scores with one
 //                         lane per (token, half of the chunks), PV with one
 //                         lane per chunk, online softmax and the bound's sums
 //                         as for the other codecs
@@ -97,6 +97,20 @@ __device__ __forceinline__ int hq_direction(const float x[4], const float4* sec,
     }
   }
   return best;
+}
+
+// the reconstruction's codeword: each component rounded to fp16 (nearest even)
+__device__ __forceinline__ float4 hq_round16(const float4 c) {
+  return make_float4(__half2float(__float2half_rn(c.x)), __half2float(__float2half_rn(c.y)),
+                     __half2float(__float2half_rn(c.z)), __half2float(__float2half_rn(c.w)));
+}
+// the same as the decode's table entry: four fp16 in two words
+__device__ __forceinline__ uint2 hq_pack16(const float4 c) {
+  return make_uint2(h2_as_u32(__floats2half2_rn(c.x, c.y)), h2_as_u32(__floats2half2_rn(c.z, c.w)));
+}
+__device__ __forceinline__ float4 hq_unpack16(const uint2 w) {
+  const float2 a = __half22float2(u32_as_h2(w.x)), b = __half22float2(u32_as_h2(w.y));
+  return make_float4(a.x, a.y, b.x, b.y);
 }
 
 // fp8 E4M3: round to nearest even, saturating at 448; and back (exact)
@@ -182,7 +196,7 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
       }
       reinterpret_cast<uint16_t*>(blk + (role ? L.vi() : 0))[kPage * ch + slot] = (uint16_t)code;
       blk[(role ? L.vr() : L.kr()) + kPage * ch + slot] = (uint8_t)rq;
-      const float4 cw = hq_codeword(code, secs[role * S + code / 24]);
+      const float4 cw = hq_round16(hq_codeword(code, secs[role * S + code / 24]));
       const float rv = e4m3_value(rq);
       const float xh[4] = {__fmul_rn(rv, cw.x), __fmul_rn(rv, cw.y), __fmul_rn(rv, cw.z),
                            __fmul_rn(rv, cw.w)};
@@ -295,13 +309,13 @@ struct HqCfg {
   static constexpr int OFF_QN = OFF_Q + NC * kHqRows * 16;                  // |q|_2 [4]
   static constexpr int OFF_BAR = (OFF_QN + 16 + 15) / 16 * 16;              // [warp][stage] u64
   static constexpr int OFF_PG = OFF_BAR + kHqWarps * kHqStages * 8;         // [warp][stage] i32
-  static constexpr int OFF_TAB = (OFF_PG + kHqWarps * kHqStages * 4 + 15) / 16 * 16;  // [2][24 S] float4
+  static constexpr int OFF_TAB = (OFF_PG + kHqWarps * kHqStages * 4 + 15) / 16 * 16;  // [2][24 S] 4 x fp16
   // merge of the CTA's warps (aliases the stages): per warp [4][D], [4][8], header
   static constexpr int MW = kHqRows * D + kHqRows * 8 + kHqHdr;
   static constexpr int MERGE = kHqWarps * MW * 4;
   static_assert(MERGE <= OFF_W, "the merge area must stay inside the stages");
   static_assert(BLOCK % 16 == 0, "bulk copies move multiples of 16 bytes");
-  static __host__ __device__ constexpr int smem(int S) { return 128 + OFF_TAB + 2 * 24 * S * 16; }
+  static __host__ __device__ constexpr int smem(int S) { return 128 + OFF_TAB + 2 * 24 * S * 8; }
 };
 
 template <int D>
@@ -370,13 +384,13 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
   __syncwarp();   // the barriers are initialized
   for (int j = 0; j < kHqStages && j < nloc; ++j) issue(j, j);
 
-  // ---- the kv head's codewords, K then V: [2][24 S] ----
-  float4* tab = reinterpret_cast<float4*>(sm + C::OFF_TAB);
+  // ---- the kv head's codewords in fp16, K then V: [2][24 S] ----
+  uint2* tab = reinterpret_cast<uint2*>(sm + C::OFF_TAB);
   {
     const float4* secs = reinterpret_cast<const float4*>(ha.sec) + (int64_t)kvh * 2 * S;
     for (int i = tid; i < 48 * S; i += blockDim.x) {
       const int role = i / (24 * S), ci = i - role * 24 * S;
-      tab[i] = hq_codeword(ci, __ldg(secs + role * S + ci / 24));
+      tab[i] = hq_pack16(hq_codeword(ci, __ldg(secs + role * S + ci / 24)));
     }
   }
   // ---- query rows (warp r = row r): q [chunk][row] as float4, |q|_2 ----
@@ -406,8 +420,8 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
     if (lane == 0) qn[r] = sqrtf(l2);
   }
   __syncthreads();
-  const float4* tabK = tab;
-  const float4* tabV = tab + 24 * S;
+  const uint2* tabK = tab;
+  const uint2* tabV = tab + 24 * S;
   // a code beyond the table (only a pool not written by this codec holds one)
   // reads the last codeword instead of memory past the table
   const int ncw = 24 * S;
@@ -475,7 +489,7 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           const int c = hc ? HC + (cc + 1) % HC : cc;
           const int idx = min((int)kidx[kPage * c + t], ncw - 1);
           const float rv = e4m3_value(krad[kPage * c + t]);
-          const float4 cw = tabK[idx];
+          const float4 cw = hq_unpack16(tabK[idx]);
           const float k0 = __fmul_rn(rv, cw.x), k1 = __fmul_rn(rv, cw.y);
           const float k2 = __fmul_rn(rv, cw.z), k3 = __fmul_rn(rv, cw.w);
 #pragma unroll
@@ -557,7 +571,7 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
         for (int tt = 0; tt < TPL; ++tt) {
           const int idx = min((int)((iw[tt / 2] >> (16 * (tt & 1))) & 0xFFFFu), ncw - 1);
           const float rv = e4m3_value((rw[tt / 4] >> (8 * (tt & 3))) & 0xFFu);
-          const float4 cw = tabV[idx];
+          const float4 cw = hq_unpack16(tabV[idx]);
           const float v0 = __fmul_rn(rv, cw.x), v1 = __fmul_rn(rv, cw.y);
           const float v2 = __fmul_rn(rv, cw.z), v3 = __fmul_rn(rv, cw.w);
           const float4 w4 = w4p[tt];

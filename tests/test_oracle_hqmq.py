@@ -8,15 +8,16 @@ Against things other than its own code:
   closed under a quaternion product written here (4x4 matrices, fp64), with
   2T's element orders (1, 1, 8, 6, 8 elements of order 1, 2, 3, 4, 6) and 60
   degrees between nearest neighbours;
-* each codeword is q_p q_s to fp32 rounding, and each secondary unit maps 2T
-  isometrically (the page's argument for calibration-free codebooks);
+* each codeword is q_p q_s to fp32 rounding (and to fp16 rounding in the
+  reconstruction), and each secondary unit maps 2T isometrically (the page's
+  argument for calibration-free codebooks);
 * the direction code is the codeword of largest inner product, by brute force
   in fp64 over all 24 S codewords;
 * covering: every direction lies within 45 degrees (the 24-cell's covering
   radius, attained at (1 + i)/sqrt 2) of a codeword for any S, and the mean
   angular error falls with S like (24 S)^(-1/3) (the page's Proposition 3.1);
 * the radius in fp8 E4M3 against torch's float8_e4m3fn cast and hand values;
-* exact recovery of chunks that are representable (r^ c with r^ in E4M3);
+* exact recovery of chunks that are representable (r^ c16 with r^ in E4M3);
 * an independent numpy reader of the documented block layout reproduces the
   decode; eps, eta and the value range cover the errors; the bound never falls
   below the error against exact attention, and Delta is tight when q is
@@ -94,6 +95,8 @@ def test_codewords_are_products_and_isometric_copies(oracle_lib):
     got = np.stack([oracle.hq_codeword(sec, i) for i in range(book.shape[0])]).astype(np.float64)
     assert np.abs(got - book).max() < 2 ** -23
     assert np.allclose(np.linalg.norm(got, axis=1), 1.0, atol=1e-6)
+    got16 = np.stack([oracle.hq_codeword16(sec, i) for i in range(book.shape[0])])
+    assert np.array_equal(got16, got.astype(np.float32).astype(np.float16).astype(np.float32))
     P = _primaries()
     for s in range(sec.shape[0]):                # right multiplication by q_s is an isometry
         blk = got[24 * s:24 * s + 24]
@@ -183,6 +186,9 @@ class _Reader:
         self.E4 = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(
             torch.float64).numpy()
         self.books = [[_book64(c.sec[h, r]) for r in range(2)] for h in range(c.cfg.hkv)]
+        # the reconstruction's codewords: fp16 of the fp32 products
+        self.books16 = [[b.astype(np.float32).astype(np.float16).astype(np.float64) for b in bh]
+                        for bh in self.books]
 
     def token(self, page, kv, slot):
         nc, blk = self.nc, self.c.pool[(page * self.c.cfg.hkv + kv) * self.bb:][:self.bb]
@@ -191,8 +197,8 @@ class _Reader:
         kr = self.E4[blk[64 * nc:80 * nc].reshape(nc, 16)[:, slot]]
         vr = self.E4[blk[80 * nc:96 * nc].reshape(nc, 16)[:, slot]]
         f = blk[96 * nc:].view(np.float32)
-        kh = (kr[:, None] * self.books[kv][0][ki]).reshape(-1)
-        vh = (vr[:, None] * self.books[kv][1][vi]).reshape(-1)
+        kh = (kr[:, None] * self.books16[kv][0][ki]).reshape(-1)
+        vh = (vr[:, None] * self.books16[kv][1][vi]).reshape(-1)
         return dict(ki=ki, vi=vi, kr=kr, vr=vr, kh=kh, vh=vh, nk=f[slot], eps=f[16 + slot],
                     rg=f[32:32 + 2 * (self.d // 32)].reshape(-1, 2))
 
@@ -243,7 +249,7 @@ def test_exact_recovery_of_representable_chunks(oracle_lib):
     rads = rng.integers(0x20, 0x60, size=(2, d // 4)).astype(np.uint8)
     for role in range(2):
         for ch in range(d // 4):
-            cw = oracle.hq_codeword(secs[0, role], int(codes[role, ch]))
+            cw = oracle.hq_codeword16(secs[0, role], int(codes[role, ch]))
             x[role, 4 * ch:4 * ch + 4] = np.float32(oracle.e4m3_value(int(rads[role, ch]))) * cw
     c = oracle.HqCache(d, 1, 1, secs)
     k = x[0].reshape(1, 1, 1, d)
