@@ -304,8 +304,8 @@ struct HqCfg {
   static constexpr int NC = D / 4;
   static constexpr int BLOCK = 24 * D + 8 * kPage + D / 4;                  // HqLayout{D}.bytes()
   static constexpr int OFF_ST = 0;                                          // [warp][stage][BLOCK]
-  static constexpr int OFF_W = OFF_ST + kHqWarps * kHqStages * BLOCK;       // [warp][16][4] f32
-  static constexpr int OFF_Q = OFF_W + kHqWarps * kPage * kHqRows * 4;      // q [chunk][row] float4
+  static constexpr int OFF_W = OFF_ST + kHqWarps * kHqStages * BLOCK;       // [warp][16][4] f32 x 2
+  static constexpr int OFF_Q = OFF_W + kHqWarps * kPage * kHqRows * 8;      // q [chunk][row] float4
   static constexpr int OFF_QN = OFF_Q + NC * kHqRows * 16;                  // |q|_2 [4]
   static constexpr int OFF_BAR = (OFF_QN + 16 + 15) / 16 * 16;              // [warp][stage] u64
   static constexpr int OFF_PG = OFF_BAR + kHqWarps * kHqStages * 8;         // [warp][stage] i32
@@ -438,11 +438,11 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
   // PV: lane owns chunk pc for tokens t0 .. t0 + TPL - 1
   const int pc = lane % NC, t0 = (lane / NC) * TPL;
 
-  float acc[kHqRows][4];
+  // PV accumulators: row r, channels (0, 1) and (2, 3) of the lane's chunk,
+  // each pair one packed fp32x2 register
+  float2 acc[kHqRows][2];
 #pragma unroll
-  for (int r = 0; r < kHqRows; ++r)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[r][e] = 0.f;
+  for (int r = 0; r < kHqRows; ++r) acc[r][0] = acc[r][1] = make_float2(0.f, 0.f);
   float m2[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f}, Asum[2] = {0.f, 0.f},
         Bsum[2] = {0.f, 0.f}, Esum[2] = {0.f, 0.f}, dmax[2] = {0.f, 0.f};
   float rhi[NB], rlo[NB], etamax = clamped ? INFINITY : 0.f;
@@ -451,7 +451,8 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
     rhi[g] = -INFINITY;
     rlo[g] = INFINITY;
   }
-  float* wts = reinterpret_cast<float*>(sm + C::OFF_W) + warp * kPage * kHqRows;
+  // the page's weights [token][row], each twice (a packed pair for PV)
+  float2* wts = reinterpret_cast<float2*>(sm + C::OFF_W) + warp * kPage * kHqRows;
   int jstop = nloc;
   for (int j = 0; j < nloc; ++j) {
     const int st = j % kHqStages;
@@ -480,7 +481,10 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
       // ---- scores: q . k^ of token t over half hc of the chunks (the upper
       // half starts one chunk later, so the two halves' loads fall in
       // different banks) ----
-      float s4[kHqRows] = {0.f, 0.f, 0.f, 0.f};
+      // per row: the channel pairs (0, 1) and (2, 3) summed as packed fp32x2
+      float2 s2[kHqRows];
+#pragma unroll
+      for (int r = 0; r < kHqRows; ++r) s2[r] = make_float2(0.f, 0.f);
       {
         const uint16_t* kidx = reinterpret_cast<const uint16_t*>(blk);
         const uint8_t* krad = blk + L.kr();
@@ -490,17 +494,23 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           const int idx = min((int)kidx[kPage * c + t], ncw - 1);
           const float rv = e4m3_value(krad[kPage * c + t]);
           const float4 cw = hq_unpack16(tabK[idx]);
-          const float k0 = __fmul_rn(rv, cw.x), k1 = __fmul_rn(rv, cw.y);
-          const float k2 = __fmul_rn(rv, cw.z), k3 = __fmul_rn(rv, cw.w);
+          const float2 rr = make_float2(rv, rv);
+          const float2 k01 = mul2(make_float2(cw.x, cw.y), rr);   // exact products
+          const float2 k23 = mul2(make_float2(cw.z, cw.w), rr);
 #pragma unroll
           for (int r = 0; r < kHqRows; ++r) {
             const float4 qv = qs[c * kHqRows + r];
-            s4[r] = fmaf(qv.w, k3, fmaf(qv.z, k2, fmaf(qv.y, k1, fmaf(qv.x, k0, s4[r]))));
+            s2[r] = fma2(make_float2(qv.x, qv.y), k01, s2[r]);
+            s2[r] = fma2(make_float2(qv.z, qv.w), k23, s2[r]);
           }
         }
       }
+      float s4[kHqRows];
 #pragma unroll
-      for (int r = 0; r < kHqRows; ++r) s4[r] += __shfl_xor_sync(0xffffffffu, s4[r], 16);
+      for (int r = 0; r < kHqRows; ++r) {
+        s4[r] = s2[r].x + s2[r].y;
+        s4[r] += __shfl_xor_sync(0xffffffffu, s4[r], 16);
+      }
       const bool vt = t < nval;
       float zt[2], dl[2];
 #pragma unroll
@@ -530,7 +540,7 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
         Bsum[k] = fmaf(Bsum[k], alpha[k], wv * en);
         Esum[k] = fmaf(Esum[k], alpha[k], wv * eta_pg);
         dmax[k] = fmaxf(dmax[k], d);
-        wts[t * 4 + r0 + k] = wv;   // 0 outside the context
+        wts[t * 4 + r0 + k] = make_float2(wv, wv);   // 0 outside the context
       }
       if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
 #pragma unroll
@@ -538,7 +548,7 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           // row r's factor sits in the lanes of half r / 2, slot r % 2
           const float ar = __shfl_sync(0xffffffffu, alpha[r & 1], 16 * (r >> 1));
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[r][e] *= ar;
+          for (int h = 0; h < 2; ++h) acc[r][h] = mul2(acc[r][h], make_float2(ar, ar));
         }
       }
       __syncwarp();
@@ -566,22 +576,22 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           rw[0] = r2.x;
           rw[1] = r2.y;
         }
-        const float4* w4p = reinterpret_cast<const float4*>(wts) + t0;
+        const float4* w4p = reinterpret_cast<const float4*>(wts) + 2 * t0;
 #pragma unroll
         for (int tt = 0; tt < TPL; ++tt) {
           const int idx = min((int)((iw[tt / 2] >> (16 * (tt & 1))) & 0xFFFFu), ncw - 1);
           const float rv = e4m3_value((rw[tt / 4] >> (8 * (tt & 3))) & 0xFFu);
           const float4 cw = hq_unpack16(tabV[idx]);
-          const float v0 = __fmul_rn(rv, cw.x), v1 = __fmul_rn(rv, cw.y);
-          const float v2 = __fmul_rn(rv, cw.z), v3 = __fmul_rn(rv, cw.w);
-          const float4 w4 = w4p[tt];
-          const float wr[4] = {w4.x, w4.y, w4.z, w4.w};
+          const float2 rr = make_float2(rv, rv);
+          const float2 v01 = mul2(make_float2(cw.x, cw.y), rr);   // exact products
+          const float2 v23 = mul2(make_float2(cw.z, cw.w), rr);
+          const float4 wa = w4p[2 * tt], wb = w4p[2 * tt + 1];   // (w0, w0, w1, w1), (w2, w2, w3, w3)
+          const float2 w2[kHqRows] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w),
+                                      make_float2(wb.x, wb.y), make_float2(wb.z, wb.w)};
 #pragma unroll
           for (int r = 0; r < kHqRows; ++r) {
-            acc[r][0] = fmaf(wr[r], v0, acc[r][0]);
-            acc[r][1] = fmaf(wr[r], v1, acc[r][1]);
-            acc[r][2] = fmaf(wr[r], v2, acc[r][2]);
-            acc[r][3] = fmaf(wr[r], v3, acc[r][3]);
+            acc[r][0] = fma2(w2[r], v01, acc[r][0]);
+            acc[r][1] = fma2(w2[r], v23, acc[r][1]);
           }
         }
       }
@@ -611,7 +621,10 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
 #pragma unroll
     for (int r = 0; r < kHqRows; ++r)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], 16);
+      for (int h = 0; h < 2; ++h) {
+        acc[r][h].x += __shfl_xor_sync(0xffffffffu, acc[r][h].x, 16);
+        acc[r][h].y += __shfl_xor_sync(0xffffffffu, acc[r][h].y, 16);
+      }
   }
   __syncthreads();   // every warp is done with its stages
   float* mw = reinterpret_cast<float*>(sm) + warp * C::MW;
@@ -619,7 +632,7 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
 #pragma unroll
     for (int r = 0; r < kHqRows; ++r)
       *reinterpret_cast<float4*>(mw + r * D + 4 * lane) =
-          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+          make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
   }
   if (lane == 0 || lane == 16) {   // the lanes of half hc hold rows 2 hc, 2 hc + 1
 #pragma unroll
