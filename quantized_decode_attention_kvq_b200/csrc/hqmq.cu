@@ -304,8 +304,8 @@ struct HqCfg {
   static constexpr int NC = D / 4;
   static constexpr int BLOCK = 24 * D + 8 * kPage + D / 4;                  // HqLayout{D}.bytes()
   static constexpr int OFF_ST = 0;                                          // [warp][stage][BLOCK]
-  static constexpr int OFF_W = OFF_ST + kHqWarps * kHqStages * BLOCK;       // [warp][16][4] f32 x 2
-  static constexpr int OFF_Q = OFF_W + kHqWarps * kPage * kHqRows * 8;      // q [chunk][row] float4
+  static constexpr int OFF_W = OFF_ST + kHqWarps * kHqStages * BLOCK;       // [warp][16][4] f32
+  static constexpr int OFF_Q = OFF_W + kHqWarps * kPage * kHqRows * 4;      // q [chunk][row] float4
   static constexpr int OFF_QN = OFF_Q + NC * kHqRows * 16;                  // |q|_2 [4]
   static constexpr int OFF_BAR = (OFF_QN + 16 + 15) / 16 * 16;              // [warp][stage] u64
   static constexpr int OFF_PG = OFF_BAR + kHqWarps * kHqStages * 8;         // [warp][stage] i32
@@ -451,8 +451,8 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
     rhi[g] = -INFINITY;
     rlo[g] = INFINITY;
   }
-  // the page's weights [token][row], each twice (a packed pair for PV)
-  float2* wts = reinterpret_cast<float2*>(sm + C::OFF_W) + warp * kPage * kHqRows;
+  // the page's weights [token][row]
+  float* wts = reinterpret_cast<float*>(sm + C::OFF_W) + warp * kPage * kHqRows;
   int jstop = nloc;
   for (int j = 0; j < nloc; ++j) {
     const int st = j % kHqStages;
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
         Bsum[k] = fmaf(Bsum[k], alpha[k], wv * en);
         Esum[k] = fmaf(Esum[k], alpha[k], wv * eta_pg);
         dmax[k] = fmaxf(dmax[k], d);
-        wts[t * 4 + r0 + k] = make_float2(wv, wv);   // 0 outside the context
+        wts[t * 4 + r0 + k] = wv;   // 0 outside the context
       }
       if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
 #pragma unroll
@@ -576,7 +576,7 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           rw[0] = r2.x;
           rw[1] = r2.y;
         }
-        const float4* w4p = reinterpret_cast<const float4*>(wts) + 2 * t0;
+        const float4* w4p = reinterpret_cast<const float4*>(wts) + t0;
 #pragma unroll
         for (int tt = 0; tt < TPL; ++tt) {
           const int idx = min((int)((iw[tt / 2] >> (16 * (tt & 1))) & 0xFFFFu), ncw - 1);
@@ -585,9 +585,9 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           const float2 rr = make_float2(rv, rv);
           const float2 v01 = mul2(make_float2(cw.x, cw.y), rr);   // exact products
           const float2 v23 = mul2(make_float2(cw.z, cw.w), rr);
-          const float4 wa = w4p[2 * tt], wb = w4p[2 * tt + 1];   // (w0, w0, w1, w1), (w2, w2, w3, w3)
-          const float2 w2[kHqRows] = {make_float2(wa.x, wa.y), make_float2(wa.z, wa.w),
-                                      make_float2(wb.x, wb.y), make_float2(wb.z, wb.w)};
+          const float4 w4 = w4p[tt];   // one load; the pairs (w, w) are built in registers
+          const float2 w2[kHqRows] = {make_float2(w4.x, w4.x), make_float2(w4.y, w4.y),
+                                      make_float2(w4.z, w4.z), make_float2(w4.w, w4.w)};
 #pragma unroll
           for (int r = 0; r < kHqRows; ++r) {
             acc[r][0] = fma2(w2[r], v01, acc[r][0]);
