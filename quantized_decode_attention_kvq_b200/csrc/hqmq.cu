@@ -7,8 +7,9 @@
 // Bounded-Error Quantized Attention" (Methodology 2) carries over with a
 // per-token Euclidean key error.
 //
-//   hqmq_append_kernel    one warp per (token, kv head): each lane codes one
-//                         (chunk, role) pair at a time (the direction through
+//   hqmq_append_kernel    one warp per (token, kv head, role) at d = 128 (per
+//                         (token, kv head) at d = 64): each lane codes one
+//                         (chunk, role) pair (the direction through
 //                         y = x conj(q_s) and 2T's closed-form best unit, the
 //                         radius by the fp8 conversion), then |k|, eps and
 //                         |v| as sequential chains over the channels, eta and
@@ -125,15 +126,16 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
 }  // namespace
 
 // ================================================================ append =====
-// One warp per (token, kv head), 8 warps per CTA looping over the items.  Lane
-// l codes (chunk l, K) then (chunk l, V) at d = 128, or (chunk l % 16, role
-// l / 16) at d = 64.
-constexpr int kHqAppendWarps = 8;
+// One warp per item, 4 warps per CTA looping over the items.  At d = 128 an
+// item is one role of one (token, kv head), lane l coding chunk l, so K and V
+// search in parallel warps; at d = 64 an item is the (token, kv head), lane l
+// coding (chunk l % 16, role l / 16).
+constexpr int kHqAppendWarps = 4;
 
 template <int D>
 __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const HqAppendArgs ha) {
   constexpr int NC = D / 4;
-  constexpr int CPL = 2 * NC / 32;   // (chunk, role) pairs per lane
+  constexpr bool SPLIT = NC == 32;   // one role per item
   constexpr int GL = 8;              // lanes per 32-channel group of V chunks
   const AppendArgs& a = ha.a;
   const HqLayout L{D};
@@ -144,12 +146,14 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
   float* xk = stg[w][0];
   float* ek = stg[w][1];
   float* xv = stg[w][2];
-  const int64_t total = (int64_t)a.num_seqs * a.num_tokens * a.hkv;
+  const int64_t total = (int64_t)a.num_seqs * a.num_tokens * a.hkv * (SPLIT ? 2 : 1);
   for (int64_t item = (int64_t)blockIdx.x * kHqAppendWarps + w; item < total;
        item += (int64_t)gridDim.x * kHqAppendWarps) {
-    const int h = (int)(item % a.hkv);
-    const int t = (int)((item / a.hkv) % a.num_tokens);
-    const int s = (int)(item / ((int64_t)a.hkv * a.num_tokens));
+    const int rsel = SPLIT ? (int)(item & 1) : 0;   // the item's role when split
+    const int64_t it = SPLIT ? item >> 1 : item;
+    const int h = (int)(it % a.hkv);
+    const int t = (int)((it / a.hkv) % a.num_tokens);
+    const int s = (int)(it / ((int64_t)a.hkv * a.num_tokens));
     if (a.valid && t >= a.valid[s]) continue;
     const int pos = a.start_pos[s] + t;
     const int lp = pos / kPage;
@@ -165,62 +169,57 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
     const int slot = pos % kPage;
     const int64_t base = s * a.seq_stride + h * a.head_stride + (int64_t)t * a.tok_stride;
     uint8_t* blk = a.pool + ((int64_t)page * a.hkv + h) * L.bytes();
+    const bool has_k = !SPLIT || rsel == 0, has_v = !SPLIT || rsel == 1;
     __syncwarp();   // the previous item's chains and searches have read the staging rows
-    {   // the kv head's secondary units, K then V, in one coalesced load
-      const float4* src = reinterpret_cast<const float4*>(ha.sec) + (int64_t)h * 2 * S;
-      for (int i = lane; i < 2 * S; i += 32) ssec[w][i] = __ldg(src + i);
+    {   // the item's secondary units (its role's, or K's then V's) in one coalesced load
+      const float4* src = reinterpret_cast<const float4*>(ha.sec) + (int64_t)h * 2 * S +
+                          (SPLIT ? rsel * S : 0);
+      for (int i = lane; i < (SPLIT ? S : 2 * S); i += 32) ssec[w][i] = __ldg(src + i);
     }
     __syncwarp();
-    const float4* secs = ssec[w];
-    bool bad_k = false, bad_v = false, bad_r = false;
+    const int role = SPLIT ? rsel : lane / 16;
+    const int ch = SPLIT ? lane : lane % 16;
+    const float4* secs = ssec[w] + (SPLIT ? 0 : role * S);
+    float x[4];
+#pragma unroll
+    for (int n = 0; n < 4; ++n) x[n] = load_elem(role ? a.v : a.k, a.in_bf16, base + 4 * ch + n);
+    bool fin = true;
+#pragma unroll
+    for (int n = 0; n < 4; ++n) fin = fin && isfinite(x[n]);
+    const float r = __fsqrt_rn(__fadd_rn(__fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[1], x[1])),
+                                         __fadd_rn(__fmul_rn(x[2], x[2]), __fmul_rn(x[3], x[3]))));
+    int code = 0;
+    uint32_t rq = 0;
+    const bool rok = isfinite(r);
+    if (rok) {
+      code = hq_direction(x, secs, S);
+      rq = e4m3_rn(r);
+    }
+    reinterpret_cast<uint16_t*>(blk + (role ? L.vi() : 0))[kPage * ch + slot] = (uint16_t)code;
+    blk[(role ? L.vr() : L.kr()) + kPage * ch + slot] = (uint8_t)rq;
+    const float4 cw = hq_round16(hq_codeword(code, secs[code / 24]));
+    const float rv = e4m3_value(rq);
+    const float xh[4] = {__fmul_rn(rv, cw.x), __fmul_rn(rv, cw.y), __fmul_rn(rv, cw.z),
+                         __fmul_rn(rv, cw.w)};
     float err = 0.f, hi = 0.f, lo = 0.f;
+    if (role == 0) {
 #pragma unroll
-    for (int u = 0; u < CPL; ++u) {
-      const int role = CPL == 2 ? u : lane / 16;
-      const int ch = CPL == 2 ? lane : lane % 16;
-      float x[4];
-#pragma unroll
-      for (int n = 0; n < 4; ++n) x[n] = load_elem(role ? a.v : a.k, a.in_bf16, base + 4 * ch + n);
-      bool fin = true;
-#pragma unroll
-      for (int n = 0; n < 4; ++n) fin = fin && isfinite(x[n]);
-      const float r = __fsqrt_rn(__fadd_rn(__fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[1], x[1])),
-                                           __fadd_rn(__fmul_rn(x[2], x[2]), __fmul_rn(x[3], x[3]))));
-      int code = 0;
-      uint32_t rq = 0;
-      if (isfinite(r)) {
-        code = hq_direction(x, secs + role * S, S);
-        rq = e4m3_rn(r);
-      } else {
-        bad_r = true;
+      for (int n = 0; n < 4; ++n) {
+        xk[4 * ch + n] = x[n];
+        ek[4 * ch + n] = __fsub_rn(x[n], xh[n]);
       }
-      reinterpret_cast<uint16_t*>(blk + (role ? L.vi() : 0))[kPage * ch + slot] = (uint16_t)code;
-      blk[(role ? L.vr() : L.kr()) + kPage * ch + slot] = (uint8_t)rq;
-      const float4 cw = hq_round16(hq_codeword(code, secs[role * S + code / 24]));
-      const float rv = e4m3_value(rq);
-      const float xh[4] = {__fmul_rn(rv, cw.x), __fmul_rn(rv, cw.y), __fmul_rn(rv, cw.z),
-                           __fmul_rn(rv, cw.w)};
-      if (role == 0) {
-        bad_k = bad_k || !fin;
+    } else {
 #pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          xk[4 * ch + n] = x[n];
-          ek[4 * ch + n] = __fsub_rn(x[n], xh[n]);
-        }
-      } else {
-        bad_v = bad_v || !fin;
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-          xv[4 * ch + n] = x[n];
-          err = fmaxf(err, fabsf(__fsub_rn(x[n], xh[n])));
-          hi = fmaxf(hi, xh[n]);
-          lo = fminf(lo, xh[n]);
-        }
+      for (int n = 0; n < 4; ++n) {
+        xv[4 * ch + n] = x[n];
+        err = fmaxf(err, fabsf(__fsub_rn(x[n], xh[n])));
+        hi = fmaxf(hi, xh[n]);
+        lo = fminf(lo, xh[n]);
       }
     }
-    bad_k = __any_sync(0xffffffffu, bad_k);
-    bad_v = __any_sync(0xffffffffu, bad_v);
-    bad_r = __any_sync(0xffffffffu, bad_r);
+    const bool bad_k = __any_sync(0xffffffffu, role == 0 && !fin);
+    const bool bad_v = __any_sync(0xffffffffu, role == 1 && !fin);
+    const bool bad_r = __any_sync(0xffffffffu, !rok);
 #pragma unroll
     for (int o = 1; o < 32; o *= 2) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, o));
 #pragma unroll
@@ -231,28 +230,43 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
     __syncwarp();
     // |k|, |k - k^| and |v|: sequential chains over the channels
     float nk2 = 0.f, e2 = 0.f, nv2 = 0.f;
+    if (has_k) {
 #pragma unroll 4
-    for (int c = 0; c < D; c += 4) {
-      const float4 k4 = *reinterpret_cast<const float4*>(xk + c);
-      const float4 e4 = *reinterpret_cast<const float4*>(ek + c);
-      const float4 v4 = *reinterpret_cast<const float4*>(xv + c);
-      nk2 = __fmaf_rn(k4.w, k4.w, __fmaf_rn(k4.z, k4.z, __fmaf_rn(k4.y, k4.y, __fmaf_rn(k4.x, k4.x, nk2))));
-      e2 = __fmaf_rn(e4.w, e4.w, __fmaf_rn(e4.z, e4.z, __fmaf_rn(e4.y, e4.y, __fmaf_rn(e4.x, e4.x, e2))));
-      nv2 = __fmaf_rn(v4.w, v4.w, __fmaf_rn(v4.z, v4.z, __fmaf_rn(v4.y, v4.y, __fmaf_rn(v4.x, v4.x, nv2))));
+      for (int c = 0; c < D; c += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(xk + c);
+        const float4 e4 = *reinterpret_cast<const float4*>(ek + c);
+        nk2 = __fmaf_rn(k4.w, k4.w, __fmaf_rn(k4.z, k4.z, __fmaf_rn(k4.y, k4.y, __fmaf_rn(k4.x, k4.x, nk2))));
+        e2 = __fmaf_rn(e4.w, e4.w, __fmaf_rn(e4.z, e4.z, __fmaf_rn(e4.y, e4.y, __fmaf_rn(e4.x, e4.x, e2))));
+      }
+    }
+    if (has_v) {
+#pragma unroll 4
+      for (int c = 0; c < D; c += 4) {
+        const float4 v4 = *reinterpret_cast<const float4*>(xv + c);
+        nv2 = __fmaf_rn(v4.w, v4.w, __fmaf_rn(v4.z, v4.z, __fmaf_rn(v4.y, v4.y, __fmaf_rn(v4.x, v4.x, nv2))));
+      }
     }
     if (lane == 0) {
       if (bad_k || bad_v || bad_r) set_error(a.err, KVQ_ERR_RANGE);
-      const float en = __fsqrt_rn(e2);
-      reinterpret_cast<float*>(blk + L.kn())[slot] = __fsqrt_rn(nk2);
-      reinterpret_cast<float*>(blk + L.ke())[slot] =
-          bad_k ? INFINITY : nextafterf(__fmaf_rn(en, 0x1p-16f, en), INFINITY);
-      const float eu = bad_k || bad_v ? INFINITY
-                                      : nextafterf(__fmaf_rn(0x1p-16f, __fsqrt_rn(nv2), err), INFINITY);
-      atomicMax(reinterpret_cast<int*>(a.eta + (int64_t)page * a.hkv + h), __float_as_int(eu));
+      int* eta = reinterpret_cast<int*>(a.eta + (int64_t)page * a.hkv + h);
+      if (has_k) {
+        const float en = __fsqrt_rn(e2);
+        reinterpret_cast<float*>(blk + L.kn())[slot] = __fsqrt_rn(nk2);
+        reinterpret_cast<float*>(blk + L.ke())[slot] =
+            bad_k ? INFINITY : nextafterf(__fmaf_rn(en, 0x1p-16f, en), INFINITY);
+        // a non-finite key makes the token's eta +inf (its value warp cannot see it)
+        if (SPLIT && bad_k) atomicMax(eta, __float_as_int(INFINITY));
+      }
+      if (has_v) {
+        const float eu = bad_v || (!SPLIT && bad_k)
+                             ? INFINITY
+                             : nextafterf(__fmaf_rn(0x1p-16f, __fsqrt_rn(nv2), err), INFINITY);
+        atomicMax(eta, __float_as_int(eu));
+      }
     }
-    // the V chunks' 32-channel groups: lanes 8 g .. 8 g + 7 (d 128), or
-    // 16 + 8 g .. (d 64); the block's range starts at [0, 0]
-    const int vlane = CPL == 2 ? lane : lane - 16;
+    // the V chunks' 32-channel groups: lanes 8 g .. 8 g + 7 of a value item
+    // (d 128), or 16 + 8 g .. (d 64); the block's range starts at [0, 0]
+    const int vlane = SPLIT ? (rsel == 1 ? lane : -1) : lane - 16;
     if (vlane >= 0 && vlane % GL == 0) {
       float* rg = reinterpret_cast<float*>(blk + L.rg()) + 2 * (vlane / GL);
       if (hi > 0.f) atomicMax(reinterpret_cast<int*>(rg), __float_as_int(hi));
@@ -278,8 +292,8 @@ cudaError_t launch_hqmq_append_d(const HqAppendArgs& a, cudaStream_t stream) {
     }
     sms = it->second;
   }
-  const int64_t items = (int64_t)a.a.num_seqs * a.a.num_tokens * a.a.hkv;
-  const int64_t blocks = std::min<int64_t>((items + kHqAppendWarps - 1) / kHqAppendWarps, 4 * sms);
+  const int64_t items = (int64_t)a.a.num_seqs * a.a.num_tokens * a.a.hkv * (D == 128 ? 2 : 1);
+  const int64_t blocks = std::min<int64_t>((items + kHqAppendWarps - 1) / kHqAppendWarps, 8 * sms);
   hqmq_append_kernel<D><<<(unsigned)blocks, kHqAppendWarps * 32, 0, stream>>>(a);
   return cudaGetLastError();
 }

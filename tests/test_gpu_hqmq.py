@@ -169,9 +169,10 @@ def test_ragged_and_empty_contexts():
     _check(inp, r, q, inp.wl.tau, "hqmq ragged")
 
 
-def test_non_finite_input_is_reported():
+@pytest.mark.parametrize("name", ["tiny", "llama8b"])   # d = 64 and d = 128 (one warp per role)
+def test_non_finite_input_is_reported(name):
     from quantized_decode_attention_kvq_b200 import kvq
-    inp = small("tiny", 0)
+    inp = small(name, 0)
     k, v = inp.kv()
     k = k.copy()
     v = v.copy()
