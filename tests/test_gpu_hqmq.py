@@ -176,8 +176,9 @@ def test_non_finite_input_is_reported(name):
     k, v = inp.kv()
     k = k.copy()
     v = v.copy()
-    k[0, 0, 3, 5] = np.inf
-    v[0, 0, 7, 9] = np.nan
+    bf16 = k.dtype == np.uint16     # bf16 bit patterns: +inf 0x7f80, a quiet NaN 0x7fc0
+    k[0, 0, 3, 5] = 0x7F80 if bf16 else np.inf
+    v[0, 0, 7, 9] = 0x7FC0 if bf16 else np.nan
     wl = inp.wl
     g, o = _caches(inp)
     pt = torch.from_numpy(inp.page_table).cuda()
