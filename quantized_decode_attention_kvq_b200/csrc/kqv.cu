@@ -509,11 +509,13 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
   };
   for (int j = 0; j < kKqStages && j < nloc; ++j) issue(j, j);
 
-  float acc1[kKqRows][E], acc2[kKqRows][E];
+  // PV accumulators of channel (and projection) e: rows (0, 1) and (2, 3) as
+  // packed fp32x2 pairs
+  float2 acc1[E][2], acc2[E][2];
 #pragma unroll
-  for (int r = 0; r < kKqRows; ++r)
+  for (int e = 0; e < E; ++e)
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc1[r][e] = acc2[r][e] = 0.f;
+    for (int h = 0; h < 2; ++h) acc1[e][h] = acc2[e][h] = make_float2(0.f, 0.f);
   float m2[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f}, Asum[2] = {0.f, 0.f},
         Bsum[2] = {0.f, 0.f}, Esum[2] = {0.f, 0.f}, dmax[2] = {0.f, 0.f};
   float rhi[NB], rlo[NB], etamax = clamped ? INFINITY : 0.f;
@@ -629,14 +631,17 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
         wts[kPage * 4 + t * 4 + r0 + k] = wa * wrn;
       }
       if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
+        // row r's factor sits in lanes with c4 & 1 == r / 2, slot r % 2
+        float ar[kKqRows];
 #pragma unroll
-        for (int r = 0; r < kKqRows; ++r) {
-          // row r's factor sits in lanes with c4 & 1 == r / 2, slot r % 2
-          const float ar = __shfl_sync(0xffffffffu, alpha[r & 1], r >> 1);
+        for (int r = 0; r < kKqRows; ++r) ar[r] = __shfl_sync(0xffffffffu, alpha[r & 1], r >> 1);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 a2 = make_float2(ar[2 * h], ar[2 * h + 1]);
 #pragma unroll
           for (int e = 0; e < E; ++e) {
-            acc1[r][e] *= ar;
-            acc2[r][e] *= ar;
+            acc1[e][h] = mul2(acc1[e][h], a2);
+            acc2[e][h] = mul2(acc2[e][h], a2);
           }
         }
       }
@@ -657,15 +662,17 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
         }
 #pragma unroll
         for (int e = 0; e < E; ++e) sg[e] = (sb >> e) & 1u ? 1.f : -1.f;
-        const float war[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
-        const float wbr[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
+        const float2 wa2[2] = {make_float2(wa4.x, wa4.y), make_float2(wa4.z, wa4.w)};
+        const float2 wb2[2] = {make_float2(wb4.x, wb4.y), make_float2(wb4.z, wb4.w)};
 #pragma unroll
-        for (int r = 0; r < kKqRows; ++r)
+        for (int e = 0; e < E; ++e) {
+          const float2 c2 = make_float2(cv[e], cv[e]), s2 = make_float2(sg[e], sg[e]);
 #pragma unroll
-          for (int e = 0; e < E; ++e) {
-            acc1[r][e] = fmaf(war[r], cv[e], acc1[r][e]);
-            acc2[r][e] = fmaf(wbr[r], sg[e], acc2[r][e]);
+          for (int h = 0; h < 2; ++h) {
+            acc1[e][h] = fma2(wa2[h], c2, acc1[e][h]);
+            acc2[e][h] = fma2(wb2[h], s2, acc2[e][h]);
           }
+        }
       }
     }
     __syncwarp();
@@ -694,8 +701,8 @@ __global__ void __launch_bounds__(kKqWarps * 32) kqv_partial_kernel(const KqvDec
   for (int r = 0; r < kKqRows; ++r)
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      mw[r * D + lane * E + e] = acc1[r][e];
-      mw[kKqRows * D + r * D + lane * E + e] = acc2[r][e];
+      mw[r * D + lane * E + e] = (r & 1) ? acc1[e][r >> 1].y : acc1[e][r >> 1].x;
+      mw[kKqRows * D + r * D + lane * E + e] = (r & 1) ? acc2[e][r >> 1].y : acc2[e][r >> 1].x;
     }
   if (lane < 2) {   // lane c4 = lane holds rows 2 lane, 2 lane + 1
 #pragma unroll
