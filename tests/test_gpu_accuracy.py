@@ -7,7 +7,8 @@ notes; the assertions check that every row stays within its bound and that the
 errors are those of the codecs, not of the kernel: at full size, seed 0, about
 12% (INT8 keys) and 34% (rotated INT4 keys) relative L2 on N(0,1) data, where
 attention spreads over thousands of tokens and the outputs are small; the
-4-bit values dominate the INT8-key codec, and 4-bit keys almost triple it."""
+4-bit values dominate the INT8-key codec, and 4-bit keys almost triple it.
+The same measurement runs for Med3x extraction and the KQV and HQMQ codecs."""
 
 import numpy as np
 import pytest
@@ -37,4 +38,51 @@ def test_error_against_dense_attention(name):
     ratio = g["bound"] / np.maximum(err, 1e-30)
     print(f"{name}: max-abs error {err.max():.3e}, relative L2 {rel:.3e}, "
           f"mean bound {g['bound'].mean():.3f}, bound / error median {np.median(ratio):.0f}")
+    assert rel < 0.5
+
+
+def _run_codec(inp, k, v, q, codec):
+    """Append the whole context into a cache of another codec and decode."""
+    from gpu_cases import to_torch
+    from quantized_decode_attention_kvq_b200 import kvq
+    wl = inp.wl
+    if codec == "kqv":
+        kw = dict(codec="kqv", rot_signs=inp.rotation_signs(), qjl_matrix=inp.qjl_matrix())
+    else:
+        kw = dict(codec="hqmq", hq_secondary=inp.hqmq_secondary(32))
+    c = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, **kw)
+    pt = torch.from_numpy(inp.page_table).cuda()
+    sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
+    c.append(to_torch(k), to_torch(v), pt, torch.zeros(wl.num_seqs, dtype=torch.int32,
+                                                       device="cuda"), sl)
+    ws = c.workspace(wl.num_seqs, wl.num_queries, wl.num_q_heads, pt.shape[1])
+    out, bound, _ = c.decode(to_torch(q), pt, sl, ws, tau=float("inf"))
+    torch.cuda.synchronize()
+    assert c.device_error() == 0
+    return (out.cpu().numpy().reshape(-1, wl.head_dim).astype(np.float64),
+            bound.cpu().numpy().reshape(-1).astype(np.float64))
+
+
+@pytest.mark.parametrize("codec", ["med3", "kqv", "hqmq"])
+def test_error_of_the_other_codecs(codec):
+    """The same measurement on llama8b data and shapes for Med3x extraction
+    (over the INT8-key codec), the KQV codec and the HQMQ codec (S = 32)."""
+    if not torch.cuda.is_available():
+        pytest.fail("the GPU tests need a CUDA device")
+    inp = synth.make("llama8b", 0)
+    k, v = inp.kv()
+    q = inp.q()
+    if codec == "med3":
+        g = run_gpu(inp, k, v, q, outliers=True)
+        assert g["err"] == 0
+        out, bound = g["out"], g["bound"]
+    else:
+        out, bound = _run_codec(inp, k, v, q, codec)
+    dense = oracle.dense(q, k, v, inp.seq_lens)
+    err = max_err(dense, out)
+    rel = rel_l2(out, dense)
+    assert np.isfinite(err).all() and (err <= bound).all()
+    ratio = bound / np.maximum(err, 1e-30)
+    print(f"{codec}: max-abs error {err.max():.3e}, relative L2 {rel:.3e}, "
+          f"mean bound {bound.mean():.3f}, bound / error median {np.median(ratio):.0f}")
     assert rel < 0.5
