@@ -456,7 +456,7 @@ class KqvCache:
 
 
 class OhCfg(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("d", "hkv", "num_pages", "S")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("d", "hkv", "num_pages", "S", "outliers")]
 
 
 def hq_primary(p: int) -> np.ndarray:
@@ -502,13 +502,14 @@ class HqCache:
     Multiplicative Quantization for KV Cache Compression", Method 1-2): every
     4-channel chunk of K and V coded by its radius (fp8 E4M3) and the index of
     the nearest product codeword q_p q_s (q_p in 2T, q_s from the secondary
-    set of its kv head and role)."""
+    set of its kv head and role); with outliers, the Med3x chunk of K and of V
+    kept in fp16 (Method 3)."""
 
-    def __init__(self, head_dim, num_kv_heads, num_pages, secondary):
+    def __init__(self, head_dim, num_kv_heads, num_pages, secondary, outliers=False):
         sec = _c(secondary, np.float32)
         assert sec.ndim == 4 and sec.shape[0] == num_kv_heads and sec.shape[1] == 2 \
             and sec.shape[3] == 4
-        self.cfg = OhCfg(head_dim, num_kv_heads, num_pages, sec.shape[2])
+        self.cfg = OhCfg(head_dim, num_kv_heads, num_pages, sec.shape[2], int(bool(outliers)))
         bb = lib().oh_block_bytes(ctypes.byref(self.cfg))
         if bb < 0:
             raise ValueError("unsupported cache configuration")

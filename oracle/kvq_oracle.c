@@ -1530,23 +1530,31 @@ int oq_decode(const oq_cfg* c, const uint8_t* pool, const float* eta, const void
 /*    one ulp up; the bound's Delta_j = kappa*s*|q|_2 (eps_j + 2^-16 |k_j|);*/
 /*  - eta_b = the block's largest max_c |v - v^| + 2^-16 |v|_2, one ulp up; */
 /*    the value range per 32-channel group starts at [0, 0] (a zeroed      */
-/*    block) and widens to every v^ appended.                                */
+/*    block) and widens to every v^ appended;                                */
+/*  - with Med3x extraction (Method 3, the page's combination for           */
+/*    outlier-heavy models; outliers = 1): the chunk oc_med3_chunk picks in */
+/*    K and in V is kept in fp16 (R32's rules) in the Tier-1 outlier        */
+/*    section appended to the block, takes code 0 and radius 0, and         */
+/*    reconstructs to its fp16 values; eps, eta and the range are measured  */
+/*    on that reconstruction.                                                */
 /* Block of one (page, kv head), 16 tokens, d/4 chunks per vector, chunk-   */
 /* major (the 16 tokens of one chunk side by side):                         */
 /*   [K codes u16 [d/4][16]][V codes u16 [d/4][16]][K radii e4m3 [d/4][16]]  */
 /*   [V radii e4m3 [d/4][16]][|k| f32 [16]][eps f32 [16]]                    */
 /*   [v^ max, min f32 [d/32][2]]                                             */
+/*   (outliers = 1) [chunk K u8 [16]][chunk V u8 [16]][k16 f16 [16][4]]      */
+/*   [v16 f16 [16][4]] (0xFF: none; the values zero then)                    */
 /* u16 little-endian.                                                        */
 /* ======================================================================== */
 typedef struct {
-  int32_t d, hkv, num_pages, S;
+  int32_t d, hkv, num_pages, S, outliers;
 } oh_cfg;
 
 #define OH_MAX_S 2730   /* 24 S codewords index in 16 bits */
 
 static int oh_ok(const oh_cfg* c) {
   return c && (c->d == 64 || c->d == 128) && c->hkv > 0 && c->num_pages >= 0 && c->S >= 1 &&
-         c->S <= OH_MAX_S;
+         c->S <= OH_MAX_S && (c->outliers == 0 || c->outliers == 1);
 }
 static int64_t oh_off_vi(const oh_cfg* c) { return (int64_t)OC_PAGE * (c->d / 4) * 2; }
 static int64_t oh_off_kr(const oh_cfg* c) { return (int64_t)OC_PAGE * (c->d / 4) * 4; }
@@ -1555,9 +1563,11 @@ static int64_t oh_off_kn(const oh_cfg* c) { return oh_off_vr(c) + (int64_t)OC_PA
 static int64_t oh_off_ke(const oh_cfg* c) { return oh_off_kn(c) + 4 * OC_PAGE; }
 static int64_t oh_off_rg(const oh_cfg* c) { return oh_off_kn(c) + 8 * OC_PAGE; }
 
+static int64_t oh_off_out(const oh_cfg* c) { return oh_off_rg(c) + (int64_t)(c->d / 32) * 2 * 4; }
+
 int64_t oh_block_bytes(const oh_cfg* c) {
   if (!oh_ok(c)) return -1;
-  return oh_off_rg(c) + (int64_t)(c->d / 32) * 2 * 4;
+  return oh_off_out(c) + (c->outliers ? OC_OUT_BYTES : 0);
 }
 
 /* Unit p of 2T (Method 1: the 24 vertices of the 24-cell). */
@@ -1657,16 +1667,19 @@ static float oh_chunk_radius(const float* x) {
 }
 
 /* Code one d-vector x: chunk codes (u16, chunk ch at idx + 2 * 16 ch) and
- * radii (at rad + 16 ch), and the fp32 reconstruction. */
+ * radii (at rad + 16 ch), and the fp32 reconstruction; chunk `skip` (an
+ * extracted one, or -1) takes code 0 and radius 0. */
 static int oh_code_vector(const float* x, int d, const float* sec, int S, uint8_t* idx,
-                          uint8_t* rad, float* xh) {
+                          uint8_t* rad, float* xh, int skip) {
   int rc = OC_OK;
   for (int ch = 0; ch < d / 4; ++ch) {
     const float* xc = x + 4 * ch;
     float r = oh_chunk_radius(xc);
     int i = 0;
     uint8_t rq = 0;
-    if (!isfinite(r)) {
+    if (ch == skip) {
+      /* kept in fp16 by the caller */
+    } else if (!isfinite(r)) {
       rc = OC_ERR_RANGE;
     } else {
       i = oh_direction(xc, sec, S);
@@ -1692,12 +1705,34 @@ static float oh_chain_norm2(const float* a, int d) {
  * [2][S][4]); returns its eta contribution and raises the block's range. */
 static int oh_quantize_token(const oh_cfg* c, uint8_t* blk, int slot, const float* k,
                              const float* v, const float* secs, float* eta_out) {
-  int d = c->d, nc = d / 4, S = c->S;
+  int d = c->d, S = c->S;
   float kh[128], vh[128], e[128];
-  int rc = oh_code_vector(k, d, secs, S, blk + 2 * slot, blk + oh_off_kr(c) + slot, kh);
+  int ck = c->outliers ? oc_med3_chunk(k, d) : -1;
+  int cv = c->outliers ? oc_med3_chunk(v, d) : -1;
+  int rc = oh_code_vector(k, d, secs, S, blk + 2 * slot, blk + oh_off_kr(c) + slot, kh, ck);
   int rv = oh_code_vector(v, d, secs + 4 * S, S, blk + oh_off_vi(c) + 2 * slot,
-                          blk + oh_off_vr(c) + slot, vh);
+                          blk + oh_off_vr(c) + slot, vh, cv);
   if (rv != OC_OK) rc = rv;
+  if (c->outliers) {   /* the extracted chunks in fp16 (R32), their reconstruction */
+    uint8_t* os = blk + oh_off_out(c);
+    os[slot] = ck < 0 ? OC_NO_OUTLIER : (uint8_t)ck;
+    os[OC_PAGE + slot] = cv < 0 ? OC_NO_OUTLIER : (uint8_t)cv;
+    for (int role = 0; role < 2; ++role) {
+      int cx = role ? cv : ck;
+      const float* x = role ? v : k;
+      float* xh = role ? vh : kh;
+      for (int i = 0; i < 4; ++i) {
+        uint16_t h = 0;
+        if (cx >= 0) {
+          float xi = x[4 * cx + i];
+          if (!isfinite(xi) || fabsf(xi) > 65504.0f) rc = OC_ERR_RANGE;
+          else h = oc_f16_rn(xi);
+          xh[4 * cx + i] = (float)oc_f16_value(h);
+        }
+        oc_wr16(os + 2 * OC_PAGE + role * OC_PAGE * 8 + (slot * 4 + i) * 2, h);
+      }
+    }
+  }
   int bad_k = 0, bad_v = 0;
   for (int i = 0; i < d; ++i) {
     bad_k |= !isfinite(k[i]);
@@ -1779,6 +1814,14 @@ void oh_read_token(const oh_cfg* c, const uint8_t* blk, int slot, const float* s
       oh_codeword16(secs + role * 4 * c->S, oc_rd16(idx + 2 * OC_PAGE * ch), cw);
       float rv = (float)oh_e4m3_value(rad[OC_PAGE * ch]);
       for (int n = 0; n < 4; ++n) out[4 * ch + n] = rv * cw[n];
+    }
+    if (c->outliers) {   /* an extracted chunk reads back its fp16 values */
+      const uint8_t* os = blk + oh_off_out(c);
+      int cx = os[role * OC_PAGE + slot];
+      if (cx != OC_NO_OUTLIER && cx < nc)
+        for (int n = 0; n < 4; ++n)
+          out[4 * cx + n] =
+              (float)oc_f16_value(oc_rd16(os + 2 * OC_PAGE + role * OC_PAGE * 8 + (slot * 4 + n) * 2));
     }
   }
 }

@@ -323,3 +323,80 @@ def test_delta_is_tight_for_a_query_along_the_error(oracle_lib):
     slack = 1 + 2 ** -10
     allowance = s * qn * 2 ** -16 * np.linalg.norm(k.astype(np.float64))
     assert exact <= diag[0, 3] <= slack * (exact * (1 + 1e-4) + allowance) + 1e-12
+
+
+def _setup_ext(name, seed, S=16, **kw):
+    inp = small(name, seed, **kw)
+    wl = inp.wl
+    k, v = inp.kv()
+    q = inp.q()
+    caches = []
+    for ext in (False, True):
+        c = oracle.HqCache(wl.head_dim, wl.num_kv_heads, inp.num_pages, inp.hqmq_secondary(S),
+                           outliers=ext)
+        assert c.append(k, v, inp.page_table, np.zeros(wl.num_seqs, np.int32),
+                        valid=np.array(inp.seq_lens, np.int32)) == 0
+        caches.append(c)
+    return inp, caches, k, v, q
+
+
+def test_med3_extraction_in_the_hqmq_codec(oracle_lib):
+    """Method 3 over the HQMQ codec: the chunk oc_med3_chunk picks (pinned in
+    test_oracle_med3) is stored in fp16 (numpy's float16 of the inputs), takes
+    code 0 and radius 0 and reconstructs to its fp16 values; every other chunk
+    is coded exactly as without extraction; the tokens' key error falls where
+    a chunk is extracted and stays where none is."""
+    inp, (plain, ext), k, v, q = _setup_ext("serving", 0, spike_seq_frac=0.5)
+    wl = inp.wl
+    d, nc = wl.head_dim, wl.head_dim // 4
+    kf, vf = inp.as_f32(k), inp.as_f32(v)
+    bp, be = plain.block_bytes, ext.block_bytes
+    assert be == bp + 288
+    extracted = fell = 0
+    for b in range(wl.num_seqs):
+        for t in range(inp.seq_lens[b]):
+            page = inp.page_table[b, t // 16]
+            slot = t % 16
+            for h in range(wl.num_kv_heads):
+                P = plain.pool[(page * wl.num_kv_heads + h) * bp:][:bp]
+                X = ext.pool[(page * wl.num_kv_heads + h) * be:][:be]
+                os_ = X[bp:]
+                kh, vh = ext.read_token(page, h, slot)
+                for role, x, xh in ((0, kf[b, h, t], kh), (1, vf[b, h, t], vh)):
+                    cx = int(os_[role * 16 + slot])
+                    want = oracle.med3_chunk(x)
+                    assert cx == (0xFF if want < 0 else want)
+                    idx_p = P[role * 32 * nc:(role + 1) * 32 * nc].view(np.uint16).reshape(nc, 16)[:, slot]
+                    idx_e = X[role * 32 * nc:(role + 1) * 32 * nc].view(np.uint16).reshape(nc, 16)[:, slot]
+                    rad_p = P[64 * nc + role * 16 * nc:][:16 * nc].reshape(nc, 16)[:, slot]
+                    rad_e = X[64 * nc + role * 16 * nc:][:16 * nc].reshape(nc, 16)[:, slot]
+                    keep = np.arange(nc) != cx
+                    assert np.array_equal(idx_p[keep], idx_e[keep])
+                    assert np.array_equal(rad_p[keep], rad_e[keep])
+                    if cx != 0xFF:
+                        extracted += 1
+                        assert idx_e[cx] == 0 and rad_e[cx] == 0
+                        h16 = os_[32 + role * 128 + slot * 8:][:8].view(np.float16)
+                        assert np.array_equal(h16, x[4 * cx:4 * cx + 4].astype(np.float16))
+                        assert np.array_equal(xh[4 * cx:4 * cx + 4], h16.astype(np.float32))
+                eps_p = P[96 * nc + 64:][:64].view(np.float32)[slot]
+                eps_e = X[96 * nc + 64:][:64].view(np.float32)[slot]
+                if os_[slot] == 0xFF:
+                    assert eps_e == eps_p
+                else:
+                    fell += eps_e < eps_p
+    assert extracted > 10
+    assert fell > 0
+
+
+@pytest.mark.parametrize("name", ["llama8b", "serving", "tiny"])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_med3_hqmq_bound_dominates_observed_error(oracle_lib, name, seed):
+    inp, (plain, ext), k, v, q = _setup_ext(name, seed, spike_seq_frac=0.5)
+    o, bound, _, _ = ext.decode(q, inp.page_table, inp.seq_lens)
+    od = oracle.dense(q, k, v, inp.seq_lens)
+    err = max_err(od, o)
+    assert (bound >= err).all()
+    # the decode over the extraction cache is attention over its reconstructions
+    o2, _, _, _ = plain.decode(q, inp.page_table, inp.seq_lens)
+    assert np.isfinite(o2).all()
