@@ -61,9 +61,9 @@ def _variant(name: str):
     """'llama8b' -> ('llama8b', ''); 'llama8b+med3' -> ('llama8b', 'med3'): the
     workload with Med3x outlier extraction in the cache; 'llama8b+kqv' and
     'llama8b+hqmq': the workload's data and shapes in a cache of the KQV or the
-    HQMQ codec."""
+    HQMQ codec; 'llama8b+hqmq+med3': the HQMQ codec with Med3x."""
     base, _, ext = name.partition("+")
-    if base not in synth.WORKLOADS or ext not in ("", "med3", "kqv", "hqmq"):
+    if base not in synth.WORKLOADS or ext not in ("", "med3", "kqv", "hqmq", "hqmq+med3"):
         raise SystemExit(f"unknown workload {name}")
     return base, ext
 
@@ -77,13 +77,14 @@ def _describe(name: str) -> str:
                 f"Hkv={wl.num_kv_heads}, d={wl.head_dim}, {ctx}, KQV codec (Hadamard-rotated "
                 f"K and V; K 4-bit Lloyd-Max, V 3-bit Lloyd-Max + 1-bit QJL sketch; fp32 "
                 f"norms), 16-token pages (seeded permutation), tau={wl.tau}")
-    if ext == "hqmq":
+    if ext.startswith("hqmq"):
         ctx = f"ctx {wl.ctx}" if wl.ctx_min is None else f"ctx U[{wl.ctx_min},{wl.ctx}]"
         return (f"{wl.name} data and shapes: B={wl.num_seqs}, Hq={wl.num_q_heads}, "
                 f"Hkv={wl.num_kv_heads}, d={wl.head_dim}, {ctx}, HQMQ codec (4-channel "
                 f"chunks of K and V: 16-bit index into 2T x {HQ_S} secondary unit "
-                f"quaternions, fp8 E4M3 radius), 16-token pages (seeded permutation), "
-                f"tau={wl.tau}")
+                f"quaternions, fp8 E4M3 radius)"
+                + (", Med3x outlier extraction" if ext.endswith("med3") else "")
+                + f", 16-token pages (seeded permutation), tau={wl.tau}")
     return _workload_desc(wl) + (
         ", Med3x outlier extraction (one 4-channel chunk of K and of V per token in fp16)"
         if ext == "med3" else "")
@@ -333,7 +334,7 @@ class GpuStep:
         if codec == "kqv":
             ckw = dict(codec="kqv", rot_signs=inp.rotation_signs(), qjl_matrix=inp.qjl_matrix())
         elif codec == "hqmq":
-            ckw = dict(codec="hqmq", hq_secondary=inp.hqmq_secondary(HQ_S))
+            ckw = dict(codec="hqmq", hq_secondary=inp.hqmq_secondary(HQ_S), outliers=outliers)
         base = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, **ckw)
         zeros = torch.zeros(wl.num_seqs, dtype=torch.int32, device="cuda")
         base.append(self.kd, self.vd, self.pt, zeros, self.sl)
@@ -675,9 +676,10 @@ def measure_workload(name, args, world, rank, local):
     reps = max(2, math.ceil(3 * L2_BYTES / max(1, _cache_bytes_estimate(wl, ext))))
     reps = min(reps, 8)
     # the KQV and HQMQ codecs have no fused step: theirs is the append and the decode
-    two_calls = args.two_calls or ext in ("kqv", "hqmq")
-    st = GpuStep(base, args.seed, reps, two_calls=two_calls, outliers=ext == "med3",
-                 codec=ext if ext in ("kqv", "hqmq") else "int")
+    codec = "kqv" if ext == "kqv" else "hqmq" if ext.startswith("hqmq") else "int"
+    two_calls = args.two_calls or codec != "int"
+    st = GpuStep(base, args.seed, reps, two_calls=two_calls, outliers=ext.endswith("med3"),
+                 codec=codec)
     ms_total, dec_ms, clocks = _timed_replay(st, args, world, rank, local)
     e2e_ms, h2d, d2h = _e2e(st, args, world)
     lad_ms = None
@@ -709,7 +711,7 @@ def measure_workload(name, args, world, rank, local):
                      "frac_vs_spec": achieved / SPEC_HBM_GBS,
                      "spec_peak": SPEC_HBM_GBS,
                      "kernel": ("kqv_partial_kernel + kqv_merge_kernel" if ext == "kqv" else
-                                "hqmq_partial_kernel + hqmq_merge_kernel" if ext == "hqmq" else
+                                "hqmq_partial_kernel + hqmq_merge_kernel" if codec == "hqmq" else
                                 "decode_mma_kernel" + ("" if st.two_calls else " (append fused)")),
                      "kernel_ms": dec_ms,
                      "timing": ("events around every decode launch" if st.two_calls else
@@ -799,8 +801,8 @@ def _cache_bytes_estimate(wl, ext="") -> int:
         + 4 * wl.head_dim // 32 + (18 if ext == "med3" else 0)
     if ext == "kqv":
         per_tok = wl.head_dim + wl.head_dim // 8 + 16 + wl.head_dim // 64
-    if ext == "hqmq":
-        per_tok = 3 * wl.head_dim // 2 + 8 + wl.head_dim // 64
+    if ext.startswith("hqmq"):
+        per_tok = 3 * wl.head_dim // 2 + 8 + wl.head_dim // 64 + (18 if ext.endswith("med3") else 0)
     ctx = wl.ctx if wl.ctx_min is None else (wl.ctx + wl.ctx_min) // 2
     return wl.num_seqs * ctx * wl.num_kv_heads * per_tok
 
@@ -815,8 +817,9 @@ def _oracle_cache(workload: str, seed: int):
     if ext == "kqv":
         c = oracle.KqvCache(wl.head_dim, wl.num_kv_heads, inp.num_pages, inp.rotation_signs(),
                             inp.qjl_matrix())
-    elif ext == "hqmq":
-        c = oracle.HqCache(wl.head_dim, wl.num_kv_heads, inp.num_pages, inp.hqmq_secondary(HQ_S))
+    elif ext.startswith("hqmq"):
+        c = oracle.HqCache(wl.head_dim, wl.num_kv_heads, inp.num_pages, inp.hqmq_secondary(HQ_S),
+                           outliers=ext.endswith("med3"))
     else:
         c = oracle.Cache(wl.head_dim, wl.num_kv_heads, inp.num_pages, k_bits=wl.k_bits,
                          k_group=wl.k_group, k_rotate=wl.k_rotate, rot_signs=inp.rot_signs,
@@ -949,7 +952,8 @@ def main():
     ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--workload", default="llama8b",
-                    choices=sorted(synth.WORKLOADS) + [w + x for x in ("+med3", "+kqv", "+hqmq")
+                    choices=sorted(synth.WORKLOADS) + [w + x for x in ("+med3", "+kqv", "+hqmq",
+                                                                        "+hqmq+med3")
                                                         for w in sorted(synth.WORKLOADS)])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])

@@ -174,7 +174,7 @@ typedef struct kvq_cache {
  * +-i, +-j, +-k as p = 2 n + [negative]; p = 8..23 (+-1 +-i +-j +-k)/2 with
  * component n negative when bit n of p - 8 is set), q_s one of the hq_s
  * secondary units of the kv head and role (k_bits = v_bits = 6, k_group =
- * v_group = 4, k_rotate 0, outliers 0):
+ * v_group = 4, k_rotate 0; outliers 0, or 1 for Med3x over this codec):
  *   code i = 24 s + p maximizing <x, q_p q_s>, evaluated as <x conj(q_s),
  *   q_p>: y = x conj(q_s) with each component a sequential fmaf chain over
  *   x0..x3; the best axis unit is max_n |y_n| (first n on ties), the best
@@ -187,6 +187,10 @@ typedef struct kvq_cache {
  *   exact in fp32).
  *   A chunk with a non-finite r gets code 0, radius 0; a token with a
  *   non-finite value sets KVQ_ERR_RANGE and eps (K) and eta to +inf.
+ *   With outliers = 1 the Med3x chunk of K and of V (chosen as for the INT
+ *   codec) takes code 0 and radius 0, is stored in fp16 in the outlier
+ *   section appended to the block (the layout above) and reconstructs to its
+ *   fp16 values.
  * Block of one (page, kv head), 16 tokens, n = head_dim / 4 chunks,
  * chunk-major (token t of chunk ch at [ch][t]):
  *   [K codes u16 [n][16]][V codes u16 [n][16]][K radii e4m3 [n][16]]

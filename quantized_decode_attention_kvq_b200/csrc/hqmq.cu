@@ -123,6 +123,34 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return __half2float(__half(h));
 }
 
+// Med3x (Method 3) over one vector whose NCH chunk norms are held one per
+// lane by an aligned group of NCH lanes (the warp, or a half-warp): the chunk
+// with the largest norm above 3 x the median (0.5 (a + b) of the two middle
+// norms; equal norms ranked by chunk index), -1 for none or when a norm is NaN.
+template <int NCH>
+__device__ __forceinline__ int med3_group(float r, int lane) {
+  const int c = lane % NCH, g0 = lane - c;
+  const unsigned gmask = NCH == 32 ? 0xffffffffu : (0xffffu << g0);
+  if (__ballot_sync(0xffffffffu, isnan(r)) & gmask) return -1;
+  int rank = 0;
+#pragma unroll 8
+  for (int j = 0; j < NCH; ++j) {
+    const float rj = __shfl_sync(0xffffffffu, r, j, NCH);
+    rank += (rj < r) || (rj == r && j < c);
+  }
+  const unsigned lo_l = __ballot_sync(0xffffffffu, rank == NCH / 2 - 1) & gmask;
+  const unsigned hi_l = __ballot_sync(0xffffffffu, rank == NCH / 2) & gmask;
+  const float a = __shfl_sync(0xffffffffu, r, __ffs(lo_l) - 1);
+  const float b = __shfl_sync(0xffffffffu, r, __ffs(hi_l) - 1);
+  const float thr = __fmul_rn(3.0f, __fmul_rn(0.5f, __fadd_rn(a, b)));
+  float best = r > thr ? r : -1.0f;   // norms are >= 0
+#pragma unroll
+  for (int o = 1; o < NCH; o *= 2) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
+  if (best < 0.0f) return -1;
+  const unsigned who = __ballot_sync(0xffffffffu, r > thr && r == best) & gmask;
+  return __ffs(who) - 1 - g0;
+}
+
 }  // namespace
 
 // ================================================================ append =====
@@ -138,7 +166,7 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
   constexpr bool SPLIT = NC == 32;   // one role per item
   constexpr int GL = 8;              // lanes per 32-channel group of V chunks
   const AppendArgs& a = ha.a;
-  const HqLayout L{D};
+  const HqLayout L{D, ha.outliers};
   const int S = ha.S;
   __shared__ __align__(16) float stg[kHqAppendWarps][3][D];   // per warp: k, k - k^, v
   __shared__ float4 ssec[kHqAppendWarps][2 * KVQ_HQMQ_MAX_S];  // per warp: the item's units
@@ -188,10 +216,14 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
     for (int n = 0; n < 4; ++n) fin = fin && isfinite(x[n]);
     const float r = __fsqrt_rn(__fadd_rn(__fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[1], x[1])),
                                          __fadd_rn(__fmul_rn(x[2], x[2]), __fmul_rn(x[3], x[3]))));
+    // Med3x: the vector's extracted chunk (its lanes are this item's, or this
+    // half-warp's at d = 64)
+    const int cx = ha.outliers ? med3_group<SPLIT ? 32 : 16>(r, lane) : -1;
+    const bool ext = cx == ch;
     int code = 0;
     uint32_t rq = 0;
-    const bool rok = isfinite(r);
-    if (rok) {
+    const bool rok = ext || isfinite(r);
+    if (!ext && rok) {
       code = hq_direction(x, secs, S);
       rq = e4m3_rn(r);
     }
@@ -199,8 +231,32 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
     blk[(role ? L.vr() : L.kr()) + kPage * ch + slot] = (uint8_t)rq;
     const float4 cw = hq_round16(hq_codeword(code, secs[code / 24]));
     const float rv = e4m3_value(rq);
-    const float xh[4] = {__fmul_rn(rv, cw.x), __fmul_rn(rv, cw.y), __fmul_rn(rv, cw.z),
-                         __fmul_rn(rv, cw.w)};
+    float xh[4] = {__fmul_rn(rv, cw.x), __fmul_rn(rv, cw.y), __fmul_rn(rv, cw.z),
+                   __fmul_rn(rv, cw.w)};
+    bool bad16 = false;
+    if (ha.outliers) {
+      // the extracted chunk in fp16 (a value that is not finite or beyond
+      // 65504 is stored as 0 and is a range error); the section's chunk index
+      // and values are written for every token (zeros when none)
+      uint8_t* os = blk + L.out_off();
+      if (ch == 0) os[role * kPage + slot] = cx < 0 ? (uint8_t)kNoOutlier : (uint8_t)cx;
+      if (ch == (cx < 0 ? 0 : cx)) {
+        __half hv[4];
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+          hv[n] = __float2half_rn(0.f);
+          if (ext) {
+            if (!isfinite(x[n]) || fabsf(x[n]) > 65504.0f)
+              bad16 = true;
+            else
+              hv[n] = __float2half_rn(x[n]);
+            xh[n] = __half2float(hv[n]);
+          }
+        }
+        *reinterpret_cast<uint2*>(os + 2 * kPage + role * kPage * 8 + slot * 8) =
+            make_uint2(h2_as_u32(__halves2half2(hv[0], hv[1])), h2_as_u32(__halves2half2(hv[2], hv[3])));
+      }
+    }
     float err = 0.f, hi = 0.f, lo = 0.f;
     if (role == 0) {
 #pragma unroll
@@ -219,7 +275,7 @@ __global__ void __launch_bounds__(kHqAppendWarps * 32) hqmq_append_kernel(const 
     }
     const bool bad_k = __any_sync(0xffffffffu, role == 0 && !fin);
     const bool bad_v = __any_sync(0xffffffffu, role == 1 && !fin);
-    const bool bad_r = __any_sync(0xffffffffu, !rok);
+    const bool bad_r = __any_sync(0xffffffffu, !rok || bad16);
 #pragma unroll
     for (int o = 1; o < 32; o *= 2) err = fmaxf(err, __shfl_xor_sync(0xffffffffu, err, o));
 #pragma unroll
@@ -313,10 +369,10 @@ constexpr int kHqStages = 2;
 constexpr int kHqHdr = 16;   // floats: range max [NB], range min [NB], eta max
 __host__ __device__ constexpr int hq_rec_floats(int d) { return kHqHdr + kHqRows * 8 + kHqRows * d; }
 
-template <int D>
+template <int D, bool OUT>
 struct HqCfg {
   static constexpr int NC = D / 4;
-  static constexpr int BLOCK = 24 * D + 8 * kPage + D / 4;                  // HqLayout{D}.bytes()
+  static constexpr int BLOCK = 24 * D + 8 * kPage + D / 4 + (OUT ? kOutBytes : 0);   // HqLayout bytes()
   static constexpr int OFF_ST = 0;                                          // [warp][stage][BLOCK]
   static constexpr int OFF_W = OFF_ST + kHqWarps * kHqStages * BLOCK;       // [warp][16][4] f32
   static constexpr int OFF_Q = OFF_W + kHqWarps * kPage * kHqRows * 4;      // q [chunk][row] float4
@@ -332,14 +388,14 @@ struct HqCfg {
   static __host__ __device__ constexpr int smem(int S) { return 128 + OFF_TAB + 2 * 24 * S * 8; }
 };
 
-template <int D>
+template <int D, bool OUT>
 __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const HqDecodeArgs ha) {
-  using C = HqCfg<D>;
+  using C = HqCfg<D, OUT>;
   constexpr int NC = C::NC, NB = D / 32, E = D / 32;
   constexpr int HC = NC / 2;          // chunks per half-warp in the scores
   constexpr int TPL = 16 * NC / 32;   // tokens per lane in PV
   const DecodeArgs& a = ha.a;
-  const HqLayout L{D};
+  const HqLayout L{D, OUT ? 1 : 0};
   const int S = ha.S;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
@@ -519,6 +575,21 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           }
         }
       }
+      if constexpr (OUT) {
+        // token t's extracted key chunk, kept in fp16 (its code and radius are
+        // 0): its score term, added by the half-warp whose chunks hold it
+        const uint8_t* os = blk + L.out_off();
+        const int cx = os[t];
+        if (cx < NC && (hc ? cx >= HC : cx < HC)) {
+          const float4 k16 = hq_unpack16(*reinterpret_cast<const uint2*>(os + 2 * kPage + t * 8));
+#pragma unroll
+          for (int r = 0; r < kHqRows; ++r) {
+            const float4 qv = qs[cx * kHqRows + r];
+            s2[r] = fma2(make_float2(qv.x, qv.y), make_float2(k16.x, k16.y), s2[r]);
+            s2[r] = fma2(make_float2(qv.z, qv.w), make_float2(k16.z, k16.w), s2[r]);
+          }
+        }
+      }
       float s4[kHqRows];
 #pragma unroll
       for (int r = 0; r < kHqRows; ++r) {
@@ -606,6 +677,27 @@ __global__ void __launch_bounds__(kHqWarps * 32, 4) hqmq_partial_kernel(const Hq
           for (int r = 0; r < kHqRows; ++r) {
             acc[r][0] = fma2(w2[r], v01, acc[r][0]);
             acc[r][1] = fma2(w2[r], v23, acc[r][1]);
+          }
+        }
+        if constexpr (OUT) {
+          // extracted value chunks (code and radius 0) of this lane's chunk:
+          // w * v16 for those tokens
+          const uint8_t* os = blk + L.out_off();
+#pragma unroll
+          for (int tt = 0; tt < TPL; ++tt) {
+            const int tk = t0 + tt;
+            if (os[kPage + tk] == pc) {
+              const float4 v16 =
+                  hq_unpack16(*reinterpret_cast<const uint2*>(os + 2 * kPage + kPage * 8 + tk * 8));
+              const float4 w4 = w4p[tt];
+              const float wr[kHqRows] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+              for (int r = 0; r < kHqRows; ++r) {
+                const float2 w2 = make_float2(wr[r], wr[r]);
+                acc[r][0] = fma2(w2, make_float2(v16.x, v16.y), acc[r][0]);
+                acc[r][1] = fma2(w2, make_float2(v16.z, v16.w), acc[r][1]);
+              }
+            }
           }
         }
       }
@@ -772,27 +864,36 @@ __global__ void __launch_bounds__(kHqWarps * 32) hqmq_merge_kernel(const HqDecod
   }
 }
 
-const void* hqmq_partial_kernel(int d) {
-  if (d == 128) return reinterpret_cast<const void*>(hqmq_partial_kernel<128>);
-  if (d == 64) return reinterpret_cast<const void*>(hqmq_partial_kernel<64>);
+const void* hqmq_partial_kernel(int d, int out) {
+  if (d == 128) return out ? reinterpret_cast<const void*>(hqmq_partial_kernel<128, true>)
+                           : reinterpret_cast<const void*>(hqmq_partial_kernel<128, false>);
+  if (d == 64) return out ? reinterpret_cast<const void*>(hqmq_partial_kernel<64, true>)
+                          : reinterpret_cast<const void*>(hqmq_partial_kernel<64, false>);
   return nullptr;
 }
-int hqmq_partial_smem(int d, int S) {
-  return d == 128 ? HqCfg<128>::smem(S) : HqCfg<64>::smem(S);
+int hqmq_partial_smem(int d, int S, int out) {
+  if (d == 128) return out ? HqCfg<128, true>::smem(S) : HqCfg<128, false>::smem(S);
+  return out ? HqCfg<64, true>::smem(S) : HqCfg<64, false>::smem(S);
 }
 int hqmq_record_floats(int d) { return hq_rec_floats(d); }
 int hqmq_threads() { return kHqWarps * 32; }
+
+template <int D, bool OUT>
+static void launch_hqmq_partial(const HqDecodeArgs& a, dim3 grid, cudaStream_t stream) {
+  hqmq_partial_kernel<D, OUT><<<grid, kHqWarps * 32, HqCfg<D, OUT>::smem(a.S), stream>>>(a);
+}
 
 cudaError_t launch_hqmq_decode(const HqDecodeArgs& a, int d, int units, int splits,
                                cudaStream_t stream) {
   if (units == 0) return cudaSuccess;
   const dim3 grid((unsigned)units, (unsigned)splits, 1);
-  const size_t smem = (size_t)hqmq_partial_smem(d, a.S);
   if (d == 128) {
-    hqmq_partial_kernel<128><<<grid, kHqWarps * 32, smem, stream>>>(a);
+    if (a.outliers) launch_hqmq_partial<128, true>(a, grid, stream);
+    else launch_hqmq_partial<128, false>(a, grid, stream);
     hqmq_merge_kernel<128><<<units, kHqWarps * 32, 0, stream>>>(a);
   } else if (d == 64) {
-    hqmq_partial_kernel<64><<<grid, kHqWarps * 32, smem, stream>>>(a);
+    if (a.outliers) launch_hqmq_partial<64, true>(a, grid, stream);
+    else launch_hqmq_partial<64, false>(a, grid, stream);
     hqmq_merge_kernel<64><<<units, kHqWarps * 32, 0, stream>>>(a);
   } else {
     return cudaErrorInvalidValue;

@@ -56,7 +56,7 @@ int check_hqmq(const kvq_cache* c) {
   if (c->k_bits != 6 || c->v_bits != 6 || c->k_group != 4 || c->v_group != 4)
     return fail(KVQ_ERR_UNSUPPORTED, "the HQMQ codec takes k_bits = v_bits = 6 and groups of 4");
   if (c->k_rotate != 0) return fail(KVQ_ERR_UNSUPPORTED, "the HQMQ codec does not rotate keys");
-  if (c->outliers != 0) return fail(KVQ_ERR_UNSUPPORTED, "the HQMQ codec has no outlier extraction");
+  if (c->outliers != 0 && c->outliers != 1) return fail(KVQ_ERR_INVALID_ARG, "outliers not 0/1");
   if (!c->hq_sec) return fail(KVQ_ERR_INVALID_ARG, "the HQMQ codec needs the secondary units");
   if (c->hq_s < 1 || c->hq_s > KVQ_HQMQ_MAX_S)
     return fail(KVQ_ERR_UNSUPPORTED, "hq_s %d unsupported (1..%d)", c->hq_s, KVQ_HQMQ_MAX_S);
@@ -200,22 +200,22 @@ int kqv_occupancy(int d, int* occ) {
 
 // blocks of the HQMQ codec's partial decode kernel resident per SM (its shared
 // memory grows with the secondary set)
-int hqmq_occupancy(int d, int S, int* occ) {
+int hqmq_occupancy(int d, int S, int out, int* occ) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int>, int> cache;
+  static std::map<std::tuple<int, int, int, int>, int> cache;
   int dev = 0;
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lk(mu);
-  auto key = std::make_tuple(dev, d, S);
+  auto key = std::make_tuple(dev, d, S, out);
   auto it = cache.find(key);
   if (it == cache.end()) {
-    const void* k = hqmq_partial_kernel(d);
-    const int smem = hqmq_partial_smem(d, KVQ_HQMQ_MAX_S);
+    const void* k = hqmq_partial_kernel(d, out);
+    const int smem = hqmq_partial_smem(d, KVQ_HQMQ_MAX_S, out);
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     int n = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, hqmq_threads(),
-                                                      hqmq_partial_smem(d, S));
+                                                      hqmq_partial_smem(d, S, out));
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     it = cache.emplace(key, n < 1 ? 1 : n).first;
   }
@@ -235,7 +235,7 @@ int make_plan(const kvq_cache* c, int num_seqs, int max_pages, Plan* p) {
   if (rc) return rc;
   int occ = 1;
   if ((rc = kqv    ? kqv_occupancy(c->head_dim, &occ)
-            : hqmq ? hqmq_occupancy(c->head_dim, c->hq_s, &occ)
+            : hqmq ? hqmq_occupancy(c->head_dim, c->hq_s, c->outliers, &occ)
                    : decode_occupancy(v, &occ)))
     return rc;
   const int64_t units = (int64_t)num_seqs * c->num_kv_heads;
@@ -356,6 +356,7 @@ int decode_impl(const kvq_cache* cache, const void* q, int q_dtype, int32_t num_
     ha.sec = cache->hq_sec;
     ha.S = cache->hq_s;
     ha.nsp = plan.splits;
+    ha.outliers = cache->outliers;
     cudaError_t e = launch_hqmq_decode(ha, cache->head_dim, (int)units, plan.splits, stream);
     if (e != cudaSuccess) return cuda_fail(e, "HQMQ decode launch");
     return KVQ_OK;
@@ -402,9 +403,9 @@ size_t kvq_block_bytes(const kvq_cache* cache) {
   }
   if (cache->codec == KVQ_CODEC_HQMQ) {
     if (cache->k_bits != 6 || cache->v_bits != 6 || cache->k_group != 4 || cache->v_group != 4 ||
-        cache->k_rotate != 0 || cache->outliers != 0)
+        cache->k_rotate != 0 || (cache->outliers != 0 && cache->outliers != 1))
       return 0;
-    return (size_t)HqLayout{cache->head_dim}.bytes();
+    return (size_t)HqLayout{cache->head_dim, cache->outliers}.bytes();
   }
   if (cache->codec != KVQ_CODEC_INT || (cache->k_bits != 8 && cache->k_bits != 4)) return 0;
   if (cache->k_group != 32 && cache->k_group != 64 && cache->k_group != 128) return 0;
@@ -471,6 +472,7 @@ int kvq_quantize_append(const kvq_cache* cache, const void* k, const void* v, in
     ha.a = a;
     ha.sec = cache->hq_sec;
     ha.S = cache->hq_s;
+    ha.outliers = cache->outliers;
     cudaError_t e = launch_hqmq_append(ha, cache->head_dim, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "HQMQ append kernel launch");
     return KVQ_OK;

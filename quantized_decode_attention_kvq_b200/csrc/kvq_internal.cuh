@@ -209,9 +209,11 @@ int kqv_threads();
 // ---- the HQMQ codec (hqmq.cu) ------------------------------------------------
 // Byte layout of one (page, kv head) block, chunk-major (token t of chunk c at
 // [c][t]): K codes u16, V codes u16, K radii e4m3, V radii e4m3, then per
-// token |k| and eps (fp32), then the block's v^ max / min per 32-channel group.
+// token |k| and eps (fp32), then the block's v^ max / min per 32-channel group,
+// then (out) the Med3x section of the Tier-1 layout.
 struct HqLayout {
   int d;
+  int out = 0;
   __host__ __device__ int nc() const { return d / 4; }
   __host__ __device__ int vi() const { return kPage * nc() * 2; }
   __host__ __device__ int kr() const { return kPage * nc() * 4; }
@@ -219,25 +221,28 @@ struct HqLayout {
   __host__ __device__ int kn() const { return vr() + kPage * nc(); }
   __host__ __device__ int ke() const { return kn() + 4 * kPage; }
   __host__ __device__ int rg() const { return kn() + 8 * kPage; }
-  __host__ __device__ int bytes() const { return rg() + (d / 32) * 8; }
+  __host__ __device__ int out_off() const { return rg() + (d / 32) * 8; }
+  __host__ __device__ int bytes() const { return out_off() + (out ? kOutBytes : 0); }
 };
 struct HqAppendArgs {
   AppendArgs a;
   const float* sec;   // [hkv][2][S][4] unit quaternions
   int S;
+  int outliers;       // Med3x extraction (0 or 1)
 };
 struct HqDecodeArgs {
   DecodeArgs a;       // out, bound, flags, part as for the Tier-1 decode; no fused append
   const float* sec;
   int S;
   int nsp;            // splits of the partial grid (records per unit)
+  int outliers;
 };
 cudaError_t launch_hqmq_append(const HqAppendArgs& a, int d, cudaStream_t s);
 // the partial kernel over (unit, split), then the merge per unit
 cudaError_t launch_hqmq_decode(const HqDecodeArgs& a, int d, int units, int splits,
                                cudaStream_t s);
-const void* hqmq_partial_kernel(int d);
-int hqmq_partial_smem(int d, int S);
+const void* hqmq_partial_kernel(int d, int out);
+int hqmq_partial_smem(int d, int S, int out);
 int hqmq_record_floats(int d);
 int hqmq_threads();
 

@@ -305,7 +305,7 @@ class PagedCache:
         if codec == "kqv":
             k_bits, v_bits, k_group, v_group, k_rotate = 4, 3, head_dim, head_dim, True
         hq_s = 0
-        if codec == "hqmq":
+        if codec == "hqmq":   # outliers: Med3x over the HQMQ codec
             k_bits, v_bits, k_group, v_group, k_rotate = 6, 6, 4, 4, False
             hq_s = int(np.asarray(hq_secondary).shape[2])   # S secondary units per (head, role)
         self.desc = kvq_cache(num_kv_heads, head_dim, PAGE_SIZE, num_pages, k_bits, k_group,

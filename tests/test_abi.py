@@ -95,6 +95,9 @@ def test_hqmq_block_size_and_checks(kvq):
     assert kvq.kvq_block_bytes(_desc(kvq, **hq)) == 24 * 128 + 128 + 32 == 3232
     assert kvq.kvq_block_bytes(_desc(kvq, head_dim=64, **hq)) == 24 * 64 + 128 + 16 == 1680
     assert kvq.kvq_block_bytes(_desc(kvq, **{**hq, "k_bits": 8})) == 0
+    # Med3x over the HQMQ codec: the same 288-byte outlier section
+    assert kvq.kvq_block_bytes(_desc(kvq, outliers=1, **hq)) == 3232 + 288
+    assert kvq.kvq_block_bytes(_desc(kvq, head_dim=64, outliers=1, **hq)) == 1680 + 288
     assert kvq.kvq_block_bytes(_desc(kvq, k_rotate=1, rot_signs=0x3000, **hq)) == 0
     d = _desc(kvq, **hq)
     assert kvq.kvq_adaptive_work_size(d, 2, 1, 32, 4) == 0

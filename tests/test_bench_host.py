@@ -29,6 +29,8 @@ def test_workload_variants():
     assert bench._variant("llama8b+kqv") == ("llama8b", "kqv")
     assert bench._variant("llama8b+hqmq") == ("llama8b", "hqmq")
     assert "HQMQ" in bench._describe("llama8b+hqmq")
+    assert bench._variant("llama8b+hqmq+med3") == ("llama8b", "hqmq+med3")
+    assert "Med3x" in bench._describe("llama8b+hqmq+med3")
     assert "Med3x" in bench._describe("serving+med3")
     assert "KQV" in bench._describe("llama8b+kqv")
     for bad in ("llama8b+x", "nosuch", "nosuch+med3"):

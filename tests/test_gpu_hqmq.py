@@ -30,19 +30,19 @@ def _cuda():
     build.build()
 
 
-def _caches(inp, S=S_DEFAULT):
+def _caches(inp, S=S_DEFAULT, outliers=False):
     from quantized_decode_attention_kvq_b200 import kvq
     wl = inp.wl
     sec = inp.hqmq_secondary(S)
     g = kvq.PagedCache(wl.num_kv_heads, wl.head_dim, inp.num_pages, codec="hqmq",
-                       hq_secondary=sec)
-    o = oracle.HqCache(wl.head_dim, wl.num_kv_heads, inp.num_pages, sec)
+                       hq_secondary=sec, outliers=outliers)
+    o = oracle.HqCache(wl.head_dim, wl.num_kv_heads, inp.num_pages, sec, outliers=outliers)
     return g, o
 
 
-def _run(inp, k, v, q, tau=None, seqs=None, bound_only=False, S=S_DEFAULT):
+def _run(inp, k, v, q, tau=None, seqs=None, bound_only=False, S=S_DEFAULT, outliers=False):
     wl = inp.wl
-    g, o = _caches(inp, S)
+    g, o = _caches(inp, S, outliers)
     pt = torch.from_numpy(inp.page_table).cuda()
     sl = torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda")
     g.append(to_torch(k), to_torch(v), pt, torch.zeros(wl.num_seqs, dtype=torch.int32,
@@ -290,3 +290,41 @@ def test_exact_fallback_on_an_hqmq_cache():
     od = oracle.dense(q, k, v, inp.seq_lens)
     assert max_err(od[fl], res[fl]).max() <= 1e-4
     assert np.array_equal(res[~fl], decoded[~fl].astype(np.float64))
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("seed", [0, 1])
+def test_med3_over_hqmq_parity(name, seed):
+    """Med3x over the HQMQ codec (the page's combination): pool bytes (the
+    outlier section included) and eta bit for bit, the decode against the
+    oracle, and the bound against dense attention."""
+    inp = small(name, seed, **SPIKES)
+    k, v = inp.kv()
+    q = inp.q()
+    r = _run(inp, k, v, q, outliers=True)
+    assert r["err"] == 0
+    pool = r["cache"].pool.cpu().numpy()
+    assert np.array_equal(pool, r["oracle"].pool), np.flatnonzero(pool != r["oracle"].pool)[:10]
+    assert np.array_equal(r["cache"].eta.cpu().numpy().view(np.uint32),
+                          r["oracle"].eta.view(np.uint32))
+    _check(inp, r, q, inp.wl.tau, f"hqmq+med3 {name} seed={seed}")
+    o_dense = oracle.dense(q, k, v, inp.seq_lens)
+    assert (max_err(o_dense, r["out"]) <= r["bound"]).all()
+
+
+def test_med3_over_hqmq_full_size_sampled():
+    inp = synth.make("llama8b", 0)
+    wl = inp.wl
+    k, v = inp.kv()
+    q = inp.q()
+    seqs = [0, wl.num_seqs - 1]
+    r = _run(inp, k, v, q, seqs=seqs, outliers=True)
+    assert r["err"] == 0
+    bb = r["oracle"].block_bytes
+    gpool = r["cache"].pool.cpu().numpy().reshape(inp.num_pages, wl.num_kv_heads, bb)
+    opool = r["oracle"].pool.reshape(inp.num_pages, wl.num_kv_heads, bb)
+    pages = np.concatenate([inp.page_table[s, :inp.pages_per_seq[s]] for s in seqs])
+    assert np.array_equal(gpool[pages], opool[pages])
+    rows, _ = _check(inp, r, q, wl.tau, "hqmq+med3 llama8b full size")
+    o_dense = oracle.dense(q[seqs], k[seqs], v[seqs], np.array(inp.seq_lens)[seqs])
+    assert (max_err(o_dense, r["out"][rows]) <= r["bound"][rows]).all()
