@@ -127,11 +127,13 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
 // lane by an aligned group of NCH lanes (the warp, or a half-warp): the chunk
 // with the largest norm above 3 x the median (0.5 (a + b) of the two middle
 // norms; equal norms ranked by chunk index), -1 for none or when a norm is NaN.
+// Every lane of the warp runs every shuffle and ballot (the two half-warps'
+// groups may have different answers), and the answer is chosen at the end.
 template <int NCH>
 __device__ __forceinline__ int med3_group(float r, int lane) {
   const int c = lane % NCH, g0 = lane - c;
   const unsigned gmask = NCH == 32 ? 0xffffffffu : (0xffffu << g0);
-  if (__ballot_sync(0xffffffffu, isnan(r)) & gmask) return -1;
+  const bool any_nan = (__ballot_sync(0xffffffffu, isnan(r)) & gmask) != 0u;
   int rank = 0;
 #pragma unroll 8
   for (int j = 0; j < NCH; ++j) {
@@ -140,15 +142,16 @@ __device__ __forceinline__ int med3_group(float r, int lane) {
   }
   const unsigned lo_l = __ballot_sync(0xffffffffu, rank == NCH / 2 - 1) & gmask;
   const unsigned hi_l = __ballot_sync(0xffffffffu, rank == NCH / 2) & gmask;
-  const float a = __shfl_sync(0xffffffffu, r, __ffs(lo_l) - 1);
-  const float b = __shfl_sync(0xffffffffu, r, __ffs(hi_l) - 1);
+  // (a group with a NaN norm may have no such lanes: any lane will do, the
+  // answer is -1 then)
+  const float a = __shfl_sync(0xffffffffu, r, lo_l ? __ffs(lo_l) - 1 : g0);
+  const float b = __shfl_sync(0xffffffffu, r, hi_l ? __ffs(hi_l) - 1 : g0);
   const float thr = __fmul_rn(3.0f, __fmul_rn(0.5f, __fadd_rn(a, b)));
   float best = r > thr ? r : -1.0f;   // norms are >= 0
 #pragma unroll
   for (int o = 1; o < NCH; o *= 2) best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, o));
-  if (best < 0.0f) return -1;
   const unsigned who = __ballot_sync(0xffffffffu, r > thr && r == best) & gmask;
-  return __ffs(who) - 1 - g0;
+  return any_nan || best < 0.0f || who == 0u ? -1 : __ffs(who) - 1 - g0;
 }
 
 }  // namespace
