@@ -3,24 +3,28 @@
 // a quaternion split into its radius and its direction on S^3; the direction
 // is coded by the product codebook {q_p q_s} of the 24 Hurwitz units (the
 // binary tetrahedral group 2T) and a random secondary set per (kv head, role),
-// the radius in fp8 E4M3.  The certified bound of "Runtime-Certified
-// Bounded-Error Quantized Attention" (Methodology 2) carries over with a
-// per-token Euclidean key error.
+// the radius in fp8 E4M3; optionally with Method 3's Med3x chunks kept in
+// fp16.  The certified bound of "Runtime-Certified Bounded-Error Quantized
+// Attention" (Methodology 2) carries over with a per-token Euclidean key
+// error.
 //
 //   hqmq_append_kernel    one warp per (token, kv head, role) at d = 128 (per
 //                         (token, kv head) at d = 64): each lane codes one
 //                         (chunk, role) pair (the direction through
 //                         y = x conj(q_s) and 2T's closed-form best unit, the
-//                         radius by the fp8 conversion), then |k|, eps and
-//                         |v| as sequential chains over the channels, eta and
-//                         the value range
+//                         radius by the fp8 conversion; or the chunk in fp16
+//                         when Med3x extracts it), then |k|, eps and |v| as
+//                         sequential chains over the channels, eta and the
+//                         value range
 //   hqmq_partial_kernel   grid (sequence x kv head, split), 4 warps, each
 //                         streaming its pages through a 2-stage bulk-copy
 //                         ring; the CTA builds its kv head's 2 x 24 S
-//                         codewords (fp16) in shared memory first.  Scores with one
-//                         lane per (token, half of the chunks), PV with one
-//                         lane per chunk, online softmax and the bound's sums
-//                         as for the other codecs
+//                         codewords (fp16) in shared memory first.  Scores
+//                         with one lane per (token, half of the chunks), PV
+//                         with one lane per chunk (packed fp32x2 arithmetic),
+//                         online softmax and the bound's sums as for the
+//                         other codecs; the extracted chunks' terms in the
+//                         Med3x instantiation
 //   hqmq_merge_kernel     per (sequence, kv head): the split records' merge,
 //                         the output, the bound and the flag
 // The arithmetic that decides a code or a stored value (the chunk norm, the
