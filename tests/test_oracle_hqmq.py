@@ -400,3 +400,56 @@ def test_med3_hqmq_bound_dominates_observed_error(oracle_lib, name, seed):
     # the decode over the extraction cache is attention over its reconstructions
     o2, _, _, _ = plain.decode(q, inp.page_table, inp.seq_lens)
     assert np.isfinite(o2).all()
+
+
+# ------------------------------------------------- planted mistakes ---------
+# (name, text in kvq_oracle.c, replacement): plausible slips in the HQMQ
+# oracle, each of which one of the pins above must catch.
+MUTANTS = [
+    ("y_component_sign", "y[1] = fmaf(x[3], b[2], fmaf(-x[2], b[3], fmaf(x[1], b[0], -x[0] * b[1])));",
+     "y[1] = fmaf(x[3], b[2], fmaf(x[2], b[3], fmaf(x[1], b[0], -x[0] * b[1])));"),
+    ("half_unit_scale", "float h = 0.5f * (((a[0] + a[1]) + a[2]) + a[3]);",
+     "float h = 0.45f * (((a[0] + a[1]) + a[2]) + a[3]);"),
+    ("product_sign", "{a[0] * b[1], a[1] * b[0], a[2] * b[3], -(a[3] * b[2])},",
+     "{a[0] * b[1], a[1] * b[0], -(a[2] * b[3]), (a[3] * b[2])},"),
+    ("primary_sign_bits", "q[n] = ((p - 8) >> n) & 1 ? -0.5f : 0.5f;",
+     "q[n] = ((p - 8) >> (3 - n)) & 1 ? -0.5f : 0.5f;"),
+    ("e4m3_ties_up", "return (uint8_t)((lo & 1) ? lo + 1 : lo);", "return (uint8_t)(lo + 1);"),
+    ("eps_doubled", "nextafterf(fmaf(en, 1.0f / 65536.0f, en), INFINITY)",
+     "nextafterf(2.0f * en, INFINITY)"),
+    ("delta_scaled_norm", "dl[j] = OC_KAPPA * sc * qn2 *", "dl[j] = OC_KAPPA * sc * 1.5 * qn2 *"),
+    ("med3_chunk_dropped", "xh[4 * cx + i] = (float)oc_f16_value(h);", "xh[4 * cx + i] = 0.0f;"),
+]
+
+# the pins a mutant is run against, cheapest first
+PROBES = [
+    (test_primary_units_are_2T, {}),
+    (test_e4m3_radius, {}),
+    (test_codewords_are_products_and_isometric_copies, {}),
+    (test_direction_is_the_best_codeword, {"S": 7}),
+    (test_exact_recovery_of_representable_chunks, {}),
+    (test_delta_is_tight_for_a_query_along_the_error, {}),
+    (test_codes_radii_and_error_annotations, {"name": "tiny"}),
+    (test_med3_extraction_in_the_hqmq_codec, {}),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return str(tmp_path_factory.mktemp("hqmq_mutants"))
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(oracle_lib, mutant_dir, name, old, new):
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation target of {name} not found once in the oracle"
+    so = oracle.compile_variant(src.replace(old, new), mutant_dir, name)
+    caught = None
+    with oracle.library_override(so):
+        for fn, kw in PROBES:
+            try:
+                fn(oracle_lib, **kw)
+            except AssertionError:
+                caught = fn.__name__
+                break
+    assert caught, f"no pin catches the planted mistake {name}"
