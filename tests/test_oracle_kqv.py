@@ -15,7 +15,9 @@ Against things other than its own code:
   (pi/2)|r|^2 |y|^2 / m (less <y, r>^2 / m) over many draws of S;
 * an independent numpy reader of the documented block layout reproduces the
   decode, and the stored eps, eta and value range cover the errors;
-* the bound never falls below the error against exact attention.
+* the bound never falls below the error against exact attention, and Delta
+  is tight for a rotated query that makes Hoelder's inequality an equality;
+* five planted mistakes compiled into copies of the oracle are each caught.
 """
 
 import math
@@ -256,3 +258,95 @@ def test_bound_dominates_observed_error(oracle_lib, name, seed):
     err = max_err(od, o)
     assert (bound >= err).all()
     assert (diag[:, 0] <= 1.0).all() and (diag[:, 1] >= 0).all() and (diag[:, 2] > 0).all()
+
+
+def test_delta_is_tight_for_a_one_hot_rotated_query(oracle_lib):
+    """One token: with q' (the rotated query) one-hot on the channel where
+    |k' - k^'| is largest, |z - z^| = s |q'| eps exactly (Hoelder's inequality
+    is tight), and the oracle's Delta exceeds it by no more than kappa and the
+    rotation allowance (a Delta with |q'|_2 in place of |q'|_1, a factor 2 or a
+    dropped term fails one side)."""
+    d = 128
+    inp = small("llama8b", 0)
+    rng = np.random.default_rng(8)
+    k = rng.standard_normal(d).astype(np.float32)
+    v = rng.standard_normal(d).astype(np.float32)
+    sig = inp.rotation_signs()
+    c = oracle.KqvCache(d, 1, 1, sig, inp.qjl_matrix())
+    assert c.append(k.reshape(1, 1, 1, d), v.reshape(1, 1, 1, d), np.zeros((1, 1), np.int32),
+                    np.zeros(1, np.int32)) == 0
+    R = _Reader(c)
+    tok = R.token(0, 0, 0)
+    kcent, _ = oracle.kqv_tables(4, d)
+    kr = _rot64(k, sig.astype(np.float64))
+    kh = float(tok["nk"]) * kcent[tok["kc"]].astype(np.float64)
+    cstar = int(np.abs(kr - kh).argmax())
+    # q with q' = 3 e_cstar: the inverse rotation is sigma o (H x') / sqrt(d)
+    onehot = np.zeros(d)
+    onehot[cstar] = 3.0
+    H = scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d)
+    q = (sig * (H @ onehot)).astype(np.float32)
+    qr = _rot64(q, sig.astype(np.float64))
+    _, _, _, diag = c.decode(q.reshape(1, 1, 1, d), np.zeros((1, 1), np.int32),
+                             np.array([1], np.int32))
+    s = float(oracle.default_scale(d))
+    exact = s * abs(qr @ (kr - kh))
+    e_inf = np.abs(kr - kh).max()
+    assert exact == pytest.approx(s * 3.0 * e_inf, rel=1e-5)
+    allowance = s * np.linalg.norm(qr) * 2 ** -16 * float(tok["nk"])
+    slack = 1 + 2 ** -10
+    assert exact * (1 - 1e-5) <= diag[0, 3] <= slack * (exact * (1 + 1e-4) + allowance) + 1e-12
+    # q' = 3 sign(k' - k^') on every channel: |q' . e| = 3 |e|_1, which only
+    # the 1-norm of q' covers (|q'|_2 eps falls short for a spread error)
+    q2 = (sig * (H @ (3.0 * np.sign(kr - kh)))).astype(np.float32)
+    qr2 = _rot64(q2, sig.astype(np.float64))
+    _, _, _, diag2 = c.decode(q2.reshape(1, 1, 1, d), np.zeros((1, 1), np.int32),
+                              np.array([1], np.int32))
+    exact2 = s * abs(qr2 @ (kr - kh))
+    assert exact2 == pytest.approx(s * 3.0 * np.abs(kr - kh).sum(), rel=1e-4)
+    assert diag2[0, 3] >= exact2
+
+
+# ------------------------------------------------- planted mistakes ---------
+# (name, text in kvq_oracle.c, replacement): plausible slips in the KQV
+# oracle, each of which one of the pins above must catch.
+MUTANTS = [
+    ("sketch_bit_sign", "if (oq_dot(S + (int64_t)i * d, r, d) >= 0.0f) bits[i / 8]",
+     "if (oq_dot(S + (int64_t)i * d, r, d) < 0.0f) bits[i / 8]"),
+    ("codebook_scale", "for (int i = 0; i < L; ++i) cent[i] = (float)(c[i] / sd);",
+     "for (int i = 0; i < L; ++i) cent[i] = (float)(c[i] / d);"),
+    ("eps_not_inf_norm", "if (nk > 0.0f && e > eps) eps = e;", "if (nk > 0.0f) eps = e;"),
+    ("delta_l2_for_l1", "dl[j] = OC_KAPPA * sc * (qn1 * (double)oq_rdf(",
+     "dl[j] = OC_KAPPA * sc * (qn2 * (double)oq_rdf("),
+    ("decode_sketch_constant", "double rho = sqrt(OQ_PI / 2.0) / d * (double)oq_rdf(",
+     "double rho = sqrt(OQ_PI) / d * (double)oq_rdf("),
+]
+
+# the pins a mutant is run against, cheapest first
+PROBES = [
+    (test_codes_bits_and_error_annotations, {"name": "tiny"}),
+    (test_decode_matches_an_independent_reader, {"name": "tiny"}),
+    (test_delta_is_tight_for_a_one_hot_rotated_query, {}),
+    (test_gaussian_codebook_close_to_the_beta_marginal, {"d": 64}),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return str(tmp_path_factory.mktemp("kqv_mutants"))
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(oracle_lib, mutant_dir, name, old, new):
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation target of {name} not found once in the oracle"
+    so = oracle.compile_variant(src.replace(old, new), mutant_dir, name)
+    caught = None
+    with oracle.library_override(so):
+        for fn, kw in PROBES:
+            try:
+                fn(oracle_lib, **kw)
+            except AssertionError:
+                caught = fn.__name__
+                break
+    assert caught, f"no pin catches the planted mistake {name}"
