@@ -13,7 +13,9 @@ Against things other than its own code:
   sequences and raises it nowhere; the bound dominates the error against
   exact attention;
 * with no chunk above the threshold, the decode equals the one without
-  extraction.
+  extraction;
+* eta covers the fp16 rounding of an extracted value (a hand case);
+* four planted mistakes compiled into copies of the oracle are each caught.
 """
 
 import math
@@ -162,3 +164,60 @@ def test_no_outlier_means_same_decode(oracle_lib):
         res.append(c.decode(q, inp.page_table, inp.seq_lens))
     if all(oracle.med3_chunk(x) < 0 for x in flat):
         assert np.array_equal(res[0][0], res[1][0]) and np.array_equal(res[0][1], res[1][1])
+
+
+def test_eta_covers_the_fp16_rounding_of_an_extracted_value(oracle_lib):
+    """d = 64: V = 0.25 everywhere except channel 9 = 50.0123, which fp16
+    rounds to 50.0 (spacing 2^-5 there); the other values are exact for the
+    INT4 group codec (a constant group), so eta is the fp16 error, 0.0123,
+    raised by one ulp."""
+    d = 64
+    k = np.ones(d, np.float32)
+    v = np.full(d, 0.25, np.float32)
+    v[9] = np.float32(50.0123)
+    c = _one_token_cache(k, v, d)
+    err16 = abs(float(v[9]) - float(np.float16(v[9])))
+    assert 0.012 < err16 < 0.013
+    assert err16 <= c.eta[0, 0] <= err16 * (1 + 1e-6) + 1e-30
+
+
+# ------------------------------------------------- planted mistakes ---------
+# (name, text in kvq_oracle.c, replacement): plausible slips in the oracle's
+# Med3x, each of which one of the pins above must catch.
+MUTANTS = [
+    ("threshold_2x", "float thr = 3.0f * med;", "float thr = 2.0f * med;"),
+    ("median_upper_only", "float med = 0.5f * (srt[nc / 2 - 1] + srt[nc / 2]);",
+     "float med = srt[nc / 2];"),
+    ("first_not_largest", "if (r[i] > thr && (best < 0 || r[i] > r[best])) best = i;",
+     "if (r[i] > thr && best < 0) best = i;"),
+    ("eta_without_fp16_error", "float err = fabsf(x - (float)oc_f16_value(hv));",
+     "float err = 0.0f;"),
+]
+
+# the pins a mutant is run against, cheapest first
+PROBES = [
+    (test_hand_worked_spike_token, {}),
+    (test_eta_covers_the_fp16_rounding_of_an_extracted_value, {}),
+    (test_chunk_choice_matches_definition, {"d": 64}),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return str(tmp_path_factory.mktemp("med3_mutants"))
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(oracle_lib, mutant_dir, name, old, new):
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation target of {name} not found once in the oracle"
+    so = oracle.compile_variant(src.replace(old, new), mutant_dir, name)
+    caught = None
+    with oracle.library_override(so):
+        for fn, kw in PROBES:
+            try:
+                fn(oracle_lib, **kw)
+            except AssertionError:
+                caught = fn.__name__
+                break
+    assert caught, f"no pin catches the planted mistake {name}"
