@@ -12,7 +12,8 @@ Against things other than its own code:
   and are the fewest that do; sets are nested in tau_cov;
 * a brute-force, pairwise version of the ranking check on the originals;
 * a hand-worked two-block case where the quantized keys invert the order;
-* the bound never below the error against exact attention.
+* the bound never below the error against exact attention;
+* five planted mistakes compiled into copies of the oracle are each caught.
 """
 
 import math
@@ -204,3 +205,52 @@ def test_adaptive_bound_dominates_observed_error(oracle_lib, name, tau_cov, v_to
     r = c.decode_adaptive(q, inp.page_table, inp.seq_lens, k, v, tau_cov=tau_cov, v_tol=v_tol)
     od = oracle.dense(q, k, v, inp.seq_lens)
     assert (r["bound"] >= max_err(od, r["out"])).all()
+
+
+# ------------------------------------------------- planted mistakes ---------
+# (name, text in kvq_oracle.c, replacement): plausible slips in the oracle's
+# adaptive precision, each of which one of the pins above must catch.
+MUTANTS = [
+    ("coverage_one_block_short", "while (kstar < npg && cum < tau_cov) cum += ord[kstar++].m;",
+     "while (kstar + 1 < npg && cum < tau_cov) cum += ord[kstar++].m;"),
+    ("ascending_order", "  if (a->m > b->m) return -1;\n  if (a->m < b->m) return 1;",
+     "  if (a->m < b->m) return -1;\n  if (a->m > b->m) return 1;"),
+    ("ranking_check_reversed", "if (L - lmin > rank_tol) fail = 1;",
+     "if (lmin - L > rank_tol) fail = 1;"),
+    ("value_promotion_on_eta_only", "vp[lp] = ord[lp].m * et[lp * OC_PAGE] > v_tol ? 1 : 0;",
+     "vp[lp] = et[lp * OC_PAGE] > v_tol ? 1 : 0;"),
+    ("promoted_values_keep_eval", "for (int ch = 0; ch < d; ++ch) o[ch] += p[j] * (double)vf[ch];\n"
+     "          } else {",
+     "for (int ch = 0; ch < d; ++ch) o[ch] += p[j] * (double)vf[ch];\n"
+     "            Ev += p[j] * et[j];\n          } else {"),
+]
+
+# the pins a mutant is run against, cheapest first
+PROBES = [
+    (test_hand_worked_inversion, {}),
+    (test_selection_is_the_smallest_top_set_covering_tau_cov, {"name": "llama8b"}),
+    (test_everything_promoted_is_dense_attention, {"name": "tiny"}),
+    (test_values_only_is_value_promotion, {"name": "llama8b"}),
+    (test_ranking_check_matches_pairwise_brute_force, {"name": "llama8b", "rank_tol": 0.0}),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return str(tmp_path_factory.mktemp("adaptive_mutants"))
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(oracle_lib, mutant_dir, name, old, new):
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation target of {name} not found once in the oracle"
+    so = oracle.compile_variant(src.replace(old, new), mutant_dir, name)
+    caught = None
+    with oracle.library_override(so):
+        for fn, kw in PROBES:
+            try:
+                fn(oracle_lib, **kw)
+            except AssertionError:
+                caught = fn.__name__
+                break
+    assert caught, f"no pin catches the planted mistake {name}"

@@ -6,7 +6,8 @@
 * hand-worked group quantizations (tests/golden/codec_hand_worked.txt);
 * the round-trip invariant |x - deq(q(x))| <= s/2 (plus fp32 slack);
 * exact recovery of representable inputs;
-* the packed page layout is a bijection and matches the documented formula.
+* the packed page layout is a bijection and matches the documented formula;
+* five planted mistakes compiled into copies of the oracle are each caught.
 """
 
 import os
@@ -292,3 +293,46 @@ def test_pack_roundtrip_through_pool(oracle_lib, kbits, kgroup, d):
             errs = [oracle.quantize_asym(v[0, h, t, g * 32:(g + 1) * 32])[4]
                     for t in range(lp * 16, min(T, lp * 16 + 16)) for g in range(d // 32)]
             assert c.eta[page, h] == np.nextafter(np.float32(max(errs)), np.float32(np.inf))
+
+
+# ------------------------------------------------- planted mistakes ---------
+# (name, text in kvq_oracle.c, replacement): plausible slips in the oracle's
+# Tier-1 codec, each of which one of the pins above must catch.
+MUTANTS = [
+    ("key_scale_rounded_down", "float t = a / (float)Q;\n  uint16_t sb = oc_f16_round(t, 1);",
+     "float t = a / (float)Q;\n  uint16_t sb = oc_f16_round(t, 0);"),
+    ("key_scale_over_q_plus_one", "float t = a / (float)Q;", "float t = a / (float)(Q + 1);"),
+    ("key_code_truncated", "float r = rintf(x[c] / s);", "float r = truncf(x[c] / s);"),
+    ("value_zero_rounded_up", "uint16_t zb = oc_f16_round(lo, 0);", "uint16_t zb = oc_f16_round(lo, 1);"),
+    ("value_sixteen_steps", "float t = (hi - z) / 15.0f;", "float t = (hi - z) / 16.0f;"),
+]
+
+# the pins a mutant is run against, cheapest first
+PROBES = [
+    (lambda lib: [test_hand_worked_groups(lib, c) for c in _gold_cases()], {}),
+    (test_roundtrip_invariant_symmetric, {"bits": 8}),
+    (test_roundtrip_invariant_asymmetric, {}),
+    (test_exact_recovery_symmetric, {"bits": 4}),
+    (test_exact_recovery_asymmetric, {}),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return str(tmp_path_factory.mktemp("codec_mutants"))
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(oracle_lib, mutant_dir, name, old, new):
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation target of {name} not found once in the oracle"
+    so = oracle.compile_variant(src.replace(old, new), mutant_dir, name)
+    caught = None
+    with oracle.library_override(so):
+        for fn, kw in PROBES:
+            try:
+                fn(oracle_lib, **kw)
+            except AssertionError:
+                caught = True
+                break
+    assert caught, f"no pin catches the planted mistake {name}"
