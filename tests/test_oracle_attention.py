@@ -4,7 +4,8 @@ Against: scipy's Sylvester Hadamard matrix, an fp64 matrix product, torch's
 fp64 scaled-dot-product attention, the two-token logistic closed form, an
 independent numpy dequantization of the group quantizers' output, brute force
 over score perturbations (the total-variation lemma behind E_key), and fp64
-dense attention on the originals (bound dominance on every query).
+dense attention on the originals (bound dominance on every query); four
+planted mistakes compiled into copies of the oracle are each caught.
 """
 
 import math
@@ -239,3 +240,48 @@ def test_empty_context_row(oracle_lib):
     o_hat, bound, flags, diag = c.decode(inp.q(), inp.page_table, [40, 0], tau=0.0)
     assert (o_hat[4:] == 0).all() and (bound[4:] == 0).all() and (flags[4:] == 0).all()
     assert (flags[:4] == 1).all()
+
+
+# ------------------------------------------------- planted mistakes ---------
+# (name, text in kvq_oracle.c, replacement): plausible slips in the oracle's
+# rotation and dense attention, each of which one of the pins above must catch.
+_DENSE_K = ("oc_load_vec(k, kv_is_f32, b * seq_stride + kv * head_stride + j * tok_stride, d, kf);\n"
+            "          double dot = 0.0;\n"
+            "          for (int ch = 0; ch < d; ++ch) dot += (double)qf[ch] * (double)kf[ch];\n"
+            "          z[j] = sc * dot;\n          if (z[j] > m) m = z[j];")
+_DENSE_P = ("double p = exp(z[j] - m) / l;\n"
+            "          oc_load_vec(v, kv_is_f32, b * seq_stride + kv * head_stride + j * tok_stride, d, vf);")
+MUTANTS = [
+    ("butterfly_sign", "y[j + h] = a - b;", "y[j + h] = b - a;"),
+    ("rotation_scale", "float c = (float)(1.0 / sqrt((double)d));", "float c = (float)(1.0 / d);"),
+    ("dense_unnormalized", _DENSE_P, _DENSE_P.replace("exp(z[j] - m) / l", "exp(z[j] - m)")),
+    ("dense_scale_twice", _DENSE_K, _DENSE_K.replace("z[j] = sc * dot;", "z[j] = sc * sc * dot;")),
+]
+
+# the pins a mutant is run against, cheapest first
+PROBES = [
+    (test_rotation_columns_are_scaled_hadamard, {"d": 64}),
+    (test_dense_two_token_closed_form, {}),
+    (test_dense_matches_torch_sdpa_fp64, {"dtype": "fp32"}),
+]
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return str(tmp_path_factory.mktemp("attention_mutants"))
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(oracle_lib, mutant_dir, name, old, new):
+    src = oracle.source_text()
+    assert src.count(old) == 1, f"mutation target of {name} not found once in the oracle"
+    so = oracle.compile_variant(src.replace(old, new), mutant_dir, name)
+    caught = None
+    with oracle.library_override(so):
+        for fn, kw in PROBES:
+            try:
+                fn(oracle_lib, **kw)
+            except AssertionError:
+                caught = fn.__name__
+                break
+    assert caught, f"no pin catches the planted mistake {name}"
