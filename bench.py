@@ -696,6 +696,8 @@ def measure_workload(name, args, world, rank, local):
     rec = {
         "value": _job_value(st.token_heads, world, ms_step),
         "unit": UNIT,
+        # the same rate counted per query head (x Hq/Hkv: each kv head serves its GQA group)
+        "value_q_heads": _job_value(st.token_heads, world, ms_step) * (wl.num_q_heads / wl.num_kv_heads),
         "ms_per_step": ms_step,
         "steps": args.steps,
         "config": {"workload": _describe(name),
@@ -767,6 +769,7 @@ def run_gpu(args):
         "metric": METRIC,
         "value": main["value"],
         "unit": UNIT,
+        "value_q_heads": main["value_q_heads"],
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
